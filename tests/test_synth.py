@@ -1,0 +1,102 @@
+"""CPU checks of the seeded input generator (synth): Philox known answers,
+the Irwin-Hall draw, bf16 rounding, the MXFP4 quantiser and the routing-gap
+conditioning.  The device generator's bit-identity is checked in
+test_gpu_synth.py."""
+import numpy as np
+import pytest
+
+import oracle
+import synth
+
+
+def test_philox4x32_10_known_answers():
+    # known-answer vectors of the Random123 distribution (Salmon et al., SC'11)
+    kat = [
+        ((0, 0, 0, 0), (0, 0), (0x6627E8D5, 0xE169C58D, 0xBC57AC4C, 0x9B00DBD8)),
+        ((0xFFFFFFFF,) * 4, (0xFFFFFFFF, 0xFFFFFFFF), (0x408F276D, 0x41C83B0E, 0xA20BC7C6, 0x6D5451FD)),
+        ((0x243F6A88, 0x85A308D3, 0x13198A2E, 0x03707344), (0xA4093822, 0x299F31D0),
+         (0xD16CFE09, 0x94FDCCEB, 0x5001E420, 0x24126EA1)),
+    ]
+    for ctr, key, want in kat:
+        got = synth.philox4x32_10(*ctr, *key)
+        assert tuple(int(g) for g in got) == want
+
+
+def test_irwin_hall_draw_moments_and_range():
+    key = synth.stream_key(123, 0, synth.T_X)
+    s = synth.irwin_hall_ints(key, 0, 0, 0, 400_000).astype(np.float64)
+    assert s.min() >= -131070 and s.max() <= 131070
+    assert abs(s.mean()) < 3 * synth.IH_SD / np.sqrt(len(s)) * 2
+    assert abs(s.std() / synth.IH_SD - 1) < 0.01
+    v = synth.normal_f32(key, 0, 0, 0, 400_000, 0.02).astype(np.float64)
+    assert abs(v.std() / 0.02 - 1) < 0.01
+    # substreams differ, elements are reproducible one by one
+    a = synth.irwin_hall_ints(key, 1, 0, 100, 10)
+    b = np.array([synth.irwin_hall_ints(key, 1, 0, 100 + i, 1)[0] for i in range(10)])
+    assert np.array_equal(a, b)
+    assert not np.array_equal(a, synth.irwin_hall_ints(key, 2, 0, 100, 10))
+
+
+def test_bf16_rne_matches_torch():
+    import torch
+    rng = np.random.default_rng(2)
+    v = np.concatenate([rng.normal(0, 1, 10000), rng.normal(0, 1e-30, 100)]).astype(np.float32)
+    want = torch.from_numpy(v).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(synth.bf16_rne(v), want)
+    assert np.array_equal(synth.bf16_to_f32(synth.bf16_rne(v)),
+                          torch.from_numpy(v).to(torch.bfloat16).float().numpy())
+
+
+def _dequant(codes, scales, K):
+    return np.stack([oracle.dequant_row(codes[r], scales[r], K) for r in range(codes.shape[0])])
+
+
+def test_quantizer_round_trips_exact_values_and_bounds_error():
+    rng = np.random.default_rng(4)
+    mags = np.array([0, 0.5, 1, 1.5, 2, 3, 4, 6])
+    R, K = 8, 128
+    vals = mags[rng.integers(0, 8, (R, K))] * rng.choice([-1.0, 1.0], (R, K))
+    vals *= np.repeat(2.0 ** rng.integers(-12, 3, (R, K // 32)), 32, axis=1)
+    vals[:, :32] = 0.0                                   # an all-zero block
+    codes, scales = synth.quantize_mxfp4(vals.astype(np.float32))
+    assert np.array_equal(_dequant(codes, scales, K), vals)
+    assert np.all(scales[:, 0] == 0)
+    # arbitrary values: error at most one grid step of the block (2 * 2^(s-127))
+    v = rng.normal(0, 0.02, (R, K)).astype(np.float32)
+    codes, scales = synth.quantize_mxfp4(v)
+    dq = _dequant(codes, scales, K)
+    step = np.repeat(2.0 ** (scales.astype(np.float64) - 127) * 2, 32, axis=1)
+    assert np.all(np.abs(dq - v) <= step)
+    # the block maximum lands in the top binade [4, 6] of the grid
+    amax_code = np.abs(dq).reshape(R, K // 32, 32).max(2) / 2.0 ** (scales.astype(np.float64) - 127)
+    assert np.all((amax_code >= 4) & (amax_code <= 6))
+
+
+def test_quantizer_ties_round_to_even():
+    # scale 127 (amax 6 in the block): 0.25 -> 0, 0.75 -> 1, 1.25 -> 1, 1.75 -> 2, 2.5 -> 2, 3.5 -> 4, 5 -> 4
+    row = np.zeros((1, 32), np.float32)
+    row[0, :8] = [6, 0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5]
+    codes, scales = synth.quantize_mxfp4(row)
+    assert scales[0, 0] == 127
+    dq = oracle.dequant_row(codes[0], scales[0], 32)
+    assert list(dq[:8]) == [6, 0, 1, 1, 2, 2, 4, 4]
+
+
+def test_tiny_workload_gap_and_bias():
+    cfg = synth.CONFIGS[0]
+    wr = synth.gen_router_w(cfg)
+    x, att = synth.gen_tokens(cfg, wr, None, range(16))
+    lg = oracle.router_logits(x, wr, None)
+    srt = -np.sort(-lg, axis=1)
+    assert np.all(srt[:, cfg.top_k - 1] - srt[:, cfg.top_k] >= cfg.min_gap)
+    b = synth.gen_router_bias(synth.CONFIGS[3])
+    ranks = np.rint(np.exp(-b.astype(np.float64) / 1.1)).astype(int)
+    assert sorted(ranks.tolist()) == list(range(1, 897))
+    assert synth.gen_router_bias(cfg) is None
+
+
+def test_counted_bytes_formula():
+    c1 = synth.CONFIGS[1]
+    # per active expert: codes + scales of gate/up and down
+    assert c1.expert_bytes() == 2 * 2048 * (3584 + 224) + 7168 * (1024 + 64)
+    assert c1.counted_bytes(16) == 16 * c1.expert_bytes() + 3 * 2048 * 7168 * 2 + 7168 * 896 * 2 + 3 * 7168 * 2
