@@ -1,0 +1,200 @@
+/*
+ * moe_decode.h -- C ABI of a single-GPU (B200, sm_100a) implementation of
+ * one decode step of a very sparse mixture-of-experts layer with MXFP4
+ * expert weights.
+ *
+ * What the layer is.  The decode-path pages describe a model whose MoE
+ * layers hold 896 routed experts with 16 active per token (aitest123, "how
+ * NVIDIA optimised Kimi K3 with a 12k-line CuTe DSL megakernel", intro;
+ * tmtpost, section on the phenomenon), native MXFP4 4-bit expert weights
+ * (tmtpost, same section), and a shared expert that runs on its own stream
+ * beside the routed experts (yeyulingfeng, section 02, second of the four
+ * optimisations; smzdm, section on the four-step rework, third step).
+ * Decode at small batch is bound by memory traffic and launch overhead
+ * (aitest123, intro; yeyulingfeng, section 01).  Per token b the layer
+ * computes
+ *
+ *   l[b][e]  = sum_h x[b][h] Wr[h][e] (+ bias[e])          fp32, never rounded
+ *   S_b      = the k experts with the largest l[b][.], equal logits going to
+ *              the lower expert id; listed in ascending expert id
+ *   w[b][j]  = exp(l_j - m) / sum_{i in S_b} exp(l_i - m),  m = max over S_b
+ *   y[b][j]  = Wd_e (silu(Wg_e x_b) * (Wu_e x_b)),  e = S_b[j], MXFP4 weights
+ *   y_s[b]   = Wsd (silu(Wsg x_b) * (Wsu x_b)),     bf16 shared-expert weights
+ *   out[b]   = bf16( residual[b] + y_s[b] + sum_{j = 0..k-1} w[b][j] y[b][j] )
+ *
+ * with the final sum taken in fp32 in exactly that order (ascending expert
+ * id), so results are bitwise reproducible run to run.
+ *
+ * MXFP4 (OCP Microscaling v1.0): each 32 consecutive elements along the
+ * reduction dimension K share one E8M0 scale byte s (value 2^(s-127)); each
+ * element is a 4-bit E2M1 code (magnitudes 0, .5, 1, 1.5, 2, 3, 4, 6; bit 3
+ * is the sign).  Two codes per byte, the even-K element in the low nibble.
+ *
+ * Conventions for every call:
+ *  - All tensor pointers are DEVICE pointers unless the name ends in _host,
+ *    16-byte aligned, row-major, densely packed, and owned by the caller.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *    stream).  Calls only enqueue work: they never synchronise, allocate or
+ *    free, so they may be captured into a CUDA graph (moe_layer_create and
+ *    moe_layer_destroy excepted).
+ *  - Errors are returned, never raised: invalid arguments are rejected on the
+ *    host with MOE_ERR_INVALID_ARG before anything is launched; a failed
+ *    launch returns MOE_ERR_CUDA.  Device-side waits are bounded; a wait that
+ *    gives up records MOE_ERR_TIMEOUT, read by moe_layer_last_device_error.
+ *  - One layer object may be used from one stream at a time.
+ */
+#ifndef MOE_DECODE_H_
+#define MOE_DECODE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__) || defined(__clang__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1, /* null/misaligned pointer, bad size, B > max_batch */
+  MOE_ERR_UNSUPPORTED = 2, /* shape the kernels do not cover, or no sm_100 device */
+  MOE_ERR_CUDA = 3,        /* a CUDA runtime call or launch failed */
+  MOE_ERR_OOM = 4,         /* scratch allocation failed in moe_layer_create */
+  MOE_ERR_TIMEOUT = 5      /* a bounded device-side wait gave up */
+} moe_status_t;
+
+typedef struct moe_layer* moe_layer_t; /* opaque, library-owned */
+
+/* Flags (moe_layer_config.flags); the defaults are the fastest path. */
+#define MOE_FLAG_NO_PDL 0x1u        /* launch without programmatic dependent launch */
+#define MOE_FLAG_NO_SIDE_STREAM 0x2u /* run the shared expert on the caller's stream */
+#define MOE_FLAG_NO_PREFETCH 0x4u   /* no L2 prefetch of the next layer's weights */
+#define MOE_FLAG_NO_GROUPED 0x8u    /* never use the tensor-core grouped expert path */
+
+typedef struct {
+  int hidden;       /* H: model width, multiple of 32 */
+  int n_experts;    /* E: routed experts, 1..1024 */
+  int top_k;        /* k: active experts per token, 1..32, k <= E */
+  int inter;        /* I: routed expert intermediate size, multiple of 32 */
+  int shared_inter; /* I_s: shared expert intermediate size, multiple of 32, 0 = none */
+  int max_batch;    /* largest B any call will pass, 1..64 (larger batches
+                       fall outside this decode path, as on the pages:
+                       yeyulingfeng, section 03, the batch-64 fallback) */
+  unsigned flags;   /* MOE_FLAG_* */
+} moe_layer_config;
+
+/* Weights: DEVICE pointers, caller-owned, borrowed (never copied, except the
+ * router matrix, see moe_layer_create); they must stay valid and unchanged
+ * while the layer exists. */
+typedef struct {
+  const void* router_w;      /* bf16 [H][E]: logit e is sum_h x[h] router_w[h][e] */
+  const float* router_bias;  /* fp32 [E], added to the logits before selection and
+                                softmax; NULL = no bias */
+  const uint8_t* w_gate_up;  /* E2M1 codes [E][2I][H/2]; rows 0..I-1 gate, I..2I-1 up */
+  const uint8_t* s_gate_up;  /* E8M0 scales [E][2I][H/32] */
+  const uint8_t* w_down;     /* E2M1 codes [E][H][I/2] */
+  const uint8_t* s_down;     /* E8M0 scales [E][H][I/32] */
+  const void* shared_gate_up;/* bf16 [2*I_s][H]; rows 0..I_s-1 gate, then up (NULL if I_s = 0) */
+  const void* shared_down;   /* bf16 [H][I_s] (NULL if I_s = 0) */
+} moe_layer_weights;
+
+/* Routing plan of one call (DEVICE pointers).  Pair p = b*k + j names slot j
+ * of token b. */
+typedef struct {
+  int32_t* topk_idx; /* [B][k] selected experts, ascending id within a token */
+  float* topk_w;     /* [B][k] softmax over the selected logits, same order */
+  int32_t* counts;   /* [E] pairs routed to each expert */
+  int32_t* offsets;  /* [E+1] exclusive prefix sum of counts; offsets[E] = B*k */
+  int32_t* pair_ids; /* [B*k] pairs sorted by (expert, b, j): expert e's pairs are
+                        pair_ids[offsets[e] .. offsets[e+1]) */
+  int32_t* active;   /* [E] capacity; the first *n_active entries are the experts
+                        with counts > 0, ascending */
+  int32_t* n_active; /* [1] */
+} moe_routing;
+
+/* Create a layer.  Checks the config (sizes above; the device must be
+ * compute capability 10.x), allocates the layer's scratch for max_batch
+ * tokens, a side stream and events, and copies router_w once into a
+ * library-owned expert-major [E][H] copy that the router kernel streams
+ * (so router_w need not outlive this call; every other weight must).
+ * Uses the current CUDA device.  Synchronises the device once.
+ * Returns MOE_ERR_INVALID_ARG / MOE_ERR_UNSUPPORTED / MOE_ERR_OOM /
+ * MOE_ERR_CUDA; on failure *out is NULL. */
+MOE_API moe_status_t moe_layer_create(const moe_layer_config* cfg, const moe_layer_weights* w,
+                              moe_layer_t* out);
+
+/* Free everything the layer owns (synchronises its streams first). NULL is a no-op. */
+MOE_API moe_status_t moe_layer_destroy(moe_layer_t layer);
+
+/* Router GEMV + top-k + softmax + bucketing for B tokens (the router row and
+ * the top-k selection of the pages: aitest123 intro, 16 of 896 experts).
+ * x: bf16 [B][H].  r: where to write the plan; NULL = the layer's own
+ * buffers (see moe_layer_routing).  One kernel launch. */
+MOE_API moe_status_t moe_router_topk(moe_layer_t layer, const void* x, int B, const moe_routing* r,
+                             void* stream);
+
+/* The selected experts and the shared expert for B tokens, given a routing
+ * plan from moe_router_topk (r NULL = the layer's own plan).
+ * y_routed: fp32 [B*k][H], row p = unweighted output of pair p's expert;
+ * y_shared: fp32 [B][H] (ignored, may be NULL, when I_s = 0).
+ * The shared expert runs on the layer's side stream, joined back before
+ * return (pages: yeyulingfeng section 02; smzdm, third step). */
+MOE_API moe_status_t moe_experts_mxfp4(moe_layer_t layer, const void* x, int B, const moe_routing* r,
+                               float* y_routed, float* y_shared, void* stream);
+
+/* out[b] = bf16(residual[b] + y_shared[b] + sum_j topk_w[b][j] y_routed[b*k+j]),
+ * fp32 sums in ascending j (= ascending expert id), rounded once to nearest
+ * even.  residual, out: bf16 [B][H]; out may equal residual.  y_shared may be
+ * NULL (treated as zero).  The residual add on the spot follows the pages'
+ * fused residual (yeyulingfeng section 02, first optimisation). */
+MOE_API moe_status_t moe_combine_residual(moe_layer_t layer, int B, const moe_routing* r,
+                                  const float* y_routed, const float* y_shared,
+                                  const void* residual, void* out, void* stream);
+
+/* The whole layer in one call: router/top-k/buckets, routed experts, shared
+ * expert on the side stream, down projection fused with the combine and
+ * residual add.  Kernels are chained with programmatic dependent launch;
+ * with `next` non-NULL the tail of this layer prefetches next's router and
+ * shared-expert weights into L2 (pages: yeyulingfeng section 02, third and
+ * fourth optimisations).  x, residual, out: bf16 [B][H]; out may equal
+ * residual.  The routing plan is left in the layer's buffers. */
+MOE_API moe_status_t moe_layer_forward(moe_layer_t layer, moe_layer_t next, const void* x,
+                               const void* residual, void* out, int B, void* stream);
+
+/* moe_layer_forward from HOST memory: copies x_host and residual_host
+ * (bf16 [B][H], pinned memory recommended) into the layer's device staging
+ * buffers, runs the layer and copies the result back to out_host, all on
+ * `stream`.  Returns once the work is enqueued; synchronise `stream` before
+ * reading out_host. */
+MOE_API moe_status_t moe_layer_forward_host(moe_layer_t layer, const void* x_host,
+                                    const void* residual_host, void* out_host, int B,
+                                    void* stream);
+
+/* Pointers to the layer's own routing-plan buffers (device memory owned by
+ * the layer, valid until destroy). */
+MOE_API moe_status_t moe_layer_routing(moe_layer_t layer, moe_routing* out);
+
+/* Reads (synchronously) and clears the layer's device error word: MOE_OK,
+ * or MOE_ERR_TIMEOUT if a bounded device-side wait gave up since the last
+ * call. */
+MOE_API moe_status_t moe_layer_last_device_error(moe_layer_t layer);
+
+/* Timing probe: when start/stop (cudaEvent_t as void*) are non-NULL,
+ * moe_layer_forward records start right before and stop right after the
+ * routed gate/up kernel, on the stream it is launched on.  NULL, NULL
+ * turns the probe off. */
+MOE_API moe_status_t moe_layer_set_probe(moe_layer_t layer, void* start, void* stop);
+
+/* Static description string of a status code. */
+MOE_API const char* moe_status_string(moe_status_t s);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_DECODE_H_ */

@@ -255,23 +255,61 @@ int oracle_layer(int B, int H, int E, int k, int I, int Is, const uint16_t* x, c
   std::vector<double> xd((size_t)B * H);
   for (size_t i = 0; i < (size_t)B * H; ++i) xd[i] = bf16_value(x[i]);
 
+  // Routed experts: first every h[p][i], then every y[p][r]; each element is
+  // the same sequential sum as in oracle_expert_ffn, the loops over
+  // independent elements are spread over threads.
   std::vector<double> yr((size_t)B * k * H), hr((size_t)B * k * I);
-#pragma omp parallel for schedule(dynamic, 1)
-  for (int p = 0; p < B * k; ++p) {
-    const int b = p / k;
-    const int e = idx[p];
-    const size_t slot = (size_t)(expert_slot ? expert_slot[e] : e);
-    oracle_expert_ffn(xd.data() + (size_t)b * H, gu_codes + slot * (2 * (size_t)I) * (H / 2),
-                      gu_scales + slot * (2 * (size_t)I) * (H / 32), d_codes + slot * (size_t)H * (I / 2),
-                      d_scales + slot * (size_t)H * (I / 32), H, I, hr.data() + (size_t)p * I,
-                      yr.data() + (size_t)p * H);
+  auto slot_of = [&](int p) { return (size_t)(expert_slot ? expert_slot[idx[p]] : idx[p]); };
+#pragma omp parallel for schedule(dynamic, 16)
+  for (long long pi = 0; pi < (long long)B * k * I; ++pi) {
+    const int p = (int)(pi / I), i = (int)(pi % I);
+    const double* xb = xd.data() + (size_t)(p / k) * H;
+    const size_t sl = slot_of(p);
+    const uint8_t* gc = gu_codes + sl * (2 * (size_t)I) * (H / 2);
+    const uint8_t* gs = gu_scales + sl * (2 * (size_t)I) * (H / 32);
+    std::vector<double> row(H);
+    dequant_row(gc + (size_t)i * (H / 2), gs + (size_t)i * (H / 32), H, row.data());
+    double g = 0.0;
+    for (int c = 0; c < H; ++c) g += row[c] * xb[c];
+    dequant_row(gc + (size_t)(I + i) * (H / 2), gs + (size_t)(I + i) * (H / 32), H, row.data());
+    double u = 0.0;
+    for (int c = 0; c < H; ++c) u += row[c] * xb[c];
+    hr[pi] = silu(g) * u;
   }
+#pragma omp parallel for schedule(dynamic, 64)
+  for (long long pr = 0; pr < (long long)B * k * H; ++pr) {
+    const int p = (int)(pr / H), r = (int)(pr % H);
+    const size_t sl = slot_of(p);
+    std::vector<double> row(I);
+    dequant_row(d_codes + sl * (size_t)H * (I / 2) + (size_t)r * (I / 2),
+                d_scales + sl * (size_t)H * (I / 32) + (size_t)r * (I / 32), I, row.data());
+    const double* h = hr.data() + (size_t)p * I;
+    double acc = 0.0;
+    for (int i = 0; i < I; ++i) acc += row[i] * h[i];
+    yr[pr] = acc;
+  }
+  // Shared expert, same structure.
   std::vector<double> ys((size_t)B * H, 0.0);
   if (Is > 0 && shared_gu && shared_d) {
-#pragma omp parallel for schedule(dynamic, 1)
-    for (int b = 0; b < B; ++b)
-      oracle_shared_ffn(xd.data() + (size_t)b * H, shared_gu, shared_d, H, Is, nullptr,
-                        ys.data() + (size_t)b * H);
+    std::vector<double> hs((size_t)B * Is);
+#pragma omp parallel for schedule(dynamic, 16)
+    for (long long bi = 0; bi < (long long)B * Is; ++bi) {
+      const int b = (int)(bi / Is), i = (int)(bi % Is);
+      const double* xb = xd.data() + (size_t)b * H;
+      double g = 0.0, u = 0.0;
+      for (int c = 0; c < H; ++c) {
+        g += bf16_value(shared_gu[(size_t)i * H + c]) * xb[c];
+        u += bf16_value(shared_gu[(size_t)(Is + i) * H + c]) * xb[c];
+      }
+      hs[bi] = silu(g) * u;
+    }
+#pragma omp parallel for schedule(dynamic, 64)
+    for (long long br = 0; br < (long long)B * H; ++br) {
+      const int b = (int)(br / H), r = (int)(br % H);
+      double acc = 0.0;
+      for (int i = 0; i < Is; ++i) acc += bf16_value(shared_d[(size_t)r * Is + i]) * hs[(size_t)b * Is + i];
+      ys[br] = acc;
+    }
   }
   if (h_routed) std::memcpy(h_routed, hr.data(), sizeof(double) * B * k * I);
   if (y_routed) std::memcpy(y_routed, yr.data(), sizeof(double) * B * k * H);

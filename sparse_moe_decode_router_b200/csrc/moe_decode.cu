@@ -1,0 +1,573 @@
+// Host side of the MoE decode library: layer object, launch plans,
+// programmatic-dependent-launch chaining, the shared-expert side stream and
+// the C ABI declared in include/moe_decode.h.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdint>
+#include <cstring>
+#include <new>
+
+#include "../../include/moe_decode.h"
+#include "kernels.cuh"
+
+using namespace moe;
+
+namespace {
+
+constexpr int kSmemBudget = 200 * 1024;  // dynamic shared memory per CTA (1 CTA per SM)
+constexpr int kMaxStages = 8;
+
+size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+struct GemvPlan {
+  bool ok = false;
+  int K = 0, out_rows = 0, R = 0, G = 0, wpr = 0, rpg = 0, n_stages = 0, stage_bytes = 0;
+  int threads = 0, smem = 0;
+};
+
+// Work decomposition of one weight stream for one register budget (tmax tokens per pass:
+// 1 -> up to 16 consumer warps, 2 -> up to 8).
+GemvPlan make_plan(int K, int out_rows, bool swiglu, bool mxfp4, int tmax) {
+  GemvPlan p;
+  if (K <= 0 || K % 32 || out_rows <= 0) return p;
+  const int C = K / 32;
+  const int wpr = (C + 31) / 32;
+  if (wpr > 16) return p;
+  const int maxw = (tmax == 1) ? 16 : 8;
+  const int rowbytes = mxfp4 ? K / 2 : K * 2;
+  const int sbytes = mxfp4 ? K / 32 : 0;
+  for (int rpg = 2; rpg >= 1; --rpg) {
+    for (int G = std::max(1, maxw / wpr); G >= 1; --G) {
+      const int R = G * rpg;
+      if (out_rows % R) continue;
+      if (mxfp4 && (R * sbytes) % 16) continue;
+      const int rows = swiglu ? 2 * R : R;
+      const int stage = (int)align_up((size_t)rows * (rowbytes + sbytes), 128);
+      const int hdr = (int)align_up(16 * kMaxStages + 256 * G * wpr + 16, 128);
+      int ns = (kSmemBudget - hdr) / stage;
+      ns = std::min(ns, kMaxStages);
+      if (ns < 3 && !(rpg == 1 && G == 1 && ns >= 2)) continue;
+      p.ok = true;
+      p.K = K;
+      p.out_rows = out_rows;
+      p.R = R;
+      p.G = G;
+      p.wpr = wpr;
+      p.rpg = rpg;
+      p.n_stages = ns;
+      p.stage_bytes = stage;
+      p.threads = (G * wpr + 1) * 32;
+      if (p.threads > (tmax == 1 ? 17 * 32 : 9 * 32)) return GemvPlan();
+      p.smem = hdr + ns * stage;
+      return p;
+    }
+  }
+  return p;
+}
+
+enum Kind { K_ROUTER = 0, K_SGU = 1, K_SDN = 2, K_GU = 3, K_DN = 4, K_DNC = 5, K_NUM = 6 };
+
+typedef void (*GemvFn)(const GemvArgs);
+
+template <int RPG, int TMAX>
+GemvFn pick_fn(Kind k) {
+  constexpr int MAXT = (TMAX == 1) ? 17 * 32 : 9 * 32;
+  switch (k) {
+    case K_ROUTER: return stream_gemv_kernel<W_BF16, EPI_ROUTER, false, RPG, TMAX, MAXT>;
+    case K_SGU: return stream_gemv_kernel<W_BF16, EPI_SWIGLU, false, RPG, TMAX, MAXT>;
+    case K_SDN: return stream_gemv_kernel<W_BF16, EPI_STORE, true, RPG, TMAX, MAXT>;
+    case K_GU: return stream_gemv_kernel<W_MXFP4, EPI_SWIGLU, false, RPG, TMAX, MAXT>;
+    case K_DN: return stream_gemv_kernel<W_MXFP4, EPI_STORE, true, RPG, TMAX, MAXT>;
+    case K_DNC: return stream_gemv_kernel<W_MXFP4, EPI_DOWN_COMBINE, true, RPG, TMAX, MAXT>;
+    default: return nullptr;
+  }
+}
+
+GemvFn gemv_fn(Kind k, int rpg, int tmax) {
+  if (tmax == 1) return rpg == 2 ? pick_fn<2, 1>(k) : pick_fn<1, 1>(k);
+  return rpg == 2 ? pick_fn<2, 2>(k) : pick_fn<1, 2>(k);
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+}  // namespace
+
+struct moe_layer {
+  moe_layer_config cfg{};
+  moe_layer_weights w{};
+  int device = 0;
+  int num_sms = 0;
+  bool pdl = true;
+  bool side_stream = true;
+  bool prefetch = true;
+  char* arena = nullptr;
+  uint16_t* wr_t = nullptr;  // router matrix, expert-major [E][H]
+  float* logits = nullptr;
+  moe_routing plan{};
+  float* h = nullptr;
+  float* y = nullptr;
+  float* hs = nullptr;
+  float* ys = nullptr;
+  int* router_cnt = nullptr;
+  int* tile_cnt = nullptr;
+  int* err = nullptr;
+  uint16_t* x_stage = nullptr;
+  uint16_t* res_stage = nullptr;
+  uint16_t* out_stage = nullptr;
+  cudaStream_t side = nullptr;
+  cudaEvent_t ev_fork = nullptr, ev_join = nullptr;
+  cudaEvent_t probe_start = nullptr, probe_stop = nullptr;
+  GemvPlan plans[K_NUM][2];  // [kind][tmax==1 ? 0 : 1]
+};
+
+namespace {
+
+moe_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+int tmax_for(int B) { return B == 1 ? 1 : 2; }
+
+template <typename... Args>
+cudaError_t launch_ex(void (*kern)(Args...), int grid, int block, int smem, cudaStream_t st, bool pdl,
+                      Args... args) {
+  cudaLaunchConfig_t c = {};
+  c.gridDim = dim3(grid);
+  c.blockDim = dim3(block);
+  c.dynamicSmemBytes = (size_t)smem;
+  c.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  c.attrs = attr;
+  c.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&c, kern, args...);
+}
+
+GemvArgs base_args(const moe_layer* L, const GemvPlan& p) {
+  GemvArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.K = p.K;
+  a.out_rows = p.out_rows;
+  a.R = p.R;
+  a.G = p.G;
+  a.wpr = p.wpr;
+  a.n_stages = p.n_stages;
+  a.stage_bytes = p.stage_bytes;
+  a.top_k = L->cfg.top_k;
+  a.n_experts = L->cfg.n_experts;
+  a.err = L->err;
+  return a;
+}
+
+cudaError_t run_gemv(moe_layer* L, Kind k, int B, const GemvArgs& a, cudaStream_t st, bool pdl) {
+  const int tm = tmax_for(B);
+  const GemvPlan& p = L->plans[k][tm == 1 ? 0 : 1];
+  GemvFn fn = gemv_fn(k, p.rpg, tm);
+  return launch_ex(fn, L->num_sms, p.threads, p.smem, st, pdl, a);
+}
+
+const GemvPlan& plan_of(const moe_layer* L, Kind k, int B) { return L->plans[k][tmax_for(B) == 1 ? 0 : 1]; }
+
+bool routing_ok(const moe_routing* r) {
+  return r && r->topk_idx && r->topk_w && r->counts && r->offsets && r->pair_ids && r->active && r->n_active;
+}
+
+cudaError_t launch_router(moe_layer* L, const void* x, int B, const moe_routing& r, cudaStream_t st) {
+  const GemvPlan& p = plan_of(L, K_ROUTER, B);
+  GemvArgs a = base_args(L, p);
+  a.w = reinterpret_cast<const uint8_t*>(L->wr_t);
+  a.act = x;
+  a.routed = 0;
+  a.n_tokens = B;
+  a.out = L->logits;
+  a.bias = L->w.router_bias;
+  a.topk_w = r.topk_w;
+  a.topk_idx = r.topk_idx;
+  a.counts = r.counts;
+  a.offsets_out = r.offsets;
+  a.pair_ids_out = r.pair_ids;
+  a.active_out = r.active;
+  a.n_active_out = r.n_active;
+  a.done_counter = L->router_cnt;
+  return run_gemv(L, K_ROUTER, B, a, st, L->pdl);
+}
+
+cudaError_t launch_shared(moe_layer* L, const void* x, int B, float* ys, cudaStream_t st, bool pdl) {
+  const int H = L->cfg.hidden, Is = L->cfg.shared_inter;
+  {
+    const GemvPlan& p = plan_of(L, K_SGU, B);
+    GemvArgs a = base_args(L, p);
+    a.w = reinterpret_cast<const uint8_t*>(L->w.shared_gate_up);
+    a.up_off = Is;
+    a.act = x;
+    a.n_tokens = B;
+    a.out = L->hs;
+    cudaError_t e = run_gemv(L, K_SGU, B, a, st, pdl);
+    if (e != cudaSuccess) return e;
+  }
+  const GemvPlan& p = plan_of(L, K_SDN, B);
+  GemvArgs a = base_args(L, p);
+  a.w = reinterpret_cast<const uint8_t*>(L->w.shared_down);
+  a.act = L->hs;
+  a.n_tokens = B;
+  a.out = ys;
+  (void)H;
+  return run_gemv(L, K_SDN, B, a, st, pdl);
+}
+
+GemvArgs routed_args(const moe_layer* L, const GemvPlan& p, const moe_routing& r, int B) {
+  GemvArgs a = base_args(L, p);
+  a.routed = 1;
+  a.n_pairs = B * L->cfg.top_k;
+  a.n_active = r.n_active;
+  a.active = r.active;
+  a.offsets = r.offsets;
+  a.pair_ids = r.pair_ids;
+  return a;
+}
+
+cudaError_t launch_gate_up(moe_layer* L, const void* x, int B, const moe_routing& r, cudaStream_t st) {
+  const int H = L->cfg.hidden, I = L->cfg.inter;
+  const GemvPlan& p = plan_of(L, K_GU, B);
+  GemvArgs a = routed_args(L, p, r, B);
+  a.w = L->w.w_gate_up;
+  a.sc = L->w.s_gate_up;
+  a.w_gstride = (long long)2 * I * (H / 2);
+  a.s_gstride = (long long)2 * I * (H / 32);
+  a.up_off = I;
+  a.act = x;
+  a.act_by_pair = 0;
+  a.out = L->h;
+  return run_gemv(L, K_GU, B, a, st, L->pdl);
+}
+
+cudaError_t launch_down(moe_layer* L, int B, const moe_routing& r, float* y, bool fused, const void* residual,
+                        void* out, const float* ys, moe_layer* next, cudaStream_t st, bool pdl) {
+  const int H = L->cfg.hidden, I = L->cfg.inter;
+  const Kind k = fused ? K_DNC : K_DN;
+  const GemvPlan& p = plan_of(L, k, B);
+  GemvArgs a = routed_args(L, p, r, B);
+  a.w = L->w.w_down;
+  a.sc = L->w.s_down;
+  a.w_gstride = (long long)H * (I / 2);
+  a.s_gstride = (long long)H * (I / 32);
+  a.act = L->h;
+  a.act_by_pair = 1;
+  a.out = y;
+  if (fused) {
+    a.comb_w = r.topk_w;
+    a.y_shared = ys;
+    a.residual = static_cast<const uint16_t*>(residual);
+    a.out_bf16 = static_cast<uint16_t*>(out);
+    a.batch = B;
+    a.tile_counter = L->tile_cnt;
+    if (next && L->prefetch) {
+      a.pf_ptr[0] = reinterpret_cast<const uint8_t*>(next->wr_t);
+      a.pf_bytes[0] = (long long)next->cfg.n_experts * next->cfg.hidden * 2;
+      if (next->cfg.shared_inter > 0) {
+        a.pf_ptr[1] = reinterpret_cast<const uint8_t*>(next->w.shared_gate_up);
+        a.pf_bytes[1] = (long long)2 * next->cfg.shared_inter * next->cfg.hidden * 2;
+      }
+    }
+  }
+  return run_gemv(L, k, B, a, st, pdl);
+}
+
+cudaError_t launch_combine(moe_layer* L, int B, const moe_routing& r, const float* y, const float* ys,
+                           const void* residual, void* out, cudaStream_t st) {
+  GemvArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.out_rows = L->cfg.hidden;
+  a.top_k = L->cfg.top_k;
+  a.comb_w = r.topk_w;
+  a.y_shared = ys;
+  a.residual = static_cast<const uint16_t*>(residual);
+  a.out_bf16 = static_cast<uint16_t*>(out);
+  a.batch = B;
+  const long long n = (long long)B * L->cfg.hidden;
+  const int grid = (int)std::min<long long>((n + 255) / 256, (long long)L->num_sms * 8);
+  return launch_ex(combine_kernel, grid, 256, 0, st, L->pdl, a, y);
+}
+
+moe_status_t check_call(const moe_layer* L, int B) {
+  if (!L) return MOE_ERR_INVALID_ARG;
+  if (B < 1 || B > L->cfg.max_batch) return MOE_ERR_INVALID_ARG;
+  return MOE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* moe_status_string(moe_status_t s) {
+  switch (s) {
+    case MOE_OK: return "ok";
+    case MOE_ERR_INVALID_ARG: return "invalid argument";
+    case MOE_ERR_UNSUPPORTED: return "unsupported shape or device";
+    case MOE_ERR_CUDA: return "CUDA error";
+    case MOE_ERR_OOM: return "out of device memory";
+    case MOE_ERR_TIMEOUT: return "device-side wait timed out";
+  }
+  return "unknown status";
+}
+
+moe_status_t moe_layer_create(const moe_layer_config* cfg, const moe_layer_weights* w, moe_layer_t* out) {
+  if (!out) return MOE_ERR_INVALID_ARG;
+  *out = nullptr;
+  if (!cfg || !w) return MOE_ERR_INVALID_ARG;
+  const moe_layer_config c = *cfg;
+  if (c.hidden <= 0 || c.hidden % 32 || c.inter <= 0 || c.inter % 32 || c.shared_inter < 0 ||
+      c.shared_inter % 32 || c.n_experts < 1 || c.n_experts > kMaxExperts || c.top_k < 1 ||
+      c.top_k > kMaxTopK || c.top_k > c.n_experts || c.max_batch < 1 || c.max_batch > kMaxBatch)
+    return MOE_ERR_INVALID_ARG;
+  if (!w->router_w || !w->w_gate_up || !w->s_gate_up || !w->w_down || !w->s_down) return MOE_ERR_INVALID_ARG;
+  if (c.shared_inter > 0 && (!w->shared_gate_up || !w->shared_down)) return MOE_ERR_INVALID_ARG;
+  const void* ptrs[] = {w->router_w, w->w_gate_up, w->s_gate_up, w->w_down, w->s_down};
+  for (const void* p : ptrs)
+    if (!aligned16(p)) return MOE_ERR_INVALID_ARG;
+  if (c.shared_inter > 0 && (!aligned16(w->shared_gate_up) || !aligned16(w->shared_down)))
+    return MOE_ERR_INVALID_ARG;
+
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
+  int major = 0, sms = 0;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  if (major != 10) return MOE_ERR_UNSUPPORTED;
+
+  moe_layer* L = new (std::nothrow) moe_layer();
+  if (!L) return MOE_ERR_OOM;
+  L->cfg = c;
+  L->w = *w;
+  L->device = dev;
+  L->num_sms = sms;
+  L->pdl = !(c.flags & MOE_FLAG_NO_PDL);
+  L->side_stream = !(c.flags & MOE_FLAG_NO_SIDE_STREAM);
+  L->prefetch = !(c.flags & MOE_FLAG_NO_PREFETCH);
+
+  const int H = c.hidden, E = c.n_experts, k = c.top_k, I = c.inter, Is = c.shared_inter, MB = c.max_batch;
+  for (int t = 0; t < 2; ++t) {
+    const int tm = t == 0 ? 1 : 2;
+    L->plans[K_ROUTER][t] = make_plan(H, E, false, false, tm);
+    L->plans[K_GU][t] = make_plan(H, I, true, true, tm);
+    L->plans[K_DN][t] = make_plan(I, H, false, true, tm);
+    L->plans[K_DNC][t] = make_plan(I, H, false, true, tm);
+    if (Is > 0) {
+      L->plans[K_SGU][t] = make_plan(H, Is, true, false, tm);
+      L->plans[K_SDN][t] = make_plan(Is, H, false, false, tm);
+    }
+    bool ok = L->plans[K_ROUTER][t].ok && L->plans[K_GU][t].ok && L->plans[K_DN][t].ok;
+    if (Is > 0) ok = ok && L->plans[K_SGU][t].ok && L->plans[K_SDN][t].ok;
+    // the router's last CTA reuses its stage ring for top-k and bucketing
+    ok = ok && (size_t)L->plans[K_ROUTER][t].n_stages * L->plans[K_ROUTER][t].stage_bytes >=
+                   8 * 1024 + 8 * kMaxExperts + 4 * (kMaxExperts + 1);
+    if (!ok) {
+      delete L;
+      return MOE_ERR_UNSUPPORTED;
+    }
+  }
+
+  // scratch arena
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off = align_up(off + bytes, 256);
+    return o;
+  };
+  const size_t o_wr = take((size_t)E * H * 2);
+  const size_t o_lg = take((size_t)MB * E * 4);
+  const size_t o_ti = take((size_t)MB * k * 4);
+  const size_t o_tw = take((size_t)MB * k * 4);
+  const size_t o_cn = take((size_t)E * 4);
+  const size_t o_of = take((size_t)(E + 1) * 4);
+  const size_t o_pi = take((size_t)MB * k * 4);
+  const size_t o_ac = take((size_t)E * 4);
+  const size_t o_na = take(4);
+  const size_t o_h = take((size_t)MB * k * I * 4);
+  const size_t o_y = take((size_t)MB * k * H * 4);
+  const size_t o_hs = take((size_t)MB * std::max(Is, 1) * 4);
+  const size_t o_ys = take((size_t)MB * H * 4);
+  const size_t o_rc = take(4);
+  const size_t o_tc = take((size_t)H * 4);
+  const size_t o_er = take(4);
+  const size_t o_xs = take((size_t)MB * H * 2);
+  const size_t o_rs = take((size_t)MB * H * 2);
+  const size_t o_os = take((size_t)MB * H * 2);
+  if (cudaMalloc(&L->arena, off) != cudaSuccess) {
+    cudaGetLastError();
+    delete L;
+    return MOE_ERR_OOM;
+  }
+  char* A = L->arena;
+  L->wr_t = reinterpret_cast<uint16_t*>(A + o_wr);
+  L->logits = reinterpret_cast<float*>(A + o_lg);
+  L->plan.topk_idx = reinterpret_cast<int32_t*>(A + o_ti);
+  L->plan.topk_w = reinterpret_cast<float*>(A + o_tw);
+  L->plan.counts = reinterpret_cast<int32_t*>(A + o_cn);
+  L->plan.offsets = reinterpret_cast<int32_t*>(A + o_of);
+  L->plan.pair_ids = reinterpret_cast<int32_t*>(A + o_pi);
+  L->plan.active = reinterpret_cast<int32_t*>(A + o_ac);
+  L->plan.n_active = reinterpret_cast<int32_t*>(A + o_na);
+  L->h = reinterpret_cast<float*>(A + o_h);
+  L->y = reinterpret_cast<float*>(A + o_y);
+  L->hs = reinterpret_cast<float*>(A + o_hs);
+  L->ys = reinterpret_cast<float*>(A + o_ys);
+  L->router_cnt = reinterpret_cast<int*>(A + o_rc);
+  L->tile_cnt = reinterpret_cast<int*>(A + o_tc);
+  L->err = reinterpret_cast<int*>(A + o_er);
+  L->x_stage = reinterpret_cast<uint16_t*>(A + o_xs);
+  L->res_stage = reinterpret_cast<uint16_t*>(A + o_rs);
+  L->out_stage = reinterpret_cast<uint16_t*>(A + o_os);
+
+  cudaError_t e = cudaMemset(L->arena, 0, off);
+  if (e == cudaSuccess) {
+    dim3 blk(32, 8), grd((E + 31) / 32, (H + 31) / 32);
+    transpose_u16_kernel<<<grd, blk>>>(static_cast<const uint16_t*>(w->router_w), L->wr_t, H, E);
+    e = cudaGetLastError();
+  }
+  if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&L->side, cudaStreamNonBlocking);
+  if (e == cudaSuccess) e = cudaEventCreateWithFlags(&L->ev_fork, cudaEventDisableTiming);
+  if (e == cudaSuccess) e = cudaEventCreateWithFlags(&L->ev_join, cudaEventDisableTiming);
+  for (int kk = 0; kk < K_NUM && e == cudaSuccess; ++kk)
+    for (int t = 0; t < 2 && e == cudaSuccess; ++t) {
+      const GemvPlan& p = L->plans[kk][t];
+      if (!p.ok) continue;
+      e = cudaFuncSetAttribute(gemv_fn((Kind)kk, p.rpg, t == 0 ? 1 : 2), cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               p.smem);
+    }
+  if (e == cudaSuccess) e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) {
+    moe_layer_destroy(L);
+    return MOE_ERR_CUDA;
+  }
+  *out = L;
+  return MOE_OK;
+}
+
+moe_status_t moe_layer_destroy(moe_layer_t L) {
+  if (!L) return MOE_OK;
+  if (L->side) cudaStreamSynchronize(L->side);
+  cudaDeviceSynchronize();
+  if (L->ev_fork) cudaEventDestroy(L->ev_fork);
+  if (L->ev_join) cudaEventDestroy(L->ev_join);
+  if (L->side) cudaStreamDestroy(L->side);
+  if (L->arena) cudaFree(L->arena);
+  delete L;
+  return MOE_OK;
+}
+
+moe_status_t moe_layer_routing(moe_layer_t L, moe_routing* out) {
+  if (!L || !out) return MOE_ERR_INVALID_ARG;
+  *out = L->plan;
+  return MOE_OK;
+}
+
+moe_status_t moe_router_topk(moe_layer_t L, const void* x, int B, const moe_routing* r, void* stream) {
+  moe_status_t s = check_call(L, B);
+  if (s != MOE_OK) return s;
+  if (!x || !aligned16(x)) return MOE_ERR_INVALID_ARG;
+  if (r && !routing_ok(r)) return MOE_ERR_INVALID_ARG;
+  const moe_routing& rr = r ? *r : L->plan;
+  return cuda_status(launch_router(L, x, B, rr, (cudaStream_t)stream));
+}
+
+moe_status_t moe_experts_mxfp4(moe_layer_t L, const void* x, int B, const moe_routing* r, float* y_routed,
+                               float* y_shared, void* stream) {
+  moe_status_t s = check_call(L, B);
+  if (s != MOE_OK) return s;
+  if (!x || !aligned16(x) || !y_routed || !aligned16(y_routed)) return MOE_ERR_INVALID_ARG;
+  if (L->cfg.shared_inter > 0 && (!y_shared || !aligned16(y_shared))) return MOE_ERR_INVALID_ARG;
+  if (r && !routing_ok(r)) return MOE_ERR_INVALID_ARG;
+  const moe_routing& rr = r ? *r : L->plan;
+  cudaStream_t st = (cudaStream_t)stream;
+  const bool has_shared = L->cfg.shared_inter > 0;
+  const bool fork = has_shared && L->side_stream;
+  cudaError_t e = cudaSuccess;
+  if (fork) {
+    e = cudaEventRecord(L->ev_fork, st);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(L->side, L->ev_fork, 0);
+    if (e == cudaSuccess) e = launch_shared(L, x, B, y_shared, L->side, false);
+    if (e == cudaSuccess) e = cudaEventRecord(L->ev_join, L->side);
+  }
+  if (e == cudaSuccess) e = launch_gate_up(L, x, B, rr, st);
+  if (e == cudaSuccess) e = launch_down(L, B, rr, y_routed, false, nullptr, nullptr, nullptr, nullptr, st, L->pdl);
+  if (e == cudaSuccess && has_shared && !fork) e = launch_shared(L, x, B, y_shared, st, L->pdl);
+  if (e == cudaSuccess && fork) e = cudaStreamWaitEvent(st, L->ev_join, 0);
+  return cuda_status(e);
+}
+
+moe_status_t moe_combine_residual(moe_layer_t L, int B, const moe_routing* r, const float* y_routed,
+                                  const float* y_shared, const void* residual, void* out, void* stream) {
+  moe_status_t s = check_call(L, B);
+  if (s != MOE_OK) return s;
+  if (!y_routed || !residual || !out || !aligned16(y_routed) || !aligned16(residual) || !aligned16(out))
+    return MOE_ERR_INVALID_ARG;
+  if (r && !routing_ok(r)) return MOE_ERR_INVALID_ARG;
+  const moe_routing& rr = r ? *r : L->plan;
+  return cuda_status(launch_combine(L, B, rr, y_routed, y_shared, residual, out, (cudaStream_t)stream));
+}
+
+moe_status_t moe_layer_forward(moe_layer_t L, moe_layer_t next, const void* x, const void* residual, void* out,
+                               int B, void* stream) {
+  moe_status_t s = check_call(L, B);
+  if (s != MOE_OK) return s;
+  if (!x || !residual || !out || !aligned16(x) || !aligned16(residual) || !aligned16(out))
+    return MOE_ERR_INVALID_ARG;
+  cudaStream_t st = (cudaStream_t)stream;
+  const bool has_shared = L->cfg.shared_inter > 0;
+  const bool fork = has_shared && L->side_stream;
+  cudaError_t e = cudaSuccess;
+  if (fork) {
+    e = cudaEventRecord(L->ev_fork, st);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(L->side, L->ev_fork, 0);
+    if (e == cudaSuccess) e = launch_shared(L, x, B, L->ys, L->side, false);
+    if (e == cudaSuccess) e = cudaEventRecord(L->ev_join, L->side);
+  }
+  if (e == cudaSuccess) e = launch_router(L, x, B, L->plan, st);
+  if (e == cudaSuccess && L->probe_start) e = cudaEventRecord(L->probe_start, st);
+  if (e == cudaSuccess) e = launch_gate_up(L, x, B, L->plan, st);
+  if (e == cudaSuccess && L->probe_stop) e = cudaEventRecord(L->probe_stop, st);
+  if (e == cudaSuccess && has_shared && !fork) e = launch_shared(L, x, B, L->ys, st, L->pdl);
+  if (e == cudaSuccess && fork) e = cudaStreamWaitEvent(st, L->ev_join, 0);
+  if (e == cudaSuccess)
+    e = launch_down(L, B, L->plan, L->y, true, residual, out, has_shared ? L->ys : nullptr, next, st,
+                    L->pdl && !fork);
+  return cuda_status(e);
+}
+
+moe_status_t moe_layer_forward_host(moe_layer_t L, const void* x_host, const void* residual_host, void* out_host,
+                                    int B, void* stream) {
+  moe_status_t s = check_call(L, B);
+  if (s != MOE_OK) return s;
+  if (!x_host || !residual_host || !out_host) return MOE_ERR_INVALID_ARG;
+  cudaStream_t st = (cudaStream_t)stream;
+  const size_t bytes = (size_t)B * L->cfg.hidden * 2;
+  cudaError_t e = cudaMemcpyAsync(L->x_stage, x_host, bytes, cudaMemcpyHostToDevice, st);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(L->res_stage, residual_host, bytes, cudaMemcpyHostToDevice, st);
+  if (e != cudaSuccess) return MOE_ERR_CUDA;
+  s = moe_layer_forward(L, nullptr, L->x_stage, L->res_stage, L->out_stage, B, stream);
+  if (s != MOE_OK) return s;
+  return cuda_status(cudaMemcpyAsync(out_host, L->out_stage, bytes, cudaMemcpyDeviceToHost, st));
+}
+
+moe_status_t moe_layer_last_device_error(moe_layer_t L) {
+  if (!L) return MOE_ERR_INVALID_ARG;
+  int v = 0;
+  if (cudaMemcpy(&v, L->err, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return MOE_ERR_CUDA;
+  if (v == 0) return MOE_OK;
+  // clear the word and the completion counters a cut-short launch may have left behind
+  cudaMemset(L->err, 0, sizeof(int));
+  cudaMemset(L->router_cnt, 0, sizeof(int));
+  cudaMemset(L->tile_cnt, 0, sizeof(int) * L->cfg.hidden);
+  return v == kErrTimeout ? MOE_ERR_TIMEOUT : MOE_ERR_INVALID_ARG;
+}
+
+moe_status_t moe_layer_set_probe(moe_layer_t L, void* start, void* stop) {
+  if (!L || ((start == nullptr) != (stop == nullptr))) return MOE_ERR_INVALID_ARG;
+  L->probe_start = (cudaEvent_t)start;
+  L->probe_stop = (cudaEvent_t)stop;
+  return MOE_OK;
+}
+
+}  // extern "C"

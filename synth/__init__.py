@@ -283,6 +283,8 @@ def _logit_gap(x_bf16_row, wr_f64, bias, k):
     lg = bf16_to_f32(x_bf16_row).astype(np.float64) @ wr_f64
     if bias is not None:
         lg = lg + bias.astype(np.float64)
+    if k >= lg.shape[0]:
+        return np.inf            # every expert is selected
     srt = np.sort(lg)[::-1]
     return srt[k - 1] - srt[k]
 

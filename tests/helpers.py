@@ -1,0 +1,34 @@
+"""Shared test helpers: tolerance metrics and oracle runs on device workloads."""
+import numpy as np
+
+from synth import bf16_to_f32
+
+# Layer output tolerance (bf16 [B][H]) stated for the layer:
+#   max|out - ref| <= 1e-2 * max|ref|  and  sum|out - ref| / sum|ref| <= 2e-3,
+# ref = the oracle's fp64 result rounded once to bf16.
+OUT_MAX_REL = 1e-2
+OUT_MEAN_REL = 2e-3
+# fp32 intermediates (unweighted expert outputs, shared-expert output) against
+# fp64: K-term fp32 dot products (K <= 7168) with per-block partial sums keep
+# the relative error near 1e-6; these bounds leave two orders of margin.
+Y_MAX_REL = 1e-4
+Y_MEAN_REL = 1e-5
+# routing weights: fp32 softmax of fp32 logits vs fp64 (|w| <= 1)
+W_ABS = 1e-5
+
+
+def bf16_close(gpu_u16, ref_u16, max_rel=OUT_MAX_REL, mean_rel=OUT_MEAN_REL):
+    g = bf16_to_f32(np.asarray(gpu_u16)).astype(np.float64)
+    r = bf16_to_f32(np.asarray(ref_u16)).astype(np.float64)
+    return metric_close(g, r, max_rel, mean_rel)
+
+
+def metric_close(g, r, max_rel, mean_rel):
+    g = np.asarray(g, dtype=np.float64)
+    r = np.asarray(r, dtype=np.float64)
+    assert g.shape == r.shape, (g.shape, r.shape)
+    assert np.all(np.isfinite(g)), "non-finite values in GPU output"
+    d = np.abs(g - r)
+    mx, mr = d.max(), d.sum() / max(np.abs(r).sum(), 1e-300)
+    ok = mx <= max_rel * np.abs(r).max() and mr <= mean_rel
+    return ok, dict(max_abs=float(mx), max_ref=float(np.abs(r).max()), mean_rel=float(mr))
