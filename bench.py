@@ -36,7 +36,7 @@ sys.path.insert(0, ROOT)
 METRIC = "MoE decode layer achieved HBM GB/s (counted bytes per layer-step / device time per layer-step)"
 UNIT = "GB/s"
 WORKLOAD_DEFAULT = 1
-POOL = 64  # distinct token batches cycled through the steps
+POOL = 64  # distinct token batches cycled through the steps (--pool)
 
 
 def parse_args():
@@ -48,6 +48,9 @@ def parse_args():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--flags", type=int, default=0, help="MOE_FLAG_* bits for ablations")
+    ap.add_argument("--experts", type=int, default=0,
+                    help="profiling aid: fewer routed experts (same per-step work, smaller footprint)")
+    ap.add_argument("--pool", type=int, default=64, help="distinct token batches cycled through the steps")
     return ap.parse_args()
 
 
@@ -337,7 +340,7 @@ def run_ours(args, cfg):
         "e2e": {"value": round(world * total_bytes / (e2e_total * 1e-3) / 1e9, 2), "unit": UNIT,
                 "h2d_bytes_per_step": 2 * B * H * 2, "d2h_bytes_per_step": B * H * 2,
                 "us_per_step": round(e2e_total / K * 1e3, 2)},
-        "gpu_launches": 5 * K,
+        "gpu_launches": 6 * K,  # router, top-k, gate/up, down+combine, shared gate/up, shared down
         "clocks": clocks,
     }
     if world == 1 and not args.no_cpu_baseline:
@@ -376,6 +379,10 @@ def main():
     args = parse_args()
     import synth
     cfg = synth.CONFIGS[args.config]
+    if args.experts:
+        cfg = cfg.with_(n_experts=args.experts, name=cfg.name + f"_E{args.experts}")
+    global POOL
+    POOL = args.pool
     if args.impl == "reference":
         run_reference(args, cfg)
     else:

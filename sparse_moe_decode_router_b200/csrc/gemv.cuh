@@ -1,0 +1,852 @@
+// Warp-item streaming GEMV for the MoE decode layer (sm_100a).
+//
+// Decode at batch <= 64 streams each active weight matrix from HBM once per
+// step and multiplies it with a handful of activation vectors.  The kernel:
+//
+//  * persistent CTAs, one per SM; each owns a contiguous range of work items
+//    (an item = R consecutive output rows of one group: one active expert,
+//    or the single dense group of the router / shared expert), sized so that
+//    each TMA copy moves 14-32 KB;
+//  * one producer lane moves every item's weight rows (codes, and for MXFP4
+//    the E8M0 scale rows) into a ring of shared-memory stages with 1-D TMA
+//    bulk copies (evict-first L2 policy: weights are read once per step);
+//    completion is counted on per-stage mbarriers;
+//  * an item is shared by a small group of warps, each owning whole rows:
+//    its lanes split K, so a row's dot product needs only an in-warp
+//    butterfly; warps never wait for each other in the steady state (the
+//    stage is handed back with one mbarrier arrive per warp, no CTA barrier);
+//  * the activation vectors an item needs sit in shared memory, staged once
+//    per "phase" (a run of groups whose tokens fit): MXFP4 streams keep them
+//    as f16 scaled by a per-vector power of two (exact for bf16 inputs,
+//    11-bit rounding for fp32 ones) in a lane-interleaved layout that makes
+//    every 16-byte read conflict-free; bf16 streams keep bf16 or fp32 as is;
+//  * MXFP4 weights are decoded in registers (cvt e2m1x2 -> f16x2) and fed to
+//    fp32-accumulating mixed-precision FMAs; each lane's 32-element chunk is
+//    one scale block, so the E8M0 scale is applied once per chunk in fp32;
+//  * epilogues: store, SwiGLU, router logits (+ bias; top-k follows in its own
+//    kernel), and the down projection fused with the
+//    routing-weight combine and residual add (the last warp to finish a row
+//    tile over all active experts sums that tile in ascending expert order).
+#pragma once
+#include <cstdint>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include "kernels.cuh"
+#include "ptx.cuh"
+
+namespace moe {
+
+enum XKind : int { X_BF16 = 0, X_F32 = 1 };
+
+#ifndef MOE_MAX_CONSUMER_WARPS
+#define MOE_MAX_CONSUMER_WARPS 12
+#endif
+constexpr int kMaxConsumerWarps = MOE_MAX_CONSUMER_WARPS;
+constexpr int kMaxStagesDev = 24;     // stage ring slots the shared-memory header reserves
+constexpr int kMaxStageUnits = 64;    // (vector, segment) units of one staging pass
+constexpr int kMaxPhases = 32;
+constexpr int kMaxSlots = 32;
+
+struct PhaseDesc {
+  int g0, g1;    // groups [g0, g1) (indices into the active list; 0..1 for dense)
+  int t0, t1;    // token range inside each group's token list (split groups only; else 0, INT_MAX)
+  int nslots;    // activation vectors staged for this phase
+  int first_item, last_item;  // CTA-local item range [first, last) of this phase
+};
+
+struct PhaseTable {
+  int n;
+  int bad;
+  PhaseDesc ph[kMaxPhases];
+  int slot_src[kMaxPhases][kMaxSlots];  // source row of each slot (token or pair)
+};
+
+// ---------------------------------------------------------------------------
+// mixed-precision FMAs: fp32 accumulator, two f16 (or bf16) products from packed pairs
+__device__ __forceinline__ float fma2_f16(uint32_t w2, uint32_t x2, float acc) {
+  asm("{\n\t.reg .f16 a0, a1, b0, b1;\n\t"
+      "mov.b32 {a0, a1}, %1;\n\t"
+      "mov.b32 {b0, b1}, %2;\n\t"
+      "fma.rn.f32.f16 %0, a0, b0, %0;\n\t"
+      "fma.rn.f32.f16 %0, a1, b1, %0;\n\t}"
+      : "+f"(acc)
+      : "r"(w2), "r"(x2));
+  return acc;
+}
+
+__device__ __forceinline__ float fma2_bf16(uint32_t w2, uint32_t x2, float acc) {
+  asm("{\n\t.reg .b16 a0, a1, b0, b1;\n\t"
+      "mov.b32 {a0, a1}, %1;\n\t"
+      "mov.b32 {b0, b1}, %2;\n\t"
+      "fma.rn.f32.bf16 %0, a0, b0, %0;\n\t"
+      "fma.rn.f32.bf16 %0, a1, b1, %0;\n\t}"
+      : "+f"(acc)
+      : "r"(w2), "r"(x2));
+  return acc;
+}
+
+// 32-element MXFP4 chunk (16 code bytes = 16 f16x2 after decode) dotted with a
+// 32-element f16 activation chunk (4 x 16 bytes, lane-interleaved), 4 chains.
+__device__ __forceinline__ float dot32_f16(const uint32_t (&w)[16], const uint4 (&xv)[4]) {
+  float p0 = 0.f, p1 = 0.f, p2 = 0.f, p3 = 0.f;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    p0 = fma2_f16(w[4 * q + 0], xv[q].x, p0);
+    p1 = fma2_f16(w[4 * q + 1], xv[q].y, p1);
+    p2 = fma2_f16(w[4 * q + 2], xv[q].z, p2);
+    p3 = fma2_f16(w[4 * q + 3], xv[q].w, p3);
+  }
+  return (p0 + p1) + (p2 + p3);
+}
+
+__device__ __forceinline__ void decode_chunk(const uint4 q, uint32_t (&w)[16]) {
+  uint32_t t[4];
+  e2m1x8_to_f16x2(q.x, t);
+  w[0] = t[0]; w[1] = t[1]; w[2] = t[2]; w[3] = t[3];
+  e2m1x8_to_f16x2(q.y, t);
+  w[4] = t[0]; w[5] = t[1]; w[6] = t[2]; w[7] = t[3];
+  e2m1x8_to_f16x2(q.z, t);
+  w[8] = t[0]; w[9] = t[1]; w[10] = t[2]; w[11] = t[3];
+  e2m1x8_to_f16x2(q.w, t);
+  w[12] = t[0]; w[13] = t[1]; w[14] = t[2]; w[15] = t[3];
+}
+
+// f16 activation layout in shared memory: element k of a K-vector, k = 32*b + 8*q + j
+// (chunk b = 32*i + l), lives at half index ((i*4 + q)*32 + l)*8 + j.  Lane l's q-th
+// 16-byte read of chunk b is then contiguous across the warp.
+__device__ __forceinline__ int xperm_index(int k) {
+  const int b = k >> 5, q = (k >> 3) & 3, j = k & 7;
+  const int i = b >> 5, l = b & 31;
+  return (((i * 4 + q) * 32 + l) << 3) + j;
+}
+
+// ---------------------------------------------------------------------------
+// Phase table: runs of groups whose activation vectors fit in `xcap` slots.
+// Built by one thread; `lo`/`hi` = the CTA's item range.
+__device__ void build_phases(const GemvArgs& a, long long lo, long long hi, int n_rt, int xcap,
+                             PhaseTable& pt) {
+  pt.n = 0;
+  pt.bad = 0;
+  if (lo >= hi) return;
+  if (!a.routed) {
+    // dense: token chunks of xcap, each over the whole item range
+    for (int t0 = 0; t0 < a.n_tokens; t0 += xcap) {
+      if (pt.n == kMaxPhases) { pt.bad = 1; return; }
+      PhaseDesc& p = pt.ph[pt.n];
+      p.g0 = 0; p.g1 = 1;
+      p.t0 = t0; p.t1 = min(a.n_tokens, t0 + xcap);
+      p.nslots = p.t1 - p.t0;
+      for (int s = 0; s < p.nslots; ++s) pt.slot_src[pt.n][s] = t0 + s;
+      p.first_item = 0;
+      p.last_item = (int)(hi - lo);
+      ++pt.n;
+    }
+    return;
+  }
+  const int gfirst = (int)(lo / n_rt), glast = (int)((hi - 1) / n_rt);
+  int cur = -1;  // open phase index
+  for (int g = gfirst; g <= glast; ++g) {
+    const int e = clamp_group(a.active[g], a.n_experts, nullptr);
+    const int b0 = a.offsets[e], cnt = a.offsets[e + 1] - b0;
+    const long long ilo = max(lo, (long long)g * n_rt), ihi = min(hi, (long long)(g + 1) * n_rt);
+    // activation rows this group needs
+    int need[kMaxSlots];
+    int nneed = 0;
+    bool split = false;
+    for (int t = 0; t < cnt; ++t) {
+      int p = a.pair_ids[b0 + t];
+      if (p < 0 || p >= a.n_pairs) p = 0;
+      const int src = a.act_by_pair ? p : p / a.top_k;
+      bool dup = false;
+      for (int u = 0; u < nneed; ++u) dup |= (need[u] == src);
+      if (!dup) {
+        if (nneed == xcap || nneed == kMaxSlots) { split = true; break; }
+        need[nneed++] = src;
+      }
+    }
+    if (split) {
+      // a group with more activation rows than slots: own phases, token chunks of xcap
+      cur = -1;
+      for (int t0 = 0; t0 < cnt; t0 += xcap) {
+        if (pt.n == kMaxPhases) { pt.bad = 1; return; }
+        PhaseDesc& p = pt.ph[pt.n];
+        p.g0 = g; p.g1 = g + 1;
+        p.t0 = t0; p.t1 = min(cnt, t0 + xcap);
+        p.nslots = 0;
+        for (int t = p.t0; t < p.t1; ++t) {
+          int pr = a.pair_ids[b0 + t];
+          if (pr < 0 || pr >= a.n_pairs) pr = 0;
+          pt.slot_src[pt.n][p.nslots++] = a.act_by_pair ? pr : pr / a.top_k;  // duplicates allowed
+        }
+        p.first_item = (int)(ilo - lo);
+        p.last_item = (int)(ihi - lo);
+        ++pt.n;
+      }
+      continue;
+    }
+    // try to extend the open phase with this group's new rows
+    if (cur >= 0) {
+      PhaseDesc& p = pt.ph[cur];
+      int add = 0;
+      for (int u = 0; u < nneed; ++u) {
+        bool have = false;
+        for (int s = 0; s < p.nslots; ++s) have |= (pt.slot_src[cur][s] == need[u]);
+        add += !have;
+      }
+      if (p.nslots + add <= xcap) {
+        for (int u = 0; u < nneed; ++u) {
+          bool have = false;
+          for (int s = 0; s < p.nslots; ++s) have |= (pt.slot_src[cur][s] == need[u]);
+          if (!have) pt.slot_src[cur][p.nslots++] = need[u];
+        }
+        p.g1 = g + 1;
+        p.last_item = (int)(ihi - lo);
+        continue;
+      }
+    }
+    if (pt.n == kMaxPhases) { pt.bad = 1; return; }
+    cur = pt.n++;
+    PhaseDesc& p = pt.ph[cur];
+    p.g0 = g; p.g1 = g + 1;
+    p.t0 = 0; p.t1 = 1 << 30;
+    p.nslots = nneed;
+    for (int u = 0; u < nneed; ++u) pt.slot_src[cur][u] = need[u];
+    p.first_item = (int)(ilo - lo);
+    p.last_item = (int)(ihi - lo);
+  }
+}
+
+// 2^e as an exact fp32 (e clamped to the normal range).
+__device__ __forceinline__ float pow2f(int e) {
+  e = max(-126, min(127, e));
+  return __uint_as_float((uint32_t)(e + 127) << 23);
+}
+
+// Staging of activation vectors into shared memory.  MXFP4 streams: f16 of
+// x * 2^-e in the lane-interleaved layout, e chosen from max|x| so that the
+// largest element sits in [2^14, 2^15) (exact for bf16 inputs, one rounding
+// for fp32 ones).  bf16 streams: a plain copy of the bf16 or fp32 row.
+// Work is split into (vector, segment) units over all consumer warps; all
+// loads are 16-byte vectors with several in flight.
+
+// max |x| over 8-element groups [g0, g1) of row `row`
+template <int XK>
+__device__ float segment_amax(const void* src_base, int row, int K, int g0, int g1, int lane) {
+  float amax = 0.f;
+  if constexpr (XK == X_F32) {
+    const float4* s = reinterpret_cast<const float4*>(static_cast<const float*>(src_base) + (size_t)row * K);
+#pragma unroll 4
+    for (int g = g0 + lane; g < g1; g += 32) {
+      const float4 v0 = __ldcg(s + 2 * g), v1 = __ldcg(s + 2 * g + 1);
+      amax = fmaxf(amax, fmaxf(fmaxf(fabsf(v0.x), fabsf(v0.y)), fmaxf(fabsf(v0.z), fabsf(v0.w))));
+      amax = fmaxf(amax, fmaxf(fmaxf(fabsf(v1.x), fabsf(v1.y)), fmaxf(fabsf(v1.z), fabsf(v1.w))));
+    }
+  } else {
+    const uint4* s = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(src_base) + (size_t)row * K);
+#pragma unroll 4
+    for (int g = g0 + lane; g < g1; g += 32) {
+      const uint4 v = __ldg(s + g);
+      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) amax = fmaxf(amax, fmaxf(fabsf(bf16lo_to_f32(w[j])), fabsf(bf16hi_to_f32(w[j]))));
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
+  return amax;
+}
+
+// 8-element groups [g0, g1) of row `row` -> f16 * 2^-e, interleaved layout
+template <int XK>
+__device__ void segment_to_f16(const void* src_base, int row, int K, int g0, int g1, float scale, unsigned char* dst,
+                               int lane) {
+#pragma unroll 4
+  for (int g = g0 + lane; g < g1; g += 32) {
+    float v[8];
+    if constexpr (XK == X_F32) {
+      const float4* s = reinterpret_cast<const float4*>(static_cast<const float*>(src_base) + (size_t)row * K);
+      const float4 v0 = __ldcg(s + 2 * g), v1 = __ldcg(s + 2 * g + 1);
+      v[0] = v0.x; v[1] = v0.y; v[2] = v0.z; v[3] = v0.w; v[4] = v1.x; v[5] = v1.y; v[6] = v1.z; v[7] = v1.w;
+    } else {
+      const uint4* s = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(src_base) + (size_t)row * K);
+      const uint4 u = __ldg(s + g);
+      const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        v[2 * j] = bf16lo_to_f32(w[j]);
+        v[2 * j + 1] = bf16hi_to_f32(w[j]);
+      }
+    }
+    uint32_t hv[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const __half2 h2 = __floats2half2_rn(v[2 * j] * scale, v[2 * j + 1] * scale);
+      hv[j] = *reinterpret_cast<const uint32_t*>(&h2);
+    }
+    // 8 consecutive elements k = 8g .. 8g+7 stay contiguous in the interleaved layout
+    *reinterpret_cast<uint4*>(dst + 2 * xperm_index(8 * g)) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
+  }
+}
+
+__device__ __forceinline__ int shift_for_amax(float amax) {
+  int e = 0;
+  if (amax > 0.f && amax < INFINITY) {
+    const int ef = (int)((__float_as_uint(amax) >> 23) & 0xFF);
+    e = (ef > 0 ? ef - 127 : -127) - 14;  // floor(log2(amax)) - 14
+    e = max(-126, min(127, e));
+  }
+  return e;
+}
+
+template <int WF, int XK>
+__device__ void stage_phase(const void* src, const int* slot_src, int nslots, int K, unsigned char* xbuf,
+                            int xrow_bytes, int* slot_e, float* s_amax, int warp, int ncw, int lane, int nct) {
+  if (nslots <= 0) return;
+  const int ngrp = K >> 3;
+  int nseg = max(1, ncw / nslots);
+  nseg = min(nseg, max(1, kMaxStageUnits / nslots));
+  const int seglen = (ngrp + nseg - 1) / nseg;
+  const int units = nslots * nseg;
+  if constexpr (WF == W_MXFP4) {
+    for (int u = warp; u < units; u += ncw) {
+      const int sl = u / nseg, q = u - sl * nseg;
+      const float m = segment_amax<XK>(src, slot_src[sl], K, q * seglen, min(ngrp, (q + 1) * seglen), lane);
+      if (lane == 0) s_amax[u] = m;
+    }
+    named_bar_sync(1, nct);
+    for (int u = warp; u < units; u += ncw) {
+      const int sl = u / nseg, q = u - sl * nseg;
+      float m = 0.f;
+      for (int i = 0; i < nseg; ++i) m = fmaxf(m, s_amax[sl * nseg + i]);
+      const int e = shift_for_amax(m);
+      if (lane == 0 && q == 0) slot_e[sl] = e;
+      segment_to_f16<XK>(src, slot_src[sl], K, q * seglen, min(ngrp, (q + 1) * seglen), pow2f(-e),
+                         xbuf + (size_t)sl * xrow_bytes, lane);
+    }
+  } else {
+    const int esz = (XK == X_F32) ? 4 : 2;
+    const int n16 = K * esz / 16;
+    const int seg16 = (n16 + nseg - 1) / nseg;
+    for (int u = warp; u < units; u += ncw) {
+      const int sl = u / nseg, q = u - sl * nseg;
+      const uint4* s = reinterpret_cast<const uint4*>(static_cast<const unsigned char*>(src) +
+                                                      (size_t)slot_src[sl] * K * esz);
+      uint4* d = reinterpret_cast<uint4*>(xbuf + (size_t)sl * xrow_bytes);
+      const int i1 = min(n16, (q + 1) * seg16);
+#pragma unroll 4
+      for (int i = q * seg16 + lane; i < i1; i += 32) d[i] = (XK == X_F32) ? __ldcg(s + i) : __ldg(s + i);
+      if (lane == 0 && q == 0) slot_e[sl] = 0;
+    }
+  }
+}
+
+// Bytes of one staged activation vector (MXFP4 streams: whole groups of 32
+// chunks in the interleaved f16 layout).
+__host__ __device__ constexpr int x_row_bytes(int wf, int xk, int K) {
+  return wf == W_MXFP4 ? ((K / 32 + 31) / 32) * 2048 : K * (xk == X_F32 ? 4 : 2);
+}
+
+// ---------------------------------------------------------------------------
+// Fused combine bookkeeping.  A warp group writes the unweighted expert
+// outputs y of its items to the scratch; every kPubBatch items it meets on a
+// group barrier (all of the group's y stores are then ordered before the
+// leader's fence), the leader issues one gpu-scope fence and one tile-counter
+// atomic per item (lanes in parallel).  The atomics' results are examined one
+// batch later (settle), so their latency hides behind the next batch: the
+// item that brings a row tile's count to the number of active experts makes
+// its warp combine that tile in ascending expert order.
+constexpr int kPubBatch = 8;
+
+__device__ __forceinline__ void group_bar(int q0, int wpi) {
+  named_bar_sync(3 + q0, wpi * 32);
+}
+
+__device__ void settle_batch(const GemvArgs& a, int prev_cnt, int prev_rt, int nprev, int n_groups, int wi,
+                             int lane) {
+  if (wi != 0) return;
+  const unsigned ready = __ballot_sync(0xFFFFFFFFu, lane < nprev && prev_cnt == n_groups - 1);
+  if (!ready) return;
+  __threadfence();
+  const int H = a.out_rows;
+  for (unsigned m = ready; m; m &= m - 1) {
+    const int src = __ffs(m) - 1;
+    const int rt = __shfl_sync(0xFFFFFFFFu, prev_rt, src);
+    for (int q = lane; q < a.batch * a.R; q += 32) {
+      const int b = q / a.R, r = rt * a.R + (q - (q / a.R) * a.R);
+      a.out_bf16[(size_t)b * H + r] = combine_one(a, a.out, H, b, r);
+    }
+    if (lane == 0) a.tile_counter[rt] = 0;
+  }
+}
+
+__device__ void publish_batch(const GemvArgs& a, const int* pend_rt, int npend, int& prev_cnt, int& prev_rt,
+                              int& nprev, int n_groups, int wi, int q0, int lane) {
+  group_bar(q0, a.wpi);  // every warp of the group has written its y rows of these items
+  if (wi != 0) return;
+  // results of the previous batch first (their atomics have long completed)
+  if (nprev > 0) settle_batch(a, prev_cnt, prev_rt, nprev, n_groups, wi, lane);
+  __threadfence();
+  int rt = 0;
+#pragma unroll
+  for (int i = 0; i < kPubBatch; ++i)
+    if (lane == i) rt = pend_rt[i];
+  prev_rt = rt;
+  prev_cnt = (lane < npend) ? atomicAdd(&a.tile_counter[rt], 1) : -1;
+  nprev = npend;
+}
+
+// ---------------------------------------------------------------------------
+// Per-item token list: up to TMAX (slot, output row, exponent) per pass.
+struct TokenPass {
+  int n;
+  int slot[4];
+  int orow[4];
+  int e[4];
+};
+
+// RPW = output rows per warp (SwiGLU: one gate row and one up row per output row).
+// An item (R = RPW * wpi output rows, one stage) is shared by a group of wpi warps.
+template <int WF, int EPI, int XK, int TMAX, int RPW>
+__global__ void __launch_bounds__(kMaxConsumerWarps * 32 + 32, 1) gemv_kernel(const GemvArgs a) {
+  constexpr bool kSwiglu = (EPI == EPI_SWIGLU);
+  constexpr int NWR = kSwiglu ? 2 * RPW : RPW;  // weight rows per warp
+  static_assert(NWR % 2 == 0, "rows are processed in pairs");
+  extern __shared__ __align__(128) unsigned char smem[];
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int ncw = a.ncw;
+  const int K = a.K;
+  const int C = K >> 5;                                   // 32-element chunks per row
+  const int rowbytes = (WF == W_MXFP4) ? (K >> 1) : (K << 1);
+  const int sblocks = K >> 5;
+  const int rows_per_item = kSwiglu ? 2 * a.R : a.R;
+  const int codes_bytes = rows_per_item * rowbytes;
+  const int xrow_bytes = x_row_bytes(WF, XK, K);
+
+  // shared memory: [barriers][phase table][slot exponents][x slots][stages]
+  uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem);
+  uint64_t* empty_bar = full_bar + a.n_stages;
+  PhaseTable* pt = reinterpret_cast<PhaseTable*>(smem + 16 * 64);
+  int* slot_e = reinterpret_cast<int*>(smem + 16 * 64 + sizeof(PhaseTable));
+  volatile int* s_flag = slot_e + kMaxSlots;
+  int* s_item_cnt = slot_e + kMaxSlots + 2;  // [n_stages] warps done with the item in that stage
+  float* s_amax = reinterpret_cast<float*>(s_item_cnt + kMaxStagesDev);  // [kMaxStageUnits] staging partial maxima
+  unsigned char* xbuf = smem + a.x_offset;
+  unsigned char* stages = smem + a.stage_offset;
+
+  if (tid == 0) {
+    for (int s = 0; s < a.n_stages; ++s) {
+      mbar_init(&full_bar[s], 1);
+      mbar_init(&empty_bar[s], a.wpi);
+    }
+    s_flag[0] = 0;  // abort: set by any wait that gives up; every loop then drains without work
+    s_flag[1] = 0;
+    for (int q = 0; q < a.n_stages; ++q) s_item_cnt[q] = 0;
+    fence_barrier_init();
+  }
+  const bool producer = (warp == ncw);
+  // Routed streams depend on the routing plan: everyone waits for the previous
+  // grid first.  Dense streams only need it for their activations, so their
+  // producer starts on the (static) weights right away.
+  if (a.routed) pdl_wait();
+
+  int n_groups = a.routed ? *a.n_active : 1;
+  if (n_groups < 0 || n_groups > a.n_experts) {
+    if (tid == 0) atomicExch(a.err, kErrBadPlan);
+    n_groups = n_groups < 0 ? 0 : a.n_experts;
+  }
+  const int n_rt = a.out_rows / a.R;
+  const long long n_items = (long long)n_groups * n_rt;
+  const long long lo = n_items * blockIdx.x / gridDim.x;
+  const long long hi = n_items * (blockIdx.x + 1) / gridDim.x;
+
+  __syncthreads();  // barriers initialised
+  // plan invariant (see the host planner): stages are a multiple of the warp groups
+  if ((a.ncw % a.wpi) != 0 || (a.n_stages % (a.ncw / a.wpi)) != 0) {
+    if (tid == 0) atomicExch(a.err, kErrBadPlan);
+    return;
+  }
+  // The producer lane builds the phase table and starts streaming at once; the
+  // consumers wait for the table on named barrier 2 (the producer only arrives).
+  const int nthreads_all = (ncw + 1) * 32;
+  if (producer) {
+    if (lane == 0) {
+      build_phases(a, lo, hi, n_rt, a.xcap, *pt);
+      if (pt->bad) atomicExch(a.err, kErrBadPlan);
+    }
+    __syncwarp();
+    asm volatile("bar.arrive 2, %0;" ::"r"(nthreads_all) : "memory");
+  } else {
+    if (!a.routed) pdl_wait();
+    named_bar_sync(2, nthreads_all);
+  }
+
+  if (producer) {
+    if (lane == 0) {
+      const uint64_t pol = l2_policy_evict_first();
+      int s = 0;
+      uint32_t ph = 0;
+      bool ok = true;
+      int pg = -1, pgrp = 0;  // cached group -> expert lookup
+      for (int p = 0; p < pt->n && ok; ++p) {
+        const int jbeg = pt->ph[p].first_item, jend = pt->ph[p].last_item;
+        int g = (int)((lo + jbeg) / n_rt);
+        int rt = (int)((lo + jbeg) - (long long)g * n_rt);
+        for (int j = jbeg; j < jend; ++j, (++rt == n_rt ? (rt = 0, ++g) : 0)) {
+          if (s_flag[0] || !mbar_wait_bounded(&empty_bar[s], ph ^ 1u)) {
+            if (!s_flag[0]) atomicExch(a.err, kErrTimeout);
+            s_flag[0] = 1;
+            ok = false;
+            break;
+          }
+          if (g != pg) {
+            pg = g;
+            pgrp = a.routed ? clamp_group(a.active[g], a.n_experts, a.err) : 0;
+          }
+          const int grp = pgrp;
+          const int r0 = rt * a.R;
+          unsigned char* st = stages + (size_t)s * a.stage_bytes;
+          const uint32_t cb = (uint32_t)(a.R * rowbytes);
+          const uint32_t sb = (WF == W_MXFP4 && !a.scales_global) ? (uint32_t)(a.R * sblocks) : 0u;
+          mbar_arrive_expect_tx(&full_bar[s], (kSwiglu ? 2u : 1u) * (cb + sb));
+          const uint8_t* wg = a.w + (long long)grp * a.w_gstride;
+          bulk_g2s(st, wg + (size_t)r0 * rowbytes, cb, &full_bar[s], pol);
+          if (kSwiglu) bulk_g2s(st + cb, wg + (size_t)(r0 + a.up_off) * rowbytes, cb, &full_bar[s], pol);
+          if (WF == W_MXFP4 && !a.scales_global) {
+            const uint8_t* sg = a.sc + (long long)grp * a.s_gstride;
+            bulk_g2s(st + codes_bytes, sg + (size_t)r0 * sblocks, sb, &full_bar[s], pol);
+            if (kSwiglu)
+              bulk_g2s(st + codes_bytes + sb, sg + (size_t)(r0 + a.up_off) * sblocks, sb, &full_bar[s], pol);
+          }
+          if (++s == a.n_stages) { s = 0; ph ^= 1u; }
+        }
+      }
+      if (!ok) {
+        // let copies already in flight land before the CTA can exit
+        for (int q = 0; q < a.n_stages; ++q) {
+          (void)mbar_wait_bounded(&full_bar[q], 0u, 1ll << 24);
+          (void)mbar_wait_bounded(&full_bar[q], 1u, 1ll << 24);
+        }
+      }
+    }
+  } else {
+    // ------------------------------ consumers ------------------------------
+    const int nct = ncw * 32;
+    long long jglob = 0;  // CTA-local item counter across phases (stage ring position)
+    for (int p = 0; p < pt->n; ++p) {
+      const PhaseDesc ph = pt->ph[p];
+      // stage this phase's activation vectors, each split over several warps
+      named_bar_sync(1, nct);
+      stage_phase<WF, XK>(a.act, &pt->slot_src[p][0], ph.nslots, K, xbuf, xrow_bytes, slot_e, s_amax, warp, ncw,
+                          lane, nct);
+      named_bar_sync(1, nct);
+      const int nit = ph.last_item - ph.first_item;
+      int c_g = -1, c_grp = 0, c_tok0 = 0, c_ntok = 1, c_tp_tb = -1;
+      int pend_rt[kPubBatch], npend = 0;  // fused combine: items written, not yet published
+      int prev_cnt = 0, prev_rt = 0, nprev = 0;  // last published batch: atomic result per lane
+      (void)pend_rt; (void)npend; (void)prev_cnt; (void)prev_rt; (void)nprev;
+      TokenPass tp;
+      tp.n = 0;
+      const int ng = ncw / a.wpi;          // warp groups, one item each at a time
+      const int q0 = warp / a.wpi;         // this warp's group
+      const int wi = warp - q0 * a.wpi;    // this warp's share of the item
+      int g = (int)((lo + ph.first_item + q0) / n_rt);
+      int rt = (int)((lo + ph.first_item + q0) - (long long)g * n_rt);
+      for (int jj = q0; jj < nit; jj += ng) {
+        if (jj != q0) {  // advance (g, rt) by ng items
+          rt += ng;
+          while (rt >= n_rt) { rt -= n_rt; ++g; }
+        }
+        const bool skip = s_flag[0] != 0;  // aborting: no work, but every barrier is still met
+        const long long jl = jglob + jj;
+        const int s = (int)(jl % a.n_stages);
+        const uint32_t par = (uint32_t)((jl / a.n_stages) & 1);
+        // group and token list: looked up once per group change, kept in registers
+        if (g != c_g) {
+          c_g = g;
+          c_grp = a.routed ? clamp_group(a.active[g], a.n_experts, nullptr) : 0;
+          c_tok0 = 0;
+          c_ntok = a.n_tokens;
+          if (a.routed) {
+            c_tok0 = a.offsets[c_grp];
+            c_ntok = a.offsets[c_grp + 1] - c_tok0;
+            if (c_tok0 < 0 || c_ntok < 1 || c_tok0 + c_ntok > a.n_pairs) {
+              if (lane == 0) atomicExch(a.err, kErrBadPlan);
+              c_tok0 = 0;
+              c_ntok = 1;
+            }
+          }
+          c_tp_tb = -1;
+        }
+        const int grp = c_grp, tok0 = c_tok0, ntok = c_ntok;
+        const int tlo = a.routed ? max(0, ph.t0) : ph.t0;
+        const int thi = a.routed ? min(ntok, ph.t1) : ph.t1;
+
+        bool have = !skip;
+        if (have && !mbar_wait_bounded(&full_bar[s], par)) {
+          if (lane == 0) atomicExch(a.err, kErrTimeout);
+          s_flag[0] = 1;
+          have = false;
+        }
+        const unsigned char* st = stages + (size_t)s * a.stage_bytes;
+        for (int tb = tlo; have && tb < thi; tb += TMAX) {
+          if (tb != c_tp_tb) {
+          c_tp_tb = tb;
+          tp.n = min(TMAX, thi - tb);
+#pragma unroll
+          for (int t = 0; t < TMAX; ++t) {
+            const int tt = min(tb + t, thi - 1);
+            int src, orow;
+            if (a.routed) {
+              int pr = a.pair_ids[tok0 + tt];
+              if (pr < 0 || pr >= a.n_pairs) pr = 0;
+              src = a.act_by_pair ? pr : pr / a.top_k;
+              orow = pr;
+            } else {
+              src = tt;
+              orow = tt;
+            }
+            int sl = 0;
+            for (int u = 0; u < ph.nslots; ++u)
+              if (pt->slot_src[p][u] == src) sl = u;
+            tp.slot[t] = sl;
+            tp.orow[t] = orow;
+            tp.e[t] = slot_e[sl];
+          }
+          }
+          float acc[NWR][TMAX];
+#pragma unroll
+          for (int r = 0; r < NWR; ++r)
+#pragma unroll
+            for (int t = 0; t < TMAX; ++t) acc[r][t] = 0.f;
+
+          // stage rows handled by this warp
+          int srow[NWR];
+#pragma unroll
+          for (int r = 0; r < NWR; ++r)
+            srow[r] = kSwiglu ? (r < RPW ? wi * RPW + r : a.R + wi * RPW + (r - RPW)) : wi * RPW + r;
+          if constexpr (WF == W_MXFP4) {
+            // scale rows: in the stage after the codes, or (short rows) straight from global
+            const uint8_t* scl = st + codes_bytes;
+            const uint8_t* sgl = a.sc + (long long)grp * a.s_gstride;
+            const int r0 = rt * a.R;
+            int gsrow[NWR];  // global row of each stage row (scales read from global)
+#pragma unroll
+            for (int r = 0; r < NWR; ++r)
+              gsrow[r] = kSwiglu && srow[r] >= a.R ? r0 + a.up_off + srow[r] - a.R : r0 + srow[r];
+            if (TMAX == 1 && NWR >= 4) {
+              // one activation vector, several rows: each chunk's loads (activations,
+              // every row's codes and scale bytes) go out together, then the rows
+              const unsigned char* xs = xbuf + (size_t)tp.slot[0] * xrow_bytes;
+              for (int b = lane; b < C; b += 32) {
+                const int ii = b >> 5;
+                uint4 xv[4], cv[NWR];
+                uint32_t sv[NWR];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) xv[q] = lds128(xs + ((((ii * 4 + q) * 32) + lane) << 4));
+#pragma unroll
+                for (int r = 0; r < NWR; ++r) {
+                  cv[r] = lds128(st + (size_t)srow[r] * rowbytes + 16 * b);
+                  sv[r] = a.scales_global ? (uint32_t)__ldg(sgl + (size_t)gsrow[r] * sblocks + b)
+                                          : lds_u8(scl + srow[r] * sblocks + b);
+                }
+#pragma unroll
+                for (int r = 0; r < NWR; ++r) {
+                  uint32_t w[16];
+                  decode_chunk(cv[r], w);
+                  acc[r][0] = fmaf(dot32_f16(w, xv), e8m0_to_f32(sv[r]), acc[r][0]);
+                }
+              }
+            } else if (TMAX == 1) {
+              // one activation vector: a two-deep software pipeline, the next
+              // chunk's activations, codes and scale bytes are loaded before
+              // this chunk is computed
+              const unsigned char* xs = xbuf + (size_t)tp.slot[0] * xrow_bytes;
+              uint4 xv[4], cv[NWR];
+              uint32_t sv[NWR];
+              auto load_chunk = [&](int bb, uint4 (&xo)[4], uint4 (&co)[NWR], uint32_t (&so)[NWR]) {
+                const int ii = bb >> 5;
+#pragma unroll
+                for (int q = 0; q < 4; ++q) xo[q] = lds128(xs + ((((ii * 4 + q) * 32) + lane) << 4));
+#pragma unroll
+                for (int r = 0; r < NWR; ++r) {
+                  co[r] = lds128(st + (size_t)srow[r] * rowbytes + 16 * bb);
+                  so[r] = a.scales_global ? (uint32_t)__ldg(sgl + (size_t)gsrow[r] * sblocks + bb)
+                                          : lds_u8(scl + srow[r] * sblocks + bb);
+                }
+              };
+              if (lane < C) load_chunk(lane, xv, cv, sv);
+              for (int b = lane; b < C; b += 32) {
+                uint4 xn[4], cn[NWR];
+                uint32_t sn[NWR];
+                if (b + 32 < C) load_chunk(b + 32, xn, cn, sn);
+#pragma unroll
+                for (int r = 0; r < NWR; ++r) {
+                  uint32_t w[16];
+                  decode_chunk(cv[r], w);
+                  acc[r][0] = fmaf(dot32_f16(w, xv), e8m0_to_f32(sv[r]), acc[r][0]);
+                }
+                if (b + 32 < C) {
+#pragma unroll
+                  for (int q = 0; q < 4; ++q) xv[q] = xn[q];
+#pragma unroll
+                  for (int r = 0; r < NWR; ++r) {
+                    cv[r] = cn[r];
+                    sv[r] = sn[r];
+                  }
+                }
+              }
+            } else
+            for (int b = lane; b < C; b += 32) {
+              const int i = b >> 5;
+#pragma unroll
+              for (int t = 0; t < TMAX; ++t) {
+                if (t < tp.n) {
+                  // the activation chunk once, then every row of this warp one at a time
+                  const unsigned char* xs = xbuf + (size_t)tp.slot[t] * xrow_bytes;
+                  uint4 xv[4];
+#pragma unroll
+                  for (int q = 0; q < 4; ++q) xv[q] = lds128(xs + ((((i * 4 + q) * 32) + lane) << 4));
+#pragma unroll
+                  for (int r = 0; r < NWR; ++r) {
+                    uint32_t w[16];
+                    decode_chunk(lds128(st + (size_t)srow[r] * rowbytes + 16 * b), w);
+                    const float sc = a.scales_global ? e8m0_to_f32(__ldg(sgl + (size_t)gsrow[r] * sblocks + b))
+                                                     : e8m0_to_f32(lds_u8(scl + srow[r] * sblocks + b));
+                    acc[r][t] = fmaf(dot32_f16(w, xv), sc, acc[r][t]);
+                  }
+                }
+              }
+            }
+          } else {
+            // bf16 weights: lane owns 8-element (16-byte) chunks, contiguous across the warp
+            const int c8 = K >> 3;
+            for (int b8 = lane; b8 < c8; b8 += 32) {
+#pragma unroll
+              for (int rp = 0; rp < NWR; rp += 2) {
+                const uint4 qa = lds128(st + (size_t)srow[rp] * rowbytes + 16 * b8);
+                const uint4 qb = lds128(st + (size_t)srow[rp + 1] * rowbytes + 16 * b8);
+#pragma unroll
+                for (int t = 0; t < TMAX; ++t) {
+                  if (t < tp.n) {
+                    const unsigned char* xs = xbuf + (size_t)tp.slot[t] * xrow_bytes;
+                    if constexpr (XK == X_BF16) {
+                      const uint4 xv = lds128(xs + 16 * b8);
+                      float pa = 0.f, pb = 0.f;
+                      pa = fma2_bf16(qa.x, xv.x, pa); pb = fma2_bf16(qb.x, xv.x, pb);
+                      pa = fma2_bf16(qa.y, xv.y, pa); pb = fma2_bf16(qb.y, xv.y, pb);
+                      pa = fma2_bf16(qa.z, xv.z, pa); pb = fma2_bf16(qb.z, xv.z, pb);
+                      pa = fma2_bf16(qa.w, xv.w, pa); pb = fma2_bf16(qb.w, xv.w, pb);
+                      acc[rp][t] += pa;
+                      acc[rp + 1][t] += pb;
+                    } else {
+                      const uint4 x0 = lds128(xs + 32 * b8), x1 = lds128(xs + 32 * b8 + 16);
+                      const float xf[8] = {__uint_as_float(x0.x), __uint_as_float(x0.y), __uint_as_float(x0.z),
+                                           __uint_as_float(x0.w), __uint_as_float(x1.x), __uint_as_float(x1.y),
+                                           __uint_as_float(x1.z), __uint_as_float(x1.w)};
+                      const uint32_t wa[4] = {qa.x, qa.y, qa.z, qa.w}, wb[4] = {qb.x, qb.y, qb.z, qb.w};
+                      float pa = 0.f, pb = 0.f;
+#pragma unroll
+                      for (int j = 0; j < 4; ++j) {
+                        pa = fmaf(bf16lo_to_f32(wa[j]), xf[2 * j], pa);
+                        pa = fmaf(bf16hi_to_f32(wa[j]), xf[2 * j + 1], pa);
+                        pb = fmaf(bf16lo_to_f32(wb[j]), xf[2 * j], pb);
+                        pb = fmaf(bf16hi_to_f32(wb[j]), xf[2 * j + 1], pb);
+                      }
+                      acc[rp][t] += pa;
+                      acc[rp + 1][t] += pb;
+                    }
+                  }
+                }
+              }
+            }
+          }
+          if (tb + TMAX >= thi) {
+            // the stage is no longer read: hand it back to the producer
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty_bar[s]);
+          }
+          // --- reduce across the warp ---
+          constexpr int V = NextPow2<NWR * TMAX>::value;
+          float v[V];
+#pragma unroll
+          for (int q = 0; q < V; ++q) v[q] = 0.f;
+#pragma unroll
+          for (int r = 0; r < NWR; ++r)
+#pragma unroll
+            for (int t = 0; t < TMAX; ++t) v[r * TMAX + t] = acc[r][t];
+          const float tot = warp_reduce_multi<V>(v, lane);
+          // lane L holds value L / (32 / V); gather what the epilogue lanes need
+          const int vi = lane / (32 / V);
+          float mine = tot;
+          // --- epilogue: lanes 0 .. (outputs-1) ---
+          const int nout = RPW * TMAX;
+          const int oi = lane;  // output index handled by this lane
+          const int rr = oi / TMAX, t = oi - (oi / TMAX) * TMAX;
+          const float g_or_y = __shfl_sync(0xFFFFFFFFu, mine, (rr * TMAX + t) * (32 / V) & 31);
+          const float up = __shfl_sync(0xFFFFFFFFu, mine, ((RPW + rr) * TMAX + t) * (32 / V) & 31);
+          (void)vi;
+          if (oi < nout && t < tp.n) {
+            int et = tp.e[0], orow_t = tp.orow[0];
+#pragma unroll
+            for (int q = 1; q < TMAX; ++q)
+              if (t == q) { et = tp.e[q]; orow_t = tp.orow[q]; }
+            const int row = rt * a.R + wi * RPW + rr;
+            float val;
+            if constexpr (kSwiglu) {
+              const float gg = (WF == W_MXFP4) ? g_or_y * pow2f(et) : g_or_y;
+              const float uu = (WF == W_MXFP4) ? up * pow2f(et) : up;
+              val = gg / (1.0f + expf(-gg)) * uu;
+            } else {
+              val = (WF == W_MXFP4) ? g_or_y * pow2f(et) : g_or_y;
+              if constexpr (EPI == EPI_ROUTER) {
+                if (a.bias) val += a.bias[row];
+              }
+            }
+            a.out[(size_t)orow_t * a.out_rows + row] = val;
+          }
+        }
+        if constexpr (EPI == EPI_DOWN_COMBINE) {
+          // publish in batches: see publish_batch()
+          pend_rt[npend++] = rt;
+          if (npend == kPubBatch) {
+            publish_batch(a, pend_rt, npend, prev_cnt, prev_rt, nprev, n_groups, wi, q0, lane);
+            npend = 0;
+          }
+        }
+      }
+      if constexpr (EPI == EPI_DOWN_COMBINE) {
+        // end of phase: publish what is left, then settle the last results
+        if (npend > 0) publish_batch(a, pend_rt, npend, prev_cnt, prev_rt, nprev, n_groups, wi, q0, lane);
+        npend = 0;
+        if (nprev > 0) settle_batch(a, prev_cnt, prev_rt, nprev, n_groups, wi, lane);
+        nprev = 0;
+      }
+      jglob += nit;
+    }
+  }
+
+  // Let the next kernel in the stream start its prologue.
+  pdl_launch_dependents();
+
+  if constexpr (EPI == EPI_DOWN_COMBINE) {
+    // tail: warm L2 with the next layer's static weights (one slice per CTA)
+    if (tid == 32 * ncw) {
+      for (int q = 0; q < 2; ++q) {
+        if (!a.pf_ptr[q] || a.pf_bytes[q] <= 0) continue;
+        const long long per = ((a.pf_bytes[q] / gridDim.x) + 15) & ~15ll;
+        const long long beg = per * blockIdx.x;
+        long long end = beg + per;
+        if (end > a.pf_bytes[q]) end = a.pf_bytes[q];
+        for (long long o = beg; o < end; o += 65536) {
+          const long long n = (end - o) < 65536 ? (end - o) : 65536;
+          if (n >= 16) prefetch_l2(a.pf_ptr[q] + o, (uint32_t)(n & ~15ll));
+        }
+      }
+    }
+  }
+
+}
+
+}  // namespace moe

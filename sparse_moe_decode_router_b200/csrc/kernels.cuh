@@ -1,28 +1,7 @@
-// Device code of the MoE decode layer (sm_100a).
-//
-// One streaming-GEMV kernel template covers the four weight streams of the
-// layer: the router (bf16, dense), the shared expert's gate/up and down
-// (bf16, dense) and the routed experts' gate/up and down (MXFP4, one group
-// per active expert).  Decode at batch <= 64 is a weight stream: every byte
-// of an active weight matrix is read once and used for a handful of tokens,
-// so the kernel is built to keep HBM busy:
-//
-//  * persistent CTAs (one per SM), each owning a contiguous range of work
-//    items; an item is R consecutive output rows of one group;
-//  * one producer warp moves each item's weight tile (codes and scales, all
-//    rows contiguous in memory) into a ring of shared-memory stages with 1-D
-//    TMA bulk copies, completion counted on mbarriers, with an L2
-//    evict-first policy for the single-use routed weights;
-//  * consumer warps are split into row groups; inside a row group each
-//    thread owns one 32-element K chunk (= one MXFP4 scale block), keeps
-//    the activations of that chunk in registers across rows, decodes the
-//    weights in registers (cvt e2m1x2 -> f16x2 -> fp32, or bf16 -> fp32)
-//    and accumulates in fp32; a fixed butterfly + ordered cross-warp sum
-//    reduces the chunk partials (bitwise reproducible);
-//  * epilogues: store, SwiGLU, router logits (+ bias, then the last CTA
-//    runs top-k, softmax and bucketing), and down projection fused with the
-//    routing-weight combine and the residual add (last CTA to finish a row
-//    tile sums that tile in ascending expert order).
+// Device code shared by the MoE decode kernels (sm_100a): kernel arguments,
+// the multi-value warp reduction, the router's top-k / softmax / bucketing
+// finish, the fixed-order combine, and the router-matrix transpose.  The
+// streaming GEMV kernel itself is in gemv.cuh.
 #pragma once
 #include <cstdint>
 #include <cuda_runtime.h>
@@ -61,10 +40,14 @@ struct GemvArgs {
   int out_rows;   // output rows per group
   int up_off;     // SwiGLU: rows between a gate row and its up row (= out_rows)
   int R;          // output rows per item
-  int G;          // row groups per CTA
-  int wpr;        // warps per row group
-  int n_stages;
+  int ncw;        // consumer warps per CTA (one more warp produces)
+  int wpi;        // warps sharing one item (R = rows per warp * wpi)
+  int n_stages;   // shared-memory stages in the ring
   int stage_bytes;
+  int stage_offset;   // byte offset of the stage ring in dynamic shared memory
+  int x_offset;       // byte offset of the staged activation vectors
+  int xcap;           // activation vectors staged at a time
+  int scales_global;  // 1: MXFP4 scale rows are read from global memory (rows too short for TMA)
   // activations: row-major [*][K], bf16 or fp32
   const void* act;
   // token lists
@@ -89,7 +72,7 @@ struct GemvArgs {
   int* active_out;
   int* n_active_out;
   int n_experts;
-  int* done_counter;
+  int* done_counter;       // top-k kernel: CTAs done (the last one buckets and resets it)
   // combine extras (EPI_DOWN_COMBINE)
   const float* comb_w;      // topk_w [B][k]
   const float* y_shared;    // [B][H] or null
@@ -133,508 +116,258 @@ struct NextPow2 {
   static constexpr int value = T <= 1 ? 1 : T <= 2 ? 2 : T <= 4 ? 4 : T <= 8 ? 8 : T <= 16 ? 16 : 32;
 };
 
-// dot products of one 32-element chunk of NW weight rows with T activation chunks
-// (tokens t >= T of the TMAX-wide arrays are left untouched)
-template <int WF, int NW, int T, int TMAX>
-__device__ __forceinline__ void chunk_dots(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ scl,
-                                           const int (&row)[NW], int rowbytes, int sblocks, int c,
-                                           const float (&x)[TMAX][32], float (&acc)[NW][TMAX]) {
-#pragma unroll
-  for (int r = 0; r < NW; ++r) {
-    float d[T];
-#pragma unroll
-    for (int t = 0; t < T; ++t) d[t] = 0.f;
-    if constexpr (WF == W_MXFP4) {
-      const uint4 q = lds128(codes + (size_t)row[r] * rowbytes + c * 16);
-      const uint32_t qw[4] = {q.x, q.y, q.z, q.w};
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        uint32_t h2[4];
-        e2m1x8_to_f16x2(qw[i], h2);
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&h2[j]));
-#pragma unroll
-          for (int t = 0; t < T; ++t) {
-            d[t] = fmaf(f.x, x[t][8 * i + 2 * j], d[t]);
-            d[t] = fmaf(f.y, x[t][8 * i + 2 * j + 1], d[t]);
-          }
-        }
-      }
-      const float s = e8m0_to_f32(scl[(size_t)row[r] * sblocks + c]);
-#pragma unroll
-      for (int t = 0; t < T; ++t) acc[r][t] = d[t] * s;
-    } else {
-      const uint8_t* base = codes + (size_t)row[r] * rowbytes + c * 64;
-#pragma unroll
-      for (int v4 = 0; v4 < 4; ++v4) {
-        const uint4 q = lds128(base + 16 * v4);
-        const uint32_t qw[4] = {q.x, q.y, q.z, q.w};
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const float lo = bf16lo_to_f32(qw[i]), hi = bf16hi_to_f32(qw[i]);
-#pragma unroll
-          for (int t = 0; t < T; ++t) {
-            d[t] = fmaf(lo, x[t][8 * v4 + 2 * i], d[t]);
-            d[t] = fmaf(hi, x[t][8 * v4 + 2 * i + 1], d[t]);
-          }
-        }
-      }
-#pragma unroll
-      for (int t = 0; t < T; ++t) acc[r][t] = d[t];
-    }
-  }
-}
-
-template <bool ACT_F32>
-__device__ __forceinline__ void load_act_chunk(const void* act, int arow, int K, int c, float (&x)[32]) {
-  if constexpr (ACT_F32) {
-    const float4* p = reinterpret_cast<const float4*>(static_cast<const float*>(act) + (size_t)arow * K + c * 32);
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const float4 v = __ldg(p + i);
-      x[4 * i] = v.x;
-      x[4 * i + 1] = v.y;
-      x[4 * i + 2] = v.z;
-      x[4 * i + 3] = v.w;
-    }
-  } else {
-    const uint4* p = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(act) + (size_t)arow * K + c * 32);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const uint4 v = __ldg(p + i);
-      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        x[8 * i + 2 * j] = bf16lo_to_f32(w[j]);
-        x[8 * i + 2 * j + 1] = bf16hi_to_f32(w[j]);
-      }
-    }
-  }
-}
-
 // Fixed-order combine of one output element: residual + y_shared + sum_j w_j y_j
 // (fp32, fused multiply-adds in ascending j = ascending expert id), bf16 once.
+// Loads are issued eight pairs at a time, ahead of their ordered sums.
 __device__ __forceinline__ uint16_t combine_one(const GemvArgs& a, const float* __restrict__ y, int H, int b,
                                                 int r) {
+  const int k = a.top_k;
   float acc = __uint_as_float((uint32_t)a.residual[(size_t)b * H + r] << 16);
   if (a.y_shared) acc += __ldcg(a.y_shared + (size_t)b * H + r);
-  const int k = a.top_k;
-  for (int j = 0; j < k; ++j) acc = fmaf(__ldcg(a.comb_w + b * k + j), __ldcg(y + ((size_t)b * k + j) * H + r), acc);
+  for (int j0 = 0; j0 < k; j0 += 8) {
+    float wv[8], yv[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      wv[j] = 0.f;
+      yv[j] = 0.f;
+      if (j0 + j < k) {
+        wv[j] = __ldcg(a.comb_w + b * k + j0 + j);
+        yv[j] = __ldcg(y + ((size_t)b * k + j0 + j) * H + r);
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      if (j0 + j < k) acc = fmaf(wv[j], yv[j], acc);
+  }
   return f32_to_bf16_rne(acc);
 }
 
 // ---------------------------------------------------------------------------
-// Router finish: top-k (warp per token), softmax over the selected logits and
-// bucketing, by the last CTA of the router grid.  logits [B][E] fp32.
-__device__ void router_finish(const GemvArgs& a, unsigned char* smem) {
-  const int E = a.n_experts, k = a.top_k, B = a.n_tokens;
-  const int nthreads = blockDim.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int nwarps = nthreads >> 5;
-  const int PL = (E + 31) / 32;  // experts per lane, lane l holds [l*PL, (l+1)*PL)
-  int* s_idx = reinterpret_cast<int*>(smem);                               // [B*k]
-  unsigned long long* s_mask = reinterpret_cast<unsigned long long*>(smem + 8 * 1024);  // [E]
-  int* s_off = reinterpret_cast<int*>(smem + 8 * 1024 + 8 * kMaxExperts);               // [E+1]
-  const float* logits = a.out;
+// Top-k, softmax and bucketing (one CTA per token, 8 warps).
+//
+// Order-preserving key of an fp32 logit (larger logit -> larger key; 0 is
+// reserved for "no expert").
+__device__ __forceinline__ uint32_t logit_key(float f) {
+  const uint32_t u = __float_as_uint(f);
+  const uint32_t k = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+  return k ? k : 1u;
+}
 
-  for (int b = warp; b < B; b += nwarps) {
-    uint32_t key[32];
+// One warp selects the k largest keys among n candidates held in a blocked
+// layout (lane l owns candidates [l*PL, l*PL + PL)), whose ids ascend with the
+// candidate index; equal keys go to the lower id.  Returns the selection as a
+// per-lane slot bitmask.
+template <int PL>
+__device__ __forceinline__ uint32_t warp_select_topk(const uint32_t (&key)[PL], int k, int lane) {
+  uint32_t sel = 0u;
+  for (int r = 0; r < k; ++r) {
+    uint32_t best = 0u;
+    int bslot = 0;
 #pragma unroll
-    for (int i = 0; i < 32; ++i) {
-      const int e = lane * PL + i;
-      uint32_t kk = 0u;  // below every real key
-      if (i < PL && e < E) {
-        const uint32_t u = __float_as_uint(__ldcg(logits + (size_t)b * E + e));
-        kk = (u & 0x80000000u) ? ~u : (u | 0x80000000u);  // order-preserving map
-        if (kk == 0u) kk = 1u;                              // keep 0 for "empty"
+    for (int i = 0; i < PL; ++i) {
+      const bool live = !((sel >> i) & 1u);
+      if (live && key[i] > best) {
+        best = key[i];
+        bslot = i;
       }
-      key[i] = kk;
     }
-    uint32_t sel = 0u;
-    for (int r = 0; r < k; ++r) {
-      uint32_t best = 0u;
-      int bslot = 0;
+    const uint32_t m = __reduce_max_sync(0xFFFFFFFFu, best);
+    const uint32_t bal = __ballot_sync(0xFFFFFFFFu, best == m && m != 0u);
+    if (lane == __ffs(bal) - 1) sel |= 1u << bslot;
+  }
+  return sel;
+}
+
+constexpr int kTopkWarps = 8;
+
+// logits [B][E] fp32 -> topk_idx/topk_w [B][k] (ascending expert id), then the
+// last CTA to finish builds counts/offsets/pair_ids/active/n_active.
+__global__ void __launch_bounds__(kTopkWarps * 32) topk_bucket_kernel(const GemvArgs a) {
+  const int E = a.n_experts, k = a.top_k, B = a.n_tokens;
+  const int b = blockIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  constexpr int NT = kTopkWarps * 32;
+  __shared__ uint32_t c_key[kTopkWarps * kMaxTopK];
+  __shared__ int c_id[kTopkWarps * kMaxTopK];
+  __shared__ float c_val[kTopkWarps * kMaxTopK];
+  __shared__ int c_n[kTopkWarps];
+  __shared__ int s_last;
+  __shared__ unsigned long long s_mask[kMaxExperts];
+  __shared__ int s_off[kMaxExperts];
+  __shared__ int s_wsum[kTopkWarps][2];
+  pdl_wait();
+  const float* lg = a.out + (size_t)b * E;
+  // stage 1: warp w takes experts [w*SL, (w+1)*SL), SL = ceil(E/8) <= 128 (4 per lane)
+  const int SL = (E + kTopkWarps - 1) / kTopkWarps;
+  const int e0 = warp * SL;
+  const int PLs = (SL + 31) / 32;
+  {
+    uint32_t key[4];
+    float val[4];
 #pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        const bool live = !((sel >> i) & 1u);
-        if (live && key[i] > best) {
-          best = key[i];
-          bslot = i;
-        }
-      }
-      const uint32_t m = __reduce_max_sync(0xFFFFFFFFu, best);
-      const uint32_t bal = __ballot_sync(0xFFFFFFFFu, best == m);
-      const int win = __ffs(bal) - 1;  // lowest lane = lowest expert ids among equals
-      if (lane == win) sel |= 1u << bslot;
+    for (int i = 0; i < 4; ++i) {
+      const int e = e0 + lane * PLs + i;
+      const bool ok = i < PLs && lane * PLs + i < SL && e < E;
+      val[i] = ok ? __ldcg(lg + e) : 0.f;
+      key[i] = ok ? logit_key(val[i]) : 0u;
     }
-    // ascending expert id: lanes in order, slots in order within a lane
-    const int nsel = __popc(sel);
-    int pre = nsel;
+    const int kk = min(k, max(0, min(SL, E - e0)));
+    const uint32_t sel = warp_select_topk<4>(key, kk, lane);
+    // write the slice's selection in ascending id order
+    const int ns = __popc(sel);
+    int pre = ns;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       const int t = __shfl_up_sync(0xFFFFFFFFu, pre, o);
       if (lane >= o) pre += t;
     }
-    pre -= nsel;
-    // softmax over the selected logits in fp32: m = largest selected logit
-    float lmax = -INFINITY;
+    pre -= ns;
 #pragma unroll
-    for (int i = 0; i < 32; ++i)
-      if ((sel >> i) & 1u) lmax = fmaxf(lmax, __ldcg(logits + (size_t)b * E + lane * PL + i));
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) lmax = fmaxf(lmax, __shfl_xor_sync(0xFFFFFFFFu, lmax, o));
-    float ex[32];
-    float zl = 0.f;
-#pragma unroll
-    for (int i = 0; i < 32; ++i) {
-      ex[i] = 0.f;
+    for (int i = 0; i < 4; ++i)
       if ((sel >> i) & 1u) {
-        ex[i] = expf(__ldcg(logits + (size_t)b * E + lane * PL + i) - lmax);
+        c_key[warp * kMaxTopK + pre] = key[i];
+        c_id[warp * kMaxTopK + pre] = e0 + lane * PLs + i;
+        c_val[warp * kMaxTopK + pre] = val[i];
+        ++pre;
       }
-    }
-    // z = sum over selected in ascending expert order (lane order, then slot order)
-#pragma unroll
-    for (int i = 0; i < 32; ++i) zl += ex[i];
-    float z = 0.f;
-    for (int l = 0; l < 32; ++l) z += __shfl_sync(0xFFFFFFFFu, zl, l);
-    int pos = pre;
-#pragma unroll
-    for (int i = 0; i < 32; ++i) {
-      if ((sel >> i) & 1u) {
-        const int e = lane * PL + i;
-        a.topk_idx[b * k + pos] = e;
-        a.topk_w[b * k + pos] = ex[i] / z;
-        s_idx[b * k + pos] = e;
-        ++pos;
-      }
-    }
+    if (lane == 31) c_n[warp] = pre;
   }
   __syncthreads();
-  // bucketing: token bitmask per expert (B <= 64), counts = popcount,
-  // offsets = exclusive scan, pair position = offset + number of earlier tokens
-  for (int e = tid; e < E; e += nthreads) s_mask[e] = 0ull;
-  __syncthreads();
-  for (int p = tid; p < B * k; p += nthreads) atomicOr(&s_mask[s_idx[p]], 1ull << (p / k));
-  __syncthreads();
+  // stage 2: warp 0 merges the <= 8*k candidates (ids ascend with the index)
   if (warp == 0) {
-    int cnt_l = 0, act_l = 0;
-    for (int i = 0; i < PL; ++i) {
-      const int e = lane * PL + i;
-      if (e < E) {
-        const int c = __popcll(s_mask[e]);
-        cnt_l += c;
-        act_l += c > 0;
+    int base[kTopkWarps];
+    int n = 0;
+#pragma unroll
+    for (int w = 0; w < kTopkWarps; ++w) {
+      base[w] = n;
+      n += c_n[w];
+    }
+    const int PL = (n + 31) / 32;  // <= 8
+    uint32_t key[8];
+    int id[8];
+    float val[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int c = lane * PL + i;
+      key[i] = 0u;
+      id[i] = 0;
+      val[i] = 0.f;
+      if (i < PL && c < n) {
+        int w = 0;
+#pragma unroll
+        for (int q = 1; q < kTopkWarps; ++q)
+          if (c >= base[q]) w = q;
+        key[i] = c_key[w * kMaxTopK + (c - base[w])];
+        id[i] = c_id[w * kMaxTopK + (c - base[w])];
+        val[i] = c_val[w * kMaxTopK + (c - base[w])];
       }
     }
-    int cpre = cnt_l, apre = act_l;
+    const uint32_t sel = warp_select_topk<8>(key, k, lane);
+    const int ns = __popc(sel);
+    int pre = ns;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-      const int t1 = __shfl_up_sync(0xFFFFFFFFu, cpre, o);
-      const int t2 = __shfl_up_sync(0xFFFFFFFFu, apre, o);
-      if (lane >= o) {
-        cpre += t1;
-        apre += t2;
+      const int t = __shfl_up_sync(0xFFFFFFFFu, pre, o);
+      if (lane >= o) pre += t;
+    }
+    pre -= ns;
+    // softmax over the selected logits in fp32 (m = largest selected logit);
+    // the xor butterfly adds commuted pairs, so every lane holds the same z
+    float lmax = -INFINITY;
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      if ((sel >> i) & 1u) lmax = fmaxf(lmax, val[i]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) lmax = fmaxf(lmax, __shfl_xor_sync(0xFFFFFFFFu, lmax, o));
+    float ex[8];
+    float z = 0.f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      ex[i] = ((sel >> i) & 1u) ? expf(val[i] - lmax) : 0.f;
+      z += ex[i];
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xFFFFFFFFu, z, o);
+    int pos = pre;
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      if ((sel >> i) & 1u) {
+        a.topk_idx[b * k + pos] = id[i];
+        a.topk_w[b * k + pos] = ex[i] / z;
+        c_id[pos] = id[i];  // this token's selection, for a single-CTA bucketing
+        ++pos;
       }
-    }
-    cpre -= cnt_l;
-    apre -= act_l;
-    for (int i = 0; i < PL; ++i) {
-      const int e = lane * PL + i;
-      if (e < E) {
-        const int c = __popcll(s_mask[e]);
-        s_off[e] = cpre;
-        a.offsets_out[e] = cpre;
-        a.counts[e] = c;
-        if (c > 0) a.active_out[apre++] = e;
-        cpre += c;
-      }
-    }
-    if (lane == 31) {
-      s_off[E] = cpre;
-      a.offsets_out[E] = cpre;
-      *a.n_active_out = apre;
-    }
   }
   __syncthreads();
-  for (int p = tid; p < B * k; p += nthreads) {
-    const int e = s_idx[p];
-    const int b = p / k;
-    const unsigned long long below = (b == 0) ? 0ull : (s_mask[e] & ((1ull << b) - 1ull));
+  // the last CTA (token) to finish buckets all pairs
+  if (gridDim.x > 1) {
+    __threadfence();
+    if (tid == 0) s_last = (atomicAdd(a.done_counter, 1) == (int)gridDim.x - 1);
+    __syncthreads();
+    pdl_launch_dependents();
+    if (!s_last) return;
+    __threadfence();
+  } else {
+    pdl_launch_dependents();
+  }
+  auto idx_of = [&](int p) { return gridDim.x > 1 ? __ldcg(a.topk_idx + p) : c_id[p]; };
+  for (int e = tid; e < E; e += NT) s_mask[e] = 0ull;
+  __syncthreads();
+  for (int p = tid; p < B * k; p += NT) atomicOr(&s_mask[idx_of(p)], 1ull << (p / k));
+  __syncthreads();
+  // counts, exclusive offsets and the active list: thread t owns experts [4t, 4t+4)
+  int cnt[4], tc = 0, ta = 0;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int e = 4 * tid + i;
+    cnt[i] = (e < E) ? __popcll(s_mask[e]) : 0;
+    tc += cnt[i];
+    ta += cnt[i] > 0;
+  }
+  int ic = tc, ia = ta;  // inclusive warp scans
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int t1 = __shfl_up_sync(0xFFFFFFFFu, ic, o);
+    const int t2 = __shfl_up_sync(0xFFFFFFFFu, ia, o);
+    if (lane >= o) {
+      ic += t1;
+      ia += t2;
+    }
+  }
+  if (lane == 31) {
+    s_wsum[warp][0] = ic;
+    s_wsum[warp][1] = ia;
+  }
+  __syncthreads();
+  int wc = 0, wa = 0;
+  for (int w = 0; w < warp; ++w) {
+    wc += s_wsum[w][0];
+    wa += s_wsum[w][1];
+  }
+  int off = wc + ic - tc, act = wa + ia - ta;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int e = 4 * tid + i;
+    if (e < E) {
+      s_off[e] = off;
+      a.offsets_out[e] = off;
+      a.counts[e] = cnt[i];
+      if (cnt[i] > 0) a.active_out[act++] = e;
+      off += cnt[i];
+    }
+  }
+  if (tid == NT - 1) {
+    a.offsets_out[E] = off;
+    *a.n_active_out = act;
+  }
+  __syncthreads();
+  for (int p = tid; p < B * k; p += NT) {
+    const int e = idx_of(p);
+    const int bb = p / k;
+    const unsigned long long below = (bb == 0) ? 0ull : (s_mask[e] & ((1ull << bb) - 1ull));
     a.pair_ids_out[s_off[e] + __popcll(below)] = p;
   }
-}
-
-// ---------------------------------------------------------------------------
-template <int WF, int EPI, bool ACT_F32, int RPG, int TMAX, int MAXT>
-__global__ void __launch_bounds__(MAXT, 1) stream_gemv_kernel(const GemvArgs a) {
-  constexpr bool kSwiglu = (EPI == EPI_SWIGLU);
-  constexpr int NW = kSwiglu ? 2 * RPG : RPG;  // weight rows per thread per item
-  extern __shared__ __align__(128) unsigned char smem[];
-
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int ncw = a.G * a.wpr;  // consumer warps
-  const int nct = ncw * 32;
-  const int K = a.K;
-  const int C = K >> 5;
-  const int rowbytes = (WF == W_MXFP4) ? (K >> 1) : (K << 1);
-  const int sblocks = K >> 5;
-  const int rows_per_item = kSwiglu ? 2 * a.R : a.R;
-  const int codes_bytes = rows_per_item * rowbytes;
-
-  uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem);
-  uint64_t* empty_bar = full_bar + a.n_stages;
-  float* red = reinterpret_cast<float*>(empty_bar + a.n_stages);       // [2][G][wpr][32]
-  volatile int* s_flags = reinterpret_cast<volatile int*>(red + 2 * a.G * a.wpr * 32);  // [4]
-  unsigned char* stages = smem + ((((size_t)2 * a.n_stages * 8 + (size_t)2 * a.G * a.wpr * 32 * 4 + 16) + 127) & ~(size_t)127);
-
-  if (tid == 0) {
-    for (int s = 0; s < a.n_stages; ++s) {
-      mbar_init(&full_bar[s], 1);
-      mbar_init(&empty_bar[s], ncw);
-    }
-    s_flags[0] = 0;  // abort
-    s_flags[1] = 0;
-    fence_barrier_init();
-  }
-  __syncthreads();
-
-  // Dense weight streams may start before the previous grid finishes (weights
-  // are static); anything produced upstream (routing plan, activations) is
-  // only read after pdl_wait().
-  const bool producer = (warp == ncw);
-  if (a.routed || !producer) pdl_wait();
-
-  // A routing plan from elsewhere is validated, never trusted: groups and
-  // token counts are clamped into range (and flagged) before they address memory.
-  int n_groups = a.routed ? *a.n_active : 1;
-  if (n_groups < 0 || n_groups > a.n_experts) {
-    if (tid == 0) atomicExch(a.err, kErrBadPlan);
-    n_groups = n_groups < 0 ? 0 : a.n_experts;
-  }
-  const int n_rt = a.out_rows / a.R;
-  const long long n_items = (long long)n_groups * n_rt;
-  const long long it0 = n_items * blockIdx.x / gridDim.x;
-  const long long it1 = n_items * (blockIdx.x + 1) / gridDim.x;
-
-  if (producer) {
-    if (lane == 0) {
-      // every weight byte is used once per step: do not let it displace
-      // activations, scratch or prefetched next-layer weights in L2
-      const uint64_t pol = l2_policy_evict_first();
-      int s = 0;
-      uint32_t ph = 0;
-      for (long long it = it0; it < it1; ++it) {
-        if (!mbar_wait_bounded(&empty_bar[s], ph ^ 1u)) {
-          atomicExch(a.err, kErrTimeout);
-          s_flags[0] = 1;
-          break;
-        }
-        if (s_flags[0]) break;
-        const int g = (int)(it / n_rt);
-        const int rt = (int)(it - (long long)g * n_rt);
-        const int grp = a.routed ? clamp_group(a.active[g], a.n_experts, a.err) : 0;
-        const int r0 = rt * a.R;
-        unsigned char* st = stages + (size_t)s * a.stage_bytes;
-        const uint32_t cb = (uint32_t)(a.R * rowbytes);
-        const uint32_t sb = (WF == W_MXFP4) ? (uint32_t)(a.R * sblocks) : 0u;
-        const uint32_t total = (kSwiglu ? 2u : 1u) * (cb + sb);
-        mbar_arrive_expect_tx(&full_bar[s], total);
-        const uint8_t* wg = a.w + (long long)grp * a.w_gstride;
-        bulk_g2s(st, wg + (size_t)r0 * rowbytes, cb, &full_bar[s], pol);
-        if (kSwiglu) bulk_g2s(st + cb, wg + (size_t)(r0 + a.up_off) * rowbytes, cb, &full_bar[s], pol);
-        if (WF == W_MXFP4) {
-          const uint8_t* sg = a.sc + (long long)grp * a.s_gstride;
-          bulk_g2s(st + codes_bytes, sg + (size_t)r0 * sblocks, sb, &full_bar[s], pol);
-          if (kSwiglu) bulk_g2s(st + codes_bytes + sb, sg + (size_t)(r0 + a.up_off) * sblocks, sb, &full_bar[s], pol);
-        }
-        if (++s == a.n_stages) {
-          s = 0;
-          ph ^= 1u;
-        }
-      }
-      if (s_flags[0]) {
-        // aborting: let copies already issued land before the CTA exits
-        for (int q = 0; q < a.n_stages; ++q) (void)mbar_wait_bounded(&full_bar[q], 0u, 1ll << 24),
-                                              (void)mbar_wait_bounded(&full_bar[q], 1u, 1ll << 24);
-      }
-    }
-  } else {
-    // ------------------------------ consumers ------------------------------
-    const int rg = warp / a.wpr;           // row group
-    const int wig = warp - rg * a.wpr;     // warp in group
-    const int c = wig * 32 + lane;         // K chunk owned by this thread
-    const bool has_chunk = c < C;
-    const int gtid = wig * 32 + lane;      // thread index inside the row group
-    float x[TMAX][32];
-    int cached_group = -1;
-    int s = 0;
-    uint32_t ph = 0;
-    int buf = 0;
-    for (long long it = it0; it < it1; ++it) {
-      const int g = (int)(it / n_rt);
-      const int rt = (int)(it - (long long)g * n_rt);
-      const int grp = a.routed ? clamp_group(a.active[g], a.n_experts, nullptr) : 0;
-      int tok0 = a.routed ? a.offsets[grp] : 0;
-      int ntok = a.routed ? (a.offsets[grp + 1] - tok0) : a.n_tokens;
-      if (a.routed && (tok0 < 0 || ntok < 1 || tok0 + ntok > a.n_pairs)) {
-        if (lane == 0) atomicExch(a.err, kErrBadPlan);
-        tok0 = 0;
-        ntok = 1;
-      }
-
-      if (!mbar_wait_bounded(&full_bar[s], ph)) {
-        atomicExch(a.err, kErrTimeout);
-        s_flags[0] = 1;
-      }
-      if (s_flags[0]) break;
-      const unsigned char* st = stages + (size_t)s * a.stage_bytes;
-
-      int rowsel[NW];
-#pragma unroll
-      for (int r = 0; r < NW; ++r) rowsel[r] = (r < RPG) ? (rg * RPG + r) : (a.R + rg * RPG + (r - RPG));
-
-      for (int tb = 0; tb < ntok; tb += TMAX) {
-        const int T = min(TMAX, ntok - tb);
-        int arow[TMAX], orow[TMAX];
-#pragma unroll
-        for (int t = 0; t < TMAX; ++t) {
-          const int tt = min(tb + t, ntok - 1);
-          if (a.routed) {
-            int p = a.pair_ids[tok0 + tt];
-            if (p < 0 || p >= a.n_pairs) p = 0;
-            arow[t] = a.act_by_pair ? p : p / a.top_k;
-            orow[t] = p;
-          } else {
-            arow[t] = tt;
-            orow[t] = tt;
-          }
-        }
-        const bool reuse = (ntok <= TMAX) && (cached_group == (a.routed ? grp : 0));
-        if (!reuse && has_chunk) {
-#pragma unroll
-          for (int t = 0; t < TMAX; ++t)
-            if (t < T) load_act_chunk<ACT_F32>(a.act, arow[t], K, c, x[t]);
-        }
-        cached_group = (ntok <= TMAX) ? (a.routed ? grp : 0) : -1;
-
-        float acc[NW][TMAX];
-#pragma unroll
-        for (int r = 0; r < NW; ++r)
-#pragma unroll
-          for (int t = 0; t < TMAX; ++t) acc[r][t] = 0.f;
-        if (has_chunk) {
-          if (T == TMAX) {
-            chunk_dots<WF, NW, TMAX, TMAX>(st, st + codes_bytes, rowsel, rowbytes, sblocks, c, x, acc);
-          } else if constexpr (TMAX > 1) {
-            if (T == 1) chunk_dots<WF, NW, 1, TMAX>(st, st + codes_bytes, rowsel, rowbytes, sblocks, c, x, acc);
-            else if (T == 2) chunk_dots<WF, NW, (TMAX > 2 ? 2 : 1), TMAX>(st, st + codes_bytes, rowsel, rowbytes, sblocks, c, x, acc);
-            else chunk_dots<WF, NW, (TMAX > 3 ? 3 : 1), TMAX>(st, st + codes_bytes, rowsel, rowbytes, sblocks, c, x, acc);
-          }
-        }
-        if (tb + TMAX >= ntok) {
-          // stage no longer needed: hand it back to the producer
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&empty_bar[s]);
-        }
-        // --- reduce over the row group ---
-        constexpr int V = NextPow2<NW * TMAX>::value;
-        float v[V];
-#pragma unroll
-        for (int i = 0; i < V; ++i) v[i] = 0.f;
-#pragma unroll
-        for (int r = 0; r < NW; ++r)
-#pragma unroll
-          for (int t = 0; t < TMAX; ++t) v[r * TMAX + t] = acc[r][t];
-        const float tot = warp_reduce_multi<V>(v, lane);
-        float* rb = red + ((size_t)(buf * a.G + rg) * a.wpr) * 32;
-        if ((lane & (32 / V - 1)) == 0) rb[wig * 32 + lane / (32 / V)] = tot;
-        named_bar_sync(1, nct);
-        // --- epilogue ---
-        const int nout = (kSwiglu ? RPG : NW) * TMAX;
-        if (gtid < nout) {
-          const int rr = gtid / TMAX, t = gtid - (gtid / TMAX) * TMAX;
-          if (t < T) {
-            float s0 = 0.f;
-            for (int w2 = 0; w2 < a.wpr; ++w2) s0 += rb[w2 * 32 + rr * TMAX + t];
-            const int orow_out = rt * a.R + rg * RPG + rr;
-            float val = s0;
-            if constexpr (kSwiglu) {
-              float s1 = 0.f;
-              for (int w2 = 0; w2 < a.wpr; ++w2) s1 += rb[w2 * 32 + (RPG + rr) * TMAX + t];
-              val = s0 / (1.0f + expf(-s0)) * s1;
-            }
-            if constexpr (EPI == EPI_ROUTER) {
-              if (a.bias) val += a.bias[orow_out];
-            }
-            int orow_t = orow[0];
-#pragma unroll
-            for (int q = 1; q < TMAX; ++q)
-              if (t == q) orow_t = orow[q];
-            a.out[(size_t)orow_t * a.out_rows + orow_out] = val;
-          }
-        }
-        buf ^= 1;
-      }
-      if constexpr (EPI == EPI_DOWN_COMBINE) {
-        // last CTA to finish row tile rt (over all active experts) combines it
-        __threadfence();
-        named_bar_sync(1, nct);
-        if (tid == 0) {
-          const int old = atomicAdd(&a.tile_counter[rt], 1);
-          s_flags[1] = (old == n_groups - 1);
-        }
-        named_bar_sync(1, nct);
-        if (s_flags[1]) {
-          __threadfence();
-          const int H = a.out_rows;
-          for (int i = tid; i < a.batch * a.R; i += nct) {
-            const int b = i / a.R, r = rt * a.R + (i - (i / a.R) * a.R);
-            a.out_bf16[(size_t)b * H + r] = combine_one(a, a.out, H, b, r);
-          }
-          if (tid == 0) a.tile_counter[rt] = 0;
-        }
-      }
-      if (++s == a.n_stages) {
-        s = 0;
-        ph ^= 1u;
-      }
-    }
-  }
-
-  // Let the next kernel in the stream start its prologue.
-  pdl_launch_dependents();
-
-  if constexpr (EPI == EPI_DOWN_COMBINE) {
-    // tail: warm L2 with the next layer's static weights (one slice per CTA)
-    if (tid == 32 * ncw && !s_flags[0]) {
-      for (int q = 0; q < 2; ++q) {
-        if (!a.pf_ptr[q] || a.pf_bytes[q] <= 0) continue;
-        const long long per = ((a.pf_bytes[q] / gridDim.x) + 15) & ~15ll;
-        const long long beg = per * blockIdx.x;
-        long long end = beg + per;
-        if (end > a.pf_bytes[q]) end = a.pf_bytes[q];
-        for (long long o = beg; o < end; o += 65536) {
-          const long long n = (end - o) < 65536 ? (end - o) : 65536;
-          if (n >= 16) prefetch_l2(a.pf_ptr[q] + o, (uint32_t)(n & ~15ll));
-        }
-      }
-    }
-  }
-
-  if constexpr (EPI == EPI_ROUTER) {
-    __syncthreads();
-    __threadfence();
-    if (tid == 0) {
-      const int old = atomicAdd(a.done_counter, 1);
-      s_flags[1] = (old == (int)gridDim.x - 1);
-    }
-    __syncthreads();
-    if (s_flags[1]) {
-      __threadfence();
-      router_finish(a, stages);
-      if (tid == 0) *a.done_counter = 0;
-    }
-  }
+  if (tid == 0 && gridDim.x > 1) *a.done_counter = 0;
 }
 
 // Staged combine: out = bf16(residual + y_shared + sum_j w_j y_j), one thread per element.

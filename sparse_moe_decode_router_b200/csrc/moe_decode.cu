@@ -9,85 +9,125 @@
 #include <new>
 
 #include "../../include/moe_decode.h"
+#include "gemv.cuh"
 #include "kernels.cuh"
 
 using namespace moe;
 
 namespace {
 
-constexpr int kSmemBudget = 200 * 1024;  // dynamic shared memory per CTA (1 CTA per SM)
-constexpr int kMaxStages = 8;
+constexpr int kSmemBudget = 227 * 1024;  // dynamic shared memory per CTA (1 CTA per SM)
+constexpr int kMaxStages = kMaxStagesDev;
+constexpr int kXBudget = 64 * 1024;       // staged activation vectors
+constexpr int kPrefetchBytes = 64 * 1024; // stages kept in flight ahead of the consumers
 
 size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
-struct GemvPlan {
-  bool ok = false;
-  int K = 0, out_rows = 0, R = 0, G = 0, wpr = 0, rpg = 0, n_stages = 0, stage_bytes = 0;
-  int threads = 0, smem = 0;
+enum Kind { K_ROUTER = 0, K_SGU = 1, K_SDN = 2, K_GU = 3, K_DN = 4, K_DNC = 5, K_NUM = 6 };
+
+// Fixed per weight stream: weight format, epilogue, activation type, output
+// rows per warp, warps per item.
+struct KindTraits { int wf, epi, xk, rpw, wpi; };
+#ifndef MOE_GU_RPW
+#define MOE_GU_RPW 1
+#endif
+#ifndef MOE_GU_WPI
+#define MOE_GU_WPI 4
+#endif
+#ifndef MOE_DN_RPW
+#define MOE_DN_RPW 4
+#endif
+#ifndef MOE_DN_WPI
+#define MOE_DN_WPI 4
+#endif
+constexpr KindTraits kTraits[K_NUM] = {
+    {W_BF16, EPI_ROUTER, X_BF16, 2, 1},        // router: 2 rows (28 KB) per item
+    {W_BF16, EPI_SWIGLU, X_BF16, 1, 1},        // shared gate/up: 1 output row (2 x 14 KB)
+    {W_BF16, EPI_STORE, X_F32, 2, 4},          // shared down: 8 rows (32 KB)
+    {W_MXFP4, EPI_SWIGLU, X_BF16, MOE_GU_RPW, MOE_GU_WPI},       // routed gate/up: 4 output rows (2 x 14 KB)
+    {W_MXFP4, EPI_STORE, X_F32, MOE_DN_RPW, MOE_DN_WPI},         // routed down: 16 rows (16 KB)
+    {W_MXFP4, EPI_DOWN_COMBINE, X_F32, MOE_DN_RPW, MOE_DN_WPI},  // routed down + combine
 };
 
-// Work decomposition of one weight stream for one register budget (tmax tokens per pass:
-// 1 -> up to 16 consumer warps, 2 -> up to 8).
-GemvPlan make_plan(int K, int out_rows, bool swiglu, bool mxfp4, int tmax) {
+struct GemvPlan {
+  bool ok = false;
+  int K = 0, out_rows = 0, R = 0, ncw = 0, wpi = 0, n_stages = 0, stage_bytes = 0, stage_offset = 0, x_offset = 0;
+  int xcap = 0, scales_global = 0, threads = 0, smem = 0;
+};
+
+// Work decomposition of one weight stream.  `slots_needed` = activation
+// vectors the stream can address (B, or B*k for the down projection),
+// `max_groups` = most groups (experts) the stream can have active,
+// `tok_per_group` = most activation vectors one group uses.
+GemvPlan make_plan(Kind kind, int K, int out_rows, int slots_needed, int max_groups, int tok_per_group,
+                   long long s_gstride, int num_sms) {
   GemvPlan p;
-  if (K <= 0 || K % 32 || out_rows <= 0) return p;
-  const int C = K / 32;
-  const int wpr = (C + 31) / 32;
-  if (wpr > 16) return p;
-  const int maxw = (tmax == 1) ? 16 : 8;
-  const int rowbytes = mxfp4 ? K / 2 : K * 2;
-  const int sbytes = mxfp4 ? K / 32 : 0;
-  for (int rpg = 2; rpg >= 1; --rpg) {
-    for (int G = std::max(1, maxw / wpr); G >= 1; --G) {
-      const int R = G * rpg;
-      if (out_rows % R) continue;
-      if (mxfp4 && (R * sbytes) % 16) continue;
-      const int rows = swiglu ? 2 * R : R;
-      const int stage = (int)align_up((size_t)rows * (rowbytes + sbytes), 128);
-      const int hdr = (int)align_up(16 * kMaxStages + 256 * G * wpr + 16, 128);
-      int ns = (kSmemBudget - hdr) / stage;
-      ns = std::min(ns, kMaxStages);
-      if (ns < 3 && !(rpg == 1 && G == 1 && ns >= 2)) continue;
-      p.ok = true;
-      p.K = K;
-      p.out_rows = out_rows;
-      p.R = R;
-      p.G = G;
-      p.wpr = wpr;
-      p.rpg = rpg;
-      p.n_stages = ns;
-      p.stage_bytes = stage;
-      p.threads = (G * wpr + 1) * 32;
-      if (p.threads > (tmax == 1 ? 17 * 32 : 9 * 32)) return GemvPlan();
-      p.smem = hdr + ns * stage;
-      return p;
-    }
-  }
+  const KindTraits t = kTraits[kind];
+  const int R = t.rpw * t.wpi;
+  if (K <= 0 || K % 32 || out_rows <= 0 || out_rows % R) return p;
+  const bool mx = t.wf == W_MXFP4;
+  const bool swiglu = t.epi == EPI_SWIGLU;
+  const int rowbytes = mx ? K / 2 : K * 2;
+  const int sbytes = mx ? K / 32 : 0;
+  const int rows = swiglu ? 2 * R : R;
+  // scale rows go through TMA only when every copy is 16-byte aligned and sized
+  const bool sg = mx && (((long long)R * sbytes) % 16 != 0 || s_gstride % 16 != 0);
+  const int stage = (int)align_up((size_t)rows * (rowbytes + (mx && !sg ? sbytes : 0)), 128);
+  // activation slots: a CTA's contiguous item range spans at most
+  // ceil(items per CTA / items per group) + 1 groups
+  const int n_rt = out_rows / R;
+  const long long items_per_cta = ((long long)max_groups * n_rt + num_sms - 1) / num_sms;
+  const int groups_per_cta = (int)std::min<long long>(max_groups, (items_per_cta + n_rt - 1) / n_rt + 1);
+  const int xrow = x_row_bytes(t.wf, t.xk, K);
+  int xcap = std::min(slots_needed, groups_per_cta * tok_per_group);
+  xcap = std::min(std::min(xcap, kMaxSlots), std::max(1, kXBudget / xrow));
+  const int hdr = (int)align_up(16 * 64 + sizeof(PhaseTable) + (kMaxSlots + 2 + kMaxStagesDev + kMaxStageUnits) * 4, 128);
+  const int x_off = hdr;
+  const int st_off = (int)align_up((size_t)x_off + (size_t)xcap * xrow, 128);
+  int ns = std::min(kMaxStages, (kSmemBudget - st_off) / stage);
+  if (ns < 2) return p;
+  const int pf = std::max(1, (kPrefetchBytes + stage - 1) / stage);
+  // consumer warps: whole groups of wpi, at most ns - pf groups consuming at once.
+  // Items go to the groups round robin, so the ring holds a multiple of the
+  // group count: every stage is then always consumed by the same group, in
+  // item order, and a group never waits on a stage whose previous phase
+  // another group has not finished.
+  int groups = std::max(1, std::min(kMaxConsumerWarps / t.wpi, std::max(1, ns - pf)));
+  while (groups > 1 && (ns / groups) * groups - groups < pf) --groups;
+  ns = (ns / groups) * groups;
+  p.ok = true;
+  p.K = K;
+  p.out_rows = out_rows;
+  p.R = R;
+  p.wpi = t.wpi;
+  p.ncw = groups * t.wpi;
+  p.n_stages = ns;
+  p.stage_bytes = stage;
+  p.stage_offset = st_off;
+  p.x_offset = x_off;
+  p.xcap = xcap;
+  p.scales_global = sg ? 1 : 0;
+  p.threads = (p.ncw + 1) * 32;
+  p.smem = st_off + ns * stage;
   return p;
 }
 
-enum Kind { K_ROUTER = 0, K_SGU = 1, K_SDN = 2, K_GU = 3, K_DN = 4, K_DNC = 5, K_NUM = 6 };
-
 typedef void (*GemvFn)(const GemvArgs);
 
-template <int RPG, int TMAX>
+template <int TMAX>
 GemvFn pick_fn(Kind k) {
-  constexpr int MAXT = (TMAX == 1) ? 17 * 32 : 9 * 32;
   switch (k) {
-    case K_ROUTER: return stream_gemv_kernel<W_BF16, EPI_ROUTER, false, RPG, TMAX, MAXT>;
-    case K_SGU: return stream_gemv_kernel<W_BF16, EPI_SWIGLU, false, RPG, TMAX, MAXT>;
-    case K_SDN: return stream_gemv_kernel<W_BF16, EPI_STORE, true, RPG, TMAX, MAXT>;
-    case K_GU: return stream_gemv_kernel<W_MXFP4, EPI_SWIGLU, false, RPG, TMAX, MAXT>;
-    case K_DN: return stream_gemv_kernel<W_MXFP4, EPI_STORE, true, RPG, TMAX, MAXT>;
-    case K_DNC: return stream_gemv_kernel<W_MXFP4, EPI_DOWN_COMBINE, true, RPG, TMAX, MAXT>;
+    case K_ROUTER: return gemv_kernel<W_BF16, EPI_ROUTER, X_BF16, TMAX, 2>;
+    case K_SGU: return gemv_kernel<W_BF16, EPI_SWIGLU, X_BF16, TMAX, 1>;
+    case K_SDN: return gemv_kernel<W_BF16, EPI_STORE, X_F32, TMAX, 2>;
+    case K_GU: return gemv_kernel<W_MXFP4, EPI_SWIGLU, X_BF16, TMAX, MOE_GU_RPW>;
+    case K_DN: return gemv_kernel<W_MXFP4, EPI_STORE, X_F32, TMAX, MOE_DN_RPW>;
+    case K_DNC: return gemv_kernel<W_MXFP4, EPI_DOWN_COMBINE, X_F32, TMAX, MOE_DN_RPW>;
     default: return nullptr;
   }
 }
 
-GemvFn gemv_fn(Kind k, int rpg, int tmax) {
-  if (tmax == 1) return rpg == 2 ? pick_fn<2, 1>(k) : pick_fn<1, 1>(k);
-  return rpg == 2 ? pick_fn<2, 2>(k) : pick_fn<1, 2>(k);
-}
+GemvFn gemv_fn(Kind k, int tmax) { return tmax == 1 ? pick_fn<1>(k) : pick_fn<2>(k); }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -149,10 +189,14 @@ GemvArgs base_args(const moe_layer* L, const GemvPlan& p) {
   a.K = p.K;
   a.out_rows = p.out_rows;
   a.R = p.R;
-  a.G = p.G;
-  a.wpr = p.wpr;
+  a.ncw = p.ncw;
+  a.wpi = p.wpi;
   a.n_stages = p.n_stages;
   a.stage_bytes = p.stage_bytes;
+  a.stage_offset = p.stage_offset;
+  a.x_offset = p.x_offset;
+  a.xcap = p.xcap;
+  a.scales_global = p.scales_global;
   a.top_k = L->cfg.top_k;
   a.n_experts = L->cfg.n_experts;
   a.err = L->err;
@@ -162,8 +206,7 @@ GemvArgs base_args(const moe_layer* L, const GemvPlan& p) {
 cudaError_t run_gemv(moe_layer* L, Kind k, int B, const GemvArgs& a, cudaStream_t st, bool pdl) {
   const int tm = tmax_for(B);
   const GemvPlan& p = L->plans[k][tm == 1 ? 0 : 1];
-  GemvFn fn = gemv_fn(k, p.rpg, tm);
-  return launch_ex(fn, L->num_sms, p.threads, p.smem, st, pdl, a);
+  return launch_ex(gemv_fn(k, tm), L->num_sms, p.threads, p.smem, st, pdl, a);
 }
 
 const GemvPlan& plan_of(const moe_layer* L, Kind k, int B) { return L->plans[k][tmax_for(B) == 1 ? 0 : 1]; }
@@ -172,6 +215,7 @@ bool routing_ok(const moe_routing* r) {
   return r && r->topk_idx && r->topk_w && r->counts && r->offsets && r->pair_ids && r->active && r->n_active;
 }
 
+// Router GEMV (logits, fp32) then top-k / softmax / bucketing, chained with PDL.
 cudaError_t launch_router(moe_layer* L, const void* x, int B, const moe_routing& r, cudaStream_t st) {
   const GemvPlan& p = plan_of(L, K_ROUTER, B);
   GemvArgs a = base_args(L, p);
@@ -181,15 +225,23 @@ cudaError_t launch_router(moe_layer* L, const void* x, int B, const moe_routing&
   a.n_tokens = B;
   a.out = L->logits;
   a.bias = L->w.router_bias;
-  a.topk_w = r.topk_w;
-  a.topk_idx = r.topk_idx;
-  a.counts = r.counts;
-  a.offsets_out = r.offsets;
-  a.pair_ids_out = r.pair_ids;
-  a.active_out = r.active;
-  a.n_active_out = r.n_active;
-  a.done_counter = L->router_cnt;
-  return run_gemv(L, K_ROUTER, B, a, st, L->pdl);
+  cudaError_t e = run_gemv(L, K_ROUTER, B, a, st, L->pdl);
+  if (e != cudaSuccess) return e;
+  GemvArgs t;
+  std::memset(&t, 0, sizeof(t));
+  t.out = L->logits;
+  t.n_experts = L->cfg.n_experts;
+  t.top_k = L->cfg.top_k;
+  t.n_tokens = B;
+  t.topk_w = r.topk_w;
+  t.topk_idx = r.topk_idx;
+  t.counts = r.counts;
+  t.offsets_out = r.offsets;
+  t.pair_ids_out = r.pair_ids;
+  t.active_out = r.active;
+  t.n_active_out = r.n_active;
+  t.done_counter = L->router_cnt;
+  return launch_ex(topk_bucket_kernel, B, kTopkWarps * 32, 0, st, L->pdl, t);
 }
 
 cudaError_t launch_shared(moe_layer* L, const void* x, int B, float* ys, cudaStream_t st, bool pdl) {
@@ -347,21 +399,20 @@ moe_status_t moe_layer_create(const moe_layer_config* cfg, const moe_layer_weigh
   L->prefetch = !(c.flags & MOE_FLAG_NO_PREFETCH);
 
   const int H = c.hidden, E = c.n_experts, k = c.top_k, I = c.inter, Is = c.shared_inter, MB = c.max_batch;
+  // plans: [0] for B = 1 (one token per pass), [1] for B > 1 (two per pass)
   for (int t = 0; t < 2; ++t) {
-    const int tm = t == 0 ? 1 : 2;
-    L->plans[K_ROUTER][t] = make_plan(H, E, false, false, tm);
-    L->plans[K_GU][t] = make_plan(H, I, true, true, tm);
-    L->plans[K_DN][t] = make_plan(I, H, false, true, tm);
-    L->plans[K_DNC][t] = make_plan(I, H, false, true, tm);
+    const int nb = t == 0 ? 1 : MB;
+    const int maxg = std::min(E, nb * k);  // experts one call can activate
+    L->plans[K_ROUTER][t] = make_plan(K_ROUTER, H, E, nb, 1, nb, 0, sms);
+    L->plans[K_GU][t] = make_plan(K_GU, H, I, nb, maxg, nb, (long long)2 * I * (H / 32), sms);
+    L->plans[K_DN][t] = make_plan(K_DN, I, H, nb * k, maxg, nb, (long long)H * (I / 32), sms);
+    L->plans[K_DNC][t] = make_plan(K_DNC, I, H, nb * k, maxg, nb, (long long)H * (I / 32), sms);
     if (Is > 0) {
-      L->plans[K_SGU][t] = make_plan(H, Is, true, false, tm);
-      L->plans[K_SDN][t] = make_plan(Is, H, false, false, tm);
+      L->plans[K_SGU][t] = make_plan(K_SGU, H, Is, nb, 1, nb, 0, sms);
+      L->plans[K_SDN][t] = make_plan(K_SDN, Is, H, nb, 1, nb, 0, sms);
     }
-    bool ok = L->plans[K_ROUTER][t].ok && L->plans[K_GU][t].ok && L->plans[K_DN][t].ok;
+    bool ok = L->plans[K_ROUTER][t].ok && L->plans[K_GU][t].ok && L->plans[K_DN][t].ok && L->plans[K_DNC][t].ok;
     if (Is > 0) ok = ok && L->plans[K_SGU][t].ok && L->plans[K_SDN][t].ok;
-    // the router's last CTA reuses its stage ring for top-k and bucketing
-    ok = ok && (size_t)L->plans[K_ROUTER][t].n_stages * L->plans[K_ROUTER][t].stage_bytes >=
-                   8 * 1024 + 8 * kMaxExperts + 4 * (kMaxExperts + 1);
     if (!ok) {
       delete L;
       return MOE_ERR_UNSUPPORTED;
@@ -389,7 +440,7 @@ moe_status_t moe_layer_create(const moe_layer_config* cfg, const moe_layer_weigh
   const size_t o_hs = take((size_t)MB * std::max(Is, 1) * 4);
   const size_t o_ys = take((size_t)MB * H * 4);
   const size_t o_rc = take(4);
-  const size_t o_tc = take((size_t)H * 4);
+  const size_t o_tc = take((size_t)H * 4);  // one counter per down-projection row tile (<= H)
   const size_t o_er = take(4);
   const size_t o_xs = take((size_t)MB * H * 2);
   const size_t o_rs = take((size_t)MB * H * 2);
@@ -433,7 +484,7 @@ moe_status_t moe_layer_create(const moe_layer_config* cfg, const moe_layer_weigh
     for (int t = 0; t < 2 && e == cudaSuccess; ++t) {
       const GemvPlan& p = L->plans[kk][t];
       if (!p.ok) continue;
-      e = cudaFuncSetAttribute(gemv_fn((Kind)kk, p.rpg, t == 0 ? 1 : 2), cudaFuncAttributeMaxDynamicSharedMemorySize,
+      e = cudaFuncSetAttribute(gemv_fn((Kind)kk, t == 0 ? 1 : 2), cudaFuncAttributeMaxDynamicSharedMemorySize,
                                p.smem);
     }
   if (e == cudaSuccess) e = cudaDeviceSynchronize();

@@ -110,6 +110,12 @@ __device__ __forceinline__ uint4 lds128(const void* p) {
   return v;
 }
 
+__device__ __forceinline__ uint32_t lds_u8(const void* p) {
+  uint32_t v;
+  asm volatile("ld.shared.u8 %0, [%1];" : "=r"(v) : "r"(smem_addr(p)));
+  return v;
+}
+
 // ---- E2M1 decode ----------------------------------------------------------------
 // Four bytes of packed E2M1 codes -> four f16x2 registers; byte j of `w`
 // becomes out[j], its low nibble in the low half.

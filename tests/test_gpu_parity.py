@@ -5,7 +5,7 @@ import numpy as np
 import pytest
 
 import synth
-from helpers import W_ABS, Y_MAX_REL, Y_MEAN_REL, bf16_close, metric_close
+from helpers import W_ABS, Y_MAX_REL, Y_MEAN_REL, Y_ROUTED_MAX_REL, Y_ROUTED_MEAN_REL, bf16_close, metric_close
 from gpu_common import (assert_routing_equal, create_layer, layer_routing_host, make_device_layer,
                         oracle_layer_for, residual_tokens, routing_buffers, routing_host, routing_struct,
                         to_host_u16)
@@ -63,7 +63,7 @@ def run_all_paths(torch, dl, B, max_batch=None, flags=0, token0=0):
 def check_against_oracle(got, ref, shared=True):
     assert_routing_equal(got["routing"], ref, W_ABS)
     assert_routing_equal(got["fused_routing"], ref, W_ABS)
-    ok, info = metric_close(got["y"], ref["y_routed"], Y_MAX_REL, Y_MEAN_REL)
+    ok, info = metric_close(got["y"], ref["y_routed"], Y_ROUTED_MAX_REL, Y_ROUTED_MEAN_REL)
     assert ok, f"routed expert outputs: {info}"
     if shared:
         ok, info = metric_close(got["ys"], ref["y_shared"], Y_MAX_REL, Y_MEAN_REL)
