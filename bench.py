@@ -146,6 +146,23 @@ def measured_peaks():
     return 6650.0, "fallback"
 
 
+def max_over_ranks(values, device="cpu"):
+    """Element-wise maximum of `values` over all ranks (the slowest replica
+    sets the job's time); identity without a process group."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return [float(v) for v in values]
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
+def job_value(world, total_bytes_per_rank, slowest_ms):
+    """Whole-job GB/s of N replicas: the bytes all ranks moved / the slowest rank's time."""
+    return world * total_bytes_per_rank / (slowest_ms * 1e-3) / 1e9
+
+
 def dist_setup(n_gpus):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -306,9 +323,7 @@ def run_ours(args, cfg):
     gu_avg_s = statistics.mean(gu_ms) * 1e-3
     gu_bytes = statistics.mean([gate_up_bytes(i) for i in range(K)])
     if dist is not None:
-        t = torch.tensor([total_ms, e2e_total], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms, e2e_total = float(t[0]), float(t[1])
+        total_ms, e2e_total = max_over_ranks([total_ms, e2e_total], "cuda")
     api.moe_layer_destroy(handle)
     if dist is not None:
         dist.destroy_process_group()
@@ -316,7 +331,7 @@ def run_ours(args, cfg):
         return
 
     ms_per_step = total_ms / K
-    value = world * total_bytes / (total_ms * 1e-3) / 1e9
+    value = job_value(world, total_bytes, total_ms)
     peak, peak_src = measured_peaks()
     achieved = gu_bytes / gu_avg_s / 1e9
     traffic = recorded_traffic("routed_gate_up", cfg.name)

@@ -658,45 +658,6 @@ __global__ void __launch_bounds__(kMaxConsumerWarps * 32 + 32, 1) gemv_kernel(co
                   acc[r][0] = fmaf(dot32_f16(w, xv), e8m0_to_f32(sv[r]), acc[r][0]);
                 }
               }
-            } else if (TMAX == 1) {
-              // one activation vector: a two-deep software pipeline, the next
-              // chunk's activations, codes and scale bytes are loaded before
-              // this chunk is computed
-              const unsigned char* xs = xbuf + (size_t)tp.slot[0] * xrow_bytes;
-              uint4 xv[4], cv[NWR];
-              uint32_t sv[NWR];
-              auto load_chunk = [&](int bb, uint4 (&xo)[4], uint4 (&co)[NWR], uint32_t (&so)[NWR]) {
-                const int ii = bb >> 5;
-#pragma unroll
-                for (int q = 0; q < 4; ++q) xo[q] = lds128(xs + ((((ii * 4 + q) * 32) + lane) << 4));
-#pragma unroll
-                for (int r = 0; r < NWR; ++r) {
-                  co[r] = lds128(st + (size_t)srow[r] * rowbytes + 16 * bb);
-                  so[r] = a.scales_global ? (uint32_t)__ldg(sgl + (size_t)gsrow[r] * sblocks + bb)
-                                          : lds_u8(scl + srow[r] * sblocks + bb);
-                }
-              };
-              if (lane < C) load_chunk(lane, xv, cv, sv);
-              for (int b = lane; b < C; b += 32) {
-                uint4 xn[4], cn[NWR];
-                uint32_t sn[NWR];
-                if (b + 32 < C) load_chunk(b + 32, xn, cn, sn);
-#pragma unroll
-                for (int r = 0; r < NWR; ++r) {
-                  uint32_t w[16];
-                  decode_chunk(cv[r], w);
-                  acc[r][0] = fmaf(dot32_f16(w, xv), e8m0_to_f32(sv[r]), acc[r][0]);
-                }
-                if (b + 32 < C) {
-#pragma unroll
-                  for (int q = 0; q < 4; ++q) xv[q] = xn[q];
-#pragma unroll
-                  for (int r = 0; r < NWR; ++r) {
-                    cv[r] = cn[r];
-                    sv[r] = sn[r];
-                  }
-                }
-              }
             } else
             for (int b = lane; b < C; b += 32) {
               const int i = b >> 5;

@@ -1,8 +1,9 @@
 """Four full-size layers chained through the residual, batch 1, 64 decode
 steps captured in one CUDA graph (programmatic dependent launch inside,
-next-layer L2 prefetch on): every layer-step output is checked against the
-oracle run on its own residual chain, and the routing of every step is
-bit-exact."""
+next-layer L2 prefetch on).  Each step is a new token: its residual stream
+starts from that token's seeded residual and passes through the four layers
+(out of layer l is the residual of layer l+1).  Every layer-step output is
+checked against the oracle run on its own chain."""
 import numpy as np
 import pytest
 
@@ -14,9 +15,9 @@ from gpu_common import create_layer, make_device_layer, oracle_threads, residual
 pytestmark = pytest.mark.gpu
 
 
-def build_stack_graph(torch, layers, handles, xs, r0, n_steps):
-    """Capture n_steps x n_layers moe_layer_forward calls into one graph.
-    Returns (graph, outs[t][l])."""
+def build_stack_graph(torch, layers, handles, xs, r0s, n_steps):
+    """Capture n_steps x n_layers moe_layer_forward calls into one graph
+    (step t starts from residual r0s[t]).  Returns (graph, outs[t][l])."""
     from sparse_moe_decode_router_b200 import api
     nl = len(handles)
     H = layers[0].cfg.hidden
@@ -27,8 +28,8 @@ def build_stack_graph(torch, layers, handles, xs, r0, n_steps):
     with torch.cuda.stream(s):
         # one eager pass outside capture is not needed: the library allocates nothing per call
         with torch.cuda.graph(g, stream=s):
-            res = r0
             for t in range(n_steps):
+                res = r0s[t]
                 for l in range(nl):
                     nxt = handles[(l + 1) % nl]
                     api.moe_layer_forward(handles[l], nxt, xs[t][l], res, outs[t][l], 1,
@@ -50,10 +51,11 @@ def test_stack4_graph_64_steps_every_step_matches_oracle():
         for t in range(n_steps):
             x_host[t][l] = xh[t:t + 1]
             xs[t][l] = xd[t:t + 1]
-    r0_h, r0 = residual_tokens(cfg, [0], 0)
+    r0_h, r0_d = residual_tokens(cfg, range(n_steps), 0)   # one fresh residual per step (token)
+    r0s = [r0_d[t:t + 1] for t in range(n_steps)]
     handles = [create_layer(dl, 1) for dl in layers]
     try:
-        g, outs = build_stack_graph(torch, layers, handles, xs, r0, n_steps)
+        g, outs = build_stack_graph(torch, layers, handles, xs, r0s, n_steps)
         g.replay()
         torch.cuda.synchronize()
         for hd in handles:
@@ -68,9 +70,9 @@ def test_stack4_graph_64_steps_every_step_matches_oracle():
         for hd in handles:
             api.moe_layer_destroy(hd)
     shared = [dl.host_shared() for dl in layers]
-    res = r0_h
     worst = 0.0
     for t in range(n_steps):
+        res = r0_h[t:t + 1]
         for l in range(nl):
             dl = layers[l]
             rt = oracle.routing(x_host[t][l], dl.router_w_host, None, k)
