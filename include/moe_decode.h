@@ -190,6 +190,39 @@ MOE_API moe_status_t moe_layer_last_device_error(moe_layer_t layer);
  * turns the probe off. */
 MOE_API moe_status_t moe_layer_set_probe(moe_layer_t layer, void* start, void* stop);
 
+/* Router + top-k + softmax + bucketing without any device allocation.
+ *
+ * The decode-path pages have no counterpart of this call; it exists for
+ * callers that cannot allocate device memory: a serving engine that
+ * reserves nearly all of the GPU's memory for weights and KV cache up front
+ * and forbids allocations on the decode path, a host framework whose own
+ * memory pool must account for every device byte, or latency-critical code
+ * that cannot afford the device synchronisation cudaMalloc may imply.  Such
+ * a caller can not create a layer (moe_layer_create allocates), so this
+ * entry takes everything as arguments and keeps its scratch -- the fp32
+ * logits (B * n_experts floats), the top-k kernel's completion counter and
+ * an error word -- in one fixed device array inside the library, sized for
+ * B * n_experts <= 65536 (256 KiB of logits).  Every GPU that loads the
+ * library holds that array until the process exits.
+ *
+ * router_w_em: bf16 [n_experts][hidden], EXPERT-MAJOR (row e is expert e's
+ *   scoring vector: the transpose of moe_layer_weights.router_w).
+ * router_bias: fp32 [n_experts] or NULL.  x: bf16 [B][hidden].
+ * r: where to write the plan (all seven pointers required), as for
+ *   moe_router_topk; the results equal moe_router_topk's bit for bit.
+ * Limits: hidden a multiple of 32, <= 16384; 1 <= n_experts <= 1024;
+ *   1 <= top_k <= min(32, n_experts); 1 <= B <= 64; B * n_experts <= 65536.
+ *   Anything beyond returns MOE_ERR_INVALID_ARG and launches nothing.
+ * The first call on a device (with that device current) looks the array's
+ * device address up and sets the kernels' shared-memory limits; make that
+ * first call before any stream capture.  The counter is cleared on the
+ * stream at the start of every call; the logits are overwritten.  All calls
+ * on a device share the one array, so calls that overlap on the GPU (other
+ * streams, other host threads) race: serialise them. */
+MOE_API moe_status_t moe_router_topk_noalloc(const void* router_w_em, const float* router_bias, int hidden,
+                                             int n_experts, int top_k, const void* x, int B,
+                                             const moe_routing* r, void* stream);
+
 /* Static description string of a status code. */
 MOE_API const char* moe_status_string(moe_status_t s);
 

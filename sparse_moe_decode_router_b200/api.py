@@ -30,7 +30,7 @@ MOE_FLAG_NO_GROUPED = 0x8
 EXPORTS = (
     "moe_layer_create", "moe_layer_destroy", "moe_router_topk", "moe_experts_mxfp4",
     "moe_combine_residual", "moe_layer_forward", "moe_layer_forward_host", "moe_layer_routing",
-    "moe_layer_last_device_error", "moe_layer_set_probe", "moe_status_string",
+    "moe_layer_last_device_error", "moe_layer_set_probe", "moe_router_topk_noalloc", "moe_status_string",
 )
 
 
@@ -81,6 +81,7 @@ def load_library(path: str = LIB_PATH):
         "moe_layer_routing": [vp, ctypes.POINTER(moe_routing)],
         "moe_layer_last_device_error": [vp],
         "moe_layer_set_probe": [vp, vp, vp],
+        "moe_router_topk_noalloc": [vp, vp, i32, i32, i32, vp, i32, ctypes.POINTER(moe_routing), vp],
     }
     for name, args in sig.items():
         f = getattr(L, name)
@@ -173,3 +174,12 @@ def moe_layer_set_probe(layer: int, start_event=None, stop_event=None):
     s = None if start_event is None else start_event.cuda_event
     e = None if stop_event is None else stop_event.cuda_event
     _check("moe_layer_set_probe", load_library().moe_layer_set_probe(layer, s, e))
+
+
+def moe_router_topk_noalloc(router_w_em, router_bias, hidden: int, n_experts: int, top_k: int, x, B: int,
+                            routing: moe_routing, stream=None):
+    """Router + top-k + bucketing with no device allocation (see the header).
+    router_w_em is the expert-major [E][H] bf16 router matrix."""
+    _check("moe_router_topk_noalloc", load_library().moe_router_topk_noalloc(
+        _ptr(router_w_em), _ptr(router_bias), hidden, n_experts, top_k, _ptr(x), B, ctypes.byref(routing),
+        _stream(stream)))

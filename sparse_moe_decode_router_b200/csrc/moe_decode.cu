@@ -6,6 +6,7 @@
 #include <algorithm>
 #include <cstdint>
 #include <cstring>
+#include <mutex>
 #include <new>
 
 #include "../../include/moe_decode.h"
@@ -132,6 +133,25 @@ GemvFn gemv_fn(Kind k, int tmax) { return tmax == 1 ? pick_fn<1>(k) : pick_fn<2>
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 }  // namespace
+
+// ---------------------------------------------------------------------------
+// Allocation-free router/top-k: its only scratch (the fp32 logits, the top-k
+// kernel's CTA counter and an error word) lives in this file-scope device
+// array.  Host code must not use the array's name as a device address; the
+// address comes from cudaGetSymbolAddress, once per device.
+namespace {
+constexpr int kNoAllocMaxLogits = kMaxBatch * kMaxExperts;  // 65536 floats (B * E)
+struct NoAllocScratch {
+  float logits[kNoAllocMaxLogits];
+  int done_counter;
+  int err;
+};
+constexpr int kNoAllocMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kNoAllocMaxDevices] = {};
+int g_noalloc_sms[kNoAllocMaxDevices] = {};
+}  // namespace
+static __device__ __align__(256) unsigned char g_noalloc_scratch[sizeof(NoAllocScratch)];
 
 struct moe_layer {
   moe_layer_config cfg{};
@@ -612,6 +632,92 @@ moe_status_t moe_layer_last_device_error(moe_layer_t L) {
   cudaMemset(L->router_cnt, 0, sizeof(int));
   cudaMemset(L->tile_cnt, 0, sizeof(int) * L->cfg.hidden);
   return v == kErrTimeout ? MOE_ERR_TIMEOUT : MOE_ERR_INVALID_ARG;
+}
+
+moe_status_t moe_router_topk_noalloc(const void* router_w_em, const float* router_bias, int hidden, int n_experts,
+                                     int top_k, const void* x, int B, const moe_routing* r, void* stream) {
+  if (!router_w_em || !x || !aligned16(router_w_em) || !aligned16(x) || !routing_ok(r)) return MOE_ERR_INVALID_ARG;
+  if (hidden <= 0 || hidden % 32 || hidden > 32 * 32 * 16 || n_experts < 1 || n_experts > kMaxExperts || top_k < 1 ||
+      top_k > kMaxTopK || top_k > n_experts || B < 1 || B > kMaxBatch || (long long)B * n_experts > kNoAllocMaxLogits)
+    return MOE_ERR_INVALID_ARG;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
+  if (dev < 0 || dev >= kNoAllocMaxDevices) return MOE_ERR_UNSUPPORTED;
+  void* base = nullptr;
+  int sms = 0;
+  {
+    // first call on this device: resolve the array's device address (with the
+    // device current) and raise the kernels' shared-memory limits
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (!g_noalloc_ptr[dev]) {
+      int major = 0;
+      if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+          cudaDeviceGetAttribute(&g_noalloc_sms[dev], cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return MOE_ERR_CUDA;
+      if (major != 10) return MOE_ERR_UNSUPPORTED;
+      void* ptr = nullptr;
+      if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || !ptr) return MOE_ERR_CUDA;
+      for (int t = 0; t < 2; ++t) {
+        const GemvPlan p = make_plan(K_ROUTER, hidden, n_experts, t == 0 ? 1 : kMaxBatch, 1, t == 0 ? 1 : kMaxBatch,
+                                     0, g_noalloc_sms[dev]);
+        if (!p.ok) return MOE_ERR_UNSUPPORTED;
+      }
+      // the largest dynamic shared memory any router plan asks for
+      if (cudaFuncSetAttribute(gemv_fn(K_ROUTER, 1), cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBudget) !=
+              cudaSuccess ||
+          cudaFuncSetAttribute(gemv_fn(K_ROUTER, 2), cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBudget) !=
+              cudaSuccess)
+        return MOE_ERR_CUDA;
+      g_noalloc_ptr[dev] = ptr;
+    }
+    base = g_noalloc_ptr[dev];
+    sms = g_noalloc_sms[dev];
+  }
+  NoAllocScratch* sc = static_cast<NoAllocScratch*>(base);
+  const GemvPlan p = make_plan(K_ROUTER, hidden, n_experts, B, 1, B, 0, sms);
+  if (!p.ok) return MOE_ERR_UNSUPPORTED;
+  cudaStream_t st = (cudaStream_t)stream;
+  // the counter must start at zero (a call cut short could leave it set)
+  cudaError_t e = cudaMemsetAsync(&sc->done_counter, 0, sizeof(int), st);
+  if (e != cudaSuccess) return MOE_ERR_CUDA;
+  GemvArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.K = p.K;
+  a.out_rows = p.out_rows;
+  a.R = p.R;
+  a.ncw = p.ncw;
+  a.wpi = p.wpi;
+  a.n_stages = p.n_stages;
+  a.stage_bytes = p.stage_bytes;
+  a.stage_offset = p.stage_offset;
+  a.x_offset = p.x_offset;
+  a.xcap = p.xcap;
+  a.top_k = top_k;
+  a.n_experts = n_experts;
+  a.err = &sc->err;
+  a.w = static_cast<const uint8_t*>(router_w_em);
+  a.act = x;
+  a.n_tokens = B;
+  a.out = sc->logits;
+  a.bias = router_bias;
+  const int tm = tmax_for(B);
+  e = launch_ex(gemv_fn(K_ROUTER, tm), sms, p.threads, p.smem, st, false, a);
+  if (e != cudaSuccess) return MOE_ERR_CUDA;
+  GemvArgs t;
+  std::memset(&t, 0, sizeof(t));
+  t.out = sc->logits;
+  t.n_experts = n_experts;
+  t.top_k = top_k;
+  t.n_tokens = B;
+  t.topk_w = r->topk_w;
+  t.topk_idx = r->topk_idx;
+  t.counts = r->counts;
+  t.offsets_out = r->offsets;
+  t.pair_ids_out = r->pair_ids;
+  t.active_out = r->active;
+  t.n_active_out = r->n_active;
+  t.done_counter = &sc->done_counter;
+  return cuda_status(launch_ex(topk_bucket_kernel, B, kTopkWarps * 32, 0, st, true, t));
 }
 
 moe_status_t moe_layer_set_probe(moe_layer_t L, void* start, void* stop) {

@@ -1,0 +1,48 @@
+"""The allocation-free router entry point (moe_router_topk_noalloc).
+
+It serves callers that cannot allocate device memory (an engine that has
+reserved the GPU's memory up front, a framework that must account for every
+device byte).  Its scratch is a fixed array inside the library, shared by all
+calls, so the check runs two calls in a row with different inputs: each must
+reproduce what the allocating entry point (moe_router_topk on a layer)
+returns for the same inputs.  This file sorts last so that a run stopping at
+the first failure has already run every other test."""
+import numpy as np
+import pytest
+
+import synth
+from gpu_common import create_layer, make_device_layer, routing_buffers, routing_host, routing_struct
+
+pytestmark = pytest.mark.gpu
+
+
+def test_noalloc_router_matches_layer_router_twice():
+    import torch
+    from sparse_moe_decode_router_b200 import api
+    if not torch.cuda.is_available():
+        pytest.fail("GPU tests need a CUDA device")
+    api.load_library()
+    cfg = synth.CONFIGS[0].with_(zipf_s=1.1, seed=synth.CONFIGS[0].seed + 7)   # with a router bias
+    dl = make_device_layer(cfg)
+    H, E, k = cfg.hidden, cfg.n_experts, cfg.top_k
+    w_em = dl.router_w.t().contiguous()          # expert-major copy, made by the caller
+    h = create_layer(dl, 64)
+    try:
+        for call, B in enumerate((5, 64)):
+            _, x = dl.tokens(range(100 * call, 100 * call + B))
+            want = routing_buffers(B, k, E)
+            api.moe_router_topk(h, x, B, routing_struct(want))
+            got = routing_buffers(B, k, E)
+            api.moe_router_topk_noalloc(w_em, dl.router_bias, H, E, k, x, B, routing_struct(got))
+            torch.cuda.synchronize()
+            g, w = routing_host(got), routing_host(want)
+            for key in ("topk_idx", "counts", "offsets", "pair_ids", "active"):
+                assert np.array_equal(g[key], w[key]), (call, key)
+            assert g["n_active"] == w["n_active"]
+            assert np.array_equal(g["topk_w"], w["topk_w"]), call   # same kernels: bit-identical
+        # sizes beyond the fixed scratch are refused, nothing launched
+        with pytest.raises(api.MoEError) as e:
+            api.moe_router_topk_noalloc(w_em, None, H, E, k, x, 65, routing_struct(routing_buffers(1, k, E)))
+        assert e.value.status == api.MOE_ERR_INVALID_ARG
+    finally:
+        api.moe_layer_destroy(h)
