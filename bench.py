@@ -114,7 +114,7 @@ class ClockSampler:
 # ------------------------------------------------------------- helpers ------
 def kernel_source_sha():
     h = hashlib.sha256()
-    for f in ("kernels.cuh", "ptx.cuh", "moe_decode.cu"):
+    for f in ("kernels.cuh", "gemv.cuh", "ptx.cuh", "moe_decode.cu"):
         with open(os.path.join(ROOT, "sparse_moe_decode_router_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]

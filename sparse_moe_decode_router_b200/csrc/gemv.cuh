@@ -348,6 +348,26 @@ __host__ __device__ constexpr int x_row_bytes(int wf, int xk, int K) {
 }
 
 // ---------------------------------------------------------------------------
+// Scale bytes of one item for this warp's rows and this lane's chunks (the
+// shape-specialised path reads them from global memory, one item ahead).
+template <int NWR, int RPW, bool kSwiglu, int kCPL>
+__device__ __forceinline__ void load_item_scales(const GemvArgs& a, int grp, int rt, int wi, int lane, int C,
+                                                 int sblocks, float (&out)[NWR][kCPL]) {
+  const uint8_t* sgl = a.sc + (long long)grp * a.s_gstride;
+  const int r0 = rt * a.R;
+#pragma unroll
+  for (int r = 0; r < NWR; ++r) {
+    const int sr = kSwiglu ? (r < RPW ? wi * RPW + r : a.R + wi * RPW + (r - RPW)) : wi * RPW + r;
+    const int gr = kSwiglu && sr >= a.R ? r0 + a.up_off + sr - a.R : r0 + sr;
+#pragma unroll
+    for (int ci = 0; ci < kCPL; ++ci) {
+      const int b = lane + 32 * ci;
+      out[r][ci] = e8m0_to_f32((b < C) ? (uint32_t)__ldg(sgl + (size_t)gr * sblocks + b) : 127u);
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
 // Fused combine bookkeeping.  A warp group writes the unweighted expert
 // outputs y of its items to the scratch; every kPubBatch items it meets on a
 // group barrier (all of the group's y stores are then ordered before the
@@ -407,16 +427,23 @@ struct TokenPass {
 
 // RPW = output rows per warp (SwiGLU: one gate row and one up row per output row).
 // An item (R = RPW * wpi output rows, one stage) is shared by a group of wpi warps.
-template <int WF, int EPI, int XK, int TMAX, int RPW>
+// KT: the reduction length as a compile-time constant (0 = taken from the
+// arguments).  Specialised instances unroll the chunk loop with constant
+// addressing and, for MXFP4, read the E8M0 scale bytes from global memory with
+// loads issued ahead of the stage wait (the stage then holds codes only).
+template <int WF, int EPI, int XK, int TMAX, int RPW, int KT>
 __global__ void __launch_bounds__(kMaxConsumerWarps * 32 + 32, 1) gemv_kernel(const GemvArgs a) {
   constexpr bool kSwiglu = (EPI == EPI_SWIGLU);
   constexpr int NWR = kSwiglu ? 2 * RPW : RPW;  // weight rows per warp
   static_assert(NWR % 2 == 0, "rows are processed in pairs");
+  constexpr bool kFast = (KT != 0) && (WF == W_MXFP4) && (TMAX == 1);
+  constexpr int kCPL = KT ? ((KT / 32) + 31) / 32 : 1;  // chunks per lane (fast path)
   extern __shared__ __align__(128) unsigned char smem[];
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int ncw = a.ncw;
-  const int K = a.K;
+  const int K = KT ? KT : a.K;
+  const bool sglobal = (KT != 0 && WF == W_MXFP4) ? true : (a.scales_global != 0);
   const int C = K >> 5;                                   // 32-element chunks per row
   const int rowbytes = (WF == W_MXFP4) ? (K >> 1) : (K << 1);
   const int sblocks = K >> 5;
@@ -508,12 +535,12 @@ __global__ void __launch_bounds__(kMaxConsumerWarps * 32 + 32, 1) gemv_kernel(co
           const int r0 = rt * a.R;
           unsigned char* st = stages + (size_t)s * a.stage_bytes;
           const uint32_t cb = (uint32_t)(a.R * rowbytes);
-          const uint32_t sb = (WF == W_MXFP4 && !a.scales_global) ? (uint32_t)(a.R * sblocks) : 0u;
+          const uint32_t sb = (WF == W_MXFP4 && !sglobal) ? (uint32_t)(a.R * sblocks) : 0u;
           mbar_arrive_expect_tx(&full_bar[s], (kSwiglu ? 2u : 1u) * (cb + sb));
           const uint8_t* wg = a.w + (long long)grp * a.w_gstride;
           bulk_g2s(st, wg + (size_t)r0 * rowbytes, cb, &full_bar[s], pol);
           if (kSwiglu) bulk_g2s(st + cb, wg + (size_t)(r0 + a.up_off) * rowbytes, cb, &full_bar[s], pol);
-          if (WF == W_MXFP4 && !a.scales_global) {
+          if (WF == W_MXFP4 && !sglobal) {
             const uint8_t* sg = a.sc + (long long)grp * a.s_gstride;
             bulk_g2s(st + codes_bytes, sg + (size_t)r0 * sblocks, sb, &full_bar[s], pol);
             if (kSwiglu)
@@ -543,6 +570,8 @@ __global__ void __launch_bounds__(kMaxConsumerWarps * 32 + 32, 1) gemv_kernel(co
       named_bar_sync(1, nct);
       const int nit = ph.last_item - ph.first_item;
       int c_g = -1, c_grp = 0, c_tok0 = 0, c_ntok = 1, c_tp_tb = -1;
+      float snext[kFast ? NWR : 1][kFast ? kCPL : 1];  // next item's scales, fp32 (fast path)
+      (void)snext;
       int pend_rt[kPubBatch], npend = 0;  // fused combine: items written, not yet published
       int prev_cnt = 0, prev_rt = 0, nprev = 0;  // last published batch: atomic result per lane
       (void)pend_rt; (void)npend; (void)prev_cnt; (void)prev_rt; (void)nprev;
@@ -583,6 +612,25 @@ __global__ void __launch_bounds__(kMaxConsumerWarps * 32 + 32, 1) gemv_kernel(co
         const int tlo = a.routed ? max(0, ph.t0) : ph.t0;
         const int thi = a.routed ? min(ntok, ph.t1) : ph.t1;
 
+        // fast path: scale bytes come from global memory one item ahead -- this
+        // item's were loaded during the previous item, the next item's go out now
+        float sreg[kFast ? NWR : 1][kFast ? kCPL : 1];
+        if constexpr (kFast) {
+          if (jj == q0) load_item_scales<NWR, RPW, kSwiglu, kCPL>(a, grp, rt, wi, lane, C, sblocks, sreg);
+          else {
+#pragma unroll
+            for (int r = 0; r < NWR; ++r)
+#pragma unroll
+              for (int ci = 0; ci < kCPL; ++ci) sreg[r][ci] = snext[r][ci];
+          }
+          const int jn = jj + ng;
+          if (jn < nit) {
+            int gn = g, rtn = rt + ng;
+            while (rtn >= n_rt) { rtn -= n_rt; ++gn; }
+            const int grpn = a.routed ? clamp_group(a.active[gn], a.n_experts, nullptr) : 0;
+            load_item_scales<NWR, RPW, kSwiglu, kCPL>(a, grpn, rtn, wi, lane, C, sblocks, snext);
+          }
+        }
         bool have = !skip;
         if (have && !mbar_wait_bounded(&full_bar[s], par)) {
           if (lane == 0) atomicExch(a.err, kErrTimeout);
@@ -626,7 +674,28 @@ __global__ void __launch_bounds__(kMaxConsumerWarps * 32 + 32, 1) gemv_kernel(co
 #pragma unroll
           for (int r = 0; r < NWR; ++r)
             srow[r] = kSwiglu ? (r < RPW ? wi * RPW + r : a.R + wi * RPW + (r - RPW)) : wi * RPW + r;
-          if constexpr (WF == W_MXFP4) {
+          if constexpr (kFast) {
+            // one activation vector, compile-time K: every chunk of this lane, unrolled,
+            // 32-bit shared addresses with constant offsets
+            const uint32_t xs_s = smem_addr(xbuf) + (uint32_t)(tp.slot[0] * xrow_bytes) + 16u * lane;
+            uint32_t rb_s[NWR];
+#pragma unroll
+            for (int r = 0; r < NWR; ++r) rb_s[r] = smem_addr(st) + (uint32_t)(srow[r] * rowbytes) + 16u * lane;
+#pragma unroll
+            for (int ci = 0; ci < kCPL; ++ci) {
+              if (lane + 32 * ci < C) {
+                uint4 xv[4];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) xv[q] = lds128_s(xs_s + (uint32_t)((ci * 4 + q) * 512));
+#pragma unroll
+                for (int r = 0; r < NWR; ++r) {
+                  uint32_t w[16];
+                  decode_chunk(lds128_s(rb_s[r] + 512u * ci), w);
+                  acc[r][0] = fmaf(dot32_f16(w, xv), sreg[r][ci], acc[r][0]);
+                }
+              }
+            }
+          } else if constexpr (WF == W_MXFP4) {
             // scale rows: in the stage after the codes, or (short rows) straight from global
             const uint8_t* scl = st + codes_bytes;
             const uint8_t* sgl = a.sc + (long long)grp * a.s_gstride;
@@ -648,7 +717,7 @@ __global__ void __launch_bounds__(kMaxConsumerWarps * 32 + 32, 1) gemv_kernel(co
 #pragma unroll
                 for (int r = 0; r < NWR; ++r) {
                   cv[r] = lds128(st + (size_t)srow[r] * rowbytes + 16 * b);
-                  sv[r] = a.scales_global ? (uint32_t)__ldg(sgl + (size_t)gsrow[r] * sblocks + b)
+                  sv[r] = sglobal ? (uint32_t)__ldg(sgl + (size_t)gsrow[r] * sblocks + b)
                                           : lds_u8(scl + srow[r] * sblocks + b);
                 }
 #pragma unroll
@@ -673,7 +742,7 @@ __global__ void __launch_bounds__(kMaxConsumerWarps * 32 + 32, 1) gemv_kernel(co
                   for (int r = 0; r < NWR; ++r) {
                     uint32_t w[16];
                     decode_chunk(lds128(st + (size_t)srow[r] * rowbytes + 16 * b), w);
-                    const float sc = a.scales_global ? e8m0_to_f32(__ldg(sgl + (size_t)gsrow[r] * sblocks + b))
+                    const float sc = sglobal ? e8m0_to_f32(__ldg(sgl + (size_t)gsrow[r] * sblocks + b))
                                                      : e8m0_to_f32(lds_u8(scl + srow[r] * sblocks + b));
                     acc[r][t] = fmaf(dot32_f16(w, xv), sc, acc[r][t]);
                   }

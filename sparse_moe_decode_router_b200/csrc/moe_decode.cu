@@ -54,6 +54,7 @@ struct GemvPlan {
   bool ok = false;
   int K = 0, out_rows = 0, R = 0, ncw = 0, wpi = 0, n_stages = 0, stage_bytes = 0, stage_offset = 0, x_offset = 0;
   int xcap = 0, scales_global = 0, threads = 0, smem = 0;
+  bool fast = false;  // run the shape-specialised one-token instance
 };
 
 // Work decomposition of one weight stream.  `slots_needed` = activation
@@ -61,7 +62,7 @@ struct GemvPlan {
 // `max_groups` = most groups (experts) the stream can have active,
 // `tok_per_group` = most activation vectors one group uses.
 GemvPlan make_plan(Kind kind, int K, int out_rows, int slots_needed, int max_groups, int tok_per_group,
-                   long long s_gstride, int num_sms) {
+                   long long s_gstride, int num_sms, bool fast = false) {
   GemvPlan p;
   const KindTraits t = kTraits[kind];
   const int R = t.rpw * t.wpi;
@@ -71,8 +72,9 @@ GemvPlan make_plan(Kind kind, int K, int out_rows, int slots_needed, int max_gro
   const int rowbytes = mx ? K / 2 : K * 2;
   const int sbytes = mx ? K / 32 : 0;
   const int rows = swiglu ? 2 * R : R;
-  // scale rows go through TMA only when every copy is 16-byte aligned and sized
-  const bool sg = mx && (((long long)R * sbytes) % 16 != 0 || s_gstride % 16 != 0);
+  // scale rows go through TMA only when every copy is 16-byte aligned and sized;
+  // the shape-specialised (fast) instances always read them from global memory
+  const bool sg = mx && (fast || ((long long)R * sbytes) % 16 != 0 || s_gstride % 16 != 0);
   const int stage = (int)align_up((size_t)rows * (rowbytes + (mx && !sg ? sbytes : 0)), 128);
   // activation slots: a CTA's contiguous item range spans at most
   // ceil(items per CTA / items per group) + 1 groups
@@ -110,25 +112,37 @@ GemvPlan make_plan(Kind kind, int K, int out_rows, int slots_needed, int max_gro
   p.scales_global = sg ? 1 : 0;
   p.threads = (p.ncw + 1) * 32;
   p.smem = st_off + ns * stage;
+  p.fast = fast;
   return p;
 }
 
 typedef void (*GemvFn)(const GemvArgs);
 
-template <int TMAX>
+// Reduction lengths with shape-specialised instances (the full-size layer).
+constexpr int kFastH = 7168;
+constexpr int kFastI = 2048;
+
+template <int TMAX, int KH, int KI>
 GemvFn pick_fn(Kind k) {
   switch (k) {
-    case K_ROUTER: return gemv_kernel<W_BF16, EPI_ROUTER, X_BF16, TMAX, 2>;
-    case K_SGU: return gemv_kernel<W_BF16, EPI_SWIGLU, X_BF16, TMAX, 1>;
-    case K_SDN: return gemv_kernel<W_BF16, EPI_STORE, X_F32, TMAX, 2>;
-    case K_GU: return gemv_kernel<W_MXFP4, EPI_SWIGLU, X_BF16, TMAX, MOE_GU_RPW>;
-    case K_DN: return gemv_kernel<W_MXFP4, EPI_STORE, X_F32, TMAX, MOE_DN_RPW>;
-    case K_DNC: return gemv_kernel<W_MXFP4, EPI_DOWN_COMBINE, X_F32, TMAX, MOE_DN_RPW>;
+    case K_ROUTER: return gemv_kernel<W_BF16, EPI_ROUTER, X_BF16, TMAX, 2, KH>;
+    case K_SGU: return gemv_kernel<W_BF16, EPI_SWIGLU, X_BF16, TMAX, 1, KH>;
+    case K_SDN: return gemv_kernel<W_BF16, EPI_STORE, X_F32, TMAX, 2, KI>;
+    case K_GU: return gemv_kernel<W_MXFP4, EPI_SWIGLU, X_BF16, TMAX, MOE_GU_RPW, KH>;
+    case K_DN: return gemv_kernel<W_MXFP4, EPI_STORE, X_F32, TMAX, MOE_DN_RPW, KI>;
+    case K_DNC: return gemv_kernel<W_MXFP4, EPI_DOWN_COMBINE, X_F32, TMAX, MOE_DN_RPW, KI>;
     default: return nullptr;
   }
 }
 
-GemvFn gemv_fn(Kind k, int tmax) { return tmax == 1 ? pick_fn<1>(k) : pick_fn<2>(k); }
+// the K each stream reduces over in the full-size layer
+int fast_k(Kind k) { return (k == K_SDN || k == K_DN || k == K_DNC) ? kFastI : kFastH; }
+
+// fast = the shape-specialised one-token instance (K must equal fast_k(k))
+GemvFn gemv_fn(Kind k, int tmax, bool fast = false) {
+  if (tmax == 1) return fast ? pick_fn<1, kFastH, kFastI>(k) : pick_fn<1, 0, 0>(k);
+  return pick_fn<2, 0, 0>(k);
+}
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -226,7 +240,7 @@ GemvArgs base_args(const moe_layer* L, const GemvPlan& p) {
 cudaError_t run_gemv(moe_layer* L, Kind k, int B, const GemvArgs& a, cudaStream_t st, bool pdl) {
   const int tm = tmax_for(B);
   const GemvPlan& p = L->plans[k][tm == 1 ? 0 : 1];
-  return launch_ex(gemv_fn(k, tm), L->num_sms, p.threads, p.smem, st, pdl, a);
+  return launch_ex(gemv_fn(k, tm, p.fast), L->num_sms, p.threads, p.smem, st, pdl, a);
 }
 
 const GemvPlan& plan_of(const moe_layer* L, Kind k, int B) { return L->plans[k][tmax_for(B) == 1 ? 0 : 1]; }
@@ -423,13 +437,14 @@ moe_status_t moe_layer_create(const moe_layer_config* cfg, const moe_layer_weigh
   for (int t = 0; t < 2; ++t) {
     const int nb = t == 0 ? 1 : MB;
     const int maxg = std::min(E, nb * k);  // experts one call can activate
-    L->plans[K_ROUTER][t] = make_plan(K_ROUTER, H, E, nb, 1, nb, 0, sms);
-    L->plans[K_GU][t] = make_plan(K_GU, H, I, nb, maxg, nb, (long long)2 * I * (H / 32), sms);
-    L->plans[K_DN][t] = make_plan(K_DN, I, H, nb * k, maxg, nb, (long long)H * (I / 32), sms);
-    L->plans[K_DNC][t] = make_plan(K_DNC, I, H, nb * k, maxg, nb, (long long)H * (I / 32), sms);
+    const bool fh = t == 0 && H == kFastH, fi = t == 0 && I == kFastI, fis = t == 0 && Is == kFastI;
+    L->plans[K_ROUTER][t] = make_plan(K_ROUTER, H, E, nb, 1, nb, 0, sms, fh);
+    L->plans[K_GU][t] = make_plan(K_GU, H, I, nb, maxg, nb, (long long)2 * I * (H / 32), sms, fh);
+    L->plans[K_DN][t] = make_plan(K_DN, I, H, nb * k, maxg, nb, (long long)H * (I / 32), sms, fi);
+    L->plans[K_DNC][t] = make_plan(K_DNC, I, H, nb * k, maxg, nb, (long long)H * (I / 32), sms, fi);
     if (Is > 0) {
-      L->plans[K_SGU][t] = make_plan(K_SGU, H, Is, nb, 1, nb, 0, sms);
-      L->plans[K_SDN][t] = make_plan(K_SDN, Is, H, nb, 1, nb, 0, sms);
+      L->plans[K_SGU][t] = make_plan(K_SGU, H, Is, nb, 1, nb, 0, sms, fh);
+      L->plans[K_SDN][t] = make_plan(K_SDN, Is, H, nb, 1, nb, 0, sms, fis);
     }
     bool ok = L->plans[K_ROUTER][t].ok && L->plans[K_GU][t].ok && L->plans[K_DN][t].ok && L->plans[K_DNC][t].ok;
     if (Is > 0) ok = ok && L->plans[K_SGU][t].ok && L->plans[K_SDN][t].ok;
@@ -504,7 +519,7 @@ moe_status_t moe_layer_create(const moe_layer_config* cfg, const moe_layer_weigh
     for (int t = 0; t < 2 && e == cudaSuccess; ++t) {
       const GemvPlan& p = L->plans[kk][t];
       if (!p.ok) continue;
-      e = cudaFuncSetAttribute(gemv_fn((Kind)kk, t == 0 ? 1 : 2), cudaFuncAttributeMaxDynamicSharedMemorySize,
+      e = cudaFuncSetAttribute(gemv_fn((Kind)kk, t == 0 ? 1 : 2, p.fast), cudaFuncAttributeMaxDynamicSharedMemorySize,
                                p.smem);
     }
   if (e == cudaSuccess) e = cudaDeviceSynchronize();

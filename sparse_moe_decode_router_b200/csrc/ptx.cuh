@@ -110,6 +110,13 @@ __device__ __forceinline__ uint4 lds128(const void* p) {
   return v;
 }
 
+// loads from a 32-bit shared-memory address (no generic-address conversion)
+__device__ __forceinline__ uint4 lds128_s(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+  return v;
+}
+
 __device__ __forceinline__ uint32_t lds_u8(const void* p) {
   uint32_t v;
   asm volatile("ld.shared.u8 %0, [%1];" : "=r"(v) : "r"(smem_addr(p)));
