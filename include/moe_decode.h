@@ -72,7 +72,9 @@ typedef struct moe_layer* moe_layer_t; /* opaque, library-owned */
 
 /* Flags (moe_layer_config.flags); the defaults are the fastest path. */
 #define MOE_FLAG_NO_PDL 0x1u        /* launch without programmatic dependent launch */
-#define MOE_FLAG_NO_SIDE_STREAM 0x2u /* run the shared expert on the caller's stream */
+#define MOE_FLAG_SIDE_STREAM 0x2u   /* fork the shared expert onto the layer's side stream and
+                                      join it before the down projection (default: it runs on
+                                      the caller's stream, overlapping the top-k) */
 #define MOE_FLAG_NO_PREFETCH 0x4u   /* no L2 prefetch of the next layer's weights */
 #define MOE_FLAG_NO_GROUPED 0x8u    /* never use the tensor-core grouped expert path */
 
@@ -142,8 +144,9 @@ MOE_API moe_status_t moe_router_topk(moe_layer_t layer, const void* x, int B, co
  * plan from moe_router_topk (r NULL = the layer's own plan).
  * y_routed: fp32 [B*k][H], row p = unweighted output of pair p's expert;
  * y_shared: fp32 [B][H] (ignored, may be NULL, when I_s = 0).
- * The shared expert runs on the layer's side stream, joined back before
- * return (pages: yeyulingfeng section 02; smzdm, third step). */
+ * With MOE_FLAG_SIDE_STREAM the shared expert runs on the layer's side
+ * stream, joined back before return (pages: yeyulingfeng section 02; smzdm,
+ * third step); otherwise on `stream` after the routed experts. */
 MOE_API moe_status_t moe_experts_mxfp4(moe_layer_t layer, const void* x, int B, const moe_routing* r,
                                float* y_routed, float* y_shared, void* stream);
 
@@ -156,9 +159,12 @@ MOE_API moe_status_t moe_combine_residual(moe_layer_t layer, int B, const moe_ro
                                   const float* y_routed, const float* y_shared,
                                   const void* residual, void* out, void* stream);
 
-/* The whole layer in one call: router/top-k/buckets, routed experts, shared
- * expert on the side stream, down projection fused with the combine and
- * residual add.  Kernels are chained with programmatic dependent launch;
+/* The whole layer in one call: router/top-k/buckets, shared expert, routed
+ * experts, down projection fused with the combine and residual add.  Kernels
+ * are chained with programmatic dependent launch on `stream`; the shared
+ * expert's gate/up kernel starts while the top-k runs (it needs only x), so
+ * it overlaps the routing latency the way the pages' side stream does
+ * (MOE_FLAG_SIDE_STREAM forks it onto a side stream instead);
  * with `next` non-NULL the tail of this layer prefetches next's router and
  * shared-expert weights into L2 (pages: yeyulingfeng section 02, third and
  * fourth optimisations).  x, residual, out: bf16 [B][H]; out may equal

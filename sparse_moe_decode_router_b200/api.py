@@ -22,7 +22,7 @@ MOE_ERR_OOM = 4
 MOE_ERR_TIMEOUT = 5
 
 MOE_FLAG_NO_PDL = 0x1
-MOE_FLAG_NO_SIDE_STREAM = 0x2
+MOE_FLAG_SIDE_STREAM = 0x2
 MOE_FLAG_NO_PREFETCH = 0x4
 MOE_FLAG_NO_GROUPED = 0x8
 

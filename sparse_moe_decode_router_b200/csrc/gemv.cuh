@@ -43,6 +43,15 @@ enum XKind : int { X_BF16 = 0, X_F32 = 1 };
 #define MOE_MAX_CONSUMER_WARPS 12
 #endif
 constexpr int kMaxConsumerWarps = MOE_MAX_CONSUMER_WARPS;
+// Split-K instances (one token, MXFP4, compile-time K): more, lighter warps.
+#ifndef MOE_MAX_SPLITK_WARPS
+#define MOE_MAX_SPLITK_WARPS 16
+#endif
+constexpr int kMaxSplitKWarps = MOE_MAX_SPLITK_WARPS;
+constexpr int kMaxWarpsAny = kMaxSplitKWarps > kMaxConsumerWarps ? kMaxSplitKWarps : kMaxConsumerWarps;
+constexpr int kSplitKRows = 8;  // weight rows per warp in the split-K instances
+// cross-warp partial sums of the split-K instances: two item buffers per group
+constexpr int kRedFloats = 2 * kMaxSplitKWarps * kSplitKRows;
 constexpr int kMaxStagesDev = 24;     // stage ring slots the shared-memory header reserves
 constexpr int kMaxStageUnits = 64;    // (vector, segment) units of one staging pass
 constexpr int kMaxPhases = 32;
@@ -63,18 +72,31 @@ struct PhaseTable {
 };
 
 // ---------------------------------------------------------------------------
-// mixed-precision FMAs: fp32 accumulator, two f16 (or bf16) products from packed pairs
-__device__ __forceinline__ float fma2_f16(uint32_t w2, uint32_t x2, float acc) {
-  asm("{\n\t.reg .f16 a0, a1, b0, b1;\n\t"
-      "mov.b32 {a0, a1}, %1;\n\t"
-      "mov.b32 {b0, b1}, %2;\n\t"
-      "fma.rn.f32.f16 %0, a0, b0, %0;\n\t"
-      "fma.rn.f32.f16 %0, a1, b1, %0;\n\t}"
-      : "+f"(acc)
-      : "r"(w2), "r"(x2));
-  return acc;
+// packed f16x2 multiply-adds (one rounding each) and the f16x2 -> fp32 sum
+__device__ __forceinline__ uint32_t hmul2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
 }
 
+__device__ __forceinline__ uint32_t hfma2(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t d;
+  asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+
+__device__ __forceinline__ float h2_sum_f32(uint32_t v) {
+  float lo, hi;
+  asm("{\n\t.reg .f16 l, h;\n\t"
+      "mov.b32 {l, h}, %2;\n\t"
+      "cvt.f32.f16 %0, l;\n\t"
+      "cvt.f32.f16 %1, h;\n\t}"
+      : "=f"(lo), "=f"(hi)
+      : "r"(v));
+  return lo + hi;
+}
+
+// mixed-precision FMAs: fp32 accumulator, two bf16 products from packed pairs
 __device__ __forceinline__ float fma2_bf16(uint32_t w2, uint32_t x2, float acc) {
   asm("{\n\t.reg .b16 a0, a1, b0, b1;\n\t"
       "mov.b32 {a0, a1}, %1;\n\t"
@@ -86,18 +108,26 @@ __device__ __forceinline__ float fma2_bf16(uint32_t w2, uint32_t x2, float acc) 
   return acc;
 }
 
-// 32-element MXFP4 chunk (16 code bytes = 16 f16x2 after decode) dotted with a
-// 32-element f16 activation chunk (4 x 16 bytes, lane-interleaved), 4 chains.
-__device__ __forceinline__ float dot32_f16(const uint32_t (&w)[16], const uint4 (&xv)[4]) {
-  float p0 = 0.f, p1 = 0.f, p2 = 0.f, p3 = 0.f;
+// 32-element MXFP4 chunk (16 code bytes = 16 f16x2 after decode, element pair
+// j in w[j]) dotted with a 32-element f16 activation chunk (4 x 16 bytes,
+// lane-interleaved).  Products and the two partial sums are packed f16x2: the
+// even pairs go to one accumulator, the odd pairs to the other, so each f16
+// lane sums eight products, each with one rounding (the products themselves
+// are exact for bf16 activations: 2 + 8 significant bits).  The activations
+// are staged with max|x| in [2^8, 2^9), so a partial sum stays below
+// 8 * 6 * 2^9 = 24576 < 65504.  The four partial sums are added in fp32.
+__device__ __forceinline__ float dot32_h2(const uint32_t (&w)[16], const uint4 (&xv)[4]) {
+  uint32_t a0 = hmul2(w[0], xv[0].x), a1 = hmul2(w[1], xv[0].y);
+  a0 = hfma2(w[2], xv[0].z, a0);
+  a1 = hfma2(w[3], xv[0].w, a1);
 #pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    p0 = fma2_f16(w[4 * q + 0], xv[q].x, p0);
-    p1 = fma2_f16(w[4 * q + 1], xv[q].y, p1);
-    p2 = fma2_f16(w[4 * q + 2], xv[q].z, p2);
-    p3 = fma2_f16(w[4 * q + 3], xv[q].w, p3);
+  for (int q = 1; q < 4; ++q) {
+    a0 = hfma2(w[4 * q + 0], xv[q].x, a0);
+    a1 = hfma2(w[4 * q + 1], xv[q].y, a1);
+    a0 = hfma2(w[4 * q + 2], xv[q].z, a0);
+    a1 = hfma2(w[4 * q + 3], xv[q].w, a1);
   }
-  return (p0 + p1) + (p2 + p3);
+  return h2_sum_f32(a0) + h2_sum_f32(a1);
 }
 
 __device__ __forceinline__ void decode_chunk(const uint4 q, uint32_t (&w)[16]) {
@@ -225,8 +255,9 @@ __device__ __forceinline__ float pow2f(int e) {
 
 // Staging of activation vectors into shared memory.  MXFP4 streams: f16 of
 // x * 2^-e in the lane-interleaved layout, e chosen from max|x| so that the
-// largest element sits in [2^14, 2^15) (exact for bf16 inputs, one rounding
-// for fp32 ones).  bf16 streams: a plain copy of the bf16 or fp32 row.
+// largest element sits in [2^8, 2^9) (exact for bf16 inputs down to 2^-25 of
+// the largest element, one rounding for fp32 ones); the headroom above keeps
+// the f16 partial sums of dot32_h2 finite.  bf16 streams: a plain copy of the bf16 or fp32 row.
 // Work is split into (vector, segment) units over all consumer warps; all
 // loads are 16-byte vectors with several in flight.
 
@@ -293,7 +324,7 @@ __device__ __forceinline__ int shift_for_amax(float amax) {
   int e = 0;
   if (amax > 0.f && amax < INFINITY) {
     const int ef = (int)((__float_as_uint(amax) >> 23) & 0xFF);
-    e = (ef > 0 ? ef - 127 : -127) - 14;  // floor(log2(amax)) - 14
+    e = (ef > 0 ? ef - 127 : -127) - 8;  // floor(log2(amax)) - 8
     e = max(-126, min(127, e));
   }
   return e;
@@ -348,72 +379,61 @@ __host__ __device__ constexpr int x_row_bytes(int wf, int xk, int K) {
 }
 
 // ---------------------------------------------------------------------------
-// Scale bytes of one item for this warp's rows and this lane's chunks (the
-// shape-specialised path reads them from global memory, one item ahead).
-template <int NWR, int RPW, bool kSwiglu, int kCPL>
-__device__ __forceinline__ void load_item_scales(const GemvArgs& a, int grp, int rt, int wi, int lane, int C,
-                                                 int sblocks, float (&out)[NWR][kCPL]) {
-  const uint8_t* sgl = a.sc + (long long)grp * a.s_gstride;
-  const int r0 = rt * a.R;
-#pragma unroll
-  for (int r = 0; r < NWR; ++r) {
-    const int sr = kSwiglu ? (r < RPW ? wi * RPW + r : a.R + wi * RPW + (r - RPW)) : wi * RPW + r;
-    const int gr = kSwiglu && sr >= a.R ? r0 + a.up_off + sr - a.R : r0 + sr;
-#pragma unroll
-    for (int ci = 0; ci < kCPL; ++ci) {
-      const int b = lane + 32 * ci;
-      out[r][ci] = e8m0_to_f32((b < C) ? (uint32_t)__ldg(sgl + (size_t)gr * sblocks + b) : 127u);
-    }
-  }
-}
-
-// ---------------------------------------------------------------------------
 // Fused combine bookkeeping.  A warp group writes the unweighted expert
-// outputs y of its items to the scratch; every kPubBatch items it meets on a
-// group barrier (all of the group's y stores are then ordered before the
-// leader's fence), the leader issues one gpu-scope fence and one tile-counter
-// atomic per item (lanes in parallel).  The atomics' results are examined one
-// batch later (settle), so their latency hides behind the next batch: the
-// item that brings a row tile's count to the number of active experts makes
-// its warp combine that tile in ascending expert order.
+// outputs y of its items to the scratch; every kPubBatch items all warps of
+// the group meet in publish_round().  After a group barrier (the group's y
+// stores are then ordered before the leader's fence) the leader warp issues
+// one gpu-scope fence and one tile-counter atomic per item (lanes in
+// parallel).  The atomics' results are examined one round later, so their
+// latency hides behind the next batch: the row tiles whose count reached the
+// number of active experts are listed in shared memory, and after a second
+// group barrier every warp of the group combines them, one output element per
+// lane, in ascending expert order.
 constexpr int kPubBatch = 8;
+
+#ifndef MOE_L2_AHEAD
+#define MOE_L2_AHEAD 0
+#endif
+constexpr int kL2Ahead = MOE_L2_AHEAD;  // items the producer prefetches into L2 ahead of the ring
+constexpr int kPubInts = kPubBatch + 1;  // per group: [0] = tiles to combine, [1..] = their row tiles
 
 __device__ __forceinline__ void group_bar(int q0, int wpi) {
   named_bar_sync(3 + q0, wpi * 32);
 }
 
-__device__ void settle_batch(const GemvArgs& a, int prev_cnt, int prev_rt, int nprev, int n_groups, int wi,
-                             int lane) {
-  if (wi != 0) return;
-  const unsigned ready = __ballot_sync(0xFFFFFFFFu, lane < nprev && prev_cnt == n_groups - 1);
-  if (!ready) return;
-  __threadfence();
-  const int H = a.out_rows;
-  for (unsigned m = ready; m; m &= m - 1) {
-    const int src = __ffs(m) - 1;
-    const int rt = __shfl_sync(0xFFFFFFFFu, prev_rt, src);
-    for (int q = lane; q < a.batch * a.R; q += 32) {
-      const int b = q / a.R, r = rt * a.R + (q - (q / a.R) * a.R);
-      a.out_bf16[(size_t)b * H + r] = combine_one(a, a.out, H, b, r);
+__device__ void publish_round(const GemvArgs& a, const int* pend_rt, int npend, int& prev_cnt, int& prev_rt,
+                              int& nprev, int n_groups, int wi, int q0, int lane, int* s_pub) {
+  group_bar(q0, a.wpi);  // every warp of the group has written its y rows of the pending items
+  if (wi == 0) {
+    // results of the previous round first (their atomics completed long ago)
+    const bool rdy = lane < nprev && prev_cnt == n_groups - 1;
+    const unsigned m = __ballot_sync(0xFFFFFFFFu, rdy);
+    if (rdy) {
+      s_pub[1 + __popc(m & ((1u << lane) - 1u))] = prev_rt;
+      a.tile_counter[prev_rt] = 0;  // every contribution has arrived: ready for the next launch
     }
-    if (lane == 0) a.tile_counter[rt] = 0;
-  }
-}
-
-__device__ void publish_batch(const GemvArgs& a, const int* pend_rt, int npend, int& prev_cnt, int& prev_rt,
-                              int& nprev, int n_groups, int wi, int q0, int lane) {
-  group_bar(q0, a.wpi);  // every warp of the group has written its y rows of these items
-  if (wi != 0) return;
-  // results of the previous batch first (their atomics have long completed)
-  if (nprev > 0) settle_batch(a, prev_cnt, prev_rt, nprev, n_groups, wi, lane);
-  __threadfence();
-  int rt = 0;
+    if (lane == 0) s_pub[0] = __popc(m);
+    if (m) __threadfence();  // acquire: the other contributors' y stores before our loads
+    if (npend > 0) {
+      __threadfence();  // release: this group's y stores before its counts
+      int rt = 0;
 #pragma unroll
-  for (int i = 0; i < kPubBatch; ++i)
-    if (lane == i) rt = pend_rt[i];
-  prev_rt = rt;
-  prev_cnt = (lane < npend) ? atomicAdd(&a.tile_counter[rt], 1) : -1;
+      for (int i = 0; i < kPubBatch; ++i)
+        if (lane == i) rt = pend_rt[i];
+      prev_rt = rt;
+      prev_cnt = (lane < npend) ? atomicAdd(&a.tile_counter[rt], 1) : -1;
+    }
+  }
   nprev = npend;
+  group_bar(q0, a.wpi);
+  const int nready = s_pub[0];
+  if (nready == 0) return;
+  const int H = a.out_rows, per_tile = a.batch * a.R;
+  for (int o = wi * 32 + lane; o < nready * per_tile; o += a.wpi * 32) {
+    const int ti = o / per_tile, q = o - ti * per_tile;
+    const int b = q / a.R, r = s_pub[1 + ti] * a.R + (q - (q / a.R) * a.R);
+    a.out_bf16[(size_t)b * H + r] = combine_one(a, a.out, H, b, r);
+  }
 }
 
 // ---------------------------------------------------------------------------
@@ -432,18 +452,29 @@ struct TokenPass {
 // addressing and, for MXFP4, read the E8M0 scale bytes from global memory with
 // loads issued ahead of the stage wait (the stage then holds codes only).
 template <int WF, int EPI, int XK, int TMAX, int RPW, int KT>
-__global__ void __launch_bounds__(kMaxConsumerWarps * 32 + 32, 1) gemv_kernel(const GemvArgs a) {
+__global__ void __launch_bounds__(((KT != 0 && WF == W_MXFP4 && TMAX == 1 &&
+                                    (EPI == EPI_SWIGLU ? 2 * RPW : RPW) == kSplitKRows)
+                                       ? kMaxSplitKWarps
+                                       : kMaxConsumerWarps) * 32 + 32,
+                                  1) gemv_kernel(const GemvArgs a) {
   constexpr bool kSwiglu = (EPI == EPI_SWIGLU);
   constexpr int NWR = kSwiglu ? 2 * RPW : RPW;  // weight rows per warp
   static_assert(NWR % 2 == 0, "rows are processed in pairs");
-  constexpr bool kFast = (KT != 0) && (WF == W_MXFP4) && (TMAX == 1);
-  constexpr int kCPL = KT ? ((KT / 32) + 31) / 32 : 1;  // chunks per lane (fast path)
+  // kFast: the split-K instance.  Lanes own one 32-element chunk each, a
+  // warp covers 32 chunks (a K slice) of NWR rows, and an item's KS slices go
+  // to KS warps of the group (times R / RPW row quarters).
+  constexpr bool kOneTokMx = (KT != 0) && (WF == W_MXFP4) && (TMAX == 1);
+  constexpr bool kFast = kOneTokMx && NWR == kSplitKRows;
+  // kUnroll: one token, compile-time K, whole rows per warp (lane-strided
+  // chunks, fully unrolled, constant shared-memory offsets)
+  constexpr bool kUnroll = kOneTokMx && !kFast;
+  constexpr int KS = KT ? ((KT / 32) + 31) / 32 : 1;  // K slices of 32 chunks (= chunks per lane when unrolled)
   extern __shared__ __align__(128) unsigned char smem[];
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int ncw = a.ncw;
   const int K = KT ? KT : a.K;
-  const bool sglobal = (KT != 0 && WF == W_MXFP4) ? true : (a.scales_global != 0);
+  const bool sglobal = a.scales_global != 0;
   const int C = K >> 5;                                   // 32-element chunks per row
   const int rowbytes = (WF == W_MXFP4) ? (K >> 1) : (K << 1);
   const int sblocks = K >> 5;
@@ -459,6 +490,8 @@ __global__ void __launch_bounds__(kMaxConsumerWarps * 32 + 32, 1) gemv_kernel(co
   volatile int* s_flag = slot_e + kMaxSlots;
   int* s_item_cnt = slot_e + kMaxSlots + 2;  // [n_stages] warps done with the item in that stage
   float* s_amax = reinterpret_cast<float*>(s_item_cnt + kMaxStagesDev);  // [kMaxStageUnits] staging partial maxima
+  int* s_pub = reinterpret_cast<int*>(s_amax + kMaxStageUnits);          // [kMaxWarpsAny][kPubInts] combine lists
+  float* s_red = reinterpret_cast<float*>(s_pub + kMaxWarpsAny * kPubInts);  // [kRedFloats] split-K partials
   unsigned char* xbuf = smem + a.x_offset;
   unsigned char* stages = smem + a.stage_offset;
 
@@ -505,7 +538,7 @@ __global__ void __launch_bounds__(kMaxConsumerWarps * 32 + 32, 1) gemv_kernel(co
     __syncwarp();
     asm volatile("bar.arrive 2, %0;" ::"r"(nthreads_all) : "memory");
   } else {
-    if (!a.routed) pdl_wait();
+    if (!a.routed && !a.pdl_late) pdl_wait();
     named_bar_sync(2, nthreads_all);
   }
 
@@ -516,6 +549,33 @@ __global__ void __launch_bounds__(kMaxConsumerWarps * 32 + 32, 1) gemv_kernel(co
       uint32_t ph = 0;
       bool ok = true;
       int pg = -1, pgrp = 0;  // cached group -> expert lookup
+      // L2 prefetch kL2Ahead items ahead of the copies into the ring, so that
+      // the bytes in flight per SM are not bounded by the ring's size: a ring
+      // copy then finds its lines in L2 (or on their way there).
+      const long long n_mine = hi - lo;
+      const bool scale_pf = WF == W_MXFP4 && ((a.R * sblocks) & 15) == 0 && (a.s_gstride & 15) == 0 &&
+                            ((a.up_off * sblocks) & 15) == 0;
+      // the prefetch cursor walks the CTA's items in order; the expert of its
+      // group is looked up once per group
+      int g2 = (int)(lo / n_rt), rt2 = (int)(lo - (long long)g2 * n_rt), cg2 = -1, grp2 = 0;
+      auto l2_ahead = [&]() {
+        if (g2 != cg2) {
+          cg2 = g2;
+          grp2 = a.routed ? clamp_group(a.active[g2], a.n_experts, nullptr) : 0;
+        }
+        const int r02 = rt2 * a.R;
+        if (++rt2 == n_rt) { rt2 = 0; ++g2; }
+        const uint8_t* wg2 = a.w + (long long)grp2 * a.w_gstride;
+        const uint32_t cb2 = (uint32_t)(a.R * rowbytes);
+        prefetch_l2(wg2 + (size_t)r02 * rowbytes, cb2);
+        if (kSwiglu) prefetch_l2(wg2 + (size_t)(r02 + a.up_off) * rowbytes, cb2);
+        if (scale_pf) {
+          const uint8_t* sg2 = a.sc + (long long)grp2 * a.s_gstride;
+          prefetch_l2(sg2 + (size_t)r02 * sblocks, (uint32_t)(a.R * sblocks));
+          if (kSwiglu) prefetch_l2(sg2 + (size_t)(r02 + a.up_off) * sblocks, (uint32_t)(a.R * sblocks));
+        }
+      };
+      for (long long jl = 0; jl < kL2Ahead && jl < n_mine; ++jl) l2_ahead();
       for (int p = 0; p < pt->n && ok; ++p) {
         const int jbeg = pt->ph[p].first_item, jend = pt->ph[p].last_item;
         int g = (int)((lo + jbeg) / n_rt);
@@ -546,6 +606,7 @@ __global__ void __launch_bounds__(kMaxConsumerWarps * 32 + 32, 1) gemv_kernel(co
             if (kSwiglu)
               bulk_g2s(st + codes_bytes + sb, sg + (size_t)(r0 + a.up_off) * sblocks, sb, &full_bar[s], pol);
           }
+          if (kL2Ahead > 0 && j + kL2Ahead < n_mine) l2_ahead();
           if (++s == a.n_stages) { s = 0; ph ^= 1u; }
         }
       }
@@ -560,7 +621,7 @@ __global__ void __launch_bounds__(kMaxConsumerWarps * 32 + 32, 1) gemv_kernel(co
   } else {
     // ------------------------------ consumers ------------------------------
     const int nct = ncw * 32;
-    long long jglob = 0;  // CTA-local item counter across phases (stage ring position)
+    int jglob = 0;  // CTA-local item counter across phases (stage ring position)
     for (int p = 0; p < pt->n; ++p) {
       const PhaseDesc ph = pt->ph[p];
       // stage this phase's activation vectors, each split over several warps
@@ -570,8 +631,6 @@ __global__ void __launch_bounds__(kMaxConsumerWarps * 32 + 32, 1) gemv_kernel(co
       named_bar_sync(1, nct);
       const int nit = ph.last_item - ph.first_item;
       int c_g = -1, c_grp = 0, c_tok0 = 0, c_ntok = 1, c_tp_tb = -1;
-      float snext[kFast ? NWR : 1][kFast ? kCPL : 1];  // next item's scales, fp32 (fast path)
-      (void)snext;
       int pend_rt[kPubBatch], npend = 0;  // fused combine: items written, not yet published
       int prev_cnt = 0, prev_rt = 0, nprev = 0;  // last published batch: atomic result per lane
       (void)pend_rt; (void)npend; (void)prev_cnt; (void)prev_rt; (void)nprev;
@@ -582,15 +641,17 @@ __global__ void __launch_bounds__(kMaxConsumerWarps * 32 + 32, 1) gemv_kernel(co
       const int wi = warp - q0 * a.wpi;    // this warp's share of the item
       int g = (int)((lo + ph.first_item + q0) / n_rt);
       int rt = (int)((lo + ph.first_item + q0) - (long long)g * n_rt);
+      // ring position of this group's first item; each step moves ng stages on
+      int s = (jglob + q0) % a.n_stages;
+      uint32_t par = (uint32_t)(((jglob + q0) / a.n_stages) & 1);
       for (int jj = q0; jj < nit; jj += ng) {
-        if (jj != q0) {  // advance (g, rt) by ng items
+        if (jj != q0) {  // advance (g, rt) and the ring position by ng items
           rt += ng;
           while (rt >= n_rt) { rt -= n_rt; ++g; }
+          s += ng;
+          if (s >= a.n_stages) { s -= a.n_stages; par ^= 1u; }
         }
         const bool skip = s_flag[0] != 0;  // aborting: no work, but every barrier is still met
-        const long long jl = jglob + jj;
-        const int s = (int)(jl % a.n_stages);
-        const uint32_t par = (uint32_t)((jl / a.n_stages) & 1);
         // group and token list: looked up once per group change, kept in registers
         if (g != c_g) {
           c_g = g;
@@ -612,25 +673,6 @@ __global__ void __launch_bounds__(kMaxConsumerWarps * 32 + 32, 1) gemv_kernel(co
         const int tlo = a.routed ? max(0, ph.t0) : ph.t0;
         const int thi = a.routed ? min(ntok, ph.t1) : ph.t1;
 
-        // fast path: scale bytes come from global memory one item ahead -- this
-        // item's were loaded during the previous item, the next item's go out now
-        float sreg[kFast ? NWR : 1][kFast ? kCPL : 1];
-        if constexpr (kFast) {
-          if (jj == q0) load_item_scales<NWR, RPW, kSwiglu, kCPL>(a, grp, rt, wi, lane, C, sblocks, sreg);
-          else {
-#pragma unroll
-            for (int r = 0; r < NWR; ++r)
-#pragma unroll
-              for (int ci = 0; ci < kCPL; ++ci) sreg[r][ci] = snext[r][ci];
-          }
-          const int jn = jj + ng;
-          if (jn < nit) {
-            int gn = g, rtn = rt + ng;
-            while (rtn >= n_rt) { rtn -= n_rt; ++gn; }
-            const int grpn = a.routed ? clamp_group(a.active[gn], a.n_experts, nullptr) : 0;
-            load_item_scales<NWR, RPW, kSwiglu, kCPL>(a, grpn, rtn, wi, lane, C, sblocks, snext);
-          }
-        }
         bool have = !skip;
         if (have && !mbar_wait_bounded(&full_bar[s], par)) {
           if (lane == 0) atomicExch(a.err, kErrTimeout);
@@ -638,6 +680,90 @@ __global__ void __launch_bounds__(kMaxConsumerWarps * 32 + 32, 1) gemv_kernel(co
           have = false;
         }
         const unsigned char* st = stages + (size_t)s * a.stage_bytes;
+        if constexpr (kFast) {
+          // ---- split-K item (one token): this warp's K slice of its NWR rows ----
+          // The group barrier below is met on every item, with or without work,
+          // so that an aborting warp can never leave the others waiting.
+          const bool work = have && tlo < thi;
+          if (work && tlo != c_tp_tb) {
+            c_tp_tb = tlo;
+            int src = tlo, orow = tlo;
+            if (a.routed) {
+              int pr = a.pair_ids[tok0 + tlo];
+              if (pr < 0 || pr >= a.n_pairs) pr = 0;
+              src = a.act_by_pair ? pr : pr / a.top_k;
+              orow = pr;
+            }
+            int sl = 0;
+            for (int u = 0; u < ph.nslots; ++u)
+              if (pt->slot_src[p][u] == src) sl = u;
+            tp.n = 1;
+            tp.slot[0] = sl;
+            tp.orow[0] = orow;
+            tp.e[0] = slot_e[sl];
+          }
+          const int ks = wi % KS, rq = wi / KS;  // K slice, row quarter
+          const int b = ks * 32 + lane;          // this lane's chunk
+          const bool bok = work && b < C;
+          int srow[NWR];
+#pragma unroll
+          for (int r = 0; r < NWR; ++r)
+            srow[r] = kSwiglu ? (r < RPW ? rq * RPW + r : a.R + rq * RPW + (r - RPW)) : rq * RPW + r;
+          // everything this warp needs from the stage, then hand it back at once
+          uint4 xv[4], cv[NWR];
+          uint32_t sv[NWR];
+          const uint32_t xs_s =
+              smem_addr(xbuf) + (uint32_t)(tp.slot[0] * xrow_bytes) + (uint32_t)(ks * 2048 + 16 * lane);
+          const uint32_t st_s = smem_addr(st) + 16u * (uint32_t)b;
+          const unsigned char* scl = st + codes_bytes;
+#pragma unroll
+          for (int q = 0; q < 4; ++q) xv[q] = bok ? lds128_s(xs_s + 512u * q) : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+          for (int r = 0; r < NWR; ++r) {
+            cv[r] = bok ? lds128_s(st_s + (uint32_t)(srow[r] * rowbytes)) : make_uint4(0u, 0u, 0u, 0u);
+            sv[r] = bok ? lds_u8(scl + srow[r] * sblocks + b) : 127u;
+          }
+          if (have) {
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty_bar[s]);
+          }
+          float v[NWR];
+#pragma unroll
+          for (int r = 0; r < NWR; ++r) {
+            uint32_t w[16];
+            decode_chunk(cv[r], w);
+            v[r] = dot32_h2(w, xv) * e8m0_to_f32(sv[r]);
+          }
+          // across the warp (lane L ends with row L / (32 / NWR)), then across the
+          // KS slices in ascending order, by the item's finishing warp
+          const float tot = warp_reduce_multi<NWR>(v, lane);
+          const int nit_g = jj / ng;  // this group's item counter
+          float* red = s_red + (size_t)(q0 * a.wpi) * 2 * NWR + (size_t)(nit_g & 1) * a.wpi * NWR;
+          if ((lane & (32 / NWR - 1)) == 0) red[wi * NWR + lane / (32 / NWR)] = tot;
+          group_bar(q0, a.wpi);
+          if (work && wi == nit_g % a.wpi) {
+            const int nrq = a.wpi / KS;
+            const int o = lane;  // output row of the item handled by this lane
+            if (o < nrq * RPW) {
+              const int orq = o / RPW, orr = o - orq * RPW;
+              float gsum = 0.f, usum = 0.f;
+#pragma unroll
+              for (int k2 = 0; k2 < KS; ++k2) {
+                gsum += red[(orq * KS + k2) * NWR + orr];
+                if constexpr (kSwiglu) usum += red[(orq * KS + k2) * NWR + RPW + orr];
+              }
+              const int row = rt * a.R + o;
+              float val;
+              if constexpr (kSwiglu) {
+                const float gg = gsum * pow2f(tp.e[0]), uu = usum * pow2f(tp.e[0]);
+                val = gg / (1.0f + expf(-gg)) * uu;
+              } else {
+                val = gsum * pow2f(tp.e[0]);
+              }
+              a.out[(size_t)tp.orow[0] * a.out_rows + row] = val;
+            }
+          }
+        } else
         for (int tb = tlo; have && tb < thi; tb += TMAX) {
           if (tb != c_tp_tb) {
           c_tp_tb = tb;
@@ -674,15 +800,33 @@ __global__ void __launch_bounds__(kMaxConsumerWarps * 32 + 32, 1) gemv_kernel(co
 #pragma unroll
           for (int r = 0; r < NWR; ++r)
             srow[r] = kSwiglu ? (r < RPW ? wi * RPW + r : a.R + wi * RPW + (r - RPW)) : wi * RPW + r;
-          if constexpr (kFast) {
-            // one activation vector, compile-time K: every chunk of this lane, unrolled,
-            // 32-bit shared addresses with constant offsets
+          if constexpr (kUnroll) {
+            const unsigned char* scl = st + codes_bytes;
+            float sreg[NWR][KS];
+#pragma unroll
+            for (int r = 0; r < NWR; ++r)
+#pragma unroll
+              for (int ci = 0; ci < KS; ++ci)
+                sreg[r][ci] = sglobal ? 1.f
+                                      : e8m0_to_f32(lane + 32 * ci < C ? lds_u8(scl + srow[r] * sblocks + lane + 32 * ci)
+                                                                       : 127u);
+            const uint8_t* sgl = a.sc + (long long)grp * a.s_gstride;
+            if (sglobal) {
+              const int r0 = rt * a.R;
+#pragma unroll
+              for (int r = 0; r < NWR; ++r) {
+                const int gr = kSwiglu && srow[r] >= a.R ? r0 + a.up_off + srow[r] - a.R : r0 + srow[r];
+#pragma unroll
+                for (int ci = 0; ci < KS; ++ci)
+                  if (lane + 32 * ci < C) sreg[r][ci] = e8m0_to_f32(__ldg(sgl + (size_t)gr * sblocks + lane + 32 * ci));
+              }
+            }
             const uint32_t xs_s = smem_addr(xbuf) + (uint32_t)(tp.slot[0] * xrow_bytes) + 16u * lane;
             uint32_t rb_s[NWR];
 #pragma unroll
             for (int r = 0; r < NWR; ++r) rb_s[r] = smem_addr(st) + (uint32_t)(srow[r] * rowbytes) + 16u * lane;
 #pragma unroll
-            for (int ci = 0; ci < kCPL; ++ci) {
+            for (int ci = 0; ci < KS; ++ci) {
               if (lane + 32 * ci < C) {
                 uint4 xv[4];
 #pragma unroll
@@ -691,7 +835,7 @@ __global__ void __launch_bounds__(kMaxConsumerWarps * 32 + 32, 1) gemv_kernel(co
                 for (int r = 0; r < NWR; ++r) {
                   uint32_t w[16];
                   decode_chunk(lds128_s(rb_s[r] + 512u * ci), w);
-                  acc[r][0] = fmaf(dot32_f16(w, xv), sreg[r][ci], acc[r][0]);
+                  acc[r][0] = fmaf(dot32_h2(w, xv), sreg[r][ci], acc[r][0]);
                 }
               }
             }
@@ -724,7 +868,7 @@ __global__ void __launch_bounds__(kMaxConsumerWarps * 32 + 32, 1) gemv_kernel(co
                 for (int r = 0; r < NWR; ++r) {
                   uint32_t w[16];
                   decode_chunk(cv[r], w);
-                  acc[r][0] = fmaf(dot32_f16(w, xv), e8m0_to_f32(sv[r]), acc[r][0]);
+                  acc[r][0] = fmaf(dot32_h2(w, xv), e8m0_to_f32(sv[r]), acc[r][0]);
                 }
               }
             } else
@@ -744,7 +888,7 @@ __global__ void __launch_bounds__(kMaxConsumerWarps * 32 + 32, 1) gemv_kernel(co
                     decode_chunk(lds128(st + (size_t)srow[r] * rowbytes + 16 * b), w);
                     const float sc = sglobal ? e8m0_to_f32(__ldg(sgl + (size_t)gsrow[r] * sblocks + b))
                                                      : e8m0_to_f32(lds_u8(scl + srow[r] * sblocks + b));
-                    acc[r][t] = fmaf(dot32_f16(w, xv), sc, acc[r][t]);
+                    acc[r][t] = fmaf(dot32_h2(w, xv), sc, acc[r][t]);
                   }
                 }
               }
@@ -838,19 +982,20 @@ __global__ void __launch_bounds__(kMaxConsumerWarps * 32 + 32, 1) gemv_kernel(co
           }
         }
         if constexpr (EPI == EPI_DOWN_COMBINE) {
-          // publish in batches: see publish_batch()
+          // publish in batches: see publish_round()
           pend_rt[npend++] = rt;
           if (npend == kPubBatch) {
-            publish_batch(a, pend_rt, npend, prev_cnt, prev_rt, nprev, n_groups, wi, q0, lane);
+            publish_round(a, pend_rt, npend, prev_cnt, prev_rt, nprev, n_groups, wi, q0, lane, s_pub + q0 * kPubInts);
             npend = 0;
           }
         }
       }
       if constexpr (EPI == EPI_DOWN_COMBINE) {
         // end of phase: publish what is left, then settle the last results
-        if (npend > 0) publish_batch(a, pend_rt, npend, prev_cnt, prev_rt, nprev, n_groups, wi, q0, lane);
+        // (npend and nprev are the same in every warp of the group)
+        if (npend > 0) publish_round(a, pend_rt, npend, prev_cnt, prev_rt, nprev, n_groups, wi, q0, lane, s_pub + q0 * kPubInts);
         npend = 0;
-        if (nprev > 0) settle_batch(a, prev_cnt, prev_rt, nprev, n_groups, wi, lane);
+        if (nprev > 0) publish_round(a, pend_rt, 0, prev_cnt, prev_rt, nprev, n_groups, wi, q0, lane, s_pub + q0 * kPubInts);
         nprev = 0;
       }
       jglob += nit;
@@ -859,6 +1004,9 @@ __global__ void __launch_bounds__(kMaxConsumerWarps * 32 + 32, 1) gemv_kernel(co
 
   // Let the next kernel in the stream start its prologue.
   pdl_launch_dependents();
+  // A stream that skipped the wait still completes only after its predecessor,
+  // so the kernels behind it inherit that dependency.
+  if (a.pdl_late) pdl_wait();
 
   if constexpr (EPI == EPI_DOWN_COMBINE) {
     // tail: warm L2 with the next layer's static weights (one slice per CTA)

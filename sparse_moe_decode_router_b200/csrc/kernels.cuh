@@ -83,6 +83,8 @@ struct GemvArgs {
   // L2 prefetch of the next layer's weights (issued by CTAs when their items are done)
   const uint8_t* pf_ptr[2];
   long long pf_bytes[2];
+  int pdl_late;     // dense stream whose activations are final at launch: no wait before
+                   // reading them; every thread waits for the preceding grid at exit instead
   int* err;
 };
 
@@ -118,16 +120,16 @@ struct NextPow2 {
 
 // Fixed-order combine of one output element: residual + y_shared + sum_j w_j y_j
 // (fp32, fused multiply-adds in ascending j = ascending expert id), bf16 once.
-// Loads are issued eight pairs at a time, ahead of their ordered sums.
+// The loads of up to sixteen pairs go out together, ahead of their ordered sums.
 __device__ __forceinline__ uint16_t combine_one(const GemvArgs& a, const float* __restrict__ y, int H, int b,
                                                 int r) {
   const int k = a.top_k;
   float acc = __uint_as_float((uint32_t)a.residual[(size_t)b * H + r] << 16);
   if (a.y_shared) acc += __ldcg(a.y_shared + (size_t)b * H + r);
-  for (int j0 = 0; j0 < k; j0 += 8) {
-    float wv[8], yv[8];
+  for (int j0 = 0; j0 < k; j0 += 16) {
+    float wv[16], yv[16];
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
+    for (int j = 0; j < 16; ++j) {
       wv[j] = 0.f;
       yv[j] = 0.f;
       if (j0 + j < k) {
@@ -136,7 +138,7 @@ __device__ __forceinline__ uint16_t combine_one(const GemvArgs& a, const float* 
       }
     }
 #pragma unroll
-    for (int j = 0; j < 8; ++j)
+    for (int j = 0; j < 16; ++j)
       if (j0 + j < k) acc = fmaf(wv[j], yv[j], acc);
   }
   return f32_to_bf16_rne(acc);
@@ -196,6 +198,9 @@ __global__ void __launch_bounds__(kTopkWarps * 32) topk_bucket_kernel(const Gemv
   __shared__ int s_off[kMaxExperts];
   __shared__ int s_wsum[kTopkWarps][2];
   pdl_wait();
+  // Dependents may launch now: a dense kernel that reads only the layer input
+  // overlaps this latency-bound work; routed kernels wait for our completion.
+  pdl_launch_dependents();
   const float* lg = a.out + (size_t)b * E;
   // stage 1: warp w takes experts [w*SL, (w+1)*SL), SL = ceil(E/8) <= 128 (4 per lane)
   const int SL = (E + kTopkWarps - 1) / kTopkWarps;
@@ -304,11 +309,8 @@ __global__ void __launch_bounds__(kTopkWarps * 32) topk_bucket_kernel(const Gemv
     __threadfence();
     if (tid == 0) s_last = (atomicAdd(a.done_counter, 1) == (int)gridDim.x - 1);
     __syncthreads();
-    pdl_launch_dependents();
     if (!s_last) return;
     __threadfence();
-  } else {
-    pdl_launch_dependents();
   }
   auto idx_of = [&](int p) { return gridDim.x > 1 ? __ldcg(a.topk_idx + p) : c_id[p]; };
   for (int e = tid; e < E; e += NT) s_mask[e] = 0ull;

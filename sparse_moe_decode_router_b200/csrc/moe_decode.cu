@@ -61,20 +61,42 @@ struct GemvPlan {
 // vectors the stream can address (B, or B*k for the down projection),
 // `max_groups` = most groups (experts) the stream can have active,
 // `tok_per_group` = most activation vectors one group uses.
+// Row quarters of the split-K (one-token MXFP4) instances: an item is
+// kSplitKRows / (2 for SwiGLU) rows per warp times this many warp rows, each
+// spread over the K slices.  Gate/up: 4 gate + 4 up rows (2 x 14 KB codes);
+// down: 32 rows (32 KB).
+#ifndef MOE_SPLITK_GU
+#define MOE_SPLITK_GU 0  // gate/up: 0 = whole rows per warp (faster there), 1 = split-K
+#endif
+#ifndef MOE_SPLITK_GU_RQ
+#define MOE_SPLITK_GU_RQ 1
+#endif
+#ifndef MOE_SPLITK_DN_RQ
+#define MOE_SPLITK_DN_RQ 4
+#endif
+
 GemvPlan make_plan(Kind kind, int K, int out_rows, int slots_needed, int max_groups, int tok_per_group,
                    long long s_gstride, int num_sms, bool fast = false) {
   GemvPlan p;
-  const KindTraits t = kTraits[kind];
-  const int R = t.rpw * t.wpi;
-  if (K <= 0 || K % 32 || out_rows <= 0 || out_rows % R) return p;
+  KindTraits t = kTraits[kind];
   const bool mx = t.wf == W_MXFP4;
   const bool swiglu = t.epi == EPI_SWIGLU;
+  const bool splitk = fast && mx && (!swiglu || MOE_SPLITK_GU);  // warps = row quarters x K slices
+  if (splitk) {
+    const int ks = (K / 32 + 31) / 32;
+    const int rq = swiglu ? MOE_SPLITK_GU_RQ : MOE_SPLITK_DN_RQ;
+    t.rpw = swiglu ? kSplitKRows / 2 : kSplitKRows;
+    t.wpi = rq * ks;
+  }
+  const int R = t.rpw * t.wpi / (splitk ? (K / 32 + 31) / 32 : 1);
+  if (K <= 0 || K % 32 || out_rows <= 0 || out_rows % R) return p;
   const int rowbytes = mx ? K / 2 : K * 2;
   const int sbytes = mx ? K / 32 : 0;
   const int rows = swiglu ? 2 * R : R;
-  // scale rows go through TMA only when every copy is 16-byte aligned and sized;
-  // the shape-specialised (fast) instances always read them from global memory
-  const bool sg = mx && (fast || ((long long)R * sbytes) % 16 != 0 || s_gstride % 16 != 0);
+  // scale rows go through TMA only when every copy is 16-byte aligned and sized
+  // (the split-K instances read them from the stage: no other way)
+  const bool sg = mx && (((long long)R * sbytes) % 16 != 0 || s_gstride % 16 != 0);
+  if (splitk && sg) return p;
   const int stage = (int)align_up((size_t)rows * (rowbytes + (mx && !sg ? sbytes : 0)), 128);
   // activation slots: a CTA's contiguous item range spans at most
   // ceil(items per CTA / items per group) + 1 groups
@@ -84,7 +106,7 @@ GemvPlan make_plan(Kind kind, int K, int out_rows, int slots_needed, int max_gro
   const int xrow = x_row_bytes(t.wf, t.xk, K);
   int xcap = std::min(slots_needed, groups_per_cta * tok_per_group);
   xcap = std::min(std::min(xcap, kMaxSlots), std::max(1, kXBudget / xrow));
-  const int hdr = (int)align_up(16 * 64 + sizeof(PhaseTable) + (kMaxSlots + 2 + kMaxStagesDev + kMaxStageUnits) * 4, 128);
+  const int hdr = (int)align_up(16 * 64 + sizeof(PhaseTable) + (kMaxSlots + 2 + kMaxStagesDev + kMaxStageUnits + kMaxWarpsAny * kPubInts + kRedFloats) * 4, 128);
   const int x_off = hdr;
   const int st_off = (int)align_up((size_t)x_off + (size_t)xcap * xrow, 128);
   int ns = std::min(kMaxStages, (kSmemBudget - st_off) / stage);
@@ -95,7 +117,9 @@ GemvPlan make_plan(Kind kind, int K, int out_rows, int slots_needed, int max_gro
   // group count: every stage is then always consumed by the same group, in
   // item order, and a group never waits on a stage whose previous phase
   // another group has not finished.
-  int groups = std::max(1, std::min(kMaxConsumerWarps / t.wpi, std::max(1, ns - pf)));
+  const int max_warps = splitk ? kMaxSplitKWarps : kMaxConsumerWarps;
+  if (t.wpi > max_warps) return p;
+  int groups = std::max(1, std::min(max_warps / t.wpi, std::max(1, ns - pf)));
   while (groups > 1 && (ns / groups) * groups - groups < pf) --groups;
   ns = (ns / groups) * groups;
   p.ok = true;
@@ -128,17 +152,18 @@ GemvFn pick_fn(Kind k) {
     case K_ROUTER: return gemv_kernel<W_BF16, EPI_ROUTER, X_BF16, TMAX, 2, KH>;
     case K_SGU: return gemv_kernel<W_BF16, EPI_SWIGLU, X_BF16, TMAX, 1, KH>;
     case K_SDN: return gemv_kernel<W_BF16, EPI_STORE, X_F32, TMAX, 2, KI>;
-    case K_GU: return gemv_kernel<W_MXFP4, EPI_SWIGLU, X_BF16, TMAX, MOE_GU_RPW, KH>;
-    case K_DN: return gemv_kernel<W_MXFP4, EPI_STORE, X_F32, TMAX, MOE_DN_RPW, KI>;
-    case K_DNC: return gemv_kernel<W_MXFP4, EPI_DOWN_COMBINE, X_F32, TMAX, MOE_DN_RPW, KI>;
+    // instances with a compile-time K and one token are the split-K ones
+    case K_GU:
+      return gemv_kernel<W_MXFP4, EPI_SWIGLU, X_BF16, TMAX, (KH && TMAX == 1 && MOE_SPLITK_GU) ? kSplitKRows / 2 : MOE_GU_RPW, KH>;
+    case K_DN: return gemv_kernel<W_MXFP4, EPI_STORE, X_F32, TMAX, (KI && TMAX == 1) ? kSplitKRows : MOE_DN_RPW, KI>;
+    case K_DNC:
+      return gemv_kernel<W_MXFP4, EPI_DOWN_COMBINE, X_F32, TMAX, (KI && TMAX == 1) ? kSplitKRows : MOE_DN_RPW, KI>;
     default: return nullptr;
   }
 }
 
-// the K each stream reduces over in the full-size layer
-int fast_k(Kind k) { return (k == K_SDN || k == K_DN || k == K_DNC) ? kFastI : kFastH; }
-
-// fast = the shape-specialised one-token instance (K must equal fast_k(k))
+// fast = the shape-specialised one-token instance (K must be kFastI for the
+// down projections, kFastH for the others)
 GemvFn gemv_fn(Kind k, int tmax, bool fast = false) {
   if (tmax == 1) return fast ? pick_fn<1, kFastH, kFastI>(k) : pick_fn<1, 0, 0>(k);
   return pick_fn<2, 0, 0>(k);
@@ -173,7 +198,7 @@ struct moe_layer {
   int device = 0;
   int num_sms = 0;
   bool pdl = true;
-  bool side_stream = true;
+  bool side_stream = false;
   bool prefetch = true;
   char* arena = nullptr;
   uint16_t* wr_t = nullptr;  // router matrix, expert-major [E][H]
@@ -278,7 +303,10 @@ cudaError_t launch_router(moe_layer* L, const void* x, int B, const moe_routing&
   return launch_ex(topk_bucket_kernel, B, kTopkWarps * 32, 0, st, L->pdl, t);
 }
 
-cudaError_t launch_shared(moe_layer* L, const void* x, int B, float* ys, cudaStream_t st, bool pdl) {
+// Shared expert: gate/up + SwiGLU, then down.  late: the gate/up kernel may
+// read x before its predecessor completes (see GemvArgs::pdl_late).
+cudaError_t launch_shared(moe_layer* L, const void* x, int B, float* ys, cudaStream_t st, bool pdl,
+                          bool late = false) {
   const int H = L->cfg.hidden, Is = L->cfg.shared_inter;
   {
     const GemvPlan& p = plan_of(L, K_SGU, B);
@@ -288,6 +316,7 @@ cudaError_t launch_shared(moe_layer* L, const void* x, int B, float* ys, cudaStr
     a.act = x;
     a.n_tokens = B;
     a.out = L->hs;
+    a.pdl_late = late && pdl ? 1 : 0;
     cudaError_t e = run_gemv(L, K_SGU, B, a, st, pdl);
     if (e != cudaSuccess) return e;
   }
@@ -429,7 +458,7 @@ moe_status_t moe_layer_create(const moe_layer_config* cfg, const moe_layer_weigh
   L->device = dev;
   L->num_sms = sms;
   L->pdl = !(c.flags & MOE_FLAG_NO_PDL);
-  L->side_stream = !(c.flags & MOE_FLAG_NO_SIDE_STREAM);
+  L->side_stream = (c.flags & MOE_FLAG_SIDE_STREAM) != 0;
   L->prefetch = !(c.flags & MOE_FLAG_NO_PREFETCH);
 
   const int H = c.hidden, E = c.n_experts, k = c.top_k, I = c.inter, Is = c.shared_inter, MB = c.max_batch;
@@ -611,10 +640,11 @@ moe_status_t moe_layer_forward(moe_layer_t L, moe_layer_t next, const void* x, c
     if (e == cudaSuccess) e = cudaEventRecord(L->ev_join, L->side);
   }
   if (e == cudaSuccess) e = launch_router(L, x, B, L->plan, st);
+  // the shared expert's gate/up reads only x: it starts while the top-k runs
+  if (e == cudaSuccess && has_shared && !fork) e = launch_shared(L, x, B, L->ys, st, L->pdl, true);
   if (e == cudaSuccess && L->probe_start) e = cudaEventRecord(L->probe_start, st);
   if (e == cudaSuccess) e = launch_gate_up(L, x, B, L->plan, st);
   if (e == cudaSuccess && L->probe_stop) e = cudaEventRecord(L->probe_stop, st);
-  if (e == cudaSuccess && has_shared && !fork) e = launch_shared(L, x, B, L->ys, st, L->pdl);
   if (e == cudaSuccess && fork) e = cudaStreamWaitEvent(st, L->ev_join, 0);
   if (e == cudaSuccess)
     e = launch_down(L, B, L->plan, L->y, true, residual, out, has_shared ? L->ys : nullptr, next, st,

@@ -117,6 +117,14 @@ __device__ __forceinline__ uint4 lds128_s(uint32_t addr) {
   return v;
 }
 
+// Read-only byte load that stays where it is written (volatile): a prefetch
+// into a register whose value is used much later.
+__device__ __forceinline__ uint32_t ldg_u8_early(const void* p) {
+  uint32_t v;
+  asm volatile("ld.global.nc.u8 %0, [%1];" : "=r"(v) : "l"(p));
+  return v;
+}
+
 __device__ __forceinline__ uint32_t lds_u8(const void* p) {
   uint32_t v;
   asm volatile("ld.shared.u8 %0, [%1];" : "=r"(v) : "r"(smem_addr(p)));

@@ -13,14 +13,17 @@ OUT_MEAN_REL = 2e-3
 # bounds leave an order of magnitude of margin.
 Y_MAX_REL = 1e-4
 Y_MEAN_REL = 1e-5
-# Routed expert outputs: the down projection reads the SwiGLU activations h
-# rounded once to f16 (scaled by a power of two, 11 significant bits, relative
-# error <= 2^-11 per element).  A dot product of such elements has a relative
-# error of at most 2^-11 ~ 4.9e-4 when every rounding error has the same sign,
-# typically ~2^-12 / sqrt(3); the mean bound is the worst case, the max bound
-# allows a few cancelling outputs.
-Y_ROUTED_MAX_REL = 2e-3
-Y_ROUTED_MEAN_REL = 4.9e-4
+# Routed expert outputs.  MXFP4 dot products take their products and their
+# partial sums over eight products in f16 (unit roundoff u = 2^-11 ~ 4.9e-4 per
+# operation), the down projection reads the SwiGLU activations h rounded once
+# to f16, and block sums are scaled and accumulated in fp32.  For the
+# random-sign data here the errors do not line up: an exact emulation of these
+# roundings on the full-size layer (one token, its 16 experts) gives a mean
+# relative error of ~7.4e-4 and a max error of ~8.8e-4 * max|y|.  The bounds
+# leave a factor of ~2.7 (mean) and ~4.5 (max) of margin; the layer output
+# keeps its own, stated tolerance above.
+Y_ROUTED_MAX_REL = 4e-3
+Y_ROUTED_MEAN_REL = 2e-3
 # routing weights: fp32 softmax of fp32 logits vs fp64 (|w| <= 1)
 W_ABS = 1e-5
 
