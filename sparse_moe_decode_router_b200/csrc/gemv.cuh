@@ -522,8 +522,11 @@ __global__ void __launch_bounds__(((KT != 0 && WF == W_MXFP4 && TMAX == 1 &&
   const long long hi = n_items * (blockIdx.x + 1) / gridDim.x;
 
   __syncthreads();  // barriers initialised
-  // plan invariant (see the host planner): stages are a multiple of the warp groups
-  if ((a.ncw % a.wpi) != 0 || (a.n_stages % (a.ncw / a.wpi)) != 0) {
+  // plan invariants (see the host planner): stages are a multiple of the warp
+  // groups, and an item's rows are exactly what the group's warps cover
+  const int kq_plan = kFast ? KS : ((WF == W_BF16 && a.ksplit > 1) ? a.ksplit : 1);
+  if ((a.ncw % a.wpi) != 0 || (a.n_stages % (a.ncw / a.wpi)) != 0 || (a.wpi % kq_plan) != 0 ||
+      a.R != RPW * (a.wpi / kq_plan)) {
     if (tid == 0) atomicExch(a.err, kErrBadPlan);
     return;
   }
@@ -631,6 +634,7 @@ __global__ void __launch_bounds__(((KT != 0 && WF == W_MXFP4 && TMAX == 1 &&
       named_bar_sync(1, nct);
       const int nit = ph.last_item - ph.first_item;
       int c_g = -1, c_grp = 0, c_tok0 = 0, c_ntok = 1, c_tp_tb = -1;
+      int nred = 0;  // K-split reduction rounds of this warp (buffer parity)
       int pend_rt[kPubBatch], npend = 0;  // fused combine: items written, not yet published
       int prev_cnt = 0, prev_rt = 0, nprev = 0;  // last published batch: atomic result per lane
       (void)pend_rt; (void)npend; (void)prev_cnt; (void)prev_rt; (void)nprev;
@@ -763,8 +767,14 @@ __global__ void __launch_bounds__(((KT != 0 && WF == W_MXFP4 && TMAX == 1 &&
               a.out[(size_t)tp.orow[0] * a.out_rows + row] = val;
             }
           }
-        } else
-        for (int tb = tlo; have && tb < thi; tb += TMAX) {
+        } else {
+        // bf16 streams may split K over the group's warps: warp wi takes K slice
+        // wi % kq of the rows of warp-row wi / kq; partial sums meet in s_red
+        const int kq = (WF == W_BF16 && a.ksplit > 1) ? a.ksplit : 1;
+        const int ksl = wi % kq, wr = wi / kq;
+        // with K split, every warp of the group runs the same token passes (the
+        // group barrier inside is met even by a warp that is aborting)
+        for (int tb = tlo; (have || kq > 1) && tb < thi; tb += TMAX) {
           if (tb != c_tp_tb) {
           c_tp_tb = tb;
           tp.n = min(TMAX, thi - tb);
@@ -799,7 +809,7 @@ __global__ void __launch_bounds__(((KT != 0 && WF == W_MXFP4 && TMAX == 1 &&
           int srow[NWR];
 #pragma unroll
           for (int r = 0; r < NWR; ++r)
-            srow[r] = kSwiglu ? (r < RPW ? wi * RPW + r : a.R + wi * RPW + (r - RPW)) : wi * RPW + r;
+            srow[r] = kSwiglu ? (r < RPW ? wr * RPW + r : a.R + wr * RPW + (r - RPW)) : wr * RPW + r;
           if constexpr (kUnroll) {
             const unsigned char* scl = st + codes_bytes;
             float sreg[NWR][KS];
@@ -896,7 +906,8 @@ __global__ void __launch_bounds__(((KT != 0 && WF == W_MXFP4 && TMAX == 1 &&
           } else {
             // bf16 weights: lane owns 8-element (16-byte) chunks, contiguous across the warp
             const int c8 = K >> 3;
-            for (int b8 = lane; b8 < c8; b8 += 32) {
+            const int per = c8 / kq, b8_hi = (ksl == kq - 1) ? c8 : (ksl + 1) * per;
+            for (int b8 = ksl * per + lane; have && b8 < b8_hi; b8 += 32) {
 #pragma unroll
               for (int rp = 0; rp < NWR; rp += 2) {
                 const uint4 qa = lds128(st + (size_t)srow[rp] * rowbytes + 16 * b8);
@@ -936,7 +947,7 @@ __global__ void __launch_bounds__(((KT != 0 && WF == W_MXFP4 && TMAX == 1 &&
               }
             }
           }
-          if (tb + TMAX >= thi) {
+          if (have && tb + TMAX >= thi) {
             // the stage is no longer read: hand it back to the producer
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty_bar[s]);
@@ -954,6 +965,17 @@ __global__ void __launch_bounds__(((KT != 0 && WF == W_MXFP4 && TMAX == 1 &&
           // lane L holds value L / (32 / V); gather what the epilogue lanes need
           const int vi = lane / (32 / V);
           float mine = tot;
+          if (kq > 1) {
+            // K slices: partial sums through shared memory (two buffers, one per
+            // alternate pass), summed in ascending slice order by slice 0's warp
+            float* red = s_red + ((size_t)q0 * 2 + (nred & 1)) * a.wpi * V;
+            ++nred;
+            if ((lane & (32 / V - 1)) == 0) red[wi * V + vi] = tot;
+            group_bar(q0, a.wpi);
+            if (ksl != 0 || !have) continue;
+            mine = 0.f;
+            for (int k2 = 0; k2 < kq; ++k2) mine += red[(wr * kq + k2) * V + vi];
+          }
           // --- epilogue: lanes 0 .. (outputs-1) ---
           const int nout = RPW * TMAX;
           const int oi = lane;  // output index handled by this lane
@@ -966,7 +988,7 @@ __global__ void __launch_bounds__(((KT != 0 && WF == W_MXFP4 && TMAX == 1 &&
 #pragma unroll
             for (int q = 1; q < TMAX; ++q)
               if (t == q) { et = tp.e[q]; orow_t = tp.orow[q]; }
-            const int row = rt * a.R + wi * RPW + rr;
+            const int row = rt * a.R + wr * RPW + rr;
             float val;
             if constexpr (kSwiglu) {
               const float gg = (WF == W_MXFP4) ? g_or_y * pow2f(et) : g_or_y;
@@ -981,6 +1003,7 @@ __global__ void __launch_bounds__(((KT != 0 && WF == W_MXFP4 && TMAX == 1 &&
             a.out[(size_t)orow_t * a.out_rows + row] = val;
           }
         }
+        }  // generic item
         if constexpr (EPI == EPI_DOWN_COMBINE) {
           // publish in batches: see publish_round()
           pend_rt[npend++] = rt;

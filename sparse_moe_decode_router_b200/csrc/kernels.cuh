@@ -83,6 +83,7 @@ struct GemvArgs {
   // L2 prefetch of the next layer's weights (issued by CTAs when their items are done)
   const uint8_t* pf_ptr[2];
   long long pf_bytes[2];
+  int ksplit;       // bf16 streams: warps of a group that split K (partial sums meet in shared memory)
   int pdl_late;     // dense stream whose activations are final at launch: no wait before
                    // reading them; every thread waits for the preceding grid at exit instead
   int* err;

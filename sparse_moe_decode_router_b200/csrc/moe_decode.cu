@@ -27,8 +27,12 @@ size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 enum Kind { K_ROUTER = 0, K_SGU = 1, K_SDN = 2, K_GU = 3, K_DN = 4, K_DNC = 5, K_NUM = 6 };
 
 // Fixed per weight stream: weight format, epilogue, activation type, output
-// rows per warp, warps per item.
-struct KindTraits { int wf, epi, xk, rpw, wpi; };
+// rows per warp row, warps per item, and how many of those warps split K
+// (item rows = rpw * wpi / ks).
+struct KindTraits { int wf, epi, xk, rpw, wpi, ks; };
+#ifndef MOE_DENSE_KSPLIT
+#define MOE_DENSE_KSPLIT 4
+#endif
 #ifndef MOE_GU_RPW
 #define MOE_GU_RPW 1
 #endif
@@ -42,18 +46,20 @@ struct KindTraits { int wf, epi, xk, rpw, wpi; };
 #define MOE_DN_WPI 4
 #endif
 constexpr KindTraits kTraits[K_NUM] = {
-    {W_BF16, EPI_ROUTER, X_BF16, 2, 1},        // router: 2 rows (28 KB) per item
-    {W_BF16, EPI_SWIGLU, X_BF16, 1, 1},        // shared gate/up: 1 output row (2 x 14 KB)
-    {W_BF16, EPI_STORE, X_F32, 2, 4},          // shared down: 8 rows (32 KB)
-    {W_MXFP4, EPI_SWIGLU, X_BF16, MOE_GU_RPW, MOE_GU_WPI},       // routed gate/up: 4 output rows (2 x 14 KB)
-    {W_MXFP4, EPI_STORE, X_F32, MOE_DN_RPW, MOE_DN_WPI},         // routed down: 16 rows (16 KB)
-    {W_MXFP4, EPI_DOWN_COMBINE, X_F32, MOE_DN_RPW, MOE_DN_WPI},  // routed down + combine
+    // router: 2 rows (28 KB) per item, K split over 4 warps
+    {W_BF16, EPI_ROUTER, X_BF16, 2, MOE_DENSE_KSPLIT, MOE_DENSE_KSPLIT},
+    // shared gate/up: 1 output row (2 x 14 KB), K split over 4 warps
+    {W_BF16, EPI_SWIGLU, X_BF16, 1, MOE_DENSE_KSPLIT, MOE_DENSE_KSPLIT},
+    {W_BF16, EPI_STORE, X_F32, 2, 4, 1},          // shared down: 8 rows (32 KB)
+    {W_MXFP4, EPI_SWIGLU, X_BF16, MOE_GU_RPW, MOE_GU_WPI, 1},       // routed gate/up: 4 output rows (2 x 14 KB)
+    {W_MXFP4, EPI_STORE, X_F32, MOE_DN_RPW, MOE_DN_WPI, 1},         // routed down: 16 rows (16 KB)
+    {W_MXFP4, EPI_DOWN_COMBINE, X_F32, MOE_DN_RPW, MOE_DN_WPI, 1},  // routed down + combine
 };
 
 struct GemvPlan {
   bool ok = false;
   int K = 0, out_rows = 0, R = 0, ncw = 0, wpi = 0, n_stages = 0, stage_bytes = 0, stage_offset = 0, x_offset = 0;
-  int xcap = 0, scales_global = 0, threads = 0, smem = 0;
+  int xcap = 0, scales_global = 0, threads = 0, smem = 0, ksplit = 1;
   bool fast = false;  // run the shape-specialised one-token instance
 };
 
@@ -88,7 +94,12 @@ GemvPlan make_plan(Kind kind, int K, int out_rows, int slots_needed, int max_gro
     t.rpw = swiglu ? kSplitKRows / 2 : kSplitKRows;
     t.wpi = rq * ks;
   }
-  const int R = t.rpw * t.wpi / (splitk ? (K / 32 + 31) / 32 : 1);
+  // bf16 K split: only where the 16-byte chunks divide evenly over the slices
+  if (t.ks > 1 && (K / 8) % t.ks != 0) {
+    t.wpi /= t.ks;
+    t.ks = 1;
+  }
+  const int R = t.rpw * t.wpi / (splitk ? (K / 32 + 31) / 32 : t.ks);
   if (K <= 0 || K % 32 || out_rows <= 0 || out_rows % R) return p;
   const int rowbytes = mx ? K / 2 : K * 2;
   const int sbytes = mx ? K / 32 : 0;
@@ -137,6 +148,7 @@ GemvPlan make_plan(Kind kind, int K, int out_rows, int slots_needed, int max_gro
   p.threads = (p.ncw + 1) * 32;
   p.smem = st_off + ns * stage;
   p.fast = fast;
+  p.ksplit = splitk ? 1 : t.ks;
   return p;
 }
 
@@ -256,6 +268,7 @@ GemvArgs base_args(const moe_layer* L, const GemvPlan& p) {
   a.x_offset = p.x_offset;
   a.xcap = p.xcap;
   a.scales_global = p.scales_global;
+  a.ksplit = p.ksplit;
   a.top_k = L->cfg.top_k;
   a.n_experts = L->cfg.n_experts;
   a.err = L->err;
@@ -544,6 +557,15 @@ moe_status_t moe_layer_create(const moe_layer_config* cfg, const moe_layer_weigh
   if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&L->side, cudaStreamNonBlocking);
   if (e == cudaSuccess) e = cudaEventCreateWithFlags(&L->ev_fork, cudaEventDisableTiming);
   if (e == cudaSuccess) e = cudaEventCreateWithFlags(&L->ev_join, cudaEventDisableTiming);
+  // The small kernels run under the same shared-memory carve-out as the
+  // streaming ones: an SM cannot change its carve-out while a CTA is resident,
+  // so a small CTA under a smaller carve-out would keep a streaming CTA (of
+  // the next kernel, launched early) off its SM until it exits.
+  const void* small_kernels[] = {reinterpret_cast<const void*>(topk_bucket_kernel),
+                                 reinterpret_cast<const void*>(combine_kernel)};
+  for (const void* f : small_kernels)
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(f, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
   for (int kk = 0; kk < K_NUM && e == cudaSuccess; ++kk)
     for (int t = 0; t < 2 && e == cudaSuccess; ++t) {
       const GemvPlan& p = L->plans[kk][t];
@@ -737,6 +759,7 @@ moe_status_t moe_router_topk_noalloc(const void* router_w_em, const float* route
   a.stage_offset = p.stage_offset;
   a.x_offset = p.x_offset;
   a.xcap = p.xcap;
+  a.ksplit = p.ksplit;
   a.top_k = top_k;
   a.n_experts = n_experts;
   a.err = &sc->err;
