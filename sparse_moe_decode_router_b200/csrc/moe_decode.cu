@@ -12,6 +12,7 @@
 #include "../../include/moe_decode.h"
 #include "gemv.cuh"
 #include "kernels.cuh"
+#include "mma_grouped.cuh"
 
 using namespace moe;
 
@@ -222,6 +223,10 @@ struct moe_layer {
   float* ys = nullptr;
   int* router_cnt = nullptr;
   int* tile_cnt = nullptr;
+  __half* xh = nullptr;       // grouped path: f16 copy of the activations of one projection
+  int* xe = nullptr;          // ... and its per-row exponents
+  int mma_stages[2] = {0, 0};  // grouped path ring depth: [gate/up, down] (0 = not usable)
+  bool grouped = false;
   int* err = nullptr;
   uint16_t* x_stage = nullptr;
   uint16_t* res_stage = nullptr;
@@ -354,7 +359,15 @@ GemvArgs routed_args(const moe_layer* L, const GemvPlan& p, const moe_routing& r
   return a;
 }
 
+// Batches above this size use the grouped tensor-core expert kernels (at or
+// below it most experts see one token and the GEMV kernels are faster).
+constexpr int kGroupedMinBatch = 8;
+
+cudaError_t launch_grouped(moe_layer* L, bool gate_up, int B, const moe_routing& r, const void* act, float* out,
+                           cudaStream_t st);
+
 cudaError_t launch_gate_up(moe_layer* L, const void* x, int B, const moe_routing& r, cudaStream_t st) {
+  if (B > kGroupedMinBatch && L->grouped) return launch_grouped(L, true, B, r, x, L->h, st);
   const int H = L->cfg.hidden, I = L->cfg.inter;
   const GemvPlan& p = plan_of(L, K_GU, B);
   GemvArgs a = routed_args(L, p, r, B);
@@ -369,8 +382,57 @@ cudaError_t launch_gate_up(moe_layer* L, const void* x, int B, const moe_routing
   return run_gemv(L, K_GU, B, a, st, L->pdl);
 }
 
+// Grouped tensor-core projection (batch > 1): f16 copy of the activation
+// rows, then the MMA kernel.  gate/up: x rows -> h; down: h rows -> y.
+cudaError_t launch_grouped(moe_layer* L, bool gate_up, int B, const moe_routing& r, const void* act, float* out,
+                           cudaStream_t st) {
+  const int H = L->cfg.hidden, I = L->cfg.inter, k = L->cfg.top_k;
+  const int K = gate_up ? H : I;
+  const int rows = gate_up ? B : B * k;
+  cudaError_t e = gate_up ? launch_ex(act_to_f16_kernel<false>, rows, 256, 0, st, L->pdl, act, K, L->xh, L->xe)
+                          : launch_ex(act_to_f16_kernel<true>, rows, 256, 0, st, L->pdl, act, K, L->xh, L->xe);
+  if (e != cudaSuccess) return e;
+  MmaArgs m;
+  std::memset(&m, 0, sizeof(m));
+  m.w = gate_up ? L->w.w_gate_up : L->w.w_down;
+  m.sc = gate_up ? L->w.s_gate_up : L->w.s_down;
+  m.w_gstride = gate_up ? (long long)2 * I * (H / 2) : (long long)H * (I / 2);
+  m.s_gstride = gate_up ? (long long)2 * I * (H / 32) : (long long)H * (I / 32);
+  m.K = K;
+  m.out_rows = gate_up ? I : H;
+  m.up_off = gate_up ? I : 0;
+  m.xh = L->xh;
+  m.xe = L->xe;
+  m.act_by_pair = gate_up ? 0 : 1;
+  m.top_k = k;
+  m.n_pairs = B * k;
+  m.n_experts = L->cfg.n_experts;
+  m.n_active = r.n_active;
+  m.active = r.active;
+  m.offsets = r.offsets;
+  m.pair_ids = r.pair_ids;
+  m.out = out;
+  m.n_stages = L->mma_stages[gate_up ? 0 : 1];
+  m.stage_bytes = (int)align_up((size_t)kMmaRows * (K / 2 + K / 32), 128);
+  m.err = L->err;
+  const int smem = kMmaHeaderBytes + m.n_stages * m.stage_bytes;
+  return gate_up ? launch_ex(grouped_mma_kernel<true>, L->num_sms, (kMmaWarps + 1) * 32, smem, st, L->pdl, m)
+                 : launch_ex(grouped_mma_kernel<false>, L->num_sms, (kMmaWarps + 1) * 32, smem, st, L->pdl, m);
+}
+
+cudaError_t launch_combine(moe_layer* L, int B, const moe_routing& r, const float* y, const float* ys,
+                           const void* residual, void* out, cudaStream_t st);
+
 cudaError_t launch_down(moe_layer* L, int B, const moe_routing& r, float* y, bool fused, const void* residual,
                         void* out, const float* ys, moe_layer* next, cudaStream_t st, bool pdl) {
+  if (B > kGroupedMinBatch && L->grouped) {
+    // tensor-core projection into y, then the fixed-order combine
+    cudaError_t e = launch_grouped(L, false, B, r, L->h, y, st);
+    if (e == cudaSuccess && fused) e = launch_combine(L, B, r, y, ys, residual, out, st);
+    (void)next;
+    (void)pdl;
+    return e;
+  }
   const int H = L->cfg.hidden, I = L->cfg.inter;
   const Kind k = fused ? K_DNC : K_DN;
   const GemvPlan& p = plan_of(L, k, B);
@@ -519,6 +581,8 @@ moe_status_t moe_layer_create(const moe_layer_config* cfg, const moe_layer_weigh
   const size_t o_rc = take(4);
   const size_t o_tc = take((size_t)H * 4);  // one counter per down-projection row tile (<= H)
   const size_t o_er = take(4);
+  const size_t o_xh = take((size_t)MB * std::max(H, k * I) * 2);
+  const size_t o_xe = take((size_t)MB * k * 4);
   const size_t o_xs = take((size_t)MB * H * 2);
   const size_t o_rs = take((size_t)MB * H * 2);
   const size_t o_os = take((size_t)MB * H * 2);
@@ -544,6 +608,8 @@ moe_status_t moe_layer_create(const moe_layer_config* cfg, const moe_layer_weigh
   L->router_cnt = reinterpret_cast<int*>(A + o_rc);
   L->tile_cnt = reinterpret_cast<int*>(A + o_tc);
   L->err = reinterpret_cast<int*>(A + o_er);
+  L->xh = reinterpret_cast<__half*>(A + o_xh);
+  L->xe = reinterpret_cast<int*>(A + o_xe);
   L->x_stage = reinterpret_cast<uint16_t*>(A + o_xs);
   L->res_stage = reinterpret_cast<uint16_t*>(A + o_rs);
   L->out_stage = reinterpret_cast<uint16_t*>(A + o_os);
@@ -561,7 +627,28 @@ moe_status_t moe_layer_create(const moe_layer_config* cfg, const moe_layer_weigh
   // streaming ones: an SM cannot change its carve-out while a CTA is resident,
   // so a small CTA under a smaller carve-out would keep a streaming CTA (of
   // the next kernel, launched early) off its SM until it exits.
+  // grouped tensor-core path (batch > 1): ring depth per projection
+  if (!(c.flags & MOE_FLAG_NO_GROUPED) && MB > 1) {
+    const int Ks[2] = {H, I};
+    bool ok = true;
+    for (int q = 0; q < 2; ++q) {
+      const int K = Ks[q];
+      if (K % (32 * kMmaWarps) != 0) { ok = false; break; }
+      const int stage = (int)align_up((size_t)kMmaRows * (K / 2 + K / 32), 128);
+      const int ns = std::min(kMmaMaxStages, (kSmemBudget - kMmaHeaderBytes) / stage);
+      if (ns < 2) { ok = false; break; }
+      L->mma_stages[q] = ns;
+    }
+    if (ok && (I % (kMmaRows / 2)) == 0 && (H % kMmaRows) == 0) L->grouped = true;
+  }
+  if (e == cudaSuccess && L->grouped) {
+    e = cudaFuncSetAttribute(grouped_mma_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBudget);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(grouped_mma_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBudget);
+  }
   const void* small_kernels[] = {reinterpret_cast<const void*>(topk_bucket_kernel),
+                                 reinterpret_cast<const void*>(act_to_f16_kernel<false>),
+                                 reinterpret_cast<const void*>(act_to_f16_kernel<true>),
                                  reinterpret_cast<const void*>(combine_kernel)};
   for (const void* f : small_kernels)
     if (e == cudaSuccess)

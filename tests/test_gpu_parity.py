@@ -190,6 +190,7 @@ def test_full_size_b64_zipf(torch_cuda, full_layers):
         out2 = torch.empty_like(out)
         api.moe_layer_forward(h, None, x_d, r_d, out2, B)
         torch.cuda.synchronize()
+        assert api.moe_layer_last_device_error(h) == api.MOE_OK
         assert np.array_equal(to_host_u16(out2), out_h)          # run to run bit-identical
     finally:
         api.moe_layer_destroy(h)
