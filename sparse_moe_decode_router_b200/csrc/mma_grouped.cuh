@@ -29,6 +29,7 @@ constexpr int kMmaWarps = 8;       // consumer warps (K slices)
 constexpr int kMmaRows = 16;       // weight rows per item
 constexpr int kMmaNTiles = 4;      // token tiles of 8 handled per pass (32 tokens)
 constexpr int kMmaMaxStages = 8;
+constexpr int kMmaPf = 4;  // blocks of activation fragments fetched ahead
 // dynamic shared memory ahead of the ring: barriers, abort flag, partial sums
 constexpr int kMmaHeaderBytes = 256 + 2 * 8 * 4 * 32 * 4 * 4;
 
@@ -59,6 +60,9 @@ struct MmaArgs {
 // f16 copy of activation rows: row r of `src` (bf16 or fp32, K elements) is
 // scaled by 2^-e, e chosen from max|x| so that the largest element sits in
 // [2^14, 2^15) (exact for bf16, one rounding for fp32); one CTA per row.
+// Within each 32-element block the elements are stored in the order the MMA's
+// B fragments want them: thread tq of a quad takes elements {2tq, 2tq+1,
+// 2tq+8, 2tq+9, 2tq+16, 2tq+17, 2tq+24, 2tq+25} as one 16-byte vector.
 template <bool kF32>
 __global__ void __launch_bounds__(256) act_to_f16_kernel(const void* __restrict__ src, int K, __half* __restrict__ dst,
                                                          int* __restrict__ exps) {
@@ -93,7 +97,9 @@ __global__ void __launch_bounds__(256) act_to_f16_kernel(const void* __restrict_
   for (int i = tid; i < K; i += 256) {
     const float v = kF32 ? __ldcg(static_cast<const float*>(src) + (size_t)r * K + i)
                          : bf16lo_to_f32(static_cast<const uint16_t*>(src)[(size_t)r * K + i]);
-    dst[(size_t)r * K + i] = __float2half_rn(v * sc);
+    const int p = i & 31;
+    const int pos = ((i >> 5) * 4 + ((p >> 1) & 3)) * 8 + (((p >> 4) * 2 + ((p >> 3) & 1)) * 2) + (p & 1);
+    dst[(size_t)r * K + pos] = __float2half_rn(v * sc);
   }
   pdl_launch_dependents();
 }
@@ -121,9 +127,9 @@ __device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4],
         "f"(c[3]));
 }
 
-__device__ __forceinline__ uint32_t ldg_u32_cg(const void* p) {
-  uint32_t v;
-  asm volatile("ld.global.cg.u32 %0, [%1];" : "=r"(v) : "l"(p));
+__device__ __forceinline__ uint4 ldg128_cg(const void* p) {
+  uint4 v;
+  asm volatile("ld.global.cg.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
   return v;
 }
 
@@ -241,6 +247,7 @@ __global__ void __launch_bounds__((kMmaWarps + 1) * 32, 1) grouped_mma_kernel(co
       s_flag[0] = 1;
       have = false;
     }
+    have = __all_sync(0xFFFFFFFFu, have);  // the MMAs below need the whole warp
     const unsigned char* st = stages + (size_t)s * a.stage_bytes;
     // token passes of up to 8 * kMmaNTiles tokens; every warp runs the same passes
     for (int t0 = 0; t0 < max(ntok, 1); t0 += 8 * kMmaNTiles) {
@@ -269,38 +276,61 @@ __global__ void __launch_bounds__((kMmaWarps + 1) * 32, 1) grouped_mma_kernel(co
         const unsigned char* rowA = st + (size_t)gq * rowbytes;
         const unsigned char* rowB = st + (size_t)(gq + 8) * rowbytes;
         const unsigned char* scl = st + codes_bytes;
-        for (int i = 0; i < nblk; ++i) {
-          const int kb = kb0 + i;
-          const uint4 wa = lds128(rowA + 16 * kb), wb = lds128(rowB + 16 * kb);
-          const float sa = e8m0_to_f32(lds_u8(scl + gq * sblocks + kb));
-          const float sbv = e8m0_to_f32(lds_u8(scl + (gq + 8) * sblocks + kb));
-          uint32_t a0[4], a1[4];
-          a0[0] = e2m1_byte_to_f16x2(wa.x, sh);
-          a0[1] = e2m1_byte_to_f16x2(wb.x, sh);
-          a0[2] = e2m1_byte_to_f16x2(wa.y, sh);
-          a0[3] = e2m1_byte_to_f16x2(wb.y, sh);
-          a1[0] = e2m1_byte_to_f16x2(wa.z, sh);
-          a1[1] = e2m1_byte_to_f16x2(wb.z, sh);
-          a1[2] = e2m1_byte_to_f16x2(wa.w, sh);
-          a1[3] = e2m1_byte_to_f16x2(wb.w, sh);
-          const int kel = kb * 32 + 2 * tq;
+        // Token tiles two at a time; their activation fragments (one 16-byte
+        // load per block, tile and lane) are fetched kMmaPf blocks ahead.  The
+        // MMAs are warp-collective: whether a tile is computed depends only on
+        // warp-uniform values; a lane without a token in a tile feeds zeros.
 #pragma unroll
-          for (int nt = 0; nt < kMmaNTiles; ++nt) {
-            if (nt < ntiles) {
-              uint32_t b00 = 0, b01 = 0, b10 = 0, b11 = 0;
-              if (xrow[nt]) {
-                b00 = ldg_u32_cg(xrow[nt] + kel);
-                b01 = ldg_u32_cg(xrow[nt] + kel + 8);
-                b10 = ldg_u32_cg(xrow[nt] + kel + 16);
-                b11 = ldg_u32_cg(xrow[nt] + kel + 24);
+        for (int pp = 0; pp < kMmaNTiles / 2; ++pp) {
+          if (2 * pp < ntiles) {
+            const bool two = 2 * pp + 1 < ntiles;  // warp-uniform
+            const uint4* xp0 = reinterpret_cast<const uint4*>(xrow[2 * pp]);
+            const uint4* xp1 = two ? reinterpret_cast<const uint4*>(xrow[2 * pp + 1]) : nullptr;
+            uint4 xq[kMmaPf][2];
+#pragma unroll
+            for (int j = 0; j < kMmaPf; ++j) {
+              const int kb = kb0 + j;
+              xq[j][0] = (xp0 && j < nblk) ? ldg128_cg(xp0 + kb * 4 + tq) : make_uint4(0u, 0u, 0u, 0u);
+              xq[j][1] = (xp1 && j < nblk) ? ldg128_cg(xp1 + kb * 4 + tq) : make_uint4(0u, 0u, 0u, 0u);
+            }
+            for (int i = 0; i < nblk; i += kMmaPf) {
+#pragma unroll
+              for (int j = 0; j < kMmaPf; ++j) {
+                const int ib = i + j;
+                if (ib < nblk) {  // warp-uniform
+                  const int kb = kb0 + ib;
+                  const uint4 wa = lds128(rowA + 16 * kb), wb = lds128(rowB + 16 * kb);
+                  const float sa = e8m0_to_f32(lds_u8(scl + gq * sblocks + kb));
+                  const float sbv = e8m0_to_f32(lds_u8(scl + (gq + 8) * sblocks + kb));
+                  uint32_t a0[4], a1[4];
+                  a0[0] = e2m1_byte_to_f16x2(wa.x, sh);
+                  a0[1] = e2m1_byte_to_f16x2(wb.x, sh);
+                  a0[2] = e2m1_byte_to_f16x2(wa.y, sh);
+                  a0[3] = e2m1_byte_to_f16x2(wb.y, sh);
+                  a1[0] = e2m1_byte_to_f16x2(wa.z, sh);
+                  a1[1] = e2m1_byte_to_f16x2(wb.z, sh);
+                  a1[2] = e2m1_byte_to_f16x2(wa.w, sh);
+                  a1[3] = e2m1_byte_to_f16x2(wb.w, sh);
+#pragma unroll
+                  for (int h = 0; h < 2; ++h) {
+                    if (h == 0 || two) {  // warp-uniform
+                      float d[4];
+                      mma_16816(d, a0, xq[j][h].x, xq[j][h].y, zero);
+                      mma_16816(d, a1, xq[j][h].z, xq[j][h].w, d);
+                      float(&ac)[4] = acc[2 * pp + h];
+                      ac[0] = fmaf(d[0], sa, ac[0]);
+                      ac[1] = fmaf(d[1], sa, ac[1]);
+                      ac[2] = fmaf(d[2], sbv, ac[2]);
+                      ac[3] = fmaf(d[3], sbv, ac[3]);
+                    }
+                  }
+                  const int nb = ib + kMmaPf;
+                  if (nb < nblk) {
+                    if (xp0) xq[j][0] = ldg128_cg(xp0 + (kb0 + nb) * 4 + tq);
+                    if (xp1) xq[j][1] = ldg128_cg(xp1 + (kb0 + nb) * 4 + tq);
+                  }
+                }
               }
-              float d[4];
-              mma_16816(d, a0, b00, b01, zero);
-              mma_16816(d, a1, b10, b11, d);
-              acc[nt][0] = fmaf(d[0], sa, acc[nt][0]);
-              acc[nt][1] = fmaf(d[1], sa, acc[nt][1]);
-              acc[nt][2] = fmaf(d[2], sbv, acc[nt][2]);
-              acc[nt][3] = fmaf(d[3], sbv, acc[nt][3]);
             }
           }
         }
@@ -328,6 +358,7 @@ __global__ void __launch_bounds__((kMmaWarps + 1) * 32, 1) grouped_mma_kernel(co
         s_flag[0] = 1;
         have = false;
       }
+      have = __all_sync(0xFFFFFFFFu, have);
       gph ^= 1u;
       if (have && warp == (int)(npass_done % kMmaWarps) && npass > 0) {
 #pragma unroll
