@@ -361,7 +361,10 @@ GemvArgs routed_args(const moe_layer* L, const GemvPlan& p, const moe_routing& r
 
 // Batches above this size use the grouped tensor-core expert kernels (at or
 // below it most experts see one token and the GEMV kernels are faster).
-constexpr int kGroupedMinBatch = 8;
+#ifndef MOE_GROUPED_MIN_BATCH
+#define MOE_GROUPED_MIN_BATCH 8
+#endif
+constexpr int kGroupedMinBatch = MOE_GROUPED_MIN_BATCH;
 
 cudaError_t launch_grouped(moe_layer* L, bool gate_up, int B, const moe_routing& r, const void* act, float* out,
                            cudaStream_t st);
@@ -628,7 +631,7 @@ moe_status_t moe_layer_create(const moe_layer_config* cfg, const moe_layer_weigh
   // so a small CTA under a smaller carve-out would keep a streaming CTA (of
   // the next kernel, launched early) off its SM until it exits.
   // grouped tensor-core path (batch > 1): ring depth per projection
-  if (!(c.flags & MOE_FLAG_NO_GROUPED) && MB > 1) {
+  if (!(c.flags & MOE_FLAG_NO_GROUPED) && MB > kGroupedMinBatch) {
     const int Ks[2] = {H, I};
     bool ok = true;
     for (int q = 0; q < 2; ++q) {
