@@ -1005,8 +1005,12 @@ __global__ void __launch_bounds__(((KT != 0 && WF == W_MXFP4 && TMAX == 1 &&
         }
         }  // generic item
         if constexpr (EPI == EPI_DOWN_COMBINE) {
-          // publish in batches: see publish_round()
-          pend_rt[npend++] = rt;
+          // publish in batches: see publish_round().  A group whose tokens are
+          // split over several phases (more activation rows than slots) runs
+          // each of its items once per phase: the item counts once, with the
+          // phase that holds the group's last tokens (the earlier phases' y
+          // stores are ordered before it by the phase barrier).
+          if (thi >= ntok) pend_rt[npend++] = rt;
           if (npend == kPubBatch) {
             publish_round(a, pend_rt, npend, prev_cnt, prev_rt, nprev, n_groups, wi, q0, lane, s_pub + q0 * kPubInts);
             npend = 0;

@@ -114,6 +114,33 @@ def test_tiny_variants_match_oracle(torch_cuda, variant):
         check_against_oracle(got, ref, shared=cfg.shared_inter > 0)
 
 
+@pytest.fixture(scope="module")
+def skewed_small(torch_cuda):
+    # K = 512 and 256 are multiples of 256, so batches above 8 take the grouped
+    # tensor-core kernels; the Zipf bias piles tokens onto a few experts
+    base = synth.CONFIGS[0]
+    return make_device_layer(base.with_(hidden=512, inter=256, shared_inter=64, zipf_s=1.1, seed=base.seed + 300))
+
+
+@pytest.mark.parametrize("B", [9, 33, 64])
+def test_grouped_kernels_match_oracle(torch_cuda, skewed_small, B):
+    """Grouped path on every token: B=33 has an expert with 27 tokens (four
+    8-token tiles), B=64 one with 56 (two passes of 32 per item)."""
+    got, ref = run_all_paths(torch_cuda, skewed_small, B, max_batch=64)
+    check_against_oracle(got, ref)
+    if B == 64:
+        assert ref["counts"].max() > 32
+
+
+def test_grouped_and_gemv_paths_agree_within_tolerance(torch_cuda, skewed_small):
+    """MOE_FLAG_NO_GROUPED keeps batch 64 on the GEMV kernels: both paths
+    meet the oracle (their sums run in different fixed orders)."""
+    got_g, ref = run_all_paths(torch_cuda, skewed_small, 64, max_batch=64)
+    got_v, _ = run_all_paths(torch_cuda, skewed_small, 64, max_batch=64, flags=8)
+    check_against_oracle(got_g, ref)
+    check_against_oracle(got_v, ref)
+
+
 @pytest.mark.parametrize("flags", [1, 2, 4, 7])
 def test_tiny_flags_give_identical_results(torch_cuda, tiny, flags):
     base, _ = run_all_paths(torch_cuda, tiny, 3, max_batch=4)
