@@ -83,12 +83,12 @@ struct GemvPlan {
 #endif
 
 GemvPlan make_plan(Kind kind, int K, int out_rows, int slots_needed, int max_groups, int tok_per_group,
-                   long long s_gstride, int num_sms, bool fast = false) {
+                   long long s_gstride, int num_sms, bool fast = false, bool splitk_ok = true) {
   GemvPlan p;
   KindTraits t = kTraits[kind];
   const bool mx = t.wf == W_MXFP4;
   const bool swiglu = t.epi == EPI_SWIGLU;
-  const bool splitk = fast && mx && (!swiglu || MOE_SPLITK_GU);  // warps = row quarters x K slices
+  const bool splitk = splitk_ok && fast && mx && (!swiglu || MOE_SPLITK_GU);  // warps = row quarters x K slices
   if (splitk) {
     const int ks = (K / 32 + 31) / 32;
     const int rq = swiglu ? MOE_SPLITK_GU_RQ : MOE_SPLITK_DN_RQ;
@@ -159,7 +159,7 @@ typedef void (*GemvFn)(const GemvArgs);
 constexpr int kFastH = 7168;
 constexpr int kFastI = 2048;
 
-template <int TMAX, int KH, int KI>
+template <int TMAX, int KH, int KI, bool kSplitDn = true>
 GemvFn pick_fn(Kind k) {
   switch (k) {
     case K_ROUTER: return gemv_kernel<W_BF16, EPI_ROUTER, X_BF16, TMAX, 2, KH>;
@@ -168,17 +168,24 @@ GemvFn pick_fn(Kind k) {
     // instances with a compile-time K and one token are the split-K ones
     case K_GU:
       return gemv_kernel<W_MXFP4, EPI_SWIGLU, X_BF16, TMAX, (KH && TMAX == 1 && MOE_SPLITK_GU) ? kSplitKRows / 2 : MOE_GU_RPW, KH>;
-    case K_DN: return gemv_kernel<W_MXFP4, EPI_STORE, X_F32, TMAX, (KI && TMAX == 1) ? kSplitKRows : MOE_DN_RPW, KI>;
+    case K_DN:
+      return gemv_kernel<W_MXFP4, EPI_STORE, X_F32, TMAX, (KI && TMAX == 1 && kSplitDn) ? kSplitKRows : MOE_DN_RPW, KI>;
     case K_DNC:
-      return gemv_kernel<W_MXFP4, EPI_DOWN_COMBINE, X_F32, TMAX, (KI && TMAX == 1) ? kSplitKRows : MOE_DN_RPW, KI>;
+      return gemv_kernel<W_MXFP4, EPI_DOWN_COMBINE, X_F32, TMAX,
+                         (KI && TMAX == 1 && kSplitDn) ? kSplitKRows : MOE_DN_RPW, KI>;
     default: return nullptr;
   }
 }
 
 // fast = the shape-specialised one-token instance (K must be kFastI for the
 // down projections, kFastH for the others)
-GemvFn gemv_fn(Kind k, int tmax, bool fast = false) {
-  if (tmax == 1) return fast ? pick_fn<1, kFastH, kFastI>(k) : pick_fn<1, 0, 0>(k);
+// small = the one-token-per-pass plans of batches 2..kSmallBatch (no split-K:
+// those instances take exactly one token per item)
+GemvFn gemv_fn(Kind k, int tmax, bool fast = false, bool small = false) {
+  if (tmax == 1) {
+    if (!fast) return pick_fn<1, 0, 0>(k);
+    return small ? pick_fn<1, kFastH, kFastI, false>(k) : pick_fn<1, kFastH, kFastI>(k);
+  }
   return pick_fn<2, 0, 0>(k);
 }
 
@@ -234,14 +241,21 @@ struct moe_layer {
   cudaStream_t side = nullptr;
   cudaEvent_t ev_fork = nullptr, ev_join = nullptr;
   cudaEvent_t probe_start = nullptr, probe_stop = nullptr;
-  GemvPlan plans[K_NUM][2];  // [kind][tmax==1 ? 0 : 1]
+  GemvPlan plans[K_NUM][3];  // [kind][plan slot: 0 batch 1, 1 two tokens per pass, 2 small batches]
 };
 
 namespace {
 
 moe_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
 
-int tmax_for(int B) { return B == 1 ? 1 : 2; }
+// Batches 2..kSmallBatch take one token per pass (most of their experts see
+// one token) on the compile-time-K instances; larger ones two per pass.
+// The dense bf16 streams keep two tokens per pass there.
+constexpr int kSmallBatch = 8;
+bool routed_kind(Kind k) { return k == K_GU || k == K_DN || k == K_DNC; }
+int slot_for(Kind k, int B) { return B == 1 ? 0 : ((B <= kSmallBatch && routed_kind(k)) ? 2 : 1); }
+int tmax_of_slot(int t) { return t == 1 ? 2 : 1; }
+int tmax_for(int B) { return B == 1 ? 1 : 2; }  // dense streams
 
 template <typename... Args>
 cudaError_t launch_ex(void (*kern)(Args...), int grid, int block, int smem, cudaStream_t st, bool pdl,
@@ -281,12 +295,12 @@ GemvArgs base_args(const moe_layer* L, const GemvPlan& p) {
 }
 
 cudaError_t run_gemv(moe_layer* L, Kind k, int B, const GemvArgs& a, cudaStream_t st, bool pdl) {
-  const int tm = tmax_for(B);
-  const GemvPlan& p = L->plans[k][tm == 1 ? 0 : 1];
-  return launch_ex(gemv_fn(k, tm, p.fast), L->num_sms, p.threads, p.smem, st, pdl, a);
+  const int sl = slot_for(k, B);
+  const GemvPlan& p = L->plans[k][sl];
+  return launch_ex(gemv_fn(k, tmax_of_slot(sl), p.fast, sl == 2), L->num_sms, p.threads, p.smem, st, pdl, a);
 }
 
-const GemvPlan& plan_of(const moe_layer* L, Kind k, int B) { return L->plans[k][tmax_for(B) == 1 ? 0 : 1]; }
+const GemvPlan& plan_of(const moe_layer* L, Kind k, int B) { return L->plans[k][slot_for(k, B)]; }
 
 bool routing_ok(const moe_routing* r) {
   return r && r->topk_idx && r->topk_w && r->counts && r->offsets && r->pair_ids && r->active && r->n_active;
@@ -541,14 +555,26 @@ moe_status_t moe_layer_create(const moe_layer_config* cfg, const moe_layer_weigh
 
   const int H = c.hidden, E = c.n_experts, k = c.top_k, I = c.inter, Is = c.shared_inter, MB = c.max_batch;
   // plans: [0] for B = 1 (one token per pass), [1] for B > 1 (two per pass)
-  for (int t = 0; t < 2; ++t) {
-    const int nb = t == 0 ? 1 : MB;
+  for (int t = 0; t < 3; ++t) {
+    const int nb = t == 0 ? 1 : (t == 2 ? std::min(MB, kSmallBatch) : MB);
     const int maxg = std::min(E, nb * k);  // experts one call can activate
-    const bool fh = t == 0 && H == kFastH, fi = t == 0 && I == kFastI, fis = t == 0 && Is == kFastI;
+    const bool one = t != 1;            // one token per pass
+    const bool fh = one && H == kFastH, fi = one && I == kFastI, fis = one && Is == kFastI;
+    const bool sk = t == 0;             // split-K down projection: batch 1 only
+    if (t == 2) {  // routed kinds only
+      L->plans[K_GU][t] = make_plan(K_GU, H, I, nb, maxg, nb, (long long)2 * I * (H / 32), sms, fh);
+      L->plans[K_DN][t] = make_plan(K_DN, I, H, nb * k, maxg, nb, (long long)H * (I / 32), sms, fi, false);
+      L->plans[K_DNC][t] = make_plan(K_DNC, I, H, nb * k, maxg, nb, (long long)H * (I / 32), sms, fi, false);
+      if (!(L->plans[K_GU][t].ok && L->plans[K_DN][t].ok && L->plans[K_DNC][t].ok)) {
+        delete L;
+        return MOE_ERR_UNSUPPORTED;
+      }
+      continue;
+    }
     L->plans[K_ROUTER][t] = make_plan(K_ROUTER, H, E, nb, 1, nb, 0, sms, fh);
     L->plans[K_GU][t] = make_plan(K_GU, H, I, nb, maxg, nb, (long long)2 * I * (H / 32), sms, fh);
-    L->plans[K_DN][t] = make_plan(K_DN, I, H, nb * k, maxg, nb, (long long)H * (I / 32), sms, fi);
-    L->plans[K_DNC][t] = make_plan(K_DNC, I, H, nb * k, maxg, nb, (long long)H * (I / 32), sms, fi);
+    L->plans[K_DN][t] = make_plan(K_DN, I, H, nb * k, maxg, nb, (long long)H * (I / 32), sms, fi, sk);
+    L->plans[K_DNC][t] = make_plan(K_DNC, I, H, nb * k, maxg, nb, (long long)H * (I / 32), sms, fi, sk);
     if (Is > 0) {
       L->plans[K_SGU][t] = make_plan(K_SGU, H, Is, nb, 1, nb, 0, sms, fh);
       L->plans[K_SDN][t] = make_plan(K_SDN, Is, H, nb, 1, nb, 0, sms, fis);
@@ -657,10 +683,10 @@ moe_status_t moe_layer_create(const moe_layer_config* cfg, const moe_layer_weigh
     if (e == cudaSuccess)
       e = cudaFuncSetAttribute(f, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
   for (int kk = 0; kk < K_NUM && e == cudaSuccess; ++kk)
-    for (int t = 0; t < 2 && e == cudaSuccess; ++t) {
+    for (int t = 0; t < 3 && e == cudaSuccess; ++t) {
       const GemvPlan& p = L->plans[kk][t];
       if (!p.ok) continue;
-      e = cudaFuncSetAttribute(gemv_fn((Kind)kk, t == 0 ? 1 : 2, p.fast), cudaFuncAttributeMaxDynamicSharedMemorySize,
+      e = cudaFuncSetAttribute(gemv_fn((Kind)kk, tmax_of_slot(t), p.fast, t == 2), cudaFuncAttributeMaxDynamicSharedMemorySize,
                                p.smem);
     }
   if (e == cudaSuccess) e = cudaDeviceSynchronize();
