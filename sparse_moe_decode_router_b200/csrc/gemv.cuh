@@ -391,10 +391,7 @@ __host__ __device__ constexpr int x_row_bytes(int wf, int xk, int K) {
 // lane, in ascending expert order.
 constexpr int kPubBatch = 8;
 
-#ifndef MOE_L2_AHEAD
-#define MOE_L2_AHEAD 0
-#endif
-constexpr int kL2Ahead = MOE_L2_AHEAD;  // items the producer prefetches into L2 ahead of the ring
+
 constexpr int kPubInts = kPubBatch + 1;  // per group: [0] = tiles to combine, [1..] = their row tiles
 
 __device__ __forceinline__ void group_bar(int q0, int wpi) {
@@ -552,33 +549,6 @@ __global__ void __launch_bounds__(((KT != 0 && WF == W_MXFP4 && TMAX == 1 &&
       uint32_t ph = 0;
       bool ok = true;
       int pg = -1, pgrp = 0;  // cached group -> expert lookup
-      // L2 prefetch kL2Ahead items ahead of the copies into the ring, so that
-      // the bytes in flight per SM are not bounded by the ring's size: a ring
-      // copy then finds its lines in L2 (or on their way there).
-      const long long n_mine = hi - lo;
-      const bool scale_pf = WF == W_MXFP4 && ((a.R * sblocks) & 15) == 0 && (a.s_gstride & 15) == 0 &&
-                            ((a.up_off * sblocks) & 15) == 0;
-      // the prefetch cursor walks the CTA's items in order; the expert of its
-      // group is looked up once per group
-      int g2 = (int)(lo / n_rt), rt2 = (int)(lo - (long long)g2 * n_rt), cg2 = -1, grp2 = 0;
-      auto l2_ahead = [&]() {
-        if (g2 != cg2) {
-          cg2 = g2;
-          grp2 = a.routed ? clamp_group(a.active[g2], a.n_experts, nullptr) : 0;
-        }
-        const int r02 = rt2 * a.R;
-        if (++rt2 == n_rt) { rt2 = 0; ++g2; }
-        const uint8_t* wg2 = a.w + (long long)grp2 * a.w_gstride;
-        const uint32_t cb2 = (uint32_t)(a.R * rowbytes);
-        prefetch_l2(wg2 + (size_t)r02 * rowbytes, cb2);
-        if (kSwiglu) prefetch_l2(wg2 + (size_t)(r02 + a.up_off) * rowbytes, cb2);
-        if (scale_pf) {
-          const uint8_t* sg2 = a.sc + (long long)grp2 * a.s_gstride;
-          prefetch_l2(sg2 + (size_t)r02 * sblocks, (uint32_t)(a.R * sblocks));
-          if (kSwiglu) prefetch_l2(sg2 + (size_t)(r02 + a.up_off) * sblocks, (uint32_t)(a.R * sblocks));
-        }
-      };
-      for (long long jl = 0; jl < kL2Ahead && jl < n_mine; ++jl) l2_ahead();
       for (int p = 0; p < pt->n && ok; ++p) {
         const int jbeg = pt->ph[p].first_item, jend = pt->ph[p].last_item;
         int g = (int)((lo + jbeg) / n_rt);
@@ -609,7 +579,6 @@ __global__ void __launch_bounds__(((KT != 0 && WF == W_MXFP4 && TMAX == 1 &&
             if (kSwiglu)
               bulk_g2s(st + codes_bytes + sb, sg + (size_t)(r0 + a.up_off) * sblocks, sb, &full_bar[s], pol);
           }
-          if (kL2Ahead > 0 && j + kL2Ahead < n_mine) l2_ahead();
           if (++s == a.n_stages) { s = 0; ph ^= 1u; }
         }
       }

@@ -60,7 +60,7 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
 // ---- bulk copies (TMA, no tensor map, no multicast) ---------------------------
 // 16-byte aligned src/dst, size a multiple of 16; completion is signalled as
 // transaction bytes on `bar`.  `policy` is an L2 cache policy from
-// l2_policy_evict_first()/l2_policy_evict_last().
+// l2_policy_evict_first().
 __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar,
                                          uint64_t policy) {
   asm volatile(
@@ -73,12 +73,6 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
 __device__ __forceinline__ uint64_t l2_policy_evict_first() {
   uint64_t p;
   asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
-  return p;
-}
-
-__device__ __forceinline__ uint64_t l2_policy_evict_last() {
-  uint64_t p;
-  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
   return p;
 }
 
@@ -114,14 +108,6 @@ __device__ __forceinline__ uint4 lds128(const void* p) {
 __device__ __forceinline__ uint4 lds128_s(uint32_t addr) {
   uint4 v;
   asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
-  return v;
-}
-
-// Read-only byte load that stays where it is written (volatile): a prefetch
-// into a register whose value is used much later.
-__device__ __forceinline__ uint32_t ldg_u8_early(const void* p) {
-  uint32_t v;
-  asm volatile("ld.global.nc.u8 %0, [%1];" : "=r"(v) : "l"(p));
   return v;
 }
 
