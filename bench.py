@@ -112,11 +112,37 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------- helpers ------
+def _code_only(src):
+    """C++ source with comments and blank lines removed (string literals kept)."""
+    out, i, n = [], 0, len(src)
+    while i < n:
+        c = src[i]
+        if c == '"':
+            j = i + 1
+            while j < n and src[j] != '"':
+                j += 2 if src[j] == "\\" else 1
+            out.append(src[i:j + 1])
+            i = j + 1
+        elif src.startswith("//", i):
+            i = src.find("\n", i)
+            i = n if i < 0 else i
+        elif src.startswith("/*", i):
+            j = src.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+        else:
+            out.append(c)
+            i += 1
+    return "\n".join(l.rstrip() for l in "".join(out).splitlines() if l.strip())
+
+
 def kernel_source_sha():
+    """Hash of the code (comments ignored) of the sources that build the
+    routed gate/up kernel: a recorded ncu traffic figure stays valid as long
+    as this hash is unchanged."""
     h = hashlib.sha256()
     for f in ("kernels.cuh", "gemv.cuh", "ptx.cuh", "moe_decode.cu"):
-        with open(os.path.join(ROOT, "sparse_moe_decode_router_b200", "csrc", f), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(ROOT, "sparse_moe_decode_router_b200", "csrc", f), encoding="utf-8") as fh:
+            h.update(_code_only(fh.read()).encode())
     return h.hexdigest()[:16]
 
 

@@ -11,22 +11,27 @@
 //    the E8M0 scale rows) into a ring of shared-memory stages with 1-D TMA
 //    bulk copies (evict-first L2 policy: weights are read once per step);
 //    completion is counted on per-stage mbarriers;
-//  * an item is shared by a small group of warps, each owning whole rows:
-//    its lanes split K, so a row's dot product needs only an in-warp
-//    butterfly; warps never wait for each other in the steady state (the
-//    stage is handed back with one mbarrier arrive per warp, no CTA barrier);
+//  * an item is taken by a group of warps.  By default each warp owns whole
+//    rows and its lanes split K, so a row's dot product needs only an in-warp
+//    butterfly and the stage is handed back with one mbarrier arrive per
+//    warp.  The bf16 router and shared gate/up split K over the group's
+//    warps, and the one-token MXFP4 down projection ("split-K" instances)
+//    gives each lane one 32-element block of a warp-wide K slice; there the
+//    warps' partial sums meet in shared memory behind a group barrier and
+//    are added in ascending slice order by one warp;
 //  * the activation vectors an item needs sit in shared memory, staged once
 //    per "phase" (a run of groups whose tokens fit): MXFP4 streams keep them
 //    as f16 scaled by a per-vector power of two (exact for bf16 inputs,
 //    11-bit rounding for fp32 ones) in a lane-interleaved layout that makes
 //    every 16-byte read conflict-free; bf16 streams keep bf16 or fp32 as is;
-//  * MXFP4 weights are decoded in registers (cvt e2m1x2 -> f16x2) and fed to
-//    fp32-accumulating mixed-precision FMAs; each lane's 32-element chunk is
-//    one scale block, so the E8M0 scale is applied once per chunk in fp32;
+//  * MXFP4 weights are decoded in registers (cvt e2m1x2 -> f16x2); products
+//    and partial sums over eight products are packed f16 (fma.rn.f16x2), the
+//    block's partial sums are added in fp32 and scaled by its E8M0 value, and
+//    blocks accumulate in fp32; bf16 weights use mixed fp32 FMAs;
 //  * epilogues: store, SwiGLU, router logits (+ bias; top-k follows in its own
-//    kernel), and the down projection fused with the
-//    routing-weight combine and residual add (the last warp to finish a row
-//    tile over all active experts sums that tile in ascending expert order).
+//    kernel), and the down projection fused with the routing-weight combine
+//    and residual add (the warp group that completes a row tile over all
+//    active experts combines it in ascending expert order).
 #pragma once
 #include <cstdint>
 #include <cuda_fp16.h>

@@ -43,3 +43,14 @@ def test_max_over_two_gloo_ranks_and_job_value():
     assert bench.max_over_ranks([1.0, 2.0]) == [1.0, 2.0]       # no process group: identity
     # two replicas, 1 GB each per run, slowest rank 2 ms -> 1000 GB/s for the job
     assert bench.job_value(2, 1e9, 2.0) == pytest.approx(1000.0)
+
+
+def test_source_hash_ignores_comments_only():
+    """The hash that ties a recorded ncu traffic figure to the kernel sources
+    changes with the code, not with comments."""
+    import bench
+    a = "int a = 1;  // one\n/* block\n comment */\nconst char* s = \"//kept\";\n"
+    b = "int a = 1;\n\nconst char* s = \"//kept\";  /* other */\n"
+    assert bench._code_only(a) == bench._code_only(b)
+    assert bench._code_only("int a = 2;") != bench._code_only("int a = 1;")
+    assert "//kept" in bench._code_only(a)
