@@ -136,12 +136,17 @@ MOE_API moe_status_t moe_layer_destroy(moe_layer_t layer);
 /* Router GEMV + top-k + softmax + bucketing for B tokens (the router row and
  * the top-k selection of the pages: aitest123 intro, 16 of 896 experts).
  * x: bf16 [B][H].  r: where to write the plan; NULL = the layer's own
- * buffers (see moe_layer_routing).  One kernel launch. */
+ * buffers (see moe_layer_routing).  Two kernel launches (router GEMV, then
+ * top-k / softmax / bucketing), chained with programmatic dependent launch. */
 MOE_API moe_status_t moe_router_topk(moe_layer_t layer, const void* x, int B, const moe_routing* r,
                              void* stream);
 
 /* The selected experts and the shared expert for B tokens, given a routing
- * plan from moe_router_topk (r NULL = the layer's own plan).
+ * plan from moe_router_topk (r NULL = the layer's own plan).  Batches above 8
+ * run the routed projections on the tensor cores (warp-level MMA, each
+ * expert's weights decoded once for all of its tokens) unless the layer was
+ * created with MOE_FLAG_NO_GROUPED; smaller ones on the streaming GEMV
+ * kernels.
  * y_routed: fp32 [B*k][H], row p = unweighted output of pair p's expert;
  * y_shared: fp32 [B][H] (ignored, may be NULL, when I_s = 0).
  * With MOE_FLAG_SIDE_STREAM the shared expert runs on the layer's side
