@@ -234,6 +234,22 @@ MOE_API moe_status_t moe_router_topk_noalloc(const void* router_w_em, const floa
                                              int n_experts, int top_k, const void* x, int B,
                                              const moe_routing* r, void* stream);
 
+/* Self-test of the failure paths (the decode-path pages have no counterpart;
+ * it exists so that tests can check, without faulting, trapping or hanging a
+ * GPU, that failures surface as status codes):
+ *   MOE_SELFTEST_WAIT_TIMEOUT: launches one small kernel on `stream` whose
+ *     bounded mbarrier wait -- the same wait the layer's kernels use -- runs
+ *     out (~0.5 ms: nothing ever arrives), synchronises `stream` and returns
+ *     the status the kernel recorded: MOE_ERR_TIMEOUT when the path works.
+ *     Allocates and frees a 4-byte device word.
+ *   MOE_SELFTEST_FAIL_NEXT_ALLOC: makes the next moe_layer_create in this
+ *     process fail its scratch allocation (returning MOE_ERR_OOM, nothing
+ *     leaked); returns MOE_OK.
+ * Any other value returns MOE_ERR_INVALID_ARG. */
+#define MOE_SELFTEST_WAIT_TIMEOUT 1
+#define MOE_SELFTEST_FAIL_NEXT_ALLOC 2
+MOE_API moe_status_t moe_selftest(int what, void* stream);
+
 /* Static description string of a status code. */
 MOE_API const char* moe_status_string(moe_status_t s);
 

@@ -30,8 +30,12 @@ MOE_FLAG_NO_GROUPED = 0x8
 EXPORTS = (
     "moe_layer_create", "moe_layer_destroy", "moe_router_topk", "moe_experts_mxfp4",
     "moe_combine_residual", "moe_layer_forward", "moe_layer_forward_host", "moe_layer_routing",
-    "moe_layer_last_device_error", "moe_layer_set_probe", "moe_router_topk_noalloc", "moe_status_string",
+    "moe_layer_last_device_error", "moe_layer_set_probe", "moe_router_topk_noalloc", "moe_selftest",
+    "moe_status_string",
 )
+
+MOE_SELFTEST_WAIT_TIMEOUT = 1
+MOE_SELFTEST_FAIL_NEXT_ALLOC = 2
 
 
 class MoEError(RuntimeError):
@@ -82,6 +86,7 @@ def load_library(path: str = LIB_PATH):
         "moe_layer_last_device_error": [vp],
         "moe_layer_set_probe": [vp, vp, vp],
         "moe_router_topk_noalloc": [vp, vp, i32, i32, i32, vp, i32, ctypes.POINTER(moe_routing), vp],
+        "moe_selftest": [i32, vp],
     }
     for name, args in sig.items():
         f = getattr(L, name)
@@ -183,3 +188,8 @@ def moe_router_topk_noalloc(router_w_em, router_bias, hidden: int, n_experts: in
     _check("moe_router_topk_noalloc", load_library().moe_router_topk_noalloc(
         _ptr(router_w_em), _ptr(router_bias), hidden, n_experts, top_k, _ptr(x), B, ctypes.byref(routing),
         _stream(stream)))
+
+
+def moe_selftest(what: int, stream=None) -> int:
+    """Failure-path self-test (see the header); returns the status code."""
+    return int(load_library().moe_selftest(int(what), _stream(stream)))

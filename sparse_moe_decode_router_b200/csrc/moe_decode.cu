@@ -4,6 +4,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cstdint>
 #include <cstring>
 #include <mutex>
@@ -502,9 +503,49 @@ moe_status_t check_call(const moe_layer* L, int B) {
   return MOE_OK;
 }
 
+// Failure-path self-test: a wait on an mbarrier that nothing will complete
+// (phase 0 of a fresh barrier) gives up after `limit` cycles and records the
+// timeout, exactly as the layer's kernels do.
+__global__ void selftest_wait_kernel(int* err, long long limit) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (!mbar_wait_bounded(&bar, 0u, limit) && threadIdx.x == 0) atomicExch(err, kErrTimeout);
+}
+
+std::atomic<bool> g_fail_next_alloc{false};  // MOE_SELFTEST_FAIL_NEXT_ALLOC
+
 }  // namespace
 
 extern "C" {
+
+moe_status_t moe_selftest(int what, void* stream) {
+  if (what == MOE_SELFTEST_FAIL_NEXT_ALLOC) {
+    g_fail_next_alloc.store(true);
+    return MOE_OK;
+  }
+  if (what != MOE_SELFTEST_WAIT_TIMEOUT) return MOE_ERR_INVALID_ARG;
+  cudaStream_t st = (cudaStream_t)stream;
+  int* d = nullptr;
+  if (cudaMalloc(&d, sizeof(int)) != cudaSuccess) {
+    cudaGetLastError();
+    return MOE_ERR_OOM;
+  }
+  int h = -1;
+  cudaError_t e = cudaMemsetAsync(d, 0, sizeof(int), st);
+  if (e == cudaSuccess) {
+    selftest_wait_kernel<<<1, 32, 0, st>>>(d, 1ll << 20);
+    e = cudaGetLastError();
+  }
+  if (e == cudaSuccess) e = cudaMemcpyAsync(&h, d, sizeof(int), cudaMemcpyDeviceToHost, st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  cudaFree(d);
+  if (e != cudaSuccess) return MOE_ERR_CUDA;
+  return h == kErrTimeout ? MOE_ERR_TIMEOUT : (h == 0 ? MOE_OK : MOE_ERR_CUDA);
+}
 
 const char* moe_status_string(moe_status_t s) {
   switch (s) {
@@ -615,7 +656,7 @@ moe_status_t moe_layer_create(const moe_layer_config* cfg, const moe_layer_weigh
   const size_t o_xs = take((size_t)MB * H * 2);
   const size_t o_rs = take((size_t)MB * H * 2);
   const size_t o_os = take((size_t)MB * H * 2);
-  if (cudaMalloc(&L->arena, off) != cudaSuccess) {
+  if (g_fail_next_alloc.exchange(false) || cudaMalloc(&L->arena, off) != cudaSuccess) {
     cudaGetLastError();
     delete L;
     return MOE_ERR_OOM;

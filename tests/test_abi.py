@@ -63,3 +63,11 @@ def test_host_side_argument_checks(lib):
     assert lib.moe_layer_destroy(None) == api.MOE_OK
     with pytest.raises(api.MoEError):
         api.moe_layer_forward(None, None, 0x1000, 0x1000, 0x1000, 1)
+
+
+def test_selftest_rejects_unknown_requests():
+    """Host-side argument check of the failure-path self-test (no CUDA call)."""
+    from sparse_moe_decode_router_b200 import api
+    api.load_library()
+    assert api.moe_selftest(0) == api.MOE_ERR_INVALID_ARG
+    assert api.moe_selftest(99) == api.MOE_ERR_INVALID_ARG
