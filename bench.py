@@ -364,7 +364,7 @@ def run_ours(args, cfg):
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5), "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "scaling": "weak", "vs_baseline": None, "dtype": "f16",
         "data": "synthetic (seeded Philox4x32-10 draws; random-init weights of the full-size layer)",
         "config": {"workload": workload_desc(cfg), "batch": B, "parallelism": f"replicas x{world}",
                    "l2": "flushed between steps (256 MiB write, outside the per-step CUDA events)",
