@@ -229,7 +229,13 @@ MOE_API moe_status_t moe_layer_set_probe(moe_layer_t layer, void* start, void* s
  * first call before any stream capture.  The counter is cleared on the
  * stream at the start of every call; the logits are overwritten.  All calls
  * on a device share the one array, so calls that overlap on the GPU (other
- * streams, other host threads) race: serialise them. */
+ * streams, other host threads) race: serialise them.
+ * Device-side errors: the router kernel's bounded waits and plan checks
+ * record a timeout or a bad plan in the array's error word, exactly as a
+ * layer's kernels record theirs, but no entry point reads that word back
+ * yet; a call whose wait gave up leaves its logits, and so the plan it
+ * writes, unspecified without reporting it.  (A layer reports the same
+ * condition through moe_layer_last_device_error.) */
 MOE_API moe_status_t moe_router_topk_noalloc(const void* router_w_em, const float* router_bias, int hidden,
                                              int n_experts, int top_k, const void* x, int B,
                                              const moe_routing* r, void* stream);
