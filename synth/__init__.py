@@ -85,6 +85,7 @@ T_SHARED_D = 5
 T_EXPERT_GU = 6
 T_EXPERT_D = 7
 T_ZIPF_PERM = 8
+T_TIES = 9
 
 # Irwin-Hall(4) of 16-bit uniforms: S = sum - 2*65535, Var(S) = 4*(65536^2-1)/12
 IH_SD = math.sqrt(4.0 * (65536.0 * 65536.0 - 1.0) / 12.0)
@@ -315,6 +316,44 @@ def gen_residual(cfg, token_ids, layer=0):
     key = stream_key(cfg.seed, layer, T_RESIDUAL)
     return np.stack([bf16_rne(normal_f32(key, int(t), 0, 0, cfg.hidden, cfg.act_sigma))
                      for t in token_ids])
+
+
+def gen_tied_router(cfg, n_copies=4, with_bias=True, layer=0):
+    """Router inputs whose logits tie exactly: bf16 Wr [H][E] with entries in
+    {-1, 0, 1}, where the E columns come in groups of n_copies identical
+    copies scattered over the expert ids (expert e belongs to group
+    perm[e] mod E/n_copies, perm a seeded permutation), and an fp32 bias in
+    {-2, ..., 2} per group, or None.  With integer activations every logit
+    is an integer of magnitude <= H + 2, exact in fp32 and fp64 whatever
+    the order of the sum.  Returns (router_w bits, bias, group)."""
+    E, H = cfg.n_experts, cfg.hidden
+    if E % n_copies:
+        raise ValueError("n_experts must be a multiple of n_copies")
+    G = E // n_copies
+    key = stream_key(cfg.seed, layer, T_TIES)
+    o0, o1, _, _ = philox4x32_10(np.arange(E, dtype=np.uint64), 0, 0, 0, *key)
+    perm = np.lexsort((np.arange(E), o0))
+    group = np.empty(E, dtype=np.int64)
+    group[perm] = np.arange(E) % G
+    c0, _, _, _ = philox4x32_10(np.arange(H * G, dtype=np.uint64), 1, 0, 0, *key)
+    base = (c0.astype(np.int64) % 3 - 1).reshape(H, G).astype(np.float32)
+    wr = bf16_rne(base[:, group])
+    bias = None
+    if with_bias:
+        bg = (o1[:G].astype(np.int64) % 5 - 2).astype(np.float32)
+        bias = bg[group]
+    return wr, bias, group
+
+
+def gen_tied_tokens(cfg, B, layer=0):
+    """bf16 activations [B][H] with entries in {-1, 0, 1} (token 0 all zero,
+    so its logits are the bias alone)."""
+    H = cfg.hidden
+    key = stream_key(cfg.seed, layer, T_TIES)
+    c0, _, _, _ = philox4x32_10(np.arange(B * H, dtype=np.uint64), 2, 0, 0, *key)
+    x = (c0.astype(np.int64) % 3 - 1).reshape(B, H).astype(np.float32)
+    x[0] = 0.0
+    return bf16_rne(x)
 
 
 def gen_host_layer(cfg, layer=0, experts=None):

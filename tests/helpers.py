@@ -27,6 +27,11 @@ Y_ROUTED_MEAN_REL = 2e-3
 # routing weights: fp32 softmax of fp32 logits vs fp64 (|w| <= 1)
 W_ABS = 1e-5
 
+# Exact-tie router workloads (synth.gen_tied_router): (n_experts, top_k,
+# copies per tied group).  They cover the top-k kernel's slice layouts: one,
+# four and four candidates per lane in the first stage.
+TIE_SHAPES = ((32, 4, 8), (896, 16, 4), (1024, 32, 4))
+
 
 def bf16_close(gpu_u16, ref_u16, max_rel=OUT_MAX_REL, mean_rel=OUT_MEAN_REL):
     g = bf16_to_f32(np.asarray(gpu_u16)).astype(np.float64)

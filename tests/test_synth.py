@@ -1,12 +1,13 @@
 """CPU checks of the seeded input generator (synth): Philox known answers,
 the Irwin-Hall draw, bf16 rounding, the MXFP4 quantiser and the routing-gap
-conditioning.  The device generator's bit-identity is checked in
-test_gpu_synth.py."""
+conditioning, and the exact-tie router inputs.  The device generator's
+bit-identity is checked in test_gpu_parity.py."""
 import numpy as np
 import pytest
 
 import oracle
 import synth
+from helpers import TIE_SHAPES
 
 
 def test_philox4x32_10_known_answers():
@@ -100,3 +101,28 @@ def test_counted_bytes_formula():
     # per active expert: codes + scales of gate/up and down
     assert c1.expert_bytes() == 2 * 2048 * (3584 + 224) + 7168 * (1024 + 64)
     assert c1.counted_bytes(16) == 16 * c1.expert_bytes() + 3 * 2048 * 7168 * 2 + 7168 * 896 * 2 + 3 * 7168 * 2
+
+
+@pytest.mark.parametrize("E,k,copies", TIE_SHAPES)
+@pytest.mark.parametrize("with_bias", [True, False])
+def test_tied_router_inputs_tie_at_the_selection_boundary(E, k, copies, with_bias):
+    """The premise of the GPU tie test: every logit is an integer (so fp32
+    and fp64 agree exactly), the copies of a group share every logit, and
+    among the first tokens some have equal k-th and (k+1)-th logits, so
+    their selected set depends on the tie rule."""
+    cfg = synth.CONFIGS[0].with_(n_experts=E, top_k=k)
+    wr, bias, group = synth.gen_tied_router(cfg, n_copies=copies, with_bias=with_bias)
+    assert np.bincount(group).tolist() == [copies] * (E // copies)
+    x = synth.gen_tied_tokens(cfg, 64)
+    assert set(np.unique(synth.bf16_to_f32(x))) <= {-1.0, 0.0, 1.0}
+    assert not np.any(synth.bf16_to_f32(x[0]))
+    lg = synth.bf16_to_f32(x).astype(np.float64) @ synth.bf16_to_f32(wr).astype(np.float64)
+    if bias is not None:
+        lg += bias
+    assert np.array_equal(lg, np.rint(lg)) and np.abs(lg).max() < 2.0 ** 24
+    for g in range(E // copies):      # copies of a group tie on every token
+        cols = lg[:, group == g]
+        assert np.all(cols == cols[:, :1])
+    srt = -np.sort(-lg, axis=1)
+    boundary = srt[:, k - 1] == srt[:, k]
+    assert boundary[:7].any() and boundary.sum() >= 4
