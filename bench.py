@@ -2,8 +2,8 @@
 """Benchmark of the sparse MXFP4 MoE decode layer (libmoe_decode.so) on B200.
 
 One step = one moe_layer_forward of the workload (router GEMV + top-k +
-bucketing, routed MXFP4 SwiGLU experts, shared expert on the side stream,
-down projection fused with the combine and residual add) on one batch of
+bucketing, routed MXFP4 SwiGLU experts, the shared expert, down projection
+fused with the combine and residual add) on one batch of
 seeded synthetic tokens; a pool of distinct tokens makes every step route to
 a different expert set.  Weights and inputs are resident in HBM before the
 timed region; L2 is flushed (256 MiB write) between steps, outside the
@@ -61,40 +61,104 @@ def workload_desc(cfg):
 
 
 # ---------------------------------------------------------------- clocks ----
-class ClockSampler:
-    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+def _load_nvml():
+    import pynvml
+    return pynvml
 
-    def __init__(self, gpu_index):
+
+class ClockSampler:
+    """SM clock and clock-event (throttle) reasons while the timed regions run.
+
+    NVML, read in-process by a thread every 5 ms (reading only: no setting is
+    changed); only samples taken between begin() and end() count.  If NVML
+    cannot be used, nvidia-smi's 50 ms loop instead, started before the
+    warm-up and waited for, so that it is already sampling when timing
+    starts."""
+    PERIOD_S = 0.005
+    REASON_BITS = (("hw_slowdown", 0x8), ("hw_thermal_slowdown", 0x40), ("sw_thermal_slowdown", 0x20),
+                   ("sw_power_cap", 0x4))
+    SMI_FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+                  "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+                  "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index, uuid=None):
         self.gpu = gpu_index
+        self.uuid = uuid
+        self.nv = None
         self.proc = None
         self.lines = []
+        self.samples = []       # (perf_counter, sm MHz, reason bits)
+        self.windows = []       # (begin, end) of the timed regions
+        self._open = None
+        self._halt = threading.Event()
 
-    def start(self):
+    # -- NVML --------------------------------------------------------------
+    def _nvml_start(self):
+        nv = _load_nvml()
+        nv.nvmlInit()
+        try:
+            h = None
+            if self.uuid:
+                u = self.uuid if self.uuid.startswith("GPU-") else "GPU-" + self.uuid
+                try:
+                    h = nv.nvmlDeviceGetHandleByUUID(u)
+                except Exception:
+                    h = None
+            if h is None:
+                h = nv.nvmlDeviceGetHandleByIndex(self.gpu)
+            try:
+                nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+                reasons = nv.nvmlDeviceGetCurrentClocksEventReasons
+            except Exception:
+                reasons = nv.nvmlDeviceGetCurrentClocksThrottleReasons
+            self.max_mhz = float(nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM))
+            self._read = lambda: (time.perf_counter(), float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)),
+                                  int(reasons(h)))
+            self.samples.append(self._read())     # a failing read fails here, not in the thread
+        except Exception:
+            try:
+                nv.nvmlShutdown()
+            except Exception:
+                pass
+            raise
+        self.nv = nv
+        self.thread = threading.Thread(target=self._poll, daemon=True)
+        self.thread.start()
+
+    def _poll(self):
+        while not self._halt.wait(self.PERIOD_S):
+            try:
+                self.samples.append(self._read())
+            except Exception:
+                return
+
+    # -- nvidia-smi ----------------------------------------------------------
+    def _smi_start(self):
         try:
             self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.SMI_FIELDS}", "--format=csv,noheader,nounits",
                  "-lms", "50"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            self.thread = threading.Thread(target=self._read, daemon=True)
-            self.thread.start()
         except OSError:
             self.proc = None
+            return
+        self.thread = threading.Thread(target=self._smi_read, daemon=True)
+        self.thread.start()
+        t0 = time.perf_counter()
+        while not self.lines and self.proc.poll() is None and time.perf_counter() - t0 < 3.0:
+            time.sleep(0.01)
 
-    def _read(self):
+    def _smi_read(self):
         for line in self.proc.stdout:
             self.lines.append(line.strip())
 
-    def stop(self):
-        if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+    def _smi_stop(self):
         self.proc.terminate()
         try:
             self.proc.wait(timeout=5)
         except subprocess.TimeoutExpired:
             self.proc.kill()
         sm, mx, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        names = [n for n, _ in self.REASON_BITS]
         for ln in self.lines:
             parts = [p.strip() for p in ln.split(",")]
             if len(parts) < 8:
@@ -108,7 +172,44 @@ class ClockSampler:
                 if v.lower() == "active":
                     reasons.add(n)
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
-                "reasons": sorted(reasons), "samples": len(sm)}
+                "reasons": sorted(reasons), "samples": len(sm), "source": "nvidia-smi, 50 ms, whole run"}
+
+    # -- public ----------------------------------------------------------------
+    def start(self):
+        try:
+            self._nvml_start()
+        except Exception:
+            self.nv = None
+            self._smi_start()
+
+    def begin(self):
+        self._open = time.perf_counter()
+
+    def end(self):
+        if self._open is not None:
+            self.windows.append((self._open, time.perf_counter()))
+            self._open = None
+
+    def stop(self):
+        if self.nv is not None:
+            self._halt.set()
+            self.thread.join(timeout=2.0)
+            try:
+                self.nv.nvmlShutdown()
+            except Exception:
+                pass
+            inside = [s for s in self.samples if any(a <= s[0] <= b for a, b in self.windows)]
+            bits = 0
+            for s in inside:
+                bits |= s[2]
+            return {"sm_mhz": statistics.median(s[1] for s in inside) if inside else None,
+                    "sm_max_mhz": self.max_mhz,
+                    "reasons": sorted(n for n, b in self.REASON_BITS if bits & b),
+                    "samples": len(inside), "source": "NVML, 5 ms, timed regions only"}
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no clock source (NVML and nvidia-smi unavailable)"],
+                    "samples": 0}
+        return self._smi_stop()
 
 
 # ------------------------------------------------------------- helpers ------
@@ -302,7 +403,11 @@ def run_ours(args, cfg):
         na = n_active[i % POOL]
         return na * 2 * cfg.inter * (H // 2 + H // 32) + B * H * 2 + B * k * cfg.inter * 4
 
-    sampler = ClockSampler(local)
+    try:
+        uuid = str(torch.cuda.get_device_properties(local).uuid)
+    except Exception:
+        uuid = None
+    sampler = ClockSampler(local, uuid)
     sampler.start()
     for i in range(args.warmup):
         flush.zero_()
@@ -316,6 +421,7 @@ def run_ours(args, cfg):
     if dist is not None:
         dist.barrier()
     torch.cuda.synchronize()
+    sampler.begin()
     for i in range(K):
         flush.zero_()
         api.moe_layer_set_probe(handle, pr[i][0], pr[i][1])
@@ -323,6 +429,7 @@ def run_ours(args, cfg):
         api.moe_layer_forward(handle, None, pool_x[i % POOL], pool_r[i % POOL], out, B, stream)
         ev[i][1].record(stream)
     torch.cuda.synchronize()
+    sampler.end()
     if dist is not None:
         dist.barrier()
     api.moe_layer_set_probe(handle, None, None)
@@ -332,12 +439,14 @@ def run_ours(args, cfg):
     # end to end through the host-buffer entry point (pinned host memory)
     e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
     torch.cuda.synchronize()
+    sampler.begin()
     for i in range(K):
         flush.zero_()
         e2e_ev[i][0].record(stream)
         api.moe_layer_forward_host(handle, pool_xh[i % POOL], pool_rh[i % POOL], out_h, B, stream)
         e2e_ev[i][1].record(stream)
     torch.cuda.synchronize()
+    sampler.end()
     clocks = sampler.stop()
     e2e_ms = [a.elapsed_time(b) for a, b in e2e_ev]
     if api.moe_layer_last_device_error(handle) != api.MOE_OK:
@@ -381,12 +490,27 @@ def run_ours(args, cfg):
         "e2e": {"value": round(world * total_bytes / (e2e_total * 1e-3) / 1e9, 2), "unit": UNIT,
                 "h2d_bytes_per_step": 2 * B * H * 2, "d2h_bytes_per_step": B * H * 2,
                 "us_per_step": round(e2e_total / K * 1e3, 2)},
-        "gpu_launches": 6 * K,  # router, top-k, gate/up, down+combine, shared gate/up, shared down
+        "gpu_launches": launches_per_step(cfg, args.flags) * K,
         "clocks": clocks,
     }
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(cfg, dl)
     print(json.dumps(line), flush=True)
+
+
+def launches_per_step(cfg, flags):
+    """Kernels of this library one moe_layer_forward launches: router GEMV and
+    top-k; the shared expert's gate/up and down; then, for batches of one to
+    eight (or with the grouped path off), routed gate/up and down+combine;
+    above eight, the grouped tensor-core path: an activation-staging kernel
+    and a grouped MMA kernel per projection, then the combine.  The grouped
+    path is taken when both reduction lengths are multiples of 256 (the
+    full-size and test shapes)."""
+    from sparse_moe_decode_router_b200.api import MOE_FLAG_NO_GROUPED
+    n = 2 + (2 if cfg.shared_inter > 0 else 0)
+    grouped = (cfg.batch > 8 and not (flags & MOE_FLAG_NO_GROUPED) and cfg.hidden % 256 == 0
+               and cfg.inter % 256 == 0)
+    return n + (5 if grouped else 2)
 
 
 def cpu_baseline(cfg, dl):
@@ -398,7 +522,7 @@ def cpu_baseline(cfg, dl):
     B = cfg.batch
     shared = dl.host_shared()
     spent, n, nbytes = 0.0, 0, 0
-    while n < 1 or (spent < 10.0 and n < 8):
+    while n < 1 or (spent < 10.0 and n < 64):
         ids = [((n % POOL) * B) + b for b in range(B)]
         x_h, _ = dl.tokens(ids)
         r_h, _ = residual_tokens(cfg, ids)
