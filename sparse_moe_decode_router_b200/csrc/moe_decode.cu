@@ -7,8 +7,10 @@
 #include <atomic>
 #include <cstdint>
 #include <cstring>
+#include <map>
 #include <mutex>
 #include <new>
+#include <utility>
 
 #include "../../include/moe_decode.h"
 #include "gemv.cuh"
@@ -191,6 +193,25 @@ GemvFn gemv_fn(Kind k, int tmax, bool fast = false, bool small = false) {
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// The dynamic shared-memory limit of a kernel instance is a per-device
+// property shared by every layer (and the allocation-free router): it is
+// raised to what a plan needs and never lowered, so that creating a layer
+// whose plans need less cannot make the launches of an earlier layer fail.
+std::mutex g_smem_mu;
+std::map<std::pair<int, const void*>, int> g_smem_limit;
+
+cudaError_t raise_smem_limit(const void* fn, int bytes) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(g_smem_mu);
+  int& cur = g_smem_limit[std::make_pair(dev, fn)];
+  if (bytes <= cur) return cudaSuccess;
+  e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess) cur = bytes;
+  return e;
+}
 
 }  // namespace
 
@@ -712,9 +733,8 @@ moe_status_t moe_layer_create(const moe_layer_config* cfg, const moe_layer_weigh
     if (ok && (I % (kMmaRows / 2)) == 0 && (H % kMmaRows) == 0) L->grouped = true;
   }
   if (e == cudaSuccess && L->grouped) {
-    e = cudaFuncSetAttribute(grouped_mma_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBudget);
-    if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(grouped_mma_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBudget);
+    e = raise_smem_limit(reinterpret_cast<const void*>(grouped_mma_kernel<true>), kSmemBudget);
+    if (e == cudaSuccess) e = raise_smem_limit(reinterpret_cast<const void*>(grouped_mma_kernel<false>), kSmemBudget);
   }
   const void* small_kernels[] = {reinterpret_cast<const void*>(topk_bucket_kernel),
                                  reinterpret_cast<const void*>(act_to_f16_kernel<false>),
@@ -727,8 +747,7 @@ moe_status_t moe_layer_create(const moe_layer_config* cfg, const moe_layer_weigh
     for (int t = 0; t < 3 && e == cudaSuccess; ++t) {
       const GemvPlan& p = L->plans[kk][t];
       if (!p.ok) continue;
-      e = cudaFuncSetAttribute(gemv_fn((Kind)kk, tmax_of_slot(t), p.fast, t == 2), cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               p.smem);
+      e = raise_smem_limit(reinterpret_cast<const void*>(gemv_fn((Kind)kk, tmax_of_slot(t), p.fast, t == 2)), p.smem);
     }
   if (e == cudaSuccess) e = cudaDeviceSynchronize();
   if (e != cudaSuccess) {
@@ -887,10 +906,8 @@ moe_status_t moe_router_topk_noalloc(const void* router_w_em, const float* route
         if (!p.ok) return MOE_ERR_UNSUPPORTED;
       }
       // the largest dynamic shared memory any router plan asks for
-      if (cudaFuncSetAttribute(gemv_fn(K_ROUTER, 1), cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBudget) !=
-              cudaSuccess ||
-          cudaFuncSetAttribute(gemv_fn(K_ROUTER, 2), cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBudget) !=
-              cudaSuccess)
+      if (raise_smem_limit(reinterpret_cast<const void*>(gemv_fn(K_ROUTER, 1)), kSmemBudget) != cudaSuccess ||
+          raise_smem_limit(reinterpret_cast<const void*>(gemv_fn(K_ROUTER, 2)), kSmemBudget) != cudaSuccess)
         return MOE_ERR_CUDA;
       g_noalloc_ptr[dev] = ptr;
     }

@@ -149,6 +149,36 @@ def test_tiny_flags_give_identical_results(torch_cuda, tiny, flags):
     assert np.array_equal(base["y"], other["y"])
 
 
+def test_layers_of_different_shapes_coexist(torch_cuda, tiny):
+    """Kernel instances are shared by every layer in the process: creating a
+    layer whose plans need less shared memory must not break the launches of
+    a larger layer created before it."""
+    from sparse_moe_decode_router_b200 import api
+    torch = torch_cuda
+    base = synth.CONFIGS[0]
+    big = make_device_layer(base.with_(hidden=512, inter=256, shared_inter=64))
+    hb = create_layer(big, 8)
+    hs = create_layer(tiny, 8)
+    try:
+        for dl, h in ((big, hb), (tiny, hs), (big, hb)):
+            c = dl.cfg
+            for B in (1, 5):
+                ids = list(range(B))
+                x_h, x_d = dl.tokens(ids)
+                r_h, r_d = residual_tokens(c, ids, dl.layer)
+                out = torch.empty((B, c.hidden), dtype=torch.bfloat16, device="cuda")
+                api.moe_layer_forward(h, None, x_d, r_d, out, B)
+                torch.cuda.synchronize()
+                assert api.moe_layer_last_device_error(h) == api.MOE_OK
+                ref = oracle_layer_for(dl, x_h, r_h)
+                assert_routing_equal(layer_routing_host(h, B, c.top_k, c.n_experts), ref, W_ABS)
+                ok, info = bf16_close(to_host_u16(out), ref["out_bf16"])
+                assert ok, (c.hidden, B, info)
+    finally:
+        api.moe_layer_destroy(hs)
+        api.moe_layer_destroy(hb)
+
+
 def test_invalid_calls_are_rejected(torch_cuda, tiny):
     from sparse_moe_decode_router_b200 import api
     torch = torch_cuda
