@@ -37,6 +37,11 @@
  *    stream).  Calls only enqueue work: they never synchronise, allocate or
  *    free, so they may be captured into a CUDA graph (moe_layer_create and
  *    moe_layer_destroy excepted).
+ *  - A call on a layer must be made with the layer's device current (the
+ *    device that was current at moe_layer_create); otherwise it returns
+ *    MOE_ERR_INVALID_ARG and launches nothing.  moe_layer_destroy and
+ *    moe_layer_last_device_error make the layer's device current themselves
+ *    and restore the caller's.
  *  - Errors are returned, never raised: invalid arguments are rejected on the
  *    host with MOE_ERR_INVALID_ARG before anything is launched; a failed
  *    launch returns MOE_ERR_CUDA.  Device-side waits are bounded; a wait that
@@ -172,7 +177,8 @@ MOE_API moe_status_t moe_combine_residual(moe_layer_t layer, int B, const moe_ro
  * (MOE_FLAG_SIDE_STREAM forks it onto a side stream instead);
  * with `next` non-NULL the tail of this layer prefetches next's router and
  * shared-expert weights into L2 (pages: yeyulingfeng section 02, third and
- * fourth optimisations).  x, residual, out: bf16 [B][H]; out may equal
+ * fourth optimisations); `next` must live on the same device (else
+ * MOE_ERR_INVALID_ARG).  x, residual, out: bf16 [B][H]; out may equal
  * residual.  The routing plan is left in the layer's buffers. */
 MOE_API moe_status_t moe_layer_forward(moe_layer_t layer, moe_layer_t next, const void* x,
                                const void* residual, void* out, int B, void* stream);
@@ -190,9 +196,11 @@ MOE_API moe_status_t moe_layer_forward_host(moe_layer_t layer, const void* x_hos
  * the layer, valid until destroy). */
 MOE_API moe_status_t moe_layer_routing(moe_layer_t layer, moe_routing* out);
 
-/* Reads (synchronously) and clears the layer's device error word: MOE_OK,
- * or MOE_ERR_TIMEOUT if a bounded device-side wait gave up since the last
- * call. */
+/* Waits for all work on the layer's device (every stream), then reads and
+ * clears the layer's device error word: MOE_OK, MOE_ERR_TIMEOUT if a bounded
+ * device-side wait gave up since the last call, or MOE_ERR_INVALID_ARG if a
+ * kernel found a routing plan inconsistent with the layer.  Synchronous: not
+ * during stream capture. */
 MOE_API moe_status_t moe_layer_last_device_error(moe_layer_t layer);
 
 /* Timing probe: when start/stop (cudaEvent_t as void*) are non-NULL,

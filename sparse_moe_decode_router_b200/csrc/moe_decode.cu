@@ -521,8 +521,28 @@ cudaError_t launch_combine(moe_layer* L, int B, const moe_routing& r, const floa
 moe_status_t check_call(const moe_layer* L, int B) {
   if (!L) return MOE_ERR_INVALID_ARG;
   if (B < 1 || B > L->cfg.max_batch) return MOE_ERR_INVALID_ARG;
+  // the layer's pointers belong to the device current at its creation
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev != L->device) return MOE_ERR_INVALID_ARG;
   return MOE_OK;
 }
+
+// Makes a layer's device current for a call that may come with another
+// device current (destroy, the error readout) and restores the caller's.
+struct DeviceGuard {
+  int prev = -1;
+  bool ok = false;
+  explicit DeviceGuard(int dev) {
+    if (cudaGetDevice(&prev) != cudaSuccess) {
+      prev = -1;
+      return;
+    }
+    ok = prev == dev || cudaSetDevice(dev) == cudaSuccess;
+  }
+  ~DeviceGuard() {
+    if (ok && prev >= 0) cudaSetDevice(prev);
+  }
+};
 
 // Failure-path self-test: a wait on an mbarrier that nothing will complete
 // (phase 0 of a fresh barrier) gives up after `limit` cycles and records the
@@ -760,6 +780,7 @@ moe_status_t moe_layer_create(const moe_layer_config* cfg, const moe_layer_weigh
 
 moe_status_t moe_layer_destroy(moe_layer_t L) {
   if (!L) return MOE_OK;
+  DeviceGuard guard(L->device);
   if (L->side) cudaStreamSynchronize(L->side);
   cudaDeviceSynchronize();
   if (L->ev_fork) cudaEventDestroy(L->ev_fork);
@@ -827,6 +848,7 @@ moe_status_t moe_layer_forward(moe_layer_t L, moe_layer_t next, const void* x, c
   if (s != MOE_OK) return s;
   if (!x || !residual || !out || !aligned16(x) || !aligned16(residual) || !aligned16(out))
     return MOE_ERR_INVALID_ARG;
+  if (next && next->device != L->device) return MOE_ERR_INVALID_ARG;  // prefetch reads local memory only
   cudaStream_t st = (cudaStream_t)stream;
   const bool has_shared = L->cfg.shared_inter > 0;
   const bool fork = has_shared && L->side_stream;
@@ -867,13 +889,21 @@ moe_status_t moe_layer_forward_host(moe_layer_t L, const void* x_host, const voi
 
 moe_status_t moe_layer_last_device_error(moe_layer_t L) {
   if (!L) return MOE_ERR_INVALID_ARG;
+  DeviceGuard guard(L->device);
+  if (!guard.ok) return MOE_ERR_CUDA;
+  // the layer may run on a non-blocking stream, which a copy on the legacy
+  // stream would not wait for: wait for all of the device's work first
+  if (cudaDeviceSynchronize() != cudaSuccess) return MOE_ERR_CUDA;
   int v = 0;
   if (cudaMemcpy(&v, L->err, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return MOE_ERR_CUDA;
   if (v == 0) return MOE_OK;
-  // clear the word and the completion counters a cut-short launch may have left behind
-  cudaMemset(L->err, 0, sizeof(int));
-  cudaMemset(L->router_cnt, 0, sizeof(int));
-  cudaMemset(L->tile_cnt, 0, sizeof(int) * L->cfg.hidden);
+  // clear the word and the completion counters a cut-short launch may have
+  // left behind, and finish before the caller's next launch on any stream
+  cudaError_t e = cudaMemset(L->err, 0, sizeof(int));
+  if (e == cudaSuccess) e = cudaMemset(L->router_cnt, 0, sizeof(int));
+  if (e == cudaSuccess) e = cudaMemset(L->tile_cnt, 0, sizeof(int) * L->cfg.hidden);
+  if (e == cudaSuccess) e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) return MOE_ERR_CUDA;
   return v == kErrTimeout ? MOE_ERR_TIMEOUT : MOE_ERR_INVALID_ARG;
 }
 
