@@ -238,15 +238,21 @@ MOE_API moe_status_t moe_layer_set_probe(moe_layer_t layer, void* start, void* s
  * stream at the start of every call; the logits are overwritten.  All calls
  * on a device share the one array, so calls that overlap on the GPU (other
  * streams, other host threads) race: serialise them.
- * Device-side errors: the router kernel's bounded waits and plan checks
- * record a timeout or a bad plan in the array's error word, exactly as a
- * layer's kernels record theirs, but no entry point reads that word back
- * yet; a call whose wait gave up leaves its logits, and so the plan it
- * writes, unspecified without reporting it.  (A layer reports the same
- * condition through moe_layer_last_device_error.) */
+ * Device-side errors: the kernels' bounded waits and plan checks record a
+ * timeout or a bad plan in the array's error word, read and cleared by
+ * moe_router_topk_noalloc_last_error; a call whose wait gave up leaves its
+ * plan unspecified. */
 MOE_API moe_status_t moe_router_topk_noalloc(const void* router_w_em, const float* router_bias, int hidden,
                                              int n_experts, int top_k, const void* x, int B,
                                              const moe_routing* r, void* stream);
+
+/* Waits for all work on the current device, then reads and clears the
+ * allocation-free router's error word of this device: MOE_OK (also when no
+ * allocation-free call has been made on it), MOE_ERR_TIMEOUT if a bounded
+ * device-side wait of one of its calls gave up since the last readout, or
+ * MOE_ERR_INVALID_ARG if a kernel found its plan inconsistent.  Synchronous:
+ * not during stream capture. */
+MOE_API moe_status_t moe_router_topk_noalloc_last_error(void);
 
 /* Self-test of the failure paths (the decode-path pages have no counterpart;
  * it exists so that tests can check, without faulting, trapping or hanging a

@@ -30,7 +30,8 @@ MOE_FLAG_NO_GROUPED = 0x8
 EXPORTS = (
     "moe_layer_create", "moe_layer_destroy", "moe_router_topk", "moe_experts_mxfp4",
     "moe_combine_residual", "moe_layer_forward", "moe_layer_forward_host", "moe_layer_routing",
-    "moe_layer_last_device_error", "moe_layer_set_probe", "moe_router_topk_noalloc", "moe_selftest",
+    "moe_layer_last_device_error", "moe_layer_set_probe", "moe_router_topk_noalloc",
+    "moe_router_topk_noalloc_last_error", "moe_selftest",
     "moe_status_string",
 )
 
@@ -86,6 +87,7 @@ def load_library(path: str = LIB_PATH):
         "moe_layer_last_device_error": [vp],
         "moe_layer_set_probe": [vp, vp, vp],
         "moe_router_topk_noalloc": [vp, vp, i32, i32, i32, vp, i32, ctypes.POINTER(moe_routing), vp],
+        "moe_router_topk_noalloc_last_error": [],
         "moe_selftest": [i32, vp],
     }
     for name, args in sig.items():
@@ -188,6 +190,12 @@ def moe_router_topk_noalloc(router_w_em, router_bias, hidden: int, n_experts: in
     _check("moe_router_topk_noalloc", load_library().moe_router_topk_noalloc(
         _ptr(router_w_em), _ptr(router_bias), hidden, n_experts, top_k, _ptr(x), B, ctypes.byref(routing),
         _stream(stream)))
+
+
+def moe_router_topk_noalloc_last_error() -> int:
+    """Reads and clears the allocation-free router's device error word of the
+    current device (see the header); returns the status code."""
+    return int(load_library().moe_router_topk_noalloc_last_error())
 
 
 def moe_selftest(what: int, stream=None) -> int:

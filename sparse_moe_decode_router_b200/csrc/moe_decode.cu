@@ -992,6 +992,26 @@ moe_status_t moe_router_topk_noalloc(const void* router_w_em, const float* route
   return cuda_status(launch_ex(topk_bucket_kernel, B, kTopkWarps * 32, 0, st, true, t));
 }
 
+moe_status_t moe_router_topk_noalloc_last_error(void) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
+  if (dev < 0 || dev >= kNoAllocMaxDevices) return MOE_ERR_UNSUPPORTED;
+  void* base = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    base = g_noalloc_ptr[dev];
+  }
+  if (!base) return MOE_OK;  // no allocation-free call on this device yet
+  // the calls may run on non-blocking streams: wait for all of the device's work
+  if (cudaDeviceSynchronize() != cudaSuccess) return MOE_ERR_CUDA;
+  int* err = &static_cast<NoAllocScratch*>(base)->err;
+  int v = 0;
+  if (cudaMemcpy(&v, err, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return MOE_ERR_CUDA;
+  if (v == 0) return MOE_OK;
+  if (cudaMemset(err, 0, sizeof(int)) != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess) return MOE_ERR_CUDA;
+  return v == kErrTimeout ? MOE_ERR_TIMEOUT : MOE_ERR_INVALID_ARG;
+}
+
 moe_status_t moe_layer_set_probe(moe_layer_t L, void* start, void* stop) {
   if (!L || ((start == nullptr) != (stop == nullptr))) return MOE_ERR_INVALID_ARG;
   L->probe_start = (cudaEvent_t)start;

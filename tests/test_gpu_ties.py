@@ -52,6 +52,7 @@ def test_equal_logits_go_to_the_lower_expert_id(E, k, copies, with_bias):
             api.moe_router_topk_noalloc(w_em, bias_d, cfg.hidden, E, k, x_d, B, routing_struct(got_na))
             torch.cuda.synchronize()
             assert api.moe_layer_last_device_error(h) == api.MOE_OK
+            assert api.moe_router_topk_noalloc_last_error() == api.MOE_OK
             assert_routing_equal(routing_host(got), ref, W_ABS)
             assert_routing_equal(routing_host(got_na), ref, W_ABS)
     finally:

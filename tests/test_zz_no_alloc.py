@@ -35,6 +35,7 @@ def test_noalloc_router_matches_layer_router_twice():
             got = routing_buffers(B, k, E)
             api.moe_router_topk_noalloc(w_em, dl.router_bias, H, E, k, x, B, routing_struct(got))
             torch.cuda.synchronize()
+            assert api.moe_router_topk_noalloc_last_error() == api.MOE_OK
             g, w = routing_host(got), routing_host(want)
             for key in ("topk_idx", "counts", "offsets", "pair_ids", "active"):
                 assert np.array_equal(g[key], w[key]), (call, key)
