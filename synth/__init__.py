@@ -36,7 +36,7 @@ from __future__ import annotations
 import ctypes
 import math
 import os
-from dataclasses import dataclass, field, replace
+from dataclasses import dataclass, replace
 
 import numpy as np
 

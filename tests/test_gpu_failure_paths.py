@@ -2,7 +2,6 @@
 hanging the GPU: a device-side wait that runs out is reported as
 MOE_ERR_TIMEOUT and leaves the context usable; a failed scratch allocation
 makes moe_layer_create return MOE_ERR_OOM and leaks nothing."""
-import numpy as np
 import pytest
 
 import synth

@@ -9,7 +9,7 @@ import pytest
 
 import oracle
 import synth
-from helpers import W_ABS, bf16_close
+from helpers import bf16_close
 from gpu_common import create_layer, make_device_layer, oracle_threads, residual_tokens, to_host_u16
 
 pytestmark = pytest.mark.gpu
