@@ -4,7 +4,14 @@ exactly those roundings (f16 activations scaled by a power of two, f16 products
 and eight-term f16 partial sums per 32-element block, fp32 across blocks, h
 rounded to f16 before the down projection) in numpy to one expert of a
 medium-size layer, and checks the resulting error against the fp64 oracle.
-It uses no GPU code; the oracle supplies the reference."""
+It uses no GPU code; the oracle supplies the reference.
+
+A second derivation concerns activations given to block-scaled tensor-core
+MMAs as MX types (E4M3 elements, one E8M0 scale per 32): one E4M3 term per
+activation breaks the routed-output bounds, while two terms (the value, then
+its residual, each with its own scale) fit them with margin, provided the
+scale keeps the block maximum within E4M3's range (448) rather than clipping
+it."""
 import numpy as np
 
 import oracle
@@ -73,3 +80,89 @@ def test_f16_block_partial_sums_fit_the_stated_bounds():
     out_r = synth.bf16_to_f32(synth.bf16_rne((w @ yr).astype(np.float32))).astype(np.float64)
     ok, info = metric_close(out_g, out_r, OUT_MAX_REL, OUT_MEAN_REL)
     assert ok, info
+
+
+def _e4m3_positive():
+    """Non-negative E4M3 values by code 0..126 (OCP FP8: bias 7, 3 mantissa
+    bits, subnormals at exponent 0, code 127 is NaN): value and code."""
+    codes = np.arange(127)
+    e, m = codes >> 3, codes & 7
+    vals = np.where(e == 0, m / 8.0 * 2.0 ** -6, (1 + m / 8.0) * 2.0 ** (e - 7.0))
+    return vals, codes
+
+
+def _q_e4m3(x):
+    """Round to the nearest E4M3 value, ties to the even code; saturate at 448."""
+    vals, codes = _e4m3_positive()
+    a = np.minimum(np.abs(x), vals[-1])
+    i = np.clip(np.searchsorted(vals, a), 1, len(vals) - 1)
+    lo, hi = vals[i - 1], vals[i]
+    dl, dh = a - lo, hi - a
+    pick_hi = (dh < dl) | ((dh == dl) & (codes[i] % 2 == 0))
+    return np.sign(x) * np.where(pick_hi, hi, lo)
+
+
+def _mx_e4m3(x, clip_scale):
+    """One MX term: per 32 elements an E8M0 scale 2^e and E4M3 elements.
+    clip_scale: e = floor(log2 amax) - 8 (the block maximum lands in [256,
+    512) and is clipped to 448); otherwise e = ceil(log2(amax / 448))."""
+    xb = x.reshape(-1, 32)
+    amax = np.abs(xb).max(1, keepdims=True)
+    safe = np.where(amax > 0, amax, 1.0)
+    e = np.floor(np.log2(safe)) - 8 if clip_scale else np.ceil(np.log2(safe / 448.0))
+    e = np.where(amax > 0, e, 0.0)
+    return (_q_e4m3(xb / 2.0 ** e) * 2.0 ** e).reshape(x.shape)
+
+
+def _mx_terms(x, n, clip_scale=False):
+    out, r = np.zeros_like(x), x.copy()
+    for _ in range(n):
+        t = _mx_e4m3(r, clip_scale)
+        out, r = out + t, r - t
+    return out
+
+
+def _dequant(codes, scales):
+    R, K = codes.shape[0], codes.shape[1] * 2
+    w = np.empty((R, K))
+    w[:, 0::2] = _E2M1[codes & 15]
+    w[:, 1::2] = _E2M1[codes >> 4]
+    return w * np.repeat(2.0 ** (scales.astype(np.float64) - 127), 32, axis=1)
+
+
+def test_e4m3_grid_pins():
+    vals, _ = _e4m3_positive()
+    assert vals[-1] == 448.0 and vals[1] == 2.0 ** -9 and vals[8] == 2.0 ** -6
+    assert _q_e4m3(np.array([1000.0, -1000.0]))[0] == 448.0
+    # 1 + 1/16 lies halfway between 1 (code 56, even) and 1.125 (code 57): even wins
+    assert _q_e4m3(np.array([1.0625, 1.1875]))[0] == 1.0
+    assert _q_e4m3(np.array([1.1875]))[0] == 1.25          # halfway 1.125 / 1.25: code 58 is even
+
+
+def test_mx_activation_terms_against_the_routed_bounds():
+    cfg = synth.CONFIGS[0].with_(hidden=2048, inter=1024, shared_inter=0, n_experts=8, top_k=2,
+                                 seed=synth.CONFIGS[0].seed + 900)
+    wr = synth.gen_router_w(cfg)
+    x_bf, _ = synth.gen_tokens(cfg, wr, None, [0])
+    x = synth.bf16_to_f32(x_bf[0]).astype(np.float64)
+    I = cfg.inter
+    experts = [synth.gen_expert(cfg, e) for e in range(2)]
+    refs = np.stack([oracle.expert_ffn(x, *ex)[1] for ex in experts])
+
+    def routed(n, clip_scale=False):
+        ys = []
+        for gc, gs, dc, ds in experts:
+            gu = _dequant(gc, gs) @ _mx_terms(x, n, clip_scale)
+            g, u = gu[:I], gu[I:]
+            h = g / (1 + np.exp(-g)) * u
+            ys.append(_dequant(dc, ds) @ _mx_terms(h, n, clip_scale))
+        return metric_close(np.stack(ys), refs, Y_ROUTED_MAX_REL, Y_ROUTED_MEAN_REL)
+
+    ok1, one = routed(1)
+    assert not ok1 and one["mean_rel"] > 10 * Y_ROUTED_MEAN_REL, one
+    ok2, two = routed(2)
+    assert ok2 and two["mean_rel"] < Y_ROUTED_MEAN_REL / 2, two
+    assert two["max_abs"] < Y_ROUTED_MAX_REL / 2 * two["max_ref"], two
+    # clipping the block maximum at 448 costs most of that margin
+    okc, clip = routed(2, clip_scale=True)
+    assert clip["mean_rel"] > 1.5 * two["mean_rel"], (clip, two)
