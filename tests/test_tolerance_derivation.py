@@ -6,7 +6,13 @@ rounded to f16 before the down projection) in numpy to one expert of a
 medium-size layer, and checks the resulting error against the fp64 oracle.
 It uses no GPU code; the oracle supplies the reference.
 
-A second derivation concerns activations given to block-scaled tensor-core
+A second derivation does the same for the grouped tensor-core kernels
+(batches above eight): activation rows scaled by a power of two so that
+their maximum lies in [2^14, 2^15) and rounded once to f16, exact products
+summed in fp32 per 32-element block, the block's E8M0 scale applied in
+fp32, h rounded to f16 the same way before the down projection.
+
+A third derivation concerns activations given to block-scaled tensor-core
 MMAs as MX types (E4M3 elements, one E8M0 scale per 32): one E4M3 term per
 activation breaks the routed-output bounds, while two terms (the value, then
 its residual, each with its own scale) fit them with margin, provided the
@@ -166,3 +172,46 @@ def test_mx_activation_terms_against_the_routed_bounds():
     # clipping the block maximum at 448 costs most of that margin
     okc, clip = routed(2, clip_scale=True)
     assert clip["mean_rel"] > 1.5 * two["mean_rel"], (clip, two)
+
+
+def _stage_f16_grouped(v):
+    """f16 copy of a row with max|v| placed in [2^14, 2^15), and its exponent."""
+    amax = float(np.abs(v).max())
+    e = int(np.floor(np.log2(amax))) - 14 if amax > 0 else 0
+    return (v * 2.0 ** -e).astype(np.float16).astype(np.float64), e
+
+
+def _grouped_rows(codes, scales, xs, e):
+    """Rows of MXFP4 times an f16-staged row: exact products, fp32 sums per
+    32-element block, the block scale applied in fp32, fp32 across blocks."""
+    R, K = codes.shape[0], xs.shape[0]
+    w = np.empty((R, K))
+    w[:, 0::2] = _E2M1[codes & 15]
+    w[:, 1::2] = _E2M1[codes >> 4]
+    blk = (w.reshape(R, K // 32, 32) * xs.reshape(K // 32, 32)[None]).astype(np.float32).sum(2, dtype=np.float32)
+    sc = (2.0 ** (scales.astype(np.float64) - 127)).astype(np.float32)
+    return (blk * sc).astype(np.float32).sum(1, dtype=np.float32).astype(np.float64) * 2.0 ** e
+
+
+def test_grouped_path_roundings_fit_the_stated_bounds():
+    cfg = synth.CONFIGS[0].with_(hidden=2048, inter=1024, shared_inter=0, n_experts=8, top_k=2,
+                                 seed=synth.CONFIGS[0].seed + 900)
+    wr = synth.gen_router_w(cfg)
+    x_bf, _ = synth.gen_tokens(cfg, wr, None, [0])
+    x = synth.bf16_to_f32(x_bf[0]).astype(np.float64)
+    I = cfg.inter
+    ys, refs = [], []
+    for expert in range(2):
+        gc, gs, dc, ds = synth.gen_expert(cfg, expert)
+        refs.append(oracle.expert_ffn(x, gc, gs, dc, ds)[1])
+        xs, ex = _stage_f16_grouped(x)
+        assert np.array_equal(xs * 2.0 ** ex, x)            # bf16 activations stage exactly
+        gu = _grouped_rows(gc, gs, xs, ex)
+        g, u = gu[:I], gu[I:]
+        h = (g / (1 + np.exp(-g)) * u).astype(np.float32).astype(np.float64)
+        hs, eh = _stage_f16_grouped(h)
+        ys.append(_grouped_rows(dc, ds, hs, eh))
+    ok, info = metric_close(np.stack(ys), np.stack(refs), Y_ROUTED_MAX_REL, Y_ROUTED_MEAN_REL)
+    assert ok, info
+    assert info["mean_rel"] < Y_ROUTED_MEAN_REL / 4, info
+    assert info["max_abs"] < Y_ROUTED_MAX_REL / 4 * info["max_ref"], info
