@@ -54,18 +54,24 @@ class FakeNvml:
         return self.sm
 
 
+# State changes sit 50 ms away from the region's edges: a sample's time stamp
+# and its reading are two steps of the polling thread, which the interpreter
+# may separate by a thread switch (5 ms by default).
+GAP = 0.05
+
+
 def _run(sampler, fake):
     sampler.start()
     fake.sm, fake.bits = 1965, 0x8            # hw_slowdown outside the timed regions: not counted
-    time.sleep(0.03)
+    time.sleep(GAP)
     fake.sm, fake.bits = 1900, 0x4            # sw_power_cap inside
-    time.sleep(0.01)
+    time.sleep(GAP)
     sampler.begin()
-    time.sleep(0.05)
+    time.sleep(2 * GAP)
     sampler.end()
-    time.sleep(0.01)
+    time.sleep(GAP)
     fake.sm, fake.bits = 1500, 0x40           # thermal slowdown after: not counted
-    time.sleep(0.03)
+    time.sleep(GAP)
     return sampler.stop()
 
 
@@ -94,9 +100,9 @@ def test_reason_bits_map_to_names(monkeypatch):
     s = bench.ClockSampler(0)
     s.start()
     fake.bits = 0x8 | 0x20 | 0x40 | 0x4 | 0x1   # 0x1 (idle) is not reported
-    time.sleep(0.01)
+    time.sleep(GAP)
     s.begin()
-    time.sleep(0.02)
+    time.sleep(2 * GAP)
     s.end()
     c = s.stop()
     assert c["reasons"] == sorted(["hw_slowdown", "sw_thermal_slowdown", "hw_thermal_slowdown", "sw_power_cap"])
