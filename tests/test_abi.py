@@ -71,3 +71,21 @@ def test_selftest_rejects_unknown_requests():
     api.load_library()
     assert api.moe_selftest(0) == api.MOE_ERR_INVALID_ARG
     assert api.moe_selftest(99) == api.MOE_ERR_INVALID_ARG
+
+
+def test_noalloc_router_rejects_invalid_calls_on_the_host(lib):
+    """Every call here is refused by the host-side checks before any CUDA
+    call, so the placeholder addresses are never dereferenced."""
+    from sparse_moe_decode_router_b200 import api
+    routing = api.make_routing(*([0x1000] * 7))
+
+    def call(w=0x1000, H=256, E=32, k=4, x=0x1000, B=1, r=routing):
+        return lib.moe_router_topk_noalloc(w, None, H, E, k, x, B, None if r is None else ctypes.byref(r), None)
+
+    bad = [dict(w=None), dict(w=0x1008), dict(x=None), dict(x=0x1004), dict(r=None),
+           dict(r=api.make_routing(*([0x1000] * 6 + [None]))),
+           dict(H=0), dict(H=250), dict(H=16384 + 32),
+           dict(E=0), dict(E=1025), dict(k=0), dict(k=33, E=64), dict(k=8, E=4),
+           dict(B=0), dict(B=65)]
+    for kw in bad:
+        assert call(**kw) == api.MOE_ERR_INVALID_ARG, kw
