@@ -11,6 +11,11 @@ per-step CUDA events.  Prints one JSON line (rank 0).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--config 1|2|3|4] [--impl ours|reference]
 
+With the default workload (the full-size batch-1 layer) on one GPU the line
+also carries `per_config`: the batch-8 and batch-64 (Zipf) layers through
+the same call, and the 4-layer x 64-step decode loop captured in one CUDA
+graph with and without the next-layer L2 prefetch.
+
 --gpus N > 1 runs under torchrun as N independent replicas (the layer does
 not shard); value = the bytes all ranks moved / the slowest rank's time.
 --impl reference times the CPU oracle on the same workload (rank 0 only).
@@ -47,6 +52,8 @@ def parse_args():
     ap.add_argument("--config", type=int, default=WORKLOAD_DEFAULT)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-per-config", action="store_true",
+                    help="skip the batch-8, batch-64 and 4-layer graph records of the default run")
     ap.add_argument("--flags", type=int, default=0, help="MOE_FLAG_* bits for ablations")
     ap.add_argument("--experts", type=int, default=0,
                     help="profiling aid: fewer routed experts (same per-step work, smaller footprint)")
@@ -58,6 +65,13 @@ def workload_desc(cfg):
     return (f"{cfg.name}: one MoE decode layer, hidden {cfg.hidden}, {cfg.n_experts} routed experts top-{cfg.top_k}, "
             f"expert intermediate {cfg.inter} (MXFP4 E2M1 + E8M0/32), shared expert intermediate "
             f"{cfg.shared_inter} (bf16), batch {cfg.batch}" + (f", Zipf({cfg.zipf_s}) router bias" if cfg.zipf_s else ""))
+
+
+def config_dict(cfg, world, flags):
+    """The `config` object of the JSON line (the same for both arms)."""
+    return {"workload": workload_desc(cfg), "batch": cfg.batch, "parallelism": f"replicas x{world}",
+            "l2": "flushed between steps (256 MiB write, outside the per-step CUDA events)",
+            "token_pool": POOL, "flags": flags}
 
 
 # ---------------------------------------------------------------- clocks ----
@@ -337,7 +351,7 @@ def run_reference(args, cfg):
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": sec * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": workload_desc(cfg), "parallelism": "rank 0 only (CPU oracle)"},
+            "config": config_dict(cfg, 1, args.flags),
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
                              "sample": f"{len(times)} of {args.steps} steps timed (90 s cap), each a full "
                                        f"layer-step of batch {B} (fp64 C++ oracle, OpenMP over {threads} threads)"},
@@ -352,6 +366,191 @@ class _DevPtr:
                                          "data": (int(ptr), False), "version": 3}
 
 
+class LayerRun:
+    """One full-size layer on the device with a pool of distinct token
+    batches, timed through moe_layer_forward (weights and inputs resident in
+    HBM, L2 flushed between steps outside the per-step events)."""
+
+    def __init__(self, cfg, flags, pool, layer=0):
+        import torch
+        from sparse_moe_decode_router_b200 import api
+        from synth.workload import make_device_layer, residual_tokens
+        self.torch, self.api, self.cfg = torch, api, cfg
+        B, H = cfg.batch, cfg.hidden
+        self.dl = make_device_layer(cfg, layer)
+        c = api.moe_layer_config(cfg.hidden, cfg.n_experts, cfg.top_k, cfg.inter, cfg.shared_inter, B, flags)
+        self.handle = api.moe_layer_create(c, self.dl.weights_struct())
+        self.pool = pool
+        self.x, self.r, self.xh, self.rh = [], [], [], []
+        for p in range(pool):
+            ids = [p * B + b for b in range(B)]
+            xh, xd = self.dl.tokens(ids)
+            rh, rd = residual_tokens(cfg, ids)
+            self.x.append(xd)
+            self.r.append(rd)
+            self.xh.append(torch.from_numpy(xh.view(np.int16)).pin_memory())
+            self.rh.append(torch.from_numpy(rh.view(np.int16)).pin_memory())
+        self.out = torch.empty((B, H), dtype=torch.bfloat16, device="cuda")
+        self.out_h = torch.empty((B, H), dtype=torch.int16).pin_memory()
+        self.flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device="cuda")
+        self.stream = torch.cuda.current_stream()
+        plan = api.moe_layer_routing(self.handle)
+        n_act_view = torch.as_tensor(_DevPtr(plan.n_active, (1,), "<i4"), device="cuda")
+        self.n_active = []
+        for p in range(pool):           # experts touched by each pool batch (read back before timing)
+            api.moe_layer_forward(self.handle, None, self.x[p], self.r[p], self.out, B, self.stream)
+            self.n_active.append(int(n_act_view.cpu()[0]))
+        torch.cuda.synchronize()
+        if api.moe_layer_last_device_error(self.handle) != api.MOE_OK:
+            raise SystemExit("device-side error during warm-up")
+
+    def step_bytes(self, i):
+        return self.cfg.counted_bytes(self.n_active[i % self.pool])
+
+    def gate_up_bytes(self, i):
+        """Routed gate/up kernel: codes + scales of the active experts, x in, h out (fp32)."""
+        c = self.cfg
+        na = self.n_active[i % self.pool]
+        return na * 2 * c.inter * (c.hidden // 2 + c.hidden // 32) + c.batch * c.hidden * 2 + \
+            c.batch * c.top_k * c.inter * 4
+
+    def forward(self, i):
+        self.api.moe_layer_forward(self.handle, None, self.x[i % self.pool], self.r[i % self.pool], self.out,
+                                   self.cfg.batch, self.stream)
+
+    def timed(self, steps, warmup, sampler=None, probe=False, host=False):
+        """Per-step device times (ms) of `steps` steps after `warmup` untimed
+        ones; probe: the routed gate/up kernel's own time instead."""
+        torch, api = self.torch, self.api
+        B = self.cfg.batch
+        for i in range(warmup):
+            self.flush.zero_()
+            self.forward(i)
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+        if probe:
+            for a, b in ev:  # materialise the events before handing them to the library
+                a.record(self.stream)
+                b.record(self.stream)
+        torch.cuda.synchronize()
+        if sampler:
+            sampler.begin()
+        for i in range(steps):
+            self.flush.zero_()
+            if probe:
+                api.moe_layer_set_probe(self.handle, ev[i][0], ev[i][1])
+                self.forward(i)
+            elif host:
+                ev[i][0].record(self.stream)
+                api.moe_layer_forward_host(self.handle, self.xh[i % self.pool], self.rh[i % self.pool], self.out_h,
+                                           B, self.stream)
+                ev[i][1].record(self.stream)
+            else:
+                ev[i][0].record(self.stream)
+                self.forward(i)
+                ev[i][1].record(self.stream)
+        torch.cuda.synchronize()
+        if sampler:
+            sampler.end()
+        if probe:
+            api.moe_layer_set_probe(self.handle, None, None)
+        if api.moe_layer_last_device_error(self.handle) != api.MOE_OK:
+            raise SystemExit("device-side error during the timed region")
+        return [a.elapsed_time(b) for a, b in ev]
+
+    def close(self):
+        self.api.moe_layer_destroy(self.handle)
+        del self.dl, self.x, self.r, self.flush
+        self.torch.cuda.empty_cache()
+
+
+def grouped_flops(cfg, n_pairs):
+    """Multiply-add work of the routed experts at one token per pair: gate/up
+    (2I x H) and down (H x I) per pair, 2 flops per multiply-add."""
+    return n_pairs * 2 * (2 * cfg.inter * cfg.hidden + cfg.hidden * cfg.inter)
+
+
+def per_config_record(cfg, flags, steps, warmup, peak, sampler):
+    run = LayerRun(cfg, flags, pool=8)
+    try:
+        ms = run.timed(steps, warmup, sampler)
+        tot = sum(run.step_bytes(i) for i in range(steps))
+        sec = sum(ms) * 1e-3
+        rec = {"workload": workload_desc(cfg), "batch": cfg.batch, "steps": steps, "warmup": warmup,
+               "us_per_step": round(sum(ms) / steps * 1e3, 2), "gb_per_s": round(tot / sec / 1e9, 2),
+               "frac_of_measured_hbm": round(tot / sec / 1e9 / peak, 4),
+               "tokens_per_s": round(cfg.batch * steps / sec, 1),
+               "counted_bytes_per_step": int(tot / steps),
+               "n_active_mean": statistics.mean(run.n_active[i % run.pool] for i in range(steps)),
+               "gpu_launches_per_step": launches_per_step(cfg, flags)}
+        if cfg.batch > 8:
+            fl = grouped_flops(cfg, cfg.batch * cfg.top_k)
+            rec["routed_tflops"] = round(fl * steps / sec / 1e12, 2)
+            rec["expert_path"] = "grouped tensor-core kernels"
+        return rec
+    finally:
+        run.close()
+
+
+def stack_record(cfg, flags, replays, peak, sampler):
+    """Config 4: n_layers full-size layers chained through the residual, an
+    n_steps decode loop captured in one CUDA graph (PDL inside, next-layer L2
+    prefetch unless MOE_FLAG_NO_PREFETCH); device time per replay / layer-steps.
+    Weights (~84 GB) exceed L2 many times over, so L2 is not flushed."""
+    import torch
+    from sparse_moe_decode_router_b200 import api
+    from synth.workload import make_device_layer, residual_tokens
+    nl, ns, H = cfg.n_layers, cfg.n_steps, cfg.hidden
+    layers = [make_device_layer(cfg, l) for l in range(nl)]
+    xs = [[None] * nl for _ in range(ns)]
+    for l in range(nl):
+        _, xd = layers[l].tokens(range(ns))
+        for t in range(ns):
+            xs[t][l] = xd[t:t + 1]
+    _, r0 = residual_tokens(cfg, range(ns), 0)
+    c = api.moe_layer_config(cfg.hidden, cfg.n_experts, cfg.top_k, cfg.inter, cfg.shared_inter, 1, flags)
+    handles = [api.moe_layer_create(c, dl.weights_struct()) for dl in layers]
+    try:
+        outs = [[torch.empty((1, H), dtype=torch.bfloat16, device="cuda") for _ in range(nl)] for _ in range(ns)]
+        g = torch.cuda.CUDAGraph()
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            with torch.cuda.graph(g, stream=s):
+                for t in range(ns):
+                    res = r0[t:t + 1]
+                    for l in range(nl):
+                        api.moe_layer_forward(handles[l], handles[(l + 1) % nl], xs[t][l], res, outs[t][l], 1,
+                                              stream=torch.cuda.current_stream())
+                        res = outs[t][l]
+        st = torch.cuda.current_stream()
+        g.replay()                      # warm-up
+        torch.cuda.synchronize()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(replays)]
+        sampler.begin()
+        for a, b in ev:
+            a.record(st)
+            g.replay()
+            b.record(st)
+        torch.cuda.synchronize()
+        sampler.end()
+        for hd in handles:
+            if api.moe_layer_last_device_error(hd) != api.MOE_OK:
+                raise SystemExit("device-side error in the stack graph")
+        del g
+        ms = statistics.median(a.elapsed_time(b) for a, b in ev)
+        per = ms * 1e3 / (nl * ns)
+        bpl = cfg.counted_bytes(cfg.top_k)       # batch 1: top_k distinct experts per layer-step
+        return {"us_per_layer_step": round(per, 2), "gb_per_s": round(bpl / (per * 1e-6) / 1e9, 2),
+                "frac_of_measured_hbm": round(bpl / (per * 1e-6) / 1e9 / peak, 4),
+                "replays": replays, "replay_ms_median": round(ms, 3), "layer_steps_per_replay": nl * ns,
+                "gpu_launches_per_layer_step": launches_per_step(cfg.with_(batch=1), flags)}
+    finally:
+        for hd in handles:
+            api.moe_layer_destroy(hd)
+        del layers, xs
+        torch.cuda.empty_cache()
+
+
 def run_ours(args, cfg):
     world, rank, local = dist_setup(args.gpus)
     import torch
@@ -363,103 +562,52 @@ def run_ours(args, cfg):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local))
     from sparse_moe_decode_router_b200 import api
-    from synth.workload import make_device_layer, residual_tokens
+    import synth
 
     api.load_library()
     B, H, k = cfg.batch, cfg.hidden, cfg.top_k
-    dl = make_device_layer(cfg, 0)
-    c = api.moe_layer_config(cfg.hidden, cfg.n_experts, cfg.top_k, cfg.inter, cfg.shared_inter, B, args.flags)
-    handle = api.moe_layer_create(c, dl.weights_struct())
-    pool_x, pool_r, pool_xh, pool_rh = [], [], [], []
-    for p in range(POOL):
-        ids = [p * B + b for b in range(B)]
-        xh, xd = dl.tokens(ids)
-        rh, rd = residual_tokens(cfg, ids)
-        pool_x.append(xd)
-        pool_r.append(rd)
-        pool_xh.append(torch.from_numpy(xh.view(np.int16)).pin_memory())
-        pool_rh.append(torch.from_numpy(rh.view(np.int16)).pin_memory())
-    out = torch.empty((B, H), dtype=torch.bfloat16, device="cuda")
-    out_h = torch.empty((B, H), dtype=torch.int16).pin_memory()
-    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device="cuda")
-    stream = torch.cuda.current_stream()
-    plan = api.moe_layer_routing(handle)
-    n_act_view = torch.as_tensor(_DevPtr(plan.n_active, (1,), "<i4"), device="cuda")
-
-    # experts touched by each pool batch (read back before any timing)
-    n_active = []
-    for p in range(POOL):
-        api.moe_layer_forward(handle, None, pool_x[p], pool_r[p], out, B, stream)
-        n_active.append(int(n_act_view.cpu()[0]))
-    torch.cuda.synchronize()
-    if api.moe_layer_last_device_error(handle) != api.MOE_OK:
-        raise SystemExit("device-side error during warm-up")
-
-    def step_bytes(i):
-        return cfg.counted_bytes(n_active[i % POOL])
-
-    # routed gate/up kernel: codes + scales of the active experts, x in, h out (fp32)
-    def gate_up_bytes(i):
-        na = n_active[i % POOL]
-        return na * 2 * cfg.inter * (H // 2 + H // 32) + B * H * 2 + B * k * cfg.inter * 4
-
+    run = LayerRun(cfg, args.flags, POOL)
     try:
         uuid = str(torch.cuda.get_device_properties(local).uuid)
     except Exception:
         uuid = None
     sampler = ClockSampler(local, uuid)
     sampler.start()
-    for i in range(args.warmup):
-        flush.zero_()
-        api.moe_layer_forward(handle, None, pool_x[i % POOL], pool_r[i % POOL], out, B, stream)
     K = args.steps
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
-    pr = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
-    for a, b in pr:  # materialise the CUDA events before handing them to the library
-        a.record(stream)
-        b.record(stream)
+    # headline: whole layer-steps, nothing but the layer between the events
     if dist is not None:
         dist.barrier()
     torch.cuda.synchronize()
-    sampler.begin()
-    for i in range(K):
-        flush.zero_()
-        api.moe_layer_set_probe(handle, pr[i][0], pr[i][1])
-        ev[i][0].record(stream)
-        api.moe_layer_forward(handle, None, pool_x[i % POOL], pool_r[i % POOL], out, B, stream)
-        ev[i][1].record(stream)
-    torch.cuda.synchronize()
-    sampler.end()
+    step_ms = run.timed(K, args.warmup, sampler)
     if dist is not None:
         dist.barrier()
-    api.moe_layer_set_probe(handle, None, None)
-    step_ms = [a.elapsed_time(b) for a, b in ev]
-    gu_ms = [a.elapsed_time(b) for a, b in pr]
-
     # end to end through the host-buffer entry point (pinned host memory)
-    e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
-    torch.cuda.synchronize()
-    sampler.begin()
-    for i in range(K):
-        flush.zero_()
-        e2e_ev[i][0].record(stream)
-        api.moe_layer_forward_host(handle, pool_xh[i % POOL], pool_rh[i % POOL], out_h, B, stream)
-        e2e_ev[i][1].record(stream)
-    torch.cuda.synchronize()
-    sampler.end()
-    clocks = sampler.stop()
-    e2e_ms = [a.elapsed_time(b) for a, b in e2e_ev]
-    if api.moe_layer_last_device_error(handle) != api.MOE_OK:
-        raise SystemExit("device-side error during the timed region")
-
+    e2e_ms = run.timed(K, min(args.warmup, 3), sampler, host=True)
+    # the dominant kernel, timed live in a separate pass (events around it)
+    gu_ms = run.timed(min(K, 100), 3, None, probe=True)
     total_ms = sum(step_ms)
-    total_bytes = sum(step_bytes(i) for i in range(K))
+    total_bytes = sum(run.step_bytes(i) for i in range(K))
     e2e_total = sum(e2e_ms)
     gu_avg_s = statistics.mean(gu_ms) * 1e-3
-    gu_bytes = statistics.mean([gate_up_bytes(i) for i in range(K)])
+    gu_bytes = statistics.mean([run.gate_up_bytes(i) for i in range(len(gu_ms))])
+    n_active_mean = statistics.mean(run.n_active[i % POOL] for i in range(K))
     if dist is not None:
         total_ms, e2e_total = max_over_ranks([total_ms, e2e_total], "cuda")
-    api.moe_layer_destroy(handle)
+    peak, peak_src = measured_peaks()
+    extra = {}
+    if world == 1 and rank == 0 and not args.no_cpu_baseline:
+        extra["cpu_baseline"] = cpu_baseline(cfg, run.dl)
+    run.close()
+    if world == 1 and not args.no_per_config and cfg.name == synth.CONFIGS[1].name:
+        extra["per_config"] = {
+            "full_b8": per_config_record(synth.CONFIGS[2], args.flags, 50, 5, peak, sampler),
+            "full_b64_zipf": per_config_record(synth.CONFIGS[3], args.flags, 20, 3, peak, sampler),
+            "full_stack4_b1_graph": {
+                "prefetch": stack_record(synth.CONFIGS[4], args.flags, 3, peak, sampler),
+                "no_prefetch": stack_record(synth.CONFIGS[4], args.flags | api.MOE_FLAG_NO_PREFETCH, 3, peak,
+                                            sampler)},
+        }
+    clocks = sampler.stop()
     if dist is not None:
         dist.destroy_process_group()
     if rank != 0:
@@ -467,7 +615,6 @@ def run_ours(args, cfg):
 
     ms_per_step = total_ms / K
     value = job_value(world, total_bytes, total_ms)
-    peak, peak_src = measured_peaks()
     achieved = gu_bytes / gu_avg_s / 1e9
     traffic = recorded_traffic("routed_gate_up", cfg.name)
     line = {
@@ -475,26 +622,24 @@ def run_ours(args, cfg):
         "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f16",
         "data": "synthetic (seeded Philox4x32-10 draws; random-init weights of the full-size layer)",
-        "config": {"workload": workload_desc(cfg), "batch": B, "parallelism": f"replicas x{world}",
-                   "l2": "flushed between steps (256 MiB write, outside the per-step CUDA events)",
-                   "token_pool": POOL, "flags": args.flags},
+        "config": config_dict(cfg, world, args.flags),
         "us_per_step": round(ms_per_step * 1e3, 2),
         "tokens_per_s": round(world * B * K / (total_ms * 1e-3), 1),
         "counted_bytes_per_step": int(total_bytes / K),
-        "n_active_mean": statistics.mean(n_active[i % POOL] for i in range(K)),
+        "n_active_mean": n_active_mean,
         "frac_of_measured_hbm": round(value / world / peak, 4),
         "roofline": {"kernel": "routed_gate_up", "bound": "hbm", "achieved": round(achieved, 1),
                      "peak": peak, "unit": "GB/s", "frac": round(achieved / peak, 4), "traffic": traffic,
                      "peak_source": peak_src, "algorithmic_bytes_per_launch": int(gu_bytes),
-                     "avg_launch_us": round(gu_avg_s * 1e6, 2)},
+                     "avg_launch_us": round(gu_avg_s * 1e6, 2),
+                     "timing": "separate pass: events recorded around the kernel on its stream"},
         "e2e": {"value": round(world * total_bytes / (e2e_total * 1e-3) / 1e9, 2), "unit": UNIT,
                 "h2d_bytes_per_step": 2 * B * H * 2, "d2h_bytes_per_step": B * H * 2,
                 "us_per_step": round(e2e_total / K * 1e3, 2)},
         "gpu_launches": launches_per_step(cfg, args.flags) * K,
         "clocks": clocks,
     }
-    if world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(cfg, dl)
+    line.update(extra)
     print(json.dumps(line), flush=True)
 
 
@@ -513,31 +658,42 @@ def launches_per_step(cfg, flags):
     return n + (5 if grouped else 2)
 
 
-def cpu_baseline(cfg, dl):
-    """The oracle as it stands on the host cores, on a bounded sample of the
-    same workload: whole layer-steps until ~10 s of CPU work (at least one)."""
+def _oracle_step(cfg, dl, n, threads):
     import oracle
     from synth.workload import residual_tokens
+    B = cfg.batch
+    ids = [((n % POOL) * B) + b for b in range(B)]
+    x_h, _ = dl.tokens(ids)
+    r_h, _ = residual_tokens(cfg, ids)
+    rt = oracle.routing(x_h, dl.router_w_host, dl.bias_host, cfg.top_k)
+    sel = np.unique(rt["topk_idx"])
+    gc, gs, dc, ds = dl.host_experts(sel)
+    shared = dl.host_shared()
+    t0 = time.perf_counter()
+    oracle.layer(x_h, r_h, dl.router_w_host, dl.bias_host, gc, gs, dc, ds, shared[0], shared[1],
+                 cfg.top_k, experts=sel, n_threads=threads)
+    return time.perf_counter() - t0, cfg.counted_bytes(len(sel))
+
+
+def cpu_baseline(cfg, dl):
+    """The oracle as it stands on the host cores, on a bounded sample of the
+    same workload: whole layer-steps with OpenMP over all host threads until
+    ~10 s of CPU work (at least one), then one layer-step on one thread."""
     threads = os.cpu_count() or 1
     B = cfg.batch
-    shared = dl.host_shared()
     spent, n, nbytes = 0.0, 0, 0
     while n < 1 or (spent < 10.0 and n < 64):
-        ids = [((n % POOL) * B) + b for b in range(B)]
-        x_h, _ = dl.tokens(ids)
-        r_h, _ = residual_tokens(cfg, ids)
-        rt = oracle.routing(x_h, dl.router_w_host, dl.bias_host, cfg.top_k)
-        sel = np.unique(rt["topk_idx"])
-        gc, gs, dc, ds = dl.host_experts(sel)
-        t0 = time.perf_counter()
-        oracle.layer(x_h, r_h, dl.router_w_host, dl.bias_host, gc, gs, dc, ds, shared[0], shared[1],
-                     cfg.top_k, experts=sel, n_threads=threads)
-        spent += time.perf_counter() - t0
-        nbytes += cfg.counted_bytes(len(sel))
+        dt, nb = _oracle_step(cfg, dl, n, threads)
+        spent += dt
+        nbytes += nb
         n += 1
+    dt1, nb1 = _oracle_step(cfg, dl, n, 1)
     return {"value": round(nbytes / spent / 1e9, 4), "unit": UNIT, "cores": threads, "kind": "oracle",
             "sample": f"{n} whole layer-step(s) of batch {B} (fp64 C++ oracle, OpenMP over {threads} threads), "
-                      f"{spent:.1f} s", "us_per_step": round(spent / n * 1e6, 1)}
+                      f"{spent:.1f} s; then one layer-step on one thread",
+            "us_per_step": round(spent / n * 1e6, 1),
+            "single_thread": {"value": round(nb1 / dt1 / 1e9, 4), "unit": UNIT, "cores": 1,
+                              "us_per_step": round(dt1 * 1e6, 1)}}
 
 
 def main():

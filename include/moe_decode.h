@@ -229,9 +229,11 @@ MOE_API moe_status_t moe_layer_set_probe(moe_layer_t layer, void* start, void* s
  * router_bias: fp32 [n_experts] or NULL.  x: bf16 [B][hidden].
  * r: where to write the plan (all seven pointers required), as for
  *   moe_router_topk; the results equal moe_router_topk's bit for bit.
- * Limits: hidden a multiple of 32, <= 16384; 1 <= n_experts <= 1024;
+ * Limits: hidden a multiple of 32, <= 16384; n_experts even, 2..1024;
  *   1 <= top_k <= min(32, n_experts); 1 <= B <= 64; B * n_experts <= 65536.
  *   Anything beyond returns MOE_ERR_INVALID_ARG and launches nothing.
+ *   MOE_ERR_UNSUPPORTED: the device is not compute capability 10.x, or (not
+ *   expected within the limits above) no launch plan fits the shape.
  * The first call on a device (with that device current) looks the array's
  * device address up and sets the kernels' shared-memory limits; make that
  * first call before any stream capture.  The counter is cleared on the

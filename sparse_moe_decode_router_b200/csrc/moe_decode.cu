@@ -910,8 +910,10 @@ moe_status_t moe_layer_last_device_error(moe_layer_t L) {
 moe_status_t moe_router_topk_noalloc(const void* router_w_em, const float* router_bias, int hidden, int n_experts,
                                      int top_k, const void* x, int B, const moe_routing* r, void* stream) {
   if (!router_w_em || !x || !aligned16(router_w_em) || !aligned16(x) || !routing_ok(r)) return MOE_ERR_INVALID_ARG;
-  if (hidden <= 0 || hidden % 32 || hidden > 32 * 32 * 16 || n_experts < 1 || n_experts > kMaxExperts || top_k < 1 ||
-      top_k > kMaxTopK || top_k > n_experts || B < 1 || B > kMaxBatch || (long long)B * n_experts > kNoAllocMaxLogits)
+  // n_experts even: the router's work items are pairs of expert rows
+  if (hidden <= 0 || hidden % 32 || hidden > 32 * 32 * 16 || n_experts < 2 || n_experts > kMaxExperts ||
+      n_experts % 2 || top_k < 1 || top_k > kMaxTopK || top_k > n_experts || B < 1 || B > kMaxBatch ||
+      (long long)B * n_experts > kNoAllocMaxLogits)
     return MOE_ERR_INVALID_ARG;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
@@ -930,11 +932,6 @@ moe_status_t moe_router_topk_noalloc(const void* router_w_em, const float* route
       if (major != 10) return MOE_ERR_UNSUPPORTED;
       void* ptr = nullptr;
       if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || !ptr) return MOE_ERR_CUDA;
-      for (int t = 0; t < 2; ++t) {
-        const GemvPlan p = make_plan(K_ROUTER, hidden, n_experts, t == 0 ? 1 : kMaxBatch, 1, t == 0 ? 1 : kMaxBatch,
-                                     0, g_noalloc_sms[dev]);
-        if (!p.ok) return MOE_ERR_UNSUPPORTED;
-      }
       // the largest dynamic shared memory any router plan asks for
       if (raise_smem_limit(reinterpret_cast<const void*>(gemv_fn(K_ROUTER, 1)), kSmemBudget) != cudaSuccess ||
           raise_smem_limit(reinterpret_cast<const void*>(gemv_fn(K_ROUTER, 2)), kSmemBudget) != cudaSuccess)
@@ -1004,11 +1001,15 @@ moe_status_t moe_router_topk_noalloc_last_error(void) {
   if (!base) return MOE_OK;  // no allocation-free call on this device yet
   // the calls may run on non-blocking streams: wait for all of the device's work
   if (cudaDeviceSynchronize() != cudaSuccess) return MOE_ERR_CUDA;
-  int* err = &static_cast<NoAllocScratch*>(base)->err;
+  NoAllocScratch* sc = static_cast<NoAllocScratch*>(base);
   int v = 0;
-  if (cudaMemcpy(&v, err, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return MOE_ERR_CUDA;
+  if (cudaMemcpy(&v, &sc->err, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return MOE_ERR_CUDA;
   if (v == 0) return MOE_OK;
-  if (cudaMemset(err, 0, sizeof(int)) != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess) return MOE_ERR_CUDA;
+  // clear the word and the top-k completion counter a cut-short call may have
+  // left set (every call also clears the counter on its stream before use)
+  if (cudaMemset(&sc->err, 0, sizeof(int)) != cudaSuccess ||
+      cudaMemset(&sc->done_counter, 0, sizeof(int)) != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess)
+    return MOE_ERR_CUDA;
   return v == kErrTimeout ? MOE_ERR_TIMEOUT : MOE_ERR_INVALID_ARG;
 }
 

@@ -86,6 +86,7 @@ T_EXPERT_GU = 6
 T_EXPERT_D = 7
 T_ZIPF_PERM = 8
 T_TIES = 9
+T_EDGE = 10
 
 # Irwin-Hall(4) of 16-bit uniforms: S = sum - 2*65535, Var(S) = 4*(65536^2-1)/12
 IH_SD = math.sqrt(4.0 * (65536.0 * 65536.0 - 1.0) / 12.0)
@@ -290,19 +291,25 @@ def _logit_gap(x_bf16_row, wr_f64, bias, k):
     return srt[k - 1] - srt[k]
 
 
-def gen_tokens(cfg, router_w_bf16, bias, token_ids, layer=0, max_attempts=64):
+def gen_tokens(cfg, router_w_bf16, bias, token_ids, layer=0, max_attempts=64, tiny_every=0, tiny_exp=-30):
     """bf16 activations x [len(token_ids)][H].  Token t is drawn from
     substream (X, layer; sub0 = t, sub1 = attempt); a draw whose fp64 router
     logits (plus bias) put less than cfg.min_gap between the k-th and
     (k+1)-th largest is redrawn with the next attempt number, so that the
-    selected expert set is decided with margin (input conditioning only)."""
+    selected expert set is decided with margin (input conditioning only).
+    tiny_every > 0 multiplies every tiny_every-th element of each draw by
+    2^tiny_exp (exact in fp32) before the bf16 rounding, so that a row mixes
+    elements some 2^30 apart in magnitude."""
     key = stream_key(cfg.seed, layer, T_X)
     wr = bf16_to_f32(router_w_bf16).astype(np.float64)
     out = np.empty((len(token_ids), cfg.hidden), dtype=np.uint16)
     attempts = np.zeros(len(token_ids), dtype=np.int32)
     for i, t in enumerate(token_ids):
         for a in range(max_attempts):
-            row = bf16_rne(normal_f32(key, int(t), a, 0, cfg.hidden, cfg.act_sigma))
+            v = normal_f32(key, int(t), a, 0, cfg.hidden, cfg.act_sigma)
+            if tiny_every > 0:
+                v[::tiny_every] *= np.float32(2.0 ** tiny_exp)
+            row = bf16_rne(v)
             if _logit_gap(row, wr, bias, cfg.top_k) >= cfg.min_gap:
                 break
         else:
@@ -354,6 +361,29 @@ def gen_tied_tokens(cfg, B, layer=0):
     x = (c0.astype(np.int64) % 3 - 1).reshape(B, H).astype(np.float32)
     x[0] = 0.0
     return bf16_rne(x)
+
+
+def gen_edge_mxfp4(cfg, n_experts, rows, K, tensor, s_lo, s_hi, zero_every=23, layer=0):
+    """MXFP4 tensors that reach the format's corners: codes uint8
+    [n_experts][rows][K/2] and scales uint8 [n_experts][rows][K/32].  Every
+    32-element block holds each of the 16 E2M1 codes (negative zero, code 8,
+    included) exactly twice, in a seeded order; scale bytes are drawn evenly
+    from [s_lo, s_hi], and every zero_every-th block (counted over the whole
+    tensor) gets s = 0, the smallest E8M0 value 2^-127.  Substream (EDGE,
+    layer; sub0 = tensor)."""
+    assert K % 32 == 0 and 0 <= s_lo <= s_hi <= 254
+    key = stream_key(cfg.seed, layer, T_EDGE)
+    nblk = n_experts * rows * (K // 32)
+    n = nblk * 32
+    o0, o1, _, _ = philox4x32_10(np.arange(n, dtype=np.uint64), int(tensor), 0, 0, *key)
+    order = np.argsort(o0.reshape(nblk, 32), axis=1, kind="stable")
+    codes = (order % 16).astype(np.uint8).reshape(n_experts, rows, K)
+    packed = (codes[..., 0::2] | (codes[..., 1::2] << np.uint8(4))).astype(np.uint8)
+    sb, _, _, _ = philox4x32_10(np.arange(nblk, dtype=np.uint64), int(tensor), 1, 0, *key)
+    s = (s_lo + sb.astype(np.int64) % (s_hi - s_lo + 1)).astype(np.int64)
+    if zero_every > 0:
+        s[::zero_every] = 0
+    return packed, s.astype(np.uint8).reshape(n_experts, rows, K // 32)
 
 
 def gen_host_layer(cfg, layer=0, experts=None):

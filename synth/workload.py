@@ -8,7 +8,8 @@ from dataclasses import dataclass
 import numpy as np
 
 from . import (T_EXPERT_D, T_EXPERT_GU, T_ROUTER_W, T_SHARED_D, T_SHARED_GU, MoEConfig,
-               dev_fill_bf16, dev_fill_mxfp4, gen_residual, gen_router_bias, gen_tokens, stream_key)
+               dev_fill_bf16, dev_fill_mxfp4, gen_edge_mxfp4, gen_residual, gen_router_bias, gen_tokens,
+               stream_key)
 
 
 def _t():
@@ -57,9 +58,11 @@ class DeviceLayer:
         return moe_layer_weights(p(self.router_w), p(self.router_bias), p(self.gu_codes), p(self.gu_scales),
                                  p(self.d_codes), p(self.d_scales), p(self.shared_gu), p(self.shared_d))
 
-    def tokens(self, token_ids):
-        """bf16 x for the given token ids (gap-conditioned), host and device."""
-        x, _ = gen_tokens(self.cfg, self.router_w_host, self.bias_host, list(token_ids), layer=self.layer)
+    def tokens(self, token_ids, tiny_every=0):
+        """bf16 x for the given token ids (gap-conditioned), host and device;
+        tiny_every > 0: every tiny_every-th element scaled by 2^-30."""
+        x, _ = gen_tokens(self.cfg, self.router_w_host, self.bias_host, list(token_ids), layer=self.layer,
+                          tiny_every=tiny_every)
         return x, u16_to_device(x, self.gu_codes.device)
 
 
@@ -92,3 +95,20 @@ def make_device_layer(cfg: MoEConfig, layer: int = 0, device="cuda") -> DeviceLa
 def residual_tokens(cfg: MoEConfig, token_ids, layer: int = 0, device="cuda"):
     r = gen_residual(cfg, list(token_ids), layer)
     return r, u16_to_device(r, device)
+
+
+def with_edge_experts(dl: DeviceLayer, gu_scales=(87, 139), d_scales=(115, 167)) -> DeviceLayer:
+    """The same layer with every routed expert replaced by corner-case MXFP4
+    tensors (synth.gen_edge_mxfp4): all 16 E2M1 codes in every block, scale
+    bytes spread over the given ranges (defaults: gate/up 2^-40 .. 2^12, down
+    2^-12 .. 2^40, chosen so that the layer's outputs stay inside fp32) and a
+    share of s = 0 blocks.  Router, shared expert and seeds are unchanged."""
+    import dataclasses
+    torch = _t()
+    c = dl.cfg
+    H, E, I = c.hidden, c.n_experts, c.inter
+    gc, gs = gen_edge_mxfp4(c, E, 2 * I, H, T_EXPERT_GU, *gu_scales, layer=dl.layer)
+    dc, ds = gen_edge_mxfp4(c, E, H, I, T_EXPERT_D, *d_scales, layer=dl.layer)
+    dev = dl.gu_codes.device
+    to = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(dev)
+    return dataclasses.replace(dl, gu_codes=to(gc), gu_scales=to(gs), d_codes=to(dc), d_scales=to(ds))

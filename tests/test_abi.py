@@ -85,7 +85,7 @@ def test_noalloc_router_rejects_invalid_calls_on_the_host(lib):
     bad = [dict(w=None), dict(w=0x1008), dict(x=None), dict(x=0x1004), dict(r=None),
            dict(r=api.make_routing(*([0x1000] * 6 + [None]))),
            dict(H=0), dict(H=250), dict(H=16384 + 32),
-           dict(E=0), dict(E=1025), dict(k=0), dict(k=33, E=64), dict(k=8, E=4),
-           dict(B=0), dict(B=65)]
+           dict(E=0), dict(E=1025), dict(E=31), dict(E=1023, k=4), dict(k=0), dict(k=33, E=64),
+           dict(k=8, E=4), dict(B=0), dict(B=65)]
     for kw in bad:
         assert call(**kw) == api.MOE_ERR_INVALID_ARG, kw

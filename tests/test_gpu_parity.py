@@ -23,14 +23,15 @@ def torch_cuda():
     return torch
 
 
-def run_all_paths(torch, dl, B, max_batch=None, flags=0, token0=0):
+def run_all_paths(torch, dl, B, max_batch=None, flags=0, token0=0, tiny_every=0):
     """Staged calls, fused forward and host forward on one batch; returns
-    GPU results and the oracle's."""
+    GPU results and the oracle's.  tiny_every > 0: activation rows with
+    every tiny_every-th element scaled by 2^-30."""
     from sparse_moe_decode_router_b200 import api
     c = dl.cfg
     H, k, E = c.hidden, c.top_k, c.n_experts
     ids = list(range(token0, token0 + B))
-    x_h, x_d = dl.tokens(ids)
+    x_h, x_d = dl.tokens(ids, tiny_every=tiny_every)
     r_h, r_d = residual_tokens(c, ids, dl.layer)
     h = create_layer(dl, max_batch or B, flags)
     try:

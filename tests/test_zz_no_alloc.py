@@ -47,3 +47,45 @@ def test_noalloc_router_matches_layer_router_twice():
         assert e.value.status == api.MOE_ERR_INVALID_ARG
     finally:
         api.moe_layer_destroy(h)
+
+
+@pytest.mark.parametrize("cfg_id,batches", [(1, (1,)), (3, (1, 64))])
+def test_noalloc_router_full_size_matches_oracle_and_layer(cfg_id, batches):
+    """Full-size router (hidden 7168, 896 experts, top-16; config 3 adds its
+    Zipf bias): the allocation-free entry against the oracle (indices,
+    counts, offsets, pairs and active list exactly, weights within the
+    routing tolerance) and against the layer's router, whose batch-1 call
+    runs a kernel instance specialised for hidden 7168, bit for bit."""
+    import torch
+    import oracle
+    from helpers import W_ABS
+    from gpu_common import assert_routing_equal
+    from sparse_moe_decode_router_b200 import api
+    if not torch.cuda.is_available():
+        pytest.fail("GPU tests need a CUDA device")
+    api.load_library()
+    cfg = synth.CONFIGS[cfg_id]
+    dl = make_device_layer(cfg)
+    H, E, k = cfg.hidden, cfg.n_experts, cfg.top_k
+    w_em = dl.router_w.t().contiguous()
+    h = create_layer(dl, max(batches))
+    try:
+        for B in batches:
+            x_h, x = dl.tokens(range(B))
+            want = routing_buffers(B, k, E)
+            api.moe_router_topk(h, x, B, routing_struct(want))
+            got = routing_buffers(B, k, E)
+            api.moe_router_topk_noalloc(w_em, dl.router_bias, H, E, k, x, B, routing_struct(got))
+            torch.cuda.synchronize()
+            assert api.moe_router_topk_noalloc_last_error() == api.MOE_OK
+            assert api.moe_layer_last_device_error(h) == api.MOE_OK
+            g, w = routing_host(got), routing_host(want)
+            ref = oracle.routing(x_h, dl.router_w_host, dl.bias_host, k)
+            assert_routing_equal(g, ref, W_ABS)
+            for key in ("topk_idx", "counts", "offsets", "pair_ids", "active"):
+                assert np.array_equal(g[key], w[key]), (B, key)
+            assert np.array_equal(g["topk_w"], w["topk_w"]), B
+    finally:
+        api.moe_layer_destroy(h)
+        del dl, w_em
+        torch.cuda.empty_cache()
