@@ -82,6 +82,11 @@ typedef struct moe_layer* moe_layer_t; /* opaque, library-owned */
                                       the caller's stream, overlapping the top-k) */
 #define MOE_FLAG_NO_PREFETCH 0x4u   /* no L2 prefetch of the next layer's weights */
 #define MOE_FLAG_NO_GROUPED 0x8u    /* never use the tensor-core grouped expert path */
+#define MOE_FLAG_MX_EXPERTS 0x10u   /* routed experts at every batch size on the tcgen05 block-scaled
+                                      kernels (E2M1 weights x E4M3 activation terms, E8M0 scales
+                                      on both); needs hidden and inter multiples of 128 and
+                                      32-byte aligned expert codes, else moe_layer_create returns
+                                      MOE_ERR_UNSUPPORTED */
 
 typedef struct {
   int hidden;       /* H: model width, multiple of 32 */

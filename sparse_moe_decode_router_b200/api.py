@@ -25,6 +25,7 @@ MOE_FLAG_NO_PDL = 0x1
 MOE_FLAG_SIDE_STREAM = 0x2
 MOE_FLAG_NO_PREFETCH = 0x4
 MOE_FLAG_NO_GROUPED = 0x8
+MOE_FLAG_MX_EXPERTS = 0x10
 
 # every entry point the header declares
 EXPORTS = (

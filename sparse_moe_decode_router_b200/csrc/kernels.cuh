@@ -122,11 +122,10 @@ struct NextPow2 {
 // Fixed-order combine of one output element: residual + y_shared + sum_j w_j y_j
 // (fp32, fused multiply-adds in ascending j = ascending expert id), bf16 once.
 // The loads of up to sixteen pairs go out together, ahead of their ordered sums.
-__device__ __forceinline__ uint16_t combine_one(const GemvArgs& a, const float* __restrict__ y, int H, int b,
-                                                int r) {
-  const int k = a.top_k;
-  float acc = __uint_as_float((uint32_t)a.residual[(size_t)b * H + r] << 16);
-  if (a.y_shared) acc += __ldcg(a.y_shared + (size_t)b * H + r);
+__device__ __forceinline__ uint16_t combine_elem(const uint16_t* __restrict__ residual, const float* y_shared,
+                                                 const float* comb_w, int k, const float* y, int H, int b, int r) {
+  float acc = __uint_as_float((uint32_t)residual[(size_t)b * H + r] << 16);
+  if (y_shared) acc += __ldcg(y_shared + (size_t)b * H + r);
   for (int j0 = 0; j0 < k; j0 += 16) {
     float wv[16], yv[16];
 #pragma unroll
@@ -134,7 +133,7 @@ __device__ __forceinline__ uint16_t combine_one(const GemvArgs& a, const float* 
       wv[j] = 0.f;
       yv[j] = 0.f;
       if (j0 + j < k) {
-        wv[j] = __ldcg(a.comb_w + b * k + j0 + j);
+        wv[j] = __ldcg(comb_w + b * k + j0 + j);
         yv[j] = __ldcg(y + ((size_t)b * k + j0 + j) * H + r);
       }
     }
@@ -143,6 +142,11 @@ __device__ __forceinline__ uint16_t combine_one(const GemvArgs& a, const float* 
       if (j0 + j < k) acc = fmaf(wv[j], yv[j], acc);
   }
   return f32_to_bf16_rne(acc);
+}
+
+__device__ __forceinline__ uint16_t combine_one(const GemvArgs& a, const float* __restrict__ y, int H, int b,
+                                                int r) {
+  return combine_elem(a.residual, a.y_shared, a.comb_w, a.top_k, y, H, b, r);
 }
 
 // ---------------------------------------------------------------------------

@@ -1,6 +1,7 @@
 // Host side of the MoE decode library: layer object, launch plans,
 // programmatic-dependent-launch chaining, the shared-expert side stream and
 // the C ABI declared in include/moe_decode.h.
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -16,6 +17,7 @@
 #include "gemv.cuh"
 #include "kernels.cuh"
 #include "mma_grouped.cuh"
+#include "mx_umma.cuh"
 
 using namespace moe;
 
@@ -256,6 +258,15 @@ struct moe_layer {
   int* xe = nullptr;          // ... and its per-row exponents
   int mma_stages[2] = {0, 0};  // grouped path ring depth: [gate/up, down] (0 = not usable)
   bool grouped = false;
+  // tcgen05 block-scaled expert path: tensor maps over the weights and over
+  // the activation-term buffers, and the buffers themselves
+  bool mx = false;      // the shapes and pointers allow it
+  bool mx_on = false;   // routed experts run on it
+  CUtensorMap tm_agu{}, tm_adn{}, tm_bx{}, tm_bh{};
+  uint8_t* aqx = nullptr;   // E4M3 terms of x per pair position [MB*k*T][H]
+  uint8_t* asfx = nullptr;  // ... their scales [MB*k*T][H/32]
+  uint8_t* aqh = nullptr;   // E4M3 terms of h [MB*k*T][I]
+  uint8_t* asfh = nullptr;  // ... their scales [MB*k*T][I/32]
   int* err = nullptr;
   uint16_t* x_stage = nullptr;
   uint16_t* res_stage = nullptr;
@@ -405,7 +416,156 @@ constexpr int kGroupedMinBatch = MOE_GROUPED_MIN_BATCH;
 cudaError_t launch_grouped(moe_layer* L, bool gate_up, int B, const moe_routing& r, const void* act, float* out,
                            cudaStream_t st);
 
-cudaError_t launch_gate_up(moe_layer* L, const void* x, int B, const moe_routing& r, cudaStream_t st) {
+cudaError_t launch_gate_up_streams(moe_layer* L, const void* x, int B, const moe_routing& r, cudaStream_t st);
+
+// ---- tcgen05 block-scaled expert path -------------------------------------
+constexpr int kMxTerms = 3;  // E4M3 terms per activation row
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no link
+// against the driver library); null if unavailable
+EncodeTiledFn encode_tiled_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+    else
+      cudaGetLastError();
+  });
+  return fn;
+}
+
+// 2-D tiled map over a row-major matrix: `inner` elements per row, `rows`
+// rows `row_bytes` apart; box = box_inner x box_rows; 128-byte swizzle
+bool encode_map(CUtensorMap* m, CUtensorMapDataType t, const void* base, uint64_t inner, uint64_t rows,
+                uint64_t row_bytes, uint32_t box_inner, uint32_t box_rows) {
+  EncodeTiledFn fn = encode_tiled_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {inner, rows};
+  const cuuint64_t strides[1] = {row_bytes};
+  const cuuint32_t box[2] = {box_inner, box_rows};
+  const cuuint32_t es[2] = {1, 1};
+  return fn(m, t, 2, const_cast<void*>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
+struct MxPlan {
+  int n_max, stage_bytes, n_stages, smem, off_up, off_b, off_sfa, off_sfb;
+};
+
+// shared-memory ring of one projection: a stage holds the A tile(s), the B
+// rows of one pass and the scale-factor chunks
+MxPlan mx_plan(bool gate_up, int B) {
+  MxPlan p;
+  p.n_max = std::min(kMxNMax, (B * kMxTerms + 15) & ~15);
+  p.off_up = gate_up ? kMxABytes : 0;
+  p.off_b = (gate_up ? 2 : 1) * kMxABytes;
+  p.off_sfa = p.off_b + p.n_max * 128;
+  p.off_sfb = p.off_sfa + (gate_up ? 1024 : 512);
+  p.stage_bytes = (int)align_up((size_t)p.off_sfb + 512, 1024);
+  p.n_stages = std::min(kMxMaxStages, (kSmemBudget - 2 * kMxHeaderBytes) / p.stage_bytes);
+  p.smem = 2 * kMxHeaderBytes + p.n_stages * p.stage_bytes;
+  return p;
+}
+
+MxArgs mx_args(const moe_layer* L, bool gate_up, int B, const moe_routing& r, const MxPlan& p, float* out) {
+  const int H = L->cfg.hidden, I = L->cfg.inter, k = L->cfg.top_k;
+  MxArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.sc = gate_up ? L->w.s_gate_up : L->w.s_down;
+  a.s_gstride = gate_up ? (long long)2 * I * (H / 32) : (long long)H * (I / 32);
+  a.a_rows = gate_up ? 2 * I : H;
+  a.K = gate_up ? H : I;
+  a.out_rows = gate_up ? I : H;
+  a.up_off = gate_up ? I : 0;
+  a.top_k = k;
+  a.n_pairs = B * k;
+  a.n_experts = L->cfg.n_experts;
+  a.n_active = r.n_active;
+  a.active = r.active;
+  a.offsets = r.offsets;
+  a.pair_ids = r.pair_ids;
+  a.asf = gate_up ? L->asfx : L->asfh;
+  a.act_rows = L->cfg.max_batch * k * kMxTerms;
+  a.n_max = p.n_max;
+  a.out_f32 = out;
+  a.next_aq = gate_up ? L->aqh : nullptr;
+  a.next_asf = gate_up ? L->asfh : nullptr;
+  a.n_stages = p.n_stages;
+  a.stage_bytes = p.stage_bytes;
+  a.off_up = p.off_up;
+  a.off_b = p.off_b;
+  a.off_sfa = p.off_sfa;
+  a.off_sfb = p.off_sfb;
+  a.err = L->err;
+  return a;
+}
+
+// gate/up on the tensor cores: x -> E4M3 terms per pair position, then the
+// block-scaled MMA kernel (h fp32 into `h`, and h's terms for the down kernel)
+cudaError_t launch_mx_gate_up(moe_layer* L, const void* x, int B, const moe_routing& r, float* h, cudaStream_t st,
+                              cudaEvent_t ev0, cudaEvent_t ev1) {
+  const int H = L->cfg.hidden, k = L->cfg.top_k;
+  cudaError_t e = launch_ex(mx_x_terms_kernel<kMxTerms>, B * k, 256, 0, st, L->pdl, static_cast<const uint16_t*>(x),
+                            H, k, B * k, static_cast<const int*>(r.pair_ids), L->aqx, L->asfx, L->err);
+  if (e != cudaSuccess) return e;
+  const MxPlan p = mx_plan(true, B);
+  const MxArgs a = mx_args(L, true, B, r, p, h);
+  if (ev0 && (e = cudaEventRecord(ev0, st)) != cudaSuccess) return e;
+  e = launch_ex(mx_expert_kernel<true, kMxTerms>, L->num_sms, kMxThreads, p.smem, st, L->pdl, L->tm_agu, L->tm_bx,
+                a);
+  if (e == cudaSuccess && ev1) e = cudaEventRecord(ev1, st);
+  return e;
+}
+
+// down projection on the tensor cores; with `residual` non-null fused with
+// the combine (and the next layer's L2 prefetch)
+cudaError_t launch_mx_down(moe_layer* L, int B, const moe_routing& r, float* y, cudaStream_t st,
+                           const void* residual = nullptr, void* out = nullptr, const float* ys = nullptr,
+                           const moe_layer* next = nullptr) {
+  const MxPlan p = mx_plan(false, B);
+  MxArgs a = mx_args(L, false, B, r, p, y);
+  if (residual) {
+    a.comb_w = r.topk_w;
+    a.y_shared = ys;
+    a.residual = static_cast<const uint16_t*>(residual);
+    a.out_bf16 = static_cast<uint16_t*>(out);
+    a.batch = B;
+    a.tile_counter = L->tile_cnt;
+    if (next && L->prefetch) {
+      a.pf_ptr[0] = reinterpret_cast<const uint8_t*>(next->wr_t);
+      a.pf_bytes[0] = (long long)next->cfg.n_experts * next->cfg.hidden * 2;
+      if (next->cfg.shared_inter > 0) {
+        a.pf_ptr[1] = reinterpret_cast<const uint8_t*>(next->w.shared_gate_up);
+        a.pf_bytes[1] = (long long)2 * next->cfg.shared_inter * next->cfg.hidden * 2;
+      }
+    }
+  }
+  return launch_ex(mx_expert_kernel<false, kMxTerms>, L->num_sms, kMxThreads, p.smem, st, L->pdl, L->tm_adn,
+                   L->tm_bh, a);
+}
+
+cudaError_t launch_gate_up(moe_layer* L, const void* x, int B, const moe_routing& r, cudaStream_t st,
+                           cudaEvent_t ev0 = nullptr, cudaEvent_t ev1 = nullptr) {
+  if (L->mx_on) return launch_mx_gate_up(L, x, B, r, L->h, st, ev0, ev1);
+  if (ev0) {
+    const cudaError_t e = cudaEventRecord(ev0, st);
+    if (e != cudaSuccess) return e;
+  }
+  cudaError_t e = launch_gate_up_streams(L, x, B, r, st);
+  if (e == cudaSuccess && ev1) e = cudaEventRecord(ev1, st);
+  return e;
+}
+
+cudaError_t launch_gate_up_streams(moe_layer* L, const void* x, int B, const moe_routing& r, cudaStream_t st) {
   if (B > kGroupedMinBatch && L->grouped) return launch_grouped(L, true, B, r, x, L->h, st);
   const int H = L->cfg.hidden, I = L->cfg.inter;
   const GemvPlan& p = plan_of(L, K_GU, B);
@@ -464,6 +624,10 @@ cudaError_t launch_combine(moe_layer* L, int B, const moe_routing& r, const floa
 
 cudaError_t launch_down(moe_layer* L, int B, const moe_routing& r, float* y, bool fused, const void* residual,
                         void* out, const float* ys, moe_layer* next, cudaStream_t st, bool pdl) {
+  if (L->mx_on) {
+    (void)pdl;
+    return fused ? launch_mx_down(L, B, r, y, st, residual, out, ys, next) : launch_mx_down(L, B, r, y, st);
+  }
   if (B > kGroupedMinBatch && L->grouped) {
     // tensor-core projection into y, then the fixed-order combine
     cudaError_t e = launch_grouped(L, false, B, r, L->h, y, st);
@@ -697,6 +861,11 @@ moe_status_t moe_layer_create(const moe_layer_config* cfg, const moe_layer_weigh
   const size_t o_xs = take((size_t)MB * H * 2);
   const size_t o_rs = take((size_t)MB * H * 2);
   const size_t o_os = take((size_t)MB * H * 2);
+  const size_t mx_rows = (size_t)MB * k * kMxTerms;
+  const size_t o_aqx = take(mx_rows * H);
+  const size_t o_sfx = take(mx_rows * (H / 32));
+  const size_t o_aqh = take(mx_rows * I);
+  const size_t o_sfh = take(mx_rows * (I / 32));
   if (g_fail_next_alloc.exchange(false) || cudaMalloc(&L->arena, off) != cudaSuccess) {
     cudaGetLastError();
     delete L;
@@ -724,6 +893,10 @@ moe_status_t moe_layer_create(const moe_layer_config* cfg, const moe_layer_weigh
   L->x_stage = reinterpret_cast<uint16_t*>(A + o_xs);
   L->res_stage = reinterpret_cast<uint16_t*>(A + o_rs);
   L->out_stage = reinterpret_cast<uint16_t*>(A + o_os);
+  L->aqx = reinterpret_cast<uint8_t*>(A + o_aqx);
+  L->asfx = reinterpret_cast<uint8_t*>(A + o_sfx);
+  L->aqh = reinterpret_cast<uint8_t*>(A + o_aqh);
+  L->asfh = reinterpret_cast<uint8_t*>(A + o_sfh);
 
   cudaError_t e = cudaMemset(L->arena, 0, off);
   if (e == cudaSuccess) {
@@ -752,11 +925,34 @@ moe_status_t moe_layer_create(const moe_layer_config* cfg, const moe_layer_weigh
     }
     if (ok && (I % (kMmaRows / 2)) == 0 && (H % kMmaRows) == 0) L->grouped = true;
   }
+  // tcgen05 block-scaled path: K and output rows in whole 128-tiles, weights
+  // 32-byte aligned (4-bit TMA), tensor maps encodable
+  if (e == cudaSuccess && H % kMxKTile == 0 && I % kMxKTile == 0 &&
+      (reinterpret_cast<uintptr_t>(w->w_gate_up) & 31u) == 0 && (reinterpret_cast<uintptr_t>(w->w_down) & 31u) == 0) {
+    const uint64_t mxr = (uint64_t)MB * k * kMxTerms;
+    L->mx = encode_map(&L->tm_agu, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, w->w_gate_up, (uint64_t)H,
+                       (uint64_t)E * 2 * I, (uint64_t)H / 2, kMxKTile, kMxRows) &&
+            encode_map(&L->tm_adn, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, w->w_down, (uint64_t)I, (uint64_t)E * H,
+                       (uint64_t)I / 2, kMxKTile, kMxRows) &&
+            encode_map(&L->tm_bx, CU_TENSOR_MAP_DATA_TYPE_UINT8, L->aqx, (uint64_t)H, mxr, (uint64_t)H, kMxKTile, 8) &&
+            encode_map(&L->tm_bh, CU_TENSOR_MAP_DATA_TYPE_UINT8, L->aqh, (uint64_t)I, mxr, (uint64_t)I, kMxKTile, 8);
+    L->mx_on = L->mx && (c.flags & MOE_FLAG_MX_EXPERTS);
+  }
+  if (e == cudaSuccess && L->mx) {
+    e = raise_smem_limit(reinterpret_cast<const void*>(mx_expert_kernel<true, kMxTerms>), kSmemBudget);
+    if (e == cudaSuccess)
+      e = raise_smem_limit(reinterpret_cast<const void*>(mx_expert_kernel<false, kMxTerms>), kSmemBudget);
+  }
+  if ((c.flags & MOE_FLAG_MX_EXPERTS) && !L->mx && e == cudaSuccess) {
+    moe_layer_destroy(L);
+    return MOE_ERR_UNSUPPORTED;
+  }
   if (e == cudaSuccess && L->grouped) {
     e = raise_smem_limit(reinterpret_cast<const void*>(grouped_mma_kernel<true>), kSmemBudget);
     if (e == cudaSuccess) e = raise_smem_limit(reinterpret_cast<const void*>(grouped_mma_kernel<false>), kSmemBudget);
   }
   const void* small_kernels[] = {reinterpret_cast<const void*>(topk_bucket_kernel),
+                                 reinterpret_cast<const void*>(mx_x_terms_kernel<kMxTerms>),
                                  reinterpret_cast<const void*>(act_to_f16_kernel<false>),
                                  reinterpret_cast<const void*>(act_to_f16_kernel<true>),
                                  reinterpret_cast<const void*>(combine_kernel)};
@@ -862,9 +1058,7 @@ moe_status_t moe_layer_forward(moe_layer_t L, moe_layer_t next, const void* x, c
   if (e == cudaSuccess) e = launch_router(L, x, B, L->plan, st);
   // the shared expert's gate/up reads only x: it starts while the top-k runs
   if (e == cudaSuccess && has_shared && !fork) e = launch_shared(L, x, B, L->ys, st, L->pdl, true);
-  if (e == cudaSuccess && L->probe_start) e = cudaEventRecord(L->probe_start, st);
-  if (e == cudaSuccess) e = launch_gate_up(L, x, B, L->plan, st);
-  if (e == cudaSuccess && L->probe_stop) e = cudaEventRecord(L->probe_stop, st);
+  if (e == cudaSuccess) e = launch_gate_up(L, x, B, L->plan, st, L->probe_start, L->probe_stop);
   if (e == cudaSuccess && fork) e = cudaStreamWaitEvent(st, L->ev_join, 0);
   if (e == cudaSuccess)
     e = launch_down(L, B, L->plan, L->y, true, residual, out, has_shared ? L->ys : nullptr, next, st,

@@ -281,3 +281,78 @@ def test_full_b1_run_to_run_bit_identical(torch_cuda, full_layers):
             assert np.array_equal(to_host_u16(o), first)
     finally:
         api.moe_layer_destroy(h)
+
+
+# ------------------------------------------- tcgen05 block-scaled path -----
+MX = 0x10  # MOE_FLAG_MX_EXPERTS
+
+
+@pytest.mark.parametrize("B", [1, 2, 7, 33, 64])
+def test_mx_tiny_all_paths_match_oracle(torch_cuda, tiny, B):
+    """Routed experts on the tcgen05 kernels (E2M1 x E4M3 terms, E8M0 scales
+    on both operands): tiny layer, one 128-row tile per projection."""
+    got, ref = run_all_paths(torch_cuda, tiny, B, max_batch=64, flags=MX)
+    check_against_oracle(got, ref)
+
+
+@pytest.mark.parametrize("B", [1, 5, 9, 33, 64])
+def test_mx_skewed_matches_oracle(torch_cuda, skewed_small, B):
+    """Several K tiles and row tiles; B = 64 has an expert with 56 tokens
+    (three passes of 21 tokens over its weights)."""
+    got, ref = run_all_paths(torch_cuda, skewed_small, B, max_batch=64, flags=MX)
+    check_against_oracle(got, ref)
+
+
+def test_mx_and_gemv_paths_agree(torch_cuda, skewed_small):
+    got_m, ref = run_all_paths(torch_cuda, skewed_small, 7, max_batch=8, flags=MX)
+    got_g, _ = run_all_paths(torch_cuda, skewed_small, 7, max_batch=8)
+    check_against_oracle(got_m, ref)
+    check_against_oracle(got_g, ref)
+    assert np.array_equal(got_m["routing"]["topk_idx"], got_g["routing"]["topk_idx"])
+
+
+@pytest.mark.parametrize("cfg_id", [1, 2])
+def test_mx_full_size_matches_oracle(torch_cuda, full_layers, cfg_id):
+    dl = full_layers(cfg_id)
+    got, ref = run_all_paths(torch_cuda, dl, dl.cfg.batch, flags=MX)
+    check_against_oracle(got, ref)
+
+
+def test_mx_full_size_b64_zipf(torch_cuda, full_layers):
+    """Batch 64, Zipf-skewed routing, tcgen05 path: routing of all 64 tokens
+    bit-exact; routed expert outputs (staged call) and layer outputs (fused
+    call) of a sample of tokens, the hottest expert's among them, against the
+    oracle run on those tokens (tokens are independent of each other)."""
+    from sparse_moe_decode_router_b200 import api
+    import oracle
+    torch = torch_cuda
+    dl = full_layers(3)
+    c = dl.cfg
+    B, H, k, E = c.batch, c.hidden, c.top_k, c.n_experts
+    ids = list(range(B))
+    x_h, x_d = dl.tokens(ids)
+    r_h, r_d = residual_tokens(c, ids)
+    ref_rt = oracle.routing(x_h, dl.router_w_host, dl.bias_host, k)
+    h = create_layer(dl, B, MX)
+    try:
+        out = torch.empty((B, H), dtype=torch.bfloat16, device="cuda")
+        api.moe_layer_forward(h, None, x_d, r_d, out, B)
+        y = torch.empty((B * k, H), dtype=torch.float32, device="cuda")
+        ys = torch.empty((B, H), dtype=torch.float32, device="cuda")
+        api.moe_experts_mxfp4(h, x_d, B, None, y, ys)
+        torch.cuda.synchronize()
+        assert api.moe_layer_last_device_error(h) == api.MOE_OK
+        got_rt = layer_routing_host(h, B, k, E)
+        out_h, y_h = to_host_u16(out), y.cpu().numpy()
+    finally:
+        api.moe_layer_destroy(h)
+    assert_routing_equal(got_rt, ref_rt, W_ABS)
+    hot = int(np.argmax(ref_rt["counts"]))
+    hot_tokens = sorted(set(np.nonzero((ref_rt["topk_idx"] == hot).any(1))[0].tolist()))
+    sample = sorted(set(hot_tokens[:3] + [0, 21, 42, 63]))
+    ref = oracle_layer_for(dl, x_h[sample], r_h[sample])
+    ok, info = bf16_close(out_h[sample], ref["out_bf16"])
+    assert ok, info
+    rows = np.concatenate([np.arange(b * k, (b + 1) * k) for b in sample])
+    ok, info = metric_close(y_h[rows], ref["y_routed"], Y_ROUTED_MAX_REL, Y_ROUTED_MEAN_REL)
+    assert ok, info
