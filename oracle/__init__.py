@@ -63,6 +63,9 @@ def lib():
         L.oracle_shared_ffn.argtypes = [vp, vp, vp, i32, i32, vp, vp]
         L.oracle_layer.argtypes = [i32] * 6 + [vp] * 11 + [i32] + [vp] * 13
         L.oracle_layer.restype = i32
+        L.oracle_layer_v.argtypes = [i32] * 6 + [vp] * 11 + [i32] + [vp] * 13 + [i32] + [vp] * 4
+        L.oracle_layer_v.restype = i32
+        L.oracle_topk_sigmoid.argtypes = [vp, vp, i32, i32, i32, vp, vp]
         _LIB = L
     return _LIB
 
@@ -114,6 +117,17 @@ def topk_softmax(logits, k):
     return idx, w
 
 
+def topk_sigmoid(logits, k, bias=None):
+    """Sigmoid scoring: select by sigmoid(l) + bias, weights sigmoid(l) / sum."""
+    lg = _c(logits, np.float64)
+    B, E = lg.shape
+    b = None if bias is None else _c(bias, np.float32)
+    idx = np.empty((B, k), dtype=np.int32)
+    w = np.empty((B, k), dtype=np.float64)
+    lib().oracle_topk_sigmoid(_p(lg), _p(b), B, E, k, _p(idx), _p(w))
+    return idx, w
+
+
 def bucket(topk_idx, E):
     idx = _c(topk_idx, np.int32)
     B, k = idx.shape
@@ -150,9 +164,12 @@ def shared_ffn(x, gu_bf16, d_bf16):
 
 
 def layer(x, residual, router_w, router_bias, gu_codes, gu_scales, d_codes, d_scales,
-          shared_gu, shared_d, top_k, experts=None, n_threads=1):
+          shared_gu, shared_d, top_k, experts=None, n_threads=1, scoring="softmax", shared_mx=None):
     """Whole layer.  Expert tensors are stacked by slot; `experts` lists the
-    expert id of each slot (None: slot i is expert i).  Returns a dict."""
+    expert id of each slot (None: slot i is expert i).  scoring: "softmax"
+    (default) or "sigmoid" (bias-corrected selection); shared_mx: MXFP4
+    shared expert (gu_codes, gu_scales, d_codes, d_scales) instead of the
+    bf16 shared_gu / shared_d.  Returns a dict."""
     x, residual = _c(x, np.uint16), _c(residual, np.uint16)
     wr = _c(router_w, np.uint16)
     B, H = x.shape
@@ -163,6 +180,11 @@ def layer(x, residual, router_w, router_bias, gu_codes, gu_scales, d_codes, d_sc
     sgu = None if shared_gu is None else _c(shared_gu, np.uint16)
     sd = None if shared_d is None else _c(shared_d, np.uint16)
     Is = 0 if sgu is None else sgu.shape[0] // 2
+    smx = None
+    if shared_mx is not None:
+        smx = tuple(_c(a, np.uint8) for a in shared_mx)
+        Is = smx[0].shape[0] // 2
+        sgu = sd = None
     bias = None if router_bias is None else _c(router_bias, np.float32)
     slot = None
     if experts is not None:
@@ -175,12 +197,14 @@ def layer(x, residual, router_w, router_bias, gu_codes, gu_scales, d_codes, d_sc
         n_active=np.empty(1, np.int32), h_routed=np.empty((B * k, I)),
         y_routed=np.empty((B * k, H)), y_shared=np.empty((B, H)), out=np.empty((B, H)),
         out_bf16=np.empty((B, H), np.uint16))
-    rc = lib().oracle_layer(
+    sc_id = {"softmax": 0, "sigmoid": 1}[scoring]
+    mx_ptrs = [None] * 4 if smx is None else [_p(a) for a in smx]
+    rc = lib().oracle_layer_v(
         B, H, E, k, I, Is, _p(x), _p(residual), _p(wr), _p(bias), _p(gc), _p(gs), _p(dc), _p(ds),
         _p(slot), _p(sgu), _p(sd), int(n_threads), _p(r["logits"]), _p(r["topk_idx"]),
         _p(r["topk_w"]), _p(r["counts"]), _p(r["offsets"]), _p(r["pair_ids"]), _p(r["active"]),
         _p(r["n_active"]), _p(r["h_routed"]), _p(r["y_routed"]), _p(r["y_shared"]), _p(r["out"]),
-        _p(r["out_bf16"]))
+        _p(r["out_bf16"]), sc_id, *mx_ptrs)
     if rc != 0:
         raise RuntimeError(f"oracle_layer failed: {rc}")
     na = int(r["n_active"][0])
@@ -189,10 +213,14 @@ def layer(x, residual, router_w, router_bias, gu_codes, gu_scales, d_codes, d_sc
     return r
 
 
-def routing(x, router_w, router_bias, top_k):
-    """Router, top-k, softmax and buckets only (cheap at every size)."""
-    lg = router_logits(x, router_w, router_bias)
-    idx, w = topk_softmax(lg, top_k)
+def routing(x, router_w, router_bias, top_k, scoring="softmax"):
+    """Router, top-k, weights and buckets only (cheap at every size)."""
+    if scoring == "sigmoid":
+        lg = router_logits(x, router_w, None)
+        idx, w = topk_sigmoid(lg, top_k, router_bias)
+    else:
+        lg = router_logits(x, router_w, router_bias)
+        idx, w = topk_softmax(lg, top_k)
     out = bucket(idx, np.asarray(router_w).shape[1])
     out.update(logits=lg, topk_idx=idx, topk_w=w)
     return out

@@ -20,7 +20,9 @@
 //   S_b          = the k largest logits, ties to the lower expert id,
 //                  listed in ascending expert id                  (top-k)
 //   w[b][j]      = exp(l_j - m) / sum_{i in S_b} exp(l_i - m)     (softmax
-//                  over the selected logits, m = their maximum)
+//                  over the selected logits, m = their maximum; the
+//                  sigmoid variant: s = sigmoid(l), selection by s + bias,
+//                  w = s_j / sum of the selected s)
 //   buckets      = counting sort of the pairs (b, j) by expert    (bucketing)
 //   g = Wg x, u = Wu x, h = silu(g) * u, y = Wd h                 (SwiGLU
 //                  expert; MXFP4 weights dequantised exactly)
@@ -158,6 +160,35 @@ void oracle_topk_softmax(const double* logits, int B, int E, int k, int32_t* idx
   }
 }
 
+// Sigmoid scoring with a selection bias (the bias-corrected router variant):
+// s_e = 1 / (1 + e^-l_e) from the raw logits; the k experts with the largest
+// s_e + bias_e are selected (equal values to the lower id; bias NULL = 0),
+// listed in ascending id, with weights s_j / sum of the selected s -- the
+// bias steers the choice only.
+void oracle_topk_sigmoid(const double* logits, const float* bias, int B, int E, int k, int32_t* idx, double* w) {
+  std::vector<Pair> p(E);
+  std::vector<double> sc(E);
+  for (int b = 0; b < B; ++b) {
+    for (int e = 0; e < E; ++e) {
+      sc[e] = 1.0 / (1.0 + std::exp(-logits[(size_t)b * E + e]));
+      p[e] = Pair{sc[e] + (bias ? (double)bias[e] : 0.0), e};
+    }
+    std::sort(p.begin(), p.end(), [](const Pair& a, const Pair& c) {
+      if (a.logit != c.logit) return a.logit > c.logit;
+      return a.expert < c.expert;
+    });
+    std::vector<int> sel(k);
+    for (int j = 0; j < k; ++j) sel[j] = p[j].expert;
+    std::sort(sel.begin(), sel.end());
+    double z = 0.0;
+    for (int j = 0; j < k; ++j) z += sc[sel[j]];
+    for (int j = 0; j < k; ++j) {
+      idx[(size_t)b * k + j] = sel[j];
+      w[(size_t)b * k + j] = sc[sel[j]] / z;
+    }
+  }
+}
+
 // Counting sort of pairs p = b*k + j by expert: counts[E], offsets[E+1]
 // (exclusive scan), pair_ids[B*k] ordered by (expert, b, j), the ascending
 // list of experts with a nonzero count and its length.
@@ -223,15 +254,27 @@ void oracle_shared_ffn(const double* x, const uint16_t* gu, const uint16_t* d, i
 // d_codes [slots][H][I/2], d_scales [slots][H][I/32]; expert_slot NULL means
 // slot = e.  Every output pointer may be NULL.  Returns 0, or -1 when a
 // selected expert has no slot, -2 on bad sizes.
-int oracle_layer(int B, int H, int E, int k, int I, int Is, const uint16_t* x, const uint16_t* residual,
-                 const uint16_t* router_w, const float* router_bias, const uint8_t* gu_codes,
-                 const uint8_t* gu_scales, const uint8_t* d_codes, const uint8_t* d_scales,
-                 const int32_t* expert_slot, const uint16_t* shared_gu, const uint16_t* shared_d,
-                 int n_threads, double* logits_out, int32_t* topk_idx_out, double* topk_w_out,
-                 int32_t* counts, int32_t* offsets, int32_t* pair_ids, int32_t* active,
-                 int32_t* n_active, double* h_routed, double* y_routed, double* y_shared,
-                 double* out, uint16_t* out_bf16) {
+//
+// Variants (scoring, shared expert format): scoring 0 = softmax over the
+// selected logits, the bias added to the logits first (as above); scoring 1
+// = oracle_topk_sigmoid on the raw logits, the bias steering selection only
+// (logits_out then holds the raw logits).  The shared expert is either bf16
+// (shared_gu / shared_d) or, when shared_mx_gu_codes is non-NULL, MXFP4
+// tensors of the routed experts' layout: gate/up codes [2Is][H/2], scales
+// [2Is][H/32], down codes [H][Is/2], scales [H][Is/32], dequantised exactly.
+int oracle_layer_v(int B, int H, int E, int k, int I, int Is, const uint16_t* x, const uint16_t* residual,
+                   const uint16_t* router_w, const float* router_bias, const uint8_t* gu_codes,
+                   const uint8_t* gu_scales, const uint8_t* d_codes, const uint8_t* d_scales,
+                   const int32_t* expert_slot, const uint16_t* shared_gu, const uint16_t* shared_d,
+                   int n_threads, double* logits_out, int32_t* topk_idx_out, double* topk_w_out,
+                   int32_t* counts, int32_t* offsets, int32_t* pair_ids, int32_t* active,
+                   int32_t* n_active, double* h_routed, double* y_routed, double* y_shared,
+                   double* out, uint16_t* out_bf16, int scoring, const uint8_t* shared_mx_gu_codes,
+                   const uint8_t* shared_mx_gu_scales, const uint8_t* shared_mx_d_codes,
+                   const uint8_t* shared_mx_d_scales) {
   if (B <= 0 || H <= 0 || E <= 0 || k <= 0 || k > E || I <= 0 || H % 32 || I % 32 || Is < 0) return -2;
+  if (scoring != 0 && scoring != 1) return -2;
+  if (shared_mx_gu_codes && Is % 32) return -2;
 #ifdef _OPENMP
   if (n_threads > 0) omp_set_num_threads(n_threads);
 #else
@@ -239,8 +282,13 @@ int oracle_layer(int B, int H, int E, int k, int I, int Is, const uint16_t* x, c
 #endif
   std::vector<double> logits((size_t)B * E), w((size_t)B * k);
   std::vector<int32_t> idx((size_t)B * k);
-  oracle_router_logits(x, router_w, router_bias, B, H, E, logits.data());
-  oracle_topk_softmax(logits.data(), B, E, k, idx.data(), w.data());
+  if (scoring == 0) {
+    oracle_router_logits(x, router_w, router_bias, B, H, E, logits.data());
+    oracle_topk_softmax(logits.data(), B, E, k, idx.data(), w.data());
+  } else {
+    oracle_router_logits(x, router_w, nullptr, B, H, E, logits.data());
+    oracle_topk_sigmoid(logits.data(), router_bias, B, E, k, idx.data(), w.data());
+  }
   for (int p = 0; p < B * k; ++p) {
     const int e = idx[p];
     const int slot = expert_slot ? expert_slot[e] : e;
@@ -290,7 +338,35 @@ int oracle_layer(int B, int H, int E, int k, int I, int Is, const uint16_t* x, c
   }
   // Shared expert, same structure.
   std::vector<double> ys((size_t)B * H, 0.0);
-  if (Is > 0 && shared_gu && shared_d) {
+  if (Is > 0 && shared_mx_gu_codes) {
+    // MXFP4 shared expert: every token, weight 1, exact dequantisation
+    std::vector<double> hs((size_t)B * Is);
+#pragma omp parallel for schedule(dynamic, 16)
+    for (long long bi = 0; bi < (long long)B * Is; ++bi) {
+      const int b = (int)(bi / Is), i = (int)(bi % Is);
+      const double* xb = xd.data() + (size_t)b * H;
+      std::vector<double> row(H);
+      dequant_row(shared_mx_gu_codes + (size_t)i * (H / 2), shared_mx_gu_scales + (size_t)i * (H / 32), H,
+                  row.data());
+      double g = 0.0;
+      for (int c = 0; c < H; ++c) g += row[c] * xb[c];
+      dequant_row(shared_mx_gu_codes + (size_t)(Is + i) * (H / 2), shared_mx_gu_scales + (size_t)(Is + i) * (H / 32),
+                  H, row.data());
+      double u = 0.0;
+      for (int c = 0; c < H; ++c) u += row[c] * xb[c];
+      hs[bi] = silu(g) * u;
+    }
+#pragma omp parallel for schedule(dynamic, 64)
+    for (long long br = 0; br < (long long)B * H; ++br) {
+      const int b = (int)(br / H), r = (int)(br % H);
+      std::vector<double> row(Is);
+      dequant_row(shared_mx_d_codes + (size_t)r * (Is / 2), shared_mx_d_scales + (size_t)r * (Is / 32), Is,
+                  row.data());
+      double acc = 0.0;
+      for (int i = 0; i < Is; ++i) acc += row[i] * hs[(size_t)b * Is + i];
+      ys[br] = acc;
+    }
+  } else if (Is > 0 && shared_gu && shared_d) {
     std::vector<double> hs((size_t)B * Is);
 #pragma omp parallel for schedule(dynamic, 16)
     for (long long bi = 0; bi < (long long)B * Is; ++bi) {
@@ -324,6 +400,21 @@ int oracle_layer(int B, int H, int E, int k, int I, int Is, const uint16_t* x, c
       if (out_bf16) out_bf16[(size_t)b * H + r] = round_bf16(o);
     }
   return 0;
+}
+
+// The layer with the default variants: softmax scoring, bf16 shared expert.
+int oracle_layer(int B, int H, int E, int k, int I, int Is, const uint16_t* x, const uint16_t* residual,
+                 const uint16_t* router_w, const float* router_bias, const uint8_t* gu_codes,
+                 const uint8_t* gu_scales, const uint8_t* d_codes, const uint8_t* d_scales,
+                 const int32_t* expert_slot, const uint16_t* shared_gu, const uint16_t* shared_d,
+                 int n_threads, double* logits_out, int32_t* topk_idx_out, double* topk_w_out,
+                 int32_t* counts, int32_t* offsets, int32_t* pair_ids, int32_t* active,
+                 int32_t* n_active, double* h_routed, double* y_routed, double* y_shared,
+                 double* out, uint16_t* out_bf16) {
+  return oracle_layer_v(B, H, E, k, I, Is, x, residual, router_w, router_bias, gu_codes, gu_scales, d_codes,
+                        d_scales, expert_slot, shared_gu, shared_d, n_threads, logits_out, topk_idx_out, topk_w_out,
+                        counts, offsets, pair_ids, active, n_active, h_routed, y_routed, y_shared, out, out_bf16, 0,
+                        nullptr, nullptr, nullptr, nullptr);
 }
 
 }  // extern "C"

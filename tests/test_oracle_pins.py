@@ -375,3 +375,83 @@ def test_layer_special_cases():
     rc = oracle.layer(a["x"], a["res"], a["wr"], None, a["gc"][sel], a["gs"][sel], a["dc"][sel],
                       a["ds"][sel], a["sgu"], a["sd"], k, experts=sel)
     assert np.array_equal(rc["out"], base["out"])
+
+
+# ------------------------------------------- router and shared variants ----
+def test_sigmoid_topk_brute_force_with_bias_and_ties():
+    """Sigmoid scoring: the selected set maximises sum(sigmoid(l) + bias) over
+    all k-subsets (lower ids win ties), whatever the bias does to the order."""
+    rng = np.random.default_rng(91)
+    for E, k in ((8, 2), (10, 3), (12, 4)):
+        for _ in range(30):
+            lg = rng.integers(-3, 4, size=(1, E)).astype(np.float64)
+            bias = (rng.integers(-2, 3, size=E) * 0.25).astype(np.float32)
+            idx, w = oracle.topk_sigmoid(lg, k, bias)
+            score = [1.0 / (1.0 + math.exp(-lg[0, e])) + float(bias[e]) for e in range(E)]
+            assert list(idx[0]) == brute_topk(score, k)
+            assert abs(w.sum() - 1.0) < 1e-12
+
+
+def test_sigmoid_weights_closed_forms():
+    # l = (0, ln 3): sigmoid = (1/2, 3/4) -> weights (2/5, 3/5)
+    idx, w = oracle.topk_sigmoid(np.array([[0.0, math.log(3.0)]]), 2)
+    assert list(idx[0]) == [0, 1]
+    assert abs(w[0, 0] - 0.4) < 1e-15 and abs(w[0, 1] - 0.6) < 1e-15
+    # the bias steers the choice but stays out of the weights: sigmoid(2.0) >
+    # sigmoid(1.9), yet +0.1 on expert 1 selects it, alone, with weight 1
+    idx, w = oracle.topk_sigmoid(np.array([[2.0, 1.9]]), 1, np.array([0.0, 0.1], np.float32))
+    assert list(idx[0]) == [1] and w[0, 0] == 1.0
+    # with k = 2 both are selected and the weights ignore the bias
+    idx, w = oracle.topk_sigmoid(np.array([[2.0, 1.9]]), 2, np.array([0.0, 0.1], np.float32))
+    s0, s1 = 1 / (1 + math.exp(-2.0)), 1 / (1 + math.exp(-1.9))
+    assert abs(w[0, 0] - s0 / (s0 + s1)) < 1e-15 and abs(w[0, 1] - s1 / (s0 + s1)) < 1e-15
+
+
+def test_sigmoid_without_bias_selects_like_softmax():
+    # sigmoid is increasing: without a bias both scorings select the same set
+    rng = np.random.default_rng(92)
+    lg = rng.normal(0, 2, size=(16, 40))
+    i1, _ = oracle.topk_sigmoid(lg, 6)
+    i2, _ = oracle.topk_softmax(lg, 6)
+    assert np.array_equal(i1, i2)
+
+
+def test_layer_sigmoid_scoring_matches_dense_formulation():
+    rng = np.random.default_rng(93)
+    B, H, E, k, I, Is = 3, 64, 6, 2, 32, 32
+    a = _tiny_layer_arrays(rng, B, H, E, k, I, Is, bias=True)
+    r = _run(a, k, scoring="sigmoid")
+    X = bf16_to_f32(a["x"]).astype(np.float64)
+    Wr = bf16_to_f32(a["wr"]).astype(np.float64)
+    lg = X @ Wr                                   # raw logits: the bias only steers
+    assert np.allclose(r["logits"], lg, rtol=0, atol=1e-12)
+    G = bf16_to_f32(a["sgu"]).astype(np.float64)
+    D = bf16_to_f32(a["sd"]).astype(np.float64)
+    for b in range(B):
+        s = 1.0 / (1.0 + np.exp(-lg[b]))
+        sel = sorted(brute_topk(list(s + a["bias"].astype(np.float64)), k))
+        assert list(r["topk_idx"][b]) == sel
+        acc = bf16_to_f32(a["res"][b]).astype(np.float64)
+        acc = acc + D @ (silu_np(G[:Is] @ X[b]) * (G[Is:] @ X[b]))
+        for e in sel:
+            h = silu_np(a["gu_vals"][e][:I] @ X[b]) * (a["gu_vals"][e][I:] @ X[b])
+            acc = acc + s[e] / s[sel].sum() * (a["d_vals"][e] @ h)
+        assert np.allclose(r["out"][b], acc, rtol=1e-12, atol=1e-12)
+
+
+def test_mxfp4_shared_expert_equals_bf16_copy_and_expert_ffn():
+    """An MXFP4 shared expert whose values are exact in bf16 gives the bf16
+    shared expert's result bit for bit, and equals the MXFP4 expert FFN."""
+    rng = np.random.default_rng(94)
+    B, H, E, k, I, Is = 2, 64, 4, 2, 32, 64
+    a = _tiny_layer_arrays(rng, B, H, E, k, I, Is)
+    gv, gc, gs = random_exact(rng, (2 * Is, H), s_choices=(119, 121, 123))
+    dv, dc, ds = random_exact(rng, (H, Is), s_choices=(119, 121, 123))
+    r_mx = _run(a, k, shared_mx=(gc, gs, dc, ds))
+    r_bf = _run(dict(a, sgu=bf16_rne(gv.astype(np.float32)), sd=bf16_rne(dv.astype(np.float32))), k)
+    assert np.array_equal(bf16_to_f32(bf16_rne(gv.astype(np.float32))).astype(np.float64), gv)
+    assert np.array_equal(r_mx["y_shared"], r_bf["y_shared"])
+    assert np.array_equal(r_mx["out"], r_bf["out"])
+    for b in range(B):
+        _, y = oracle.expert_ffn(bf16_to_f32(a["x"][b]).astype(np.float64), gc, gs, dc, ds)
+        assert np.array_equal(r_mx["y_shared"][b], y)
