@@ -87,6 +87,13 @@ typedef struct moe_layer* moe_layer_t; /* opaque, library-owned */
                                       on both); needs hidden and inter multiples of 128 and
                                       32-byte aligned expert codes, else moe_layer_create returns
                                       MOE_ERR_UNSUPPORTED */
+#define MOE_FLAG_ROUTER_SIGMOID 0x20u /* bias-corrected sigmoid router: scores s_e = 1/(1+e^-l_e)
+                                      from the raw logits, the k largest s_e + bias_e selected
+                                      (equal values to the lower id), weights s_j / sum of the
+                                      selected s (the bias steers the choice only).  Default:
+                                      softmax over the selected logits, bias added to the
+                                      logits first.  The pages do not state the scoring
+                                      function; this is the variant of DeepSeek-style routers */
 
 typedef struct {
   int hidden;       /* H: model width, multiple of 32 */
@@ -111,8 +118,16 @@ typedef struct {
   const uint8_t* s_gate_up;  /* E8M0 scales [E][2I][H/32] */
   const uint8_t* w_down;     /* E2M1 codes [E][H][I/2] */
   const uint8_t* s_down;     /* E8M0 scales [E][H][I/32] */
-  const void* shared_gate_up;/* bf16 [2*I_s][H]; rows 0..I_s-1 gate, then up (NULL if I_s = 0) */
-  const void* shared_down;   /* bf16 [H][I_s] (NULL if I_s = 0) */
+  const void* shared_gate_up;/* bf16 [2*I_s][H]; rows 0..I_s-1 gate, then up (NULL if I_s = 0
+                                or if the shared expert is given in MXFP4 below) */
+  const void* shared_down;   /* bf16 [H][I_s] (NULL as for shared_gate_up) */
+  /* The shared expert in MXFP4 instead (all four non-NULL, the two bf16
+   * pointers NULL, I_s > 0): the routed experts' layout for one expert.
+   * The pages do not say the shared expert's format; bf16 is the default. */
+  const uint8_t* shared_mx_gate_up;   /* E2M1 codes [2*I_s][H/2] */
+  const uint8_t* shared_mx_s_gate_up; /* E8M0 scales [2*I_s][H/32] */
+  const uint8_t* shared_mx_down;      /* E2M1 codes [H][I_s/2] */
+  const uint8_t* shared_mx_s_down;    /* E8M0 scales [H][I_s/32] */
 } moe_layer_weights;
 
 /* Routing plan of one call (DEVICE pointers).  Pair p = b*k + j names slot j

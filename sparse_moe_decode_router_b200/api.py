@@ -26,6 +26,7 @@ MOE_FLAG_SIDE_STREAM = 0x2
 MOE_FLAG_NO_PREFETCH = 0x4
 MOE_FLAG_NO_GROUPED = 0x8
 MOE_FLAG_MX_EXPERTS = 0x10
+MOE_FLAG_ROUTER_SIGMOID = 0x20
 
 # every entry point the header declares
 EXPORTS = (
@@ -55,7 +56,8 @@ class moe_layer_config(ctypes.Structure):
 class moe_layer_weights(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in (
         "router_w", "router_bias", "w_gate_up", "s_gate_up", "w_down", "s_down",
-        "shared_gate_up", "shared_down")]
+        "shared_gate_up", "shared_down", "shared_mx_gate_up", "shared_mx_s_gate_up",
+        "shared_mx_down", "shared_mx_s_down")]
 
 
 class moe_routing(ctypes.Structure):

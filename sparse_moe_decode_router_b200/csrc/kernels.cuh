@@ -86,6 +86,9 @@ struct GemvArgs {
   int ksplit;       // bf16 streams: warps of a group that split K (partial sums meet in shared memory)
   int pdl_late;     // dense stream whose activations are final at launch: no wait before
                    // reading them; every thread waits for the preceding grid at exit instead
+  int scoring;      // top-k: 0 = softmax over the selected logits (bias already in the
+                    // logits); 1 = sigmoid scores, selection by score + bias, weights
+                    // score / sum of the selected scores
   int* err;
 };
 
@@ -213,13 +216,18 @@ __global__ void __launch_bounds__(kTopkWarps * 32) topk_bucket_kernel(const Gemv
   const int PLs = (SL + 31) / 32;
   {
     uint32_t key[4];
-    float val[4];
+    float val[4];  // the value the weights are made of: the logit, or the sigmoid score
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       const int e = e0 + lane * PLs + i;
       const bool ok = i < PLs && lane * PLs + i < SL && e < E;
       val[i] = ok ? __ldcg(lg + e) : 0.f;
-      key[i] = ok ? logit_key(val[i]) : 0u;
+      if (a.scoring == 1) {
+        val[i] = 1.0f / (1.0f + expf(-val[i]));
+        key[i] = ok ? logit_key(val[i] + (a.bias ? __ldg(a.bias + e) : 0.f)) : 0u;
+      } else {
+        key[i] = ok ? logit_key(val[i]) : 0u;
+      }
     }
     const int kk = min(k, max(0, min(SL, E - e0)));
     const uint32_t sel = warp_select_topk<4>(key, kk, lane);
@@ -281,8 +289,9 @@ __global__ void __launch_bounds__(kTopkWarps * 32) topk_bucket_kernel(const Gemv
       if (lane >= o) pre += t;
     }
     pre -= ns;
-    // softmax over the selected logits in fp32 (m = largest selected logit);
-    // the xor butterfly adds commuted pairs, so every lane holds the same z
+    // softmax over the selected logits in fp32 (m = largest selected logit),
+    // or the selected sigmoid scores as they are; the xor butterfly adds
+    // commuted pairs, so every lane holds the same z
     float lmax = -INFINITY;
 #pragma unroll
     for (int i = 0; i < 8; ++i)
@@ -293,7 +302,7 @@ __global__ void __launch_bounds__(kTopkWarps * 32) topk_bucket_kernel(const Gemv
     float z = 0.f;
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-      ex[i] = ((sel >> i) & 1u) ? expf(val[i] - lmax) : 0.f;
+      ex[i] = ((sel >> i) & 1u) ? (a.scoring == 1 ? val[i] : expf(val[i] - lmax)) : 0.f;
       z += ex[i];
     }
 #pragma unroll

@@ -30,7 +30,8 @@ constexpr int kPrefetchBytes = 64 * 1024; // stages kept in flight ahead of the 
 
 size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
-enum Kind { K_ROUTER = 0, K_SGU = 1, K_SDN = 2, K_GU = 3, K_DN = 4, K_DNC = 5, K_NUM = 6 };
+enum Kind { K_ROUTER = 0, K_SGU = 1, K_SDN = 2, K_GU = 3, K_DN = 4, K_DNC = 5, K_SGU_MX = 6, K_SDN_MX = 7,
+            K_NUM = 8 };
 
 // Fixed per weight stream: weight format, epilogue, activation type, output
 // rows per warp row, warps per item, and how many of those warps split K
@@ -60,6 +61,9 @@ constexpr KindTraits kTraits[K_NUM] = {
     {W_MXFP4, EPI_SWIGLU, X_BF16, MOE_GU_RPW, MOE_GU_WPI, 1},       // routed gate/up: 4 output rows (2 x 14 KB)
     {W_MXFP4, EPI_STORE, X_F32, MOE_DN_RPW, MOE_DN_WPI, 1},         // routed down: 16 rows (16 KB)
     {W_MXFP4, EPI_DOWN_COMBINE, X_F32, MOE_DN_RPW, MOE_DN_WPI, 1},  // routed down + combine
+    // MXFP4 shared expert: the routed instances in dense mode (every token, one group)
+    {W_MXFP4, EPI_SWIGLU, X_BF16, MOE_GU_RPW, MOE_GU_WPI, 1},
+    {W_MXFP4, EPI_STORE, X_F32, MOE_DN_RPW, MOE_DN_WPI, 1},
 };
 
 struct GemvPlan {
@@ -172,8 +176,10 @@ GemvFn pick_fn(Kind k) {
     case K_SDN: return gemv_kernel<W_BF16, EPI_STORE, X_F32, TMAX, 2, KI>;
     // instances with a compile-time K and one token are the split-K ones
     case K_GU:
+    case K_SGU_MX:
       return gemv_kernel<W_MXFP4, EPI_SWIGLU, X_BF16, TMAX, (KH && TMAX == 1 && MOE_SPLITK_GU) ? kSplitKRows / 2 : MOE_GU_RPW, KH>;
     case K_DN:
+    case K_SDN_MX:
       return gemv_kernel<W_MXFP4, EPI_STORE, X_F32, TMAX, (KI && TMAX == 1 && kSplitDn) ? kSplitKRows : MOE_DN_RPW, KI>;
     case K_DNC:
       return gemv_kernel<W_MXFP4, EPI_DOWN_COMBINE, X_F32, TMAX,
@@ -244,6 +250,8 @@ struct moe_layer {
   bool pdl = true;
   bool side_stream = false;
   bool prefetch = true;
+  bool sigmoid = false;  // router scoring (MOE_FLAG_ROUTER_SIGMOID)
+  bool shared_mx = false; // the shared expert's weights are MXFP4
   char* arena = nullptr;
   uint16_t* wr_t = nullptr;  // router matrix, expert-major [E][H]
   float* logits = nullptr;
@@ -348,7 +356,7 @@ cudaError_t launch_router(moe_layer* L, const void* x, int B, const moe_routing&
   a.routed = 0;
   a.n_tokens = B;
   a.out = L->logits;
-  a.bias = L->w.router_bias;
+  a.bias = L->sigmoid ? nullptr : L->w.router_bias;  // sigmoid scoring: the bias steers selection only
   cudaError_t e = run_gemv(L, K_ROUTER, B, a, st, L->pdl);
   if (e != cudaSuccess) return e;
   GemvArgs t;
@@ -365,6 +373,8 @@ cudaError_t launch_router(moe_layer* L, const void* x, int B, const moe_routing&
   t.active_out = r.active;
   t.n_active_out = r.n_active;
   t.done_counter = L->router_cnt;
+  t.scoring = L->sigmoid ? 1 : 0;
+  t.bias = L->sigmoid ? L->w.router_bias : nullptr;
   return launch_ex(topk_bucket_kernel, B, kTopkWarps * 32, 0, st, L->pdl, t);
 }
 
@@ -373,26 +383,30 @@ cudaError_t launch_router(moe_layer* L, const void* x, int B, const moe_routing&
 cudaError_t launch_shared(moe_layer* L, const void* x, int B, float* ys, cudaStream_t st, bool pdl,
                           bool late = false) {
   const int H = L->cfg.hidden, Is = L->cfg.shared_inter;
+  const bool mx = L->shared_mx;
+  const Kind kgu = mx ? K_SGU_MX : K_SGU, kdn = mx ? K_SDN_MX : K_SDN;
   {
-    const GemvPlan& p = plan_of(L, K_SGU, B);
+    const GemvPlan& p = plan_of(L, kgu, B);
     GemvArgs a = base_args(L, p);
-    a.w = reinterpret_cast<const uint8_t*>(L->w.shared_gate_up);
+    a.w = mx ? L->w.shared_mx_gate_up : reinterpret_cast<const uint8_t*>(L->w.shared_gate_up);
+    a.sc = mx ? L->w.shared_mx_s_gate_up : nullptr;
     a.up_off = Is;
     a.act = x;
     a.n_tokens = B;
     a.out = L->hs;
     a.pdl_late = late && pdl ? 1 : 0;
-    cudaError_t e = run_gemv(L, K_SGU, B, a, st, pdl);
+    cudaError_t e = run_gemv(L, kgu, B, a, st, pdl);
     if (e != cudaSuccess) return e;
   }
-  const GemvPlan& p = plan_of(L, K_SDN, B);
+  const GemvPlan& p = plan_of(L, kdn, B);
   GemvArgs a = base_args(L, p);
-  a.w = reinterpret_cast<const uint8_t*>(L->w.shared_down);
+  a.w = mx ? L->w.shared_mx_down : reinterpret_cast<const uint8_t*>(L->w.shared_down);
+  a.sc = mx ? L->w.shared_mx_s_down : nullptr;
   a.act = L->hs;
   a.n_tokens = B;
   a.out = ys;
   (void)H;
-  return run_gemv(L, K_SDN, B, a, st, pdl);
+  return run_gemv(L, kdn, B, a, st, pdl);
 }
 
 GemvArgs routed_args(const moe_layer* L, const GemvPlan& p, const moe_routing& r, int B) {
@@ -774,11 +788,20 @@ moe_status_t moe_layer_create(const moe_layer_config* cfg, const moe_layer_weigh
       c.top_k > kMaxTopK || c.top_k > c.n_experts || c.max_batch < 1 || c.max_batch > kMaxBatch)
     return MOE_ERR_INVALID_ARG;
   if (!w->router_w || !w->w_gate_up || !w->s_gate_up || !w->w_down || !w->s_down) return MOE_ERR_INVALID_ARG;
-  if (c.shared_inter > 0 && (!w->shared_gate_up || !w->shared_down)) return MOE_ERR_INVALID_ARG;
+  const bool smx = w->shared_mx_gate_up != nullptr;
+  if (smx && (!w->shared_mx_s_gate_up || !w->shared_mx_down || !w->shared_mx_s_down || w->shared_gate_up ||
+              w->shared_down || c.shared_inter <= 0))
+    return MOE_ERR_INVALID_ARG;
+  if (c.shared_inter > 0 && !smx && (!w->shared_gate_up || !w->shared_down)) return MOE_ERR_INVALID_ARG;
+  if (smx) {
+    const void* sp[] = {w->shared_mx_gate_up, w->shared_mx_s_gate_up, w->shared_mx_down, w->shared_mx_s_down};
+    for (const void* p : sp)
+      if (!aligned16(p)) return MOE_ERR_INVALID_ARG;
+  }
   const void* ptrs[] = {w->router_w, w->w_gate_up, w->s_gate_up, w->w_down, w->s_down};
   for (const void* p : ptrs)
     if (!aligned16(p)) return MOE_ERR_INVALID_ARG;
-  if (c.shared_inter > 0 && (!aligned16(w->shared_gate_up) || !aligned16(w->shared_down)))
+  if (c.shared_inter > 0 && !smx && (!aligned16(w->shared_gate_up) || !aligned16(w->shared_down)))
     return MOE_ERR_INVALID_ARG;
 
   int dev = 0;
@@ -798,6 +821,8 @@ moe_status_t moe_layer_create(const moe_layer_config* cfg, const moe_layer_weigh
   L->pdl = !(c.flags & MOE_FLAG_NO_PDL);
   L->side_stream = (c.flags & MOE_FLAG_SIDE_STREAM) != 0;
   L->prefetch = !(c.flags & MOE_FLAG_NO_PREFETCH);
+  L->sigmoid = (c.flags & MOE_FLAG_ROUTER_SIGMOID) != 0;
+  L->shared_mx = smx;
 
   const int H = c.hidden, E = c.n_experts, k = c.top_k, I = c.inter, Is = c.shared_inter, MB = c.max_batch;
   // plans: [0] for B = 1 (one token per pass), [1] for B > 1 (two per pass)
@@ -821,12 +846,13 @@ moe_status_t moe_layer_create(const moe_layer_config* cfg, const moe_layer_weigh
     L->plans[K_GU][t] = make_plan(K_GU, H, I, nb, maxg, nb, (long long)2 * I * (H / 32), sms, fh);
     L->plans[K_DN][t] = make_plan(K_DN, I, H, nb * k, maxg, nb, (long long)H * (I / 32), sms, fi, sk);
     L->plans[K_DNC][t] = make_plan(K_DNC, I, H, nb * k, maxg, nb, (long long)H * (I / 32), sms, fi, sk);
+    const Kind kgu = smx ? K_SGU_MX : K_SGU, kdn = smx ? K_SDN_MX : K_SDN;
     if (Is > 0) {
-      L->plans[K_SGU][t] = make_plan(K_SGU, H, Is, nb, 1, nb, 0, sms, fh);
-      L->plans[K_SDN][t] = make_plan(K_SDN, Is, H, nb, 1, nb, 0, sms, fis);
+      L->plans[kgu][t] = make_plan(kgu, H, Is, nb, 1, nb, smx ? (long long)2 * Is * (H / 32) : 0, sms, fh);
+      L->plans[kdn][t] = make_plan(kdn, Is, H, nb, 1, nb, smx ? (long long)H * (Is / 32) : 0, sms, fis, sk);
     }
     bool ok = L->plans[K_ROUTER][t].ok && L->plans[K_GU][t].ok && L->plans[K_DN][t].ok && L->plans[K_DNC][t].ok;
-    if (Is > 0) ok = ok && L->plans[K_SGU][t].ok && L->plans[K_SDN][t].ok;
+    if (Is > 0) ok = ok && L->plans[kgu][t].ok && L->plans[kdn][t].ok;
     if (!ok) {
       delete L;
       return MOE_ERR_UNSUPPORTED;

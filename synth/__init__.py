@@ -87,6 +87,8 @@ T_EXPERT_D = 7
 T_ZIPF_PERM = 8
 T_TIES = 9
 T_EDGE = 10
+T_SHARED_MX_GU = 11
+T_SHARED_MX_D = 12
 
 # Irwin-Hall(4) of 16-bit uniforms: S = sum - 2*65535, Var(S) = 4*(65536^2-1)/12
 IH_SD = math.sqrt(4.0 * (65536.0 * 65536.0 - 1.0) / 12.0)
@@ -198,6 +200,8 @@ class MoEConfig:
     shared_sigma: float = 0.02
     act_sigma: float = 1.0
     min_gap: float = 1e-3        # logit gap between the k-th and (k+1)-th expert
+    scoring: str = "softmax"     # "sigmoid": the gap is taken on sigmoid(logit) + bias
+    shared_format: str = "bf16"  # "mxfp4": the shared expert quantised like the routed ones
 
     def with_(self, **kw) -> "MoEConfig":
         return replace(self, **kw)
@@ -281,8 +285,10 @@ def gen_router_bias(cfg, layer=0):
     return (-cfg.zipf_s * np.log(rank.astype(np.float64))).astype(np.float32)
 
 
-def _logit_gap(x_bf16_row, wr_f64, bias, k):
+def _logit_gap(x_bf16_row, wr_f64, bias, k, scoring="softmax"):
     lg = bf16_to_f32(x_bf16_row).astype(np.float64) @ wr_f64
+    if scoring == "sigmoid":
+        lg = 1.0 / (1.0 + np.exp(-lg))
     if bias is not None:
         lg = lg + bias.astype(np.float64)
     if k >= lg.shape[0]:
@@ -296,7 +302,8 @@ def gen_tokens(cfg, router_w_bf16, bias, token_ids, layer=0, max_attempts=64, ti
     substream (X, layer; sub0 = t, sub1 = attempt); a draw whose fp64 router
     logits (plus bias) put less than cfg.min_gap between the k-th and
     (k+1)-th largest is redrawn with the next attempt number, so that the
-    selected expert set is decided with margin (input conditioning only).
+    selected expert set is decided with margin (input conditioning only;
+    with cfg.scoring == "sigmoid" the margin is on sigmoid(logit) + bias).
     tiny_every > 0 multiplies every tiny_every-th element of each draw by
     2^tiny_exp (exact in fp32) before the bf16 rounding, so that a row mixes
     elements some 2^30 apart in magnitude."""
@@ -310,7 +317,7 @@ def gen_tokens(cfg, router_w_bf16, bias, token_ids, layer=0, max_attempts=64, ti
             if tiny_every > 0:
                 v[::tiny_every] *= np.float32(2.0 ** tiny_exp)
             row = bf16_rne(v)
-            if _logit_gap(row, wr, bias, cfg.top_k) >= cfg.min_gap:
+            if _logit_gap(row, wr, bias, cfg.top_k, cfg.scoring) >= cfg.min_gap:
                 break
         else:
             raise RuntimeError(f"no draw with logit gap >= {cfg.min_gap} for token {t}")

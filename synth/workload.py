@@ -7,7 +7,8 @@ from dataclasses import dataclass
 
 import numpy as np
 
-from . import (T_EXPERT_D, T_EXPERT_GU, T_ROUTER_W, T_SHARED_D, T_SHARED_GU, MoEConfig,
+from . import (T_EXPERT_D, T_EXPERT_GU, T_ROUTER_W, T_SHARED_D, T_SHARED_GU, T_SHARED_MX_D, T_SHARED_MX_GU,
+               MoEConfig,
                dev_fill_bf16, dev_fill_mxfp4, gen_edge_mxfp4, gen_residual, gen_router_bias, gen_tokens,
                stream_key)
 
@@ -41,6 +42,7 @@ class DeviceLayer:
     shared_d: object      # bf16 [H][Is]
     router_w_host: np.ndarray
     bias_host: np.ndarray | None
+    shared_mx: tuple | None = None   # MXFP4 shared expert: (gu codes, gu scales, d codes, d scales)
 
     def host_experts(self, experts):
         """Host copies of the listed experts' packed tensors (slot order)."""
@@ -50,13 +52,20 @@ class DeviceLayer:
                      (self.gu_codes, self.gu_scales, self.d_codes, self.d_scales))
 
     def host_shared(self):
+        if self.shared_gu is None:
+            return None, None
         return to_host_u16(self.shared_gu), to_host_u16(self.shared_d)
+
+    def host_shared_mx(self):
+        return None if self.shared_mx is None else tuple(t.cpu().numpy() for t in self.shared_mx)
 
     def weights_struct(self):
         from sparse_moe_decode_router_b200.api import moe_layer_weights
         p = lambda t: None if t is None else t.data_ptr()
+        mx = self.shared_mx if self.shared_mx is not None else (None,) * 4
         return moe_layer_weights(p(self.router_w), p(self.router_bias), p(self.gu_codes), p(self.gu_scales),
-                                 p(self.d_codes), p(self.d_scales), p(self.shared_gu), p(self.shared_d))
+                                 p(self.d_codes), p(self.d_scales), p(self.shared_gu), p(self.shared_d),
+                                 *(p(t) for t in mx))
 
     def tokens(self, token_ids, tiny_every=0):
         """bf16 x for the given token ids (gap-conditioned), host and device;
@@ -80,8 +89,18 @@ def make_device_layer(cfg: MoEConfig, layer: int = 0, device="cuda") -> DeviceLa
                    cfg.expert_sigma)
     wr = torch.empty((H, E), dtype=torch.bfloat16, device=dev)
     dev_fill_bf16(wr.data_ptr(), H * E, stream_key(cfg.seed, layer, T_ROUTER_W), 0, 0, cfg.router_sigma)
-    sgu = sd = None
-    if Is > 0:
+    sgu = sd = smx = None
+    if Is > 0 and cfg.shared_format == "mxfp4":
+        smx = (torch.empty((1, 2 * Is, H // 2), dtype=torch.uint8, device=dev),
+               torch.empty((1, 2 * Is, H // 32), dtype=torch.uint8, device=dev),
+               torch.empty((1, H, Is // 2), dtype=torch.uint8, device=dev),
+               torch.empty((1, H, Is // 32), dtype=torch.uint8, device=dev))
+        dev_fill_mxfp4(smx[0].data_ptr(), smx[1].data_ptr(), 1, 2 * Is, H, stream_key(cfg.seed, layer, T_SHARED_MX_GU),
+                       0, cfg.shared_sigma)
+        dev_fill_mxfp4(smx[2].data_ptr(), smx[3].data_ptr(), 1, H, Is, stream_key(cfg.seed, layer, T_SHARED_MX_D),
+                       0, cfg.shared_sigma)
+        smx = tuple(t[0] for t in smx)
+    elif Is > 0:
         sgu = torch.empty((2 * Is, H), dtype=torch.bfloat16, device=dev)
         sd = torch.empty((H, Is), dtype=torch.bfloat16, device=dev)
         dev_fill_bf16(sgu.data_ptr(), 2 * Is * H, stream_key(cfg.seed, layer, T_SHARED_GU), 0, 0, cfg.shared_sigma)
@@ -89,7 +108,7 @@ def make_device_layer(cfg: MoEConfig, layer: int = 0, device="cuda") -> DeviceLa
     bias_host = gen_router_bias(cfg, layer)
     bias = None if bias_host is None else torch.from_numpy(bias_host).to(dev)
     torch.cuda.synchronize(dev)
-    return DeviceLayer(cfg, layer, wr, bias, gu_c, gu_s, d_c, d_s, sgu, sd, to_host_u16(wr), bias_host)
+    return DeviceLayer(cfg, layer, wr, bias, gu_c, gu_s, d_c, d_s, sgu, sd, to_host_u16(wr), bias_host, smx)
 
 
 def residual_tokens(cfg: MoEConfig, token_ids, layer: int = 0, device="cuda"):

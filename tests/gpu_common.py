@@ -86,12 +86,13 @@ def oracle_threads():
 def oracle_layer_for(dl, x_host, res_host):
     """The oracle on a device workload: routing first, then only the experts it selects."""
     c = dl.cfg
-    rt = oracle.routing(x_host, dl.router_w_host, dl.bias_host, c.top_k)
+    rt = oracle.routing(x_host, dl.router_w_host, dl.bias_host, c.top_k, scoring=c.scoring)
     sel = np.unique(rt["topk_idx"])
     gc, gs, dc, ds = dl.host_experts(sel)
     sgu, sd = dl.host_shared() if c.shared_inter > 0 else (None, None)
     return oracle.layer(x_host, res_host, dl.router_w_host, dl.bias_host, gc, gs, dc, ds, sgu, sd, c.top_k,
-                        experts=sel, n_threads=oracle_threads())
+                        experts=sel, n_threads=oracle_threads(), scoring=c.scoring,
+                        shared_mx=dl.host_shared_mx())
 
 
 __all__ = ["make_device_layer", "residual_tokens", "to_host_u16"]

@@ -61,13 +61,16 @@ def run_all_paths(torch, dl, B, max_batch=None, flags=0, token0=0, tiny_every=0)
     return got, ref
 
 
-def check_against_oracle(got, ref, shared=True):
+def check_against_oracle(got, ref, shared=True, shared_mx=False):
+    """shared_mx: the shared expert is MXFP4 and runs on the MXFP4 streaming
+    kernels, so its output gets the routed experts' tolerance."""
     assert_routing_equal(got["routing"], ref, W_ABS)
     assert_routing_equal(got["fused_routing"], ref, W_ABS)
     ok, info = metric_close(got["y"], ref["y_routed"], Y_ROUTED_MAX_REL, Y_ROUTED_MEAN_REL)
     assert ok, f"routed expert outputs: {info}"
     if shared:
-        ok, info = metric_close(got["ys"], ref["y_shared"], Y_MAX_REL, Y_MEAN_REL)
+        tol = (Y_ROUTED_MAX_REL, Y_ROUTED_MEAN_REL) if shared_mx else (Y_MAX_REL, Y_MEAN_REL)
+        ok, info = metric_close(got["ys"], ref["y_shared"], *tol)
         assert ok, f"shared expert output: {info}"
     ok, info = bf16_close(got["out_fused"], ref["out_bf16"])
     assert ok, f"layer output: {info}"
