@@ -9,12 +9,13 @@ a different expert set.  Weights and inputs are resident in HBM before the
 timed region; L2 is flushed (256 MiB write) between steps, outside the
 per-step CUDA events.  Prints one JSON line (rank 0).
 
-  python bench.py [--gpus N] [--steps K] [--warmup W] [--config 1|2|3|4] [--impl ours|reference]
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--config 1|2|3|5] [--impl ours|reference]
 
 With the default workload (the full-size batch-1 layer) on one GPU the line
-also carries `per_config`: the batch-8 and batch-64 (Zipf) layers through
-the same call, and the 4-layer x 64-step decode loop captured in one CUDA
-graph with and without the next-layer L2 prefetch.
+also carries `per_config`: the batch-8, batch-64 (Zipf) and speculative
+verify (8 correlated positions of one sequence) layers through the same
+call, and the 4-layer x 64-step decode loop captured in one CUDA graph with
+and without the next-layer L2 prefetch.
 
 --gpus N > 1 runs under torchrun as N independent replicas (the layer does
 not shard); value = the bytes all ranks moved / the slowest rank's time.
@@ -602,6 +603,7 @@ def run_ours(args, cfg):
         extra["per_config"] = {
             "full_b8": per_config_record(synth.CONFIGS[2], args.flags, 50, 5, peak, sampler),
             "full_b64_zipf": per_config_record(synth.CONFIGS[3], args.flags, 20, 3, peak, sampler),
+            "full_b8_verify": per_config_record(synth.CONFIGS[5], args.flags, 50, 5, peak, sampler),
             "full_stack4_b1_graph": {
                 "prefetch": stack_record(synth.CONFIGS[4], args.flags, 3, peak, sampler),
                 "no_prefetch": stack_record(synth.CONFIGS[4], args.flags | api.MOE_FLAG_NO_PREFETCH, 3, peak,

@@ -202,6 +202,7 @@ class MoEConfig:
     min_gap: float = 1e-3        # logit gap between the k-th and (k+1)-th expert
     scoring: str = "softmax"     # "sigmoid": the gap is taken on sigmoid(logit) + bias
     shared_format: str = "bf16"  # "mxfp4": the shared expert quantised like the routed ones
+    verify_corr: float = 0.0     # > 0: a batch is `batch` positions of one sequence (see gen_tokens)
 
     def with_(self, **kw) -> "MoEConfig":
         return replace(self, **kw)
@@ -228,6 +229,9 @@ CONFIGS = {
     3: MoEConfig("full_b64_zipf", 7168, 896, 16, 2048, 2048, 64, BASE_SEED + 3, zipf_s=1.1),
     4: MoEConfig("full_stack4_b1", 7168, 896, 16, 2048, 2048, 1, BASE_SEED + 4,
                  n_layers=4, n_steps=64),
+    # speculative-decoding verify step: 8 positions of one sequence (a token
+    # and its drafts), whose activations share most of their direction
+    5: MoEConfig("full_b8_verify", 7168, 896, 16, 2048, 2048, 8, BASE_SEED + 5, verify_corr=0.9),
 }
 
 
@@ -304,6 +308,10 @@ def gen_tokens(cfg, router_w_bf16, bias, token_ids, layer=0, max_attempts=64, ti
     (k+1)-th largest is redrawn with the next attempt number, so that the
     selected expert set is decided with margin (input conditioning only;
     with cfg.scoring == "sigmoid" the margin is on sigmoid(logit) + bias).
+    cfg.verify_corr = c > 0 makes a batch the positions of one sequence:
+    x = sqrt(c) * (the sequence's draw) + sqrt(1 - c) * (the token's draw),
+    in fp32, before the rounding (so the positions route to overlapping
+    experts, as a speculative-decoding verify step does).
     tiny_every > 0 multiplies every tiny_every-th element of each draw by
     2^tiny_exp (exact in fp32) before the bf16 rounding, so that a row mixes
     elements some 2^30 apart in magnitude."""
@@ -311,9 +319,18 @@ def gen_tokens(cfg, router_w_bf16, bias, token_ids, layer=0, max_attempts=64, ti
     wr = bf16_to_f32(router_w_bf16).astype(np.float64)
     out = np.empty((len(token_ids), cfg.hidden), dtype=np.uint16)
     attempts = np.zeros(len(token_ids), dtype=np.int32)
+    c_base = np.float32(math.sqrt(cfg.verify_corr))
+    c_own = np.float32(math.sqrt(1.0 - cfg.verify_corr))
     for i, t in enumerate(token_ids):
+        base = None
+        if cfg.verify_corr > 0:
+            # positions of one sequence: token t is position t % batch of
+            # sequence t // batch; all share that sequence's draw (sub1 = 2^20)
+            base = normal_f32(key, int(t) // cfg.batch, 1 << 20, 0, cfg.hidden, cfg.act_sigma)
         for a in range(max_attempts):
             v = normal_f32(key, int(t), a, 0, cfg.hidden, cfg.act_sigma)
+            if base is not None:
+                v = (c_base * base + c_own * v).astype(np.float32)
             if tiny_every > 0:
                 v[::tiny_every] *= np.float32(2.0 ** tiny_exp)
             row = bf16_rne(v)

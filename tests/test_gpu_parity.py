@@ -359,3 +359,14 @@ def test_mx_full_size_b64_zipf(torch_cuda, full_layers):
     rows = np.concatenate([np.arange(b * k, (b + 1) * k) for b in sample])
     ok, info = metric_close(y_h[rows], ref["y_routed"], Y_ROUTED_MAX_REL, Y_ROUTED_MEAN_REL)
     assert ok, info
+
+
+@pytest.mark.parametrize("flags", [0, MX], ids=["cuda_cores", "tcgen05"])
+def test_full_size_verify_b8_matches_oracle(torch_cuda, full_layers, flags):
+    """Speculative-decoding verify shape: 8 positions of one sequence whose
+    activations share most of their direction, so they route to far fewer
+    distinct experts than 8 independent tokens (about 40 of 128)."""
+    dl = full_layers(5)
+    got, ref = run_all_paths(torch_cuda, dl, 8, flags=flags)
+    check_against_oracle(got, ref)
+    assert ref["n_active"] < 64
