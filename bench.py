@@ -646,15 +646,21 @@ def run_ours(args, cfg):
 
 
 def launches_per_step(cfg, flags):
-    """Kernels of this library one moe_layer_forward launches: router GEMV and
-    top-k; the shared expert's gate/up and down; then, for batches of one to
-    eight (or with the grouped path off), routed gate/up and down+combine;
-    above eight, the grouped tensor-core path: an activation-staging kernel
-    and a grouped MMA kernel per projection, then the combine.  The grouped
-    path is taken when both reduction lengths are multiples of 256 (the
-    full-size and test shapes)."""
-    from sparse_moe_decode_router_b200.api import MOE_FLAG_NO_GROUPED
-    n = 2 + (2 if cfg.shared_inter > 0 else 0)
+    """Kernels of this library one moe_layer_forward launches: the router
+    (whose last CTA selects the top-k and builds the buckets, and which also
+    streams a bf16 shared expert's gate/up rows), the shared expert's down
+    projection (an MXFP4 shared expert: its gate/up and down); then the routed
+    experts: on the tcgen05 kernels (MOE_FLAG_MX_EXPERTS) the activation-term
+    kernel, gate/up and down+combine; for batches above eight (grouped path
+    on, both reduction lengths multiples of 256) the warp-MMA path: an
+    activation-staging kernel and a grouped MMA kernel per projection, then
+    the combine; otherwise the streaming gate/up and down+combine."""
+    from sparse_moe_decode_router_b200.api import MOE_FLAG_MX_EXPERTS, MOE_FLAG_NO_GROUPED
+    n = 1
+    if cfg.shared_inter > 0:
+        n += 2 if cfg.shared_format == "mxfp4" else 1
+    if flags & MOE_FLAG_MX_EXPERTS:
+        return n + 3
     grouped = (cfg.batch > 8 and not (flags & MOE_FLAG_NO_GROUPED) and cfg.hidden % 256 == 0
                and cfg.inter % 256 == 0)
     return n + (5 if grouped else 2)

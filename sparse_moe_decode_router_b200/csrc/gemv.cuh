@@ -460,6 +460,9 @@ __global__ void __launch_bounds__(((KT != 0 && WF == W_MXFP4 && TMAX == 1 &&
                                        : kMaxConsumerWarps) * 32 + 32,
                                   1) gemv_kernel(const GemvArgs a) {
   constexpr bool kSwiglu = (EPI == EPI_SWIGLU);
+  // router: expert rows, then (optionally) the shared expert's gate/up rows as
+  // extra items, then the top-k / weights / buckets in the last CTA
+  constexpr bool kRouter = (EPI == EPI_ROUTER);
   constexpr int NWR = kSwiglu ? 2 * RPW : RPW;  // weight rows per warp
   static_assert(NWR % 2 == 0, "rows are processed in pairs");
   // kFast: the split-K instance.  Lanes own one 32-element chunk each, a
@@ -518,7 +521,8 @@ __global__ void __launch_bounds__(((KT != 0 && WF == W_MXFP4 && TMAX == 1 &&
     if (tid == 0) atomicExch(a.err, kErrBadPlan);
     n_groups = n_groups < 0 ? 0 : a.n_experts;
   }
-  const int n_rt = a.out_rows / a.R;
+  const int n_router = a.out_rows / a.R;                   // router: items of expert rows
+  const int n_rt = n_router + (kRouter ? a.n_items2 : 0);  // ... then shared gate/up items
   const long long n_items = (long long)n_groups * n_rt;
   const long long lo = n_items * blockIdx.x / gridDim.x;
   const long long hi = n_items * (blockIdx.x + 1) / gridDim.x;
@@ -576,7 +580,14 @@ __global__ void __launch_bounds__(((KT != 0 && WF == W_MXFP4 && TMAX == 1 &&
           const uint32_t sb = (WF == W_MXFP4 && !sglobal) ? (uint32_t)(a.R * sblocks) : 0u;
           mbar_arrive_expect_tx(&full_bar[s], (kSwiglu ? 2u : 1u) * (cb + sb));
           const uint8_t* wg = a.w + (long long)grp * a.w_gstride;
-          bulk_g2s(st, wg + (size_t)r0 * rowbytes, cb, &full_bar[s], pol);
+          if (kRouter && rt >= n_router) {
+            // shared gate/up item: its gate row and up row (R = 2 rows of stage)
+            const int j2 = rt - n_router;
+            bulk_g2s(st, a.w2 + (size_t)j2 * rowbytes, (uint32_t)rowbytes, &full_bar[s], pol);
+            bulk_g2s(st + rowbytes, a.w2 + (size_t)(j2 + a.up_off2) * rowbytes, (uint32_t)rowbytes, &full_bar[s], pol);
+          } else {
+            bulk_g2s(st, wg + (size_t)r0 * rowbytes, cb, &full_bar[s], pol);
+          }
           if (kSwiglu) bulk_g2s(st + cb, wg + (size_t)(r0 + a.up_off) * rowbytes, cb, &full_bar[s], pol);
           if (WF == W_MXFP4 && !sglobal) {
             const uint8_t* sg = a.sc + (long long)grp * a.s_gstride;
@@ -957,7 +968,14 @@ __global__ void __launch_bounds__(((KT != 0 && WF == W_MXFP4 && TMAX == 1 &&
           const float g_or_y = __shfl_sync(0xFFFFFFFFu, mine, (rr * TMAX + t) * (32 / V) & 31);
           const float up = __shfl_sync(0xFFFFFFFFu, mine, ((RPW + rr) * TMAX + t) * (32 / V) & 31);
           (void)vi;
-          if (oi < nout && t < tp.n) {
+          if (kRouter && rt >= n_router) {
+            // shared gate/up item: stage row 0 is the gate row, row 1 the up row
+            const float second = __shfl_sync(0xFFFFFFFFu, mine, (TMAX + t) * (32 / V) & 31);
+            if (oi < TMAX && t < tp.n) {
+              const int orow_t = (t == 0) ? tp.orow[0] : tp.orow[TMAX - 1];
+              a.out2[(size_t)orow_t * a.n_items2 + (rt - n_router)] = g_or_y / (1.0f + expf(-g_or_y)) * second;
+            }
+          } else if (oi < nout && t < tp.n) {
             int et = tp.e[0], orow_t = tp.orow[0];
 #pragma unroll
             for (int q = 1; q < TMAX; ++q)
@@ -1000,6 +1018,32 @@ __global__ void __launch_bounds__(((KT != 0 && WF == W_MXFP4 && TMAX == 1 &&
         nprev = 0;
       }
       jglob += nit;
+    }
+  }
+
+  if constexpr (kRouter) {
+    if (a.topk_idx) {
+      // every CTA's logits are written: the last CTA to get here selects the
+      // top-k of every token (one warp per token), then builds the buckets
+      __syncthreads();
+      if (tid == 0) {
+        __threadfence();
+        s_flag[1] = (atomicAdd(a.done_counter, 1) == (int)gridDim.x - 1) ? 1 : 0;
+      }
+      __syncthreads();
+      if (s_flag[1]) {
+        __threadfence();
+        const int nw = blockDim.x >> 5;
+        for (int b = warp; b < a.n_tokens; b += nw) topk_token_warp(a, a.out, b, lane);
+        __threadfence();
+        __syncthreads();
+        // the stage ring is idle now: bucket scratch
+        unsigned long long* s_mask = reinterpret_cast<unsigned long long*>(stages);
+        int* s_off = reinterpret_cast<int*>(stages + 8 * kMaxExperts);
+        int* s_wsum = s_off + kMaxExperts;
+        bucket_block(a, a.n_tokens, tid, (int)blockDim.x, s_mask, s_off, s_wsum);
+        if (tid == 0) *a.done_counter = 0;
+      }
     }
   }
 

@@ -87,8 +87,16 @@ struct GemvArgs {
   int pdl_late;     // dense stream whose activations are final at launch: no wait before
                    // reading them; every thread waits for the preceding grid at exit instead
   int scoring;      // top-k: 0 = softmax over the selected logits (bias already in the
-                    // logits); 1 = sigmoid scores, selection by score + bias, weights
+                    // logits); 1 = sigmoid scores, selection by score + sel_bias, weights
                     // score / sum of the selected scores
+  const float* sel_bias;  // sigmoid scoring: the selection bias [E] (or null)
+  // router kernel: the shared expert's gate/up rows as extra items (same
+  // activation, same bf16 format): gate row i at w2 + i*rowbytes, up row at
+  // w2 + (i + up_off2)*rowbytes, h_s = silu(gate . x) * (up . x) into out2 [B][n_items2]
+  const uint8_t* w2;
+  float* out2;
+  int n_items2;
+  int up_off2;
   int* err;
 };
 
@@ -188,150 +196,78 @@ __device__ __forceinline__ uint32_t warp_select_topk(const uint32_t (&key)[PL], 
   return sel;
 }
 
-constexpr int kTopkWarps = 8;
+// ---------------------------------------------------------------------------
+// Routing finish inside the router kernel (its last CTA): one warp per token
+// selects the k largest scores of all E experts (lane l owns experts
+// [l*PL, l*PL + PL), PL = ceil(E/32) <= 32, ids ascending with the slot),
+// equal scores going to the lower id; then the weights (softmax over the
+// selected logits, or the selected sigmoid scores normalised), written in
+// ascending expert id.
+__device__ void topk_token_warp(const GemvArgs& a, const float* __restrict__ lg, int b, int lane) {
+  const int E = a.n_experts, k = a.top_k;
+  const int PL = (E + 31) / 32;
+  uint32_t key[32];
+  float val[32];
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    const int e = lane * PL + i;
+    const bool ok = i < PL && e < E;
+    float v = ok ? __ldcg(lg + (size_t)b * E + e) : 0.f;
+    if (a.scoring == 1) {
+      v = 1.0f / (1.0f + expf(-v));
+      key[i] = ok ? logit_key(v + (a.sel_bias ? __ldg(a.sel_bias + e) : 0.f)) : 0u;
+    } else {
+      key[i] = ok ? logit_key(v) : 0u;
+    }
+    val[i] = v;
+  }
+  const uint32_t sel = warp_select_topk<32>(key, k, lane);
+  const int ns = __popc(sel);
+  int pre = ns;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int t = __shfl_up_sync(0xFFFFFFFFu, pre, o);
+    if (lane >= o) pre += t;
+  }
+  pre -= ns;
+  float lmax = -INFINITY;
+#pragma unroll
+  for (int i = 0; i < 32; ++i)
+    if ((sel >> i) & 1u) lmax = fmaxf(lmax, val[i]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) lmax = fmaxf(lmax, __shfl_xor_sync(0xFFFFFFFFu, lmax, o));
+  float z = 0.f;
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    if ((sel >> i) & 1u) {
+      val[i] = a.scoring == 1 ? val[i] : expf(val[i] - lmax);
+      z += val[i];
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xFFFFFFFFu, z, o);
+  int pos = pre;
+#pragma unroll
+  for (int i = 0; i < 32; ++i)
+    if ((sel >> i) & 1u) {
+      a.topk_idx[b * k + pos] = lane * PL + i;
+      a.topk_w[b * k + pos] = val[i] / z;
+      ++pos;
+    }
+}
 
-// logits [B][E] fp32 -> topk_idx/topk_w [B][k] (ascending expert id), then the
-// last CTA to finish builds counts/offsets/pair_ids/active/n_active.
-__global__ void __launch_bounds__(kTopkWarps * 32) topk_bucket_kernel(const GemvArgs a) {
-  const int E = a.n_experts, k = a.top_k, B = a.n_tokens;
-  const int b = blockIdx.x;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  constexpr int NT = kTopkWarps * 32;
-  __shared__ uint32_t c_key[kTopkWarps * kMaxTopK];
-  __shared__ int c_id[kTopkWarps * kMaxTopK];
-  __shared__ float c_val[kTopkWarps * kMaxTopK];
-  __shared__ int c_n[kTopkWarps];
-  __shared__ int s_last;
-  __shared__ unsigned long long s_mask[kMaxExperts];
-  __shared__ int s_off[kMaxExperts];
-  __shared__ int s_wsum[kTopkWarps][2];
-  pdl_wait();
-  // Dependents may launch now: a dense kernel that reads only the layer input
-  // overlaps this latency-bound work; routed kernels wait for our completion.
-  pdl_launch_dependents();
-  const float* lg = a.out + (size_t)b * E;
-  // stage 1: warp w takes experts [w*SL, (w+1)*SL), SL = ceil(E/8) <= 128 (4 per lane)
-  const int SL = (E + kTopkWarps - 1) / kTopkWarps;
-  const int e0 = warp * SL;
-  const int PLs = (SL + 31) / 32;
-  {
-    uint32_t key[4];
-    float val[4];  // the value the weights are made of: the logit, or the sigmoid score
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int e = e0 + lane * PLs + i;
-      const bool ok = i < PLs && lane * PLs + i < SL && e < E;
-      val[i] = ok ? __ldcg(lg + e) : 0.f;
-      if (a.scoring == 1) {
-        val[i] = 1.0f / (1.0f + expf(-val[i]));
-        key[i] = ok ? logit_key(val[i] + (a.bias ? __ldg(a.bias + e) : 0.f)) : 0u;
-      } else {
-        key[i] = ok ? logit_key(val[i]) : 0u;
-      }
-    }
-    const int kk = min(k, max(0, min(SL, E - e0)));
-    const uint32_t sel = warp_select_topk<4>(key, kk, lane);
-    // write the slice's selection in ascending id order
-    const int ns = __popc(sel);
-    int pre = ns;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int t = __shfl_up_sync(0xFFFFFFFFu, pre, o);
-      if (lane >= o) pre += t;
-    }
-    pre -= ns;
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-      if ((sel >> i) & 1u) {
-        c_key[warp * kMaxTopK + pre] = key[i];
-        c_id[warp * kMaxTopK + pre] = e0 + lane * PLs + i;
-        c_val[warp * kMaxTopK + pre] = val[i];
-        ++pre;
-      }
-    if (lane == 31) c_n[warp] = pre;
-  }
+// Buckets of the B*k pairs from topk_idx (global, written by this block
+// before a __syncthreads): counts, exclusive offsets, pair ids sorted by
+// (expert, b, j), the active list.  nt threads (a multiple of 32, nt*4 >= E);
+// scratch: s_mask [E] u64, s_off [E] int, s_wsum [2*32] int.
+__device__ void bucket_block(const GemvArgs& a, int B, int tid, int nt, unsigned long long* s_mask, int* s_off,
+                             int* s_wsum) {
+  const int E = a.n_experts, k = a.top_k;
+  const int lane = tid & 31, warp = tid >> 5;
+  for (int e = tid; e < E; e += nt) s_mask[e] = 0ull;
   __syncthreads();
-  // stage 2: warp 0 merges the <= 8*k candidates (ids ascend with the index)
-  if (warp == 0) {
-    int base[kTopkWarps];
-    int n = 0;
-#pragma unroll
-    for (int w = 0; w < kTopkWarps; ++w) {
-      base[w] = n;
-      n += c_n[w];
-    }
-    const int PL = (n + 31) / 32;  // <= 8
-    uint32_t key[8];
-    int id[8];
-    float val[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int c = lane * PL + i;
-      key[i] = 0u;
-      id[i] = 0;
-      val[i] = 0.f;
-      if (i < PL && c < n) {
-        int w = 0;
-#pragma unroll
-        for (int q = 1; q < kTopkWarps; ++q)
-          if (c >= base[q]) w = q;
-        key[i] = c_key[w * kMaxTopK + (c - base[w])];
-        id[i] = c_id[w * kMaxTopK + (c - base[w])];
-        val[i] = c_val[w * kMaxTopK + (c - base[w])];
-      }
-    }
-    const uint32_t sel = warp_select_topk<8>(key, k, lane);
-    const int ns = __popc(sel);
-    int pre = ns;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int t = __shfl_up_sync(0xFFFFFFFFu, pre, o);
-      if (lane >= o) pre += t;
-    }
-    pre -= ns;
-    // softmax over the selected logits in fp32 (m = largest selected logit),
-    // or the selected sigmoid scores as they are; the xor butterfly adds
-    // commuted pairs, so every lane holds the same z
-    float lmax = -INFINITY;
-#pragma unroll
-    for (int i = 0; i < 8; ++i)
-      if ((sel >> i) & 1u) lmax = fmaxf(lmax, val[i]);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) lmax = fmaxf(lmax, __shfl_xor_sync(0xFFFFFFFFu, lmax, o));
-    float ex[8];
-    float z = 0.f;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      ex[i] = ((sel >> i) & 1u) ? (a.scoring == 1 ? val[i] : expf(val[i] - lmax)) : 0.f;
-      z += ex[i];
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xFFFFFFFFu, z, o);
-    int pos = pre;
-#pragma unroll
-    for (int i = 0; i < 8; ++i)
-      if ((sel >> i) & 1u) {
-        a.topk_idx[b * k + pos] = id[i];
-        a.topk_w[b * k + pos] = ex[i] / z;
-        c_id[pos] = id[i];  // this token's selection, for a single-CTA bucketing
-        ++pos;
-      }
-  }
+  for (int p = tid; p < B * k; p += nt) atomicOr(&s_mask[__ldcg(a.topk_idx + p)], 1ull << (p / k));
   __syncthreads();
-  // the last CTA (token) to finish buckets all pairs
-  if (gridDim.x > 1) {
-    __threadfence();
-    if (tid == 0) s_last = (atomicAdd(a.done_counter, 1) == (int)gridDim.x - 1);
-    __syncthreads();
-    if (!s_last) return;
-    __threadfence();
-  }
-  auto idx_of = [&](int p) { return gridDim.x > 1 ? __ldcg(a.topk_idx + p) : c_id[p]; };
-  for (int e = tid; e < E; e += NT) s_mask[e] = 0ull;
-  __syncthreads();
-  for (int p = tid; p < B * k; p += NT) atomicOr(&s_mask[idx_of(p)], 1ull << (p / k));
-  __syncthreads();
-  // counts, exclusive offsets and the active list: thread t owns experts [4t, 4t+4)
   int cnt[4], tc = 0, ta = 0;
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
@@ -340,7 +276,7 @@ __global__ void __launch_bounds__(kTopkWarps * 32) topk_bucket_kernel(const Gemv
     tc += cnt[i];
     ta += cnt[i] > 0;
   }
-  int ic = tc, ia = ta;  // inclusive warp scans
+  int ic = tc, ia = ta;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
     const int t1 = __shfl_up_sync(0xFFFFFFFFu, ic, o);
@@ -351,14 +287,14 @@ __global__ void __launch_bounds__(kTopkWarps * 32) topk_bucket_kernel(const Gemv
     }
   }
   if (lane == 31) {
-    s_wsum[warp][0] = ic;
-    s_wsum[warp][1] = ia;
+    s_wsum[2 * warp] = ic;
+    s_wsum[2 * warp + 1] = ia;
   }
   __syncthreads();
   int wc = 0, wa = 0;
   for (int w = 0; w < warp; ++w) {
-    wc += s_wsum[w][0];
-    wa += s_wsum[w][1];
+    wc += s_wsum[2 * w];
+    wa += s_wsum[2 * w + 1];
   }
   int off = wc + ic - tc, act = wa + ia - ta;
 #pragma unroll
@@ -372,18 +308,17 @@ __global__ void __launch_bounds__(kTopkWarps * 32) topk_bucket_kernel(const Gemv
       off += cnt[i];
     }
   }
-  if (tid == NT - 1) {
+  if (4 * tid < E && 4 * tid + 4 >= E) {  // the thread owning the last expert
     a.offsets_out[E] = off;
     *a.n_active_out = act;
   }
   __syncthreads();
-  for (int p = tid; p < B * k; p += NT) {
-    const int e = idx_of(p);
+  for (int p = tid; p < B * k; p += nt) {
+    const int e = __ldcg(a.topk_idx + p);
     const int bb = p / k;
     const unsigned long long below = (bb == 0) ? 0ull : (s_mask[e] & ((1ull << bb) - 1ull));
     a.pair_ids_out[s_off[e] + __popcll(below)] = p;
   }
-  if (tid == 0 && gridDim.x > 1) *a.done_counter = 0;
 }
 
 // Staged combine: out = bf16(residual + y_shared + sum_j w_j y_j), one thread per element.

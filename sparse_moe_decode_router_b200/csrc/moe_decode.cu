@@ -27,6 +27,7 @@ constexpr int kSmemBudget = 227 * 1024;  // dynamic shared memory per CTA (1 CTA
 constexpr int kMaxStages = kMaxStagesDev;
 constexpr int kXBudget = 64 * 1024;       // staged activation vectors
 constexpr int kPrefetchBytes = 64 * 1024; // stages kept in flight ahead of the consumers
+constexpr int kRouterBucketBytes = 8 * kMaxExperts + 4 * kMaxExperts + 4 * 64;  // s_mask, s_off, s_wsum
 
 size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
@@ -157,6 +158,9 @@ GemvPlan make_plan(Kind kind, int K, int out_rows, int slots_needed, int max_gro
   p.scales_global = sg ? 1 : 0;
   p.threads = (p.ncw + 1) * 32;
   p.smem = st_off + ns * stage;
+  // the router kernel's last CTA builds the buckets in its idle stage ring
+  if (kind == K_ROUTER) p.smem = std::max(p.smem, st_off + kRouterBucketBytes);
+  if (p.smem > kSmemBudget) return GemvPlan{};
   p.fast = fast;
   p.ksplit = splitk ? 1 : t.ks;
   return p;
@@ -347,8 +351,13 @@ bool routing_ok(const moe_routing* r) {
   return r && r->topk_idx && r->topk_w && r->counts && r->offsets && r->pair_ids && r->active && r->n_active;
 }
 
-// Router GEMV (logits, fp32) then top-k / softmax / bucketing, chained with PDL.
-cudaError_t launch_router(moe_layer* L, const void* x, int B, const moe_routing& r, cudaStream_t st) {
+// Router GEMV (logits, fp32) whose last CTA selects the top-k, computes the
+// weights and builds the buckets.  with_shared: the shared expert's bf16
+// gate/up rows ride along as extra items (same activation x), so the
+// routing finish overlaps the shared expert's weight stream; h_s lands in
+// L->hs.
+cudaError_t launch_router(moe_layer* L, const void* x, int B, const moe_routing& r, cudaStream_t st,
+                          bool with_shared = false) {
   const GemvPlan& p = plan_of(L, K_ROUTER, B);
   GemvArgs a = base_args(L, p);
   a.w = reinterpret_cast<const uint8_t*>(L->wr_t);
@@ -357,35 +366,33 @@ cudaError_t launch_router(moe_layer* L, const void* x, int B, const moe_routing&
   a.n_tokens = B;
   a.out = L->logits;
   a.bias = L->sigmoid ? nullptr : L->w.router_bias;  // sigmoid scoring: the bias steers selection only
-  cudaError_t e = run_gemv(L, K_ROUTER, B, a, st, L->pdl);
-  if (e != cudaSuccess) return e;
-  GemvArgs t;
-  std::memset(&t, 0, sizeof(t));
-  t.out = L->logits;
-  t.n_experts = L->cfg.n_experts;
-  t.top_k = L->cfg.top_k;
-  t.n_tokens = B;
-  t.topk_w = r.topk_w;
-  t.topk_idx = r.topk_idx;
-  t.counts = r.counts;
-  t.offsets_out = r.offsets;
-  t.pair_ids_out = r.pair_ids;
-  t.active_out = r.active;
-  t.n_active_out = r.n_active;
-  t.done_counter = L->router_cnt;
-  t.scoring = L->sigmoid ? 1 : 0;
-  t.bias = L->sigmoid ? L->w.router_bias : nullptr;
-  return launch_ex(topk_bucket_kernel, B, kTopkWarps * 32, 0, st, L->pdl, t);
+  a.scoring = L->sigmoid ? 1 : 0;
+  a.sel_bias = L->sigmoid ? L->w.router_bias : nullptr;
+  a.topk_w = r.topk_w;
+  a.topk_idx = r.topk_idx;
+  a.counts = r.counts;
+  a.offsets_out = r.offsets;
+  a.pair_ids_out = r.pair_ids;
+  a.active_out = r.active;
+  a.n_active_out = r.n_active;
+  a.done_counter = L->router_cnt;
+  if (with_shared) {
+    a.w2 = reinterpret_cast<const uint8_t*>(L->w.shared_gate_up);
+    a.out2 = L->hs;
+    a.n_items2 = L->cfg.shared_inter;
+    a.up_off2 = L->cfg.shared_inter;
+  }
+  return run_gemv(L, K_ROUTER, B, a, st, L->pdl);
 }
 
 // Shared expert: gate/up + SwiGLU, then down.  late: the gate/up kernel may
 // read x before its predecessor completes (see GemvArgs::pdl_late).
 cudaError_t launch_shared(moe_layer* L, const void* x, int B, float* ys, cudaStream_t st, bool pdl,
-                          bool late = false) {
+                          bool late = false, bool down_only = false) {
   const int H = L->cfg.hidden, Is = L->cfg.shared_inter;
   const bool mx = L->shared_mx;
   const Kind kgu = mx ? K_SGU_MX : K_SGU, kdn = mx ? K_SDN_MX : K_SDN;
-  {
+  if (!down_only) {
     const GemvPlan& p = plan_of(L, kgu, B);
     GemvArgs a = base_args(L, p);
     a.w = mx ? L->w.shared_mx_gate_up : reinterpret_cast<const uint8_t*>(L->w.shared_gate_up);
@@ -977,8 +984,7 @@ moe_status_t moe_layer_create(const moe_layer_config* cfg, const moe_layer_weigh
     e = raise_smem_limit(reinterpret_cast<const void*>(grouped_mma_kernel<true>), kSmemBudget);
     if (e == cudaSuccess) e = raise_smem_limit(reinterpret_cast<const void*>(grouped_mma_kernel<false>), kSmemBudget);
   }
-  const void* small_kernels[] = {reinterpret_cast<const void*>(topk_bucket_kernel),
-                                 reinterpret_cast<const void*>(mx_x_terms_kernel<kMxTerms>),
+  const void* small_kernels[] = {reinterpret_cast<const void*>(mx_x_terms_kernel<kMxTerms>),
                                  reinterpret_cast<const void*>(act_to_f16_kernel<false>),
                                  reinterpret_cast<const void*>(act_to_f16_kernel<true>),
                                  reinterpret_cast<const void*>(combine_kernel)};
@@ -1081,9 +1087,11 @@ moe_status_t moe_layer_forward(moe_layer_t L, moe_layer_t next, const void* x, c
     if (e == cudaSuccess) e = launch_shared(L, x, B, L->ys, L->side, false);
     if (e == cudaSuccess) e = cudaEventRecord(L->ev_join, L->side);
   }
-  if (e == cudaSuccess) e = launch_router(L, x, B, L->plan, st);
-  // the shared expert's gate/up reads only x: it starts while the top-k runs
-  if (e == cudaSuccess && has_shared && !fork) e = launch_shared(L, x, B, L->ys, st, L->pdl, true);
+  // the bf16 shared expert's gate/up rows stream inside the router kernel
+  const bool fuse_sgu = has_shared && !fork && !L->shared_mx;
+  if (e == cudaSuccess) e = launch_router(L, x, B, L->plan, st, fuse_sgu);
+  if (e == cudaSuccess && has_shared && !fork)
+    e = launch_shared(L, x, B, L->ys, st, L->pdl, true, /*down_only*/ fuse_sgu);
   if (e == cudaSuccess) e = launch_gate_up(L, x, B, L->plan, st, L->probe_start, L->probe_stop);
   if (e == cudaSuccess && fork) e = cudaStreamWaitEvent(st, L->ev_join, 0);
   if (e == cudaSuccess)
@@ -1189,24 +1197,16 @@ moe_status_t moe_router_topk_noalloc(const void* router_w_em, const float* route
   a.n_tokens = B;
   a.out = sc->logits;
   a.bias = router_bias;
+  a.topk_w = r->topk_w;
+  a.topk_idx = r->topk_idx;
+  a.counts = r->counts;
+  a.offsets_out = r->offsets;
+  a.pair_ids_out = r->pair_ids;
+  a.active_out = r->active;
+  a.n_active_out = r->n_active;
+  a.done_counter = &sc->done_counter;
   const int tm = tmax_for(B);
-  e = launch_ex(gemv_fn(K_ROUTER, tm), sms, p.threads, p.smem, st, false, a);
-  if (e != cudaSuccess) return MOE_ERR_CUDA;
-  GemvArgs t;
-  std::memset(&t, 0, sizeof(t));
-  t.out = sc->logits;
-  t.n_experts = n_experts;
-  t.top_k = top_k;
-  t.n_tokens = B;
-  t.topk_w = r->topk_w;
-  t.topk_idx = r->topk_idx;
-  t.counts = r->counts;
-  t.offsets_out = r->offsets;
-  t.pair_ids_out = r->pair_ids;
-  t.active_out = r->active;
-  t.n_active_out = r->n_active;
-  t.done_counter = &sc->done_counter;
-  return cuda_status(launch_ex(topk_bucket_kernel, B, kTopkWarps * 32, 0, st, true, t));
+  return cuda_status(launch_ex(gemv_fn(K_ROUTER, tm), sms, p.threads, p.smem, st, false, a));
 }
 
 moe_status_t moe_router_topk_noalloc_last_error(void) {

@@ -121,7 +121,9 @@ def test_failing_nvml_falls_back(monkeypatch):
     assert c["samples"] == 0 or c["source"].startswith("nvidia-smi")
 
 
-@pytest.mark.parametrize("cfg_id,flags,want", [(1, 0, 6), (2, 0, 6), (3, 0, 9), (3, 0x8, 6)])
+@pytest.mark.parametrize("cfg_id,flags,want", [(1, 0, 4), (2, 0, 4), (3, 0, 7), (3, 0x8, 4), (1, 0x10, 5),
+                                                (3, 0x10, 5)])
 def test_launches_per_step(cfg_id, flags, want):
     assert bench.launches_per_step(synth.CONFIGS[cfg_id], flags) == want
-    assert bench.launches_per_step(synth.CONFIGS[cfg_id].with_(shared_inter=0), flags) == want - 2
+    assert bench.launches_per_step(synth.CONFIGS[cfg_id].with_(shared_inter=0), flags) == want - 1
+    assert bench.launches_per_step(synth.CONFIGS[cfg_id].with_(shared_format="mxfp4"), flags) == want + 1
