@@ -87,6 +87,14 @@ typedef struct moe_layer* moe_layer_t; /* opaque, library-owned */
                                       on both); needs hidden and inter multiples of 128 and
                                       32-byte aligned expert codes, else moe_layer_create returns
                                       MOE_ERR_UNSUPPORTED */
+#define MOE_FLAG_PERSISTENT 0x40u    /* batch-1 moe_layer_forward as one cooperative kernel (one CTA
+                                      per SM, in-kernel grid barriers between the routing, the
+                                      experts and the combine; the pages' persistent kernels,
+                                      yeyulingfeng section 02).  Same results bit for bit as the
+                                      chained kernels; larger batches use the chain.  Needs a
+                                      bf16 (or no) shared expert and no side stream, else
+                                      moe_layer_create returns MOE_ERR_UNSUPPORTED; takes
+                                      precedence over MOE_FLAG_MX_EXPERTS at batch 1 */
 #define MOE_FLAG_ROUTER_SIGMOID 0x20u /* bias-corrected sigmoid router: scores s_e = 1/(1+e^-l_e)
                                       from the raw logits, the k largest s_e + bias_e selected
                                       (equal values to the lower id), weights s_j / sum of the

@@ -27,6 +27,7 @@ MOE_FLAG_NO_PREFETCH = 0x4
 MOE_FLAG_NO_GROUPED = 0x8
 MOE_FLAG_MX_EXPERTS = 0x10
 MOE_FLAG_ROUTER_SIGMOID = 0x20
+MOE_FLAG_PERSISTENT = 0x40
 
 # every entry point the header declares
 EXPORTS = (

@@ -453,12 +453,15 @@ struct TokenPass {
 // arguments).  Specialised instances unroll the chunk loop with constant
 // addressing and, for MXFP4, read the E8M0 scale bytes from global memory with
 // loads issued ahead of the stage wait (the stage then holds codes only).
+//
+// The body runs as a device function so that the persistent single-launch
+// layer can run several streams back to back in one kernel; a block may then
+// have more threads than this stream's plan uses: the extra warps leave at
+// once, and every barrier below counts only the plan's (ncw + 1) warps.
+constexpr int kBarAll = 15;  // named barrier over all of a stream's warps
+
 template <int WF, int EPI, int XK, int TMAX, int RPW, int KT>
-__global__ void __launch_bounds__(((KT != 0 && WF == W_MXFP4 && TMAX == 1 &&
-                                    (EPI == EPI_SWIGLU ? 2 * RPW : RPW) == kSplitKRows)
-                                       ? kMaxSplitKWarps
-                                       : kMaxConsumerWarps) * 32 + 32,
-                                  1) gemv_kernel(const GemvArgs a) {
+__device__ __forceinline__ void gemv_body(const GemvArgs& a, unsigned char* smem) {
   constexpr bool kSwiglu = (EPI == EPI_SWIGLU);
   // router: expert rows, then (optionally) the shared expert's gate/up rows as
   // extra items, then the top-k / weights / buckets in the last CTA
@@ -474,10 +477,10 @@ __global__ void __launch_bounds__(((KT != 0 && WF == W_MXFP4 && TMAX == 1 &&
   // chunks, fully unrolled, constant shared-memory offsets)
   constexpr bool kUnroll = kOneTokMx && !kFast;
   constexpr int KS = KT ? ((KT / 32) + 31) / 32 : 1;  // K slices of 32 chunks (= chunks per lane when unrolled)
-  extern __shared__ __align__(128) unsigned char smem[];
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int ncw = a.ncw;
+  if (warp > ncw) return;  // beyond this stream's plan (persistent layer only)
   const int K = KT ? KT : a.K;
   const bool sglobal = a.scales_global != 0;
   const int C = K >> 5;                                   // 32-element chunks per row
@@ -527,7 +530,8 @@ __global__ void __launch_bounds__(((KT != 0 && WF == W_MXFP4 && TMAX == 1 &&
   const long long lo = n_items * blockIdx.x / gridDim.x;
   const long long hi = n_items * (blockIdx.x + 1) / gridDim.x;
 
-  __syncthreads();  // barriers initialised
+  const int nthreads_all = (ncw + 1) * 32;
+  named_bar_sync(kBarAll, nthreads_all);  // barriers initialised
   // plan invariants (see the host planner): stages are a multiple of the warp
   // groups, and an item's rows are exactly what the group's warps cover
   const int kq_plan = kFast ? KS : ((WF == W_BF16 && a.ksplit > 1) ? a.ksplit : 1);
@@ -538,7 +542,6 @@ __global__ void __launch_bounds__(((KT != 0 && WF == W_MXFP4 && TMAX == 1 &&
   }
   // The producer lane builds the phase table and starts streaming at once; the
   // consumers wait for the table on named barrier 2 (the producer only arrives).
-  const int nthreads_all = (ncw + 1) * 32;
   if (producer) {
     if (lane == 0) {
       build_phases(a, lo, hi, n_rt, a.xcap, *pt);
@@ -1025,23 +1028,23 @@ __global__ void __launch_bounds__(((KT != 0 && WF == W_MXFP4 && TMAX == 1 &&
     if (a.topk_idx) {
       // every CTA's logits are written: the last CTA to get here selects the
       // top-k of every token (one warp per token), then builds the buckets
-      __syncthreads();
+      named_bar_sync(kBarAll, nthreads_all);
       if (tid == 0) {
         __threadfence();
         s_flag[1] = (atomicAdd(a.done_counter, 1) == (int)gridDim.x - 1) ? 1 : 0;
       }
-      __syncthreads();
+      named_bar_sync(kBarAll, nthreads_all);
       if (s_flag[1]) {
         __threadfence();
-        const int nw = blockDim.x >> 5;
+        const int nw = nthreads_all >> 5;
         for (int b = warp; b < a.n_tokens; b += nw) topk_token_warp(a, a.out, b, lane);
         __threadfence();
-        __syncthreads();
+        named_bar_sync(kBarAll, nthreads_all);
         // the stage ring is idle now: bucket scratch
         unsigned long long* s_mask = reinterpret_cast<unsigned long long*>(stages);
         int* s_off = reinterpret_cast<int*>(stages + 8 * kMaxExperts);
         int* s_wsum = s_off + kMaxExperts;
-        bucket_block(a, a.n_tokens, tid, (int)blockDim.x, s_mask, s_off, s_wsum);
+        bucket_block(a, a.n_tokens, tid, nthreads_all, kBarAll, s_mask, s_off, s_wsum);
         if (tid == 0) *a.done_counter = 0;
       }
     }
@@ -1070,6 +1073,16 @@ __global__ void __launch_bounds__(((KT != 0 && WF == W_MXFP4 && TMAX == 1 &&
     }
   }
 
+}
+
+template <int WF, int EPI, int XK, int TMAX, int RPW, int KT>
+__global__ void __launch_bounds__(((KT != 0 && WF == W_MXFP4 && TMAX == 1 &&
+                                    (EPI == EPI_SWIGLU ? 2 * RPW : RPW) == kSplitKRows)
+                                       ? kMaxSplitKWarps
+                                       : kMaxConsumerWarps) * 32 + 32,
+                                  1) gemv_kernel(const GemvArgs a) {
+  extern __shared__ __align__(128) unsigned char smem[];
+  gemv_body<WF, EPI, XK, TMAX, RPW, KT>(a, smem);
 }
 
 }  // namespace moe

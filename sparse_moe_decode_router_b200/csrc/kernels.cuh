@@ -257,17 +257,18 @@ __device__ void topk_token_warp(const GemvArgs& a, const float* __restrict__ lg,
 }
 
 // Buckets of the B*k pairs from topk_idx (global, written by this block
-// before a __syncthreads): counts, exclusive offsets, pair ids sorted by
-// (expert, b, j), the active list.  nt threads (a multiple of 32, nt*4 >= E);
+// before a barrier): counts, exclusive offsets, pair ids sorted by
+// (expert, b, j), the active list.  nt threads (a multiple of 32, nt*4 >= E)
+// meeting on named barrier `bar`;
 // scratch: s_mask [E] u64, s_off [E] int, s_wsum [2*32] int.
-__device__ void bucket_block(const GemvArgs& a, int B, int tid, int nt, unsigned long long* s_mask, int* s_off,
-                             int* s_wsum) {
+__device__ void bucket_block(const GemvArgs& a, int B, int tid, int nt, int bar, unsigned long long* s_mask,
+                             int* s_off, int* s_wsum) {
   const int E = a.n_experts, k = a.top_k;
   const int lane = tid & 31, warp = tid >> 5;
   for (int e = tid; e < E; e += nt) s_mask[e] = 0ull;
-  __syncthreads();
+  named_bar_sync(bar, nt);
   for (int p = tid; p < B * k; p += nt) atomicOr(&s_mask[__ldcg(a.topk_idx + p)], 1ull << (p / k));
-  __syncthreads();
+  named_bar_sync(bar, nt);
   int cnt[4], tc = 0, ta = 0;
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
@@ -290,7 +291,7 @@ __device__ void bucket_block(const GemvArgs& a, int B, int tid, int nt, unsigned
     s_wsum[2 * warp] = ic;
     s_wsum[2 * warp + 1] = ia;
   }
-  __syncthreads();
+  named_bar_sync(bar, nt);
   int wc = 0, wa = 0;
   for (int w = 0; w < warp; ++w) {
     wc += s_wsum[2 * w];
@@ -312,7 +313,7 @@ __device__ void bucket_block(const GemvArgs& a, int B, int tid, int nt, unsigned
     a.offsets_out[E] = off;
     *a.n_active_out = act;
   }
-  __syncthreads();
+  named_bar_sync(bar, nt);
   for (int p = tid; p < B * k; p += nt) {
     const int e = __ldcg(a.topk_idx + p);
     const int bb = p / k;

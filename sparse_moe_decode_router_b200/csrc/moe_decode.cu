@@ -18,6 +18,7 @@
 #include "kernels.cuh"
 #include "mma_grouped.cuh"
 #include "mx_umma.cuh"
+#include "persistent.cuh"
 
 using namespace moe;
 
@@ -256,6 +257,8 @@ struct moe_layer {
   bool prefetch = true;
   bool sigmoid = false;  // router scoring (MOE_FLAG_ROUTER_SIGMOID)
   bool shared_mx = false; // the shared expert's weights are MXFP4
+  int persist = 0;        // persistent batch-1 kernel: 0 off, 1 generic instance, 2 shape-specialised
+  int* grid_bar = nullptr;
   char* arena = nullptr;
   uint16_t* wr_t = nullptr;  // router matrix, expert-major [E][H]
   float* logits = nullptr;
@@ -356,8 +359,7 @@ bool routing_ok(const moe_routing* r) {
 // gate/up rows ride along as extra items (same activation x), so the
 // routing finish overlaps the shared expert's weight stream; h_s lands in
 // L->hs.
-cudaError_t launch_router(moe_layer* L, const void* x, int B, const moe_routing& r, cudaStream_t st,
-                          bool with_shared = false) {
+GemvArgs router_args(const moe_layer* L, const void* x, int B, const moe_routing& r, bool with_shared) {
   const GemvPlan& p = plan_of(L, K_ROUTER, B);
   GemvArgs a = base_args(L, p);
   a.w = reinterpret_cast<const uint8_t*>(L->wr_t);
@@ -382,7 +384,24 @@ cudaError_t launch_router(moe_layer* L, const void* x, int B, const moe_routing&
     a.n_items2 = L->cfg.shared_inter;
     a.up_off2 = L->cfg.shared_inter;
   }
-  return run_gemv(L, K_ROUTER, B, a, st, L->pdl);
+  return a;
+}
+
+cudaError_t launch_router(moe_layer* L, const void* x, int B, const moe_routing& r, cudaStream_t st,
+                          bool with_shared = false) {
+  return run_gemv(L, K_ROUTER, B, router_args(L, x, B, r, with_shared), st, L->pdl);
+}
+
+GemvArgs shared_down_args(const moe_layer* L, int B, float* ys) {
+  const bool mx = L->shared_mx;
+  const GemvPlan& p = plan_of(L, mx ? K_SDN_MX : K_SDN, B);
+  GemvArgs a = base_args(L, p);
+  a.w = mx ? L->w.shared_mx_down : reinterpret_cast<const uint8_t*>(L->w.shared_down);
+  a.sc = mx ? L->w.shared_mx_s_down : nullptr;
+  a.act = L->hs;
+  a.n_tokens = B;
+  a.out = ys;
+  return a;
 }
 
 // Shared expert: gate/up + SwiGLU, then down.  late: the gate/up kernel may
@@ -405,15 +424,8 @@ cudaError_t launch_shared(moe_layer* L, const void* x, int B, float* ys, cudaStr
     cudaError_t e = run_gemv(L, kgu, B, a, st, pdl);
     if (e != cudaSuccess) return e;
   }
-  const GemvPlan& p = plan_of(L, kdn, B);
-  GemvArgs a = base_args(L, p);
-  a.w = mx ? L->w.shared_mx_down : reinterpret_cast<const uint8_t*>(L->w.shared_down);
-  a.sc = mx ? L->w.shared_mx_s_down : nullptr;
-  a.act = L->hs;
-  a.n_tokens = B;
-  a.out = ys;
   (void)H;
-  return run_gemv(L, kdn, B, a, st, pdl);
+  return run_gemv(L, kdn, B, shared_down_args(L, B, ys), st, pdl);
 }
 
 GemvArgs routed_args(const moe_layer* L, const GemvPlan& p, const moe_routing& r, int B) {
@@ -586,8 +598,7 @@ cudaError_t launch_gate_up(moe_layer* L, const void* x, int B, const moe_routing
   return e;
 }
 
-cudaError_t launch_gate_up_streams(moe_layer* L, const void* x, int B, const moe_routing& r, cudaStream_t st) {
-  if (B > kGroupedMinBatch && L->grouped) return launch_grouped(L, true, B, r, x, L->h, st);
+GemvArgs gate_up_args(const moe_layer* L, const void* x, int B, const moe_routing& r) {
   const int H = L->cfg.hidden, I = L->cfg.inter;
   const GemvPlan& p = plan_of(L, K_GU, B);
   GemvArgs a = routed_args(L, p, r, B);
@@ -599,7 +610,12 @@ cudaError_t launch_gate_up_streams(moe_layer* L, const void* x, int B, const moe
   a.act = x;
   a.act_by_pair = 0;
   a.out = L->h;
-  return run_gemv(L, K_GU, B, a, st, L->pdl);
+  return a;
+}
+
+cudaError_t launch_gate_up_streams(moe_layer* L, const void* x, int B, const moe_routing& r, cudaStream_t st) {
+  if (B > kGroupedMinBatch && L->grouped) return launch_grouped(L, true, B, r, x, L->h, st);
+  return run_gemv(L, K_GU, B, gate_up_args(L, x, B, r), st, L->pdl);
 }
 
 // Grouped tensor-core projection (batch > 1): f16 copy of the activation
@@ -642,6 +658,8 @@ cudaError_t launch_grouped(moe_layer* L, bool gate_up, int B, const moe_routing&
 
 cudaError_t launch_combine(moe_layer* L, int B, const moe_routing& r, const float* y, const float* ys,
                            const void* residual, void* out, cudaStream_t st);
+GemvArgs down_args(const moe_layer* L, int B, const moe_routing& r, float* y, bool fused, const void* residual,
+                   void* out, const float* ys, const moe_layer* next);
 
 cudaError_t launch_down(moe_layer* L, int B, const moe_routing& r, float* y, bool fused, const void* residual,
                         void* out, const float* ys, moe_layer* next, cudaStream_t st, bool pdl) {
@@ -657,6 +675,12 @@ cudaError_t launch_down(moe_layer* L, int B, const moe_routing& r, float* y, boo
     (void)pdl;
     return e;
   }
+  const Kind k = fused ? K_DNC : K_DN;
+  return run_gemv(L, k, B, down_args(L, B, r, y, fused, residual, out, ys, next), st, pdl);
+}
+
+GemvArgs down_args(const moe_layer* L, int B, const moe_routing& r, float* y, bool fused, const void* residual,
+                   void* out, const float* ys, const moe_layer* next) {
   const int H = L->cfg.hidden, I = L->cfg.inter;
   const Kind k = fused ? K_DNC : K_DN;
   const GemvPlan& p = plan_of(L, k, B);
@@ -684,7 +708,49 @@ cudaError_t launch_down(moe_layer* L, int B, const moe_routing& r, float* y, boo
       }
     }
   }
-  return run_gemv(L, k, B, a, st, pdl);
+  return a;
+}
+
+// the persistent kernel's instances: the streams of the batch-1 chain
+// (shape-specialised: compile-time K, split-K down; generic: runtime K)
+#define PERSIST_FAST persistent_b1_kernel<kFastH, kFastI, MOE_SPLITK_GU ? kSplitKRows / 2 : MOE_GU_RPW, kSplitKRows>
+#define PERSIST_GENERIC persistent_b1_kernel<0, 0, MOE_GU_RPW, MOE_DN_RPW>
+
+// The whole batch-1 step as one cooperative kernel (MOE_FLAG_PERSISTENT).
+cudaError_t launch_persistent(moe_layer* L, moe_layer* next, const void* x, const void* residual, void* out,
+                              cudaStream_t st) {
+  PersistArgs p;
+  std::memset(&p, 0, sizeof(p));
+  const bool has_shared = L->cfg.shared_inter > 0;
+  p.router = router_args(L, x, 1, L->plan, has_shared);
+  if (has_shared) {
+    p.sdown = shared_down_args(L, 1, L->ys);
+    p.has_sdown = 1;
+  }
+  p.gu = gate_up_args(L, x, 1, L->plan);
+  p.dnc = down_args(L, 1, L->plan, L->y, true, residual, out, has_shared ? L->ys : nullptr, next);
+  p.grid_bar = L->grid_bar;
+  p.err = L->err;
+  int threads = 0, smem = 0;
+  const Kind kinds[4] = {K_ROUTER, K_SDN, K_GU, K_DNC};
+  for (Kind kk : kinds) {
+    if (kk == K_SDN && !has_shared) continue;
+    threads = std::max(threads, L->plans[kk][0].threads);
+    smem = std::max(smem, L->plans[kk][0].smem);
+  }
+  cudaError_t e = cudaMemsetAsync(L->grid_bar, 0, sizeof(int), st);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t c = {};
+  c.gridDim = dim3(L->num_sms);
+  c.blockDim = dim3(threads);
+  c.dynamicSmemBytes = (size_t)smem;
+  c.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  c.attrs = attr;
+  c.numAttrs = 1;
+  return L->persist == 2 ? cudaLaunchKernelEx(&c, PERSIST_FAST, p) : cudaLaunchKernelEx(&c, PERSIST_GENERIC, p);
 }
 
 cudaError_t launch_combine(moe_layer* L, int B, const moe_routing& r, const float* y, const float* ys,
@@ -889,6 +955,7 @@ moe_status_t moe_layer_create(const moe_layer_config* cfg, const moe_layer_weigh
   const size_t o_rc = take(4);
   const size_t o_tc = take((size_t)H * 4);  // one counter per down-projection row tile (<= H)
   const size_t o_er = take(4);
+  const size_t o_gb = take(4);
   const size_t o_xh = take((size_t)MB * std::max(H, k * I) * 2);
   const size_t o_xe = take((size_t)MB * k * 4);
   const size_t o_xs = take((size_t)MB * H * 2);
@@ -921,6 +988,7 @@ moe_status_t moe_layer_create(const moe_layer_config* cfg, const moe_layer_weigh
   L->router_cnt = reinterpret_cast<int*>(A + o_rc);
   L->tile_cnt = reinterpret_cast<int*>(A + o_tc);
   L->err = reinterpret_cast<int*>(A + o_er);
+  L->grid_bar = reinterpret_cast<int*>(A + o_gb);
   L->xh = reinterpret_cast<__half*>(A + o_xh);
   L->xe = reinterpret_cast<int*>(A + o_xe);
   L->x_stage = reinterpret_cast<uint16_t*>(A + o_xs);
@@ -975,6 +1043,31 @@ moe_status_t moe_layer_create(const moe_layer_config* cfg, const moe_layer_weigh
     e = raise_smem_limit(reinterpret_cast<const void*>(mx_expert_kernel<true, kMxTerms>), kSmemBudget);
     if (e == cudaSuccess)
       e = raise_smem_limit(reinterpret_cast<const void*>(mx_expert_kernel<false, kMxTerms>), kSmemBudget);
+  }
+  // persistent batch-1 kernel: needs the bf16 (or no) shared expert, no side
+  // stream, and one shape-specialised or one generic instance for all streams
+  if (e == cudaSuccess && (c.flags & MOE_FLAG_PERSISTENT)) {
+    const bool fast = H == kFastH && I == kFastI && (Is == 0 || Is == kFastI);
+    const bool generic = H != kFastH && I != kFastI && Is != kFastI;
+    if (L->shared_mx || L->side_stream || !(fast || generic)) {
+      moe_layer_destroy(L);
+      return MOE_ERR_UNSUPPORTED;
+    }
+    int threads = 0, smem = 0;
+    for (Kind kk : {K_ROUTER, K_SDN, K_GU, K_DNC}) {
+      if (kk == K_SDN && Is == 0) continue;
+      threads = std::max(threads, L->plans[kk][0].threads);
+      smem = std::max(smem, L->plans[kk][0].smem);
+    }
+    const void* fn = fast ? reinterpret_cast<const void*>(PERSIST_FAST) : reinterpret_cast<const void*>(PERSIST_GENERIC);
+    e = raise_smem_limit(fn, smem);
+    int per_sm = 0;
+    if (e == cudaSuccess) e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, threads, smem);
+    if (e == cudaSuccess && per_sm < 1) {
+      moe_layer_destroy(L);
+      return MOE_ERR_UNSUPPORTED;
+    }
+    L->persist = fast ? 2 : 1;
   }
   if ((c.flags & MOE_FLAG_MX_EXPERTS) && !L->mx && e == cudaSuccess) {
     moe_layer_destroy(L);
@@ -1087,6 +1180,7 @@ moe_status_t moe_layer_forward(moe_layer_t L, moe_layer_t next, const void* x, c
     if (e == cudaSuccess) e = launch_shared(L, x, B, L->ys, L->side, false);
     if (e == cudaSuccess) e = cudaEventRecord(L->ev_join, L->side);
   }
+  if (B == 1 && L->persist && !fork) return cuda_status(launch_persistent(L, next, x, residual, out, st));
   // the bf16 shared expert's gate/up rows stream inside the router kernel
   const bool fuse_sgu = has_shared && !fork && !L->shared_mx;
   if (e == cudaSuccess) e = launch_router(L, x, B, L->plan, st, fuse_sgu);
