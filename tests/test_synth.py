@@ -126,3 +126,50 @@ def test_tied_router_inputs_tie_at_the_selection_boundary(E, k, copies, with_bia
     srt = -np.sort(-lg, axis=1)
     boundary = srt[:, k - 1] == srt[:, k]
     assert boundary[:7].any() and boundary.sum() >= 4
+
+
+def test_verify_positions_share_their_sequence_draw():
+    """Verify-shape batches: the 8 positions of one sequence mix the
+    sequence's draw (weight sqrt(0.9)) with their own, so they are strongly
+    correlated with each other and route to far fewer distinct experts than
+    independent tokens; positions of different sequences are independent."""
+    cfg = synth.CONFIGS[5].with_(hidden=1024, n_experts=256)
+    wr = synth.gen_router_w(cfg)
+    x, _ = synth.gen_tokens(cfg, wr, None, range(16))
+    xf = synth.bf16_to_f32(x).astype(np.float64)
+    c = np.corrcoef(xf)
+    within = c[:8, :8][~np.eye(8, dtype=bool)]
+    across = c[:8, 8:]
+    assert within.min() > 0.8 and np.abs(across).max() < 0.2
+    ind = synth.CONFIGS[2].with_(hidden=1024, n_experts=256)
+    xi, _ = synth.gen_tokens(ind, synth.gen_router_w(ind), None, range(8))
+    lg_v = xf[:8] @ synth.bf16_to_f32(wr).astype(np.float64)
+    lg_i = synth.bf16_to_f32(xi).astype(np.float64) @ synth.bf16_to_f32(synth.gen_router_w(ind)).astype(np.float64)
+    top = lambda lg: len(np.unique(np.argsort(-lg, axis=1)[:, :16]))
+    assert top(lg_v) < 0.6 * top(lg_i)
+
+
+def test_edge_mxfp4_generator_covers_the_format():
+    cfg = synth.CONFIGS[0]
+    codes, scales = synth.gen_edge_mxfp4(cfg, 3, 8, 128, synth.T_EXPERT_GU, 87, 139)
+    nib = np.stack([codes & 15, codes >> 4], -1).reshape(-1, 32)
+    assert all((np.bincount(b, minlength=16) == 2).all() for b in nib)   # every code twice per block
+    s = scales.reshape(-1)
+    assert (s == 0).sum() == len(s[::23]) and s[s > 0].min() >= 87 and s.max() <= 139
+    again = synth.gen_edge_mxfp4(cfg, 3, 8, 128, synth.T_EXPERT_GU, 87, 139)
+    assert np.array_equal(again[0], codes) and np.array_equal(again[1], scales)   # seeded
+    other = synth.gen_edge_mxfp4(cfg, 3, 8, 128, synth.T_EXPERT_D, 87, 139)
+    assert not np.array_equal(other[0], codes)
+
+
+def test_wide_range_tokens_keep_the_routing_margin():
+    cfg = synth.CONFIGS[0]
+    wr = synth.gen_router_w(cfg)
+    x, _ = synth.gen_tokens(cfg, wr, None, range(6), tiny_every=7)
+    xf = np.abs(synth.bf16_to_f32(x).astype(np.float64))
+    ratio = xf[:, ::7].max(axis=1) / xf.max(axis=1)
+    assert (ratio < 2.0 ** -26).all()                       # elements ~2^30 below the row's maximum
+    for row in x:
+        lg = synth.bf16_to_f32(row).astype(np.float64) @ synth.bf16_to_f32(wr).astype(np.float64)
+        srt = np.sort(lg)[::-1]
+        assert srt[cfg.top_k - 1] - srt[cfg.top_k] >= cfg.min_gap
