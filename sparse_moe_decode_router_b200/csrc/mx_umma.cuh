@@ -54,13 +54,16 @@ namespace moe {
 constexpr int kMxRows = 128;       // M: weight rows per MMA (one TMEM lane each)
 constexpr int kMxKTile = 128;      // K elements per pipeline stage (one 128-byte swizzle row)
 constexpr int kMxNMax = 64;        // B columns per pass (tokens x terms, padded to 16)
-constexpr int kMxMaxStages = 8;
+constexpr int kMxMaxStages = 12;   // TMEM: scale chunks of 12 stages fit below column 432
 constexpr int kMxThreads = 256;
 constexpr int kMxTmemCols = 512;
 constexpr int kMxAccCols = 128;    // per accumulator buffer: gate [0, 64), up [64, 128)
-constexpr int kMxSfaCol0 = 256;    // per stage 8 columns: gate chunk, up chunk
-constexpr int kMxSfbCol0 = 384;    // per stage 4 columns
+constexpr int kMxSfaCol0 = 256;    // per stage 8 columns: gate chunk, up chunk (256 + 8*12 <= 384)
+constexpr int kMxSfbCol0 = 384;    // per stage 4 columns (384 + 4*12 <= 512)
+static_assert(kMxSfaCol0 + 8 * kMxMaxStages <= kMxSfbCol0 && kMxSfbCol0 + 4 * kMxMaxStages <= kMxTmemCols,
+              "scale-factor columns");
 constexpr int kMxHeaderBytes = 1024;
+static_assert(8 * (2 * kMxMaxStages + 6) + 32 <= kMxHeaderBytes, "header");
 constexpr int kMxABytes = kMxRows * kMxKTile;  // one A tile in shared memory (16 KB, expanded)
 constexpr uint32_t kMxATx = kMxRows * kMxKTile / 2;  // bytes one A tile moves (packed)
 
