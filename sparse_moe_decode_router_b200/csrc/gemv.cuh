@@ -405,6 +405,7 @@ __device__ __forceinline__ void group_bar(int q0, int wpi) {
 
 __device__ void publish_round(const GemvArgs& a, const int* pend_rt, int npend, int& prev_cnt, int& prev_rt,
                               int& nprev, int n_groups, int wi, int q0, int lane, int* s_pub) {
+  if (npend > 0) __threadfence();  // this thread's y stores, visible at gpu scope
   group_bar(q0, a.wpi);  // every warp of the group has written its y rows of the pending items
   if (wi == 0) {
     // results of the previous round first (their atomics completed long ago)
@@ -1027,12 +1028,11 @@ __device__ __forceinline__ void gemv_body(const GemvArgs& a, unsigned char* smem
   if constexpr (kRouter) {
     if (a.topk_idx) {
       // every CTA's logits are written: the last CTA to get here selects the
-      // top-k of every token (one warp per token), then builds the buckets
+      // top-k of every token (one warp per token), then builds the buckets.
+      // Each thread makes its own logit stores visible at gpu scope first.
+      __threadfence();
       named_bar_sync(kBarAll, nthreads_all);
-      if (tid == 0) {
-        __threadfence();
-        s_flag[1] = (atomicAdd(a.done_counter, 1) == (int)gridDim.x - 1) ? 1 : 0;
-      }
+      if (tid == 0) s_flag[1] = (atomicAdd(a.done_counter, 1) == (int)gridDim.x - 1) ? 1 : 0;
       named_bar_sync(kBarAll, nthreads_all);
       if (s_flag[1]) {
         __threadfence();

@@ -258,8 +258,8 @@ __device__ void topk_token_warp(const GemvArgs& a, const float* __restrict__ lg,
 
 // Buckets of the B*k pairs from topk_idx (global, written by this block
 // before a barrier): counts, exclusive offsets, pair ids sorted by
-// (expert, b, j), the active list.  nt threads (a multiple of 32, nt*4 >= E)
-// meeting on named barrier `bar`;
+// (expert, b, j), the active list.  nt threads (a multiple of 32, at most
+// 32 warps) meeting on named barrier `bar`, each owning ceil(E/nt) experts;
 // scratch: s_mask [E] u64, s_off [E] int, s_wsum [2*32] int.
 __device__ void bucket_block(const GemvArgs& a, int B, int tid, int nt, int bar, unsigned long long* s_mask,
                              int* s_off, int* s_wsum) {
@@ -269,13 +269,15 @@ __device__ void bucket_block(const GemvArgs& a, int B, int tid, int nt, int bar,
   named_bar_sync(bar, nt);
   for (int p = tid; p < B * k; p += nt) atomicOr(&s_mask[__ldcg(a.topk_idx + p)], 1ull << (p / k));
   named_bar_sync(bar, nt);
-  int cnt[4], tc = 0, ta = 0;
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int e = 4 * tid + i;
-    cnt[i] = (e < E) ? __popcll(s_mask[e]) : 0;
-    tc += cnt[i];
-    ta += cnt[i] > 0;
+  // thread t owns the experts [t*per, (t+1)*per): counts, then block scans
+  // of the pair counts and of the active flags
+  const int per = (E + nt - 1) / nt;
+  const int e_lo = min(E, tid * per), e_hi = min(E, e_lo + per);
+  int tc = 0, ta = 0;
+  for (int e = e_lo; e < e_hi; ++e) {
+    const int c = __popcll(s_mask[e]);
+    tc += c;
+    ta += c > 0;
   }
   int ic = tc, ia = ta;
 #pragma unroll
@@ -298,18 +300,15 @@ __device__ void bucket_block(const GemvArgs& a, int B, int tid, int nt, int bar,
     wa += s_wsum[2 * w + 1];
   }
   int off = wc + ic - tc, act = wa + ia - ta;
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int e = 4 * tid + i;
-    if (e < E) {
-      s_off[e] = off;
-      a.offsets_out[e] = off;
-      a.counts[e] = cnt[i];
-      if (cnt[i] > 0) a.active_out[act++] = e;
-      off += cnt[i];
-    }
+  for (int e = e_lo; e < e_hi; ++e) {
+    const int c = __popcll(s_mask[e]);
+    s_off[e] = off;
+    a.offsets_out[e] = off;
+    a.counts[e] = c;
+    if (c > 0) a.active_out[act++] = e;
+    off += c;
   }
-  if (4 * tid < E && 4 * tid + 4 >= E) {  // the thread owning the last expert
+  if (e_lo < E && e_hi == E) {  // the thread owning the last expert
     a.offsets_out[E] = off;
     *a.n_active_out = act;
   }

@@ -676,9 +676,9 @@ __global__ void __launch_bounds__(kMxThreads, 1)
       if (!kSwiglu && a.comb_w && w.pass == w.npass - 1) {
         // the item is complete: count it for its row tile; the last expert to
         // arrive combines the tile's rows for every token
+        __threadfence();         // this thread's y stores, visible at gpu scope
         if (!epi_sync()) break;  // the four epilogue warps' y stores are done
         if (warp == 4 && lane == 0) {
-          __threadfence();
           const int prev = atomicAdd(&a.tile_counter[u.rt], 1);
           const bool last = prev == n_groups - 1;
           if (last) a.tile_counter[u.rt] = 0;  // every contribution is in: ready for the next launch
