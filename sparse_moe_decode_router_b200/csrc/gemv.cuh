@@ -258,7 +258,11 @@ __device__ __forceinline__ float pow2f(int e) {
   return __uint_as_float((uint32_t)(e + 127) << 23);
 }
 
-// Staging of activation vectors into shared memory.  MXFP4 streams: f16 of
+// Staging of activation vectors into shared memory.  Activations come from
+// the preceding kernel, which under programmatic dependent launch may still
+// be writing them while this grid starts: they are read through L2 only
+// (ld.global.cg), never through the non-coherent read-only path, which is
+// reserved for weights that no kernel writes.  MXFP4 streams: f16 of
 // x * 2^-e in the lane-interleaved layout, e chosen from max|x| so that the
 // largest element sits in [2^8, 2^9) (exact for bf16 inputs down to 2^-25 of
 // the largest element, one rounding for fp32 ones); the headroom above keeps
@@ -282,7 +286,7 @@ __device__ float segment_amax(const void* src_base, int row, int K, int g0, int 
     const uint4* s = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(src_base) + (size_t)row * K);
 #pragma unroll 4
     for (int g = g0 + lane; g < g1; g += 32) {
-      const uint4 v = __ldg(s + g);
+      const uint4 v = __ldcg(s + g);
       const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
       for (int j = 0; j < 4; ++j) amax = fmaxf(amax, fmaxf(fabsf(bf16lo_to_f32(w[j])), fabsf(bf16hi_to_f32(w[j]))));
@@ -306,7 +310,7 @@ __device__ void segment_to_f16(const void* src_base, int row, int K, int g0, int
       v[0] = v0.x; v[1] = v0.y; v[2] = v0.z; v[3] = v0.w; v[4] = v1.x; v[5] = v1.y; v[6] = v1.z; v[7] = v1.w;
     } else {
       const uint4* s = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(src_base) + (size_t)row * K);
-      const uint4 u = __ldg(s + g);
+      const uint4 u = __ldcg(s + g);
       const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
@@ -371,7 +375,7 @@ __device__ void stage_phase(const void* src, const int* slot_src, int nslots, in
       uint4* d = reinterpret_cast<uint4*>(xbuf + (size_t)sl * xrow_bytes);
       const int i1 = min(n16, (q + 1) * seg16);
 #pragma unroll 4
-      for (int i = q * seg16 + lane; i < i1; i += 32) d[i] = (XK == X_F32) ? __ldcg(s + i) : __ldg(s + i);
+      for (int i = q * seg16 + lane; i < i1; i += 32) d[i] = __ldcg(s + i);
       if (lane == 0 && q == 0) slot_e[sl] = 0;
     }
   }

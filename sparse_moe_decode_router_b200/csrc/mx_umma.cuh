@@ -238,7 +238,7 @@ __global__ void __launch_bounds__(256) mx_x_terms_kernel(const uint16_t* __restr
     float v[32];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      const uint4 u = __ldg(src + i);
+      const uint4 u = __ldcg(src + i);  // written by a preceding kernel: coherent path
       const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
@@ -445,6 +445,8 @@ __global__ void __launch_bounds__(kMxThreads, 1)
     }
   } else if (plan_ok && warp == 2) {
     // ------------------------- scale-factor chunks ----------------------------
+    // Weight scales are static (read-only path); the activation scales come
+    // from the preceding kernel and are read through L2 (coherent path).
     // Lane l covers rows l + 32*m (m = 0..3) of the A tile(s) and B columns
     // l + 32*m (m = 0..1).  Where a scale row is a multiple of 16 bytes long,
     // one 16-byte load per row fetches four stages' scale bytes, and the next
@@ -469,7 +471,7 @@ __global__ void __launch_bounds__(kMxThreads, 1)
         for (int m = 0; m < 2; ++m) {
           const int n = lane + 32 * m, row = u.tok * kTerms + n;
           bb[m] = (n < u.n && row < a.act_rows)
-                      ? __ldg(reinterpret_cast<const uint4*>(a.asf + (size_t)row * sblk + 4 * kg))
+                      ? __ldcg(reinterpret_cast<const uint4*>(a.asf + (size_t)row * sblk + 4 * kg))
                       : make_uint4(0u, 0u, 0u, 0u);
         }
       };
@@ -512,7 +514,7 @@ __global__ void __launch_bounds__(kMxThreads, 1)
             for (int m = 0; m < 2; ++m) {
               const int n = lane + 32 * m, row = u.tok * kTerms + n;
               vb[m] = (n < u.n && row < a.act_rows)
-                          ? __ldg(reinterpret_cast<const uint32_t*>(a.asf + (size_t)row * sblk + 4 * kt))
+                          ? __ldcg(reinterpret_cast<const uint32_t*>(a.asf + (size_t)row * sblk + 4 * kt))
                           : 0u;
             }
           }
