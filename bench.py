@@ -256,7 +256,8 @@ def kernel_source_sha():
     routed gate/up kernel: a recorded ncu traffic figure stays valid as long
     as this hash is unchanged."""
     h = hashlib.sha256()
-    for f in ("kernels.cuh", "gemv.cuh", "ptx.cuh", "moe_decode.cu"):
+    for f in ("kernels.cuh", "gemv.cuh", "ptx.cuh", "moe_decode.cu", "mx_umma.cuh", "persistent.cuh",
+              "mma_grouped.cuh"):
         with open(os.path.join(ROOT, "sparse_moe_decode_router_b200", "csrc", f), encoding="utf-8") as fh:
             h.update(_code_only(fh.read()).encode())
     return h.hexdigest()[:16]
@@ -618,7 +619,9 @@ def run_ours(args, cfg):
     ms_per_step = total_ms / K
     value = job_value(world, total_bytes, total_ms)
     achieved = gu_bytes / gu_avg_s / 1e9
-    traffic = recorded_traffic("routed_gate_up", cfg.name)
+    from sparse_moe_decode_router_b200.api import MOE_FLAG_MX_EXPERTS
+    gu_tag = "routed_gate_up_tcgen05" if args.flags & MOE_FLAG_MX_EXPERTS else "routed_gate_up"
+    traffic = recorded_traffic(gu_tag, cfg.name)
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5), "higher_is_better": True,
@@ -630,7 +633,7 @@ def run_ours(args, cfg):
         "counted_bytes_per_step": int(total_bytes / K),
         "n_active_mean": n_active_mean,
         "frac_of_measured_hbm": round(value / world / peak, 4),
-        "roofline": {"kernel": "routed_gate_up", "bound": "hbm", "achieved": round(achieved, 1),
+        "roofline": {"kernel": gu_tag, "bound": "hbm", "achieved": round(achieved, 1),
                      "peak": peak, "unit": "GB/s", "frac": round(achieved / peak, 4), "traffic": traffic,
                      "peak_source": peak_src, "algorithmic_bytes_per_launch": int(gu_bytes),
                      "avg_launch_us": round(gu_avg_s * 1e6, 2),
