@@ -21,6 +21,7 @@ their corners.
 import numpy as np
 import pytest
 
+import oracle
 import synth
 from gpu_common import (assert_routing_equal, create_layer, layer_routing_host, make_device_layer,
                         oracle_layer_for, residual_tokens, to_host_u16)
@@ -142,7 +143,7 @@ def test_inputs_written_on_stream_before_the_layer(torch_cuda, which, B, reps):
         r_buf = torch.empty_like(x_src)
         out = torch.empty_like(x_src)
         g = _graph_with_producer(torch, api, h, B, H, x_src, r_src, x_buf, r_buf, out)
-        outs, plans, xs, rs = [], [], [], []
+        outs, plans, xs, rs, xbufs = [], [], [], [], []
         for rep in range(reps):
             ids = list(range(1000 + rep * B, 1000 + (rep + 1) * B))
             x_h, x_d = dl.tokens(ids)
@@ -153,14 +154,23 @@ def test_inputs_written_on_stream_before_the_layer(torch_cuda, which, B, reps):
             outs.append(out.clone())
             torch.cuda.synchronize()
             plans.append(layer_routing_host(h, B, k, E))
+            xbufs.append(to_host_u16(x_buf))
             xs.append(x_h)
             rs.append(r_h)
         assert api.moe_layer_last_device_error(h) == api.MOE_OK
         del g
     finally:
         api.moe_layer_destroy(h)
+    bad = []
     for rep in range(reps):
+        assert np.array_equal(xbufs[rep], xs[rep]), f"replay {rep}: the producer did not write x"
         ref = oracle_layer_for(dl, xs[rep], rs[rep])
-        assert_routing_equal(plans[rep], ref, W_ABS)
-        ok, info = bf16_close(to_host_u16(outs[rep]), ref["out_bf16"])
-        assert ok, (rep, info)
+        try:
+            assert_routing_equal(plans[rep], ref, W_ABS)
+            ok, info = bf16_close(to_host_u16(outs[rep]), ref["out_bf16"])
+            assert ok, info
+        except AssertionError as e:
+            prev = oracle.routing(xs[rep - 1], dl.router_w_host, dl.bias_host, k)["topk_idx"] if rep else None
+            bad.append((rep, str(e)[:80], plans[rep]["topk_idx"].tolist(), ref["topk_idx"].tolist(),
+                        None if prev is None else prev.tolist()))
+    assert not bad, bad
