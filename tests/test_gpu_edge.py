@@ -104,7 +104,10 @@ def test_full_size_shifted_scales_match_oracle(torch_cuda, shift):
 def _graph_with_producer(torch, api, h, B, H, x_src, r_src, x_buf, r_buf, out):
     """One graph: a kernel writes x and residual from the source buffers (an
     elementwise multiply by one, so a real kernel node, not a memcpy node),
-    then the fused layer on the same stream, PDL chaining on."""
+    then the fused layer on the same stream, PDL chaining on.  Returns the
+    graph and the tensors its nodes read besides the caller's: they must
+    outlive every replay (freed, their memory would go back to the caching
+    allocator and be handed to the next input copied in).  """
     one = torch.ones((), dtype=torch.bfloat16, device="cuda")
     pad = torch.zeros(16 * 1024 * 1024, dtype=torch.float32, device="cuda")
     g = torch.cuda.CUDAGraph()
@@ -121,7 +124,7 @@ def _graph_with_producer(torch, api, h, B, H, x_src, r_src, x_buf, r_buf, out):
             torch.mul(r_src, one, out=r_buf)
             torch.mul(x_src, one, out=x_buf)       # the layer's direct predecessor
             api.moe_layer_forward(h, None, x_buf, r_buf, out, B, stream=torch.cuda.current_stream())
-    return g
+    return g, (one, pad)
 
 
 @pytest.mark.parametrize("which,B,reps", [("tiny", 1, 12), ("tiny", 33, 6), ("full", 1, 6)])
@@ -142,7 +145,7 @@ def test_inputs_written_on_stream_before_the_layer(torch_cuda, which, B, reps):
         x_buf = torch.empty_like(x_src)
         r_buf = torch.empty_like(x_src)
         out = torch.empty_like(x_src)
-        g = _graph_with_producer(torch, api, h, B, H, x_src, r_src, x_buf, r_buf, out)
+        g, keep = _graph_with_producer(torch, api, h, B, H, x_src, r_src, x_buf, r_buf, out)
         outs, plans, xs, rs, xbufs = [], [], [], [], []
         for rep in range(reps):
             ids = list(range(1000 + rep * B, 1000 + (rep + 1) * B))
@@ -158,7 +161,7 @@ def test_inputs_written_on_stream_before_the_layer(torch_cuda, which, B, reps):
             xs.append(x_h)
             rs.append(r_h)
         assert api.moe_layer_last_device_error(h) == api.MOE_OK
-        del g
+        del g, keep
     finally:
         api.moe_layer_destroy(h)
     bad = []
