@@ -83,10 +83,13 @@ typedef struct moe_layer* moe_layer_t; /* opaque, library-owned */
 #define MOE_FLAG_NO_PREFETCH 0x4u   /* no L2 prefetch of the next layer's weights */
 #define MOE_FLAG_NO_GROUPED 0x8u    /* never use the tensor-core grouped expert path */
 #define MOE_FLAG_MX_EXPERTS 0x10u   /* routed experts at every batch size on the tcgen05 block-scaled
-                                      kernels (E2M1 weights x E4M3 activation terms, E8M0 scales
-                                      on both); needs hidden and inter multiples of 128 and
-                                      32-byte aligned expert codes, else moe_layer_create returns
-                                      MOE_ERR_UNSUPPORTED */
+                                      kernels (kind::mxf4: packed E2M1 weights x five E2M1 terms
+                                      per activation value, E8M0 scales on both); needs hidden and
+                                      inter multiples of 128, else moe_layer_create returns
+                                      MOE_ERR_UNSUPPORTED.  The layer then keeps a copy of the
+                                      expert scales (s_gate_up, s_down) in the tensor cores'
+                                      scale-factor layout, taken at moe_layer_create: as for the
+                                      router matrix, later changes to them are not seen */
 #define MOE_FLAG_PERSISTENT 0x40u    /* batch-1 moe_layer_forward as one cooperative kernel (one CTA
                                       per SM, in-kernel grid barriers between the routing, the
                                       experts and the combine; the pages' persistent kernels,
@@ -116,7 +119,8 @@ typedef struct {
 } moe_layer_config;
 
 /* Weights: DEVICE pointers, caller-owned, borrowed (never copied, except the
- * router matrix, see moe_layer_create); they must stay valid and unchanged
+ * router matrix and, where the tcgen05 expert kernels can run, the expert
+ * scale arrays: see moe_layer_create); they must stay valid and unchanged
  * while the layer exists. */
 typedef struct {
   const void* router_w;      /* bf16 [H][E]: logit e is sum_h x[h] router_w[h][e] */
@@ -156,7 +160,11 @@ typedef struct {
  * compute capability 10.x), allocates the layer's scratch for max_batch
  * tokens, a side stream and events, and copies router_w once into a
  * library-owned expert-major [E][H] copy that the router kernel streams
- * (so router_w need not outlive this call; every other weight must).
+ * (so router_w need not outlive this call; every other weight must).  Where
+ * hidden and inter are multiples of 128 it also copies s_gate_up and s_down
+ * into the scale-factor chunk layout of the tcgen05 expert kernels (128
+ * rows x 4 blocks of 32 per 512-byte chunk), the same number of bytes as
+ * the scale arrays themselves.
  * Uses the current CUDA device.  Synchronises the device once.
  * Returns MOE_ERR_INVALID_ARG / MOE_ERR_UNSUPPORTED / MOE_ERR_OOM /
  * MOE_ERR_CUDA; on failure *out is NULL. */

@@ -1040,11 +1040,10 @@ __device__ __forceinline__ void gemv_body(const GemvArgs& a, unsigned char* smem
       named_bar_sync(kBarAll, nthreads_all);
       if (s_flag[1]) {
         __threadfence();
-        const int nw = nthreads_all >> 5;
-        for (int b = warp; b < a.n_tokens; b += nw) topk_token_warp(a, a.out, b, lane);
+        // the stage ring is idle now: top-k candidates, then bucket scratch
+        topk_tail(a, a.out, tid, nthreads_all, kBarAll, stages + kBucketScratchBytes);
         __threadfence();
         named_bar_sync(kBarAll, nthreads_all);
-        // the stage ring is idle now: bucket scratch
         unsigned long long* s_mask = reinterpret_cast<unsigned long long*>(stages);
         int* s_off = reinterpret_cast<int*>(stages + 8 * kMaxExperts);
         int* s_wsum = s_off + kMaxExperts;

@@ -196,32 +196,14 @@ __device__ __forceinline__ uint32_t warp_select_topk(const uint32_t (&key)[PL], 
   return sel;
 }
 
-// ---------------------------------------------------------------------------
-// Routing finish inside the router kernel (its last CTA): one warp per token
-// selects the k largest scores of all E experts (lane l owns experts
-// [l*PL, l*PL + PL), PL = ceil(E/32) <= 32, ids ascending with the slot),
-// equal scores going to the lower id; then the weights (softmax over the
-// selected logits, or the selected sigmoid scores normalised), written in
-// ascending expert id.
-__device__ void topk_token_warp(const GemvArgs& a, const float* __restrict__ lg, int b, int lane) {
-  const int E = a.n_experts, k = a.top_k;
-  const int PL = (E + 31) / 32;
-  uint32_t key[32];
-  float val[32];
-#pragma unroll
-  for (int i = 0; i < 32; ++i) {
-    const int e = lane * PL + i;
-    const bool ok = i < PL && e < E;
-    float v = ok ? __ldcg(lg + (size_t)b * E + e) : 0.f;
-    if (a.scoring == 1) {
-      v = 1.0f / (1.0f + expf(-v));
-      key[i] = ok ? logit_key(v + (a.sel_bias ? __ldg(a.sel_bias + e) : 0.f)) : 0u;
-    } else {
-      key[i] = ok ? logit_key(v) : 0u;
-    }
-    val[i] = v;
-  }
-  const uint32_t sel = warp_select_topk<32>(key, k, lane);
+// Weights of token b's selection and its output, ascending expert id: the
+// warp holds PL candidates per lane (ids ascending with lane*PL + slot),
+// `sel` marks the selected slots, val their logits (softmax) or sigmoid
+// scores (bias-corrected sigmoid: normalised over the selection).
+template <int PL>
+__device__ __forceinline__ void topk_write(const GemvArgs& a, int b, uint32_t sel, float (&val)[PL],
+                                           const int (&id)[PL], int lane) {
+  const int k = a.top_k;
   const int ns = __popc(sel);
   int pre = ns;
 #pragma unroll
@@ -232,13 +214,13 @@ __device__ void topk_token_warp(const GemvArgs& a, const float* __restrict__ lg,
   pre -= ns;
   float lmax = -INFINITY;
 #pragma unroll
-  for (int i = 0; i < 32; ++i)
+  for (int i = 0; i < PL; ++i)
     if ((sel >> i) & 1u) lmax = fmaxf(lmax, val[i]);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) lmax = fmaxf(lmax, __shfl_xor_sync(0xFFFFFFFFu, lmax, o));
   float z = 0.f;
 #pragma unroll
-  for (int i = 0; i < 32; ++i) {
+  for (int i = 0; i < PL; ++i) {
     if ((sel >> i) & 1u) {
       val[i] = a.scoring == 1 ? val[i] : expf(val[i] - lmax);
       z += val[i];
@@ -248,12 +230,123 @@ __device__ void topk_token_warp(const GemvArgs& a, const float* __restrict__ lg,
   for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xFFFFFFFFu, z, o);
   int pos = pre;
 #pragma unroll
-  for (int i = 0; i < 32; ++i)
+  for (int i = 0; i < PL; ++i)
     if ((sel >> i) & 1u) {
-      a.topk_idx[b * k + pos] = lane * PL + i;
+      a.topk_idx[b * k + pos] = id[i];
       a.topk_w[b * k + pos] = val[i] / z;
       ++pos;
     }
+}
+
+// Selection keys and values of experts [lo, hi) of token b, lane l owning
+// [lo + l*PL, lo + l*PL + PL) (PL = ceil((hi - lo)/32) <= 32)
+__device__ __forceinline__ void topk_load(const GemvArgs& a, const float* __restrict__ lg, int b, int lo, int hi,
+                                          int lane, uint32_t (&key)[32], float (&val)[32], int (&id)[32]) {
+  const int E = a.n_experts;
+  const int PL = (hi - lo + 31) / 32;
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    const int e = lo + lane * PL + i;
+    const bool ok = i < PL && e < hi;
+    float v = ok ? __ldcg(lg + (size_t)b * E + e) : 0.f;
+    if (a.scoring == 1) {
+      v = 1.0f / (1.0f + expf(-v));
+      key[i] = ok ? logit_key(v + (a.sel_bias ? __ldg(a.sel_bias + e) : 0.f)) : 0u;
+    } else {
+      key[i] = ok ? logit_key(v) : 0u;
+    }
+    val[i] = v;
+    id[i] = e;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Routing finish inside the router kernel (its last CTA, nthreads threads
+// meeting on named barrier `bar`): per token the k largest scores of all E
+// experts, equal scores going to the lower id; then the weights (softmax
+// over the selected logits, or the selected sigmoid scores normalised),
+// written in ascending expert id.
+//
+// With at least as many tokens as warps, one warp per token scans all E
+// experts.  With fewer, each token gets wpt warps: warp w selects the top-k
+// of its contiguous slice of the experts into shared memory (ids ascending
+// within and across slices), and the token's first warp selects the top-k
+// of those wpt*k candidates.  Every member of the overall top-k is in its
+// slice's top-k (at most k-1 experts of the slice precede it in the order
+// score desc, id asc), so the result is the same as one warp's scan.
+// Scratch: kTopkCandBytes of shared memory.
+constexpr int kBucketScratchBytes = 8 * kMaxExperts + 4 * kMaxExperts + 4 * 64;  // s_mask, s_off, s_wsum
+constexpr int kTopkMaxCand = 256;  // candidates one merging warp takes (8 per lane)
+constexpr int kTopkCandBytes = 12 * 32 * kMaxTopK;  // at most 32 warps x k candidates
+
+__device__ void topk_tail(const GemvArgs& a, const float* __restrict__ lg, int tid, int nthreads, int bar,
+                          unsigned char* scratch) {
+  const int B = a.n_tokens, E = a.n_experts, k = a.top_k;
+  const int nw = nthreads >> 5, warp = tid >> 5, lane = tid & 31;
+  int wpt = B > 0 ? nw / B : 1;
+  wpt = min(wpt, kTopkMaxCand / k);
+  if (wpt < 2) {
+    for (int b = warp; b < B; b += nw) {
+      uint32_t key[32];
+      float val[32];
+      int id[32];
+      topk_load(a, lg, b, 0, E, lane, key, val, id);
+      const uint32_t sel = warp_select_topk<32>(key, k, lane);
+      topk_write<32>(a, b, sel, val, id, lane);
+    }
+    return;
+  }
+  uint32_t* ck = reinterpret_cast<uint32_t*>(scratch);
+  float* cv = reinterpret_cast<float*>(scratch + 4 * 32 * kMaxTopK);
+  int* ci = reinterpret_cast<int*>(scratch + 8 * 32 * kMaxTopK);
+  const int S = (E + wpt - 1) / wpt;  // experts per slice
+  if (warp < B * wpt) {
+    const int b = warp / wpt, w = warp - b * wpt;
+    const int lo = min(E, w * S), hi = min(E, lo + S);
+    uint32_t key[32];
+    float val[32];
+    int id[32];
+    topk_load(a, lg, b, lo, hi, lane, key, val, id);
+    const uint32_t sel = warp_select_topk<32>(key, k, lane);
+    const int ns = __popc(sel);
+    int pre = ns;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int t = __shfl_up_sync(0xFFFFFFFFu, pre, o);
+      if (lane >= o) pre += t;
+    }
+    const int total = __shfl_sync(0xFFFFFFFFu, pre, 31);  // min(k, slice size)
+    pre -= ns;
+    const int base = warp * k;
+#pragma unroll
+    for (int i = 0; i < 32; ++i)
+      if ((sel >> i) & 1u) {
+        ck[base + pre] = key[i];
+        cv[base + pre] = val[i];
+        ci[base + pre] = id[i];
+        ++pre;
+      }
+    for (int j = total + lane; j < k; j += 32) ck[base + j] = 0u;  // empty slots (key 0: no expert)
+  }
+  named_bar_sync(bar, nthreads);
+  if (warp < B * wpt && (warp % wpt) == 0) {
+    const int b = warp / wpt;
+    const int nc = wpt * k;             // <= kTopkMaxCand
+    const int PL = (nc + 31) / 32;      // <= 8
+    uint32_t key[8];
+    float val[8];
+    int id[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int c = lane * PL + i;
+      const bool ok = i < PL && c < nc;
+      key[i] = ok ? ck[warp * k + c] : 0u;
+      val[i] = ok ? cv[warp * k + c] : 0.f;
+      id[i] = ok ? ci[warp * k + c] : 0;
+    }
+    const uint32_t sel = warp_select_topk<8>(key, k, lane);
+    topk_write<8>(a, b, sel, val, id, lane);
+  }
 }
 
 // Buckets of the B*k pairs from topk_idx (global, written by this block

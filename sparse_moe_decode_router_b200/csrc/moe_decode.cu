@@ -28,7 +28,7 @@ constexpr int kSmemBudget = 227 * 1024;  // dynamic shared memory per CTA (1 CTA
 constexpr int kMaxStages = kMaxStagesDev;
 constexpr int kXBudget = 64 * 1024;       // staged activation vectors
 constexpr int kPrefetchBytes = 64 * 1024; // stages kept in flight ahead of the consumers
-constexpr int kRouterBucketBytes = 8 * kMaxExperts + 4 * kMaxExperts + 4 * 64;  // s_mask, s_off, s_wsum
+constexpr int kRouterBucketBytes = kBucketScratchBytes + kTopkCandBytes;  // routing finish scratch
 
 size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
@@ -278,10 +278,13 @@ struct moe_layer {
   bool mx = false;      // the shapes and pointers allow it
   bool mx_on = false;   // routed experts run on it
   CUtensorMap tm_agu{}, tm_adn{}, tm_bx{}, tm_bh{};
-  uint8_t* aqx = nullptr;   // E4M3 terms of x per pair position [MB*k*T][H]
-  uint8_t* asfx = nullptr;  // ... their scales [MB*k*T][H/32]
-  uint8_t* aqh = nullptr;   // E4M3 terms of h [MB*k*T][I]
-  uint8_t* asfh = nullptr;  // ... their scales [MB*k*T][I/32]
+  uint8_t* aqx = nullptr;   // E2M1 terms of x per pair position [MB*k*T][H/2]
+  uint8_t* bsfx = nullptr;  // ... their scales, chunk layout [MB*k][H/128][512]
+  uint8_t* aqh = nullptr;   // E2M1 terms of h [MB*k*T][I/2]
+  uint8_t* bsfh = nullptr;  // ... their scales, chunk layout [MB*k][I/128][512]
+  char* mx_mem = nullptr;   // the weight scales in chunk layout (copied at create):
+  uint8_t* wsf_gu = nullptr;  // gate/up [E * 2I/128][H/128][512]
+  uint8_t* wsf_dn = nullptr;  // down [E * H/128][I/128][512]
   int* err = nullptr;
   uint16_t* x_stage = nullptr;
   uint16_t* res_stage = nullptr;
@@ -452,7 +455,6 @@ cudaError_t launch_grouped(moe_layer* L, bool gate_up, int B, const moe_routing&
 cudaError_t launch_gate_up_streams(moe_layer* L, const void* x, int B, const moe_routing& r, cudaStream_t st);
 
 // ---- tcgen05 block-scaled expert path -------------------------------------
-constexpr int kMxTerms = 3;  // E4M3 terms per activation row
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
@@ -494,17 +496,22 @@ struct MxPlan {
   int n_max, stage_bytes, n_stages, smem, off_up, off_b, off_sfa, off_sfb;
 };
 
+// B columns of one pass: the same for both projections of a call (the
+// gate/up epilogue writes the down projection's scale chunks per pass)
+int mx_n_max(int B) { return std::min(kMxNMax, (B * kMxTerms + 15) & ~15); }
+
 // shared-memory ring of one projection: a stage holds the A tile(s), the B
-// rows of one pass and the scale-factor chunks
+// rows of one pass and the scale-factor chunks (two per operand)
 MxPlan mx_plan(bool gate_up, int B) {
   MxPlan p;
-  p.n_max = std::min(kMxNMax, (B * kMxTerms + 15) & ~15);
-  p.off_up = gate_up ? kMxABytes : 0;
-  p.off_b = (gate_up ? 2 : 1) * kMxABytes;
-  p.off_sfa = p.off_b + p.n_max * 128;
-  p.off_sfb = p.off_sfa + (gate_up ? 1024 : 512);
-  p.stage_bytes = (int)align_up((size_t)p.off_sfb + 512, 1024);
-  p.n_stages = std::min(kMxMaxStages, (kSmemBudget - 2 * kMxHeaderBytes) / p.stage_bytes);
+  p.n_max = mx_n_max(B);
+  p.off_up = gate_up ? kMxATile : 0;
+  p.off_b = (gate_up ? 2 : 1) * kMxATile;
+  p.off_sfa = p.off_b + (int)align_up((size_t)p.n_max * 128, 1024);
+  p.off_sfb = p.off_sfa + (gate_up ? 4 : 2) * kMxChunkBytes;
+  p.stage_bytes = (int)align_up((size_t)p.off_sfb + 2 * kMxChunkBytes, 1024);
+  p.n_stages = std::min(gate_up ? kMxMaxStagesGU : kMxMaxStagesDn,
+                        (kSmemBudget - 2 * kMxHeaderBytes) / p.stage_bytes);
   p.smem = 2 * kMxHeaderBytes + p.n_stages * p.stage_bytes;
   return p;
 }
@@ -513,12 +520,11 @@ MxArgs mx_args(const moe_layer* L, bool gate_up, int B, const moe_routing& r, co
   const int H = L->cfg.hidden, I = L->cfg.inter, k = L->cfg.top_k;
   MxArgs a;
   std::memset(&a, 0, sizeof(a));
-  a.sc = gate_up ? L->w.s_gate_up : L->w.s_down;
-  a.s_gstride = gate_up ? (long long)2 * I * (H / 32) : (long long)H * (I / 32);
-  a.a_rows = gate_up ? 2 * I : H;
+  a.wsf = gate_up ? L->wsf_gu : L->wsf_dn;
+  a.a_tiles = (gate_up ? 2 * I : H) / kMxRows;
+  a.up_tile = gate_up ? I / kMxRows : 0;
   a.K = gate_up ? H : I;
   a.out_rows = gate_up ? I : H;
-  a.up_off = gate_up ? I : 0;
   a.top_k = k;
   a.n_pairs = B * k;
   a.n_experts = L->cfg.n_experts;
@@ -526,12 +532,11 @@ MxArgs mx_args(const moe_layer* L, bool gate_up, int B, const moe_routing& r, co
   a.active = r.active;
   a.offsets = r.offsets;
   a.pair_ids = r.pair_ids;
-  a.asf = gate_up ? L->asfx : L->asfh;
-  a.act_rows = L->cfg.max_batch * k * kMxTerms;
+  a.bsf = gate_up ? L->bsfx : L->bsfh;
   a.n_max = p.n_max;
   a.out_f32 = out;
   a.next_aq = gate_up ? L->aqh : nullptr;
-  a.next_asf = gate_up ? L->asfh : nullptr;
+  a.next_bsf = gate_up ? L->bsfh : nullptr;
   a.n_stages = p.n_stages;
   a.stage_bytes = p.stage_bytes;
   a.off_up = p.off_up;
@@ -542,13 +547,15 @@ MxArgs mx_args(const moe_layer* L, bool gate_up, int B, const moe_routing& r, co
   return a;
 }
 
-// gate/up on the tensor cores: x -> E4M3 terms per pair position, then the
+// gate/up on the tensor cores: x -> E2M1 terms per pair position, then the
 // block-scaled MMA kernel (h fp32 into `h`, and h's terms for the down kernel)
 cudaError_t launch_mx_gate_up(moe_layer* L, const void* x, int B, const moe_routing& r, float* h, cudaStream_t st,
                               cudaEvent_t ev0, cudaEvent_t ev1) {
   const int H = L->cfg.hidden, k = L->cfg.top_k;
   cudaError_t e = launch_ex(mx_x_terms_kernel<kMxTerms>, B * k, 256, 0, st, L->pdl, static_cast<const uint16_t*>(x),
-                            H, k, B * k, static_cast<const int*>(r.pair_ids), L->aqx, L->asfx, L->err);
+                            H, k, B * k, L->cfg.n_experts, mx_n_max(B) / kMxTerms,
+                            static_cast<const int*>(r.pair_ids), static_cast<const int*>(r.topk_idx),
+                            static_cast<const int*>(r.offsets), L->aqx, L->bsfx, L->err);
   if (e != cudaSuccess) return e;
   const MxPlan p = mx_plan(true, B);
   const MxArgs a = mx_args(L, true, B, r, p, h);
@@ -962,10 +969,10 @@ moe_status_t moe_layer_create(const moe_layer_config* cfg, const moe_layer_weigh
   const size_t o_rs = take((size_t)MB * H * 2);
   const size_t o_os = take((size_t)MB * H * 2);
   const size_t mx_rows = (size_t)MB * k * kMxTerms;
-  const size_t o_aqx = take(mx_rows * H);
-  const size_t o_sfx = take(mx_rows * (H / 32));
-  const size_t o_aqh = take(mx_rows * I);
-  const size_t o_sfh = take(mx_rows * (I / 32));
+  const size_t o_aqx = take(mx_rows * (H / 2));
+  const size_t o_sfx = take((size_t)MB * k * ((H + kMxKChunk - 1) / kMxKChunk) * kMxChunkBytes);
+  const size_t o_aqh = take(mx_rows * (I / 2));
+  const size_t o_sfh = take((size_t)MB * k * ((I + kMxKChunk - 1) / kMxKChunk) * kMxChunkBytes);
   if (g_fail_next_alloc.exchange(false) || cudaMalloc(&L->arena, off) != cudaSuccess) {
     cudaGetLastError();
     delete L;
@@ -995,9 +1002,9 @@ moe_status_t moe_layer_create(const moe_layer_config* cfg, const moe_layer_weigh
   L->res_stage = reinterpret_cast<uint16_t*>(A + o_rs);
   L->out_stage = reinterpret_cast<uint16_t*>(A + o_os);
   L->aqx = reinterpret_cast<uint8_t*>(A + o_aqx);
-  L->asfx = reinterpret_cast<uint8_t*>(A + o_sfx);
+  L->bsfx = reinterpret_cast<uint8_t*>(A + o_sfx);
   L->aqh = reinterpret_cast<uint8_t*>(A + o_aqh);
-  L->asfh = reinterpret_cast<uint8_t*>(A + o_sfh);
+  L->bsfh = reinterpret_cast<uint8_t*>(A + o_sfh);
 
   cudaError_t e = cudaMemset(L->arena, 0, off);
   if (e == cudaSuccess) {
@@ -1026,17 +1033,39 @@ moe_status_t moe_layer_create(const moe_layer_config* cfg, const moe_layer_weigh
     }
     if (ok && (I % (kMmaRows / 2)) == 0 && (H % kMmaRows) == 0) L->grouped = true;
   }
-  // tcgen05 block-scaled path: K and output rows in whole 128-tiles, weights
-  // 32-byte aligned (4-bit TMA), tensor maps encodable
-  if (e == cudaSuccess && H % kMxKTile == 0 && I % kMxKTile == 0 &&
-      (reinterpret_cast<uintptr_t>(w->w_gate_up) & 31u) == 0 && (reinterpret_cast<uintptr_t>(w->w_down) & 31u) == 0) {
+  // tcgen05 block-scaled path: K and output rows in whole 128-tiles, tensor
+  // maps encodable (packed E2M1 rows as bytes: 128 per copy), and room for the
+  // weight scales in chunk layout, which are copied here once
+  if (e == cudaSuccess && H % kMxKChunk == 0 && I % kMxKChunk == 0) {
     const uint64_t mxr = (uint64_t)MB * k * kMxTerms;
-    L->mx = encode_map(&L->tm_agu, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, w->w_gate_up, (uint64_t)H,
-                       (uint64_t)E * 2 * I, (uint64_t)H / 2, kMxKTile, kMxRows) &&
-            encode_map(&L->tm_adn, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, w->w_down, (uint64_t)I, (uint64_t)E * H,
-                       (uint64_t)I / 2, kMxKTile, kMxRows) &&
-            encode_map(&L->tm_bx, CU_TENSOR_MAP_DATA_TYPE_UINT8, L->aqx, (uint64_t)H, mxr, (uint64_t)H, kMxKTile, 8) &&
-            encode_map(&L->tm_bh, CU_TENSOR_MAP_DATA_TYPE_UINT8, L->aqh, (uint64_t)I, mxr, (uint64_t)I, kMxKTile, 8);
+    L->mx = encode_map(&L->tm_agu, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->w_gate_up, (uint64_t)H / 2,
+                       (uint64_t)E * 2 * I, (uint64_t)H / 2, 128, kMxRows) &&
+            encode_map(&L->tm_adn, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->w_down, (uint64_t)I / 2, (uint64_t)E * H,
+                       (uint64_t)I / 2, 128, kMxRows) &&
+            encode_map(&L->tm_bx, CU_TENSOR_MAP_DATA_TYPE_UINT8, L->aqx, (uint64_t)H / 2, mxr, (uint64_t)H / 2, 128,
+                       kMxBBox) &&
+            encode_map(&L->tm_bh, CU_TENSOR_MAP_DATA_TYPE_UINT8, L->aqh, (uint64_t)I / 2, mxr, (uint64_t)I / 2, 128,
+                       kMxBBox);
+    if (L->mx) {
+      // the scale arrays hold one byte per 32 weights: the chunk copies are the same size
+      const size_t gu_bytes = (size_t)E * 2 * I * (H / 32), dn_bytes = (size_t)E * H * (I / 32);
+      if (cudaMalloc(&L->mx_mem, gu_bytes + dn_bytes) != cudaSuccess) {
+        cudaGetLastError();
+        L->mx = false;
+        if (c.flags & MOE_FLAG_MX_EXPERTS) {
+          moe_layer_destroy(L);
+          return MOE_ERR_OOM;
+        }
+      } else {
+        L->wsf_gu = reinterpret_cast<uint8_t*>(L->mx_mem);
+        L->wsf_dn = L->wsf_gu + gu_bytes;
+        const long long tiles_gu = (long long)E * 2 * I / kMxRows, tiles_dn = (long long)E * H / kMxRows;
+        mx_pack_scales_kernel<<<4 * L->num_sms, 256>>>(w->s_gate_up, tiles_gu, H, L->wsf_gu);
+        mx_pack_scales_kernel<<<4 * L->num_sms, 256>>>(w->s_down, tiles_dn, I, L->wsf_dn);
+        e = cudaGetLastError();
+        if (e == cudaSuccess) e = cudaDeviceSynchronize();
+      }
+    }
     L->mx_on = L->mx && (c.flags & MOE_FLAG_MX_EXPERTS);
   }
   if (e == cudaSuccess && L->mx) {
@@ -1108,6 +1137,7 @@ moe_status_t moe_layer_destroy(moe_layer_t L) {
   if (L->ev_join) cudaEventDestroy(L->ev_join);
   if (L->side) cudaStreamDestroy(L->side);
   if (L->arena) cudaFree(L->arena);
+  if (L->mx_mem) cudaFree(L->mx_mem);
   delete L;
   return MOE_OK;
 }

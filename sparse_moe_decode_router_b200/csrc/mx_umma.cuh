@@ -1,44 +1,50 @@
 // Routed MXFP4 expert projections on the 5th-generation tensor cores
-// (tcgen05 block-scaled MMA, sm_100a).
+// (tcgen05 block-scaled MMA, kind::mxf4, sm_100a).
 //
 // The decode-path pages use batch-specialised expert kernels (smzdm, section on
 // the four-step rework, first step); here one kernel design serves every batch
 // size by leaving all per-weight work to the TMA unit and the tensor cores:
 //
-//  * weights (A operand, M = 128 rows of one expert per MMA) are E2M1 codes
-//    copied by tiled TMA with the 16U4_ALIGN16B element type, which expands
-//    each 16 packed 4-bit values into a 16-byte shared-memory chunk (8 bytes
-//    of data, 8 of gap) -- the layout `tcgen05.mma.kind::mxf8f6f4` reads for a
-//    4-bit operand -- under the 128-byte swizzle.  No CUDA-core instruction
-//    touches a weight;
-//  * the weights' E8M0 block scales (one per row and 32 K elements) are
-//    gathered by one warp into the scale-factor chunk layout (128 rows x 4
-//    K-blocks in 512 bytes: row r = r0 + 32*r1 at byte 16*r0 + 4*r1 + block)
-//    and copied into tensor memory with `tcgen05.cp.32x128b.warpx4`;
-//  * activations (B operand) are MX values too: each token's activation row
-//    is split into kTerms E4M3 terms (the value, then what the first term
-//    missed, ...), each with its own E8M0 scale per 32 elements chosen so the
-//    block maximum fits E4M3's 448 without clipping.  A token's terms are
-//    separate B columns; the epilogue adds them.  Three terms carry about 12
-//    significant bits, more than the 11 of the f16 the CUDA-core kernels use;
+//  * weights (A operand, M = 128 rows of one expert per MMA) stay in their
+//    packed E2M1 form from HBM to the tensor core: a tiled TMA copies 128 rows
+//    x 128 bytes (256 K elements) per stage under the 128-byte swizzle, which
+//    is the K-major layout `tcgen05.mma.kind::mxf4` reads.  Shared memory holds
+//    exactly the bytes that HBM delivers, and every row segment a copy reads is
+//    one full 128-byte line;
+//  * the weights' E8M0 block scales (one per row and 32 K elements) are copied
+//    once, when the layer is created, into the scale-factor chunk layout that
+//    `tcgen05.cp.32x128b.warpx4` takes (128 rows x 4 K-blocks in 512 bytes: row
+//    r = r0 + 32*r1 at byte 16*r0 + 4*r1 + block), chunks of one row tile
+//    consecutive along K.  A stage's scales are then one 1-D bulk copy;
+//  * activations (B operand) are MX values too: each activation row is split
+//    into kTerms E2M1 terms (the value, then what the first term missed, ...),
+//    each with its own E8M0 scale per 32 elements chosen so the block maximum
+//    fits E2M1's 6 without clipping.  A token's terms are separate B columns;
+//    the epilogue adds them.  Five terms keep the block's error below about
+//    2^-14 of its largest element, finer than the f16 activations of the
+//    CUDA-core kernels;
 //  * B columns are rows of a buffer ordered like the routing plan's pair list
 //    (position q of pair_ids, term t -> row q*kTerms + t), so an expert's
-//    tokens are one contiguous run of rows: one tiled TMA per 8 rows;
+//    tokens are one contiguous run of rows (tiled TMA, 16 rows per copy).  The
+//    producer of the terms writes their scales straight into chunks keyed by
+//    the first position of the pass that reads them, so B's scales are a bulk
+//    copy as well;
 //  * the accumulators live in tensor memory (fp32, M = 128 lanes x N
 //    columns, two buffers so the epilogue of one item overlaps the MMAs of
 //    the next) and are read back with `tcgen05.ld.32x32b`.
 //
-// Warp roles (256 threads, one CTA per SM): warp 0 issues the TMA copies,
-// warp 1 owns the tensor memory and one of its lanes issues the MMAs, warp 2
-// builds the scale-factor chunks, warps 4..7 are the epilogue (warp w reads
-// TMEM lanes 32*(w%4) .. +31).  Every wait is bounded: a wait that gives up
-// records MOE_ERR_TIMEOUT in the error word and the CTA drains without work.
+// Warp roles (192 threads, one CTA per SM): warp 0 issues every copy (TMA
+// tiles and bulk scale chunks), warp 1 owns the tensor memory and one of its
+// lanes issues the scale copies into tensor memory and the MMAs, warps 2..5
+// are the epilogue (warp w reads TMEM lanes 32*(w%4) .. +31).  Every wait is
+// bounded: a wait that gives up records MOE_ERR_TIMEOUT in the error word and
+// the CTA drains without work.
 //
 // Epilogues: gate/up -> h = silu(g) * u per (row, token), written as fp32
-// (optional) and as the down projection's E4M3 terms; down -> y fp32 per
+// (optional) and as the down projection's E2M1 terms; down -> y fp32 per
 // (pair, row).  An item is 128 output rows of one active expert (gate/up:
 // 128 gate rows and the matching 128 up rows as two MMAs into two
-// accumulators), all K, for up to kMxNMax / kTerms tokens per pass; experts
+// accumulators), all K, for up to n_max / kTerms tokens per pass; experts
 // with more tokens take several passes over the same weights.
 #pragma once
 #include <cstdint>
@@ -51,29 +57,35 @@
 
 namespace moe {
 
-constexpr int kMxRows = 128;       // M: weight rows per MMA (one TMEM lane each)
-constexpr int kMxKTile = 128;      // K elements per pipeline stage (one 128-byte swizzle row)
-constexpr int kMxNMax = 64;        // B columns per pass (tokens x terms, padded to 16)
-constexpr int kMxMaxStages = 12;   // TMEM: scale chunks of 12 stages fit below column 432
-constexpr int kMxThreads = 256;
+constexpr int kMxRows = 128;        // M: weight rows per MMA (one TMEM lane each)
+constexpr int kMxKStage = 256;      // K elements per pipeline stage (one 128-byte swizzle row)
+constexpr int kMxKChunk = 128;      // K elements per scale-factor chunk (4 blocks of 32)
+constexpr int kMxChunkBytes = 512;  // one chunk: 128 rows (or B columns) x 4 E8M0 bytes
+constexpr int kMxATile = kMxRows * kMxKStage / 2;  // one A tile (16 KB, packed)
+constexpr int kMxBBox = 16;         // B rows per TMA copy (2 KB)
+constexpr int kMxTerms = 5;         // E2M1 terms per activation value
+constexpr int kMxNMax = 80;         // B columns per pass: 16 tokens x 5 terms
+constexpr int kMxTokMax = kMxNMax / kMxTerms;
+constexpr int kMxThreads = 192;
 constexpr int kMxTmemCols = 512;
-constexpr int kMxAccCols = 128;    // per accumulator buffer: gate [0, 64), up [64, 128)
-constexpr int kMxSfaCol0 = 256;    // per stage 8 columns: gate chunk, up chunk (256 + 8*12 <= 384)
-constexpr int kMxSfbCol0 = 384;    // per stage 4 columns (384 + 4*12 <= 512)
-static_assert(kMxSfaCol0 + 8 * kMxMaxStages <= kMxSfbCol0 && kMxSfbCol0 + 4 * kMxMaxStages <= kMxTmemCols,
-              "scale-factor columns");
+constexpr int kMxAccCols = 2 * kMxNMax;   // per accumulator buffer: gate [0, 80), up [80, 160)
+constexpr int kMxSfCol0 = 2 * kMxAccCols; // scale factors after the two buffers (column 320)
+constexpr int kMxSfColsGU = 24;           // per stage: gate, up and B, two chunks of 4 columns each
+constexpr int kMxSfColsDn = 16;           // per stage: A and B
+constexpr int kMxMaxStagesGU = (kMxTmemCols - kMxSfCol0) / kMxSfColsGU;  // 8
+constexpr int kMxMaxStagesDn = (kMxTmemCols - kMxSfCol0) / kMxSfColsDn;  // 12
+constexpr int kMxMaxStages = kMxMaxStagesDn;
+static_assert(kMxNMax % 16 == 0 && kMxNMax <= 128, "B columns: multiples of 16, one scale chunk");
+static_assert(kMxSfCol0 + kMxMaxStagesGU * kMxSfColsGU <= kMxTmemCols, "tensor memory");
 constexpr int kMxHeaderBytes = 1024;
 static_assert(8 * (2 * kMxMaxStages + 6) + 32 <= kMxHeaderBytes, "header");
-constexpr int kMxABytes = kMxRows * kMxKTile;  // one A tile in shared memory (16 KB, expanded)
-constexpr uint32_t kMxATx = kMxRows * kMxKTile / 2;  // bytes one A tile moves (packed)
 
 struct MxArgs {
-  const uint8_t* sc;        // weight E8M0 scales [E][rows][K/32]
-  long long s_gstride;      // bytes per expert in sc
-  int a_rows;               // weight rows per expert in the A tensor map (2I or H)
+  const uint8_t* wsf;       // weight scales, chunk layout [E * a_tiles][K/128][512]
+  int a_tiles;              // 128-row tiles per expert in the A matrix (2I/128 or H/128)
+  int up_tile;              // gate/up: tiles from a gate tile to its up tile (I/128); 0 for down
   int K;                    // reduction length, multiple of 128
   int out_rows;             // output rows per expert (I or H), multiple of 128
-  int up_off;               // gate/up: rows from a gate row to its up row (= I); 0 for down
   int top_k;
   int n_pairs;              // B * top_k of this call
   int n_experts;
@@ -81,12 +93,11 @@ struct MxArgs {
   const int* active;
   const int* offsets;
   const int* pair_ids;
-  const uint8_t* asf;       // activation term scales [act_rows][K/32]
-  int act_rows;             // rows of the activation-term buffers (capacity)
+  const uint8_t* bsf;       // activation scales, chunk layout [pass-start position][K/128][512]
   int n_max;                // B columns one pass may use (multiple of 16, <= kMxNMax)
   float* out_f32;           // gate/up: h [pair][I] (may be null); down: y [pair][H]
-  uint8_t* next_aq;         // gate/up: the down projection's E4M3 terms [act_rows][I]
-  uint8_t* next_asf;        // ... and their scales [act_rows][I/32]
+  uint8_t* next_aq;         // gate/up: the down projection's E2M1 terms [pos*kTerms + t][I/2]
+  uint8_t* next_bsf;        // ... and their scale chunks [pos][I/128][512]
   int n_stages;
   int stage_bytes;          // multiple of 1024
   int off_up, off_b, off_sfa, off_sfb;  // byte offsets inside a stage
@@ -116,13 +127,14 @@ __device__ __forceinline__ void tc_commit(uint64_t* bar) {
                : "memory");
 }
 
-// D[tmem] (+)= A[smem] * B[smem], block-scaled: A scales at sfa, B scales at sfb
-__device__ __forceinline__ void tc_mma_mx(uint32_t d, uint64_t adesc, uint64_t bdesc, uint32_t idesc, uint32_t sfa,
-                                          uint32_t sfb, uint32_t accumulate) {
+// D[tmem] (+)= A[smem] * B[smem], both packed E2M1, K = 64, block-scaled by
+// E8M0 factors (two per row and column: 32-element blocks) at sfa and sfb
+__device__ __forceinline__ void tc_mma_mxf4(uint32_t d, uint64_t adesc, uint64_t bdesc, uint32_t idesc, uint32_t sfa,
+                                            uint32_t sfb, uint32_t accumulate) {
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d),
+      "tcgen05.mma.cta_group::1.kind::mxf4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d),
       "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
       : "memory");
 }
@@ -159,11 +171,12 @@ __device__ __forceinline__ uint64_t desc_sf(uint32_t saddr) {
          ((uint64_t)1 << 46);
 }
 
-// instruction descriptor, kind::mxf8f6f4 block-scaled: A E2M1, B E4M3, both
-// K-major, E8M0 scale factors, M = 128, N columns; the K-block of each scale
-// vector is set per MMA (bits 29-30 for A, 4-5 for B)
+// instruction descriptor, kind::mxf4 block-scaled: A and B E2M1, both
+// K-major, E8M0 scale factors, M = 128, N columns, K = 64; the byte of each
+// scale word that the MMA starts at (0 or 2: two 32-element blocks per MMA)
+// is set per MMA (bits 29-30 for A, 4-5 for B)
 __host__ __device__ constexpr uint32_t mx_idesc(int n) {
-  return (5u << 7) | (0u << 10) | ((uint32_t)(n >> 3) << 17) | (1u << 23) | ((uint32_t)(kMxRows >> 4) << 24);
+  return (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | (1u << 23) | ((uint32_t)(kMxRows >> 4) << 24);
 }
 
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y, uint64_t* bar,
@@ -189,14 +202,14 @@ __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
 
 // ---------------------------------------------------------------------------
 // MX activation terms.  A term of a 32-element block: scale 2^e with e the
-// smallest integer that keeps max|v| * 2^-e <= 448 (E4M3's largest finite
-// value), then each element rounded to nearest even E4M3 (saturating).
+// smallest integer that keeps max|v| * 2^-e <= 6 (E2M1's largest value), then
+// each element rounded to the nearest E2M1 value, ties to the even code.
 __device__ __forceinline__ int mx_scale_exp(float amax) {
   if (!(amax > 0.f)) return 0;
   const uint32_t u = __float_as_uint(amax);
   const int ef = (int)((u >> 23) & 0xFFu);
   const int E = ef ? ef - 127 : -127;
-  const int e = E - 8 + ((u & 0x7FFFFFu) > 0x600000u ? 1 : 0);  // 448 = 1.75 * 2^8
+  const int e = E - 2 + ((u & 0x7FFFFFu) > 0x400000u ? 1 : 0);  // 6 = 1.5 * 2^2
   return max(-127, min(127, e));
 }
 
@@ -205,34 +218,62 @@ __device__ __forceinline__ float pow2_exact(int e) {
   return __uint_as_float(e >= -126 ? (uint32_t)(e + 127) << 23 : 0x00400000u);
 }
 
-__device__ __forceinline__ uint32_t f32_to_e4m3(float v) {
-  uint16_t d;
-  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %1;" : "=h"(d) : "f"(v));
-  return d & 0xFFu;
+// E2M1 code (sign bit 3) of v, round to nearest even, saturating at 6.  The
+// value is converted into both halves of the byte, so the nibble order of
+// the packed conversion does not matter.
+__device__ __forceinline__ uint32_t f32_to_e2m1(float v) {
+  uint32_t r;
+  asm("{\n\t.reg .b8 t;\n\tcvt.rn.satfinite.e2m1x2.f32 t, %1, %1;\n\tmov.b32 %0, {t, t, t, t};\n\t}"
+      : "=r"(r)
+      : "f"(v));
+  return r & 0xFu;
 }
 
-__device__ __forceinline__ float e4m3_to_f32(uint32_t b) {
-  uint32_t h2;
-  const uint16_t in = (uint16_t)(b | (b << 8));
-  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(in));
-  return __half2float(__ushort_as_half((unsigned short)(h2 & 0xFFFFu)));
+// value of an E2M1 code: magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6
+__device__ __forceinline__ float e2m1_to_f32(uint32_t c) {
+  const uint32_t m = c & 7u;
+  const float mag = m < 2u ? 0.5f * (float)m
+                           : __uint_as_float(((m >> 1) + 126u) << 23) * (1.0f + 0.5f * (float)(m & 1u));
+  return (c & 8u) ? -mag : mag;
+}
+
+// byte of a B column's scale in its chunk: column n = r0 + 32*r1, K-block kb
+__device__ __forceinline__ int sf_chunk_byte(int n, int kb) { return 16 * (n & 31) + 4 * (n >> 5) + kb; }
+
+// first position of the pass that reads position q (passes of tpp tokens
+// from the expert's offset); -1 if the routing plan is inconsistent
+__device__ __forceinline__ int pass_start(int q, int top_k, int n_pairs, int n_experts, int tpp,
+                                          const int* __restrict__ pair_ids, const int* __restrict__ topk_idx,
+                                          const int* __restrict__ offsets) {
+  const int p = __ldcg(pair_ids + q);
+  if (p < 0 || p >= n_pairs) return -1;
+  const int e = __ldcg(topk_idx + p);
+  if (e < 0 || e >= n_experts) return -1;
+  const int off = __ldcg(offsets + e), end = __ldcg(offsets + e + 1);
+  if (off < 0 || q < off || q >= end) return -1;
+  return off + (q - off) / tpp * tpp;
 }
 
 // x (bf16 [B][K]) -> terms of the gate/up activations, one CTA per position
-// q of the pair list: rows q*kTerms + t of aq [.][K] and asf [.][K/32].
+// q of the pair list: rows q*kTerms + t of aq [.][K/2] (packed E2M1, even
+// element in the low nibble) and their scales into the chunks of q's pass.
 template <int kTerms>
 __global__ void __launch_bounds__(256) mx_x_terms_kernel(const uint16_t* __restrict__ x, int K, int top_k, int n_pairs,
-                                                         const int* __restrict__ pair_ids, uint8_t* __restrict__ aq,
-                                                         uint8_t* __restrict__ asf, int* err) {
+                                                         int n_experts, int tpp, const int* __restrict__ pair_ids,
+                                                         const int* __restrict__ topk_idx,
+                                                         const int* __restrict__ offsets, uint8_t* __restrict__ aq,
+                                                         uint8_t* __restrict__ bsf, int* err) {
   pdl_wait();
   const int q = blockIdx.x;
-  int p = pair_ids[q];
-  if (p < 0 || p >= n_pairs) {
+  const int p0 = pass_start(q, top_k, n_pairs, n_experts, tpp, pair_ids, topk_idx, offsets);
+  if (p0 < 0) {
     if (threadIdx.x == 0) atomicExch(err, kErrBadPlan);
-    p = 0;
+    pdl_launch_dependents();
+    return;
   }
-  const int b = p / top_k;
-  const int nblk = K >> 5;
+  const int b = __ldcg(pair_ids + q) / top_k;
+  const int n0 = (q - p0) * kTerms;  // this position's first B column in its pass
+  const int nblk = K >> 5, KC = K / kMxKChunk;
   for (int blk = threadIdx.x; blk < nblk; blk += blockDim.x) {
     const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)b * K + 32 * blk);
     float v[32];
@@ -246,6 +287,7 @@ __global__ void __launch_bounds__(256) mx_x_terms_kernel(const uint16_t* __restr
         v[8 * i + 2 * j + 1] = bf16hi_to_f32(w[j]);
       }
     }
+    uint8_t* chunk = bsf + ((size_t)p0 * KC + (blk >> 2)) * kMxChunkBytes;
 #pragma unroll
     for (int t = 0; t < kTerms; ++t) {
       float amax = 0.f;
@@ -253,27 +295,45 @@ __global__ void __launch_bounds__(256) mx_x_terms_kernel(const uint16_t* __restr
       for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(v[i]));
       const int e = mx_scale_exp(amax);
       const float inv = pow2_exact(-e), sc = pow2_exact(e);
-      uint32_t packed[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) packed[i] = 0u;
+      uint32_t packed[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
       for (int i = 0; i < 32; ++i) {
-        const uint32_t c = f32_to_e4m3(v[i] * inv);
-        packed[i >> 2] |= c << (8 * (i & 3));
-        v[i] -= e4m3_to_f32(c) * sc;
+        const uint32_t c = f32_to_e2m1(v[i] * inv);
+        packed[i >> 3] |= c << (4 * (i & 7));
+        v[i] -= e2m1_to_f32(c) * sc;
       }
-      uint4* dst = reinterpret_cast<uint4*>(aq + ((size_t)q * kTerms + t) * K + 32 * blk);
-      dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
-      dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
-      asf[((size_t)q * kTerms + t) * nblk + blk] = (uint8_t)(e + 127);
+      *reinterpret_cast<uint4*>(aq + ((size_t)q * kTerms + t) * (K / 2) + 16 * blk) =
+          make_uint4(packed[0], packed[1], packed[2], packed[3]);
+      chunk[sf_chunk_byte(n0 + t, blk & 3)] = (uint8_t)(e + 127);
     }
   }
   pdl_launch_dependents();
 }
 
+// Weight scales [n_tiles * 128 rows][K/32] -> chunk layout [n_tiles][K/128][512]
+// (layer creation, once per projection)
+__global__ void mx_pack_scales_kernel(const uint8_t* __restrict__ sc, long long n_tiles, int K,
+                                      uint8_t* __restrict__ out) {
+  const int sblk = K / 32, KC = K / kMxKChunk;
+  const long long n = n_tiles * KC * 32;  // one thread per (chunk, r0)
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
+    const int r0 = (int)(i & 31);
+    const long long c = i >> 5;
+    const int kc = (int)(c % KC);
+    const long long tile = c / KC;
+    uint32_t w[4];
+#pragma unroll
+    for (int r1 = 0; r1 < 4; ++r1) {
+      const uint8_t* s = sc + (tile * kMxRows + r0 + 32 * r1) * sblk + 4 * kc;
+      w[r1] = (uint32_t)s[0] | ((uint32_t)s[1] << 8) | ((uint32_t)s[2] << 16) | ((uint32_t)s[3] << 24);
+    }
+    *reinterpret_cast<uint4*>(out + c * kMxChunkBytes + 16 * r0) = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+}
+
 // ---------------------------------------------------------------------------
 // Per-CTA item walk shared by every role: items are (active group, 128-row
-// tile), contiguous ranges per CTA; each item runs one pass per kMxNMax /
+// tile), contiguous ranges per CTA; each item runs one pass per n_max /
 // kTerms tokens of its expert.
 struct MxUnit {
   int e;      // expert
@@ -288,18 +348,17 @@ struct MxWalk {
   const MxArgs& a;
   long long it, hi;
   int n_rt, pass, npass, e, tok0, cnt;
-  bool bad;
   __device__ MxWalk(const MxArgs& args, long long lo, long long hi_, int nrt)
-      : a(args), it(lo), hi(hi_), n_rt(nrt), pass(0), npass(0), e(0), tok0(0), cnt(0), bad(false) {
+      : a(args), it(lo), hi(hi_), n_rt(nrt), pass(0), npass(0), e(0), tok0(0), cnt(0) {
     if (it < hi) load();
   }
   __device__ void load() {
     const int g = (int)(it / n_rt);
-    e = a.active[g];
-    if (e < 0 || e >= a.n_experts) { bad = true; e = 0; }
-    tok0 = a.offsets[e];
-    cnt = a.offsets[e + 1] - tok0;
-    if (tok0 < 0 || cnt < 1 || tok0 + cnt > a.n_pairs) { bad = true; tok0 = 0; cnt = 1; }
+    e = __ldcg(a.active + g);
+    if (e < 0 || e >= a.n_experts) e = 0;
+    tok0 = __ldcg(a.offsets + e);
+    cnt = __ldcg(a.offsets + e + 1) - tok0;
+    if (tok0 < 0 || cnt < 1 || tok0 + cnt > a.n_pairs) { tok0 = 0; cnt = 1; }
     const int tpp = a.n_max / kTerms;
     npass = (cnt + tpp - 1) / tpp;
     pass = 0;
@@ -321,7 +380,6 @@ struct MxWalk {
   }
 };
 
-template <int kTerms>
 __device__ __forceinline__ float warp_amax(float v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
@@ -332,7 +390,9 @@ template <bool kSwiglu, int kTerms>
 __global__ void __launch_bounds__(kMxThreads, 1)
     mx_expert_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                      const MxArgs a) {
-  static_assert(kMxNMax % 16 == 0 && kTerms >= 1 && kTerms <= 3, "terms");
+  static_assert(kTerms >= 1 && kTerms * kMxTokMax <= kMxNMax, "terms");
+  constexpr int kSfCols = kSwiglu ? kMxSfColsGU : kMxSfColsDn;
+  constexpr int kMaxNs = kSwiglu ? kMxMaxStagesGU : kMxMaxStagesDn;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   // header: barriers and flags; the stage ring starts at the next 1024-byte boundary
@@ -349,11 +409,11 @@ __global__ void __launch_bounds__(kMxThreads, 1)
   volatile int* s_abort = reinterpret_cast<volatile int*>(hdr + 8 * (2 * kMxMaxStages + 6) + 16);
   volatile int* s_last = s_abort + 1;
 
-  const int K = a.K, KT = K / kMxKTile, sblk = K / 32;
+  const int K = a.K, KC = K / kMxKChunk, KS = (KC + 1) / 2;
   const int ns = a.n_stages;
   if (tid == 0) {
     for (int s = 0; s < kMxMaxStages; ++s) {
-      mbar_init(&full_bar[s], 2);    // the TMA thread's expect-tx arrive + the scale-factor warp
+      mbar_init(&full_bar[s], 1);    // the TMA thread's expect-tx arrive
       mbar_init(&empty_bar[s], 1);   // tcgen05.commit after the stage's MMAs
     }
     for (int b = 0; b < 2; ++b) {
@@ -384,7 +444,7 @@ __global__ void __launch_bounds__(kMxThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *s_tmem;
 
-  int n_groups = *a.n_active;
+  int n_groups = __ldcg(a.n_active);
   if (n_groups < 0 || n_groups > a.n_experts) {
     if (tid == 0) atomicExch(a.err, kErrBadPlan);
     n_groups = n_groups < 0 ? 0 : a.n_experts;
@@ -393,8 +453,8 @@ __global__ void __launch_bounds__(kMxThreads, 1)
   const long long n_items = (long long)n_groups * n_rt;
   const long long lo = n_items * blockIdx.x / gridDim.x;
   const long long hi = n_items * (blockIdx.x + 1) / gridDim.x;
-  const bool plan_ok = ns >= 1 && ns <= kMxMaxStages && (K % kMxKTile) == 0 && (a.out_rows % kMxRows) == 0 &&
-                       a.n_max >= 16 && a.n_max <= kMxNMax && (a.n_max % 16) == 0;
+  const bool plan_ok = ns >= 1 && ns <= kMaxNs && (K % kMxKChunk) == 0 && (a.out_rows % kMxRows) == 0 &&
+                       a.n_max >= 16 && a.n_max <= kMxNMax && (a.n_max % 16) == 0 && a.n_max >= kTerms;
   if (!plan_ok) {
     if (tid == 0) atomicExch(a.err, kErrBadPlan);
   }
@@ -408,19 +468,33 @@ __global__ void __launch_bounds__(kMxThreads, 1)
       uint32_t ph = 0;
       for (MxWalk<kTerms> w(a, lo, hi, n_rt); w.valid() && !*s_abort; w.next()) {
         const MxUnit u = w.unit();
-        const int arow = u.e * a.a_rows + u.rt * kMxRows;
-        for (int kt = 0; kt < KT; ++kt) {
+        const long long tile = (long long)u.e * a.a_tiles + u.rt;  // the gate (or only) 128-row tile
+        const int arow = (int)(tile * kMxRows);
+        const uint8_t* sfa_g = a.wsf + tile * KC * kMxChunkBytes;
+        const uint8_t* sfa_u = a.wsf + (tile + a.up_tile) * KC * kMxChunkBytes;
+        const uint8_t* sfb = a.bsf + (size_t)u.tok * KC * kMxChunkBytes;
+        const int nbox = u.n / kMxBBox;
+        for (int kt = 0; kt < KS; ++kt) {
           if (!mbar_wait_bounded(&empty_bar[s], ph ^ 1u, *s_abort ? lim_short : lim_long)) {
             atomicExch(a.err, kErrTimeout);
             *s_abort = 1;
             break;
           }
-          const uint32_t st = smem_addr(ring + (size_t)s * a.stage_bytes);
-          mbar_arrive_expect_tx(&full_bar[s], (kSwiglu ? 2u : 1u) * kMxATx + (uint32_t)u.n * 128u);
-          tma_load_2d(st, &tmA, kt * kMxKTile, arow, &full_bar[s], pol);
-          if (kSwiglu) tma_load_2d(st + a.off_up, &tmA, kt * kMxKTile, arow + a.up_off, &full_bar[s], pol);
-          for (int j = 0; j < u.n / 8; ++j)
-            tma_load_2d_nohint(st + a.off_b + 1024 * j, &tmB, kt * kMxKTile, u.tok * kTerms + 8 * j, &full_bar[s]);
+          const int nck = min(2, KC - 2 * kt);  // scale chunks of this stage (1 in a last half stage)
+          const uint32_t cb = (uint32_t)(nck * kMxChunkBytes);
+          unsigned char* st = ring + (size_t)s * a.stage_bytes;
+          const uint32_t sa = smem_addr(st);
+          mbar_arrive_expect_tx(&full_bar[s], (kSwiglu ? 2u : 1u) * ((uint32_t)kMxATile + cb) +
+                                                  (uint32_t)nbox * (kMxBBox * 128u) + cb);
+          tma_load_2d(sa, &tmA, kt * 128, arow, &full_bar[s], pol);
+          if (kSwiglu) tma_load_2d(sa + a.off_up, &tmA, kt * 128, arow + a.up_tile * kMxRows, &full_bar[s], pol);
+          for (int j = 0; j < nbox; ++j)
+            tma_load_2d_nohint(sa + a.off_b + j * kMxBBox * 128, &tmB, kt * 128, u.tok * kTerms + kMxBBox * j,
+                               &full_bar[s]);
+          const size_t ck = (size_t)2 * kt * kMxChunkBytes;
+          bulk_g2s(st + a.off_sfa, sfa_g + ck, cb, &full_bar[s], pol);
+          if (kSwiglu) bulk_g2s(st + a.off_sfa + 2 * kMxChunkBytes, sfa_u + ck, cb, &full_bar[s], pol);
+          bulk_g2s_nohint(st + a.off_sfb, sfb + ck, cb, &full_bar[s]);
           if (++s == ns) { s = 0; ph ^= 1u; }
         }
       }
@@ -443,101 +517,6 @@ __global__ void __launch_bounds__(kMxThreads, 1)
         }
       }
     }
-  } else if (plan_ok && warp == 2) {
-    // ------------------------- scale-factor chunks ----------------------------
-    // Weight scales are static (read-only path); the activation scales come
-    // from the preceding kernel and are read through L2 (coherent path).
-    // Lane l covers rows l + 32*m (m = 0..3) of the A tile(s) and B columns
-    // l + 32*m (m = 0..1).  Where a scale row is a multiple of 16 bytes long,
-    // one 16-byte load per row fetches four stages' scale bytes, and the next
-    // group of four is requested before the current one is stored, so the
-    // loads' latency overlaps the stages.
-    const bool wide = (sblk % 16) == 0;
-    int s = 0;
-    uint32_t ph = 0;
-    for (MxWalk<kTerms> w(a, lo, hi, n_rt); w.valid() && !*s_abort; w.next()) {
-      const MxUnit u = w.unit();
-      const uint8_t* sg = a.sc + (long long)u.e * a.s_gstride;
-      const int r0 = u.rt * kMxRows;
-      // 16-byte groups (4 K-tiles) of this lane's rows: A gate, A up, B
-      auto load_group = [&](int kg, uint4 (&ga)[4], uint4 (&ua)[4], uint4 (&bb)[2]) {
-#pragma unroll
-        for (int m = 0; m < 4; ++m) {
-          ga[m] = __ldg(reinterpret_cast<const uint4*>(sg + (size_t)(r0 + lane + 32 * m) * sblk + 4 * kg));
-          if (kSwiglu)
-            ua[m] = __ldg(reinterpret_cast<const uint4*>(sg + (size_t)(r0 + a.up_off + lane + 32 * m) * sblk + 4 * kg));
-        }
-#pragma unroll
-        for (int m = 0; m < 2; ++m) {
-          const int n = lane + 32 * m, row = u.tok * kTerms + n;
-          bb[m] = (n < u.n && row < a.act_rows)
-                      ? __ldcg(reinterpret_cast<const uint4*>(a.asf + (size_t)row * sblk + 4 * kg))
-                      : make_uint4(0u, 0u, 0u, 0u);
-        }
-      };
-      uint4 cg[4], cu[4], cb[2], ng[4], nu[4], nb[2];
-      if (wide) load_group(0, cg, cu, cb);
-      bool stop = false;
-      for (int kg = 0; kg < KT && !stop; kg += 4) {
-        if (wide && kg + 4 < KT) load_group(kg + 4, ng, nu, nb);
-#pragma unroll
-        for (int j4 = 0; j4 < 4; ++j4) {
-          const int kt = kg + j4;
-          if (kt >= KT) break;
-          bool ok = mbar_wait_bounded(&empty_bar[s], ph ^ 1u, *s_abort ? lim_short : lim_long);
-          ok = __all_sync(0xFFFFFFFFu, ok);
-          if (!ok) {
-            if (lane == 0) atomicExch(a.err, kErrTimeout);
-            *s_abort = 1;
-            stop = true;
-            break;
-          }
-          uint32_t vg[4], vu[4], vb[4];
-          if (wide) {
-#pragma unroll
-            for (int m = 0; m < 4; ++m) {
-              vg[m] = j4 == 0 ? cg[m].x : j4 == 1 ? cg[m].y : j4 == 2 ? cg[m].z : cg[m].w;
-              vu[m] = j4 == 0 ? cu[m].x : j4 == 1 ? cu[m].y : j4 == 2 ? cu[m].z : cu[m].w;
-            }
-#pragma unroll
-            for (int m = 0; m < 2; ++m)
-              vb[m] = j4 == 0 ? cb[m].x : j4 == 1 ? cb[m].y : j4 == 2 ? cb[m].z : cb[m].w;
-          } else {
-#pragma unroll
-            for (int m = 0; m < 4; ++m) {
-              vg[m] = __ldg(reinterpret_cast<const uint32_t*>(sg + (size_t)(r0 + lane + 32 * m) * sblk + 4 * kt));
-              vu[m] = kSwiglu ? __ldg(reinterpret_cast<const uint32_t*>(sg + (size_t)(r0 + a.up_off + lane + 32 * m) *
-                                                                                 sblk + 4 * kt))
-                              : 0u;
-            }
-#pragma unroll
-            for (int m = 0; m < 2; ++m) {
-              const int n = lane + 32 * m, row = u.tok * kTerms + n;
-              vb[m] = (n < u.n && row < a.act_rows)
-                          ? __ldcg(reinterpret_cast<const uint32_t*>(a.asf + (size_t)row * sblk + 4 * kt))
-                          : 0u;
-            }
-          }
-          vb[2] = vb[3] = 0u;  // B columns 64..127 (beyond kMxNMax)
-          unsigned char* st = ring + (size_t)s * a.stage_bytes;
-          *reinterpret_cast<uint4*>(st + a.off_sfa + 16 * lane) = make_uint4(vg[0], vg[1], vg[2], vg[3]);
-          if (kSwiglu)
-            *reinterpret_cast<uint4*>(st + a.off_sfa + 512 + 16 * lane) = make_uint4(vu[0], vu[1], vu[2], vu[3]);
-          *reinterpret_cast<uint4*>(st + a.off_sfb + 16 * lane) = make_uint4(vb[0], vb[1], vb[2], vb[3]);
-          // generic-proxy stores -> visible to tcgen05.cp (async proxy)
-          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&full_bar[s]);
-          if (++s == ns) { s = 0; ph ^= 1u; }
-        }
-        if (wide) {
-#pragma unroll
-          for (int m = 0; m < 4; ++m) { cg[m] = ng[m]; cu[m] = nu[m]; }
-#pragma unroll
-          for (int m = 0; m < 2; ++m) cb[m] = nb[m];
-        }
-      }
-    }
   } else if (plan_ok && warp == 1) {
     // ------------------------------ MMA issuer --------------------------------
     if (lane == 0) {
@@ -553,10 +532,10 @@ __global__ void __launch_bounds__(kMxThreads, 1)
         }
         tc_fence_after();
         const uint32_t d_g = tmem + (uint32_t)(b * kMxAccCols);
-        const uint32_t d_u = d_g + (uint32_t)(kMxAccCols / 2);
+        const uint32_t d_u = d_g + (uint32_t)kMxNMax;
         const uint32_t idesc = mx_idesc(u.n);
         bool ok = true;
-        for (int kt = 0; kt < KT && ok; ++kt) {
+        for (int kt = 0; kt < KS && ok; ++kt) {
           if (!mbar_wait_bounded(&full_bar[s], ph, *s_abort ? lim_short : lim_long)) {
             atomicExch(a.err, kErrTimeout);
             *s_abort = 1;
@@ -564,22 +543,26 @@ __global__ void __launch_bounds__(kMxThreads, 1)
             break;
           }
           tc_fence_after();
+          const int nck = min(2, KC - 2 * kt);
           const uint32_t st = smem_addr(ring + (size_t)s * a.stage_bytes);
-          const uint32_t sfa_g = tmem + (uint32_t)(kMxSfaCol0 + 8 * s), sfa_u = sfa_g + 4u;
-          const uint32_t sfb = tmem + (uint32_t)(kMxSfbCol0 + 4 * s);
-          tc_cp_32x128_x4(sfa_g, desc_sf(st + a.off_sfa));
-          if (kSwiglu) tc_cp_32x128_x4(sfa_u, desc_sf(st + a.off_sfa + 512));
-          tc_cp_32x128_x4(sfb, desc_sf(st + a.off_sfb));
+          const uint32_t sf = tmem + (uint32_t)(kMxSfCol0 + kSfCols * s);
+          const uint32_t sfa_g = sf, sfa_u = sf + 8u, sfb = sf + (kSwiglu ? 16u : 8u);
+          for (int c = 0; c < nck; ++c) {
+            tc_cp_32x128_x4(sfa_g + 4u * c, desc_sf(st + a.off_sfa + c * kMxChunkBytes));
+            if (kSwiglu) tc_cp_32x128_x4(sfa_u + 4u * c, desc_sf(st + a.off_sfa + (2 + c) * kMxChunkBytes));
+            tc_cp_32x128_x4(sfb + 4u * c, desc_sf(st + a.off_sfb + c * kMxChunkBytes));
+          }
           const uint64_t ad = desc_sw128(st), bd = desc_sw128(st + a.off_b);
           const uint64_t ud = kSwiglu ? desc_sw128(st + a.off_up) : 0ull;
-#pragma unroll
-          for (int j = 0; j < kMxKTile / 32; ++j) {
-            // K-block j of the stage: +32 bytes in every swizzled row; scale byte j
-            const uint32_t id = idesc | ((uint32_t)j << 29) | ((uint32_t)j << 4);
+          for (int j = 0; j < 2 * nck; ++j) {
+            // MMA j of the stage: +32 bytes in every swizzled row; its two
+            // scale bytes start at byte 2*(j%2) of chunk j/2's words
+            const uint32_t sb = 2u * (uint32_t)(j & 1), col = 4u * (uint32_t)(j >> 1);
+            const uint32_t id = idesc | (sb << 29) | (sb << 4);
             const uint32_t acc = (kt > 0 || j > 0) ? 1u : 0u;
-            const uint32_t sel = (uint32_t)j << 30;
-            tc_mma_mx(d_g, ad + 2u * j, bd + 2u * j, id, sfa_g | sel, sfb | sel, acc);
-            if (kSwiglu) tc_mma_mx(d_u, ud + 2u * j, bd + 2u * j, id, sfa_u | sel, sfb | sel, acc);
+            const uint32_t tag = sb << 30;
+            tc_mma_mxf4(d_g, ad + 2u * j, bd + 2u * j, id, (sfa_g + col) | tag, (sfb + col) | tag, acc);
+            if (kSwiglu) tc_mma_mxf4(d_u, ud + 2u * j, bd + 2u * j, id, (sfa_u + col) | tag, (sfb + col) | tag, acc);
           }
           tc_commit(&empty_bar[s]);  // the stage is free once these MMAs have read it
           if (++s == ns) { s = 0; ph ^= 1u; }
@@ -592,9 +575,9 @@ __global__ void __launch_bounds__(kMxThreads, 1)
       if (!mbar_wait_bounded(done_bar, 0u, lim_long)) atomicExch(a.err, kErrTimeout);
     }
     __syncwarp();
-  } else if (plan_ok && warp >= 4) {
+  } else if (plan_ok && warp >= 2) {
     // ------------------------------ epilogue ----------------------------------
-    const int q = warp & 3;
+    const int q = warp & 3;  // TMEM lane quadrant of this warp
     const uint32_t lane_base = tmem + ((uint32_t)(32 * q) << 16);
     int uc = 0;
     uint32_t epi_ph = 0;
@@ -612,6 +595,7 @@ __global__ void __launch_bounds__(kMxThreads, 1)
       }
       return ok;
     };
+    const int KCn = a.out_rows / kMxKChunk;  // gate/up: chunks per row of the down projection's B
     for (MxWalk<kTerms> w(a, lo, hi, n_rt); w.valid(); w.next(), ++uc) {
       const MxUnit u = w.unit();
       const int b = uc & 1;
@@ -623,55 +607,57 @@ __global__ void __launch_bounds__(kMxThreads, 1)
         break;
       }
       tc_fence_after();
-      float g[kMxNMax], up[kSwiglu ? kMxNMax : 1];
+      // per token: the sum of its kTerms columns, ascending
+      float gs[kMxTokMax], us[kMxTokMax];
+#pragma unroll
+      for (int i = 0; i < kMxTokMax; ++i) gs[i] = us[i] = 0.f;
 #pragma unroll
       for (int c = 0; c < kMxNMax / 16; ++c) {
         if (16 * c < u.n) {  // warp-uniform
-          float t16[16];
-          tc_ld16(lane_base + (uint32_t)(b * kMxAccCols + 16 * c), t16);
+          float g16[16], u16[16];
+          tc_ld16(lane_base + (uint32_t)(b * kMxAccCols + 16 * c), g16);
+          if (kSwiglu) tc_ld16(lane_base + (uint32_t)(b * kMxAccCols + kMxNMax + 16 * c), u16);
+          tc_wait_ld();
 #pragma unroll
-          for (int i = 0; i < 16; ++i) g[16 * c + i] = t16[i];
-          if (kSwiglu) {
-            tc_ld16(lane_base + (uint32_t)(b * kMxAccCols + kMxAccCols / 2 + 16 * c), t16);
-#pragma unroll
-            for (int i = 0; i < 16; ++i) up[16 * c + i] = t16[i];
+          for (int i = 0; i < 16; ++i) {
+            gs[(16 * c + i) / kTerms] += g16[i];
+            if (kSwiglu) us[(16 * c + i) / kTerms] += u16[i];
           }
         }
       }
-      tc_wait_ld();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&acc_empty[b]);
       const int row = u.rt * kMxRows + 32 * q + lane;  // output row of this lane
 #pragma unroll
-      for (int i = 0; i < kMxNMax / kTerms; ++i) {
+      for (int i = 0; i < kMxTokMax; ++i) {
         if (i < u.ntok) {  // warp-uniform
-          float gs = 0.f, us = 0.f;
-#pragma unroll
-          for (int t = 0; t < kTerms; ++t) {
-            gs += g[i * kTerms + t];
-            if (kSwiglu) us += up[i * kTerms + t];
-          }
           const int pos = u.tok + i;
-          int pr = a.pair_ids[pos];
+          int pr = __ldcg(a.pair_ids + pos);
           if (pr < 0 || pr >= a.n_pairs) pr = 0;
           if (kSwiglu) {
-            const float hv = gs / (1.0f + expf(-gs)) * us;
+            const float hv = gs[i] / (1.0f + expf(-gs[i])) * us[i];
             if (a.out_f32) a.out_f32[(size_t)pr * a.out_rows + row] = hv;
-            // the down projection's terms: this warp's 32 rows are one 32-element block of h
+            // the down projection's terms: this warp's 32 rows are one
+            // 32-element block of h; lanes 8m .. 8m+7 make one 32-bit word
             float r = hv;
-            const int blk = row >> 5;
+            uint8_t* chunk = a.next_bsf + ((size_t)u.tok * KCn + u.rt) * kMxChunkBytes;
 #pragma unroll
             for (int t = 0; t < kTerms; ++t) {
-              const int e = mx_scale_exp(warp_amax<kTerms>(fabsf(r)));
-              const uint32_t c = f32_to_e4m3(r * pow2_exact(-e));
-              r -= e4m3_to_f32(c) * pow2_exact(e);
+              const int e = mx_scale_exp(warp_amax(fabsf(r)));
+              const uint32_t c = f32_to_e2m1(r * pow2_exact(-e));
+              r -= e2m1_to_f32(c) * pow2_exact(e);
+              uint32_t v = c << (4 * (lane & 7));
+#pragma unroll
+              for (int o = 1; o < 8; o <<= 1) v |= __shfl_xor_sync(0xFFFFFFFFu, v, o);
               const size_t drow = (size_t)pos * kTerms + t;
-              a.next_aq[drow * a.out_rows + row] = (uint8_t)c;
-              if (lane == 0) a.next_asf[drow * (a.out_rows / 32) + blk] = (uint8_t)(e + 127);
+              if ((lane & 7) == 0)
+                *reinterpret_cast<uint32_t*>(a.next_aq + drow * (a.out_rows / 2) + (u.rt * kMxRows + 32 * q) / 2 +
+                                             (lane >> 3) * 4) = v;
+              if (lane == 0) chunk[sf_chunk_byte(i * kTerms + t, q)] = (uint8_t)(e + 127);
             }
           } else {
-            a.out_f32[(size_t)pr * a.out_rows + row] = gs;
+            a.out_f32[(size_t)pr * a.out_rows + row] = gs[i];
           }
         }
       }
@@ -680,7 +666,7 @@ __global__ void __launch_bounds__(kMxThreads, 1)
         // arrive combines the tile's rows for every token
         __threadfence();         // this thread's y stores, visible at gpu scope
         if (!epi_sync()) break;  // the four epilogue warps' y stores are done
-        if (warp == 4 && lane == 0) {
+        if (warp == 2 && lane == 0) {
           const int prev = atomicAdd(&a.tile_counter[u.rt], 1);
           const bool last = prev == n_groups - 1;
           if (last) a.tile_counter[u.rt] = 0;  // every contribution is in: ready for the next launch

@@ -292,16 +292,17 @@ MX = 0x10  # MOE_FLAG_MX_EXPERTS
 
 @pytest.mark.parametrize("B", [1, 2, 7, 33, 64])
 def test_mx_tiny_all_paths_match_oracle(torch_cuda, tiny, B):
-    """Routed experts on the tcgen05 kernels (E2M1 x E4M3 terms, E8M0 scales
-    on both operands): tiny layer, one 128-row tile per projection."""
+    """Routed experts on the tcgen05 kernels (E2M1 weights x E2M1 activation
+    terms, E8M0 scales on both operands): tiny layer, one 128-row tile per
+    projection; the down projection's K (128) is half a pipeline stage."""
     got, ref = run_all_paths(torch_cuda, tiny, B, max_batch=64, flags=MX)
     check_against_oracle(got, ref)
 
 
 @pytest.mark.parametrize("B", [1, 5, 9, 33, 64])
 def test_mx_skewed_matches_oracle(torch_cuda, skewed_small, B):
-    """Several K tiles and row tiles; B = 64 has an expert with 56 tokens
-    (three passes of 21 tokens over its weights)."""
+    """Several K stages and row tiles; B = 64 has an expert with 56 tokens
+    (four passes of up to 16 tokens over its weights)."""
     got, ref = run_all_paths(torch_cuda, skewed_small, B, max_batch=64, flags=MX)
     check_against_oracle(got, ref)
 
