@@ -409,7 +409,6 @@ __device__ __forceinline__ void group_bar(int q0, int wpi) {
 
 __device__ void publish_round(const GemvArgs& a, const int* pend_rt, int npend, int& prev_cnt, int& prev_rt,
                               int& nprev, int n_groups, int wi, int q0, int lane, int* s_pub) {
-  if (npend > 0) __threadfence();  // this thread's y stores, visible at gpu scope
   group_bar(q0, a.wpi);  // every warp of the group has written its y rows of the pending items
   if (wi == 0) {
     // results of the previous round first (their atomics completed long ago)
@@ -420,9 +419,9 @@ __device__ void publish_round(const GemvArgs& a, const int* pend_rt, int npend, 
       a.tile_counter[prev_rt] = 0;  // every contribution has arrived: ready for the next launch
     }
     if (lane == 0) s_pub[0] = __popc(m);
-    if (m) __threadfence();  // acquire: the other contributors' y stores before our loads
+    if (m) fence_acq_rel_gpu();  // acquire: the other contributors' y stores before our loads
     if (npend > 0) {
-      __threadfence();  // release: this group's y stores before its counts
+      fence_acq_rel_gpu();  // release: this group's y stores (ordered by the group barrier) before its counts
       int rt = 0;
 #pragma unroll
       for (int i = 0; i < kPubBatch; ++i)
@@ -1032,18 +1031,19 @@ __device__ __forceinline__ void gemv_body(const GemvArgs& a, unsigned char* smem
   if constexpr (kRouter) {
     if (a.topk_idx) {
       // every CTA's logits are written: the last CTA to get here selects the
-      // top-k of every token (one warp per token), then builds the buckets.
-      // Each thread makes its own logit stores visible at gpu scope first.
-      __threadfence();
-      named_bar_sync(kBarAll, nthreads_all);
-      if (tid == 0) s_flag[1] = (atomicAdd(a.done_counter, 1) == (int)gridDim.x - 1) ? 1 : 0;
+      // top-k of every token, then builds the buckets
+      named_bar_sync(kBarAll, nthreads_all);  // this CTA's logit stores, performed CTA-wide
+      if (tid == 0) {
+        fence_acq_rel_gpu();  // release: ... and at gpu scope, before the count
+        const bool last = atomicAdd(a.done_counter, 1) == (int)gridDim.x - 1;
+        if (last) fence_acq_rel_gpu();  // acquire: every CTA's logits before the reads below
+        s_flag[1] = last ? 1 : 0;
+      }
       named_bar_sync(kBarAll, nthreads_all);
       if (s_flag[1]) {
-        __threadfence();
         // the stage ring is idle now: top-k candidates, then bucket scratch
         topk_tail(a, a.out, tid, nthreads_all, kBarAll, stages + kBucketScratchBytes);
-        __threadfence();
-        named_bar_sync(kBarAll, nthreads_all);
+        named_bar_sync(kBarAll, nthreads_all);  // topk_idx stores performed CTA-wide
         unsigned long long* s_mask = reinterpret_cast<unsigned long long*>(stages);
         int* s_off = reinterpret_cast<int*>(stages + 8 * kMaxExperts);
         int* s_wsum = s_off + kMaxExperts;

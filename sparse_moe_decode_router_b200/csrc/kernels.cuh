@@ -238,16 +238,16 @@ __device__ __forceinline__ void topk_write(const GemvArgs& a, int b, uint32_t se
     }
 }
 
-// Selection keys and values of experts [lo, hi) of token b, lane l owning
-// [lo + l*PL, lo + l*PL + PL) (PL = ceil((hi - lo)/32) <= 32)
+// Selection keys and values of experts [lo, hi) of token b (hi - lo <= 32*PL),
+// lane l owning [lo + l*PL, lo + l*PL + PL)
+template <int PL>
 __device__ __forceinline__ void topk_load(const GemvArgs& a, const float* __restrict__ lg, int b, int lo, int hi,
-                                          int lane, uint32_t (&key)[32], float (&val)[32], int (&id)[32]) {
+                                          int lane, uint32_t (&key)[PL], float (&val)[PL], int (&id)[PL]) {
   const int E = a.n_experts;
-  const int PL = (hi - lo + 31) / 32;
 #pragma unroll
-  for (int i = 0; i < 32; ++i) {
+  for (int i = 0; i < PL; ++i) {
     const int e = lo + lane * PL + i;
-    const bool ok = i < PL && e < hi;
+    const bool ok = e < hi;
     float v = ok ? __ldcg(lg + (size_t)b * E + e) : 0.f;
     if (a.scoring == 1) {
       v = 1.0f / (1.0f + expf(-v));
@@ -267,85 +267,76 @@ __device__ __forceinline__ void topk_load(const GemvArgs& a, const float* __rest
 // over the selected logits, or the selected sigmoid scores normalised),
 // written in ascending expert id.
 //
-// With at least as many tokens as warps, one warp per token scans all E
-// experts.  With fewer, each token gets wpt warps: warp w selects the top-k
-// of its contiguous slice of the experts into shared memory (ids ascending
-// within and across slices), and the token's first warp selects the top-k
-// of those wpt*k candidates.  Every member of the overall top-k is in its
-// slice's top-k (at most k-1 experts of the slice precede it in the order
-// score desc, id asc), so the result is the same as one warp's scan.
-// Scratch: kTopkCandBytes of shared memory.
+// Two levels, every warp of the CTA busy: the experts are cut into slices of
+// at most 128 (4 per lane, in registers); a warp takes a (token, slice) pair
+// and writes the slice's top-k to shared memory, ids ascending within and
+// across slices; then one warp per token selects the top-k of those
+// candidates (at most 8 per lane).  Every member of the overall top-k is in
+// its slice's top-k (at most k-1 experts of the slice precede it in the
+// order score desc, id asc), so the result equals a scan of all E experts.
+// Tokens go in rounds of as many as the scratch holds.
 constexpr int kBucketScratchBytes = 8 * kMaxExperts + 4 * kMaxExperts + 4 * 64;  // s_mask, s_off, s_wsum
-constexpr int kTopkMaxCand = 256;  // candidates one merging warp takes (8 per lane)
-constexpr int kTopkCandBytes = 12 * 32 * kMaxTopK;  // at most 32 warps x k candidates
+constexpr int kTopkSlice = 128;
+constexpr int kTopkCandBytes = 48 * 1024;  // scratch: candidates (key, value, id) of one round
 
 __device__ void topk_tail(const GemvArgs& a, const float* __restrict__ lg, int tid, int nthreads, int bar,
                           unsigned char* scratch) {
   const int B = a.n_tokens, E = a.n_experts, k = a.top_k;
   const int nw = nthreads >> 5, warp = tid >> 5, lane = tid & 31;
-  int wpt = B > 0 ? nw / B : 1;
-  wpt = min(wpt, kTopkMaxCand / k);
-  if (wpt < 2) {
-    for (int b = warp; b < B; b += nw) {
-      uint32_t key[32];
-      float val[32];
-      int id[32];
-      topk_load(a, lg, b, 0, E, lane, key, val, id);
-      const uint32_t sel = warp_select_topk<32>(key, k, lane);
-      topk_write<32>(a, b, sel, val, id, lane);
-    }
-    return;
-  }
+  const int n_sl = (E + kTopkSlice - 1) / kTopkSlice;  // <= 8: at most 8*k <= 256 candidates per token
+  const int per_tok = n_sl * k;
+  const int tb = max(1, min(B, kTopkCandBytes / (12 * per_tok)));  // tokens per round
   uint32_t* ck = reinterpret_cast<uint32_t*>(scratch);
-  float* cv = reinterpret_cast<float*>(scratch + 4 * 32 * kMaxTopK);
-  int* ci = reinterpret_cast<int*>(scratch + 8 * 32 * kMaxTopK);
-  const int S = (E + wpt - 1) / wpt;  // experts per slice
-  if (warp < B * wpt) {
-    const int b = warp / wpt, w = warp - b * wpt;
-    const int lo = min(E, w * S), hi = min(E, lo + S);
-    uint32_t key[32];
-    float val[32];
-    int id[32];
-    topk_load(a, lg, b, lo, hi, lane, key, val, id);
-    const uint32_t sel = warp_select_topk<32>(key, k, lane);
-    const int ns = __popc(sel);
-    int pre = ns;
+  float* cv = reinterpret_cast<float*>(scratch + 4 * (kTopkCandBytes / 12));
+  int* ci = reinterpret_cast<int*>(scratch + 8 * (kTopkCandBytes / 12));
+  for (int b0 = 0; b0 < B; b0 += tb) {
+    const int nb = min(tb, B - b0);
+    for (int job = warp; job < nb * n_sl; job += nw) {
+      const int bl = job / n_sl, sl = job - bl * n_sl;
+      const int lo = sl * kTopkSlice, hi = min(E, lo + kTopkSlice);
+      uint32_t key[4];
+      float val[4];
+      int id[4];
+      topk_load<4>(a, lg, b0 + bl, lo, hi, lane, key, val, id);
+      const uint32_t sel = warp_select_topk<4>(key, k, lane);
+      const int ns = __popc(sel);
+      int pre = ns;
 #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int t = __shfl_up_sync(0xFFFFFFFFu, pre, o);
-      if (lane >= o) pre += t;
-    }
-    const int total = __shfl_sync(0xFFFFFFFFu, pre, 31);  // min(k, slice size)
-    pre -= ns;
-    const int base = warp * k;
-#pragma unroll
-    for (int i = 0; i < 32; ++i)
-      if ((sel >> i) & 1u) {
-        ck[base + pre] = key[i];
-        cv[base + pre] = val[i];
-        ci[base + pre] = id[i];
-        ++pre;
+      for (int o = 1; o < 32; o <<= 1) {
+        const int t = __shfl_up_sync(0xFFFFFFFFu, pre, o);
+        if (lane >= o) pre += t;
       }
-    for (int j = total + lane; j < k; j += 32) ck[base + j] = 0u;  // empty slots (key 0: no expert)
-  }
-  named_bar_sync(bar, nthreads);
-  if (warp < B * wpt && (warp % wpt) == 0) {
-    const int b = warp / wpt;
-    const int nc = wpt * k;             // <= kTopkMaxCand
-    const int PL = (nc + 31) / 32;      // <= 8
-    uint32_t key[8];
-    float val[8];
-    int id[8];
+      const int total = __shfl_sync(0xFFFFFFFFu, pre, 31);  // min(k, slice size)
+      pre -= ns;
+      const int base = job * k;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int c = lane * PL + i;
-      const bool ok = i < PL && c < nc;
-      key[i] = ok ? ck[warp * k + c] : 0u;
-      val[i] = ok ? cv[warp * k + c] : 0.f;
-      id[i] = ok ? ci[warp * k + c] : 0;
+      for (int i = 0; i < 4; ++i)
+        if ((sel >> i) & 1u) {
+          ck[base + pre] = key[i];
+          cv[base + pre] = val[i];
+          ci[base + pre] = id[i];
+          ++pre;
+        }
+      for (int j = total + lane; j < k; j += 32) ck[base + j] = 0u;  // empty slots (key 0: no expert)
     }
-    const uint32_t sel = warp_select_topk<8>(key, k, lane);
-    topk_write<8>(a, b, sel, val, id, lane);
+    named_bar_sync(bar, nthreads);
+    for (int bl = warp; bl < nb; bl += nw) {
+      const int PL = (per_tok + 31) / 32;  // <= 8
+      uint32_t key[8];
+      float val[8];
+      int id[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int c = lane * PL + i;
+        const bool ok = i < PL && c < per_tok;
+        key[i] = ok ? ck[bl * per_tok + c] : 0u;
+        val[i] = ok ? cv[bl * per_tok + c] : 0.f;
+        id[i] = ok ? ci[bl * per_tok + c] : 0;
+      }
+      const uint32_t sel = warp_select_topk<8>(key, k, lane);
+      topk_write<8>(a, b0 + bl, sel, val, id, lane);
+    }
+    named_bar_sync(bar, nthreads);  // the next round reuses the scratch
   }
 }
 

@@ -309,10 +309,10 @@ int tmax_of_slot(int t) { return t == 1 ? 2 : 1; }
 int tmax_for(int B) { return B == 1 ? 1 : 2; }  // dense streams
 
 template <typename... Args>
-cudaError_t launch_ex(void (*kern)(Args...), int grid, int block, int smem, cudaStream_t st, bool pdl,
+cudaError_t launch_ex(void (*kern)(Args...), dim3 grid, int block, int smem, cudaStream_t st, bool pdl,
                       Args... args) {
   cudaLaunchConfig_t c = {};
-  c.gridDim = dim3(grid);
+  c.gridDim = grid;
   c.blockDim = dim3(block);
   c.dynamicSmemBytes = (size_t)smem;
   c.stream = st;
@@ -552,13 +552,17 @@ MxArgs mx_args(const moe_layer* L, bool gate_up, int B, const moe_routing& r, co
 cudaError_t launch_mx_gate_up(moe_layer* L, const void* x, int B, const moe_routing& r, float* h, cudaStream_t st,
                               cudaEvent_t ev0, cudaEvent_t ev1) {
   const int H = L->cfg.hidden, k = L->cfg.top_k;
-  cudaError_t e = launch_ex(mx_x_terms_kernel<kMxTerms>, B * k, 256, 0, st, L->pdl, static_cast<const uint16_t*>(x),
+  // batch 1: every position holds the same token, whose terms are made once
+  const int by_token = B == 1 ? 1 : 0;
+  const dim3 grid(by_token ? 1 : B * k, (H / 32 + 7) / 8);
+  cudaError_t e = launch_ex(mx_x_terms_kernel<kMxTerms>, grid, 256, 0, st, L->pdl, static_cast<const uint16_t*>(x),
                             H, k, B * k, L->cfg.n_experts, mx_n_max(B) / kMxTerms,
                             static_cast<const int*>(r.pair_ids), static_cast<const int*>(r.topk_idx),
-                            static_cast<const int*>(r.offsets), L->aqx, L->bsfx, L->err);
+                            static_cast<const int*>(r.offsets), by_token, L->aqx, L->bsfx, L->err);
   if (e != cudaSuccess) return e;
   const MxPlan p = mx_plan(true, B);
-  const MxArgs a = mx_args(L, true, B, r, p, h);
+  MxArgs a = mx_args(L, true, B, r, p, h);
+  a.b_by_token = by_token;
   if (ev0 && (e = cudaEventRecord(ev0, st)) != cudaSuccess) return e;
   e = launch_ex(mx_expert_kernel<true, kMxTerms>, L->num_sms, kMxThreads, p.smem, st, L->pdl, L->tm_agu, L->tm_bx,
                 a);

@@ -94,6 +94,7 @@ struct MxArgs {
   const int* offsets;
   const int* pair_ids;
   const uint8_t* bsf;       // activation scales, chunk layout [pass-start position][K/128][512]
+  int b_by_token;           // batch 1 gate/up: every pass reads B rows 0.. and chunk 0 (the token's terms)
   int n_max;                // B columns one pass may use (multiple of 16, <= kMxNMax)
   float* out_f32;           // gate/up: h [pair][I] (may be null); down: y [pair][H]
   uint8_t* next_aq;         // gate/up: the down projection's E2M1 terms [pos*kTerms + t][I/2]
@@ -237,6 +238,12 @@ __device__ __forceinline__ float e2m1_to_f32(uint32_t c) {
   return (c & 8u) ? -mag : mag;
 }
 
+__device__ __forceinline__ float warp_amax(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
+  return v;
+}
+
 // byte of a B column's scale in its chunk: column n = r0 + 32*r1, K-block kb
 __device__ __forceinline__ int sf_chunk_byte(int n, int kb) { return 16 * (n & 31) + 4 * (n >> 5) + kb; }
 
@@ -254,57 +261,47 @@ __device__ __forceinline__ int pass_start(int q, int top_k, int n_pairs, int n_e
   return off + (q - off) / tpp * tpp;
 }
 
-// x (bf16 [B][K]) -> terms of the gate/up activations, one CTA per position
-// q of the pair list: rows q*kTerms + t of aq [.][K/2] (packed E2M1, even
-// element in the low nibble) and their scales into the chunks of q's pass.
+// x (bf16 [B][K]) -> terms of the gate/up activations: row q*kTerms + t of
+// aq [.][K/2] (packed E2M1, even element in the low nibble) and the scales
+// into the chunks of q's pass.  Grid (rows, ceil(K/256)), 8 warps: warp w of
+// CTA (q, g) takes the 32-element block 8g + w of row q, one element per lane.
+// Rows are pair positions; with by_token (batch 1) row 0 is the token itself,
+// which every position reads, and its chunk is chunk 0 (columns = terms).
 template <int kTerms>
 __global__ void __launch_bounds__(256) mx_x_terms_kernel(const uint16_t* __restrict__ x, int K, int top_k, int n_pairs,
                                                          int n_experts, int tpp, const int* __restrict__ pair_ids,
                                                          const int* __restrict__ topk_idx,
-                                                         const int* __restrict__ offsets, uint8_t* __restrict__ aq,
-                                                         uint8_t* __restrict__ bsf, int* err) {
+                                                         const int* __restrict__ offsets, int by_token,
+                                                         uint8_t* __restrict__ aq, uint8_t* __restrict__ bsf, int* err) {
   pdl_wait();
   const int q = blockIdx.x;
-  const int p0 = pass_start(q, top_k, n_pairs, n_experts, tpp, pair_ids, topk_idx, offsets);
-  if (p0 < 0) {
-    if (threadIdx.x == 0) atomicExch(err, kErrBadPlan);
-    pdl_launch_dependents();
-    return;
-  }
-  const int b = __ldcg(pair_ids + q) / top_k;
-  const int n0 = (q - p0) * kTerms;  // this position's first B column in its pass
-  const int nblk = K >> 5, KC = K / kMxKChunk;
-  for (int blk = threadIdx.x; blk < nblk; blk += blockDim.x) {
-    const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)b * K + 32 * blk);
-    float v[32];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const uint4 u = __ldcg(src + i);  // written by a preceding kernel: coherent path
-      const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        v[8 * i + 2 * j] = bf16lo_to_f32(w[j]);
-        v[8 * i + 2 * j + 1] = bf16hi_to_f32(w[j]);
-      }
+  int b = q, p0 = q;
+  if (!by_token) {
+    p0 = pass_start(q, top_k, n_pairs, n_experts, tpp, pair_ids, topk_idx, offsets);
+    if (p0 < 0) {
+      if (threadIdx.x == 0) atomicExch(err, kErrBadPlan);
+      pdl_launch_dependents();
+      return;
     }
-    uint8_t* chunk = bsf + ((size_t)p0 * KC + (blk >> 2)) * kMxChunkBytes;
+    b = __ldcg(pair_ids + q) / top_k;
+  }
+  const int n0 = (q - p0) * kTerms;  // this row's first B column in its pass
+  const int lane = threadIdx.x & 31, blk = blockIdx.y * 8 + (threadIdx.x >> 5);
+  if (blk < (K >> 5)) {
+    // written by a preceding kernel: coherent path
+    float v = __uint_as_float((uint32_t)__ldcg(x + (size_t)b * K + 32 * blk + lane) << 16);
+    uint8_t* chunk = bsf + ((size_t)p0 * (K / kMxKChunk) + (blk >> 2)) * kMxChunkBytes;
 #pragma unroll
     for (int t = 0; t < kTerms; ++t) {
-      float amax = 0.f;
+      const int e = mx_scale_exp(warp_amax(fabsf(v)));
+      const uint32_t c = f32_to_e2m1(v * pow2_exact(-e));
+      v -= e2m1_to_f32(c) * pow2_exact(e);
+      uint32_t w = c << (4 * (lane & 7));
 #pragma unroll
-      for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(v[i]));
-      const int e = mx_scale_exp(amax);
-      const float inv = pow2_exact(-e), sc = pow2_exact(e);
-      uint32_t packed[4] = {0u, 0u, 0u, 0u};
-#pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        const uint32_t c = f32_to_e2m1(v[i] * inv);
-        packed[i >> 3] |= c << (4 * (i & 7));
-        v[i] -= e2m1_to_f32(c) * sc;
-      }
-      *reinterpret_cast<uint4*>(aq + ((size_t)q * kTerms + t) * (K / 2) + 16 * blk) =
-          make_uint4(packed[0], packed[1], packed[2], packed[3]);
-      chunk[sf_chunk_byte(n0 + t, blk & 3)] = (uint8_t)(e + 127);
+      for (int o = 1; o < 8; o <<= 1) w |= __shfl_xor_sync(0xFFFFFFFFu, w, o);
+      if ((lane & 7) == 0)
+        *reinterpret_cast<uint32_t*>(aq + ((size_t)q * kTerms + t) * (K / 2) + 16 * blk + (lane >> 3) * 4) = w;
+      if (lane == 0) chunk[sf_chunk_byte(n0 + t, blk & 3)] = (uint8_t)(e + 127);
     }
   }
   pdl_launch_dependents();
@@ -379,12 +376,6 @@ struct MxWalk {
     if (++it < hi) load();
   }
 };
-
-__device__ __forceinline__ float warp_amax(float v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
-  return v;
-}
 
 template <bool kSwiglu, int kTerms>
 __global__ void __launch_bounds__(kMxThreads, 1)
@@ -472,7 +463,8 @@ __global__ void __launch_bounds__(kMxThreads, 1)
         const int arow = (int)(tile * kMxRows);
         const uint8_t* sfa_g = a.wsf + tile * KC * kMxChunkBytes;
         const uint8_t* sfa_u = a.wsf + (tile + a.up_tile) * KC * kMxChunkBytes;
-        const uint8_t* sfb = a.bsf + (size_t)u.tok * KC * kMxChunkBytes;
+        const int bpos = a.b_by_token ? 0 : u.tok;  // B rows bpos*kTerms.. and scale chunk bpos
+        const uint8_t* sfb = a.bsf + (size_t)bpos * KC * kMxChunkBytes;
         const int nbox = u.n / kMxBBox;
         for (int kt = 0; kt < KS; ++kt) {
           if (!mbar_wait_bounded(&empty_bar[s], ph ^ 1u, *s_abort ? lim_short : lim_long)) {
@@ -489,7 +481,7 @@ __global__ void __launch_bounds__(kMxThreads, 1)
           tma_load_2d(sa, &tmA, kt * 128, arow, &full_bar[s], pol);
           if (kSwiglu) tma_load_2d(sa + a.off_up, &tmA, kt * 128, arow + a.up_tile * kMxRows, &full_bar[s], pol);
           for (int j = 0; j < nbox; ++j)
-            tma_load_2d_nohint(sa + a.off_b + j * kMxBBox * 128, &tmB, kt * 128, u.tok * kTerms + kMxBBox * j,
+            tma_load_2d_nohint(sa + a.off_b + j * kMxBBox * 128, &tmB, kt * 128, bpos * kTerms + kMxBBox * j,
                                &full_bar[s]);
           const size_t ck = (size_t)2 * kt * kMxChunkBytes;
           bulk_g2s(st + a.off_sfa, sfa_g + ck, cb, &full_bar[s], pol);
@@ -664,17 +656,19 @@ __global__ void __launch_bounds__(kMxThreads, 1)
       if (!kSwiglu && a.comb_w && w.pass == w.npass - 1) {
         // the item is complete: count it for its row tile; the last expert to
         // arrive combines the tile's rows for every token
-        __threadfence();         // this thread's y stores, visible at gpu scope
-        if (!epi_sync()) break;  // the four epilogue warps' y stores are done
+        if (!epi_sync()) break;  // the four epilogue warps' y stores, performed CTA-wide
         if (warp == 2 && lane == 0) {
+          fence_acq_rel_gpu();  // release: ... and at gpu scope, before the count
           const int prev = atomicAdd(&a.tile_counter[u.rt], 1);
           const bool last = prev == n_groups - 1;
-          if (last) a.tile_counter[u.rt] = 0;  // every contribution is in: ready for the next launch
+          if (last) {
+            fence_acq_rel_gpu();  // acquire: the other experts' y rows before the combine's loads
+            a.tile_counter[u.rt] = 0;  // every contribution is in: ready for the next launch
+          }
           *s_last = last ? 1 : 0;
         }
         if (!epi_sync()) break;
         if (*s_last) {
-          __threadfence();
           const int H = a.out_rows;
           for (int bb = 0; bb < a.batch; ++bb)
             a.out_bf16[(size_t)bb * H + row] =

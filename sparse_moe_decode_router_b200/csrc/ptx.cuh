@@ -89,6 +89,14 @@ __device__ __forceinline__ void prefetch_l2(const void* src, uint32_t bytes) {
   asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
 }
 
+// ---- gpu-scope ordering around completion counters ---------------------------
+// Release: after a CTA barrier (which orders every thread's prior stores at
+// CTA scope), one thread's fence before its counter atomic makes all of them
+// visible at gpu scope first (fences are cumulative).  Acquire: the thread
+// that reads the final count fences before a CTA barrier, after which every
+// thread may read what the other CTAs published.
+__device__ __forceinline__ void fence_acq_rel_gpu() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
+
 // ---- programmatic dependent launch ------------------------------------------
 // Wait until the grids this one depends on have completed and their writes are
 // visible.  The "memory" clobber keeps the compiler from hoisting any load of
