@@ -382,6 +382,7 @@ class LayerRun:
         self.dl = make_device_layer(cfg, layer)
         c = api.moe_layer_config(cfg.hidden, cfg.n_experts, cfg.top_k, cfg.inter, cfg.shared_inter, B, flags)
         self.handle = api.moe_layer_create(c, self.dl.weights_struct())
+        self.path = api.moe_layer_expert_path(self.handle, B)   # MOE_PATH_* of the routed experts
         self.pool = pool
         self.x, self.r, self.xh, self.rh = [], [], [], []
         for p in range(pool):
@@ -483,11 +484,11 @@ def per_config_record(cfg, flags, steps, warmup, peak, sampler):
                "tokens_per_s": round(cfg.batch * steps / sec, 1),
                "counted_bytes_per_step": int(tot / steps),
                "n_active_mean": statistics.mean(run.n_active[i % run.pool] for i in range(steps)),
-               "gpu_launches_per_step": launches_per_step(cfg, flags)}
-        if cfg.batch > 8:
+               "gpu_launches_per_step": launches_per_step(cfg, run.path),
+               "expert_path": PATH_NAMES[run.path]}
+        if run.path != 0:
             fl = grouped_flops(cfg, cfg.batch * cfg.top_k)
             rec["routed_tflops"] = round(fl * steps / sec / 1e12, 2)
-            rec["expert_path"] = "grouped tensor-core kernels"
         return rec
     finally:
         run.close()
@@ -545,7 +546,8 @@ def stack_record(cfg, flags, replays, peak, sampler):
         return {"us_per_layer_step": round(per, 2), "gb_per_s": round(bpl / (per * 1e-6) / 1e9, 2),
                 "frac_of_measured_hbm": round(bpl / (per * 1e-6) / 1e9 / peak, 4),
                 "replays": replays, "replay_ms_median": round(ms, 3), "layer_steps_per_replay": nl * ns,
-                "gpu_launches_per_layer_step": launches_per_step(cfg.with_(batch=1), flags)}
+                "gpu_launches_per_layer_step": launches_per_step(cfg.with_(batch=1),
+                                                                 api.moe_layer_expert_path(handles[0], 1))}
     finally:
         for hd in handles:
             api.moe_layer_destroy(hd)
@@ -569,6 +571,7 @@ def run_ours(args, cfg):
     api.load_library()
     B, H, k = cfg.batch, cfg.hidden, cfg.top_k
     run = LayerRun(cfg, args.flags, POOL)
+    path = run.path
     try:
         uuid = str(torch.cuda.get_device_properties(local).uuid)
     except Exception:
@@ -619,8 +622,8 @@ def run_ours(args, cfg):
     ms_per_step = total_ms / K
     value = job_value(world, total_bytes, total_ms)
     achieved = gu_bytes / gu_avg_s / 1e9
-    from sparse_moe_decode_router_b200.api import MOE_FLAG_MX_EXPERTS
-    gu_tag = "routed_gate_up_tcgen05" if args.flags & MOE_FLAG_MX_EXPERTS else "routed_gate_up"
+    from sparse_moe_decode_router_b200.api import MOE_PATH_TCGEN05
+    gu_tag = "routed_gate_up_tcgen05" if path == MOE_PATH_TCGEN05 else "routed_gate_up"
     traffic = recorded_traffic(gu_tag, cfg.name)
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": K,
@@ -641,32 +644,29 @@ def run_ours(args, cfg):
         "e2e": {"value": round(world * total_bytes / (e2e_total * 1e-3) / 1e9, 2), "unit": UNIT,
                 "h2d_bytes_per_step": 2 * B * H * 2, "d2h_bytes_per_step": B * H * 2,
                 "us_per_step": round(e2e_total / K * 1e3, 2)},
-        "gpu_launches": launches_per_step(cfg, args.flags) * K,
+        "gpu_launches": launches_per_step(cfg, path) * K,
         "clocks": clocks,
     }
     line.update(extra)
     print(json.dumps(line), flush=True)
 
 
-def launches_per_step(cfg, flags):
+PATH_NAMES = {0: "CUDA-core GEMV kernels", 1: "grouped warp-MMA kernels", 2: "tcgen05 block-scaled kernels"}
+
+
+def launches_per_step(cfg, path):
     """Kernels of this library one moe_layer_forward launches: the router
     (whose last CTA selects the top-k and builds the buckets, and which also
     streams a bf16 shared expert's gate/up rows), the shared expert's down
     projection (an MXFP4 shared expert: its gate/up and down); then the routed
-    experts: on the tcgen05 kernels (MOE_FLAG_MX_EXPERTS) the activation-term
-    kernel, gate/up and down+combine; for batches above eight (grouped path
-    on, both reduction lengths multiples of 256) the warp-MMA path: an
-    activation-staging kernel and a grouped MMA kernel per projection, then
-    the combine; otherwise the streaming gate/up and down+combine."""
-    from sparse_moe_decode_router_b200.api import MOE_FLAG_MX_EXPERTS, MOE_FLAG_NO_GROUPED
+    experts on the kernels moe_layer_expert_path names (`path`): tcgen05 =
+    the activation-term kernel, gate/up and down+combine; grouped warp-MMA =
+    an activation-staging kernel and a grouped MMA kernel per projection,
+    then the combine; GEMV = the streaming gate/up and down+combine."""
     n = 1
     if cfg.shared_inter > 0:
         n += 2 if cfg.shared_format == "mxfp4" else 1
-    if flags & MOE_FLAG_MX_EXPERTS:
-        return n + 3
-    grouped = (cfg.batch > 8 and not (flags & MOE_FLAG_NO_GROUPED) and cfg.hidden % 256 == 0
-               and cfg.inter % 256 == 0)
-    return n + (5 if grouped else 2)
+    return n + {2: 3, 1: 5, 0: 2}[path]
 
 
 def _oracle_step(cfg, dl, n, threads):

@@ -81,8 +81,11 @@ typedef struct moe_layer* moe_layer_t; /* opaque, library-owned */
                                       join it before the down projection (default: it runs on
                                       the caller's stream, overlapping the top-k) */
 #define MOE_FLAG_NO_PREFETCH 0x4u   /* no L2 prefetch of the next layer's weights */
-#define MOE_FLAG_NO_GROUPED 0x8u    /* never use the tensor-core grouped expert path */
-#define MOE_FLAG_MX_EXPERTS 0x10u   /* routed experts at every batch size on the tcgen05 block-scaled
+#define MOE_FLAG_NO_GROUPED 0x8u    /* routed experts on the CUDA-core GEMV kernels at every batch
+                                      size: no tensor-core expert kernels unless
+                                      MOE_FLAG_MX_EXPERTS (see moe_layer_expert_path) */
+#define MOE_FLAG_MX_EXPERTS 0x10u   /* routed experts at every batch size, batch 1 included (by
+                                      default they run there above batch 1), on the tcgen05 block-scaled
                                       kernels (kind::mxf4: packed E2M1 weights x five E2M1 terms
                                       per activation value, E8M0 scales on both); needs hidden and
                                       inter multiples of 128, else moe_layer_create returns
@@ -98,6 +101,10 @@ typedef struct moe_layer* moe_layer_t; /* opaque, library-owned */
                                       bf16 (or no) shared expert and no side stream, else
                                       moe_layer_create returns MOE_ERR_UNSUPPORTED; takes
                                       precedence over MOE_FLAG_MX_EXPERTS at batch 1 */
+#define MOE_FLAG_WARP_MMA 0x80u      /* batches above 8 on the grouped warp-level MMA kernels
+                                      (mma.sync, f16) instead of the tcgen05 kernels, batches
+                                      2..8 on the CUDA-core GEMVs (the earlier tensor-core path,
+                                      kept for comparison) */
 #define MOE_FLAG_ROUTER_SIGMOID 0x20u /* bias-corrected sigmoid router: scores s_e = 1/(1+e^-l_e)
                                       from the raw logits, the k largest s_e + bias_e selected
                                       (equal values to the lower id), weights s_j / sum of the
@@ -177,8 +184,9 @@ MOE_API moe_status_t moe_layer_destroy(moe_layer_t layer);
 /* Router GEMV + top-k + softmax + bucketing for B tokens (the router row and
  * the top-k selection of the pages: aitest123 intro, 16 of 896 experts).
  * x: bf16 [B][H].  r: where to write the plan; NULL = the layer's own
- * buffers (see moe_layer_routing).  Two kernel launches (router GEMV, then
- * top-k / softmax / bucketing), chained with programmatic dependent launch. */
+ * buffers (see moe_layer_routing).  One kernel launch: the router GEMV, whose
+ * last CTA to finish selects the top-k, computes the weights and builds the
+ * buckets. */
 MOE_API moe_status_t moe_router_topk(moe_layer_t layer, const void* x, int B, const moe_routing* r,
                              void* stream);
 
@@ -231,6 +239,17 @@ MOE_API moe_status_t moe_layer_forward_host(moe_layer_t layer, const void* x_hos
 /* Pointers to the layer's own routing-plan buffers (device memory owned by
  * the layer, valid until destroy). */
 MOE_API moe_status_t moe_layer_routing(moe_layer_t layer, moe_routing* out);
+
+/* Which kernels a call at batch B runs the routed experts on.  By default:
+ * batch 1 on the CUDA-core GEMVs, larger batches on the tcgen05 kernels where
+ * the shapes allow them (hidden and inter multiples of 128), else above batch
+ * 8 on the grouped warp-MMA kernels, else the GEMVs; MOE_FLAG_MX_EXPERTS,
+ * MOE_FLAG_WARP_MMA and MOE_FLAG_NO_GROUPED change this as they say.  Returns one of MOE_PATH_*,
+ * or -1 for a NULL layer or B outside 1..max_batch.  Host only. */
+#define MOE_PATH_GEMV 0     /* streaming GEMVs, MXFP4 decoded in registers (CUDA cores) */
+#define MOE_PATH_GROUPED 1  /* grouped warp-level MMA kernels (mma.sync, f16) */
+#define MOE_PATH_TCGEN05 2  /* tcgen05 block-scaled MMA kernels (kind::mxf4) */
+MOE_API int moe_layer_expert_path(moe_layer_t layer, int B);
 
 /* Waits for all work on the layer's device (every stream), then reads and
  * clears the layer's device error word: MOE_OK, MOE_ERR_TIMEOUT if a bounded

@@ -26,6 +26,8 @@ MOE_FLAG_SIDE_STREAM = 0x2
 MOE_FLAG_NO_PREFETCH = 0x4
 MOE_FLAG_NO_GROUPED = 0x8
 MOE_FLAG_MX_EXPERTS = 0x10
+MOE_FLAG_WARP_MMA = 0x80
+MOE_PATH_GEMV, MOE_PATH_GROUPED, MOE_PATH_TCGEN05 = 0, 1, 2
 MOE_FLAG_ROUTER_SIGMOID = 0x20
 MOE_FLAG_PERSISTENT = 0x40
 
@@ -34,7 +36,7 @@ EXPORTS = (
     "moe_layer_create", "moe_layer_destroy", "moe_router_topk", "moe_experts_mxfp4",
     "moe_combine_residual", "moe_layer_forward", "moe_layer_forward_host", "moe_layer_routing",
     "moe_layer_last_device_error", "moe_layer_set_probe", "moe_router_topk_noalloc",
-    "moe_router_topk_noalloc_last_error", "moe_selftest",
+    "moe_router_topk_noalloc_last_error", "moe_selftest", "moe_layer_expert_path",
     "moe_status_string",
 )
 
@@ -98,6 +100,8 @@ def load_library(path: str = LIB_PATH):
         f = getattr(L, name)
         f.argtypes = args
         f.restype = st
+    L.moe_layer_expert_path.argtypes = [vp, i32]
+    L.moe_layer_expert_path.restype = ctypes.c_int
     L.moe_status_string.argtypes = [ctypes.c_int]
     L.moe_status_string.restype = ctypes.c_char_p
     _LIB = L
@@ -169,6 +173,14 @@ def moe_layer_forward(layer: int, next_layer: int | None, x, residual, out, B: i
 def moe_layer_forward_host(layer: int, x_host, residual_host, out_host, B: int, stream=None):
     _check("moe_layer_forward_host", load_library().moe_layer_forward_host(
         layer, _ptr(x_host), _ptr(residual_host), _ptr(out_host), B, _stream(stream)))
+
+
+def moe_layer_expert_path(layer: int, B: int) -> int:
+    """MOE_PATH_* of the kernels a call at batch B runs the routed experts on."""
+    p = load_library().moe_layer_expert_path(layer, B)
+    if p < 0:
+        raise ValueError(f"moe_layer_expert_path: bad layer or batch {B}")
+    return p
 
 
 def moe_layer_routing(layer: int) -> moe_routing:

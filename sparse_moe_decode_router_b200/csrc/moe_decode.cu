@@ -275,8 +275,9 @@ struct moe_layer {
   bool grouped = false;
   // tcgen05 block-scaled expert path: tensor maps over the weights and over
   // the activation-term buffers, and the buffers themselves
-  bool mx = false;      // the shapes and pointers allow it
-  bool mx_on = false;   // routed experts run on it
+  bool mx = false;         // the shapes allow it and its scale copies exist
+  bool mx_forced = false;  // MOE_FLAG_MX_EXPERTS: at every batch size
+  bool mx_default = false; // above batch 1 unless MOE_FLAG_NO_GROUPED / MOE_FLAG_WARP_MMA
   CUtensorMap tm_agu{}, tm_adn{}, tm_bx{}, tm_bh{};
   uint8_t* aqx = nullptr;   // E2M1 terms of x per pair position [MB*k*T][H/2]
   uint8_t* bsfx = nullptr;  // ... their scales, chunk layout [MB*k][H/128][512]
@@ -597,9 +598,18 @@ cudaError_t launch_mx_down(moe_layer* L, int B, const moe_routing& r, float* y, 
                    L->tm_bh, a);
 }
 
+// Kernels of a call's routed experts: the tcgen05 kernels where forced, and
+// by default above batch 1 (at batch 1 the CUDA-core GEMVs are as fast);
+// else the grouped warp-MMA kernels above kGroupedMinBatch, else the GEMVs.
+int expert_path(const moe_layer* L, int B) {
+  if (L->mx && (L->mx_forced || (B > 1 && L->mx_default))) return MOE_PATH_TCGEN05;
+  if (B > kGroupedMinBatch && L->grouped) return MOE_PATH_GROUPED;
+  return MOE_PATH_GEMV;
+}
+
 cudaError_t launch_gate_up(moe_layer* L, const void* x, int B, const moe_routing& r, cudaStream_t st,
                            cudaEvent_t ev0 = nullptr, cudaEvent_t ev1 = nullptr) {
-  if (L->mx_on) return launch_mx_gate_up(L, x, B, r, L->h, st, ev0, ev1);
+  if (expert_path(L, B) == MOE_PATH_TCGEN05) return launch_mx_gate_up(L, x, B, r, L->h, st, ev0, ev1);
   if (ev0) {
     const cudaError_t e = cudaEventRecord(ev0, st);
     if (e != cudaSuccess) return e;
@@ -625,7 +635,7 @@ GemvArgs gate_up_args(const moe_layer* L, const void* x, int B, const moe_routin
 }
 
 cudaError_t launch_gate_up_streams(moe_layer* L, const void* x, int B, const moe_routing& r, cudaStream_t st) {
-  if (B > kGroupedMinBatch && L->grouped) return launch_grouped(L, true, B, r, x, L->h, st);
+  if (expert_path(L, B) == MOE_PATH_GROUPED) return launch_grouped(L, true, B, r, x, L->h, st);
   return run_gemv(L, K_GU, B, gate_up_args(L, x, B, r), st, L->pdl);
 }
 
@@ -674,11 +684,12 @@ GemvArgs down_args(const moe_layer* L, int B, const moe_routing& r, float* y, bo
 
 cudaError_t launch_down(moe_layer* L, int B, const moe_routing& r, float* y, bool fused, const void* residual,
                         void* out, const float* ys, moe_layer* next, cudaStream_t st, bool pdl) {
-  if (L->mx_on) {
+  const int path = expert_path(L, B);
+  if (path == MOE_PATH_TCGEN05) {
     (void)pdl;
     return fused ? launch_mx_down(L, B, r, y, st, residual, out, ys, next) : launch_mx_down(L, B, r, y, st);
   }
-  if (B > kGroupedMinBatch && L->grouped) {
+  if (path == MOE_PATH_GROUPED) {
     // tensor-core projection into y, then the fixed-order combine
     cudaError_t e = launch_grouped(L, false, B, r, L->h, y, st);
     if (e == cudaSuccess && fused) e = launch_combine(L, B, r, y, ys, residual, out, st);
@@ -1070,7 +1081,8 @@ moe_status_t moe_layer_create(const moe_layer_config* cfg, const moe_layer_weigh
         if (e == cudaSuccess) e = cudaDeviceSynchronize();
       }
     }
-    L->mx_on = L->mx && (c.flags & MOE_FLAG_MX_EXPERTS);
+    L->mx_forced = (c.flags & MOE_FLAG_MX_EXPERTS) != 0;
+    L->mx_default = !(c.flags & (MOE_FLAG_NO_GROUPED | MOE_FLAG_WARP_MMA));
   }
   if (e == cudaSuccess && L->mx) {
     e = raise_smem_limit(reinterpret_cast<const void*>(mx_expert_kernel<true, kMxTerms>), kSmemBudget);
@@ -1144,6 +1156,11 @@ moe_status_t moe_layer_destroy(moe_layer_t L) {
   if (L->mx_mem) cudaFree(L->mx_mem);
   delete L;
   return MOE_OK;
+}
+
+int moe_layer_expert_path(moe_layer_t L, int B) {
+  if (!L || B < 1 || B > L->cfg.max_batch) return -1;
+  return expert_path(L, B);
 }
 
 moe_status_t moe_layer_routing(moe_layer_t L, moe_routing* out) {

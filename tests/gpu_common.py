@@ -24,6 +24,13 @@ def view_device(ptr, shape, typestr):
     return torch().as_tensor(DevPtr(ptr, shape, typestr), device="cuda")
 
 
+# MOE_FLAG_* selecting the routed-expert kernels (the default: batch 1 on the
+# CUDA-core GEMVs, larger batches on tcgen05)
+CUDA_CORES = 0x8   # MOE_FLAG_NO_GROUPED: the GEMVs at every batch size
+MX = 0x10          # MOE_FLAG_MX_EXPERTS: tcgen05 at every batch size
+WARP_MMA = 0x80    # MOE_FLAG_WARP_MMA: grouped warp-level MMA above batch 8
+
+
 def create_layer(dl, max_batch, flags=0):
     from sparse_moe_decode_router_b200 import api
     c = dl.cfg

@@ -121,9 +121,11 @@ def test_failing_nvml_falls_back(monkeypatch):
     assert c["samples"] == 0 or c["source"].startswith("nvidia-smi")
 
 
-@pytest.mark.parametrize("cfg_id,flags,want", [(1, 0, 4), (2, 0, 4), (3, 0, 7), (3, 0x8, 4), (1, 0x10, 5),
-                                                (3, 0x10, 5)])
-def test_launches_per_step(cfg_id, flags, want):
-    assert bench.launches_per_step(synth.CONFIGS[cfg_id], flags) == want
-    assert bench.launches_per_step(synth.CONFIGS[cfg_id].with_(shared_inter=0), flags) == want - 1
-    assert bench.launches_per_step(synth.CONFIGS[cfg_id].with_(shared_format="mxfp4"), flags) == want + 1
+@pytest.mark.parametrize("path,want", [(0, 4), (1, 7), (2, 5)], ids=["gemv", "warp_mma", "tcgen05"])
+def test_launches_per_step(path, want):
+    """Router + shared down + the routed experts' kernels of each path (the
+    path itself comes from moe_layer_expert_path)."""
+    for cfg_id in (1, 2, 3):
+        assert bench.launches_per_step(synth.CONFIGS[cfg_id], path) == want
+        assert bench.launches_per_step(synth.CONFIGS[cfg_id].with_(shared_inter=0), path) == want - 1
+        assert bench.launches_per_step(synth.CONFIGS[cfg_id].with_(shared_format="mxfp4"), path) == want + 1

@@ -63,7 +63,7 @@ def _check_edge_weights(dl):
     assert (ds == 0).any() and ds[ds > 0].min() <= 116 and ds.max() >= 166
 
 
-@pytest.mark.parametrize("flags", [0, 0x10], ids=["cuda_cores", "tcgen05"])
+@pytest.mark.parametrize("flags", [0x8, 0x10], ids=["cuda_cores", "tcgen05"])
 @pytest.mark.parametrize("B", [1, 2, 7])
 def test_edge_mxfp4_gemv_path_matches_oracle(torch_cuda, edge_tiny, B, flags):
     _check_edge_weights(edge_tiny)
@@ -72,11 +72,11 @@ def test_edge_mxfp4_gemv_path_matches_oracle(torch_cuda, edge_tiny, B, flags):
     check_against_oracle(got, ref)
 
 
-@pytest.mark.parametrize("flags", [0, 0x10], ids=["cuda_cores", "tcgen05"])
+@pytest.mark.parametrize("flags", [0x80, 0x10], ids=["cuda_cores_warp_mma", "tcgen05"])
 @pytest.mark.parametrize("B", [5, 9, 33])
 def test_edge_mxfp4_grouped_and_gemv_paths_match_oracle(torch_cuda, edge_medium, B, flags):
-    """Without the tcgen05 flag, B = 5 stays on the GEMV kernels and 9, 33
-    take the grouped warp-MMA kernels; with it, all run on tcgen05."""
+    """With MOE_FLAG_WARP_MMA, B = 5 stays on the GEMV kernels and 9, 33 take
+    the grouped warp-MMA kernels; with MOE_FLAG_MX_EXPERTS, all run on tcgen05."""
     _check_edge_weights(edge_medium)
     got, ref = run_all_paths(torch_cuda, edge_medium, B, max_batch=64, tiny_every=7, flags=flags)
     check_against_oracle(got, ref)

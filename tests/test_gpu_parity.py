@@ -6,7 +6,8 @@ import pytest
 
 import synth
 from helpers import W_ABS, Y_MAX_REL, Y_MEAN_REL, Y_ROUTED_MAX_REL, Y_ROUTED_MEAN_REL, bf16_close, metric_close
-from gpu_common import (assert_routing_equal, create_layer, layer_routing_host, make_device_layer,
+from gpu_common import (CUDA_CORES, MX, WARP_MMA, assert_routing_equal, create_layer, layer_routing_host,
+                        make_device_layer,
                         oracle_layer_for, residual_tokens, routing_buffers, routing_host, routing_struct,
                         to_host_u16)
 
@@ -128,19 +129,39 @@ def skewed_small(torch_cuda):
 
 @pytest.mark.parametrize("B", [9, 33, 64])
 def test_grouped_kernels_match_oracle(torch_cuda, skewed_small, B):
-    """Grouped path on every token: B=33 has an expert with 27 tokens (four
-    8-token tiles), B=64 one with 56 (two passes of 32 per item)."""
-    got, ref = run_all_paths(torch_cuda, skewed_small, B, max_batch=64)
+    """Grouped warp-MMA path on every token: B=33 has an expert with 27 tokens
+    (four 8-token tiles), B=64 one with 56 (two passes of 32 per item)."""
+    got, ref = run_all_paths(torch_cuda, skewed_small, B, max_batch=64, flags=WARP_MMA)
     check_against_oracle(got, ref)
     if B == 64:
         assert ref["counts"].max() > 32
 
 
+def test_expert_path_selection(torch_cuda, skewed_small):
+    """moe_layer_expert_path: batch 1 on the GEMVs and larger batches on
+    tcgen05 by default; each selection flag as the header states."""
+    from sparse_moe_decode_router_b200 import api
+    G, W, T = api.MOE_PATH_GEMV, api.MOE_PATH_GROUPED, api.MOE_PATH_TCGEN05
+    want = {0: {1: G, 5: T, 9: T, 64: T}, CUDA_CORES: {1: G, 5: G, 9: G, 64: G},
+            WARP_MMA: {1: G, 5: G, 9: W, 64: W}, MX: {1: T, 5: T, 9: T, 64: T}}
+    for flags, paths in want.items():
+        h = create_layer(skewed_small, 64, flags)
+        try:
+            assert {B: api.moe_layer_expert_path(h, B) for B in paths} == paths, flags
+            with pytest.raises(ValueError):
+                api.moe_layer_expert_path(h, 65)
+        finally:
+            api.moe_layer_destroy(h)
+
+
 def test_grouped_and_gemv_paths_agree_within_tolerance(torch_cuda, skewed_small):
-    """MOE_FLAG_NO_GROUPED keeps batch 64 on the GEMV kernels: both paths
-    meet the oracle (their sums run in different fixed orders)."""
-    got_g, ref = run_all_paths(torch_cuda, skewed_small, 64, max_batch=64)
-    got_v, _ = run_all_paths(torch_cuda, skewed_small, 64, max_batch=64, flags=8)
+    """MOE_FLAG_NO_GROUPED keeps batch 64 on the GEMV kernels: the GEMV,
+    warp-MMA and tcgen05 paths all meet the oracle (their sums run in
+    different fixed orders); the default at batch 64 is tcgen05."""
+    got_g, ref = run_all_paths(torch_cuda, skewed_small, 64, max_batch=64, flags=WARP_MMA)
+    got_v, _ = run_all_paths(torch_cuda, skewed_small, 64, max_batch=64, flags=CUDA_CORES)
+    got_d, _ = run_all_paths(torch_cuda, skewed_small, 64, max_batch=64)
+    check_against_oracle(got_d, ref)
     check_against_oracle(got_g, ref)
     check_against_oracle(got_v, ref)
 
@@ -217,19 +238,23 @@ def full_layers(torch_cuda):
     cache.clear()
 
 
-@pytest.mark.parametrize("cfg_id", [1, 2])
-def test_full_size_matches_oracle(torch_cuda, full_layers, cfg_id):
+@pytest.mark.parametrize("cfg_id,flags", [(1, 0), (2, 0), (2, CUDA_CORES)],
+                         ids=["b1", "b8_default", "b8_cuda_cores"])
+def test_full_size_matches_oracle(torch_cuda, full_layers, cfg_id, flags):
+    """Batch 1 (CUDA-core GEMVs by default) and batch 8 (tcgen05 by default,
+    and on the GEMVs)."""
     dl = full_layers(cfg_id)
-    got, ref = run_all_paths(torch_cuda, dl, dl.cfg.batch)
+    got, ref = run_all_paths(torch_cuda, dl, dl.cfg.batch, flags=flags)
     check_against_oracle(got, ref)
     if cfg_id == 2:
         assert 100 <= ref["n_active"] <= 128
 
 
 def test_full_size_b64_zipf(torch_cuda, full_layers):
-    """Batch 64 with the Zipf-skewed router: routing of all 64 tokens bit-exact,
-    layer outputs of a sample of tokens against the oracle run on those tokens
-    (tokens are independent of each other)."""
+    """Batch 64 with the Zipf-skewed router on the grouped warp-MMA kernels
+    (the tcgen05 kernels, the default there, have their own test below):
+    routing of all 64 tokens bit-exact, layer outputs of a sample of tokens
+    against the oracle run on those tokens (tokens are independent)."""
     from sparse_moe_decode_router_b200 import api
     import oracle
     torch = torch_cuda
@@ -241,7 +266,7 @@ def test_full_size_b64_zipf(torch_cuda, full_layers):
     r_h, r_d = residual_tokens(c, ids)
     ref_rt = oracle.routing(x_h, dl.router_w_host, dl.bias_host, k)
     assert ref_rt["n_active"] > 300 and ref_rt["counts"].max() >= 8   # skewed: hot experts
-    h = create_layer(dl, B)
+    h = create_layer(dl, B, WARP_MMA)
     try:
         out = torch.empty((B, H), dtype=torch.bfloat16, device="cuda")
         api.moe_layer_forward(h, None, x_d, r_d, out, B)
@@ -287,7 +312,6 @@ def test_full_b1_run_to_run_bit_identical(torch_cuda, full_layers):
 
 
 # ------------------------------------------- tcgen05 block-scaled path -----
-MX = 0x10  # MOE_FLAG_MX_EXPERTS
 
 
 @pytest.mark.parametrize("B", [1, 2, 7, 33, 64])
@@ -362,7 +386,7 @@ def test_mx_full_size_b64_zipf(torch_cuda, full_layers):
     assert ok, info
 
 
-@pytest.mark.parametrize("flags", [0, MX], ids=["cuda_cores", "tcgen05"])
+@pytest.mark.parametrize("flags", [CUDA_CORES, MX], ids=["cuda_cores", "tcgen05"])
 def test_full_size_verify_b8_matches_oracle(torch_cuda, full_layers, flags):
     """Speculative-decoding verify shape: 8 positions of one sequence whose
     activations share most of their direction, so they route to far fewer

@@ -14,6 +14,7 @@ pytestmark = pytest.mark.gpu
 
 SIGMOID = 0x20
 MX = 0x10
+CUDA_CORES = 0x8  # MOE_FLAG_NO_GROUPED: the GEMVs at every batch size
 
 
 @pytest.fixture(scope="module")
@@ -40,14 +41,14 @@ def shared_mx_layer(torch_cuda):
     return make_device_layer(cfg)
 
 
-@pytest.mark.parametrize("flags", [0, MX], ids=["cuda_cores", "tcgen05"])
+@pytest.mark.parametrize("flags", [CUDA_CORES, MX], ids=["cuda_cores", "tcgen05"])
 @pytest.mark.parametrize("B", [1, 5, 33])
 def test_sigmoid_router_matches_oracle(torch_cuda, sigmoid_layer, B, flags):
     got, ref = run_all_paths(torch_cuda, sigmoid_layer, B, max_batch=64, flags=SIGMOID | flags)
     check_against_oracle(got, ref)
 
 
-@pytest.mark.parametrize("flags", [0, MX], ids=["cuda_cores", "tcgen05"])
+@pytest.mark.parametrize("flags", [CUDA_CORES, MX], ids=["cuda_cores", "tcgen05"])
 @pytest.mark.parametrize("B", [1, 5, 33])
 def test_mxfp4_shared_expert_matches_oracle(torch_cuda, shared_mx_layer, B, flags):
     got, ref = run_all_paths(torch_cuda, shared_mx_layer, B, max_batch=64, flags=flags)
