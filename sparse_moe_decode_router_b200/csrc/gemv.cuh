@@ -555,6 +555,27 @@ __device__ __forceinline__ void gemv_body(const GemvArgs& a, unsigned char* smem
     asm volatile("bar.arrive 2, %0;" ::"r"(nthreads_all) : "memory");
   } else {
     if (!a.routed && !a.pdl_late) pdl_wait();
+    if (a.dep_counter && tid == 0) {
+      // the preceding kernel's outputs this stream reads are published (bounded wait)
+      const long long t0 = clock64();
+      bool ok = true;
+      while (true) {
+        int v;
+        asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(a.dep_counter) : "memory");
+        if (v >= a.dep_target) break;
+        if (clock64() - t0 > (1ll << 31)) { ok = false; break; }
+        __nanosleep(64);
+      }
+      if (!ok) {
+        atomicExch(a.err, kErrTimeout);
+        s_flag[0] = 1;
+      }
+      fence_acq_rel_gpu();
+      if (atomicAdd(a.dep_pass, 1) == (int)gridDim.x - 1) {  // every CTA of this grid is past the wait
+        *a.dep_counter = 0;
+        *a.dep_pass = 0;
+      }
+    }
     named_bar_sync(2, nthreads_all);
   }
 
@@ -1035,11 +1056,15 @@ __device__ __forceinline__ void gemv_body(const GemvArgs& a, unsigned char* smem
       named_bar_sync(kBarAll, nthreads_all);  // this CTA's logit stores, performed CTA-wide
       if (tid == 0) {
         fence_acq_rel_gpu();  // release: ... and at gpu scope, before the count
+        if (a.pub_counter) atomicAdd(a.pub_counter, 1);
         const bool last = atomicAdd(a.done_counter, 1) == (int)gridDim.x - 1;
         if (last) fence_acq_rel_gpu();  // acquire: every CTA's logits before the reads below
         s_flag[1] = last ? 1 : 0;
       }
       named_bar_sync(kBarAll, nthreads_all);
+      // the next kernel may launch now: what it may read before its own wait
+      // (h_s, behind pub_counter) is published; the routing finish follows
+      pdl_launch_dependents();
       if (s_flag[1]) {
         // the stage ring is idle now: top-k candidates, then bucket scratch
         topk_tail(a, a.out, tid, nthreads_all, kBarAll, stages + kBucketScratchBytes);

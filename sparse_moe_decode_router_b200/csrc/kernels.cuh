@@ -97,6 +97,17 @@ struct GemvArgs {
   float* out2;
   int n_items2;
   int up_off2;
+  // router kernel: every CTA adds 1 to *pub_counter once its outputs (logits,
+  // h_s) are written, then lets the next grid launch, before the routing
+  // finish.  A dense stream that reads only those outputs (the shared down
+  // projection) waits for *dep_counter to reach dep_target (the router's
+  // grid) instead of the whole router grid; the last of its CTAs to get past
+  // resets *dep_counter and *dep_pass.  It runs with pdl_late, so it still
+  // completes only after the router grid.
+  int* pub_counter;
+  int* dep_counter;
+  int dep_target;
+  int* dep_pass;
   int* err;
 };
 

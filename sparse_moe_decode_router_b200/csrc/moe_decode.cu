@@ -268,6 +268,7 @@ struct moe_layer {
   float* hs = nullptr;
   float* ys = nullptr;
   int* router_cnt = nullptr;
+  int* pub_cnt = nullptr;     // [2]: router CTAs with outputs published, shared-down CTAs past the wait
   int* tile_cnt = nullptr;
   __half* xh = nullptr;       // grouped path: f16 copy of the activations of one projection
   int* xe = nullptr;          // ... and its per-row exponents
@@ -346,10 +347,11 @@ GemvArgs base_args(const moe_layer* L, const GemvPlan& p) {
   return a;
 }
 
-cudaError_t run_gemv(moe_layer* L, Kind k, int B, const GemvArgs& a, cudaStream_t st, bool pdl) {
+cudaError_t run_gemv(moe_layer* L, Kind k, int B, const GemvArgs& a, cudaStream_t st, bool pdl, int grid = 0) {
   const int sl = slot_for(k, B);
   const GemvPlan& p = L->plans[k][sl];
-  return launch_ex(gemv_fn(k, tmax_of_slot(sl), p.fast, sl == 2), L->num_sms, p.threads, p.smem, st, pdl, a);
+  return launch_ex(gemv_fn(k, tmax_of_slot(sl), p.fast, sl == 2), grid > 0 ? grid : L->num_sms, p.threads, p.smem,
+                   st, pdl, a);
 }
 
 const GemvPlan& plan_of(const moe_layer* L, Kind k, int B) { return L->plans[k][slot_for(k, B)]; }
@@ -393,7 +395,10 @@ GemvArgs router_args(const moe_layer* L, const void* x, int B, const moe_routing
 
 cudaError_t launch_router(moe_layer* L, const void* x, int B, const moe_routing& r, cudaStream_t st,
                           bool with_shared = false) {
-  return run_gemv(L, K_ROUTER, B, router_args(L, x, B, r, with_shared), st, L->pdl);
+  GemvArgs a = router_args(L, x, B, r, with_shared);
+  // the shared down projection launched next starts on this count (see launch_shared)
+  if (with_shared && L->pdl) a.pub_counter = L->pub_cnt;
+  return run_gemv(L, K_ROUTER, B, a, st, L->pdl);
 }
 
 GemvArgs shared_down_args(const moe_layer* L, int B, float* ys) {
@@ -410,8 +415,11 @@ GemvArgs shared_down_args(const moe_layer* L, int B, float* ys) {
 
 // Shared expert: gate/up + SwiGLU, then down.  late: the gate/up kernel may
 // read x before its predecessor completes (see GemvArgs::pdl_late).
+// after_router: the down projection follows the router kernel that computed
+// h_s; it starts once every router CTA has published (pub_cnt), overlapping
+// the router's routing finish, and completes only after the router grid.
 cudaError_t launch_shared(moe_layer* L, const void* x, int B, float* ys, cudaStream_t st, bool pdl,
-                          bool late = false, bool down_only = false) {
+                          bool late = false, bool down_only = false, bool after_router = false) {
   const int H = L->cfg.hidden, Is = L->cfg.shared_inter;
   const bool mx = L->shared_mx;
   const Kind kgu = mx ? K_SGU_MX : K_SGU, kdn = mx ? K_SDN_MX : K_SDN;
@@ -429,7 +437,17 @@ cudaError_t launch_shared(moe_layer* L, const void* x, int B, float* ys, cudaStr
     if (e != cudaSuccess) return e;
   }
   (void)H;
-  return run_gemv(L, kdn, B, shared_down_args(L, B, ys), st, pdl);
+  GemvArgs d = shared_down_args(L, B, ys);
+  if (after_router && pdl && L->num_sms > 1) {
+    d.dep_counter = L->pub_cnt;
+    d.dep_target = L->num_sms;  // the router's grid
+    d.dep_pass = L->pub_cnt + 1;
+    d.pdl_late = 1;
+    // one CTA fewer than SMs: the router's last CTA keeps its SM for the
+    // routing finish, and no CTA of this stream waits for that SM to free
+    return run_gemv(L, kdn, B, d, st, pdl, L->num_sms - 1);
+  }
+  return run_gemv(L, kdn, B, d, st, pdl);
 }
 
 GemvArgs routed_args(const moe_layer* L, const GemvPlan& p, const moe_routing& r, int B) {
@@ -975,6 +993,7 @@ moe_status_t moe_layer_create(const moe_layer_config* cfg, const moe_layer_weigh
   const size_t o_hs = take((size_t)MB * std::max(Is, 1) * 4);
   const size_t o_ys = take((size_t)MB * H * 4);
   const size_t o_rc = take(4);
+  const size_t o_pc = take(8);
   const size_t o_tc = take((size_t)H * 4);  // one counter per down-projection row tile (<= H)
   const size_t o_er = take(4);
   const size_t o_gb = take(4);
@@ -1008,6 +1027,7 @@ moe_status_t moe_layer_create(const moe_layer_config* cfg, const moe_layer_weigh
   L->hs = reinterpret_cast<float*>(A + o_hs);
   L->ys = reinterpret_cast<float*>(A + o_ys);
   L->router_cnt = reinterpret_cast<int*>(A + o_rc);
+  L->pub_cnt = reinterpret_cast<int*>(A + o_pc);
   L->tile_cnt = reinterpret_cast<int*>(A + o_tc);
   L->err = reinterpret_cast<int*>(A + o_er);
   L->grid_bar = reinterpret_cast<int*>(A + o_gb);
@@ -1236,7 +1256,7 @@ moe_status_t moe_layer_forward(moe_layer_t L, moe_layer_t next, const void* x, c
   const bool fuse_sgu = has_shared && !fork && !L->shared_mx;
   if (e == cudaSuccess) e = launch_router(L, x, B, L->plan, st, fuse_sgu);
   if (e == cudaSuccess && has_shared && !fork)
-    e = launch_shared(L, x, B, L->ys, st, L->pdl, true, /*down_only*/ fuse_sgu);
+    e = launch_shared(L, x, B, L->ys, st, L->pdl, true, /*down_only*/ fuse_sgu, /*after_router*/ fuse_sgu);
   if (e == cudaSuccess) e = launch_gate_up(L, x, B, L->plan, st, L->probe_start, L->probe_stop);
   if (e == cudaSuccess && fork) e = cudaStreamWaitEvent(st, L->ev_join, 0);
   if (e == cudaSuccess)
@@ -1274,6 +1294,7 @@ moe_status_t moe_layer_last_device_error(moe_layer_t L) {
   // left behind, and finish before the caller's next launch on any stream
   cudaError_t e = cudaMemset(L->err, 0, sizeof(int));
   if (e == cudaSuccess) e = cudaMemset(L->router_cnt, 0, sizeof(int));
+  if (e == cudaSuccess) e = cudaMemset(L->pub_cnt, 0, 2 * sizeof(int));
   if (e == cudaSuccess) e = cudaMemset(L->tile_cnt, 0, sizeof(int) * L->cfg.hidden);
   if (e == cudaSuccess) e = cudaDeviceSynchronize();
   if (e != cudaSuccess) return MOE_ERR_CUDA;
