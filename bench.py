@@ -662,10 +662,15 @@ def launches_per_step(cfg, path):
     experts on the kernels moe_layer_expert_path names (`path`): tcgen05 =
     the activation-term kernel, gate/up and down+combine; grouped warp-MMA =
     an activation-staging kernel and a grouped MMA kernel per projection,
-    then the combine; GEMV = the streaming gate/up and down+combine."""
+    then the combine; GEMV = the streaming gate/up and down+combine.  Above
+    batch 1 on the tcgen05 path the router and the bf16 shared expert run on
+    the dense tensor-core kernels (the router's launch, the shared down's) and
+    the routing finish is a launch of its own."""
     n = 1
     if cfg.shared_inter > 0:
         n += 2 if cfg.shared_format == "mxfp4" else 1
+    if path == 2 and cfg.batch > 1:
+        n += 1
     return n + {2: 3, 1: 5, 0: 2}[path]
 
 

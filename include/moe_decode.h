@@ -184,18 +184,22 @@ MOE_API moe_status_t moe_layer_destroy(moe_layer_t layer);
 /* Router GEMV + top-k + softmax + bucketing for B tokens (the router row and
  * the top-k selection of the pages: aitest123 intro, 16 of 896 experts).
  * x: bf16 [B][H].  r: where to write the plan; NULL = the layer's own
- * buffers (see moe_layer_routing).  One kernel launch: the router GEMV, whose
- * last CTA to finish selects the top-k, computes the weights and builds the
- * buckets. */
+ * buffers (see moe_layer_routing).  At batch 1 one kernel launch: the
+ * router GEMV on the CUDA cores, whose last CTA to finish selects the top-k,
+ * computes the weights and builds the buckets.  Above batch 1, where the
+ * routed experts take the tcgen05 kernels (moe_layer_expert_path), two: the
+ * router on the tensor cores (the same launch and split as moe_layer_forward
+ * uses, so the same logits), then the routing finish (one CTA per token, the
+ * last one builds the buckets). */
 MOE_API moe_status_t moe_router_topk(moe_layer_t layer, const void* x, int B, const moe_routing* r,
                              void* stream);
 
 /* The selected experts and the shared expert for B tokens, given a routing
- * plan from moe_router_topk (r NULL = the layer's own plan).  Batches above 8
- * run the routed projections on the tensor cores (warp-level MMA, each
- * expert's weights decoded once for all of its tokens) unless the layer was
- * created with MOE_FLAG_NO_GROUPED; smaller ones on the streaming GEMV
- * kernels.
+ * plan from moe_router_topk (r NULL = the layer's own plan).  The routed
+ * projections run on the kernels moe_layer_expert_path names for B (by
+ * default the streaming GEMVs at batch 1, the tcgen05 kernels above it); a
+ * bf16 shared expert runs, above batch 1 on that path, on the dense
+ * tensor-core kernels with moe_layer_forward's split (the same sums).
  * y_routed: fp32 [B*k][H], row p = unweighted output of pair p's expert;
  * y_shared: fp32 [B][H] (ignored, may be NULL, when I_s = 0).
  * With MOE_FLAG_SIDE_STREAM the shared expert runs on the layer's side
@@ -283,7 +287,12 @@ MOE_API moe_status_t moe_layer_set_probe(moe_layer_t layer, void* start, void* s
  *   scoring vector: the transpose of moe_layer_weights.router_w).
  * router_bias: fp32 [n_experts] or NULL.  x: bf16 [B][hidden].
  * r: where to write the plan (all seven pointers required), as for
- *   moe_router_topk; the results equal moe_router_topk's bit for bit.
+ *   moe_router_topk; the results equal moe_router_topk's bit for bit
+ *   wherever the layer's router runs on the CUDA cores (batch 1, or a layer
+ *   created with MOE_FLAG_NO_GROUPED or MOE_FLAG_WARP_MMA).  Above batch 1 on
+ *   the default path the layer computes the logits on the tensor cores in
+ *   another summation order: the same selection and buckets, the weights
+ *   equal to fp32 rounding.
  * Limits: hidden a multiple of 32, <= 16384; n_experts even, 2..1024;
  *   1 <= top_k <= min(32, n_experts); 1 <= B <= 64; B * n_experts <= 65536.
  *   Anything beyond returns MOE_ERR_INVALID_ARG and launches nothing.

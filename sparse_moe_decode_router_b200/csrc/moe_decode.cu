@@ -18,6 +18,7 @@
 #include "kernels.cuh"
 #include "mma_grouped.cuh"
 #include "mx_umma.cuh"
+#include "dense_umma.cuh"
 #include "persistent.cuh"
 
 using namespace moe;
@@ -284,6 +285,15 @@ struct moe_layer {
   uint8_t* bsfx = nullptr;  // ... their scales, chunk layout [MB*k][H/128][512]
   uint8_t* aqh = nullptr;   // E2M1 terms of h [MB*k*T][I/2]
   uint8_t* bsfh = nullptr;  // ... their scales, chunk layout [MB*k][I/128][512]
+  // dense bf16 streams on tcgen05 above batch 1 (router + shared expert)
+  bool dense = false;
+  CUtensorMap tm_wr{}, tm_sgu{}, tm_sdn{}, tm_ht{};
+  uint16_t* hterms = nullptr;  // bf16 terms of h_s [MB * kDnHTerms][I_s]
+  float* dws1 = nullptr;       // stream-K partials of the router + shared gate/up launch
+  float* dws2 = nullptr;       // ... of the shared down launch
+  int dparts1 = 0, dparts2 = 0;
+  int* dtile_cnt = nullptr;    // [tiles of both launches]
+  char* dense_mem = nullptr;
   char* mx_mem = nullptr;   // the weight scales in chunk layout (copied at create):
   uint8_t* wsf_gu = nullptr;  // gate/up [E * 2I/128][H/128][512]
   uint8_t* wsf_dn = nullptr;  // down [E * H/128][I/128][512]
@@ -623,6 +633,115 @@ int expert_path(const moe_layer* L, int B) {
   if (L->mx && (L->mx_forced || (B > 1 && L->mx_default))) return MOE_PATH_TCGEN05;
   if (B > kGroupedMinBatch && L->grouped) return MOE_PATH_GROUPED;
   return MOE_PATH_GEMV;
+}
+
+// ---- dense bf16 streams on tcgen05 (batches above 1) ----------------------
+// Above batch 1, where the routed experts run on the tcgen05 kernels and no
+// side stream is used: the router and the bf16 shared expert's gate/up in one
+// launch, the shared down projection in a second, then the routing finish.
+bool dense_for(const moe_layer* L, int B) {
+  return L->dense && B > 1 && !L->side_stream && expert_path(L, B) == MOE_PATH_TCGEN05;
+}
+
+int dn_tiles_k1(const moe_layer* L) {
+  const int E = L->cfg.n_experts, Is = L->cfg.shared_inter;
+  return (E + kDnRows - 1) / kDnRows + ((Is > 0 && !L->shared_mx) ? Is / kDnRows : 0);
+}
+
+void dn_fill_plan(DenseArgs& a) {
+  const bool glu = a.n_streams > 1 ? (a.st[0].up_rows || a.st[1].up_rows) : a.st[0].up_rows != 0;
+  a.off_up = glu ? kDnATile : 0;
+  a.off_b = (glu ? 2 : 1) * kDnATile;
+  a.stage_bytes = (int)align_up((size_t)a.off_b + (size_t)a.n * 128, 1024);
+  a.n_stages = std::min(kDnMaxStages, (kSmemBudget - 2 * kDnHeaderBytes) / a.stage_bytes);
+}
+
+int dn_smem(const DenseArgs& a) { return 2 * kDnHeaderBytes + a.n_stages * a.stage_bytes; }
+
+// the router's tiles (stream 0), then the bf16 shared expert's gate/up tiles
+// (stream 1); skip_mask: the streams left out (the staged entry points),
+// with the same split of the rest as the fused launch, so the same sums
+enum { kDnSkipRouter = 1, kDnSkipShared = 2 };
+DenseArgs dn_args_k1(const moe_layer* L, int B, int skip_mask = 0) {
+  DenseArgs a;
+  std::memset(&a, 0, sizeof(a));
+  const int E = L->cfg.n_experts, Is = L->cfg.shared_inter;
+  a.st[0].n_tiles = (E + kDnRows - 1) / kDnRows;
+  a.st[0].out_rows = E;
+  a.st[0].out = L->logits;
+  a.st[0].bias = L->sigmoid ? nullptr : L->w.router_bias;  // sigmoid scoring: the bias steers selection only
+  a.n_streams = 1;
+  if (Is > 0 && !L->shared_mx) {
+    DenseStream& g = a.st[1];
+    g.n_tiles = Is / kDnRows;
+    g.up_rows = Is;
+    g.out_rows = Is;
+    g.out = L->hs;
+    g.next_terms = L->hterms;
+    a.n_streams = 2;
+  }
+  a.skip_mask = skip_mask & ((1 << a.n_streams) - 1);
+  a.K = L->cfg.hidden;
+  a.B = B;
+  a.terms = 1;
+  a.n = (B + 15) & ~15;
+  a.ws = L->dws1;
+  a.ws_parts = L->dparts1;
+  a.tile_cnt = L->dtile_cnt;
+  a.err = L->err;
+  dn_fill_plan(a);
+  return a;
+}
+
+DenseArgs dn_args_sdn(const moe_layer* L, int B, float* ys) {
+  DenseArgs a;
+  std::memset(&a, 0, sizeof(a));
+  const int H = L->cfg.hidden;
+  a.st[0].n_tiles = H / kDnRows;
+  a.st[0].out_rows = H;
+  a.st[0].out = ys;
+  a.n_streams = 1;
+  a.K = L->cfg.shared_inter;
+  a.B = B;
+  a.terms = kDnHTerms;
+  a.n = (B * kDnHTerms + 15) & ~15;
+  a.ws = L->dws2;
+  a.ws_parts = L->dparts2;
+  a.tile_cnt = L->dtile_cnt + dn_tiles_k1(L);
+  a.err = L->err;
+  dn_fill_plan(a);
+  return a;
+}
+
+// the most parts any tile of a launch is cut into, on a grid of G CTAs
+int dn_max_parts(const DenseArgs& a, int G) {
+  const DnSplit d = dn_split(a, G);
+  long long m = 1;
+  for (long long t = 0; t < d.T0 + d.T1; ++t) m = std::max(m, d.owner((t + 1) * d.S - 1) - d.owner(t * d.S) + 1);
+  return (int)m;
+}
+
+cudaError_t launch_dense_k1(moe_layer* L, const void* x, int B, cudaStream_t st, int skip_mask = 0) {
+  const int H = L->cfg.hidden;
+  // the activations: a tensor map over this call's x (B rows; rows past B read as zero)
+  CUtensorMap tmx;
+  if (!encode_map(&tmx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, (uint64_t)H, (uint64_t)B, (uint64_t)H * 2, kDnKBox,
+                  kDnBBox))
+    return cudaErrorInvalidValue;
+  const DenseArgs a = dn_args_k1(L, B, skip_mask);
+  return launch_ex(dense_bf16_kernel, L->num_sms, kDnThreads, dn_smem(a), st, L->pdl, L->tm_wr,
+                   a.n_streams > 1 ? L->tm_sgu : L->tm_wr, tmx, a);
+}
+
+cudaError_t launch_dense_sdn(moe_layer* L, int B, float* ys, cudaStream_t st) {
+  const DenseArgs a = dn_args_sdn(L, B, ys);
+  return launch_ex(dense_bf16_kernel, L->num_sms, kDnThreads, dn_smem(a), st, L->pdl, L->tm_sdn, L->tm_sdn,
+                   L->tm_ht, a);
+}
+
+cudaError_t launch_routing_finish(moe_layer* L, const void* x, int B, const moe_routing& r, cudaStream_t st) {
+  const GemvArgs a = router_args(L, x, B, r, false);
+  return launch_ex(routing_finish_kernel, B, 256, kBucketScratchBytes + kTopkCandBytes, st, L->pdl, a);
 }
 
 cudaError_t launch_gate_up(moe_layer* L, const void* x, int B, const moe_routing& r, cudaStream_t st,
@@ -1104,6 +1223,50 @@ moe_status_t moe_layer_create(const moe_layer_config* cfg, const moe_layer_weigh
     L->mx_forced = (c.flags & MOE_FLAG_MX_EXPERTS) != 0;
     L->mx_default = !(c.flags & (MOE_FLAG_NO_GROUPED | MOE_FLAG_WARP_MMA));
   }
+  // dense bf16 streams on tcgen05 above batch 1: tensor maps over the router
+  // copy and the bf16 shared expert, the h_s terms buffer, the stream-K
+  // workspaces (sized for the most parts any tile is cut into) and counters
+  if (e == cudaSuccess && L->mx && MB > 1 && H % kDnRows == 0 && (Is == 0 || smx || Is % kDnRows == 0)) {
+    const bool sh = Is > 0 && !smx;
+    CUtensorMap probe;  // a map of two rows with a 16-row box, as the activations of batch 2 take
+    bool ok = encode_map(&L->tm_wr, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, L->wr_t, (uint64_t)H, (uint64_t)E,
+                         (uint64_t)H * 2, kDnKBox, kDnRows) &&
+              encode_map(&probe, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, L->x_stage, (uint64_t)H, 2, (uint64_t)H * 2,
+                         kDnKBox, kDnBBox);
+    if (ok && sh)
+      ok = encode_map(&L->tm_sgu, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w->shared_gate_up, (uint64_t)H,
+                      (uint64_t)2 * Is, (uint64_t)H * 2, kDnKBox, kDnRows) &&
+           encode_map(&L->tm_sdn, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w->shared_down, (uint64_t)Is, (uint64_t)H,
+                      (uint64_t)Is * 2, kDnKBox, kDnRows);
+    if (ok) {
+      const int t1 = dn_tiles_k1(L), t2 = sh ? H / kDnRows : 0;
+      L->dparts1 = dn_max_parts(dn_args_k1(L, 2), L->num_sms);
+      L->dparts2 = sh ? dn_max_parts(dn_args_sdn(L, 2, L->ys), L->num_sms) : 1;
+      const size_t part = (size_t)2 * kDnNMax * kDnRows * sizeof(float);
+      const size_t b_ht = align_up((size_t)MB * kDnHTerms * std::max(Is, 1) * 2, 256);
+      const size_t b_w1 = (size_t)t1 * L->dparts1 * part, b_w2 = (size_t)std::max(t2, 1) * L->dparts2 * part;
+      const size_t b_tc = (size_t)(t1 + t2) * sizeof(int);
+      if (cudaMalloc(&L->dense_mem, b_ht + b_w1 + b_w2 + b_tc) != cudaSuccess) {
+        cudaGetLastError();
+        ok = false;
+      } else {
+        L->hterms = reinterpret_cast<uint16_t*>(L->dense_mem);
+        L->dws1 = reinterpret_cast<float*>(L->dense_mem + b_ht);
+        L->dws2 = reinterpret_cast<float*>(L->dense_mem + b_ht + b_w1);
+        L->dtile_cnt = reinterpret_cast<int*>(L->dense_mem + b_ht + b_w1 + b_w2);
+        e = cudaMemset(L->dense_mem, 0, b_ht + b_w1 + b_w2 + b_tc);
+        if (e == cudaSuccess && sh)
+          ok = encode_map(&L->tm_ht, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, L->hterms, (uint64_t)Is,
+                          (uint64_t)MB * kDnHTerms, (uint64_t)Is * 2, kDnKBox, kDnBBox);
+      }
+    }
+    if (e == cudaSuccess && ok) {
+      e = raise_smem_limit(reinterpret_cast<const void*>(dense_bf16_kernel), kSmemBudget);
+      if (e == cudaSuccess)
+        e = raise_smem_limit(reinterpret_cast<const void*>(routing_finish_kernel), kBucketScratchBytes + kTopkCandBytes);
+    }
+    L->dense = ok && e == cudaSuccess;
+  }
   if (e == cudaSuccess && L->mx) {
     e = raise_smem_limit(reinterpret_cast<const void*>(mx_expert_kernel<true, kMxTerms>), kSmemBudget);
     if (e == cudaSuccess)
@@ -1174,6 +1337,7 @@ moe_status_t moe_layer_destroy(moe_layer_t L) {
   if (L->side) cudaStreamDestroy(L->side);
   if (L->arena) cudaFree(L->arena);
   if (L->mx_mem) cudaFree(L->mx_mem);
+  if (L->dense_mem) cudaFree(L->dense_mem);
   delete L;
   return MOE_OK;
 }
@@ -1195,6 +1359,13 @@ moe_status_t moe_router_topk(moe_layer_t L, const void* x, int B, const moe_rout
   if (!x || !aligned16(x)) return MOE_ERR_INVALID_ARG;
   if (r && !routing_ok(r)) return MOE_ERR_INVALID_ARG;
   const moe_routing& rr = r ? *r : L->plan;
+  if (dense_for(L, B)) {
+    // the router on the dense tensor-core kernel (same split as the fused
+    // forward's router launch, so the same logits), then the routing finish
+    cudaError_t e = launch_dense_k1(L, x, B, (cudaStream_t)stream, kDnSkipShared);
+    if (e == cudaSuccess) e = launch_routing_finish(L, x, B, rr, (cudaStream_t)stream);
+    return cuda_status(e);
+  }
   return cuda_status(launch_router(L, x, B, rr, (cudaStream_t)stream));
 }
 
@@ -1218,7 +1389,15 @@ moe_status_t moe_experts_mxfp4(moe_layer_t L, const void* x, int B, const moe_ro
   }
   if (e == cudaSuccess) e = launch_gate_up(L, x, B, rr, st);
   if (e == cudaSuccess) e = launch_down(L, B, rr, y_routed, false, nullptr, nullptr, nullptr, nullptr, st, L->pdl);
-  if (e == cudaSuccess && has_shared && !fork) e = launch_shared(L, x, B, y_shared, st, L->pdl);
+  if (e == cudaSuccess && has_shared && !fork) {
+    if (dense_for(L, B) && !L->shared_mx) {
+      // the bf16 shared expert on the dense tensor-core kernels, as in moe_layer_forward
+      e = launch_dense_k1(L, x, B, st, kDnSkipRouter);
+      if (e == cudaSuccess) e = launch_dense_sdn(L, B, y_shared, st);
+    } else {
+      e = launch_shared(L, x, B, y_shared, st, L->pdl);
+    }
+  }
   if (e == cudaSuccess && fork) e = cudaStreamWaitEvent(st, L->ev_join, 0);
   return cuda_status(e);
 }
@@ -1252,6 +1431,17 @@ moe_status_t moe_layer_forward(moe_layer_t L, moe_layer_t next, const void* x, c
     if (e == cudaSuccess) e = cudaEventRecord(L->ev_join, L->side);
   }
   if (B == 1 && L->persist && !fork) return cuda_status(launch_persistent(L, next, x, residual, out, st));
+  if (dense_for(L, B)) {
+    // router + shared gate/up, shared down, routing finish, routed experts
+    if (e == cudaSuccess) e = launch_dense_k1(L, x, B, st);
+    if (e == cudaSuccess && has_shared)
+      e = L->shared_mx ? launch_shared(L, x, B, L->ys, st, L->pdl) : launch_dense_sdn(L, B, L->ys, st);
+    if (e == cudaSuccess) e = launch_routing_finish(L, x, B, L->plan, st);
+    if (e == cudaSuccess) e = launch_gate_up(L, x, B, L->plan, st, L->probe_start, L->probe_stop);
+    if (e == cudaSuccess)
+      e = launch_down(L, B, L->plan, L->y, true, residual, out, has_shared ? L->ys : nullptr, next, st, L->pdl);
+    return cuda_status(e);
+  }
   // the bf16 shared expert's gate/up rows stream inside the router kernel
   const bool fuse_sgu = has_shared && !fork && !L->shared_mx;
   if (e == cudaSuccess) e = launch_router(L, x, B, L->plan, st, fuse_sgu);

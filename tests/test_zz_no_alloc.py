@@ -5,13 +5,17 @@ reserved the GPU's memory up front, a framework that must account for every
 device byte).  Its scratch is a fixed array inside the library, shared by all
 calls, so the check runs two calls in a row with different inputs: each must
 reproduce what the allocating entry point (moe_router_topk on a layer)
-returns for the same inputs.  This file sorts last so that a run stopping at
-the first failure has already run every other test."""
+returns for the same inputs.  The layers here are created with
+MOE_FLAG_NO_GROUPED so that their router runs the same CUDA-core kernel at
+every batch size (above batch 1 the default path computes the logits on the
+tensor cores, in another summation order: the same selection, weights equal
+to fp32 rounding).  This file sorts last so that a run stopping at the first
+failure has already run every other test."""
 import numpy as np
 import pytest
 
 import synth
-from gpu_common import create_layer, make_device_layer, routing_buffers, routing_host, routing_struct
+from gpu_common import CUDA_CORES, create_layer, make_device_layer, routing_buffers, routing_host, routing_struct
 
 pytestmark = pytest.mark.gpu
 
@@ -26,7 +30,7 @@ def test_noalloc_router_matches_layer_router_twice():
     dl = make_device_layer(cfg)
     H, E, k = cfg.hidden, cfg.n_experts, cfg.top_k
     w_em = dl.router_w.t().contiguous()          # expert-major copy, made by the caller
-    h = create_layer(dl, 64)
+    h = create_layer(dl, 64, CUDA_CORES)
     try:
         for call, B in enumerate((5, 64)):
             _, x = dl.tokens(range(100 * call, 100 * call + B))
@@ -68,7 +72,7 @@ def test_noalloc_router_full_size_matches_oracle_and_layer(cfg_id, batches):
     dl = make_device_layer(cfg)
     H, E, k = cfg.hidden, cfg.n_experts, cfg.top_k
     w_em = dl.router_w.t().contiguous()
-    h = create_layer(dl, max(batches))
+    h = create_layer(dl, max(batches), CUDA_CORES)
     try:
         for B in batches:
             x_h, x = dl.tokens(range(B))
