@@ -49,6 +49,8 @@ constexpr int kDnTmemCols = 256;                  // two accumulator buffers: [g
 constexpr int kDnMaxStages = 16;
 constexpr int kDnHTerms = 2;                      // bf16 terms of h_s (B columns per token of the shared down)
 constexpr int kDnHeaderBytes = 1024;
+constexpr int kDnRedUnits = 4;                    // last part of a tile: units (4 rows x 1 token) per thread ...
+constexpr int kDnRedParts = 4;                    // ... and parts whose loads are in flight together
 static_assert(8 * (2 * kDnMaxStages + 6) + 32 <= kDnHeaderBytes, "header");
 
 struct DenseStream {
@@ -163,6 +165,13 @@ __device__ __forceinline__ void tc_mma_f16(uint32_t d, uint64_t adesc, uint64_t 
 // instruction descriptor, kind::f16: A and B bf16, K-major, fp32 accumulate, M = 128, N columns
 __host__ __device__ constexpr uint32_t dn_idesc(int n) {
   return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(kDnRows >> 4) << 24);
+}
+
+__device__ __forceinline__ void add4(float4& s, const float4& v) {
+  s.x += v.x;
+  s.y += v.y;
+  s.z += v.z;
+  s.w += v.w;
 }
 
 __device__ __forceinline__ uint16_t f32_to_bf16_bits(float f) {
@@ -346,6 +355,7 @@ __global__ void __launch_bounds__(kDnThreads, 1)
     const int q = warp & 3;
     const uint32_t lane_base = tmem + ((uint32_t)(32 * q) << 16);
     const int rloc = 32 * q + lane;  // row of the tile held by this lane
+    const int et = (warp - 2) * 32 + lane;  // 0..127 over the four epilogue warps
     int uc = 0;
     uint32_t epi_ph = 0;
     auto epi_sync = [&]() -> bool {
@@ -410,34 +420,76 @@ __global__ void __launch_bounds__(kDnThreads, 1)
       }
       if (!epi_sync()) break;
       if (*s_last) {
-        const int row = r.lt * kDnRows + rloc;  // output row of this lane
+        // the tile's parts, added in ascending K order.  A unit is four rows
+        // of one token (a float4 of each part's column); thread et takes the
+        // units et, et + 128, ... (a warp reads 512 contiguous bytes per
+        // load), kDnRedUnits units and kDnRedParts parts at a time
         const float* w0 = a.ws + ((size_t)r.tile * a.ws_parts * 2) * kDnNMax * kDnRows;
         const int np = min(r.nparts, a.ws_parts);
-        for (int bt = 0; bt < a.B; ++bt) {
-          float g = 0.f, uu = 0.f;
+        const size_t pstr = (size_t)2 * kDnNMax * kDnRows;
+        const int n_units = a.B * (kDnRows / 4);
+        const float4 zero4 = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int u0 = et; u0 < n_units; u0 += kDnRedUnits * 128) {
+          float4 g[kDnRedUnits], uu[kDnRedUnits];
+#pragma unroll
+          for (int j = 0; j < kDnRedUnits; ++j) g[j] = uu[j] = zero4;
           for (int t = 0; t < a.terms; ++t) {
-            const int col = bt * a.terms + t;
-            float sg = 0.f, su = 0.f;
-            for (int p = 0; p < np; ++p) {  // ascending K order
-              const float* pp = w0 + (size_t)p * 2 * kDnNMax * kDnRows;
-              sg += __ldcg(pp + (size_t)col * kDnRows + rloc);
-              if (glu) su += __ldcg(pp + (size_t)(kDnNMax + col) * kDnRows + rloc);
-            }
-            g += sg;
-            uu += su;
-          }
-          if (row < S.out_rows) {
-            if (glu) {
-              const float h = g / (1.0f + expf(-g)) * uu;
-              S.out[(size_t)bt * S.out_rows + row] = h;
-              if (S.next_terms) {
-                const uint16_t t0 = f32_to_bf16_bits(h);
-                const uint16_t t1 = f32_to_bf16_bits(h - __uint_as_float((uint32_t)t0 << 16));
-                S.next_terms[((size_t)bt * kDnHTerms) * S.out_rows + row] = t0;
-                S.next_terms[((size_t)bt * kDnHTerms + 1) * S.out_rows + row] = t1;
+            float4 sg[kDnRedUnits], su[kDnRedUnits];
+#pragma unroll
+            for (int j = 0; j < kDnRedUnits; ++j) sg[j] = su[j] = zero4;
+            for (int p0 = 0; p0 < np; p0 += kDnRedParts) {
+              float4 vg[kDnRedParts][kDnRedUnits], vu[kDnRedParts][kDnRedUnits];
+#pragma unroll
+              for (int i = 0; i < kDnRedParts; ++i) {
+#pragma unroll
+                for (int j = 0; j < kDnRedUnits; ++j) {
+                  const int u = u0 + 128 * j;
+                  const bool on = p0 + i < np && u < n_units;
+                  const float* src = w0 + (size_t)(p0 + i) * pstr +
+                                     (size_t)((u >> 5) * a.terms + t) * kDnRows + 4 * (u & 31);
+                  vg[i][j] = on ? __ldcg(reinterpret_cast<const float4*>(src)) : zero4;
+                  vu[i][j] = (on && glu) ? __ldcg(reinterpret_cast<const float4*>(src + kDnNMax * kDnRows)) : zero4;
+                }
               }
-            } else {
-              S.out[(size_t)bt * S.out_rows + row] = g + (S.bias ? S.bias[row] : 0.f);
+#pragma unroll
+              for (int i = 0; i < kDnRedParts; ++i) {
+                if (p0 + i >= np) break;
+#pragma unroll
+                for (int j = 0; j < kDnRedUnits; ++j) {
+                  add4(sg[j], vg[i][j]);
+                  add4(su[j], vu[i][j]);
+                }
+              }
+            }
+#pragma unroll
+            for (int j = 0; j < kDnRedUnits; ++j) {
+              add4(g[j], sg[j]);
+              add4(uu[j], su[j]);
+            }
+          }
+#pragma unroll
+          for (int j = 0; j < kDnRedUnits; ++j) {
+            const int u = u0 + 128 * j;
+            if (u >= n_units) break;
+            const int bt = u >> 5, row0 = r.lt * kDnRows + 4 * (u & 31);
+            const float gv[4] = {g[j].x, g[j].y, g[j].z, g[j].w};
+            const float uv[4] = {uu[j].x, uu[j].y, uu[j].z, uu[j].w};
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              const int row = row0 + c;
+              if (row >= S.out_rows) break;
+              if (glu) {
+                const float h = gv[c] / (1.0f + expf(-gv[c])) * uv[c];
+                S.out[(size_t)bt * S.out_rows + row] = h;
+                if (S.next_terms) {
+                  const uint16_t t0 = f32_to_bf16_bits(h);
+                  const uint16_t t1 = f32_to_bf16_bits(h - __uint_as_float((uint32_t)t0 << 16));
+                  S.next_terms[((size_t)bt * kDnHTerms) * S.out_rows + row] = t0;
+                  S.next_terms[((size_t)bt * kDnHTerms + 1) * S.out_rows + row] = t1;
+                }
+              } else {
+                S.out[(size_t)bt * S.out_rows + row] = gv[c] + (S.bias ? S.bias[row] : 0.f);
+              }
             }
           }
         }

@@ -280,7 +280,8 @@ struct moe_layer {
   bool mx = false;         // the shapes allow it and its scale copies exist
   bool mx_forced = false;  // MOE_FLAG_MX_EXPERTS: at every batch size
   bool mx_default = false; // above batch 1 unless MOE_FLAG_NO_GROUPED / MOE_FLAG_WARP_MMA
-  CUtensorMap tm_agu{}, tm_adn{}, tm_bx{}, tm_bh{};
+  CUtensorMap tm_agu{}, tm_adn{}, tm_bx{}, tm_bh{}, tm_bh8{};
+  bool swap_dn = false;     // the down projection takes the swapped-operand kernel (H a multiple of 256)
   uint8_t* aqx = nullptr;   // E2M1 terms of x per pair position [MB*k*T][H/2]
   uint8_t* bsfx = nullptr;  // ... their scales, chunk layout [MB*k][H/128][512]
   uint8_t* aqh = nullptr;   // E2M1 terms of h [MB*k*T][I/2]
@@ -566,6 +567,7 @@ MxArgs mx_args(const moe_layer* L, bool gate_up, int B, const moe_routing& r, co
   a.out_f32 = out;
   a.next_aq = gate_up ? L->aqh : nullptr;
   a.next_bsf = gate_up ? L->bsfh : nullptr;
+  a.next_rpp = L->swap_dn ? kSwRowsPerTok : kMxTerms;
   a.n_stages = p.n_stages;
   a.stage_bytes = p.stage_bytes;
   a.off_up = p.off_up;
@@ -583,7 +585,7 @@ cudaError_t launch_mx_gate_up(moe_layer* L, const void* x, int B, const moe_rout
   const int H = L->cfg.hidden, k = L->cfg.top_k;
   // batch 1: every position holds the same token, whose terms are made once
   const int by_token = B == 1 ? 1 : 0;
-  const dim3 grid(by_token ? 1 : B * k, (H / 32 + 7) / 8);
+  const dim3 grid(B, (H / 32 + 7) / 8);
   cudaError_t e = launch_ex(mx_x_terms_kernel<kMxTerms>, grid, 256, 0, st, L->pdl, static_cast<const uint16_t*>(x),
                             H, k, B * k, L->cfg.n_experts, mx_n_max(B) / kMxTerms,
                             static_cast<const int*>(r.pair_ids), static_cast<const int*>(r.topk_idx),
@@ -599,11 +601,61 @@ cudaError_t launch_mx_gate_up(moe_layer* L, const void* x, int B, const moe_rout
   return e;
 }
 
+// down projection with the operands swapped (see mx_down_swap_kernel)
+cudaError_t launch_mx_down_swap(moe_layer* L, int B, const moe_routing& r, float* y, cudaStream_t st,
+                                const void* residual, void* out, const float* ys, const moe_layer* next) {
+  const int H = L->cfg.hidden, I = L->cfg.inter, k = L->cfg.top_k;
+  SwArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.wsf = L->wsf_dn;
+  a.a_tiles = H / kMxRows;
+  a.K = I;
+  a.out_rows = H;
+  a.top_k = k;
+  a.n_pairs = B * k;
+  a.n_experts = L->cfg.n_experts;
+  a.n_active = r.n_active;
+  a.active = r.active;
+  a.offsets = r.offsets;
+  a.pair_ids = r.pair_ids;
+  a.asf = L->bsfh;
+  // gate/up passes hold all of an expert's (at most B) tokens below batch 16
+  // and 16 from there: min(B, 16) tokens per pass gives the same pass starts
+  a.tpp = std::min(B, kSwTokMax);
+  a.off_w = (int)align_up((size_t)a.tpp * kSwRowsPerTok * 128, 1024);
+  a.off_sfa = a.off_w + 2 * kMxATile;
+  a.off_sfw = a.off_sfa + 2 * kMxChunkBytes;
+  a.stage_bytes = (int)align_up((size_t)a.off_sfw + 4 * kMxChunkBytes, 1024);
+  a.n_stages = std::min(kSwMaxStages, (kSmemBudget - 2 * kMxHeaderBytes) / a.stage_bytes);
+  a.y = y;
+  if (residual) {
+    a.comb_w = r.topk_w;
+    a.y_shared = ys;
+    a.residual = static_cast<const uint16_t*>(residual);
+    a.out_bf16 = static_cast<uint16_t*>(out);
+    a.batch = B;
+    a.tile_counter = L->tile_cnt;
+    if (next && L->prefetch) {
+      a.pf_ptr[0] = reinterpret_cast<const uint8_t*>(next->wr_t);
+      a.pf_bytes[0] = (long long)next->cfg.n_experts * next->cfg.hidden * 2;
+      if (next->cfg.shared_inter > 0) {
+        a.pf_ptr[1] = reinterpret_cast<const uint8_t*>(next->w.shared_gate_up);
+        a.pf_bytes[1] = (long long)2 * next->cfg.shared_inter * next->cfg.hidden * 2;
+      }
+    }
+  }
+  a.err = L->err;
+  const int smem = 2 * kMxHeaderBytes + a.n_stages * a.stage_bytes;
+  return launch_ex(mx_down_swap_kernel<kMxTerms>, L->num_sms, kMxThreads, smem, st, L->pdl, L->tm_adn, L->tm_bh8,
+                   a);
+}
+
 // down projection on the tensor cores; with `residual` non-null fused with
 // the combine (and the next layer's L2 prefetch)
 cudaError_t launch_mx_down(moe_layer* L, int B, const moe_routing& r, float* y, cudaStream_t st,
                            const void* residual = nullptr, void* out = nullptr, const float* ys = nullptr,
                            const moe_layer* next = nullptr) {
+  if (L->swap_dn) return launch_mx_down_swap(L, B, r, y, st, residual, out, ys, next);
   const MxPlan p = mx_plan(false, B);
   MxArgs a = mx_args(L, false, B, r, p, y);
   if (residual) {
@@ -1124,7 +1176,7 @@ moe_status_t moe_layer_create(const moe_layer_config* cfg, const moe_layer_weigh
   const size_t mx_rows = (size_t)MB * k * kMxTerms;
   const size_t o_aqx = take(mx_rows * (H / 2));
   const size_t o_sfx = take((size_t)MB * k * ((H + kMxKChunk - 1) / kMxKChunk) * kMxChunkBytes);
-  const size_t o_aqh = take(mx_rows * (I / 2));
+  const size_t o_aqh = take((size_t)MB * k * kSwRowsPerTok * (I / 2));  // 8 rows per position (>= kMxTerms)
   const size_t o_sfh = take((size_t)MB * k * ((I + kMxKChunk - 1) / kMxKChunk) * kMxChunkBytes);
   if (g_fail_next_alloc.exchange(false) || cudaMalloc(&L->arena, off) != cudaSuccess) {
     cudaGetLastError();
@@ -1200,6 +1252,10 @@ moe_status_t moe_layer_create(const moe_layer_config* cfg, const moe_layer_weigh
                        kMxBBox) &&
             encode_map(&L->tm_bh, CU_TENSOR_MAP_DATA_TYPE_UINT8, L->aqh, (uint64_t)I / 2, mxr, (uint64_t)I / 2, 128,
                        kMxBBox);
+    // the swapped down projection reads h's terms 8 rows per position (box 8 rows)
+    L->swap_dn = L->mx && H % kSwN == 0 &&
+                 encode_map(&L->tm_bh8, CU_TENSOR_MAP_DATA_TYPE_UINT8, L->aqh, (uint64_t)I / 2,
+                            (uint64_t)MB * k * kSwRowsPerTok, (uint64_t)I / 2, 128, kSwRowsPerTok);
     if (L->mx) {
       // the scale arrays hold one byte per 32 weights: the chunk copies are the same size
       const size_t gu_bytes = (size_t)E * 2 * I * (H / 32), dn_bytes = (size_t)E * H * (I / 32);
@@ -1271,6 +1327,8 @@ moe_status_t moe_layer_create(const moe_layer_config* cfg, const moe_layer_weigh
     e = raise_smem_limit(reinterpret_cast<const void*>(mx_expert_kernel<true, kMxTerms>), kSmemBudget);
     if (e == cudaSuccess)
       e = raise_smem_limit(reinterpret_cast<const void*>(mx_expert_kernel<false, kMxTerms>), kSmemBudget);
+    if (e == cudaSuccess)
+      e = raise_smem_limit(reinterpret_cast<const void*>(mx_down_swap_kernel<kMxTerms>), kSmemBudget);
   }
   // persistent batch-1 kernel: needs the bf16 (or no) shared expert, no side
   // stream, and one shape-specialised or one generic instance for all streams

@@ -97,8 +97,9 @@ struct MxArgs {
   int b_by_token;           // batch 1 gate/up: every pass reads B rows 0.. and chunk 0 (the token's terms)
   int n_max;                // B columns one pass may use (multiple of 16, <= kMxNMax)
   float* out_f32;           // gate/up: h [pair][I] (may be null); down: y [pair][H]
-  uint8_t* next_aq;         // gate/up: the down projection's E2M1 terms [pos*kTerms + t][I/2]
-  uint8_t* next_bsf;        // ... and their scale chunks [pos][I/128][512]
+  uint8_t* next_aq;         // gate/up: the down projection's E2M1 terms [pos*next_rpp + t][I/2]
+  uint8_t* next_bsf;        // ... and their scale chunks [pos][I/128][512] (pass row i*next_rpp + t)
+  int next_rpp;             // rows per pair position of those terms (kTerms, or 8 for the swapped down)
   int n_stages;
   int stage_bytes;          // multiple of 1024
   int off_up, off_b, off_sfa, off_sfb;  // byte offsets inside a stage
@@ -263,45 +264,77 @@ __device__ __forceinline__ int pass_start(int q, int top_k, int n_pairs, int n_e
 
 // x (bf16 [B][K]) -> terms of the gate/up activations: row q*kTerms + t of
 // aq [.][K/2] (packed E2M1, even element in the low nibble) and the scales
-// into the chunks of q's pass.  Grid (rows, ceil(K/256)), 8 warps: warp w of
-// CTA (q, g) takes the 32-element block 8g + w of row q, one element per lane.
-// Rows are pair positions; with by_token (batch 1) row 0 is the token itself,
-// which every position reads, and its chunk is chunk 0 (columns = terms).
+// into the chunks of q's pass, for every pair position q of the token.
+// Grid (B, ceil(K/256)), 8 warps: warp w of CTA (b, g) takes the 32-element
+// block 8g + w of token b, one element per lane, makes its terms once and
+// writes them to the token's top_k positions (found by a scan of pair_ids).
+// With by_token (batch 1) row 0 is the token itself, which every position
+// reads, and its chunk is chunk 0 (columns = terms).
 template <int kTerms>
 __global__ void __launch_bounds__(256) mx_x_terms_kernel(const uint16_t* __restrict__ x, int K, int top_k, int n_pairs,
                                                          int n_experts, int tpp, const int* __restrict__ pair_ids,
                                                          const int* __restrict__ topk_idx,
                                                          const int* __restrict__ offsets, int by_token,
                                                          uint8_t* __restrict__ aq, uint8_t* __restrict__ bsf, int* err) {
+  __shared__ int s_q[kMaxTopK], s_p0[kMaxTopK];
   pdl_wait();
-  const int q = blockIdx.x;
-  int b = q, p0 = q;
-  if (!by_token) {
-    p0 = pass_start(q, top_k, n_pairs, n_experts, tpp, pair_ids, topk_idx, offsets);
-    if (p0 < 0) {
-      if (threadIdx.x == 0) atomicExch(err, kErrBadPlan);
-      pdl_launch_dependents();
-      return;
-    }
-    b = __ldcg(pair_ids + q) / top_k;
+  const int b = blockIdx.x, tid = threadIdx.x;
+  const int nq = by_token ? 1 : top_k;
+  if (nq < 1 || nq > kMaxTopK) {
+    if (tid == 0) atomicExch(err, kErrBadPlan);
+    pdl_launch_dependents();
+    return;
   }
-  const int n0 = (q - p0) * kTerms;  // this row's first B column in its pass
-  const int lane = threadIdx.x & 31, blk = blockIdx.y * 8 + (threadIdx.x >> 5);
+  if (tid < nq) s_q[tid] = by_token ? 0 : -1;
+  __syncthreads();
+  if (!by_token) {
+    // the token's pairs b*top_k + j sit at the positions q with pair_ids[q] = that pair
+    const int pb = b * top_k;
+    for (int q = tid; q < n_pairs; q += blockDim.x) {
+      const int p = __ldcg(pair_ids + q);
+      if (p >= pb && p < pb + top_k) s_q[p - pb] = q;
+    }
+    __syncthreads();
+  }
+  bool bad = false;
+  if (tid < nq) {
+    const int q = s_q[tid];
+    const int p0 = by_token ? 0 : (q < 0 ? -1 : pass_start(q, top_k, n_pairs, n_experts, tpp, pair_ids, topk_idx, offsets));
+    s_p0[tid] = p0;
+    bad = p0 < 0;
+  }
+  if (__syncthreads_or(bad)) {
+    if (tid == 0) atomicExch(err, kErrBadPlan);
+    pdl_launch_dependents();
+    return;
+  }
+  const int lane = tid & 31, blk = blockIdx.y * 8 + (tid >> 5);
   if (blk < (K >> 5)) {
     // written by a preceding kernel: coherent path
     float v = __uint_as_float((uint32_t)__ldcg(x + (size_t)b * K + 32 * blk + lane) << 16);
-    uint8_t* chunk = bsf + ((size_t)p0 * (K / kMxKChunk) + (blk >> 2)) * kMxChunkBytes;
+    uint32_t w[kTerms];
+    int ex[kTerms];
 #pragma unroll
     for (int t = 0; t < kTerms; ++t) {
       const int e = mx_scale_exp(warp_amax(fabsf(v)));
       const uint32_t c = f32_to_e2m1(v * pow2_exact(-e));
       v -= e2m1_to_f32(c) * pow2_exact(e);
-      uint32_t w = c << (4 * (lane & 7));
+      uint32_t ww = c << (4 * (lane & 7));
 #pragma unroll
-      for (int o = 1; o < 8; o <<= 1) w |= __shfl_xor_sync(0xFFFFFFFFu, w, o);
-      if ((lane & 7) == 0)
-        *reinterpret_cast<uint32_t*>(aq + ((size_t)q * kTerms + t) * (K / 2) + 16 * blk + (lane >> 3) * 4) = w;
-      if (lane == 0) chunk[sf_chunk_byte(n0 + t, blk & 3)] = (uint8_t)(e + 127);
+      for (int o = 1; o < 8; o <<= 1) ww |= __shfl_xor_sync(0xFFFFFFFFu, ww, o);
+      w[t] = ww;
+      ex[t] = e;
+    }
+    for (int j = 0; j < nq; ++j) {
+      const int q = s_q[j], p0 = s_p0[j];
+      const int n0 = (q - p0) * kTerms;  // this position's first B column in its pass
+      uint8_t* chunk = bsf + ((size_t)p0 * (K / kMxKChunk) + (blk >> 2)) * kMxChunkBytes;
+#pragma unroll
+      for (int t = 0; t < kTerms; ++t) {
+        if ((lane & 7) == 0)
+          *reinterpret_cast<uint32_t*>(aq + ((size_t)q * kTerms + t) * (K / 2) + 16 * blk + (lane >> 3) * 4) = w[t];
+        if (lane == 0) chunk[sf_chunk_byte(n0 + t, blk & 3)] = (uint8_t)(ex[t] + 127);
+      }
     }
   }
   pdl_launch_dependents();
@@ -642,11 +675,11 @@ __global__ void __launch_bounds__(kMxThreads, 1)
               uint32_t v = c << (4 * (lane & 7));
 #pragma unroll
               for (int o = 1; o < 8; o <<= 1) v |= __shfl_xor_sync(0xFFFFFFFFu, v, o);
-              const size_t drow = (size_t)pos * kTerms + t;
+              const size_t drow = (size_t)pos * a.next_rpp + t;
               if ((lane & 7) == 0)
                 *reinterpret_cast<uint32_t*>(a.next_aq + drow * (a.out_rows / 2) + (u.rt * kMxRows + 32 * q) / 2 +
                                              (lane >> 3) * 4) = v;
-              if (lane == 0) chunk[sf_chunk_byte(i * kTerms + t, q)] = (uint8_t)(e + 127);
+              if (lane == 0) chunk[sf_chunk_byte(i * a.next_rpp + t, q)] = (uint8_t)(e + 127);
             }
           } else {
             a.out_f32[(size_t)pr * a.out_rows + row] = gs[i];
@@ -679,6 +712,351 @@ __global__ void __launch_bounds__(kMxThreads, 1)
     }
   }
   // all roles done: free the tensor memory (warp 1 owns it)
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kMxTmemCols) : "memory");
+  }
+  pdl_launch_dependents();
+}
+
+// ---------------------------------------------------------------------------
+// Down projection with the operands swapped: the activation terms are the A
+// operand (M = 128 rows: row 8*i + t = token i of the pass, term t; rows
+// with t >= kTerms and beyond the pass are padding whose results are
+// dropped) and the weights the B operand (N = 256: two 128-row tiles of
+// W_down).  One MMA then covers 256 weight rows x 64 K instead of 128, and
+// a stage of 32 KB of weights takes 4 MMAs and 6 scale copies instead of 8
+// and 8: the tensor pipe issues 10 operations per 32 KB, not 16.  The
+// accumulator (128 x 256 fp32) takes half of tensor memory, so there is one
+// buffer: the MMAs of the next item wait until the epilogue has read it.
+constexpr int kSwRowsPerTok = 8;                    // A rows per token (kTerms used)
+constexpr int kSwTokMax = kMxRows / kSwRowsPerTok;  // 16 tokens per pass
+constexpr int kSwN = 256;                           // weight rows per MMA (two tiles)
+constexpr int kSwSfColsStage = 24;                  // activations 2 chunks x 4 + weights 2 chunks x 8
+constexpr int kSwMaxStages = (kMxTmemCols - kSwN) / kSwSfColsStage;  // 10
+static_assert(kMxHeaderBytes >= 8 * (2 * kSwMaxStages + 6) + 32, "header");
+
+struct SwArgs {
+  const uint8_t* wsf;       // weight scales, chunk layout [E * H/128][I/128][512]
+  int a_tiles;              // 128-row tiles per expert (H / 128)
+  int K;                    // I, multiple of 128
+  int out_rows;             // H, multiple of 256
+  int top_k, n_pairs, n_experts;
+  const int* n_active;
+  const int* active;
+  const int* offsets;
+  const int* pair_ids;
+  const uint8_t* asf;       // activation scale chunks [pass-start position][K/128][512], row m = 8*i + t
+  int tpp;                  // tokens per pass (<= kSwTokMax)
+  int n_stages, stage_bytes, off_w, off_sfa, off_sfw;  // the activation rows sit at offset 0 of a stage
+  float* y;                 // [pair][H]
+  const float* comb_w;      // fused combine as MxArgs: topk_w [B][k]
+  const float* y_shared;
+  const uint16_t* residual;
+  uint16_t* out_bf16;
+  int batch;
+  int* tile_counter;        // [H / 256], zero between launches
+  const uint8_t* pf_ptr[2];
+  long long pf_bytes[2];
+  int* err;
+};
+
+struct SwUnit { int e, rt, tok, ntok; };
+
+struct SwWalk {
+  const SwArgs& a;
+  long long it, hi;
+  int n_rt, pass, npass, e, tok0, cnt;
+  __device__ SwWalk(const SwArgs& args, long long lo, long long hi_, int nrt)
+      : a(args), it(lo), hi(hi_), n_rt(nrt), pass(0), npass(0), e(0), tok0(0), cnt(0) {
+    if (it < hi) load();
+  }
+  __device__ void load() {
+    const int g = (int)(it / n_rt);
+    e = __ldcg(a.active + g);
+    if (e < 0 || e >= a.n_experts) e = 0;
+    tok0 = __ldcg(a.offsets + e);
+    cnt = __ldcg(a.offsets + e + 1) - tok0;
+    if (tok0 < 0 || cnt < 1 || tok0 + cnt > a.n_pairs) { tok0 = 0; cnt = 1; }
+    npass = (cnt + a.tpp - 1) / a.tpp;
+    pass = 0;
+  }
+  __device__ bool valid() const { return it < hi; }
+  __device__ SwUnit unit() const {
+    SwUnit u;
+    u.e = e;
+    u.rt = (int)(it % n_rt);
+    u.tok = tok0 + pass * a.tpp;
+    u.ntok = min(a.tpp, cnt - pass * a.tpp);
+    return u;
+  }
+  __device__ void next() {
+    if (++pass < npass) return;
+    if (++it < hi) load();
+  }
+};
+
+template <int kTerms>
+__global__ void __launch_bounds__(kMxThreads, 1)
+    mx_down_swap_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmA,
+                        const SwArgs a) {
+  static_assert(kTerms >= 1 && kTerms <= kSwRowsPerTok, "terms");
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const uint32_t raw = smem_addr(smem_raw);
+  unsigned char* hdr = smem_raw;
+  unsigned char* ring = smem_raw + (((raw + kMxHeaderBytes + 1023u) & ~1023u) - raw);
+  uint64_t* full_bar = reinterpret_cast<uint64_t*>(hdr);
+  uint64_t* empty_bar = full_bar + kSwMaxStages;
+  uint64_t* acc_full = empty_bar + kSwMaxStages;
+  uint64_t* acc_empty = acc_full + 1;
+  uint64_t* done_bar = acc_empty + 1;
+  uint64_t* epi_bar = done_bar + 1;
+  volatile uint32_t* s_tmem = reinterpret_cast<volatile uint32_t*>(hdr + 8 * (2 * kSwMaxStages + 6));
+  volatile int* s_abort = reinterpret_cast<volatile int*>(hdr + 8 * (2 * kSwMaxStages + 6) + 16);
+  volatile int* s_last = s_abort + 1;
+
+  const int K = a.K, KC = K / kMxKChunk, KS = (KC + 1) / 2;
+  const int ns = a.n_stages;
+  if (tid == 0) {
+    for (int s = 0; s < kSwMaxStages; ++s) {
+      mbar_init(&full_bar[s], 1);
+      mbar_init(&empty_bar[s], 1);
+    }
+    mbar_init(acc_full, 1);
+    mbar_init(acc_empty, 4);
+    mbar_init(done_bar, 1);
+    mbar_init(epi_bar, 4);
+    *s_abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_addr((const void*)s_tmem)),
+                 "r"(kMxTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmW);
+    tma_prefetch_desc(&tmA);
+  }
+  pdl_wait();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *s_tmem;
+
+  int n_groups = __ldcg(a.n_active);
+  if (n_groups < 0 || n_groups > a.n_experts) {
+    if (tid == 0) atomicExch(a.err, kErrBadPlan);
+    n_groups = n_groups < 0 ? 0 : a.n_experts;
+  }
+  const int n_rt = a.out_rows / kSwN;
+  const long long n_items = (long long)n_groups * n_rt;
+  const long long lo = n_items * blockIdx.x / gridDim.x;
+  const long long hi = n_items * (blockIdx.x + 1) / gridDim.x;
+  const bool plan_ok = ns >= 1 && ns <= kSwMaxStages && (K % kMxKChunk) == 0 && (a.out_rows % kSwN) == 0 &&
+                       a.tpp >= 1 && a.tpp <= kSwTokMax && a.off_w >= a.tpp * kSwRowsPerTok * 128 &&
+                       a.off_w + 2 * kMxATile >= kMxRows * 128;
+  if (!plan_ok && tid == 0) atomicExch(a.err, kErrBadPlan);
+  const long long lim_long = 1ll << 31, lim_short = 1ll << 20;
+
+  if (plan_ok && warp == 0) {
+    // ------------------------------ TMA producer ------------------------------
+    if (lane == 0) {
+      const uint64_t pol = l2_policy_evict_first();
+      int s = 0;
+      uint32_t ph = 0;
+      for (SwWalk w(a, lo, hi, n_rt); w.valid() && !*s_abort; w.next()) {
+        const SwUnit u = w.unit();
+        const long long tile0 = (long long)u.e * a.a_tiles + 2 * u.rt;  // the item's two 128-row weight tiles
+        const uint8_t* sfw0 = a.wsf + tile0 * KC * kMxChunkBytes;
+        const uint8_t* sfw1 = sfw0 + (size_t)KC * kMxChunkBytes;
+        const uint8_t* sfa = a.asf + (size_t)u.tok * KC * kMxChunkBytes;
+        for (int kt = 0; kt < KS; ++kt) {
+          if (!mbar_wait_bounded(&empty_bar[s], ph ^ 1u, *s_abort ? lim_short : lim_long)) {
+            atomicExch(a.err, kErrTimeout);
+            *s_abort = 1;
+            break;
+          }
+          const int nck = min(2, KC - 2 * kt);
+          const uint32_t cb = (uint32_t)(nck * kMxChunkBytes);
+          unsigned char* st = ring + (size_t)s * a.stage_bytes;
+          const uint32_t sa = smem_addr(st);
+          mbar_arrive_expect_tx(&full_bar[s], (uint32_t)u.ntok * (kSwRowsPerTok * 128u) + 2u * kMxATile + 3u * cb);
+          for (int i = 0; i < u.ntok; ++i)
+            tma_load_2d_nohint(sa + i * kSwRowsPerTok * 128, &tmA, kt * 128, (u.tok + i) * kSwRowsPerTok, &full_bar[s]);
+          tma_load_2d(sa + a.off_w, &tmW, kt * 128, (int)(tile0 * kMxRows), &full_bar[s], pol);
+          tma_load_2d(sa + a.off_w + kMxATile, &tmW, kt * 128, (int)((tile0 + 1) * kMxRows), &full_bar[s], pol);
+          const size_t ck = (size_t)2 * kt * kMxChunkBytes;
+          bulk_g2s_nohint(st + a.off_sfa, sfa + ck, cb, &full_bar[s]);
+          bulk_g2s(st + a.off_sfw, sfw0 + ck, cb, &full_bar[s], pol);
+          bulk_g2s(st + a.off_sfw + 2 * kMxChunkBytes, sfw1 + ck, cb, &full_bar[s], pol);
+          if (++s == ns) { s = 0; ph ^= 1u; }
+        }
+      }
+      if (*s_abort) {
+        for (int q = 0; q < ns; ++q) {
+          (void)mbar_wait_bounded(&full_bar[q], 0u, lim_short);
+          (void)mbar_wait_bounded(&full_bar[q], 1u, lim_short);
+        }
+      }
+      for (int qq = 0; qq < 2; ++qq) {
+        if (!a.pf_ptr[qq] || a.pf_bytes[qq] <= 0) continue;
+        const long long per = ((a.pf_bytes[qq] / gridDim.x) + 15) & ~15ll;
+        const long long beg = per * blockIdx.x;
+        const long long end = min(beg + per, a.pf_bytes[qq]);
+        for (long long o = beg; o < end; o += 65536) {
+          const long long nb = min(end - o, 65536ll);
+          if (nb >= 16) prefetch_l2(a.pf_ptr[qq] + o, (uint32_t)(nb & ~15ll));
+        }
+      }
+    }
+  } else if (plan_ok && warp == 1) {
+    // ------------------------------ MMA issuer --------------------------------
+    if (lane == 0) {
+      int s = 0, uc = 0;
+      uint32_t ph = 0;
+      const uint32_t idesc = mx_idesc(kSwN);
+      for (SwWalk w(a, lo, hi, n_rt); w.valid() && !*s_abort; w.next(), ++uc) {
+        if (!mbar_wait_bounded(acc_empty, ((uint32_t)uc & 1u) ^ 1u, lim_long)) {
+          atomicExch(a.err, kErrTimeout);
+          *s_abort = 1;
+          break;
+        }
+        tc_fence_after();
+        bool ok = true;
+        for (int kt = 0; kt < KS && ok; ++kt) {
+          if (!mbar_wait_bounded(&full_bar[s], ph, *s_abort ? lim_short : lim_long)) {
+            atomicExch(a.err, kErrTimeout);
+            *s_abort = 1;
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const int nck = min(2, KC - 2 * kt);
+          const uint32_t st = smem_addr(ring + (size_t)s * a.stage_bytes);
+          const uint32_t sfa = tmem + (uint32_t)(kSwN + kSwSfColsStage * s), sfw = sfa + 8u;
+          for (int c = 0; c < nck; ++c) {
+            tc_cp_32x128_x4(sfa + 4u * c, desc_sf(st + a.off_sfa + c * kMxChunkBytes));
+            // weight rows 0..127 of the item -> columns 0..3 of the pair, rows 128..255 -> 4..7
+            tc_cp_32x128_x4(sfw + 8u * c, desc_sf(st + a.off_sfw + c * kMxChunkBytes));
+            tc_cp_32x128_x4(sfw + 8u * c + 4u, desc_sf(st + a.off_sfw + (2 + c) * kMxChunkBytes));
+          }
+          const uint64_t ad = desc_sw128(st), bd = desc_sw128(st + a.off_w);
+          for (int j = 0; j < 2 * nck; ++j) {
+            const uint32_t sb = 2u * (uint32_t)(j & 1), cj = (uint32_t)(j >> 1);
+            const uint32_t id = idesc | (sb << 29) | (sb << 4);
+            const uint32_t acc = (kt > 0 || j > 0) ? 1u : 0u;
+            const uint32_t tag = sb << 30;
+            tc_mma_mxf4(tmem, ad + 2u * j, bd + 2u * j, id, (sfa + 4u * cj) | tag, (sfw + 8u * cj) | tag, acc);
+          }
+          tc_commit(&empty_bar[s]);
+          if (++s == ns) { s = 0; ph ^= 1u; }
+        }
+        if (!ok) break;
+        tc_commit(acc_full);
+      }
+      tc_commit(done_bar);
+      if (!mbar_wait_bounded(done_bar, 0u, lim_long)) atomicExch(a.err, kErrTimeout);
+    }
+    __syncwarp();
+  } else if (plan_ok && warp >= 2) {
+    // ------------------------------ epilogue ----------------------------------
+    // warp w reads TMEM lanes 32*(w%4).. = tokens 4*(w%4) .. +3 of the pass,
+    // 8 lanes (terms) each; the terms are summed across those lanes
+    const int q = warp & 3;
+    const uint32_t lane_base = tmem + ((uint32_t)(32 * q) << 16);
+    const int tq = 4 * q + (lane >> 3), t = lane & 7;  // token of the pass, term
+    int uc = 0;
+    uint32_t epi_ph = 0;
+    auto epi_sync = [&]() -> bool {
+      __syncwarp();
+      if (lane == 0) mbar_arrive(epi_bar);
+      bool ok = mbar_wait_bounded(epi_bar, epi_ph, *s_abort ? lim_short : lim_long);
+      ok = __all_sync(0xFFFFFFFFu, ok);
+      epi_ph ^= 1u;
+      if (!ok) {
+        if (lane == 0) atomicExch(a.err, kErrTimeout);
+        *s_abort = 1;
+      }
+      return ok;
+    };
+    const int et = (warp - 2) * 32 + lane;  // 0..127 over the four epilogue warps
+    for (SwWalk w(a, lo, hi, n_rt); w.valid(); w.next(), ++uc) {
+      const SwUnit u = w.unit();
+      bool ok = !*s_abort && mbar_wait_bounded(acc_full, (uint32_t)uc & 1u, lim_long);
+      ok = __all_sync(0xFFFFFFFFu, ok);
+      if (!ok) {
+        if (lane == 0 && !*s_abort) atomicExch(a.err, kErrTimeout);
+        *s_abort = 1;
+        break;
+      }
+      tc_fence_after();
+      const int row0 = u.rt * kSwN;
+      int pr = 0;
+      const bool mine = tq < u.ntok;  // this lane's token is in the pass
+      if (mine) {
+        pr = __ldcg(a.pair_ids + u.tok + tq);
+        if (pr < 0 || pr >= a.n_pairs) pr = 0;
+      }
+      if (4 * q < u.ntok) {  // warp-uniform: the quadrant holds tokens of the pass
+        float v[16];
+        tc_ld16(lane_base, v);
+#pragma unroll 1
+        for (int c = 0; c < kSwN / 16; ++c) {
+          tc_wait_ld();
+          float cur[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) cur[i] = t < kTerms ? v[i] : 0.f;
+          if (c + 1 < kSwN / 16) tc_ld16(lane_base + (uint32_t)(16 * (c + 1)), v);
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            // the terms of a token: a fixed pairwise tree over its 8 lanes
+            cur[i] += __shfl_xor_sync(0xFFFFFFFFu, cur[i], 1);
+            cur[i] += __shfl_xor_sync(0xFFFFFFFFu, cur[i], 2);
+            cur[i] += __shfl_xor_sync(0xFFFFFFFFu, cur[i], 4);
+          }
+          if (mine && t == 0) {
+            float4* dst = reinterpret_cast<float4*>(a.y + (size_t)pr * a.out_rows + row0 + 16 * c);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) dst[i] = make_float4(cur[4 * i], cur[4 * i + 1], cur[4 * i + 2], cur[4 * i + 3]);
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(acc_empty);
+      if (a.comb_w && w.pass == w.npass - 1) {
+        if (!epi_sync()) break;  // the four epilogue warps' y stores, performed CTA-wide
+        if (warp == 2 && lane == 0) {
+          fence_acq_rel_gpu();
+          const int prev = atomicAdd(&a.tile_counter[u.rt], 1);
+          const bool last = prev == n_groups - 1;
+          if (last) {
+            fence_acq_rel_gpu();
+            a.tile_counter[u.rt] = 0;
+          }
+          *s_last = last ? 1 : 0;
+        }
+        if (!epi_sync()) break;
+        if (*s_last) {
+          const int H = a.out_rows;
+          for (int bb = 0; bb < a.batch; ++bb) {
+            a.out_bf16[(size_t)bb * H + row0 + et] =
+                combine_elem(a.residual, a.y_shared, a.comb_w, a.top_k, a.y, H, bb, row0 + et);
+            a.out_bf16[(size_t)bb * H + row0 + 128 + et] =
+                combine_elem(a.residual, a.y_shared, a.comb_w, a.top_k, a.y, H, bb, row0 + 128 + et);
+          }
+        }
+        if (!epi_sync()) break;
+      }
+    }
+  }
   __syncwarp();
   tc_fence_before();
   __syncthreads();
