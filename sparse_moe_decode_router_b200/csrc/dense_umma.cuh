@@ -167,13 +167,6 @@ __host__ __device__ constexpr uint32_t dn_idesc(int n) {
   return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(kDnRows >> 4) << 24);
 }
 
-__device__ __forceinline__ void add4(float4& s, const float4& v) {
-  s.x += v.x;
-  s.y += v.y;
-  s.z += v.z;
-  s.w += v.w;
-}
-
 __device__ __forceinline__ uint16_t f32_to_bf16_bits(float f) {
   uint16_t h;
   asm("cvt.rn.bf16.f32 %0, %1;" : "=h"(h) : "f"(f));
@@ -509,7 +502,7 @@ __global__ void __launch_bounds__(kDnThreads, 1)
 }
 
 // Routing finish of batches above 1, after a router stream without one:
-// CTA b selects token b's top-k (per-slice tops, then the merge), the last
+// CTA b selects token b's top-k (topk_token_block), the last
 // CTA to finish builds the buckets.  Dynamic shared memory: kBucketScratchBytes
 // + kTopkCandBytes.
 __global__ void __launch_bounds__(256) routing_finish_kernel(const GemvArgs a) {
@@ -517,12 +510,8 @@ __global__ void __launch_bounds__(256) routing_finish_kernel(const GemvArgs a) {
   __shared__ int s_last;
   pdl_wait();
   const int tid = threadIdx.x, b = blockIdx.x;
-  const int E = a.n_experts, k = a.top_k;
-  GemvArgs t = a;
-  t.n_tokens = 1;
-  t.topk_idx = a.topk_idx + (size_t)b * k;
-  t.topk_w = a.topk_w + (size_t)b * k;
-  topk_tail(t, a.out + (size_t)b * E, tid, blockDim.x, 1, smem + kBucketScratchBytes);
+  const int E = a.n_experts;
+  topk_token_block(a, a.out + (size_t)b * E, b, tid, blockDim.x, 1, false, smem + kBucketScratchBytes);
   __syncthreads();  // this CTA's topk stores, performed CTA-wide
   if (tid == 0) {
     fence_acq_rel_gpu();

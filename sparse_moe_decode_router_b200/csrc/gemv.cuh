@@ -1066,13 +1066,18 @@ __device__ __forceinline__ void gemv_body(const GemvArgs& a, unsigned char* smem
       // (h_s, behind pub_counter) is published; the routing finish follows
       pdl_launch_dependents();
       if (s_flag[1]) {
-        // the stage ring is idle now: top-k candidates, then bucket scratch
-        topk_tail(a, a.out, tid, nthreads_all, kBarAll, stages + kBucketScratchBytes);
-        named_bar_sync(kBarAll, nthreads_all);  // topk_idx stores performed CTA-wide
-        unsigned long long* s_mask = reinterpret_cast<unsigned long long*>(stages);
-        int* s_off = reinterpret_cast<int*>(stages + 8 * kMaxExperts);
-        int* s_wsum = s_off + kMaxExperts;
-        bucket_block(a, a.n_tokens, tid, nthreads_all, kBarAll, s_mask, s_off, s_wsum);
+        // the stage ring is idle now: top-k scratch, then bucket scratch
+        if (a.n_tokens == 1) {
+          // one token: the whole CTA selects it and writes the plan as it goes
+          topk_token_block(a, a.out, 0, tid, nthreads_all, kBarAll, true, stages);
+        } else {
+          topk_tail(a, a.out, tid, nthreads_all, kBarAll, stages + kBucketScratchBytes);
+          named_bar_sync(kBarAll, nthreads_all);  // topk_idx stores performed CTA-wide
+          unsigned long long* s_mask = reinterpret_cast<unsigned long long*>(stages);
+          int* s_off = reinterpret_cast<int*>(stages + 8 * kMaxExperts);
+          int* s_wsum = s_off + kMaxExperts;
+          bucket_block(a, a.n_tokens, tid, nthreads_all, kBarAll, s_mask, s_off, s_wsum);
+        }
         if (tid == 0) *a.done_counter = 0;
       }
     }

@@ -207,14 +207,33 @@ __device__ __forceinline__ uint32_t warp_select_topk(const uint32_t (&key)[PL], 
   return sel;
 }
 
-// Weights of token b's selection and its output, ascending expert id: the
-// warp holds PL candidates per lane (ids ascending with lane*PL + slot),
-// `sel` marks the selected slots, val their logits (softmax) or sigmoid
-// scores (bias-corrected sigmoid: normalised over the selection).
-template <int PL>
-__device__ __forceinline__ void topk_write(const GemvArgs& a, int b, uint32_t sel, float (&val)[PL],
-                                           const int (&id)[PL], int lane) {
+// Weights of token b's selection and its output, ascending expert id, in one
+// fixed order: lane j < k of the warp holds the j-th selected expert (id and
+// logit, or sigmoid score); the softmax max and the normaliser are warp
+// reductions over the lanes in position order (every top-k path uses this,
+// so they give the same bits).
+__device__ __forceinline__ void topk_emit(const GemvArgs& a, int b, float v, int id, int lane) {
   const int k = a.top_k;
+  const bool on = lane < k;
+  float m = on ? v : -INFINITY;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+  const float e = on ? (a.scoring == 1 ? v : expf(v - m)) : 0.f;
+  float z = e;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xFFFFFFFFu, z, o);
+  if (on) {
+    a.topk_idx[b * k + lane] = id;
+    a.topk_w[b * k + lane] = e / z;
+  }
+}
+
+// The warp-selected candidates (PL per lane, ids ascending with lane*PL +
+// slot; `sel` marks the selection) in position order through `scratch`
+// (k floats + k ints of this warp), then topk_emit.
+template <int PL>
+__device__ __forceinline__ void topk_write(const GemvArgs& a, int b, uint32_t sel, const float (&val)[PL],
+                                           const int (&id)[PL], int lane, float* sv, int* si) {
   const int ns = __popc(sel);
   int pre = ns;
 #pragma unroll
@@ -223,30 +242,18 @@ __device__ __forceinline__ void topk_write(const GemvArgs& a, int b, uint32_t se
     if (lane >= o) pre += t;
   }
   pre -= ns;
-  float lmax = -INFINITY;
-#pragma unroll
-  for (int i = 0; i < PL; ++i)
-    if ((sel >> i) & 1u) lmax = fmaxf(lmax, val[i]);
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) lmax = fmaxf(lmax, __shfl_xor_sync(0xFFFFFFFFu, lmax, o));
-  float z = 0.f;
-#pragma unroll
-  for (int i = 0; i < PL; ++i) {
-    if ((sel >> i) & 1u) {
-      val[i] = a.scoring == 1 ? val[i] : expf(val[i] - lmax);
-      z += val[i];
-    }
-  }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xFFFFFFFFu, z, o);
+  __syncwarp();
   int pos = pre;
 #pragma unroll
   for (int i = 0; i < PL; ++i)
     if ((sel >> i) & 1u) {
-      a.topk_idx[b * k + pos] = id[i];
-      a.topk_w[b * k + pos] = val[i] / z;
+      sv[pos] = val[i];
+      si[pos] = id[i];
       ++pos;
     }
+  __syncwarp();
+  const bool on = lane < a.top_k;
+  topk_emit(a, b, on ? sv[lane] : 0.f, on ? si[lane] : 0, lane);
 }
 
 // Selection keys and values of experts [lo, hi) of token b (hi - lo <= 32*PL),
@@ -345,7 +352,8 @@ __device__ void topk_tail(const GemvArgs& a, const float* __restrict__ lg, int t
         id[i] = ok ? ci[bl * per_tok + c] : 0;
       }
       const uint32_t sel = warp_select_topk<8>(key, k, lane);
-      topk_write<8>(a, b0 + bl, sel, val, id, lane);
+      // this token's candidate slots are free once the warp has them in registers
+      topk_write<8>(a, b0 + bl, sel, val, id, lane, cv + bl * per_tok, ci + bl * per_tok);
     }
     named_bar_sync(bar, nthreads);  // the next round reuses the scratch
   }
@@ -414,6 +422,173 @@ __device__ void bucket_block(const GemvArgs& a, int B, int tid, int nt, int bar,
     const unsigned long long below = (bb == 0) ? 0ull : (s_mask[e] & ((1ull << bb) - 1ull));
     a.pair_ids_out[s_off[e] + __popcll(below)] = p;
   }
+}
+
+// Top-k of one token with a whole block (nt threads: 2 to 32 warps).  The
+// order is (key descending, id ascending): the pages' tie rule as the rest of
+// the library applies it.  Warp w takes the ids [w*S, (w+1)*S), S = E / nw
+// rounded up, PL of them per lane (id = lo + lane + 32*i); each lane sorts
+// its own in registers, then the warp takes its k best by k rounds of "the
+// best lane head wins and pops" (one max-reduction and one ballot per round;
+// a second reduction only when keys tie).  Warp 0 merges the nw sorted lists
+// the same way, orders the k winners by id and writes them through
+// topk_emit.  With bucket_b1 (a batch of one token) the routing plan is
+// written here too: the active list is the selection, offsets count the
+// selected ids below each expert, the pairs are in order.
+constexpr int kTopkBlockScratch = 12 * 32 * kMaxTopK + 8 * 2 * kMaxTopK + 64;
+
+struct TopkHead {
+  uint32_t hi, lo;  // key (0: none) and ~id
+  float v;
+};
+
+__device__ __forceinline__ bool topk_before(const TopkHead& a, const TopkHead& b) {
+  return a.hi > b.hi || (a.hi == b.hi && a.lo > b.lo);
+}
+
+// the lane whose head is first in the order among all lanes (-1: every head empty)
+__device__ __forceinline__ int topk_round_winner(const TopkHead& h) {
+  const uint32_t m = __reduce_max_sync(0xFFFFFFFFu, h.hi);
+  if (m == 0u) return -1;
+  unsigned bal = __ballot_sync(0xFFFFFFFFu, h.hi == m);
+  if (__popc(bal) > 1) {
+    const uint32_t ml = __reduce_max_sync(0xFFFFFFFFu, h.hi == m ? h.lo : 0u);
+    bal = __ballot_sync(0xFFFFFFFFu, h.hi == m && h.lo == ml);
+  }
+  return __ffs(bal) - 1;
+}
+
+template <int PLM>
+__device__ void topk_token_block_pl(const GemvArgs& a, const float* __restrict__ lg, int b, int tid, int nt, int bar,
+                                    bool bucket_b1, unsigned char* scratch) {
+  const int E = a.n_experts, k = a.top_k;
+  const int lane = tid & 31, warp = tid >> 5, nw = nt >> 5;
+  const int S = (E + nw - 1) / nw, lo = warp * S, hi = min(E, lo + S);
+  uint32_t* c_hi = reinterpret_cast<uint32_t*>(scratch);  // [nw][k] each warp's list, in order
+  uint32_t* c_lo = c_hi + 32 * kMaxTopK;
+  float* c_v = reinterpret_cast<float*>(c_lo + 32 * kMaxTopK);
+  int* s_id = reinterpret_cast<int*>(c_v + 32 * kMaxTopK);  // the selection, ascending id
+  float* s_v = reinterpret_cast<float*>(s_id + kMaxTopK);
+  TopkHead h[PLM];
+#pragma unroll
+  for (int i = 0; i < PLM; ++i) {
+    const int e = lo + lane + 32 * i;
+    const bool ok = e < hi;
+    float v = ok ? __ldcg(lg + e) : 0.f;
+    uint32_t key;
+    if (a.scoring == 1) {
+      v = 1.0f / (1.0f + expf(-v));
+      key = ok ? logit_key(v + (a.sel_bias ? __ldg(a.sel_bias + e) : 0.f)) : 0u;
+    } else {
+      key = ok ? logit_key(v) : 0u;
+    }
+    h[i].hi = key;
+    h[i].lo = ~(uint32_t)e;
+    h[i].v = v;
+  }
+  // lane-local sort, first in the order at h[0] (odd-even transposition)
+#pragma unroll
+  for (int pass = 0; pass < PLM; ++pass) {
+#pragma unroll
+    for (int i = pass & 1; i + 1 < PLM; i += 2) {
+      if (topk_before(h[i + 1], h[i])) {
+        const TopkHead t = h[i];
+        h[i] = h[i + 1];
+        h[i + 1] = t;
+      }
+    }
+  }
+  if (lane < k) c_hi[warp * k + lane] = 0u;
+  __syncwarp();
+  for (int r = 0; r < k; ++r) {
+    const int w = topk_round_winner(h[0]);
+    if (w < 0) break;
+    if (lane == w) {
+      c_hi[warp * k + r] = h[0].hi;
+      c_lo[warp * k + r] = h[0].lo;
+      c_v[warp * k + r] = h[0].v;
+#pragma unroll
+      for (int i = 0; i + 1 < PLM; ++i) h[i] = h[i + 1];
+      h[PLM - 1].hi = 0u;
+    }
+  }
+  named_bar_sync(bar, nt);
+  if (warp == 0) {
+    // merge: lane l < nw walks list l
+    int ptr = 0;
+    TopkHead cur;
+    cur.hi = lane < nw ? c_hi[lane * k] : 0u;
+    cur.lo = lane < nw ? c_lo[lane * k] : 0u;
+    cur.v = lane < nw ? c_v[lane * k] : 0.f;
+    int my_id = 0;
+    float my_v = 0.f;
+    for (int r = 0; r < k; ++r) {
+      const int w = topk_round_winner(cur);
+      const uint32_t wl = __shfl_sync(0xFFFFFFFFu, cur.lo, w < 0 ? 0 : w);
+      const float wv = __shfl_sync(0xFFFFFFFFu, cur.v, w < 0 ? 0 : w);
+      if (lane == r) {
+        my_id = (int)~wl;
+        my_v = wv;
+      }
+      if (lane == w) {
+        ++ptr;
+        const bool more = ptr < k;
+        cur.hi = more ? c_hi[lane * k + ptr] : 0u;
+        cur.lo = more ? c_lo[lane * k + ptr] : 0u;
+        cur.v = more ? c_v[lane * k + ptr] : 0.f;
+      }
+    }
+    // ascending id: lane r's rank among the k winners
+    int rank = 0;
+    for (int i = 0; i < k; ++i) {
+      const int oi = __shfl_sync(0xFFFFFFFFu, my_id, i);
+      rank += (lane < k && oi < my_id) ? 1 : 0;
+    }
+    if (lane < k) {
+      s_id[rank] = my_id;
+      s_v[rank] = my_v;
+    }
+    __syncwarp();
+    const bool on = lane < k;
+    const int id = on ? s_id[lane] : 0;
+    topk_emit(a, b, on ? s_v[lane] : 0.f, id, lane);
+    if (bucket_b1) {
+      if (on) {
+        a.active_out[lane] = id;
+        a.pair_ids_out[lane] = lane;
+      }
+      if (lane == 0) {
+        a.offsets_out[E] = k;
+        *a.n_active_out = k;
+      }
+    }
+  }
+  if (bucket_b1) {
+    named_bar_sync(bar, nt);  // the selection, ascending, in s_id
+    for (int e = tid; e < E; e += nt) {
+      int below = 0;
+      bool on = false;
+      for (int i = 0; i < k; ++i) {
+        const int si = s_id[i];
+        below += si < e ? 1 : 0;
+        on = on || si == e;
+      }
+      a.offsets_out[e] = below;
+      a.counts[e] = on ? 1 : 0;
+    }
+  }
+}
+
+__device__ void topk_token_block(const GemvArgs& a, const float* __restrict__ lg, int b, int tid, int nt, int bar,
+                                 bool bucket_b1, unsigned char* scratch) {
+  const int nw = nt >> 5, E = a.n_experts;
+  const int per_lane = ((E + nw - 1) / nw + 31) / 32;
+  if (nw < 2 || nw > 32 || a.top_k < 1 || a.top_k > kMaxTopK || a.top_k > E || per_lane > 16) {
+    if (tid == 0) atomicExch(a.err, kErrBadPlan);
+    return;
+  }
+  if (per_lane <= 4) topk_token_block_pl<4>(a, lg, b, tid, nt, bar, bucket_b1, scratch);
+  else topk_token_block_pl<16>(a, lg, b, tid, nt, bar, bucket_b1, scratch);
 }
 
 // Staged combine: out = bf16(residual + y_shared + sum_j w_j y_j), one thread per element.

@@ -280,8 +280,10 @@ struct moe_layer {
   bool mx = false;         // the shapes allow it and its scale copies exist
   bool mx_forced = false;  // MOE_FLAG_MX_EXPERTS: at every batch size
   bool mx_default = false; // above batch 1 unless MOE_FLAG_NO_GROUPED / MOE_FLAG_WARP_MMA
-  CUtensorMap tm_agu{}, tm_adn{}, tm_bx{}, tm_bh{}, tm_bh8{};
-  bool swap_dn = false;     // the down projection takes the swapped-operand kernel (H a multiple of 256)
+  CUtensorMap tm_agu{}, tm_adn{}, tm_bx{}, tm_bh{}, tm_bx8{}, tm_bh8{};
+  bool swap = false;        // both projections take the swapped-operand kernels (H a multiple of 256)
+  float* sw_ws = nullptr;   // their stream-K partial sums [num_sms][2][16 x 256]
+  int* sw_cnt = nullptr;    // ... and per-item part counters [E * max(I/128, H/256)]
   uint8_t* aqx = nullptr;   // E2M1 terms of x per pair position [MB*k*T][H/2]
   uint8_t* bsfx = nullptr;  // ... their scales, chunk layout [MB*k][H/128][512]
   uint8_t* aqh = nullptr;   // E2M1 terms of h [MB*k*T][I/2]
@@ -567,7 +569,7 @@ MxArgs mx_args(const moe_layer* L, bool gate_up, int B, const moe_routing& r, co
   a.out_f32 = out;
   a.next_aq = gate_up ? L->aqh : nullptr;
   a.next_bsf = gate_up ? L->bsfh : nullptr;
-  a.next_rpp = L->swap_dn ? kSwRowsPerTok : kMxTerms;
+  a.next_rpp = L->swap ? kSwRowsPerTok : kMxTerms;
   a.n_stages = p.n_stages;
   a.stage_bytes = p.stage_bytes;
   a.off_up = p.off_up;
@@ -578,6 +580,46 @@ MxArgs mx_args(const moe_layer* L, bool gate_up, int B, const moe_routing& r, co
   return a;
 }
 
+// tokens per pass of the swapped kernels: every expert's (at most B) tokens
+// below batch 16, 16 from there
+int sw_tokens_per_pass(int B) { return std::min(B, kSwTokMax); }
+
+// arguments of a swapped-operand projection, without its outputs; the stage
+// ring holds the pass's activation rows, the two weight tiles and the scale
+// chunks (two per operand tile)
+SwArgs sw_args(const moe_layer* L, bool gate_up, int B, const moe_routing& r) {
+  const int H = L->cfg.hidden, I = L->cfg.inter, k = L->cfg.top_k;
+  SwArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.wsf = gate_up ? L->wsf_gu : L->wsf_dn;
+  a.a_tiles = (gate_up ? 2 * I : H) / kMxRows;
+  a.tile2 = gate_up ? I / kMxRows : 1;
+  a.K = gate_up ? H : I;
+  a.out_rows = gate_up ? I : H;
+  a.n_rt = gate_up ? I / kMxRows : H / kSwN;
+  a.top_k = k;
+  a.n_pairs = B * k;
+  a.n_experts = L->cfg.n_experts;
+  a.n_active = r.n_active;
+  a.active = r.active;
+  a.offsets = r.offsets;
+  a.pair_ids = r.pair_ids;
+  a.asf = gate_up ? L->bsfx : L->bsfh;
+  a.tpp = sw_tokens_per_pass(B);
+  a.split = B <= kSwTokMax ? 1 : 0;  // one pass per expert
+  a.off_w = (int)align_up((size_t)a.tpp * kSwRowsPerTok * 128, 1024);
+  a.off_sfa = a.off_w + 2 * kMxATile;
+  a.off_sfw = a.off_sfa + 2 * kMxChunkBytes;
+  a.stage_bytes = (int)align_up((size_t)a.off_sfw + 4 * kMxChunkBytes, 1024);
+  a.n_stages = std::min(kSwMaxStages, (kSmemBudget - 2 * kMxHeaderBytes) / a.stage_bytes);
+  a.ws = L->sw_ws;
+  a.item_cnt = L->sw_cnt;
+  a.err = L->err;
+  return a;
+}
+
+int sw_smem(const SwArgs& a) { return 2 * kMxHeaderBytes + a.n_stages * a.stage_bytes; }
+
 // gate/up on the tensor cores: x -> E2M1 terms per pair position, then the
 // block-scaled MMA kernel (h fp32 into `h`, and h's terms for the down kernel)
 cudaError_t launch_mx_gate_up(moe_layer* L, const void* x, int B, const moe_routing& r, float* h, cudaStream_t st,
@@ -586,11 +628,25 @@ cudaError_t launch_mx_gate_up(moe_layer* L, const void* x, int B, const moe_rout
   // batch 1: every position holds the same token, whose terms are made once
   const int by_token = B == 1 ? 1 : 0;
   const dim3 grid(B, (H / 32 + 7) / 8);
+  const int rpp = L->swap ? kSwRowsPerTok : kMxTerms;
+  const int tpp = L->swap ? sw_tokens_per_pass(B) : mx_n_max(B) / kMxTerms;
   cudaError_t e = launch_ex(mx_x_terms_kernel<kMxTerms>, grid, 256, 0, st, L->pdl, static_cast<const uint16_t*>(x),
-                            H, k, B * k, L->cfg.n_experts, mx_n_max(B) / kMxTerms,
+                            H, k, B * k, L->cfg.n_experts, tpp, rpp,
                             static_cast<const int*>(r.pair_ids), static_cast<const int*>(r.topk_idx),
                             static_cast<const int*>(r.offsets), by_token, L->aqx, L->bsfx, L->err);
   if (e != cudaSuccess) return e;
+  if (L->swap) {
+    SwArgs a = sw_args(L, true, B, r);
+    a.a_by_token = by_token;
+    a.h = h;
+    a.next_aq = L->aqh;
+    a.next_bsf = L->bsfh;
+    if (ev0 && (e = cudaEventRecord(ev0, st)) != cudaSuccess) return e;
+    e = launch_ex(mx_swap_kernel<true, kMxTerms>, L->num_sms, kMxThreads, sw_smem(a), st, L->pdl, L->tm_agu,
+                  L->tm_bx8, a);
+    if (e == cudaSuccess && ev1) e = cudaEventRecord(ev1, st);
+    return e;
+  }
   const MxPlan p = mx_plan(true, B);
   MxArgs a = mx_args(L, true, B, r, p, h);
   a.b_by_token = by_token;
@@ -601,32 +657,11 @@ cudaError_t launch_mx_gate_up(moe_layer* L, const void* x, int B, const moe_rout
   return e;
 }
 
-// down projection with the operands swapped (see mx_down_swap_kernel)
+// down projection with the operands swapped; with `residual` non-null fused
+// with the combine (and the next layer's L2 prefetch)
 cudaError_t launch_mx_down_swap(moe_layer* L, int B, const moe_routing& r, float* y, cudaStream_t st,
                                 const void* residual, void* out, const float* ys, const moe_layer* next) {
-  const int H = L->cfg.hidden, I = L->cfg.inter, k = L->cfg.top_k;
-  SwArgs a;
-  std::memset(&a, 0, sizeof(a));
-  a.wsf = L->wsf_dn;
-  a.a_tiles = H / kMxRows;
-  a.K = I;
-  a.out_rows = H;
-  a.top_k = k;
-  a.n_pairs = B * k;
-  a.n_experts = L->cfg.n_experts;
-  a.n_active = r.n_active;
-  a.active = r.active;
-  a.offsets = r.offsets;
-  a.pair_ids = r.pair_ids;
-  a.asf = L->bsfh;
-  // gate/up passes hold all of an expert's (at most B) tokens below batch 16
-  // and 16 from there: min(B, 16) tokens per pass gives the same pass starts
-  a.tpp = std::min(B, kSwTokMax);
-  a.off_w = (int)align_up((size_t)a.tpp * kSwRowsPerTok * 128, 1024);
-  a.off_sfa = a.off_w + 2 * kMxATile;
-  a.off_sfw = a.off_sfa + 2 * kMxChunkBytes;
-  a.stage_bytes = (int)align_up((size_t)a.off_sfw + 4 * kMxChunkBytes, 1024);
-  a.n_stages = std::min(kSwMaxStages, (kSmemBudget - 2 * kMxHeaderBytes) / a.stage_bytes);
+  SwArgs a = sw_args(L, false, B, r);
   a.y = y;
   if (residual) {
     a.comb_w = r.topk_w;
@@ -635,19 +670,17 @@ cudaError_t launch_mx_down_swap(moe_layer* L, int B, const moe_routing& r, float
     a.out_bf16 = static_cast<uint16_t*>(out);
     a.batch = B;
     a.tile_counter = L->tile_cnt;
-    if (next && L->prefetch) {
-      a.pf_ptr[0] = reinterpret_cast<const uint8_t*>(next->wr_t);
-      a.pf_bytes[0] = (long long)next->cfg.n_experts * next->cfg.hidden * 2;
-      if (next->cfg.shared_inter > 0) {
-        a.pf_ptr[1] = reinterpret_cast<const uint8_t*>(next->w.shared_gate_up);
-        a.pf_bytes[1] = (long long)2 * next->cfg.shared_inter * next->cfg.hidden * 2;
-      }
+  }
+  if (next && L->prefetch) {
+    a.pf_ptr[0] = reinterpret_cast<const uint8_t*>(next->wr_t);
+    a.pf_bytes[0] = (long long)next->cfg.n_experts * next->cfg.hidden * 2;
+    if (next->cfg.shared_inter > 0) {
+      a.pf_ptr[1] = reinterpret_cast<const uint8_t*>(next->w.shared_gate_up);
+      a.pf_bytes[1] = (long long)2 * next->cfg.shared_inter * next->cfg.hidden * 2;
     }
   }
-  a.err = L->err;
-  const int smem = 2 * kMxHeaderBytes + a.n_stages * a.stage_bytes;
-  return launch_ex(mx_down_swap_kernel<kMxTerms>, L->num_sms, kMxThreads, smem, st, L->pdl, L->tm_adn, L->tm_bh8,
-                   a);
+  return launch_ex(mx_swap_kernel<false, kMxTerms>, L->num_sms, kMxThreads, sw_smem(a), st, L->pdl, L->tm_adn,
+                   L->tm_bh8, a);
 }
 
 // down projection on the tensor cores; with `residual` non-null fused with
@@ -655,7 +688,7 @@ cudaError_t launch_mx_down_swap(moe_layer* L, int B, const moe_routing& r, float
 cudaError_t launch_mx_down(moe_layer* L, int B, const moe_routing& r, float* y, cudaStream_t st,
                            const void* residual = nullptr, void* out = nullptr, const float* ys = nullptr,
                            const moe_layer* next = nullptr) {
-  if (L->swap_dn) return launch_mx_down_swap(L, B, r, y, st, residual, out, ys, next);
+  if (L->swap) return launch_mx_down_swap(L, B, r, y, st, residual, out, ys, next);
   const MxPlan p = mx_plan(false, B);
   MxArgs a = mx_args(L, false, B, r, p, y);
   if (residual) {
@@ -868,6 +901,7 @@ cudaError_t launch_grouped(moe_layer* L, bool gate_up, int B, const moe_routing&
 
 cudaError_t launch_combine(moe_layer* L, int B, const moe_routing& r, const float* y, const float* ys,
                            const void* residual, void* out, cudaStream_t st);
+constexpr int kMxFusedCombineMaxB = 2;  // tensor-core down projection: combine inside up to this batch
 GemvArgs down_args(const moe_layer* L, int B, const moe_routing& r, float* y, bool fused, const void* residual,
                    void* out, const float* ys, const moe_layer* next);
 
@@ -876,7 +910,14 @@ cudaError_t launch_down(moe_layer* L, int B, const moe_routing& r, float* y, boo
   const int path = expert_path(L, B);
   if (path == MOE_PATH_TCGEN05) {
     (void)pdl;
-    return fused ? launch_mx_down(L, B, r, y, st, residual, out, ys, next) : launch_mx_down(L, B, r, y, st);
+    if (!fused) return launch_mx_down(L, B, r, y, st);
+    if (B <= kMxFusedCombineMaxB) return launch_mx_down(L, B, r, y, st, residual, out, ys, next);
+    // larger batches: the combine runs over every SM after the projection
+    // (in the projection kernel the last expert of a row tile would combine
+    // the tile's rows for all B tokens alone)
+    cudaError_t e = launch_mx_down(L, B, r, y, st, nullptr, nullptr, nullptr, next);
+    if (e == cudaSuccess) e = launch_combine(L, B, r, y, ys, residual, out, st);
+    return e;
   }
   if (path == MOE_PATH_GROUPED) {
     // tensor-core projection into y, then the fixed-order combine
@@ -1173,11 +1214,12 @@ moe_status_t moe_layer_create(const moe_layer_config* cfg, const moe_layer_weigh
   const size_t o_xs = take((size_t)MB * H * 2);
   const size_t o_rs = take((size_t)MB * H * 2);
   const size_t o_os = take((size_t)MB * H * 2);
-  const size_t mx_rows = (size_t)MB * k * kMxTerms;
-  const size_t o_aqx = take(mx_rows * (H / 2));
+  const size_t o_aqx = take((size_t)MB * k * kSwRowsPerTok * (H / 2));  // 8 rows per position (>= kMxTerms)
   const size_t o_sfx = take((size_t)MB * k * ((H + kMxKChunk - 1) / kMxKChunk) * kMxChunkBytes);
   const size_t o_aqh = take((size_t)MB * k * kSwRowsPerTok * (I / 2));  // 8 rows per position (>= kMxTerms)
   const size_t o_sfh = take((size_t)MB * k * ((I + kMxKChunk - 1) / kMxKChunk) * kMxChunkBytes);
+  const size_t o_sww = take((size_t)sms * 2 * kSwSlotFloats * 4);
+  const size_t o_swc = take((size_t)E * std::max(I / kMxRows, H / kSwN + 1) * 4);
   if (g_fail_next_alloc.exchange(false) || cudaMalloc(&L->arena, off) != cudaSuccess) {
     cudaGetLastError();
     delete L;
@@ -1211,6 +1253,8 @@ moe_status_t moe_layer_create(const moe_layer_config* cfg, const moe_layer_weigh
   L->bsfx = reinterpret_cast<uint8_t*>(A + o_sfx);
   L->aqh = reinterpret_cast<uint8_t*>(A + o_aqh);
   L->bsfh = reinterpret_cast<uint8_t*>(A + o_sfh);
+  L->sw_ws = reinterpret_cast<float*>(A + o_sww);
+  L->sw_cnt = reinterpret_cast<int*>(A + o_swc);
 
   cudaError_t e = cudaMemset(L->arena, 0, off);
   if (e == cudaSuccess) {
@@ -1252,10 +1296,12 @@ moe_status_t moe_layer_create(const moe_layer_config* cfg, const moe_layer_weigh
                        kMxBBox) &&
             encode_map(&L->tm_bh, CU_TENSOR_MAP_DATA_TYPE_UINT8, L->aqh, (uint64_t)I / 2, mxr, (uint64_t)I / 2, 128,
                        kMxBBox);
-    // the swapped down projection reads h's terms 8 rows per position (box 8 rows)
-    L->swap_dn = L->mx && H % kSwN == 0 &&
-                 encode_map(&L->tm_bh8, CU_TENSOR_MAP_DATA_TYPE_UINT8, L->aqh, (uint64_t)I / 2,
-                            (uint64_t)MB * k * kSwRowsPerTok, (uint64_t)I / 2, 128, kSwRowsPerTok);
+    // the swapped kernels read x's and h's terms 8 rows per position (box 8 rows)
+    L->swap = L->mx && H % kSwN == 0 &&
+              encode_map(&L->tm_bx8, CU_TENSOR_MAP_DATA_TYPE_UINT8, L->aqx, (uint64_t)H / 2,
+                         (uint64_t)MB * k * kSwRowsPerTok, (uint64_t)H / 2, 128, kSwRowsPerTok) &&
+              encode_map(&L->tm_bh8, CU_TENSOR_MAP_DATA_TYPE_UINT8, L->aqh, (uint64_t)I / 2,
+                         (uint64_t)MB * k * kSwRowsPerTok, (uint64_t)I / 2, 128, kSwRowsPerTok);
     if (L->mx) {
       // the scale arrays hold one byte per 32 weights: the chunk copies are the same size
       const size_t gu_bytes = (size_t)E * 2 * I * (H / 32), dn_bytes = (size_t)E * H * (I / 32);
@@ -1328,7 +1374,9 @@ moe_status_t moe_layer_create(const moe_layer_config* cfg, const moe_layer_weigh
     if (e == cudaSuccess)
       e = raise_smem_limit(reinterpret_cast<const void*>(mx_expert_kernel<false, kMxTerms>), kSmemBudget);
     if (e == cudaSuccess)
-      e = raise_smem_limit(reinterpret_cast<const void*>(mx_down_swap_kernel<kMxTerms>), kSmemBudget);
+      e = raise_smem_limit(reinterpret_cast<const void*>(mx_swap_kernel<false, kMxTerms>), kSmemBudget);
+    if (e == cudaSuccess)
+      e = raise_smem_limit(reinterpret_cast<const void*>(mx_swap_kernel<true, kMxTerms>), kSmemBudget);
   }
   // persistent batch-1 kernel: needs the bf16 (or no) shared expert, no side
   // stream, and one shape-specialised or one generic instance for all streams

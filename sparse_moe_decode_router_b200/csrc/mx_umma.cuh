@@ -239,6 +239,13 @@ __device__ __forceinline__ float e2m1_to_f32(uint32_t c) {
   return (c & 8u) ? -mag : mag;
 }
 
+__device__ __forceinline__ void add4(float4& s, const float4& v) {
+  s.x += v.x;
+  s.y += v.y;
+  s.z += v.z;
+  s.w += v.w;
+}
+
 __device__ __forceinline__ float warp_amax(float v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
@@ -248,21 +255,7 @@ __device__ __forceinline__ float warp_amax(float v) {
 // byte of a B column's scale in its chunk: column n = r0 + 32*r1, K-block kb
 __device__ __forceinline__ int sf_chunk_byte(int n, int kb) { return 16 * (n & 31) + 4 * (n >> 5) + kb; }
 
-// first position of the pass that reads position q (passes of tpp tokens
-// from the expert's offset); -1 if the routing plan is inconsistent
-__device__ __forceinline__ int pass_start(int q, int top_k, int n_pairs, int n_experts, int tpp,
-                                          const int* __restrict__ pair_ids, const int* __restrict__ topk_idx,
-                                          const int* __restrict__ offsets) {
-  const int p = __ldcg(pair_ids + q);
-  if (p < 0 || p >= n_pairs) return -1;
-  const int e = __ldcg(topk_idx + p);
-  if (e < 0 || e >= n_experts) return -1;
-  const int off = __ldcg(offsets + e), end = __ldcg(offsets + e + 1);
-  if (off < 0 || q < off || q >= end) return -1;
-  return off + (q - off) / tpp * tpp;
-}
-
-// x (bf16 [B][K]) -> terms of the gate/up activations: row q*kTerms + t of
+// x (bf16 [B][K]) -> terms of the gate/up activations: row q*rpp + t of
 // aq [.][K/2] (packed E2M1, even element in the low nibble) and the scales
 // into the chunks of q's pass, for every pair position q of the token.
 // Grid (B, ceil(K/256)), 8 warps: warp w of CTA (b, g) takes the 32-element
@@ -272,20 +265,28 @@ __device__ __forceinline__ int pass_start(int q, int top_k, int n_pairs, int n_e
 // reads, and its chunk is chunk 0 (columns = terms).
 template <int kTerms>
 __global__ void __launch_bounds__(256) mx_x_terms_kernel(const uint16_t* __restrict__ x, int K, int top_k, int n_pairs,
-                                                         int n_experts, int tpp, const int* __restrict__ pair_ids,
+                                                         int n_experts, int tpp, int rpp,
+                                                         const int* __restrict__ pair_ids,
                                                          const int* __restrict__ topk_idx,
                                                          const int* __restrict__ offsets, int by_token,
                                                          uint8_t* __restrict__ aq, uint8_t* __restrict__ bsf, int* err) {
-  __shared__ int s_q[kMaxTopK], s_p0[kMaxTopK];
+  __shared__ int s_q[kMaxTopK], s_p0[kMaxTopK], s_e[kMaxTopK];
   pdl_wait();
   const int b = blockIdx.x, tid = threadIdx.x;
+  const int lane = tid & 31, blk = blockIdx.y * 8 + (tid >> 5);
   const int nq = by_token ? 1 : top_k;
-  if (nq < 1 || nq > kMaxTopK) {
+  if (nq < 1 || nq > kMaxTopK || rpp < kTerms || tpp * rpp > kMxRows) {
     if (tid == 0) atomicExch(err, kErrBadPlan);
     pdl_launch_dependents();
     return;
   }
-  if (tid < nq) s_q[tid] = by_token ? 0 : -1;
+  // written by preceding kernels: coherent loads, all issued before the first wait
+  const bool has_blk = blk < (K >> 5);
+  const uint16_t xv = has_blk ? __ldcg(x + (size_t)b * K + 32 * blk + lane) : (uint16_t)0;
+  if (tid < nq) {
+    s_q[tid] = by_token ? 0 : -1;
+    s_e[tid] = by_token ? 0 : __ldcg(topk_idx + b * top_k + tid);
+  }
   __syncthreads();
   if (!by_token) {
     // the token's pairs b*top_k + j sit at the positions q with pair_ids[q] = that pair
@@ -298,8 +299,16 @@ __global__ void __launch_bounds__(256) mx_x_terms_kernel(const uint16_t* __restr
   }
   bool bad = false;
   if (tid < nq) {
-    const int q = s_q[tid];
-    const int p0 = by_token ? 0 : (q < 0 ? -1 : pass_start(q, top_k, n_pairs, n_experts, tpp, pair_ids, topk_idx, offsets));
+    // the first position of the pass that holds q: passes of tpp tokens from the expert's offset
+    const int q = s_q[tid], e = s_e[tid];
+    int p0 = 0;
+    if (!by_token) {
+      p0 = -1;
+      if (q >= 0 && e >= 0 && e < n_experts) {
+        const int off = __ldcg(offsets + e), end = __ldcg(offsets + e + 1);
+        if (off >= 0 && q >= off && q < end) p0 = off + (q - off) / tpp * tpp;
+      }
+    }
     s_p0[tid] = p0;
     bad = p0 < 0;
   }
@@ -308,10 +317,8 @@ __global__ void __launch_bounds__(256) mx_x_terms_kernel(const uint16_t* __restr
     pdl_launch_dependents();
     return;
   }
-  const int lane = tid & 31, blk = blockIdx.y * 8 + (tid >> 5);
-  if (blk < (K >> 5)) {
-    // written by a preceding kernel: coherent path
-    float v = __uint_as_float((uint32_t)__ldcg(x + (size_t)b * K + 32 * blk + lane) << 16);
+  if (has_blk) {
+    float v = __uint_as_float((uint32_t)xv << 16);
     uint32_t w[kTerms];
     int ex[kTerms];
 #pragma unroll
@@ -327,12 +334,12 @@ __global__ void __launch_bounds__(256) mx_x_terms_kernel(const uint16_t* __restr
     }
     for (int j = 0; j < nq; ++j) {
       const int q = s_q[j], p0 = s_p0[j];
-      const int n0 = (q - p0) * kTerms;  // this position's first B column in its pass
+      const int n0 = (q - p0) * rpp;  // this position's first row (column) in its pass's scale chunks
       uint8_t* chunk = bsf + ((size_t)p0 * (K / kMxKChunk) + (blk >> 2)) * kMxChunkBytes;
 #pragma unroll
       for (int t = 0; t < kTerms; ++t) {
         if ((lane & 7) == 0)
-          *reinterpret_cast<uint32_t*>(aq + ((size_t)q * kTerms + t) * (K / 2) + 16 * blk + (lane >> 3) * 4) = w[t];
+          *reinterpret_cast<uint32_t*>(aq + ((size_t)q * rpp + t) * (K / 2) + 16 * blk + (lane >> 3) * 4) = w[t];
         if (lane == 0) chunk[sf_chunk_byte(n0 + t, blk & 3)] = (uint8_t)(ex[t] + 127);
       }
     }
@@ -723,37 +730,70 @@ __global__ void __launch_bounds__(kMxThreads, 1)
 }
 
 // ---------------------------------------------------------------------------
-// Down projection with the operands swapped: the activation terms are the A
-// operand (M = 128 rows: row 8*i + t = token i of the pass, term t; rows
-// with t >= kTerms and beyond the pass are padding whose results are
-// dropped) and the weights the B operand (N = 256: two 128-row tiles of
-// W_down).  One MMA then covers 256 weight rows x 64 K instead of 128, and
-// a stage of 32 KB of weights takes 4 MMAs and 6 scale copies instead of 8
-// and 8: the tensor pipe issues 10 operations per 32 KB, not 16.  The
-// accumulator (128 x 256 fp32) takes half of tensor memory, so there is one
-// buffer: the MMAs of the next item wait until the epilogue has read it.
+// Expert projections with the operands swapped: the activation terms are
+// the A operand (M = 128 rows: row 8*i + t = token i of the pass, term t;
+// rows with t >= kTerms and beyond the pass are padding whose results are
+// dropped) and the weights the B operand (N = 256: two 128-row weight tiles
+// side by side).  An item is (active expert, 256 weight rows): for gate/up
+// the gate tile and the up tile of the same 128 rows of h, for the down
+// projection two consecutive 128-row tiles of W_down.  One MMA covers 256
+// weight rows x 64 K, so a stage of 32 KB of weights takes 4 MMAs and 6
+// scale copies.  The accumulator (128 x 256 fp32) takes half of tensor
+// memory, so there is one buffer: the epilogue frees it as soon as it has
+// read it.
+//
+// Work split.  When every expert's tokens fit one pass (batch <= 16) the
+// launch's (item, K stage) list is cut into equal stretches, one per CTA
+// ("stream-K"): every SM streams the same number of weight bytes.  A
+// stretch holds the end of one item, whole items and the start of another;
+// the pieces ("parts") of a split item write their term-summed partial sums
+// to a workspace slot of their CTA, and the last part to arrive (a counter
+// per item) adds the parts in ascending K order and runs the epilogue.
+// Larger batches cut the item list into equal runs of whole items (each
+// expert's passes of 16 tokens stay in one CTA).
+//
+// Epilogue.  Warp w reads TMEM lanes 32*(w%4).. = tokens 4*(w%4) .. +3 of
+// the pass, 8 lanes (terms) each.  The terms of a token are summed across
+// its 8 lanes by recursive halving: after three exchange steps lane l of
+// the group holds the sums of columns 32c + 4l .. 32c + 4l + 3 of each
+// 32-column chunk c.  Gate/up then forms h = silu(g) * u for those rows and
+// splits h into the down projection's E2M1 terms (32-row blocks: the max
+// over the group's 8 lanes); the down projection stores y and, for the last
+// expert of a 256-row tile, runs the fused combine.
 constexpr int kSwRowsPerTok = 8;                    // A rows per token (kTerms used)
 constexpr int kSwTokMax = kMxRows / kSwRowsPerTok;  // 16 tokens per pass
 constexpr int kSwN = 256;                           // weight rows per MMA (two tiles)
 constexpr int kSwSfColsStage = 24;                  // activations 2 chunks x 4 + weights 2 chunks x 8
 constexpr int kSwMaxStages = (kMxTmemCols - kSwN) / kSwSfColsStage;  // 10
+constexpr int kSwSlotFloats = kSwTokMax * kSwN;     // one workspace slot: a part's sums for a pass
 static_assert(kMxHeaderBytes >= 8 * (2 * kSwMaxStages + 6) + 32, "header");
 
 struct SwArgs {
-  const uint8_t* wsf;       // weight scales, chunk layout [E * H/128][I/128][512]
-  int a_tiles;              // 128-row tiles per expert (H / 128)
-  int K;                    // I, multiple of 128
-  int out_rows;             // H, multiple of 256
+  const uint8_t* wsf;       // weight scales, chunk layout [weight tiles][K/128][512]
+  int a_tiles;              // 128-row weight tiles per expert (gate/up: 2I/128, down: H/128)
+  int tile2;                // tiles from an item's first weight tile to its second (gate/up: I/128, down: 1)
+  int K;                    // gate/up H, down I; multiple of 128
+  int out_rows;             // gate/up I, down H: rows of the projection's output per pair
+  int n_rt;                 // items per expert (gate/up I/128, down H/256)
   int top_k, n_pairs, n_experts;
   const int* n_active;
   const int* active;
   const int* offsets;
   const int* pair_ids;
   const uint8_t* asf;       // activation scale chunks [pass-start position][K/128][512], row m = 8*i + t
+  int a_by_token;           // batch-1 gate/up: every position reads row set 0 and chunk 0 (the token)
   int tpp;                  // tokens per pass (<= kSwTokMax)
+  int split;                // 1: stream-K over (item, stage); needs every expert's tokens in one pass
   int n_stages, stage_bytes, off_w, off_sfa, off_sfw;  // the activation rows sit at offset 0 of a stage
+  float* ws;                // stream-K partial sums: [grid][2 slots][kSwSlotFloats]
+  int* item_cnt;            // [n_experts * n_rt], zero between launches
+  // gate/up
+  float* h;                 // h fp32 [pair][I], or null
+  uint8_t* next_aq;         // h's E2M1 terms [pos*8 + t][I/2]
+  uint8_t* next_bsf;        // their scale chunks [pass-start position][I/128][512], row 8*i + t
+  // down
   float* y;                 // [pair][H]
-  const float* comb_w;      // fused combine as MxArgs: topk_w [B][k]
+  const float* comb_w;      // fused combine (topk_w [B][k]) or null
   const float* y_shared;
   const uint16_t* residual;
   uint16_t* out_bf16;
@@ -764,45 +804,119 @@ struct SwArgs {
   int* err;
 };
 
-struct SwUnit { int e, rt, tok, ntok; };
+// the launch's work list in K-stage units: stage it of item it / KS
+struct SwSplit {
+  long long T, G;  // stages of the list; CTAs that take a stretch (the others have none)
+  __device__ long long first(long long c) const { return c >= G ? T : c * T / G; }
+  // the CTA whose stretch holds stage s: the largest c with first(c) <= s
+  __device__ long long owner(long long s) const { return ((s + 1) * G + T - 1) / T - 1; }
+};
+
+struct SwRun {
+  int e, rt, tok, ntok;  // expert, item within the expert, first position and tokens of the pass
+  long long item;        // item index in the launch's list
+  int k0, nk;            // first K stage and stages of the run
+  int part, nparts;      // this run's piece of the item (stream-K), and the item's pieces
+  bool last_pass;
+};
 
 struct SwWalk {
   const SwArgs& a;
-  long long it, hi;
-  int n_rt, pass, npass, e, tok0, cnt;
-  __device__ SwWalk(const SwArgs& args, long long lo, long long hi_, int nrt)
-      : a(args), it(lo), hi(hi_), n_rt(nrt), pass(0), npass(0), e(0), tok0(0), cnt(0) {
+  const SwSplit& sp;
+  long long it, hi, item;
+  int KS, pass, npass, e, tok0, cnt;
+  __device__ SwWalk(const SwArgs& args, const SwSplit& split, long long lo, long long hi_, int ks)
+      : a(args), sp(split), it(lo), hi(hi_), item(0), KS(ks), pass(0), npass(0), e(0), tok0(0), cnt(0) {
     if (it < hi) load();
   }
   __device__ void load() {
-    const int g = (int)(it / n_rt);
+    item = it / KS;
+    const int g = (int)(item / a.n_rt);
     e = __ldcg(a.active + g);
     if (e < 0 || e >= a.n_experts) e = 0;
     tok0 = __ldcg(a.offsets + e);
     cnt = __ldcg(a.offsets + e + 1) - tok0;
     if (tok0 < 0 || cnt < 1 || tok0 + cnt > a.n_pairs) { tok0 = 0; cnt = 1; }
-    npass = (cnt + a.tpp - 1) / a.tpp;
+    npass = a.split ? 1 : (cnt + a.tpp - 1) / a.tpp;
     pass = 0;
   }
   __device__ bool valid() const { return it < hi; }
-  __device__ SwUnit unit() const {
-    SwUnit u;
-    u.e = e;
-    u.rt = (int)(it % n_rt);
-    u.tok = tok0 + pass * a.tpp;
-    u.ntok = min(a.tpp, cnt - pass * a.tpp);
-    return u;
+  __device__ SwRun run() const {
+    SwRun r;
+    r.e = e;
+    r.item = item;
+    r.rt = (int)(item % a.n_rt);
+    r.tok = tok0 + pass * a.tpp;
+    r.ntok = min(a.tpp, cnt - pass * a.tpp);
+    r.k0 = (int)(it - item * KS);
+    r.nk = (int)(min(hi, (item + 1) * KS) - it);
+    if (a.split) {
+      const long long c0 = sp.owner(item * KS);
+      r.part = (int)(sp.owner(it) - c0);
+      r.nparts = (int)(sp.owner((item + 1) * KS - 1) - c0 + 1);
+    } else {
+      r.part = 0;
+      r.nparts = 1;
+    }
+    r.last_pass = pass == npass - 1;
+    return r;
   }
   __device__ void next() {
     if (++pass < npass) return;
-    if (++it < hi) load();
+    it = min(hi, (item + 1) * KS);
+    if (it < hi) load();
   }
 };
 
-template <int kTerms>
+__device__ __forceinline__ void tc_ld32(uint32_t taddr, float (&v)[32]) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
+        "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]),
+        "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+        "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// sum of 32 columns over the 8 lanes of a group (xor 4, 2, 1 exchanges);
+// lane l8 of the group returns columns 4*l8 .. 4*l8 + 3
+__device__ __forceinline__ float4 group_reduce_scatter(const float (&v)[32], int l8) {
+  const bool k2 = (l8 & 4) != 0, k1 = (l8 & 2) != 0, k0 = (l8 & 1) != 0;
+  float w[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const float mine = k2 ? v[16 + i] : v[i], send = k2 ? v[i] : v[16 + i];
+    w[i] = mine + __shfl_xor_sync(0xFFFFFFFFu, send, 4);
+  }
+  float x[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const float mine = k1 ? w[8 + i] : w[i], send = k1 ? w[i] : w[8 + i];
+    x[i] = mine + __shfl_xor_sync(0xFFFFFFFFu, send, 2);
+  }
+  float y[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float mine = k0 ? x[4 + i] : x[i], send = k0 ? x[i] : x[4 + i];
+    y[i] = mine + __shfl_xor_sync(0xFFFFFFFFu, send, 1);
+  }
+  return make_float4(y[0], y[1], y[2], y[3]);
+}
+
+__device__ __forceinline__ float group_amax(float v) {
+  v = fmaxf(v, __shfl_xor_sync(0xFFFFFFFFu, v, 1));
+  v = fmaxf(v, __shfl_xor_sync(0xFFFFFFFFu, v, 2));
+  return fmaxf(v, __shfl_xor_sync(0xFFFFFFFFu, v, 4));
+}
+
+template <bool kGU, int kTerms>
 __global__ void __launch_bounds__(kMxThreads, 1)
-    mx_down_swap_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmA,
-                        const SwArgs a) {
+    mx_swap_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmA,
+                   const SwArgs a) {
   static_assert(kTerms >= 1 && kTerms <= kSwRowsPerTok, "terms");
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -855,15 +969,26 @@ __global__ void __launch_bounds__(kMxThreads, 1)
     if (tid == 0) atomicExch(a.err, kErrBadPlan);
     n_groups = n_groups < 0 ? 0 : a.n_experts;
   }
-  const int n_rt = a.out_rows / kSwN;
-  const long long n_items = (long long)n_groups * n_rt;
-  const long long lo = n_items * blockIdx.x / gridDim.x;
-  const long long hi = n_items * (blockIdx.x + 1) / gridDim.x;
-  const bool plan_ok = ns >= 1 && ns <= kSwMaxStages && (K % kMxKChunk) == 0 && (a.out_rows % kSwN) == 0 &&
-                       a.tpp >= 1 && a.tpp <= kSwTokMax && a.off_w >= a.tpp * kSwRowsPerTok * 128 &&
-                       a.off_w + 2 * kMxATile >= kMxRows * 128;
+  const long long n_items = (long long)n_groups * a.n_rt;
+  SwSplit sp;
+  long long lo, hi;
+  if (a.split) {
+    sp.T = n_items * KS;
+    sp.G = max(1ll, min((long long)gridDim.x, sp.T / 2));
+    lo = sp.first(blockIdx.x);
+    hi = sp.first(blockIdx.x + 1);
+  } else {
+    sp.T = n_items * KS;
+    sp.G = gridDim.x;
+    lo = n_items * blockIdx.x / gridDim.x * KS;
+    hi = n_items * (blockIdx.x + 1) / gridDim.x * KS;
+  }
+  const bool plan_ok = ns >= 1 && ns <= kSwMaxStages && (K % kMxKChunk) == 0 && a.n_rt >= 1 && a.tpp >= 1 &&
+                       a.tpp <= kSwTokMax && a.off_w >= a.tpp * kSwRowsPerTok * 128 &&
+                       a.off_w + 2 * kMxATile >= kMxRows * 128 && (!a.split || gridDim.x <= 4096);
   if (!plan_ok && tid == 0) atomicExch(a.err, kErrBadPlan);
   const long long lim_long = 1ll << 31, lim_short = 1ll << 20;
+  const int step = kGU ? 1 : 2;  // weight tiles per item along the expert's rows
 
   if (plan_ok && warp == 0) {
     // ------------------------------ TMA producer ------------------------------
@@ -871,13 +996,15 @@ __global__ void __launch_bounds__(kMxThreads, 1)
       const uint64_t pol = l2_policy_evict_first();
       int s = 0;
       uint32_t ph = 0;
-      for (SwWalk w(a, lo, hi, n_rt); w.valid() && !*s_abort; w.next()) {
-        const SwUnit u = w.unit();
-        const long long tile0 = (long long)u.e * a.a_tiles + 2 * u.rt;  // the item's two 128-row weight tiles
+      for (SwWalk w(a, sp, lo, hi, KS); w.valid() && !*s_abort; w.next()) {
+        const SwRun r = w.run();
+        const long long tile0 = (long long)r.e * a.a_tiles + (long long)step * r.rt;
+        const long long tile1 = tile0 + a.tile2;
         const uint8_t* sfw0 = a.wsf + tile0 * KC * kMxChunkBytes;
-        const uint8_t* sfw1 = sfw0 + (size_t)KC * kMxChunkBytes;
-        const uint8_t* sfa = a.asf + (size_t)u.tok * KC * kMxChunkBytes;
-        for (int kt = 0; kt < KS; ++kt) {
+        const uint8_t* sfw1 = a.wsf + tile1 * KC * kMxChunkBytes;
+        const int arow = a.a_by_token ? 0 : r.tok;
+        const uint8_t* sfa = a.asf + (size_t)arow * KC * kMxChunkBytes;
+        for (int kt = r.k0; kt < r.k0 + r.nk; ++kt) {
           if (!mbar_wait_bounded(&empty_bar[s], ph ^ 1u, *s_abort ? lim_short : lim_long)) {
             atomicExch(a.err, kErrTimeout);
             *s_abort = 1;
@@ -887,11 +1014,12 @@ __global__ void __launch_bounds__(kMxThreads, 1)
           const uint32_t cb = (uint32_t)(nck * kMxChunkBytes);
           unsigned char* st = ring + (size_t)s * a.stage_bytes;
           const uint32_t sa = smem_addr(st);
-          mbar_arrive_expect_tx(&full_bar[s], (uint32_t)u.ntok * (kSwRowsPerTok * 128u) + 2u * kMxATile + 3u * cb);
-          for (int i = 0; i < u.ntok; ++i)
-            tma_load_2d_nohint(sa + i * kSwRowsPerTok * 128, &tmA, kt * 128, (u.tok + i) * kSwRowsPerTok, &full_bar[s]);
+          mbar_arrive_expect_tx(&full_bar[s], (uint32_t)r.ntok * (kSwRowsPerTok * 128u) + 2u * kMxATile + 3u * cb);
+          for (int i = 0; i < r.ntok; ++i)
+            tma_load_2d_nohint(sa + i * kSwRowsPerTok * 128, &tmA, kt * 128,
+                               (a.a_by_token ? 0 : r.tok + i) * kSwRowsPerTok, &full_bar[s]);
           tma_load_2d(sa + a.off_w, &tmW, kt * 128, (int)(tile0 * kMxRows), &full_bar[s], pol);
-          tma_load_2d(sa + a.off_w + kMxATile, &tmW, kt * 128, (int)((tile0 + 1) * kMxRows), &full_bar[s], pol);
+          tma_load_2d(sa + a.off_w + kMxATile, &tmW, kt * 128, (int)(tile1 * kMxRows), &full_bar[s], pol);
           const size_t ck = (size_t)2 * kt * kMxChunkBytes;
           bulk_g2s_nohint(st + a.off_sfa, sfa + ck, cb, &full_bar[s]);
           bulk_g2s(st + a.off_sfw, sfw0 + ck, cb, &full_bar[s], pol);
@@ -922,7 +1050,8 @@ __global__ void __launch_bounds__(kMxThreads, 1)
       int s = 0, uc = 0;
       uint32_t ph = 0;
       const uint32_t idesc = mx_idesc(kSwN);
-      for (SwWalk w(a, lo, hi, n_rt); w.valid() && !*s_abort; w.next(), ++uc) {
+      for (SwWalk w(a, sp, lo, hi, KS); w.valid() && !*s_abort; w.next(), ++uc) {
+        const SwRun r = w.run();
         if (!mbar_wait_bounded(acc_empty, ((uint32_t)uc & 1u) ^ 1u, lim_long)) {
           atomicExch(a.err, kErrTimeout);
           *s_abort = 1;
@@ -930,7 +1059,7 @@ __global__ void __launch_bounds__(kMxThreads, 1)
         }
         tc_fence_after();
         bool ok = true;
-        for (int kt = 0; kt < KS && ok; ++kt) {
+        for (int kt = r.k0; kt < r.k0 + r.nk; ++kt) {
           if (!mbar_wait_bounded(&full_bar[s], ph, *s_abort ? lim_short : lim_long)) {
             atomicExch(a.err, kErrTimeout);
             *s_abort = 1;
@@ -943,7 +1072,7 @@ __global__ void __launch_bounds__(kMxThreads, 1)
           const uint32_t sfa = tmem + (uint32_t)(kSwN + kSwSfColsStage * s), sfw = sfa + 8u;
           for (int c = 0; c < nck; ++c) {
             tc_cp_32x128_x4(sfa + 4u * c, desc_sf(st + a.off_sfa + c * kMxChunkBytes));
-            // weight rows 0..127 of the item -> columns 0..3 of the pair, rows 128..255 -> 4..7
+            // the first weight tile -> columns 0..3 of the chunk's pair, the second -> 4..7
             tc_cp_32x128_x4(sfw + 8u * c, desc_sf(st + a.off_sfw + c * kMxChunkBytes));
             tc_cp_32x128_x4(sfw + 8u * c + 4u, desc_sf(st + a.off_sfw + (2 + c) * kMxChunkBytes));
           }
@@ -951,7 +1080,7 @@ __global__ void __launch_bounds__(kMxThreads, 1)
           for (int j = 0; j < 2 * nck; ++j) {
             const uint32_t sb = 2u * (uint32_t)(j & 1), cj = (uint32_t)(j >> 1);
             const uint32_t id = idesc | (sb << 29) | (sb << 4);
-            const uint32_t acc = (kt > 0 || j > 0) ? 1u : 0u;
+            const uint32_t acc = (kt > r.k0 || j > 0) ? 1u : 0u;
             const uint32_t tag = sb << 30;
             tc_mma_mxf4(tmem, ad + 2u * j, bd + 2u * j, id, (sfa + 4u * cj) | tag, (sfw + 8u * cj) | tag, acc);
           }
@@ -967,11 +1096,10 @@ __global__ void __launch_bounds__(kMxThreads, 1)
     __syncwarp();
   } else if (plan_ok && warp >= 2) {
     // ------------------------------ epilogue ----------------------------------
-    // warp w reads TMEM lanes 32*(w%4).. = tokens 4*(w%4) .. +3 of the pass,
-    // 8 lanes (terms) each; the terms are summed across those lanes
     const int q = warp & 3;
     const uint32_t lane_base = tmem + ((uint32_t)(32 * q) << 16);
-    const int tq = 4 * q + (lane >> 3), t = lane & 7;  // token of the pass, term
+    const int l8 = lane & 7, ti = 4 * q + (lane >> 3);  // term (and column quarter), token of the pass
+    const int et = (warp - 2) * 32 + lane;              // 0..127 over the four epilogue warps
     int uc = 0;
     uint32_t epi_ph = 0;
     auto epi_sync = [&]() -> bool {
@@ -986,9 +1114,8 @@ __global__ void __launch_bounds__(kMxThreads, 1)
       }
       return ok;
     };
-    const int et = (warp - 2) * 32 + lane;  // 0..127 over the four epilogue warps
-    for (SwWalk w(a, lo, hi, n_rt); w.valid(); w.next(), ++uc) {
-      const SwUnit u = w.unit();
+    for (SwWalk w(a, sp, lo, hi, KS); w.valid(); w.next(), ++uc) {
+      const SwRun r = w.run();
       bool ok = !*s_abort && mbar_wait_bounded(acc_full, (uint32_t)uc & 1u, lim_long);
       ok = __all_sync(0xFFFFFFFFu, ok);
       if (!ok) {
@@ -997,55 +1124,126 @@ __global__ void __launch_bounds__(kMxThreads, 1)
         break;
       }
       tc_fence_after();
-      const int row0 = u.rt * kSwN;
-      int pr = 0;
-      const bool mine = tq < u.ntok;  // this lane's token is in the pass
-      if (mine) {
-        pr = __ldcg(a.pair_ids + u.tok + tq);
-        if (pr < 0 || pr >= a.n_pairs) pr = 0;
-      }
-      if (4 * q < u.ntok) {  // warp-uniform: the quadrant holds tokens of the pass
-        float v[16];
-        tc_ld16(lane_base, v);
-#pragma unroll 1
-        for (int c = 0; c < kSwN / 16; ++c) {
+      const bool quad = 4 * q < r.ntok;  // warp-uniform: the quadrant holds tokens of the pass
+      const bool mine = ti < r.ntok;
+      float4 res[kSwN / 32];
+      if (quad) {
+        float v[32];
+        tc_ld32(lane_base, v);
+#pragma unroll
+        for (int c = 0; c < kSwN / 32; ++c) {
           tc_wait_ld();
-          float cur[16];
+          float cur[32];
 #pragma unroll
-          for (int i = 0; i < 16; ++i) cur[i] = t < kTerms ? v[i] : 0.f;
-          if (c + 1 < kSwN / 16) tc_ld16(lane_base + (uint32_t)(16 * (c + 1)), v);
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            // the terms of a token: a fixed pairwise tree over its 8 lanes
-            cur[i] += __shfl_xor_sync(0xFFFFFFFFu, cur[i], 1);
-            cur[i] += __shfl_xor_sync(0xFFFFFFFFu, cur[i], 2);
-            cur[i] += __shfl_xor_sync(0xFFFFFFFFu, cur[i], 4);
-          }
-          if (mine && t == 0) {
-            float4* dst = reinterpret_cast<float4*>(a.y + (size_t)pr * a.out_rows + row0 + 16 * c);
-#pragma unroll
-            for (int i = 0; i < 4; ++i) dst[i] = make_float4(cur[4 * i], cur[4 * i + 1], cur[4 * i + 2], cur[4 * i + 3]);
-          }
+          for (int i = 0; i < 32; ++i) cur[i] = l8 < kTerms ? v[i] : 0.f;
+          if (c + 1 < kSwN / 32) tc_ld32(lane_base + (uint32_t)(32 * (c + 1)), v);
+          res[c] = group_reduce_scatter(cur, l8);
         }
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(acc_empty);
-      if (a.comb_w && w.pass == w.npass - 1) {
+      if (lane == 0) mbar_arrive(acc_empty);  // the accumulator is free for the next run
+      bool fin = true;
+      if (r.nparts > 1) {
+        // a piece of a split item: its sums to the CTA's slot, then the count
+        const long long c_me = blockIdx.x;
+        const int my_slot = (int)(2 * c_me + (sp.first(c_me) >= r.item * KS ? 0 : 1));
+        if (quad && mine) {
+          float4* dst = reinterpret_cast<float4*>(a.ws + (size_t)my_slot * kSwSlotFloats + (size_t)ti * kSwN + 4 * l8);
+#pragma unroll
+          for (int c = 0; c < kSwN / 32; ++c) dst[8 * c] = res[c];
+        }
+        if (!epi_sync()) break;
+        if (warp == 2 && lane == 0) {
+          fence_acq_rel_gpu();
+          const int prev = atomicAdd(&a.item_cnt[r.item], 1);
+          const bool last = prev == r.nparts - 1;
+          if (last) {
+            fence_acq_rel_gpu();
+            a.item_cnt[r.item] = 0;
+          }
+          *s_last = last ? 1 : 0;
+        }
+        if (!epi_sync()) break;
+        fin = *s_last != 0;
+        if (fin && quad) {
+          // every piece, ascending K order
+          const long long c0 = sp.owner(r.item * KS);
+#pragma unroll
+          for (int c = 0; c < kSwN / 32; ++c) res[c] = make_float4(0.f, 0.f, 0.f, 0.f);
+          for (int p = 0; p < r.nparts; ++p) {
+            const long long cp = c0 + p;
+            const int slot = (int)(2 * cp + (sp.first(cp) >= r.item * KS ? 0 : 1));
+            const float4* src =
+                reinterpret_cast<const float4*>(a.ws + (size_t)slot * kSwSlotFloats + (size_t)ti * kSwN + 4 * l8);
+            float4 pv[kSwN / 32];
+#pragma unroll
+            for (int c = 0; c < kSwN / 32; ++c) pv[c] = mine ? __ldcg(src + 8 * c) : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+            for (int c = 0; c < kSwN / 32; ++c) add4(res[c], pv[c]);
+          }
+        }
+      }
+      if (fin && quad) {
+        int pr = 0;
+        if (mine) {
+          pr = __ldcg(a.pair_ids + r.tok + ti);
+          if (pr < 0 || pr >= a.n_pairs) pr = 0;
+        }
+        if (kGU) {
+          // h rows rt*128 + 32c + 4*l8 .. +3: gate in chunk c, up in chunk c + 4
+          const int KCn = a.out_rows / kMxKChunk;
+          uint8_t* chunk = a.next_bsf + ((size_t)r.tok * KCn + r.rt) * kMxChunkBytes;
+          const size_t pos = (size_t)r.tok + ti;
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            const float4 g4 = res[c], u4 = res[c + 4];
+            float hv[4] = {g4.x / (1.0f + expf(-g4.x)) * u4.x, g4.y / (1.0f + expf(-g4.y)) * u4.y,
+                           g4.z / (1.0f + expf(-g4.z)) * u4.z, g4.w / (1.0f + expf(-g4.w)) * u4.w};
+            const int row = r.rt * kMxRows + 32 * c + 4 * l8;
+            if (mine && a.h)
+              *reinterpret_cast<float4*>(a.h + (size_t)pr * a.out_rows + row) = make_float4(hv[0], hv[1], hv[2], hv[3]);
+#pragma unroll
+            for (int t = 0; t < kTerms; ++t) {
+              const float am = group_amax(fmaxf(fmaxf(fabsf(hv[0]), fabsf(hv[1])), fmaxf(fabsf(hv[2]), fabsf(hv[3]))));
+              const int e = mx_scale_exp(am);
+              uint32_t packed = 0;
+#pragma unroll
+              for (int j = 0; j < 4; ++j) {
+                const uint32_t cd = f32_to_e2m1(hv[j] * pow2_exact(-e));
+                hv[j] -= e2m1_to_f32(cd) * pow2_exact(e);
+                packed |= cd << (4 * j);
+              }
+              if (mine) {
+                *reinterpret_cast<uint16_t*>(a.next_aq + (pos * kSwRowsPerTok + t) * (a.out_rows / 2) + row / 2) =
+                    (uint16_t)packed;
+                if (l8 == 0) chunk[sf_chunk_byte(ti * kSwRowsPerTok + t, c)] = (uint8_t)(e + 127);
+              }
+            }
+          }
+        } else if (mine) {
+          float4* dst = reinterpret_cast<float4*>(a.y + (size_t)pr * a.out_rows + r.rt * kSwN + 4 * l8);
+#pragma unroll
+          for (int c = 0; c < kSwN / 32; ++c) dst[8 * c] = res[c];
+        }
+      }
+      if (!kGU && fin && a.comb_w && r.last_pass) {
+        // the item is complete: count it for its row tile; the last expert to
+        // arrive combines the tile's rows for every token
         if (!epi_sync()) break;  // the four epilogue warps' y stores, performed CTA-wide
         if (warp == 2 && lane == 0) {
           fence_acq_rel_gpu();
-          const int prev = atomicAdd(&a.tile_counter[u.rt], 1);
+          const int prev = atomicAdd(&a.tile_counter[r.rt], 1);
           const bool last = prev == n_groups - 1;
           if (last) {
             fence_acq_rel_gpu();
-            a.tile_counter[u.rt] = 0;
+            a.tile_counter[r.rt] = 0;
           }
           *s_last = last ? 1 : 0;
         }
         if (!epi_sync()) break;
         if (*s_last) {
-          const int H = a.out_rows;
+          const int H = a.out_rows, row0 = r.rt * kSwN;
           for (int bb = 0; bb < a.batch; ++bb) {
             a.out_bf16[(size_t)bb * H + row0 + et] =
                 combine_elem(a.residual, a.y_shared, a.comb_w, a.top_k, a.y, H, bb, row0 + et);
@@ -1053,8 +1251,8 @@ __global__ void __launch_bounds__(kMxThreads, 1)
                 combine_elem(a.residual, a.y_shared, a.comb_w, a.top_k, a.y, H, bb, row0 + 128 + et);
           }
         }
-        if (!epi_sync()) break;
       }
+      if (!epi_sync()) break;  // s_last and the workspace slots are reused by the next run
     }
   }
   __syncwarp();

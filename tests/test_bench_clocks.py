@@ -126,7 +126,8 @@ def test_launches_per_step(path, want):
     """Router + shared down + the routed experts' kernels of each path (the
     path itself comes from moe_layer_expert_path)."""
     for cfg_id in (1, 2, 3):
-        extra = 1 if path == 2 and synth.CONFIGS[cfg_id].batch > 1 else 0   # the routing finish launch
+        b = synth.CONFIGS[cfg_id].batch
+        extra = (1 if path == 2 and b > 1 else 0) + (1 if path == 2 and b > 2 else 0)  # routing finish, combine
         want_c = want + extra
         assert bench.launches_per_step(synth.CONFIGS[cfg_id], path) == want_c
         assert bench.launches_per_step(synth.CONFIGS[cfg_id].with_(shared_inter=0), path) == want_c - 1
