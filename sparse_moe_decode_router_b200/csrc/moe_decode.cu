@@ -283,7 +283,7 @@ struct moe_layer {
   CUtensorMap tm_agu{}, tm_adn{}, tm_bx{}, tm_bh{}, tm_bx8{}, tm_bh8{};
   bool swap = false;        // both projections take the swapped-operand kernels (H a multiple of 256)
   float* sw_ws = nullptr;   // their stream-K partial sums [num_sms][2][16 x 256]
-  int* sw_cnt = nullptr;    // ... and per-item part counters [E * max(I/128, H/256)]
+  int* sw_cnt = nullptr;    // ... and per-unit part counters [(E + B*k/16 + 1) * max(I/128, H/256)]
   uint8_t* aqx = nullptr;   // E2M1 terms of x per pair position [MB*k*T][H/2]
   uint8_t* bsfx = nullptr;  // ... their scales, chunk layout [MB*k][H/128][512]
   uint8_t* aqh = nullptr;   // E2M1 terms of h [MB*k*T][I/2]
@@ -606,19 +606,19 @@ SwArgs sw_args(const moe_layer* L, bool gate_up, int B, const moe_routing& r) {
   a.pair_ids = r.pair_ids;
   a.asf = gate_up ? L->bsfx : L->bsfh;
   a.tpp = sw_tokens_per_pass(B);
-  a.split = B <= kSwTokMax ? 1 : 0;  // one pass per expert
+  a.one_pass = B <= a.tpp ? 1 : 0;  // an expert holds at most B tokens
   a.off_w = (int)align_up((size_t)a.tpp * kSwRowsPerTok * 128, 1024);
   a.off_sfa = a.off_w + 2 * kMxATile;
   a.off_sfw = a.off_sfa + 2 * kMxChunkBytes;
   a.stage_bytes = (int)align_up((size_t)a.off_sfw + 4 * kMxChunkBytes, 1024);
-  a.n_stages = std::min(kSwMaxStages, (kSmemBudget - 2 * kMxHeaderBytes) / a.stage_bytes);
+  a.n_stages = std::min(kSwMaxStages, (kSmemBudget - 2 * kMxHeaderBytes - kSwTableBytes) / a.stage_bytes);
   a.ws = L->sw_ws;
   a.item_cnt = L->sw_cnt;
   a.err = L->err;
   return a;
 }
 
-int sw_smem(const SwArgs& a) { return 2 * kMxHeaderBytes + a.n_stages * a.stage_bytes; }
+int sw_smem(const SwArgs& a) { return 2 * kMxHeaderBytes + kSwTableBytes + a.n_stages * a.stage_bytes; }
 
 // gate/up on the tensor cores: x -> E2M1 terms per pair position, then the
 // block-scaled MMA kernel (h fp32 into `h`, and h's terms for the down kernel)
@@ -638,7 +638,8 @@ cudaError_t launch_mx_gate_up(moe_layer* L, const void* x, int B, const moe_rout
   if (L->swap) {
     SwArgs a = sw_args(L, true, B, r);
     a.a_by_token = by_token;
-    a.h = h;
+    a.h = nullptr;  // on this path the down projection reads h's terms only
+    (void)h;
     a.next_aq = L->aqh;
     a.next_bsf = L->bsfh;
     if (ev0 && (e = cudaEventRecord(ev0, st)) != cudaSuccess) return e;
@@ -1219,7 +1220,8 @@ moe_status_t moe_layer_create(const moe_layer_config* cfg, const moe_layer_weigh
   const size_t o_aqh = take((size_t)MB * k * kSwRowsPerTok * (I / 2));  // 8 rows per position (>= kMxTerms)
   const size_t o_sfh = take((size_t)MB * k * ((I + kMxKChunk - 1) / kMxKChunk) * kMxChunkBytes);
   const size_t o_sww = take((size_t)sms * 2 * kSwSlotFloats * 4);
-  const size_t o_swc = take((size_t)E * std::max(I / kMxRows, H / kSwN + 1) * 4);
+  // units of the swapped kernels: passes over all groups (<= E + B*k/16) x items per expert
+  const size_t o_swc = take((size_t)(E + MB * k / kSwTokMax + 1) * std::max(I / kMxRows, H / kSwN + 1) * 4);
   if (g_fail_next_alloc.exchange(false) || cudaMalloc(&L->arena, off) != cudaSuccess) {
     cudaGetLastError();
     delete L;

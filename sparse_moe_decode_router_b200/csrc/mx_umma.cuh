@@ -766,6 +766,10 @@ constexpr int kSwN = 256;                           // weight rows per MMA (two 
 constexpr int kSwSfColsStage = 24;                  // activations 2 chunks x 4 + weights 2 chunks x 8
 constexpr int kSwMaxStages = (kMxTmemCols - kSwN) / kSwSfColsStage;  // 10
 constexpr int kSwSlotFloats = kSwTokMax * kSwN;     // one workspace slot: a part's sums for a pass
+constexpr int kSwGrpMax = 64;                       // groups a CTA keeps in its table
+constexpr int kSwPrefBytes = 2 * (kMaxExperts + 8);  // pass prefix (16-bit: at most E + B*k/16 passes)
+constexpr int kSwStageOut = 4 * kMxTerms * 64;       // gate/up epilogue warp: 4 tokens x terms x 64 bytes of h
+constexpr int kSwTableBytes = kSwPrefBytes + 16 * kSwGrpMax + 4 * kSwStageOut;
 static_assert(kMxHeaderBytes >= 8 * (2 * kSwMaxStages + 6) + 32, "header");
 
 struct SwArgs {
@@ -783,10 +787,10 @@ struct SwArgs {
   const uint8_t* asf;       // activation scale chunks [pass-start position][K/128][512], row m = 8*i + t
   int a_by_token;           // batch-1 gate/up: every position reads row set 0 and chunk 0 (the token)
   int tpp;                  // tokens per pass (<= kSwTokMax)
-  int split;                // 1: stream-K over (item, stage); needs every expert's tokens in one pass
+  int one_pass;             // 1: every expert's tokens fit one pass (batch <= tpp): no pass prefix
   int n_stages, stage_bytes, off_w, off_sfa, off_sfw;  // the activation rows sit at offset 0 of a stage
   float* ws;                // stream-K partial sums: [grid][2 slots][kSwSlotFloats]
-  int* item_cnt;            // [n_experts * n_rt], zero between launches
+  int* item_cnt;            // per unit: pieces arrived, zero between launches
   // gate/up
   float* h;                 // h fp32 [pair][I], or null
   uint8_t* next_aq;         // h's E2M1 terms [pos*8 + t][I/2]
@@ -804,7 +808,31 @@ struct SwArgs {
   int* err;
 };
 
-// the launch's work list in K-stage units: stage it of item it / KS
+// (expert, first position, tokens) of active group g, checked against the plan
+template <typename Args>
+__device__ __forceinline__ int3 sw_group_entry(const Args& a, int g) {
+  int e = __ldcg(a.active + g);
+  if (e < 0 || e >= a.n_experts) e = 0;
+  int tok0 = __ldcg(a.offsets + e);
+  int cnt = __ldcg(a.offsets + e + 1) - tok0;
+  if (tok0 < 0 || cnt < 1 || tok0 + cnt > a.n_pairs) {
+    tok0 = 0;
+    cnt = 1;
+  }
+  return make_int3(e, tok0, cnt);
+}
+
+// the group whose passes hold global pass gp: the largest g with pref[g] <= gp
+__device__ __forceinline__ int sw_group_of_pass(const uint16_t* pref, int n_groups, int gp) {
+  int lo = 0, hi = n_groups - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (pref[mid] <= gp) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
+// the launch's work list in K-stage units: stage it of unit it / KS
 struct SwSplit {
   long long T, G;  // stages of the list; CTAs that take a stretch (the others have none)
   __device__ long long first(long long c) const { return c >= G ? T : c * T / G; }
@@ -814,56 +842,66 @@ struct SwSplit {
 
 struct SwRun {
   int e, rt, tok, ntok;  // expert, item within the expert, first position and tokens of the pass
-  long long item;        // item index in the launch's list
+  long long unit;        // unit index in the launch's list
   int k0, nk;            // first K stage and stages of the run
-  int part, nparts;      // this run's piece of the item (stream-K), and the item's pieces
-  bool last_pass;
+  int part, nparts;      // this run's piece of the unit (stream-K), and the unit's pieces
 };
 
+// The launch's units are (active group, pass of tpp tokens, item): unit
+// gp*n_rt + rt for the gp-th pass over all groups (a group's passes are
+// consecutive).  pref[g] is the first pass of group g (null when every group
+// has one pass); a CTA keeps (expert, first position, tokens) of the groups
+// its stretch touches in shared memory (grp, from group g_first), so the
+// walk makes no global loads.
 struct SwWalk {
   const SwArgs& a;
   const SwSplit& sp;
-  long long it, hi, item;
-  int KS, pass, npass, e, tok0, cnt;
-  __device__ SwWalk(const SwArgs& args, const SwSplit& split, long long lo, long long hi_, int ks)
-      : a(args), sp(split), it(lo), hi(hi_), item(0), KS(ks), pass(0), npass(0), e(0), tok0(0), cnt(0) {
+  const uint16_t* pref;
+  const int4* grp;
+  long long it, hi, unit;
+  int KS, n_groups, g_first, n_tab, pass, e, tok0, cnt;
+  __device__ SwWalk(const SwArgs& args, const SwSplit& split, const uint16_t* pref_, const int4* grp_, int n_groups_,
+                    int g_first_, int n_tab_, long long lo, long long hi_, int ks)
+      : a(args), sp(split), pref(pref_), grp(grp_), it(lo), hi(hi_), unit(0), KS(ks), n_groups(n_groups_),
+        g_first(g_first_), n_tab(n_tab_), pass(0), e(0), tok0(0), cnt(0) {
     if (it < hi) load();
   }
   __device__ void load() {
-    item = it / KS;
-    const int g = (int)(item / a.n_rt);
-    e = __ldcg(a.active + g);
-    if (e < 0 || e >= a.n_experts) e = 0;
-    tok0 = __ldcg(a.offsets + e);
-    cnt = __ldcg(a.offsets + e + 1) - tok0;
-    if (tok0 < 0 || cnt < 1 || tok0 + cnt > a.n_pairs) { tok0 = 0; cnt = 1; }
-    npass = a.split ? 1 : (cnt + a.tpp - 1) / a.tpp;
-    pass = 0;
+    unit = it / KS;
+    const int gp = (int)(unit / a.n_rt);
+    int g = gp;
+    if (pref) g = sw_group_of_pass(pref, n_groups, gp);
+    pass = pref ? gp - pref[g] : 0;
+    const int j = g - g_first;
+    if (j >= 0 && j < n_tab) {
+      const int4 t = grp[j];
+      e = t.x;
+      tok0 = t.y;
+      cnt = t.z;
+    } else {
+      const int3 t = sw_group_entry(a, g);
+      e = t.x;
+      tok0 = t.y;
+      cnt = t.z;
+    }
   }
   __device__ bool valid() const { return it < hi; }
   __device__ SwRun run() const {
     SwRun r;
     r.e = e;
-    r.item = item;
-    r.rt = (int)(item % a.n_rt);
+    r.unit = unit;
+    r.rt = (int)(unit % a.n_rt);
     r.tok = tok0 + pass * a.tpp;
-    r.ntok = min(a.tpp, cnt - pass * a.tpp);
-    r.k0 = (int)(it - item * KS);
-    r.nk = (int)(min(hi, (item + 1) * KS) - it);
-    if (a.split) {
-      const long long c0 = sp.owner(item * KS);
-      r.part = (int)(sp.owner(it) - c0);
-      r.nparts = (int)(sp.owner((item + 1) * KS - 1) - c0 + 1);
-    } else {
-      r.part = 0;
-      r.nparts = 1;
-    }
-    r.last_pass = pass == npass - 1;
+    r.ntok = max(1, min(a.tpp, cnt - pass * a.tpp));
+    r.k0 = (int)(it - unit * KS);
+    r.nk = (int)(min(hi, (unit + 1) * KS) - it);
+    const long long c0 = sp.owner(unit * KS);
+    r.part = (int)(sp.owner(it) - c0);
+    r.nparts = (int)(sp.owner((unit + 1) * KS - 1) - c0 + 1);
     return r;
   }
   __device__ void next() {
-    if (++pass < npass) return;
-    it = min(hi, (item + 1) * KS);
+    it = min(hi, (unit + 1) * KS);
     if (it < hi) load();
   }
 };
@@ -922,7 +960,10 @@ __global__ void __launch_bounds__(kMxThreads, 1)
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const uint32_t raw = smem_addr(smem_raw);
   unsigned char* hdr = smem_raw;
-  unsigned char* ring = smem_raw + (((raw + kMxHeaderBytes + 1023u) & ~1023u) - raw);
+  unsigned char* ring = smem_raw + (((raw + kMxHeaderBytes + kSwTableBytes + 1023u) & ~1023u) - raw);
+  uint16_t* s_pref = reinterpret_cast<uint16_t*>(hdr + kMxHeaderBytes);              // [n_groups + 1]
+  int4* s_grp = reinterpret_cast<int4*>(hdr + kMxHeaderBytes + kSwPrefBytes);          // [kSwGrpMax]
+  unsigned char* s_out = hdr + kMxHeaderBytes + kSwPrefBytes + 16 * kSwGrpMax;        // [4 warps][kSwStageOut]
   uint64_t* full_bar = reinterpret_cast<uint64_t*>(hdr);
   uint64_t* empty_bar = full_bar + kSwMaxStages;
   uint64_t* acc_full = empty_bar + kSwMaxStages;
@@ -958,34 +999,77 @@ __global__ void __launch_bounds__(kMxThreads, 1)
     tma_prefetch_desc(&tmW);
     tma_prefetch_desc(&tmA);
   }
-  pdl_wait();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *s_tmem;
 
+  // The routing plan is complete before this grid starts: the kernel before
+  // (the activation terms, or gate/up for the down projection) waited for its
+  // producer before letting this grid launch.  So the plan, the partition and
+  // the first stages' weights (static) are read before the wait for the
+  // preceding kernel; the activations and every output follow it.
   int n_groups = __ldcg(a.n_active);
   if (n_groups < 0 || n_groups > a.n_experts) {
     if (tid == 0) atomicExch(a.err, kErrBadPlan);
     n_groups = n_groups < 0 ? 0 : a.n_experts;
   }
-  const long long n_items = (long long)n_groups * a.n_rt;
-  SwSplit sp;
-  long long lo, hi;
-  if (a.split) {
-    sp.T = n_items * KS;
-    sp.G = max(1ll, min((long long)gridDim.x, sp.T / 2));
-    lo = sp.first(blockIdx.x);
-    hi = sp.first(blockIdx.x + 1);
-  } else {
-    sp.T = n_items * KS;
-    sp.G = gridDim.x;
-    lo = n_items * blockIdx.x / gridDim.x * KS;
-    hi = n_items * (blockIdx.x + 1) / gridDim.x * KS;
+  // passes of the groups: prefix over the active list (one block scan), unless
+  // every group has one pass
+  const uint16_t* pref = nullptr;
+  int n_gp = n_groups;  // passes over all groups
+  if (!a.one_pass && n_groups > 0) {
+    const int nt = blockDim.x, per = (n_groups + nt - 1) / nt;
+    const int g0 = min(n_groups, tid * per), g1 = min(n_groups, g0 + per);
+    int c = 0;
+    for (int g = g0; g < g1; ++g) {
+      const int np = (sw_group_entry(a, g).z + a.tpp - 1) / a.tpp;
+      s_pref[g] = (uint16_t)np;  // this thread's own entries: passes, then their prefix below
+      c += np;
+    }
+    int inc = c;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xFFFFFFFFu, inc, o);
+      if (lane >= o) inc += v;
+    }
+    int* s_wsum = reinterpret_cast<int*>(s_grp);  // scratch until the table is written
+    if (lane == 31) s_wsum[warp] = inc;
+    __syncthreads();
+    int base = 0;
+    for (int w2 = 0; w2 < warp; ++w2) base += s_wsum[w2];
+    int run = base + inc - c;
+    for (int g = g0; g < g1; ++g) {
+      const int np = s_pref[g];
+      s_pref[g] = (uint16_t)run;
+      run += np;
+    }
+    if (g0 < n_groups && g1 == n_groups) s_pref[n_groups] = (uint16_t)run;
+    __syncthreads();
+    n_gp = s_pref[n_groups];
+    pref = s_pref;
   }
+  const long long n_units = (long long)n_gp * a.n_rt;
+  SwSplit sp;
+  sp.T = n_units * KS;
+  sp.G = max(1ll, min((long long)gridDim.x, sp.T / 2));
+  const long long lo = sp.first(blockIdx.x), hi = sp.first(blockIdx.x + 1);
+  // the groups of this CTA's stretch, in shared memory
+  int g_first = 0, n_tab = 0;
+  if (lo < hi) {
+    const int gp0 = (int)(lo / KS / a.n_rt), gp1 = (int)((hi - 1) / KS / a.n_rt);
+    g_first = pref ? sw_group_of_pass(pref, n_groups, gp0) : gp0;
+    const int g_last = pref ? sw_group_of_pass(pref, n_groups, gp1) : gp1;
+    n_tab = min(kSwGrpMax, g_last - g_first + 1);
+    for (int j = tid; j < n_tab; j += blockDim.x) {
+      const int3 t = sw_group_entry(a, g_first + j);
+      s_grp[j] = make_int4(t.x, t.y, t.z, 0);
+    }
+  }
+  __syncthreads();
   const bool plan_ok = ns >= 1 && ns <= kSwMaxStages && (K % kMxKChunk) == 0 && a.n_rt >= 1 && a.tpp >= 1 &&
                        a.tpp <= kSwTokMax && a.off_w >= a.tpp * kSwRowsPerTok * 128 &&
-                       a.off_w + 2 * kMxATile >= kMxRows * 128 && (!a.split || gridDim.x <= 4096);
+                       a.off_w + 2 * kMxATile >= kMxRows * 128;
   if (!plan_ok && tid == 0) atomicExch(a.err, kErrBadPlan);
   const long long lim_long = 1ll << 31, lim_short = 1ll << 20;
   const int step = kGU ? 1 : 2;  // weight tiles per item along the expert's rows
@@ -994,9 +1078,35 @@ __global__ void __launch_bounds__(kMxThreads, 1)
     // ------------------------------ TMA producer ------------------------------
     if (lane == 0) {
       const uint64_t pol = l2_policy_evict_first();
+      // the first stages' weight tiles and scales before the wait
+      const long long npf = min((long long)ns, hi - lo);
+      {
+        int s = 0;
+        long long q = 0;
+        for (SwWalk w(a, sp, pref, s_grp, n_groups, g_first, n_tab, lo, hi, KS); w.valid() && q < npf; w.next()) {
+          const SwRun r = w.run();
+          const long long tile0 = (long long)r.e * a.a_tiles + (long long)step * r.rt;
+          const long long tile1 = tile0 + a.tile2;
+          for (int kt = r.k0; kt < r.k0 + r.nk && q < npf; ++kt, ++q, ++s) {
+            const int nck = min(2, KC - 2 * kt);
+            const uint32_t cb = (uint32_t)(nck * kMxChunkBytes);
+            unsigned char* st = ring + (size_t)s * a.stage_bytes;
+            const uint32_t sa = smem_addr(st);
+            mbar_arrive_expect_tx(&full_bar[s], (uint32_t)r.ntok * (kSwRowsPerTok * 128u) + 2u * kMxATile + 3u * cb);
+            tma_load_2d(sa + a.off_w, &tmW, kt * 128, (int)(tile0 * kMxRows), &full_bar[s], pol);
+            tma_load_2d(sa + a.off_w + kMxATile, &tmW, kt * 128, (int)(tile1 * kMxRows), &full_bar[s], pol);
+            const size_t ck = (size_t)2 * kt * kMxChunkBytes;
+            bulk_g2s(st + a.off_sfw, a.wsf + tile0 * KC * kMxChunkBytes + ck, cb, &full_bar[s], pol);
+            bulk_g2s(st + a.off_sfw + 2 * kMxChunkBytes, a.wsf + tile1 * KC * kMxChunkBytes + ck, cb, &full_bar[s],
+                     pol);
+          }
+        }
+      }
+      pdl_wait();
       int s = 0;
       uint32_t ph = 0;
-      for (SwWalk w(a, sp, lo, hi, KS); w.valid() && !*s_abort; w.next()) {
+      long long q = 0;  // stage counter of this CTA
+      for (SwWalk w(a, sp, pref, s_grp, n_groups, g_first, n_tab, lo, hi, KS); w.valid() && !*s_abort; w.next()) {
         const SwRun r = w.run();
         const long long tile0 = (long long)r.e * a.a_tiles + (long long)step * r.rt;
         const long long tile1 = tile0 + a.tile2;
@@ -1004,26 +1114,29 @@ __global__ void __launch_bounds__(kMxThreads, 1)
         const uint8_t* sfw1 = a.wsf + tile1 * KC * kMxChunkBytes;
         const int arow = a.a_by_token ? 0 : r.tok;
         const uint8_t* sfa = a.asf + (size_t)arow * KC * kMxChunkBytes;
-        for (int kt = r.k0; kt < r.k0 + r.nk; ++kt) {
-          if (!mbar_wait_bounded(&empty_bar[s], ph ^ 1u, *s_abort ? lim_short : lim_long)) {
-            atomicExch(a.err, kErrTimeout);
-            *s_abort = 1;
-            break;
-          }
+        for (int kt = r.k0; kt < r.k0 + r.nk; ++kt, ++q) {
           const int nck = min(2, KC - 2 * kt);
           const uint32_t cb = (uint32_t)(nck * kMxChunkBytes);
           unsigned char* st = ring + (size_t)s * a.stage_bytes;
           const uint32_t sa = smem_addr(st);
-          mbar_arrive_expect_tx(&full_bar[s], (uint32_t)r.ntok * (kSwRowsPerTok * 128u) + 2u * kMxATile + 3u * cb);
+          const size_t ck = (size_t)2 * kt * kMxChunkBytes;
+          if (q >= npf) {
+            if (!mbar_wait_bounded(&empty_bar[s], ph ^ 1u, *s_abort ? lim_short : lim_long)) {
+              atomicExch(a.err, kErrTimeout);
+              *s_abort = 1;
+              break;
+            }
+            mbar_arrive_expect_tx(&full_bar[s], (uint32_t)r.ntok * (kSwRowsPerTok * 128u) + 2u * kMxATile + 3u * cb);
+            tma_load_2d(sa + a.off_w, &tmW, kt * 128, (int)(tile0 * kMxRows), &full_bar[s], pol);
+            tma_load_2d(sa + a.off_w + kMxATile, &tmW, kt * 128, (int)(tile1 * kMxRows), &full_bar[s], pol);
+            bulk_g2s(st + a.off_sfw, sfw0 + ck, cb, &full_bar[s], pol);
+            bulk_g2s(st + a.off_sfw + 2 * kMxChunkBytes, sfw1 + ck, cb, &full_bar[s], pol);
+          }
+          // the activation rows and their scales: written by the preceding kernel
           for (int i = 0; i < r.ntok; ++i)
             tma_load_2d_nohint(sa + i * kSwRowsPerTok * 128, &tmA, kt * 128,
                                (a.a_by_token ? 0 : r.tok + i) * kSwRowsPerTok, &full_bar[s]);
-          tma_load_2d(sa + a.off_w, &tmW, kt * 128, (int)(tile0 * kMxRows), &full_bar[s], pol);
-          tma_load_2d(sa + a.off_w + kMxATile, &tmW, kt * 128, (int)(tile1 * kMxRows), &full_bar[s], pol);
-          const size_t ck = (size_t)2 * kt * kMxChunkBytes;
           bulk_g2s_nohint(st + a.off_sfa, sfa + ck, cb, &full_bar[s]);
-          bulk_g2s(st + a.off_sfw, sfw0 + ck, cb, &full_bar[s], pol);
-          bulk_g2s(st + a.off_sfw + 2 * kMxChunkBytes, sfw1 + ck, cb, &full_bar[s], pol);
           if (++s == ns) { s = 0; ph ^= 1u; }
         }
       }
@@ -1046,11 +1159,12 @@ __global__ void __launch_bounds__(kMxThreads, 1)
     }
   } else if (plan_ok && warp == 1) {
     // ------------------------------ MMA issuer --------------------------------
+    pdl_wait();
     if (lane == 0) {
       int s = 0, uc = 0;
       uint32_t ph = 0;
       const uint32_t idesc = mx_idesc(kSwN);
-      for (SwWalk w(a, sp, lo, hi, KS); w.valid() && !*s_abort; w.next(), ++uc) {
+      for (SwWalk w(a, sp, pref, s_grp, n_groups, g_first, n_tab, lo, hi, KS); w.valid() && !*s_abort; w.next(), ++uc) {
         const SwRun r = w.run();
         if (!mbar_wait_bounded(acc_empty, ((uint32_t)uc & 1u) ^ 1u, lim_long)) {
           atomicExch(a.err, kErrTimeout);
@@ -1096,6 +1210,7 @@ __global__ void __launch_bounds__(kMxThreads, 1)
     __syncwarp();
   } else if (plan_ok && warp >= 2) {
     // ------------------------------ epilogue ----------------------------------
+    pdl_wait();  // outputs (and the workspace) are written after the preceding kernel
     const int q = warp & 3;
     const uint32_t lane_base = tmem + ((uint32_t)(32 * q) << 16);
     const int l8 = lane & 7, ti = 4 * q + (lane >> 3);  // term (and column quarter), token of the pass
@@ -1114,8 +1229,11 @@ __global__ void __launch_bounds__(kMxThreads, 1)
       }
       return ok;
     };
-    for (SwWalk w(a, sp, lo, hi, KS); w.valid(); w.next(), ++uc) {
+    for (SwWalk w(a, sp, pref, s_grp, n_groups, g_first, n_tab, lo, hi, KS); w.valid(); w.next(), ++uc) {
       const SwRun r = w.run();
+      // the lane's pair, loaded while the MMAs run
+      int pr = 0;
+      if (ti < r.ntok) pr = __ldcg(a.pair_ids + r.tok + ti);
       bool ok = !*s_abort && mbar_wait_bounded(acc_full, (uint32_t)uc & 1u, lim_long);
       ok = __all_sync(0xFFFFFFFFu, ok);
       if (!ok) {
@@ -1128,16 +1246,21 @@ __global__ void __launch_bounds__(kMxThreads, 1)
       const bool mine = ti < r.ntok;
       float4 res[kSwN / 32];
       if (quad) {
+        // a rolled loop (the epilogue shares the SM with the other roles'
+        // code); the results shift down so every index stays static
         float v[32];
         tc_ld32(lane_base, v);
-#pragma unroll
+#pragma unroll 1
         for (int c = 0; c < kSwN / 32; ++c) {
           tc_wait_ld();
           float cur[32];
 #pragma unroll
           for (int i = 0; i < 32; ++i) cur[i] = l8 < kTerms ? v[i] : 0.f;
           if (c + 1 < kSwN / 32) tc_ld32(lane_base + (uint32_t)(32 * (c + 1)), v);
-          res[c] = group_reduce_scatter(cur, l8);
+          const float4 r4 = group_reduce_scatter(cur, l8);
+#pragma unroll
+          for (int j = 0; j + 1 < kSwN / 32; ++j) res[j] = res[j + 1];
+          res[kSwN / 32 - 1] = r4;
         }
       }
       tc_fence_before();
@@ -1147,7 +1270,7 @@ __global__ void __launch_bounds__(kMxThreads, 1)
       if (r.nparts > 1) {
         // a piece of a split item: its sums to the CTA's slot, then the count
         const long long c_me = blockIdx.x;
-        const int my_slot = (int)(2 * c_me + (sp.first(c_me) >= r.item * KS ? 0 : 1));
+        const int my_slot = (int)(2 * c_me + (sp.first(c_me) >= r.unit * KS ? 0 : 1));
         if (quad && mine) {
           float4* dst = reinterpret_cast<float4*>(a.ws + (size_t)my_slot * kSwSlotFloats + (size_t)ti * kSwN + 4 * l8);
 #pragma unroll
@@ -1156,11 +1279,11 @@ __global__ void __launch_bounds__(kMxThreads, 1)
         if (!epi_sync()) break;
         if (warp == 2 && lane == 0) {
           fence_acq_rel_gpu();
-          const int prev = atomicAdd(&a.item_cnt[r.item], 1);
+          const int prev = atomicAdd(&a.item_cnt[r.unit], 1);
           const bool last = prev == r.nparts - 1;
           if (last) {
             fence_acq_rel_gpu();
-            a.item_cnt[r.item] = 0;
+            a.item_cnt[r.unit] = 0;
           }
           *s_last = last ? 1 : 0;
         }
@@ -1168,12 +1291,12 @@ __global__ void __launch_bounds__(kMxThreads, 1)
         fin = *s_last != 0;
         if (fin && quad) {
           // every piece, ascending K order
-          const long long c0 = sp.owner(r.item * KS);
+          const long long c0 = sp.owner(r.unit * KS);
 #pragma unroll
           for (int c = 0; c < kSwN / 32; ++c) res[c] = make_float4(0.f, 0.f, 0.f, 0.f);
           for (int p = 0; p < r.nparts; ++p) {
             const long long cp = c0 + p;
-            const int slot = (int)(2 * cp + (sp.first(cp) >= r.item * KS ? 0 : 1));
+            const int slot = (int)(2 * cp + (sp.first(cp) >= r.unit * KS ? 0 : 1));
             const float4* src =
                 reinterpret_cast<const float4*>(a.ws + (size_t)slot * kSwSlotFloats + (size_t)ti * kSwN + 4 * l8);
             float4 pv[kSwN / 32];
@@ -1185,24 +1308,32 @@ __global__ void __launch_bounds__(kMxThreads, 1)
         }
       }
       if (fin && quad) {
-        int pr = 0;
-        if (mine) {
-          pr = __ldcg(a.pair_ids + r.tok + ti);
-          if (pr < 0 || pr >= a.n_pairs) pr = 0;
-        }
+        if (pr < 0 || pr >= a.n_pairs) pr = 0;
         if (kGU) {
-          // h rows rt*128 + 32c + 4*l8 .. +3: gate in chunk c, up in chunk c + 4
-          const int KCn = a.out_rows / kMxKChunk;
-          uint8_t* chunk = a.next_bsf + ((size_t)r.tok * KCn + r.rt) * kMxChunkBytes;
-          const size_t pos = (size_t)r.tok + ti;
+          // h rows rt*128 + 32c + 4*l8 .. +3: gate in chunk c, up in chunk c + 4.
+          // The packed terms go through this warp's staging bytes ([token of
+          // the warp][term][64 bytes = the item's 128 rows]) and out as
+          // 16-byte stores; the four block scales of a (token, term) are one
+          // 32-bit word of the pass's chunk.
+          unsigned char* stg = s_out + (warp - 2) * kSwStageOut;
+          const int lg = lane >> 3;
+          uint32_t sfw[kTerms];
 #pragma unroll
+          for (int t = 0; t < kTerms; ++t) sfw[t] = 0u;
+#pragma unroll 1
           for (int c = 0; c < 4; ++c) {
-            const float4 g4 = res[c], u4 = res[c + 4];
+            // chunk c sits at res[0] (gate) and res[4] (up): the chunks shift down after each pass
+            const float4 g4 = res[0], u4 = res[4];
+#pragma unroll
+            for (int j = 0; j < 3; ++j) {
+              res[j] = res[j + 1];
+              res[4 + j] = res[5 + j];
+            }
             float hv[4] = {g4.x / (1.0f + expf(-g4.x)) * u4.x, g4.y / (1.0f + expf(-g4.y)) * u4.y,
                            g4.z / (1.0f + expf(-g4.z)) * u4.z, g4.w / (1.0f + expf(-g4.w)) * u4.w};
-            const int row = r.rt * kMxRows + 32 * c + 4 * l8;
             if (mine && a.h)
-              *reinterpret_cast<float4*>(a.h + (size_t)pr * a.out_rows + row) = make_float4(hv[0], hv[1], hv[2], hv[3]);
+              *reinterpret_cast<float4*>(a.h + (size_t)pr * a.out_rows + r.rt * kMxRows + 32 * c + 4 * l8) =
+                  make_float4(hv[0], hv[1], hv[2], hv[3]);
 #pragma unroll
             for (int t = 0; t < kTerms; ++t) {
               const float am = group_amax(fmaxf(fmaxf(fabsf(hv[0]), fabsf(hv[1])), fmaxf(fabsf(hv[2]), fabsf(hv[3]))));
@@ -1214,27 +1345,43 @@ __global__ void __launch_bounds__(kMxThreads, 1)
                 hv[j] -= e2m1_to_f32(cd) * pow2_exact(e);
                 packed |= cd << (4 * j);
               }
-              if (mine) {
-                *reinterpret_cast<uint16_t*>(a.next_aq + (pos * kSwRowsPerTok + t) * (a.out_rows / 2) + row / 2) =
-                    (uint16_t)packed;
-                if (l8 == 0) chunk[sf_chunk_byte(ti * kSwRowsPerTok + t, c)] = (uint8_t)(e + 127);
-              }
+              *reinterpret_cast<uint16_t*>(stg + (lg * kTerms + t) * 64 + 16 * c + 2 * l8) = (uint16_t)packed;
+              sfw[t] |= (uint32_t)(e + 127) << (8 * c);
             }
           }
+          __syncwarp();
+          const int KCn = a.out_rows / kMxKChunk;
+          if (mine && l8 == 0) {
+            uint8_t* chunk = a.next_bsf + ((size_t)r.tok * KCn + r.rt) * kMxChunkBytes;
+#pragma unroll
+            for (int t = 0; t < kTerms; ++t)
+              *reinterpret_cast<uint32_t*>(chunk + sf_chunk_byte(ti * kSwRowsPerTok + t, 0)) = sfw[t];
+          }
+          for (int idx = lane; idx < 4 * kTerms * 4; idx += 32) {
+            const int tg = idx / (kTerms * 4), t = (idx >> 2) % kTerms, part = idx & 3;
+            const int tok_i = 4 * q + tg;  // token of the pass
+            if (tok_i < r.ntok) {
+              const uint4 v = *reinterpret_cast<const uint4*>(stg + (tg * kTerms + t) * 64 + 16 * part);
+              const size_t pos = (size_t)r.tok + tok_i;
+              *reinterpret_cast<uint4*>(a.next_aq + (pos * kSwRowsPerTok + t) * (a.out_rows / 2) + r.rt * 64 +
+                                        16 * part) = v;
+            }
+          }
+          __syncwarp();  // the staging bytes are rewritten by the next run
         } else if (mine) {
           float4* dst = reinterpret_cast<float4*>(a.y + (size_t)pr * a.out_rows + r.rt * kSwN + 4 * l8);
 #pragma unroll
           for (int c = 0; c < kSwN / 32; ++c) dst[8 * c] = res[c];
         }
       }
-      if (!kGU && fin && a.comb_w && r.last_pass) {
-        // the item is complete: count it for its row tile; the last expert to
-        // arrive combines the tile's rows for every token
+      if (!kGU && fin && a.comb_w) {
+        // the unit is complete: count it for its row tile; the last unit (of
+        // all groups and passes) to arrive combines the tile's rows
         if (!epi_sync()) break;  // the four epilogue warps' y stores, performed CTA-wide
         if (warp == 2 && lane == 0) {
           fence_acq_rel_gpu();
           const int prev = atomicAdd(&a.tile_counter[r.rt], 1);
-          const bool last = prev == n_groups - 1;
+          const bool last = prev == n_gp - 1;
           if (last) {
             fence_acq_rel_gpu();
             a.tile_counter[r.rt] = 0;
@@ -1252,9 +1399,11 @@ __global__ void __launch_bounds__(kMxThreads, 1)
           }
         }
       }
-      if (!epi_sync()) break;  // s_last and the workspace slots are reused by the next run
+      if (r.nparts > 1 || (!kGU && fin && a.comb_w))
+        if (!epi_sync()) break;  // s_last is rewritten by the next run
     }
   }
+  if (!plan_ok) pdl_wait();  // no role ran: still complete only after the preceding grid
   __syncwarp();
   tc_fence_before();
   __syncthreads();
