@@ -290,6 +290,10 @@ __global__ void __launch_bounds__(kDnThreads, 1)
         }
       }
     }
+    // every copy of this CTA is issued: the next grid may start its prologue
+    // on SMs as they free up (it waits for this grid before reading its outputs)
+    __syncwarp();
+    pdl_launch_dependents();
   } else {
     // activations (B operand) and the workspace come from the preceding kernels
     pdl_wait();

@@ -1157,6 +1157,10 @@ __global__ void __launch_bounds__(kMxThreads, 1)
         }
       }
     }
+    // every copy of this CTA is issued: the next grid may start its prologue
+    // on SMs as they free up (it waits for this grid before reading its outputs)
+    __syncwarp();
+    pdl_launch_dependents();
   } else if (plan_ok && warp == 1) {
     // ------------------------------ MMA issuer --------------------------------
     pdl_wait();
@@ -1320,29 +1324,41 @@ __global__ void __launch_bounds__(kMxThreads, 1)
           uint32_t sfw[kTerms];
 #pragma unroll
           for (int t = 0; t < kTerms; ++t) sfw[t] = 0u;
-#pragma unroll 1
-          for (int c = 0; c < 4; ++c) {
-            // chunk c sits at res[0] (gate) and res[4] (up): the chunks shift down after each pass
-            const float4 g4 = res[0], u4 = res[4];
+          // h for the four 32-row blocks, then the terms block by block with the
+          // four blocks' (independent) reductions interleaved
+          // (lanes of absent tokens hold whatever the padding rows produced,
+          // possibly Inf or NaN: zeros keep them off the division's slow path)
+          float hv[4][4];
 #pragma unroll
-            for (int j = 0; j < 3; ++j) {
-              res[j] = res[j + 1];
-              res[4 + j] = res[5 + j];
-            }
-            float hv[4] = {g4.x / (1.0f + expf(-g4.x)) * u4.x, g4.y / (1.0f + expf(-g4.y)) * u4.y,
-                           g4.z / (1.0f + expf(-g4.z)) * u4.z, g4.w / (1.0f + expf(-g4.w)) * u4.w};
+          for (int c = 0; c < 4; ++c) {
+            const float4 z4 = make_float4(0.f, 0.f, 0.f, 0.f);
+            const float4 g4 = mine ? res[c] : z4, u4 = mine ? res[c + 4] : z4;
+            hv[c][0] = g4.x / (1.0f + expf(-g4.x)) * u4.x;
+            hv[c][1] = g4.y / (1.0f + expf(-g4.y)) * u4.y;
+            hv[c][2] = g4.z / (1.0f + expf(-g4.z)) * u4.z;
+            hv[c][3] = g4.w / (1.0f + expf(-g4.w)) * u4.w;
             if (mine && a.h)
               *reinterpret_cast<float4*>(a.h + (size_t)pr * a.out_rows + r.rt * kMxRows + 32 * c + 4 * l8) =
-                  make_float4(hv[0], hv[1], hv[2], hv[3]);
+                  make_float4(hv[c][0], hv[c][1], hv[c][2], hv[c][3]);
+          }
 #pragma unroll
-            for (int t = 0; t < kTerms; ++t) {
-              const float am = group_amax(fmaxf(fmaxf(fabsf(hv[0]), fabsf(hv[1])), fmaxf(fabsf(hv[2]), fabsf(hv[3]))));
-              const int e = mx_scale_exp(am);
+          for (int t = 0; t < kTerms; ++t) {
+            float am[4];
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+              am[c] = fmaxf(fmaxf(fabsf(hv[c][0]), fabsf(hv[c][1])), fmaxf(fabsf(hv[c][2]), fabsf(hv[c][3])));
+#pragma unroll
+            for (int o = 1; o < 8; o <<= 1)
+#pragma unroll
+              for (int c = 0; c < 4; ++c) am[c] = fmaxf(am[c], __shfl_xor_sync(0xFFFFFFFFu, am[c], o));
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              const int e = mx_scale_exp(am[c]);
               uint32_t packed = 0;
 #pragma unroll
               for (int j = 0; j < 4; ++j) {
-                const uint32_t cd = f32_to_e2m1(hv[j] * pow2_exact(-e));
-                hv[j] -= e2m1_to_f32(cd) * pow2_exact(e);
+                const uint32_t cd = f32_to_e2m1(hv[c][j] * pow2_exact(-e));
+                hv[c][j] -= e2m1_to_f32(cd) * pow2_exact(e);
                 packed |= cd << (4 * j);
               }
               *reinterpret_cast<uint16_t*>(stg + (lg * kTerms + t) * 64 + 16 * c + 2 * l8) = (uint16_t)packed;
