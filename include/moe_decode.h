@@ -218,11 +218,14 @@ MOE_API moe_status_t moe_combine_residual(moe_layer_t layer, int B, const moe_ro
                                   const void* residual, void* out, void* stream);
 
 /* The whole layer in one call: router/top-k/buckets, shared expert, routed
- * experts, down projection fused with the combine and residual add.  Kernels
- * are chained with programmatic dependent launch on `stream`; the shared
- * expert's gate/up kernel starts while the top-k runs (it needs only x), so
- * it overlaps the routing latency the way the pages' side stream does
- * (MOE_FLAG_SIDE_STREAM forks it onto a side stream instead);
+ * experts, then the combine with the residual add (fused into the down
+ * projection on the CUDA-core path and on the tcgen05 path up to batch 2;
+ * above batch 2 on the tcgen05 path a launch of its own over every SM).
+ * Kernels are chained with programmatic dependent launch on `stream`: at
+ * batch 1 a bf16 shared expert's gate/up rows ride in the router kernel and
+ * its down projection runs beside the routing finish, overlapping the
+ * routing latency the way the pages' side stream does (MOE_FLAG_SIDE_STREAM
+ * forks the shared expert onto a side stream instead);
  * with `next` non-NULL the tail of this layer prefetches next's router and
  * shared-expert weights into L2 (pages: yeyulingfeng section 02, third and
  * fourth optimisations); `next` must live on the same device (else

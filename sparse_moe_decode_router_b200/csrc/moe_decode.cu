@@ -280,7 +280,7 @@ struct moe_layer {
   bool mx = false;         // the shapes allow it and its scale copies exist
   bool mx_forced = false;  // MOE_FLAG_MX_EXPERTS: at every batch size
   bool mx_default = false; // above batch 1 unless MOE_FLAG_NO_GROUPED / MOE_FLAG_WARP_MMA
-  CUtensorMap tm_agu{}, tm_adn{}, tm_bx{}, tm_bh{}, tm_bx8{}, tm_bh8{};
+  CUtensorMap tm_agu{}, tm_adn{}, tm_bx{}, tm_bh{}, tm_bx8{}, tm_bh8{}, tm_bx128{}, tm_bh128{};
   bool swap = false;        // both projections take the swapped-operand kernels (H a multiple of 256)
   float* sw_ws = nullptr;   // their stream-K partial sums [num_sms][2][16 x 256]
   int* sw_cnt = nullptr;    // ... and per-unit part counters [(E + B*k/16 + 1) * max(I/128, H/256)]
@@ -644,7 +644,7 @@ cudaError_t launch_mx_gate_up(moe_layer* L, const void* x, int B, const moe_rout
     a.next_bsf = L->bsfh;
     if (ev0 && (e = cudaEventRecord(ev0, st)) != cudaSuccess) return e;
     e = launch_ex(mx_swap_kernel<true, kMxTerms>, L->num_sms, kMxThreads, sw_smem(a), st, L->pdl, L->tm_agu,
-                  L->tm_bx8, a);
+                  L->tm_bx8, L->tm_bx128, a);
     if (e == cudaSuccess && ev1) e = cudaEventRecord(ev1, st);
     return e;
   }
@@ -681,7 +681,7 @@ cudaError_t launch_mx_down_swap(moe_layer* L, int B, const moe_routing& r, float
     }
   }
   return launch_ex(mx_swap_kernel<false, kMxTerms>, L->num_sms, kMxThreads, sw_smem(a), st, L->pdl, L->tm_adn,
-                   L->tm_bh8, a);
+                   L->tm_bh8, L->tm_bh128, a);
 }
 
 // down projection on the tensor cores; with `residual` non-null fused with
@@ -1303,7 +1303,12 @@ moe_status_t moe_layer_create(const moe_layer_config* cfg, const moe_layer_weigh
               encode_map(&L->tm_bx8, CU_TENSOR_MAP_DATA_TYPE_UINT8, L->aqx, (uint64_t)H / 2,
                          (uint64_t)MB * k * kSwRowsPerTok, (uint64_t)H / 2, 128, kSwRowsPerTok) &&
               encode_map(&L->tm_bh8, CU_TENSOR_MAP_DATA_TYPE_UINT8, L->aqh, (uint64_t)I / 2,
-                         (uint64_t)MB * k * kSwRowsPerTok, (uint64_t)I / 2, 128, kSwRowsPerTok);
+                         (uint64_t)MB * k * kSwRowsPerTok, (uint64_t)I / 2, 128, kSwRowsPerTok) &&
+              // a whole pass of 16 tokens in one copy (128 rows)
+              encode_map(&L->tm_bx128, CU_TENSOR_MAP_DATA_TYPE_UINT8, L->aqx, (uint64_t)H / 2,
+                         (uint64_t)MB * k * kSwRowsPerTok, (uint64_t)H / 2, 128, kMxRows) &&
+              encode_map(&L->tm_bh128, CU_TENSOR_MAP_DATA_TYPE_UINT8, L->aqh, (uint64_t)I / 2,
+                         (uint64_t)MB * k * kSwRowsPerTok, (uint64_t)I / 2, 128, kMxRows);
     if (L->mx) {
       // the scale arrays hold one byte per 32 weights: the chunk copies are the same size
       const size_t gu_bytes = (size_t)E * 2 * I * (H / 32), dn_bytes = (size_t)E * H * (I / 32);

@@ -906,6 +906,16 @@ struct SwWalk {
   }
 };
 
+// a pass of more than 4 tokens takes its activation rows as one 128-row copy
+// (rows beyond the pass are padding; it needs the whole 16 KB A tile in the
+// stage), fewer tokens one 8-row copy each
+__device__ __forceinline__ bool sw_act_whole(const SwArgs& a, const SwRun& r) {
+  return !a.a_by_token && r.ntok > 4 && a.off_w >= kMxRows * 128;
+}
+__device__ __forceinline__ uint32_t sw_act_bytes(const SwArgs& a, const SwRun& r) {
+  return sw_act_whole(a, r) ? (uint32_t)kMxRows * 128u : (uint32_t)r.ntok * (kSwRowsPerTok * 128u);
+}
+
 __device__ __forceinline__ void tc_ld32(uint32_t taddr, float (&v)[32]) {
   uint32_t r[32];
   asm volatile(
@@ -954,7 +964,7 @@ __device__ __forceinline__ float group_amax(float v) {
 template <bool kGU, int kTerms>
 __global__ void __launch_bounds__(kMxThreads, 1)
     mx_swap_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmA,
-                   const SwArgs a) {
+                   const __grid_constant__ CUtensorMap tmA16, const SwArgs a) {
   static_assert(kTerms >= 1 && kTerms <= kSwRowsPerTok, "terms");
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -998,6 +1008,7 @@ __global__ void __launch_bounds__(kMxThreads, 1)
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tmW);
     tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmA16);
   }
   tc_fence_before();
   __syncthreads();
@@ -1092,7 +1103,7 @@ __global__ void __launch_bounds__(kMxThreads, 1)
             const uint32_t cb = (uint32_t)(nck * kMxChunkBytes);
             unsigned char* st = ring + (size_t)s * a.stage_bytes;
             const uint32_t sa = smem_addr(st);
-            mbar_arrive_expect_tx(&full_bar[s], (uint32_t)r.ntok * (kSwRowsPerTok * 128u) + 2u * kMxATile + 3u * cb);
+            mbar_arrive_expect_tx(&full_bar[s], sw_act_bytes(a, r) + 2u * kMxATile + 3u * cb);
             tma_load_2d(sa + a.off_w, &tmW, kt * 128, (int)(tile0 * kMxRows), &full_bar[s], pol);
             tma_load_2d(sa + a.off_w + kMxATile, &tmW, kt * 128, (int)(tile1 * kMxRows), &full_bar[s], pol);
             const size_t ck = (size_t)2 * kt * kMxChunkBytes;
@@ -1126,16 +1137,20 @@ __global__ void __launch_bounds__(kMxThreads, 1)
               *s_abort = 1;
               break;
             }
-            mbar_arrive_expect_tx(&full_bar[s], (uint32_t)r.ntok * (kSwRowsPerTok * 128u) + 2u * kMxATile + 3u * cb);
+            mbar_arrive_expect_tx(&full_bar[s], sw_act_bytes(a, r) + 2u * kMxATile + 3u * cb);
             tma_load_2d(sa + a.off_w, &tmW, kt * 128, (int)(tile0 * kMxRows), &full_bar[s], pol);
             tma_load_2d(sa + a.off_w + kMxATile, &tmW, kt * 128, (int)(tile1 * kMxRows), &full_bar[s], pol);
             bulk_g2s(st + a.off_sfw, sfw0 + ck, cb, &full_bar[s], pol);
             bulk_g2s(st + a.off_sfw + 2 * kMxChunkBytes, sfw1 + ck, cb, &full_bar[s], pol);
           }
           // the activation rows and their scales: written by the preceding kernel
-          for (int i = 0; i < r.ntok; ++i)
-            tma_load_2d_nohint(sa + i * kSwRowsPerTok * 128, &tmA, kt * 128,
-                               (a.a_by_token ? 0 : r.tok + i) * kSwRowsPerTok, &full_bar[s]);
+          if (sw_act_whole(a, r)) {
+            tma_load_2d_nohint(sa, &tmA16, kt * 128, r.tok * kSwRowsPerTok, &full_bar[s]);
+          } else {
+            for (int i = 0; i < r.ntok; ++i)
+              tma_load_2d_nohint(sa + i * kSwRowsPerTok * 128, &tmA, kt * 128,
+                                 (a.a_by_token ? 0 : r.tok + i) * kSwRowsPerTok, &full_bar[s]);
+          }
           bulk_g2s_nohint(st + a.off_sfa, sfa + ck, cb, &full_bar[s]);
           if (++s == ns) { s = 0; ph ^= 1u; }
         }
