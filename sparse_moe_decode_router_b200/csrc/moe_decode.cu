@@ -819,9 +819,14 @@ cudaError_t launch_dense_k1(moe_layer* L, const void* x, int B, cudaStream_t st,
                    a.n_streams > 1 ? L->tm_sgu : L->tm_wr, tmx, a);
 }
 
-cudaError_t launch_dense_sdn(moe_layer* L, int B, float* ys, cudaStream_t st) {
+// the shared down projection leaves kSdnFreeSms SMs to the routing finish
+// and the activation terms, which run beside it in the fused forward
+constexpr int kSdnFreeSms = 16;
+int sdn_grid(const moe_layer* L) { return std::max(1, L->num_sms - kSdnFreeSms); }
+
+cudaError_t launch_dense_sdn(moe_layer* L, int B, float* ys, cudaStream_t st, bool pdl = true) {
   const DenseArgs a = dn_args_sdn(L, B, ys);
-  return launch_ex(dense_bf16_kernel, L->num_sms, kDnThreads, dn_smem(a), st, L->pdl, L->tm_sdn, L->tm_sdn,
+  return launch_ex(dense_bf16_kernel, sdn_grid(L), kDnThreads, dn_smem(a), st, L->pdl && pdl, L->tm_sdn, L->tm_sdn,
                    L->tm_ht, a);
 }
 
@@ -1350,7 +1355,9 @@ moe_status_t moe_layer_create(const moe_layer_config* cfg, const moe_layer_weigh
     if (ok) {
       const int t1 = dn_tiles_k1(L), t2 = sh ? H / kDnRows : 0;
       L->dparts1 = dn_max_parts(dn_args_k1(L, 2), L->num_sms);
-      L->dparts2 = sh ? dn_max_parts(dn_args_sdn(L, 2, L->ys), L->num_sms) : 1;
+      L->dparts2 = sh ? std::max(dn_max_parts(dn_args_sdn(L, 2, L->ys), L->num_sms),
+                                 dn_max_parts(dn_args_sdn(L, 2, L->ys), sdn_grid(L)))
+                      : 1;
       const size_t part = (size_t)2 * kDnNMax * kDnRows * sizeof(float);
       const size_t b_ht = align_up((size_t)MB * kDnHTerms * std::max(Is, 1) * 2, 256);
       const size_t b_w1 = (size_t)t1 * L->dparts1 * part, b_w2 = (size_t)std::max(t2, 1) * L->dparts2 * part;
@@ -1492,7 +1499,9 @@ moe_status_t moe_experts_mxfp4(moe_layer_t L, const void* x, int B, const moe_ro
   const moe_routing& rr = r ? *r : L->plan;
   cudaStream_t st = (cudaStream_t)stream;
   const bool has_shared = L->cfg.shared_inter > 0;
-  const bool fork = has_shared && L->side_stream;
+  // as in moe_layer_forward: a bf16 shared expert above batch 1 on the
+  // tensor-core path runs the dense kernels whatever the side-stream flag
+  const bool fork = has_shared && L->side_stream && !(dense_for(L, B) && !L->shared_mx);
   cudaError_t e = cudaSuccess;
   if (fork) {
     e = cudaEventRecord(L->ev_fork, st);
@@ -1535,7 +1544,10 @@ moe_status_t moe_layer_forward(moe_layer_t L, moe_layer_t next, const void* x, c
   if (next && next->device != L->device) return MOE_ERR_INVALID_ARG;  // prefetch reads local memory only
   cudaStream_t st = (cudaStream_t)stream;
   const bool has_shared = L->cfg.shared_inter > 0;
-  const bool fork = has_shared && L->side_stream;
+  // above batch 1 on the tensor-core path a bf16 shared expert's down
+  // projection takes the side stream anyway (below)
+  const bool dense = dense_for(L, B);
+  const bool fork = has_shared && L->side_stream && !(dense && !L->shared_mx);
   cudaError_t e = cudaSuccess;
   if (fork) {
     e = cudaEventRecord(L->ev_fork, st);
@@ -1544,13 +1556,27 @@ moe_status_t moe_layer_forward(moe_layer_t L, moe_layer_t next, const void* x, c
     if (e == cudaSuccess) e = cudaEventRecord(L->ev_join, L->side);
   }
   if (B == 1 && L->persist && !fork) return cuda_status(launch_persistent(L, next, x, residual, out, st));
-  if (dense_for(L, B)) {
-    // router + shared gate/up, shared down, routing finish, routed experts
+  if (dense) {
+    // router (+ shared gate/up), then the shared down projection on the side
+    // stream beside the routing finish, the activation terms and the routed
+    // experts (its grid leaves SMs free for the first two); the combine waits
+    // for it
     if (e == cudaSuccess) e = launch_dense_k1(L, x, B, st);
-    if (e == cudaSuccess && has_shared)
-      e = L->shared_mx ? launch_shared(L, x, B, L->ys, st, L->pdl) : launch_dense_sdn(L, B, L->ys, st);
+    bool join = fork;  // an MXFP4 shared expert forked above
+    if (e == cudaSuccess && has_shared && !fork) {
+      if (L->shared_mx) {
+        e = launch_shared(L, x, B, L->ys, st, L->pdl);
+      } else {
+        e = cudaEventRecord(L->ev_fork, st);
+        if (e == cudaSuccess) e = cudaStreamWaitEvent(L->side, L->ev_fork, 0);
+        if (e == cudaSuccess) e = launch_dense_sdn(L, B, L->ys, L->side, false);
+        if (e == cudaSuccess) e = cudaEventRecord(L->ev_join, L->side);
+        join = true;
+      }
+    }
     if (e == cudaSuccess) e = launch_routing_finish(L, x, B, L->plan, st);
     if (e == cudaSuccess) e = launch_gate_up(L, x, B, L->plan, st, L->probe_start, L->probe_stop);
+    if (e == cudaSuccess && join) e = cudaStreamWaitEvent(st, L->ev_join, 0);
     if (e == cudaSuccess)
       e = launch_down(L, B, L->plan, L->y, true, residual, out, has_shared ? L->ys : nullptr, next, st, L->pdl);
     return cuda_status(e);
