@@ -331,6 +331,17 @@ def test_mx_skewed_matches_oracle(torch_cuda, skewed_small, B):
     check_against_oracle(got, ref)
 
 
+@pytest.mark.parametrize("B", [1, 9, 33])
+def test_mx_weights_as_a_kernel_matches_oracle(torch_cuda, B):
+    """Hidden 384 (a multiple of 128, not of 256): the tcgen05 path keeps the
+    kernels with the weights as the A operand (128-row tiles of one
+    projection, activation terms as N columns)."""
+    base = synth.CONFIGS[0]
+    dl = make_device_layer(base.with_(hidden=384, inter=256, shared_inter=64, seed=base.seed + 700))
+    got, ref = run_all_paths(torch_cuda, dl, B, max_batch=64, flags=MX)
+    check_against_oracle(got, ref)
+
+
 def test_mx_and_gemv_paths_agree(torch_cuda, skewed_small):
     got_m, ref = run_all_paths(torch_cuda, skewed_small, 7, max_batch=8, flags=MX)
     got_g, _ = run_all_paths(torch_cuda, skewed_small, 7, max_batch=8)
