@@ -627,7 +627,7 @@ cudaError_t launch_mx_gate_up(moe_layer* L, const void* x, int B, const moe_rout
   const int H = L->cfg.hidden, k = L->cfg.top_k;
   // batch 1: every position holds the same token, whose terms are made once
   const int by_token = B == 1 ? 1 : 0;
-  const dim3 grid(B, (H / 32 + 7) / 8);
+  const dim3 grid(B, (H / 32 + 255) / 256);
   const int rpp = L->swap ? kSwRowsPerTok : kMxTerms;
   const int tpp = L->swap ? sw_tokens_per_pass(B) : mx_n_max(B) / kMxTerms;
   cudaError_t e = launch_ex(mx_x_terms_kernel<kMxTerms>, grid, 256, 0, st, L->pdl, static_cast<const uint16_t*>(x),

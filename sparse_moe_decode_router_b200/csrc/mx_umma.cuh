@@ -258,9 +258,10 @@ __device__ __forceinline__ int sf_chunk_byte(int n, int kb) { return 16 * (n & 3
 // x (bf16 [B][K]) -> terms of the gate/up activations: row q*rpp + t of
 // aq [.][K/2] (packed E2M1, even element in the low nibble) and the scales
 // into the chunks of q's pass, for every pair position q of the token.
-// Grid (B, ceil(K/256)), 8 warps: warp w of CTA (b, g) takes the 32-element
-// block 8g + w of token b, one element per lane, makes its terms once and
-// writes them to the token's top_k positions (found by a scan of pair_ids).
+// Grid (B, ceil(K/8192)), 256 threads: thread i of CTA (b, g) takes the
+// 32-element block 256g + i of token b in registers (no cross-lane steps),
+// makes its terms once and writes them, 16 bytes per term, to the token's
+// top_k positions (found by a scan of pair_ids).
 // With by_token (batch 1) row 0 is the token itself, which every position
 // reads, and its chunk is chunk 0 (columns = terms).
 template <int kTerms>
@@ -273,7 +274,7 @@ __global__ void __launch_bounds__(256) mx_x_terms_kernel(const uint16_t* __restr
   __shared__ int s_q[kMaxTopK], s_p0[kMaxTopK], s_e[kMaxTopK];
   pdl_wait();
   const int b = blockIdx.x, tid = threadIdx.x;
-  const int lane = tid & 31, blk = blockIdx.y * 8 + (tid >> 5);
+  const int blk = blockIdx.y * blockDim.x + tid;
   const int nq = by_token ? 1 : top_k;
   if (nq < 1 || nq > kMaxTopK || rpp < kTerms || tpp * rpp > kMxRows) {
     if (tid == 0) atomicExch(err, kErrBadPlan);
@@ -282,7 +283,12 @@ __global__ void __launch_bounds__(256) mx_x_terms_kernel(const uint16_t* __restr
   }
   // written by preceding kernels: coherent loads, all issued before the first wait
   const bool has_blk = blk < (K >> 5);
-  const uint16_t xv = has_blk ? __ldcg(x + (size_t)b * K + 32 * blk + lane) : (uint16_t)0;
+  uint4 xr[4];
+  if (has_blk) {
+    const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)b * K + 32 * blk);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) xr[i] = __ldcg(src + i);
+  }
   if (tid < nq) {
     s_q[tid] = by_token ? 0 : -1;
     s_e[tid] = by_token ? 0 : __ldcg(topk_idx + b * top_k + tid);
@@ -318,18 +324,33 @@ __global__ void __launch_bounds__(256) mx_x_terms_kernel(const uint16_t* __restr
     return;
   }
   if (has_blk) {
-    float v = __uint_as_float((uint32_t)xv << 16);
-    uint32_t w[kTerms];
+    float v[32];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint32_t u[4] = {xr[i].x, xr[i].y, xr[i].z, xr[i].w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        v[8 * i + 2 * j] = __uint_as_float(u[j] << 16);
+        v[8 * i + 2 * j + 1] = __uint_as_float(u[j] & 0xFFFF0000u);
+      }
+    }
+    uint4 w[kTerms];
     int ex[kTerms];
 #pragma unroll
     for (int t = 0; t < kTerms; ++t) {
-      const int e = mx_scale_exp(warp_amax(fabsf(v)));
-      const uint32_t c = f32_to_e2m1(v * pow2_exact(-e));
-      v -= e2m1_to_f32(c) * pow2_exact(e);
-      uint32_t ww = c << (4 * (lane & 7));
+      float am = 0.f;
 #pragma unroll
-      for (int o = 1; o < 8; o <<= 1) ww |= __shfl_xor_sync(0xFFFFFFFFu, ww, o);
-      w[t] = ww;
+      for (int j = 0; j < 32; ++j) am = fmaxf(am, fabsf(v[j]));
+      const int e = mx_scale_exp(am);
+      const float down = pow2_exact(-e), up = pow2_exact(e);
+      uint32_t wd[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        const uint32_t c = f32_to_e2m1(v[j] * down);
+        v[j] -= e2m1_to_f32(c) * up;
+        wd[j >> 3] |= c << (4 * (j & 7));  // element 2m in the low nibble of byte m
+      }
+      w[t] = make_uint4(wd[0], wd[1], wd[2], wd[3]);
       ex[t] = e;
     }
     for (int j = 0; j < nq; ++j) {
@@ -338,9 +359,8 @@ __global__ void __launch_bounds__(256) mx_x_terms_kernel(const uint16_t* __restr
       uint8_t* chunk = bsf + ((size_t)p0 * (K / kMxKChunk) + (blk >> 2)) * kMxChunkBytes;
 #pragma unroll
       for (int t = 0; t < kTerms; ++t) {
-        if ((lane & 7) == 0)
-          *reinterpret_cast<uint32_t*>(aq + ((size_t)q * rpp + t) * (K / 2) + 16 * blk + (lane >> 3) * 4) = w[t];
-        if (lane == 0) chunk[sf_chunk_byte(n0 + t, blk & 3)] = (uint8_t)(ex[t] + 127);
+        *reinterpret_cast<uint4*>(aq + ((size_t)q * rpp + t) * (K / 2) + 16 * blk) = w[t];
+        chunk[sf_chunk_byte(n0 + t, blk & 3)] = (uint8_t)(ex[t] + 127);
       }
     }
   }
