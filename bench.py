@@ -666,13 +666,17 @@ def launches_per_step(cfg, path):
     batch 1 on the tcgen05 path the router and the bf16 shared expert run on
     the dense tensor-core kernels (the router's launch, the shared down's) and
     the routing finish is a launch of its own; above batch 2 the combine
-    follows the tcgen05 down projection as a launch of its own."""
+    follows the tcgen05 down projection as a launch of its own.  Where the
+    hidden size is a multiple of 256 the tcgen05 gate/up kernel writes h in
+    fp32 and a small kernel makes its E2M1 terms (one launch more)."""
     n = 1
     if cfg.shared_inter > 0:
         n += 2 if cfg.shared_format == "mxfp4" else 1
     if path == 2 and cfg.batch > 1:
         n += 1
     if path == 2 and cfg.batch > 2:
+        n += 1
+    if path == 2 and cfg.hidden % 256 == 0:
         n += 1
     return n + {2: 3, 1: 5, 0: 2}[path]
 

@@ -627,7 +627,7 @@ cudaError_t launch_mx_gate_up(moe_layer* L, const void* x, int B, const moe_rout
   const int H = L->cfg.hidden, k = L->cfg.top_k;
   // batch 1: every position holds the same token, whose terms are made once
   const int by_token = B == 1 ? 1 : 0;
-  const dim3 grid(B, (H / 32 + 255) / 256);
+  const dim3 grid(B, (H / 32 + 31) / 32);
   const int rpp = L->swap ? kSwRowsPerTok : kMxTerms;
   const int tpp = L->swap ? sw_tokens_per_pass(B) : mx_n_max(B) / kMxTerms;
   cudaError_t e = launch_ex(mx_x_terms_kernel<kMxTerms>, grid, 256, 0, st, L->pdl, static_cast<const uint16_t*>(x),
@@ -636,9 +636,13 @@ cudaError_t launch_mx_gate_up(moe_layer* L, const void* x, int B, const moe_rout
                             static_cast<const int*>(r.offsets), by_token, L->aqx, L->bsfx, L->err);
   if (e != cudaSuccess) return e;
   if (L->swap) {
+    // gate/up writes h in fp32 (L->h); a small kernel then makes its terms
+    // for the down projection (the conversion costs far more CUDA-core time
+    // in the gate/up epilogue, beside the running copies and MMAs)
     SwArgs a = sw_args(L, true, B, r);
     a.a_by_token = by_token;
-    a.h = nullptr;  // on this path the down projection reads h's terms only
+    a.h = L->h;
+    a.h_only = 1;
     (void)h;
     a.next_aq = L->aqh;
     a.next_bsf = L->bsfh;
@@ -646,7 +650,13 @@ cudaError_t launch_mx_gate_up(moe_layer* L, const void* x, int B, const moe_rout
     e = launch_ex(mx_swap_kernel<true, kMxTerms>, L->num_sms, kMxThreads, sw_smem(a), st, L->pdl, L->tm_agu,
                   L->tm_bx8, L->tm_bx128, a);
     if (e == cudaSuccess && ev1) e = cudaEventRecord(ev1, st);
-    return e;
+    if (e != cudaSuccess) return e;
+    const int I = L->cfg.inter;
+    const long long n_thr = (long long)B * k * (I / 32) * 8;
+    return launch_ex(mx_h_terms_kernel<kMxTerms>, (int)((n_thr + 255) / 256), 256, 0, st, L->pdl,
+                     static_cast<const float*>(L->h), I, k, B * k, L->cfg.n_experts, sw_tokens_per_pass(B),
+                     kSwRowsPerTok, static_cast<const int*>(r.pair_ids), static_cast<const int*>(r.topk_idx),
+                     static_cast<const int*>(r.offsets), L->aqh, L->bsfh, L->err);
   }
   const MxPlan p = mx_plan(true, B);
   MxArgs a = mx_args(L, true, B, r, p, h);
@@ -1426,6 +1436,7 @@ moe_status_t moe_layer_create(const moe_layer_config* cfg, const moe_layer_weigh
     if (e == cudaSuccess) e = raise_smem_limit(reinterpret_cast<const void*>(grouped_mma_kernel<false>), kSmemBudget);
   }
   const void* small_kernels[] = {reinterpret_cast<const void*>(mx_x_terms_kernel<kMxTerms>),
+                                 reinterpret_cast<const void*>(mx_h_terms_kernel<kMxTerms>),
                                  reinterpret_cast<const void*>(act_to_f16_kernel<false>),
                                  reinterpret_cast<const void*>(act_to_f16_kernel<true>),
                                  reinterpret_cast<const void*>(combine_kernel)};

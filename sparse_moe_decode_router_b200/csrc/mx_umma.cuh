@@ -258,10 +258,10 @@ __device__ __forceinline__ int sf_chunk_byte(int n, int kb) { return 16 * (n & 3
 // x (bf16 [B][K]) -> terms of the gate/up activations: row q*rpp + t of
 // aq [.][K/2] (packed E2M1, even element in the low nibble) and the scales
 // into the chunks of q's pass, for every pair position q of the token.
-// Grid (B, ceil(K/8192)), 256 threads: thread i of CTA (b, g) takes the
-// 32-element block 256g + i of token b in registers (no cross-lane steps),
-// makes its terms once and writes them, 16 bytes per term, to the token's
-// top_k positions (found by a scan of pair_ids).
+// Grid (B, ceil(K/1024)), 256 threads: eight lanes of CTA (b, g) take one
+// 32-element block of token b (four elements each; the block's maximum is a
+// three-step exchange within the eight lanes), make its terms once and write
+// them to the token's top_k positions (found by a scan of pair_ids).
 // With by_token (batch 1) row 0 is the token itself, which every position
 // reads, and its chunk is chunk 0 (columns = terms).
 template <int kTerms>
@@ -274,7 +274,7 @@ __global__ void __launch_bounds__(256) mx_x_terms_kernel(const uint16_t* __restr
   __shared__ int s_q[kMaxTopK], s_p0[kMaxTopK], s_e[kMaxTopK];
   pdl_wait();
   const int b = blockIdx.x, tid = threadIdx.x;
-  const int blk = blockIdx.y * blockDim.x + tid;
+  const int l8 = tid & 7, blk = blockIdx.y * (blockDim.x >> 3) + (tid >> 3);
   const int nq = by_token ? 1 : top_k;
   if (nq < 1 || nq > kMaxTopK || rpp < kTerms || tpp * rpp > kMxRows) {
     if (tid == 0) atomicExch(err, kErrBadPlan);
@@ -282,13 +282,9 @@ __global__ void __launch_bounds__(256) mx_x_terms_kernel(const uint16_t* __restr
     return;
   }
   // written by preceding kernels: coherent loads, all issued before the first wait
-  const bool has_blk = blk < (K >> 5);
-  uint4 xr[4];
-  if (has_blk) {
-    const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)b * K + 32 * blk);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) xr[i] = __ldcg(src + i);
-  }
+  const bool has_blk = blk < (K >> 5);  // uniform over a block's eight lanes
+  uint2 xr = make_uint2(0u, 0u);
+  if (has_blk) xr = __ldcg(reinterpret_cast<const uint2*>(x + (size_t)b * K + 32 * blk + 4 * l8));
   if (tid < nq) {
     s_q[tid] = by_token ? 0 : -1;
     s_e[tid] = by_token ? 0 : __ldcg(topk_idx + b * top_k + tid);
@@ -323,45 +319,102 @@ __global__ void __launch_bounds__(256) mx_x_terms_kernel(const uint16_t* __restr
     pdl_launch_dependents();
     return;
   }
+  // every lane takes part in the exchanges (lanes of a block past K hold zeros)
+  float v[4] = {__uint_as_float(xr.x << 16), __uint_as_float(xr.x & 0xFFFF0000u), __uint_as_float(xr.y << 16),
+                __uint_as_float(xr.y & 0xFFFF0000u)};
+  uint32_t w[kTerms];
+  int ex[kTerms];
+#pragma unroll
+  for (int t = 0; t < kTerms; ++t) {
+    float am = fmaxf(fmaxf(fabsf(v[0]), fabsf(v[1])), fmaxf(fabsf(v[2]), fabsf(v[3])));
+#pragma unroll
+    for (int o = 1; o < 8; o <<= 1) am = fmaxf(am, __shfl_xor_sync(0xFFFFFFFFu, am, o));
+    const int e = mx_scale_exp(am);
+    const float down = pow2_exact(-e), up = pow2_exact(e);
+    uint32_t pk = 0u;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const uint32_t c = f32_to_e2m1(v[j] * down);
+      v[j] -= e2m1_to_f32(c) * up;
+      pk |= c << (4 * j);  // element 2m in the low nibble of byte m
+    }
+    w[t] = pk;
+    ex[t] = e;
+  }
   if (has_blk) {
-    float v[32];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const uint32_t u[4] = {xr[i].x, xr[i].y, xr[i].z, xr[i].w};
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        v[8 * i + 2 * j] = __uint_as_float(u[j] << 16);
-        v[8 * i + 2 * j + 1] = __uint_as_float(u[j] & 0xFFFF0000u);
-      }
-    }
-    uint4 w[kTerms];
-    int ex[kTerms];
-#pragma unroll
-    for (int t = 0; t < kTerms; ++t) {
-      float am = 0.f;
-#pragma unroll
-      for (int j = 0; j < 32; ++j) am = fmaxf(am, fabsf(v[j]));
-      const int e = mx_scale_exp(am);
-      const float down = pow2_exact(-e), up = pow2_exact(e);
-      uint32_t wd[4] = {0u, 0u, 0u, 0u};
-#pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        const uint32_t c = f32_to_e2m1(v[j] * down);
-        v[j] -= e2m1_to_f32(c) * up;
-        wd[j >> 3] |= c << (4 * (j & 7));  // element 2m in the low nibble of byte m
-      }
-      w[t] = make_uint4(wd[0], wd[1], wd[2], wd[3]);
-      ex[t] = e;
-    }
     for (int j = 0; j < nq; ++j) {
       const int q = s_q[j], p0 = s_p0[j];
       const int n0 = (q - p0) * rpp;  // this position's first row (column) in its pass's scale chunks
       uint8_t* chunk = bsf + ((size_t)p0 * (K / kMxKChunk) + (blk >> 2)) * kMxChunkBytes;
 #pragma unroll
       for (int t = 0; t < kTerms; ++t) {
-        *reinterpret_cast<uint4*>(aq + ((size_t)q * rpp + t) * (K / 2) + 16 * blk) = w[t];
-        chunk[sf_chunk_byte(n0 + t, blk & 3)] = (uint8_t)(ex[t] + 127);
+        *reinterpret_cast<uint16_t*>(aq + ((size_t)q * rpp + t) * (K / 2) + 16 * blk + 2 * l8) = (uint16_t)w[t];
+        if (l8 == 0) chunk[sf_chunk_byte(n0 + t, blk & 3)] = (uint8_t)(ex[t] + 127);
       }
+    }
+  }
+  pdl_launch_dependents();
+}
+
+// h (fp32 [pair][I], written by the gate/up kernel) -> the down projection's
+// E2M1 terms: row q*rpp + t of aq [.][I/2] and the scales into the chunks of
+// q's pass (passes of tpp tokens from the expert's offset), for every pair
+// position q.  Eight lanes per (position, 32-element block), four elements
+// each; grid (ceil(n_pairs * I/32 * 8 / 256)).
+template <int kTerms>
+__global__ void __launch_bounds__(256) mx_h_terms_kernel(const float* __restrict__ h, int I, int top_k, int n_pairs,
+                                                         int n_experts, int tpp, int rpp,
+                                                         const int* __restrict__ pair_ids,
+                                                         const int* __restrict__ topk_idx,
+                                                         const int* __restrict__ offsets, uint8_t* __restrict__ aq,
+                                                         uint8_t* __restrict__ bsf, int* err) {
+  pdl_wait();
+  const int nb = I >> 5;  // blocks per row
+  const long long gi = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  const long long gb = gi >> 3;  // (position, block); a block's eight lanes share it
+  const int l8 = threadIdx.x & 7;
+  const bool on = gb < (long long)n_pairs * nb && rpp >= kTerms && tpp * rpp <= kMxRows;
+  int q = 0, blk = 0, p = 0, p0 = -1;
+  if (on) {
+    q = (int)(gb / nb);
+    blk = (int)(gb - (long long)q * nb);
+    // the pair at position q, its expert and the first position of q's pass
+    p = __ldcg(pair_ids + q);
+    const int e = (p >= 0 && p < n_pairs) ? __ldcg(topk_idx + p) : -1;
+    if (e >= 0 && e < n_experts) {
+      const int off = __ldcg(offsets + e), end = __ldcg(offsets + e + 1);
+      if (off >= 0 && q >= off && q < end) p0 = off + (q - off) / tpp * tpp;
+    }
+    if (p0 < 0 && l8 == 0) atomicExch(err, kErrBadPlan);
+  }
+  const bool ok = on && p0 >= 0;  // uniform over a block's eight lanes
+  float v[4] = {0.f, 0.f, 0.f, 0.f};
+  if (ok) {
+    const float4 f = __ldcg(reinterpret_cast<const float4*>(h + (size_t)p * I + 32 * blk + 4 * l8));
+    v[0] = f.x;
+    v[1] = f.y;
+    v[2] = f.z;
+    v[3] = f.w;
+  }
+  const int n0 = (q - p0) * rpp;
+  uint8_t* chunk = bsf + ((size_t)max(p0, 0) * (I / kMxKChunk) + (blk >> 2)) * kMxChunkBytes;
+#pragma unroll
+  for (int t = 0; t < kTerms; ++t) {
+    float am = fmaxf(fmaxf(fabsf(v[0]), fabsf(v[1])), fmaxf(fabsf(v[2]), fabsf(v[3])));
+#pragma unroll
+    for (int o = 1; o < 8; o <<= 1) am = fmaxf(am, __shfl_xor_sync(0xFFFFFFFFu, am, o));
+    const int ex = mx_scale_exp(am);
+    const float down = pow2_exact(-ex), up = pow2_exact(ex);
+    uint32_t pk = 0u;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const uint32_t c = f32_to_e2m1(v[j] * down);
+      v[j] -= e2m1_to_f32(c) * up;
+      pk |= c << (4 * j);
+    }
+    if (ok) {
+      *reinterpret_cast<uint16_t*>(aq + ((size_t)q * rpp + t) * (I / 2) + 16 * blk + 2 * l8) = (uint16_t)pk;
+      if (l8 == 0) chunk[sf_chunk_byte(n0 + t, blk & 3)] = (uint8_t)(ex + 127);
     }
   }
   pdl_launch_dependents();
@@ -813,6 +866,7 @@ struct SwArgs {
   int* item_cnt;            // per unit: pieces arrived, zero between launches
   // gate/up
   float* h;                 // h fp32 [pair][I], or null
+  int h_only;               // 1: h fp32 only; its terms come from mx_h_terms_kernel
   uint8_t* next_aq;         // h's E2M1 terms [pos*8 + t][I/2]
   uint8_t* next_bsf;        // their scale chunks [pass-start position][I/128][512], row 8*i + t
   // down
@@ -1348,7 +1402,18 @@ __global__ void __launch_bounds__(kMxThreads, 1)
       }
       if (fin && quad) {
         if (pr < 0 || pr >= a.n_pairs) pr = 0;
-        if (kGU) {
+        if (kGU && a.h_only) {
+          // h rows rt*128 + 32c + 4*l8 .. +3 in fp32 (gate in chunk c, up in chunk c + 4)
+          if (mine) {
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              const float4 g4 = res[c], u4 = res[c + 4];
+              *reinterpret_cast<float4*>(a.h + (size_t)pr * a.out_rows + r.rt * kMxRows + 32 * c + 4 * l8) =
+                  make_float4(g4.x / (1.0f + expf(-g4.x)) * u4.x, g4.y / (1.0f + expf(-g4.y)) * u4.y,
+                              g4.z / (1.0f + expf(-g4.z)) * u4.z, g4.w / (1.0f + expf(-g4.w)) * u4.w);
+            }
+          }
+        } else if (kGU) {
           // h rows rt*128 + 32c + 4*l8 .. +3: gate in chunk c, up in chunk c + 4.
           // The packed terms go through this warp's staging bytes ([token of
           // the warp][term][64 bytes = the item's 128 rows]) and out as
