@@ -80,10 +80,10 @@ struct DenseArgs {
 };
 
 // stream-K partition: stage i of the launch's list (tiles of stream 0, then
-// stream 1; S stages per tile) weighs 1, or 2 for a SwiGLU stream.  CTA c of
+// stream 1; S stages per tile) weighs 2, or 3 for a SwiGLU stream.  CTA c of
 // the first G owns stages [first(c), first(c + 1)); G is at most half the
 // stages, so every such range holds at least one stage (a range's weight is
-// at least 2) and the parts of a tile are the ranges of consecutive CTAs.
+// at least 4) and the parts of a tile are the ranges of consecutive CTAs.
 // CTAs from G on have no work.
 struct DnSplit {
   long long S, T0, T1, w0, w1, W0, W, G;
@@ -109,8 +109,11 @@ __host__ __device__ inline DnSplit dn_split(const DenseArgs& a, int G) {
   d.S = a.K / kDnKBox;
   d.T0 = a.st[0].n_tiles;
   d.T1 = a.n_streams > 1 ? a.st[1].n_tiles : 0;
-  d.w0 = a.st[0].up_rows ? 2 : 1;
-  d.w1 = (a.n_streams > 1 && a.st[1].up_rows) ? 2 : 1;
+  // a stage's cost: its A tiles' bytes plus a fixed part per stage (the
+  // barrier round trip, the copies' and MMAs' issue): one tile weighs 2, a
+  // gate/up pair 3 (measured: a one-tile stage takes ~0.68 of a pair's time)
+  d.w0 = a.st[0].up_rows ? 3 : 2;
+  d.w1 = (a.n_streams > 1 && a.st[1].up_rows) ? 3 : 2;
   d.W0 = d.T0 * d.S * d.w0;
   d.W = d.W0 + d.T1 * d.S * d.w1;
   const long long half = (d.T0 + d.T1) * d.S / 2;
