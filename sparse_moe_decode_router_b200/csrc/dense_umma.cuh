@@ -516,6 +516,7 @@ __global__ void __launch_bounds__(256) routing_finish_kernel(const GemvArgs a) {
   extern __shared__ __align__(128) unsigned char smem[];
   __shared__ int s_last;
   pdl_wait();
+  pdl_launch_dependents();  // the activation terms read the plan after their own wait
   const int tid = threadIdx.x, b = blockIdx.x;
   const int E = a.n_experts;
   topk_token_block(a, a.out + (size_t)b * E, b, tid, blockDim.x, 1, false, smem + kBucketScratchBytes);

@@ -273,6 +273,9 @@ __global__ void __launch_bounds__(256) mx_x_terms_kernel(const uint16_t* __restr
                                                          uint8_t* __restrict__ aq, uint8_t* __restrict__ bsf, int* err) {
   __shared__ int s_q[kMaxTopK], s_p0[kMaxTopK], s_e[kMaxTopK];
   pdl_wait();
+  // the next kernel (the gate/up projection) may start its prologue and
+  // static-weight copies now; it reads these outputs after its own wait
+  pdl_launch_dependents();
   const int b = blockIdx.x, tid = threadIdx.x;
   const int l8 = tid & 7, blk = blockIdx.y * (blockDim.x >> 3) + (tid >> 3);
   const int nq = by_token ? 1 : top_k;
@@ -369,6 +372,7 @@ __global__ void __launch_bounds__(256) mx_h_terms_kernel(const float* __restrict
                                                          const int* __restrict__ offsets, uint8_t* __restrict__ aq,
                                                          uint8_t* __restrict__ bsf, int* err) {
   pdl_wait();
+  pdl_launch_dependents();  // as in mx_x_terms_kernel: the down projection's prologue may start
   const int nb = I >> 5;  // blocks per row
   const long long gi = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   const long long gb = gi >> 3;  // (position, block); a block's eight lanes share it
