@@ -473,6 +473,8 @@ def grouped_flops(cfg, n_pairs):
 
 
 def per_config_record(cfg, flags, steps, warmup, peak, sampler):
+    from sparse_moe_decode_router_b200 import api
+    persistent = bool(flags & api.MOE_FLAG_PERSISTENT) and cfg.batch == 1  # one cooperative launch
     run = LayerRun(cfg, flags, pool=8)
     try:
         ms = run.timed(steps, warmup, sampler)
@@ -484,7 +486,7 @@ def per_config_record(cfg, flags, steps, warmup, peak, sampler):
                "tokens_per_s": round(cfg.batch * steps / sec, 1),
                "counted_bytes_per_step": int(tot / steps),
                "n_active_mean": statistics.mean(run.n_active[i % run.pool] for i in range(steps)),
-               "gpu_launches_per_step": launches_per_step(cfg, run.path),
+               "gpu_launches_per_step": (1 if persistent else launches_per_step(cfg, run.path)),
                "expert_path": PATH_NAMES[run.path]}
         if run.path != 0:
             fl = grouped_flops(cfg, cfg.batch * cfg.top_k)
@@ -608,6 +610,12 @@ def run_ours(args, cfg):
             "full_b8": per_config_record(synth.CONFIGS[2], args.flags, 50, 5, peak, sampler),
             "full_b64_zipf": per_config_record(synth.CONFIGS[3], args.flags, 20, 3, peak, sampler),
             "full_b8_verify": per_config_record(synth.CONFIGS[5], args.flags, 50, 5, peak, sampler),
+            # batch-1 variants beside the default chain: the persistent single
+            # launch, and the routed experts on the tensor cores
+            "full_b1_persistent": per_config_record(synth.CONFIGS[1], args.flags | api.MOE_FLAG_PERSISTENT, 50, 5,
+                                                    peak, sampler),
+            "full_b1_tcgen05": per_config_record(synth.CONFIGS[1], args.flags | api.MOE_FLAG_MX_EXPERTS, 50, 5,
+                                                 peak, sampler),
             "full_stack4_b1_graph": {
                 "prefetch": stack_record(synth.CONFIGS[4], args.flags, 3, peak, sampler),
                 "no_prefetch": stack_record(synth.CONFIGS[4], args.flags | api.MOE_FLAG_NO_PREFETCH, 3, peak,
