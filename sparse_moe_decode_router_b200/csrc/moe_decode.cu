@@ -319,7 +319,13 @@ moe_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE
 // The dense bf16 streams keep two tokens per pass there.
 constexpr int kSmallBatch = 8;
 bool routed_kind(Kind k) { return k == K_GU || k == K_DN || k == K_DNC; }
-int slot_for(Kind k, int B) { return B == 1 ? 0 : ((B <= kSmallBatch && routed_kind(k)) ? 2 : 1); }
+// The routed down projection at batch 1 takes the one-token plans of the
+// small batches (whole rows per warp): measured faster there than the
+// split-K instance, whose cross-warp reduction stalls on barriers.
+int slot_for(Kind k, int B) {
+  if (B == 1 && (k == K_DN || k == K_DNC)) return 2;
+  return B == 1 ? 0 : ((B <= kSmallBatch && routed_kind(k)) ? 2 : 1);
+}
 int tmax_of_slot(int t) { return t == 1 ? 2 : 1; }
 int tmax_for(int B) { return B == 1 ? 1 : 2; }  // dense streams
 
@@ -981,7 +987,7 @@ GemvArgs down_args(const moe_layer* L, int B, const moe_routing& r, float* y, bo
 
 // the persistent kernel's instances: the streams of the batch-1 chain
 // (shape-specialised: compile-time K, split-K down; generic: runtime K)
-#define PERSIST_FAST persistent_b1_kernel<kFastH, kFastI, MOE_SPLITK_GU ? kSplitKRows / 2 : MOE_GU_RPW, kSplitKRows>
+#define PERSIST_FAST persistent_b1_kernel<kFastH, kFastI, MOE_SPLITK_GU ? kSplitKRows / 2 : MOE_GU_RPW, MOE_DN_RPW>
 #define PERSIST_GENERIC persistent_b1_kernel<0, 0, MOE_GU_RPW, MOE_DN_RPW>
 
 // The whole batch-1 step as one cooperative kernel (MOE_FLAG_PERSISTENT).
@@ -1003,8 +1009,8 @@ cudaError_t launch_persistent(moe_layer* L, moe_layer* next, const void* x, cons
   const Kind kinds[4] = {K_ROUTER, K_SDN, K_GU, K_DNC};
   for (Kind kk : kinds) {
     if (kk == K_SDN && !has_shared) continue;
-    threads = std::max(threads, L->plans[kk][0].threads);
-    smem = std::max(smem, L->plans[kk][0].smem);
+    threads = std::max(threads, plan_of(L, kk, 1).threads);
+    smem = std::max(smem, plan_of(L, kk, 1).smem);
   }
   cudaError_t e = cudaMemsetAsync(L->grid_bar, 0, sizeof(int), st);
   if (e != cudaSuccess) return e;
@@ -1414,8 +1420,8 @@ moe_status_t moe_layer_create(const moe_layer_config* cfg, const moe_layer_weigh
     int threads = 0, smem = 0;
     for (Kind kk : {K_ROUTER, K_SDN, K_GU, K_DNC}) {
       if (kk == K_SDN && Is == 0) continue;
-      threads = std::max(threads, L->plans[kk][0].threads);
-      smem = std::max(smem, L->plans[kk][0].smem);
+      threads = std::max(threads, plan_of(L, kk, 1).threads);
+      smem = std::max(smem, plan_of(L, kk, 1).smem);
     }
     const void* fn = fast ? reinterpret_cast<const void*>(PERSIST_FAST) : reinterpret_cast<const void*>(PERSIST_GENERIC);
     e = raise_smem_limit(fn, smem);
