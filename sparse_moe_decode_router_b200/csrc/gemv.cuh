@@ -44,10 +44,22 @@ namespace moe {
 
 enum XKind : int { X_BF16 = 0, X_F32 = 1 };
 
+// 16 consumer warps: four 4-warp groups per SM (measured faster than 12 on the
+// one-token down projection; 20 spills its registers)
 #ifndef MOE_MAX_CONSUMER_WARPS
-#define MOE_MAX_CONSUMER_WARPS 12
+#define MOE_MAX_CONSUMER_WARPS 16
 #endif
 constexpr int kMaxConsumerWarps = MOE_MAX_CONSUMER_WARPS;
+// the MXFP4 gate/up streams (two weight rows per output, K = hidden) keep 12:
+// measured faster there (the 16-warp launch bound cuts their registers to 96)
+#ifndef MOE_GU_CONSUMER_WARPS
+#define MOE_GU_CONSUMER_WARPS 12
+#endif
+// consumer warps of a whole-row (not split-K) instance: its launch bound and its plans
+__host__ __device__ constexpr int consumer_warps_for(int wf, int epi) {
+  return (wf == W_MXFP4 && epi == EPI_SWIGLU && MOE_GU_CONSUMER_WARPS < kMaxConsumerWarps) ? MOE_GU_CONSUMER_WARPS
+                                                                                        : kMaxConsumerWarps;
+}
 // Split-K instances (one token, MXFP4, compile-time K): more, lighter warps.
 #ifndef MOE_MAX_SPLITK_WARPS
 #define MOE_MAX_SPLITK_WARPS 16
@@ -463,6 +475,10 @@ struct TokenPass {
 // have more threads than this stream's plan uses: the extra warps leave at
 // once, and every barrier below counts only the plan's (ncw + 1) warps.
 constexpr int kBarAll = 15;  // named barrier over all of a stream's warps
+// named barriers: 1 (consumers), 2 (phase table), 3 + group (item groups), kBarAll
+constexpr int kMaxItemGroups = kBarAll - 3;
+// warps per item that keep ncw / wpi <= kMaxItemGroups for any ncw <= kMaxWarpsAny
+constexpr int kMinItemWarps = (kMaxWarpsAny + kMaxItemGroups - 1) / kMaxItemGroups;
 
 template <int WF, int EPI, int XK, int TMAX, int RPW, int KT>
 __device__ __forceinline__ void gemv_body(const GemvArgs& a, unsigned char* smem) {
@@ -540,7 +556,7 @@ __device__ __forceinline__ void gemv_body(const GemvArgs& a, unsigned char* smem
   // groups, and an item's rows are exactly what the group's warps cover
   const int kq_plan = kFast ? KS : ((WF == W_BF16 && a.ksplit > 1) ? a.ksplit : 1);
   if ((a.ncw % a.wpi) != 0 || (a.n_stages % (a.ncw / a.wpi)) != 0 || (a.wpi % kq_plan) != 0 ||
-      a.R != RPW * (a.wpi / kq_plan)) {
+      a.R != RPW * (a.wpi / kq_plan) || a.ncw > kMaxWarpsAny || a.wpi < kMinItemWarps) {
     if (tid == 0) atomicExch(a.err, kErrBadPlan);
     return;
   }
@@ -1112,7 +1128,7 @@ template <int WF, int EPI, int XK, int TMAX, int RPW, int KT>
 __global__ void __launch_bounds__(((KT != 0 && WF == W_MXFP4 && TMAX == 1 &&
                                     (EPI == EPI_SWIGLU ? 2 * RPW : RPW) == kSplitKRows)
                                        ? kMaxSplitKWarps
-                                       : kMaxConsumerWarps) * 32 + 32,
+                                       : consumer_warps_for(WF, EPI)) * 32 + 32,
                                   1) gemv_kernel(const GemvArgs a) {
   extern __shared__ __align__(128) unsigned char smem[];
   gemv_body<WF, EPI, XK, TMAX, RPW, KT>(a, smem);

@@ -141,9 +141,9 @@ GemvPlan make_plan(Kind kind, int K, int out_rows, int slots_needed, int max_gro
   // group count: every stage is then always consumed by the same group, in
   // item order, and a group never waits on a stage whose previous phase
   // another group has not finished.
-  const int max_warps = splitk ? kMaxSplitKWarps : kMaxConsumerWarps;
-  if (t.wpi > max_warps) return p;
-  int groups = std::max(1, std::min(max_warps / t.wpi, std::max(1, ns - pf)));
+  const int max_warps = splitk ? kMaxSplitKWarps : consumer_warps_for(t.wf, t.epi);
+  if (t.wpi > max_warps || t.wpi < kMinItemWarps) return p;
+  int groups = std::max(1, std::min(std::min(max_warps / t.wpi, kMaxItemGroups), std::max(1, ns - pf)));
   while (groups > 1 && (ns / groups) * groups - groups < pf) --groups;
   ns = (ns / groups) * groups;
   p.ok = true;
