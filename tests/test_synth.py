@@ -212,3 +212,23 @@ def test_full_size_bench_tokens_keep_the_routing_margin(cfg_id):
     if cfg.verify_corr > 0:
         # positions of one sequence share experts (a verify step's routing)
         assert np.unique(rt["topk_idx"]).size < 0.75 * cfg.batch * k
+
+
+def test_stack_workload_tokens_keep_the_routing_margin_on_every_layer():
+    """The four-layer graph workload: each layer has its own router draw and
+    its own token substream (token id = decode step); every (layer, step)
+    token routes with the margin under the oracle's logits, and the layers'
+    routers are different draws."""
+    cfg = synth.CONFIGS[4]
+    k = cfg.top_k
+    first = None
+    for layer in range(cfg.n_layers):
+        wr = synth.gen_router_w(cfg, layer)
+        if first is None:
+            first = wr
+        else:
+            assert not np.array_equal(wr, first)
+        x, _ = synth.gen_tokens(cfg, wr, None, range(cfg.n_steps), layer=layer)
+        lg = oracle.router_logits(x, wr, None)
+        srt = -np.sort(-lg, axis=1)
+        assert np.all(srt[:, k - 1] - srt[:, k] >= cfg.min_gap)
